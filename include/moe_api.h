@@ -1,0 +1,186 @@
+/*
+ * moe_api.h -- C ABI of libmoe.so: one sparse Mixture-of-Experts layer with
+ * MLX-affine quantised weights on NVIDIA B200 (sm_100a).
+ *
+ * The layer (TurboFieldfare introduction page, discuss.pytorch.kr, section
+ * "TurboFieldfare's expert streaming structure", router pseudo-code and the
+ * three-phase description; weight format from section "How TurboFieldfare
+ * saves memory"):
+ *   xn  = rmsnorm_no_scale(h)                       (no learned weight, eps inside the RMS)
+ *   xs  = xn * router_scale / sqrt(H)
+ *   logit_e = sum_i (s_e,g * q_e,i + b_e,g) * xs_i  (8-bit affine codes, groups of 64)
+ *   idx = highest k logits (ties -> lower expert index; ordered by logit desc, index asc)
+ *   w   = softmax(logit[idx]) * per_expert_scale[idx]   (no renormalisation)
+ *   xe  = bf16(xn)                                  (what the experts consume)
+ *   m   = sum_s w_s * FFN_idx_s(xe) + FFN_shared(xe) (shared expert: no routing weight)
+ *   FFN(x) = Wd (silu(Wg x) * (Wu x)),  W = scale * q + bias, 4-bit codes, groups of 64
+ *   out = (h + rmsnorm_no_scale(m)) * layer_scalar  (normalisation, residual, layer scalar)
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     16-byte aligned.  The library never allocates on these paths; scratch
+ *     comes from a caller-provided workspace (see moe_workspace_size).
+ *   - bf16 values are passed as their 16-bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on that stream and returns; none synchronises.
+ *   - Return value: MOE_OK (0) or a negative MOE_E* code.  Argument errors are
+ *     detected on the host before anything is enqueued; the reason is then in
+ *     moe_last_error() (per host thread).  Inputs are assumed finite.
+ *   - T == 0 is a valid empty call: nothing is enqueued, MOE_OK is returned.
+ *
+ * Limits: H, I, Is multiples of 64 and <= 8192; 1 <= k <= min(E, 32);
+ * E <= 1024 and a multiple of 8; 0 <= T <= 65535; T * k <= 65536.
+ */
+#ifndef MOE_API_H
+#define MOE_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_EINVAL (-1)     /* bad size, null pointer, k > E, ... */
+#define MOE_EALIGN (-2)     /* a pointer is not 16-byte aligned */
+#define MOE_EWORKSPACE (-3) /* workspace missing or smaller than moe_workspace_size() */
+#define MOE_ECUDA (-4)      /* a CUDA launch failed; the CUDA error string is in moe_last_error() */
+
+/*
+ * Quantised matrix set in the kernel ("tiled") layout, produced once per
+ * weight tensor by moe_prepare_qmat from the MLX layout.  n_mat matrices of
+ * [rows, cols] (rows % 32 == 0, cols % 64 == 0):
+ *   q : uint32 words.  For matrix m, row block rb = row / 32, column chunk
+ *       c = col / 32: a 512-byte block at word offset
+ *       ((m * rows/32 + rb) * cols/32 + c) * 128; inside it, lane l = row % 32
+ *       holds 4 consecutive words (the row's MLX words 4c .. 4c+3, i.e.
+ *       columns 32c .. 32c+31, eight 4-bit codes per word, low nibble first).
+ *   sb: uint32 per (matrix, row, group of 64 columns): low 16 bits = bf16
+ *       scale, high 16 bits = bf16 bias; for matrix m, row block rb, group g,
+ *       lane l at word offset ((m * rows/32 + rb) * cols/64 + g) * 32 + l.
+ * One row block of one matrix is therefore contiguous, so a warp whose lanes
+ * are 32 consecutive rows reads 512 contiguous bytes per column chunk.
+ */
+typedef struct {
+    const uint32_t *q;
+    const uint32_t *sb;
+} moe_qmat;
+
+/* One MoE layer's weights, all device pointers. */
+typedef struct {
+    int H;  /* hidden size */
+    int E;  /* routed experts */
+    int k;  /* experts per token */
+    int I;  /* routed expert intermediate size */
+    int Is; /* shared expert intermediate size */
+    /* router projection, MLX layout: codes [E, H/4] (four 8-bit codes per word,
+     * low byte first), bf16 scale and bias [E, H/64] */
+    const uint32_t *router_q;
+    const uint16_t *router_s;
+    const uint16_t *router_b;
+    const uint16_t *router_scale;     /* [H] bf16 */
+    const uint16_t *per_expert_scale; /* [E] bf16 */
+    /* routed experts, tiled layout: gate/up are E matrices [I, H], down E x [H, I] */
+    moe_qmat gate, up, down;
+    /* shared expert, tiled layout: gate/up [Is, H], down [H, Is] */
+    moe_qmat sh_gate, sh_up, sh_down;
+} moe_layer_w;
+
+typedef struct {
+    int post_norm;      /* 1: out = (h + rmsnorm_no_scale(m)) * layer_scalar; 0: (h + m) * layer_scalar */
+    float layer_scalar; /* default 1.0 */
+    float eps;          /* default 1e-6, inside every RMS */
+    int force_path;     /* 0 auto, 1 CUDA-core dequant-GEMV, 2 tensor-core grouped GEMM */
+} moe_opts;
+
+/* Text of the last error on this host thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+/*
+ * Repack n_mat MLX-layout matrices [rows, cols] (codes q [n_mat, rows, cols/8]
+ * uint32, scale/bias [n_mat, rows, cols/64] bf16) into the tiled layout
+ * described at moe_qmat.  q_out has the same number of words as q;
+ * sb_out has n_mat * rows * cols/64 words.  Off the hot path; done once per
+ * weight tensor.  rows % 32 == 0, cols % 64 == 0.
+ */
+MOE_API int moe_prepare_qmat(const uint32_t *q, const uint16_t *scale, const uint16_t *bias, int n_mat, int rows,
+                     int cols, uint32_t *q_out, uint32_t *sb_out, void *stream);
+
+/*
+ * Bytes of workspace that moe_router / moe_expert_ffn / moe_layer_forward
+ * need for calls with up to T_max tokens on layers shaped like `w`.
+ * Returns 0 on invalid arguments.
+ */
+MOE_API size_t moe_workspace_size(const moe_layer_w *w, int T_max);
+
+/*
+ * Router logits only (the first three lines of the router pseudo-code):
+ *   h [T, H] bf16  ->  logits [T, E] fp64, and (if xe != NULL) xe [T, H] bf16.
+ * Accumulates in fp64 so that the top-k decision does not depend on the
+ * summation order.
+ */
+MOE_API int moe_router_logits(const moe_layer_w *w, const uint16_t *h, int T, double *logits, uint16_t *xe,
+                      void *stream);
+
+/*
+ * Top-k + gate weights (last two lines of the router pseudo-code):
+ *   logits [T, E] fp64 -> idx [T, k] int32 (logit desc, index asc; equal
+ *   logits -> lower index), wts [T, k] fp32 = softmax over the k selected
+ *   logits * per_expert_scale[idx].
+ */
+MOE_API int moe_router_topk(const double *logits, int T, int E, int k, const uint16_t *per_expert_scale, int32_t *idx,
+                    float *wts, void *stream);
+
+/*
+ * Whole router: h [T, H] bf16 -> idx [T, k], wts [T, k], xe [T, H] bf16 (xe
+ * may be NULL).  Uses T * E * 8 bytes of the workspace for the logits.
+ */
+MOE_API int moe_router(const moe_layer_w *w, const uint16_t *h, int T, int32_t *idx, float *wts, uint16_t *xe,
+               void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Token -> expert bucketing of the T*k (token, slot) pairs:
+ *   offsets [E+1]: exclusive prefix sum of pairs per expert;
+ *   perm [T*k]   : pair ids p = t*k + s grouped by expert, ascending p inside
+ *                  an expert (stable);
+ *   inv [T*k]    : inv[perm[j]] = j (may be NULL);
+ *   active [E+1] : active[0] = number of experts with at least one pair,
+ *                  active[1..] = those experts ascending (may be NULL).
+ * idx values must lie in [0, E); T * k <= 65536.
+ */
+MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, int32_t *inv,
+               int32_t *active, void *stream);
+
+/*
+ * Expert part of the layer: m [T, H] fp32 = sum_s wts[t,s] * FFN_idx[t,s](xe_t)
+ * (+ FFN_shared(xe_t) when with_shared).  Inputs: xe [T, H] bf16, idx/wts
+ * [T, k], and the bucketing of idx (offsets, perm, active from moe_bucket).
+ */
+MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *idx, const float *wts,
+                   const int32_t *offsets, const int32_t *perm, const int32_t *active, int with_shared,
+                   float *m_out, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream);
+
+/*
+ * One whole MoE layer: router -> bucketing -> routed + shared experts ->
+ * weighted combine -> normalisation, residual, layer scalar.
+ *   h_in [T, H] bf16 -> h_out [T, H] bf16 (h_out may not alias h_in).
+ * opts may be NULL (post_norm 1, layer_scalar 1, eps 1e-6, auto path).
+ */
+MOE_API int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T, void *ws,
+                      size_t ws_bytes, const moe_opts *opts, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_API_H */

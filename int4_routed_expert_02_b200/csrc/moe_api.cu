@@ -1,0 +1,330 @@
+// moe_api.cu -- the C ABI of libmoe.so: argument checks, workspace carving,
+// and the launch sequence of each call.  See include/moe_api.h.
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+cudaError_t ensure_smem(const void *kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    static std::mutex mu;
+    static std::unordered_map<const void *, size_t> done;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find(kernel);
+    if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done[kernel] = bytes;
+    return e;
+}
+
+}  // namespace moe
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where) {
+    return fail(MOE_ECUDA, "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDim = 8192;
+constexpr int kMaxT = 65535;
+
+#define CHECK_PTR(p)                                                                 \
+    do {                                                                             \
+        if (!(p)) return fail(MOE_EINVAL, "%s: %s is NULL", fn, #p);                 \
+        if (!aligned16(p)) return fail(MOE_EALIGN, "%s: %s is not 16-byte aligned", fn, #p); \
+    } while (0)
+
+#define CHECK_OPT_PTR(p)                                                             \
+    do {                                                                             \
+        if ((p) && !aligned16(p)) return fail(MOE_EALIGN, "%s: %s is not 16-byte aligned", fn, #p); \
+    } while (0)
+
+int check_dims(const char *fn, const moe_layer_w *w) {
+    if (!w) return fail(MOE_EINVAL, "%s: layer is NULL", fn);
+    if (w->H < 64 || w->H % 64 || w->H > kMaxDim) return fail(MOE_EINVAL, "%s: H=%d must be a multiple of 64 in [64, %d]", fn, w->H, kMaxDim);
+    if (w->I < 64 || w->I % 64 || w->I > kMaxDim) return fail(MOE_EINVAL, "%s: I=%d must be a multiple of 64 in [64, %d]", fn, w->I, kMaxDim);
+    if (w->Is < 64 || w->Is % 64 || w->Is > kMaxDim) return fail(MOE_EINVAL, "%s: Is=%d must be a multiple of 64 in [64, %d]", fn, w->Is, kMaxDim);
+    if (w->E < 8 || w->E % 8 || w->E > moe::kMaxE) return fail(MOE_EINVAL, "%s: E=%d must be a multiple of 8 in [8, %d]", fn, w->E, moe::kMaxE);
+    if (w->k < 1 || w->k > w->E || w->k > moe::kMaxK) return fail(MOE_EINVAL, "%s: k=%d must be in [1, min(E, %d)]", fn, w->k, moe::kMaxK);
+    return MOE_OK;
+}
+
+int check_router_ptrs(const char *fn, const moe_layer_w *w) {
+    CHECK_PTR(w->router_q);
+    CHECK_PTR(w->router_s);
+    CHECK_PTR(w->router_b);
+    CHECK_PTR(w->router_scale);
+    CHECK_PTR(w->per_expert_scale);
+    return MOE_OK;
+}
+
+int check_expert_ptrs(const char *fn, const moe_layer_w *w, int with_shared) {
+    CHECK_PTR(w->gate.q);
+    CHECK_PTR(w->gate.sb);
+    CHECK_PTR(w->up.q);
+    CHECK_PTR(w->up.sb);
+    CHECK_PTR(w->down.q);
+    CHECK_PTR(w->down.sb);
+    if (with_shared) {
+        CHECK_PTR(w->sh_gate.q);
+        CHECK_PTR(w->sh_gate.sb);
+        CHECK_PTR(w->sh_up.q);
+        CHECK_PTR(w->sh_up.sb);
+        CHECK_PTR(w->sh_down.q);
+        CHECK_PTR(w->sh_down.sb);
+    }
+    return MOE_OK;
+}
+
+int check_T(const char *fn, int T) {
+    if (T < 0 || T > kMaxT) return fail(MOE_EINVAL, "%s: T=%d must be in [0, %d]", fn, T, kMaxT);
+    return MOE_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace carve-up for calls of up to T tokens.
+struct WsLayout {
+    size_t logits, idx, wts, xe, offsets, perm, inv, active, a_routed, a_shared, y, sh, total;
+};
+
+WsLayout ws_layout(const moe_layer_w *w, int T) {
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t Tk = (size_t)T * w->k;
+    L.logits = take(sizeof(double) * T * w->E);
+    L.idx = take(sizeof(int32_t) * Tk);
+    L.wts = take(sizeof(float) * Tk);
+    L.xe = take(sizeof(uint16_t) * T * w->H);
+    L.offsets = take(sizeof(int32_t) * (w->E + 1));
+    L.perm = take(sizeof(int32_t) * Tk);
+    L.inv = take(sizeof(int32_t) * Tk);
+    L.active = take(sizeof(int32_t) * (w->E + 1));
+    L.a_routed = take(sizeof(float) * Tk * w->I);
+    L.a_shared = take(sizeof(float) * T * w->Is);
+    L.y = take(sizeof(float) * Tk * w->H);
+    L.sh = take(sizeof(float) * T * w->H);
+    L.total = off;
+    return L;
+}
+
+template <typename P>
+P *at(void *ws, size_t off) {
+    return reinterpret_cast<P *>(static_cast<char *>(ws) + off);
+}
+
+int check_ws(const char *fn, const moe_layer_w *w, int T, void *ws, size_t ws_bytes) {
+    const size_t need = ws_layout(w, T).total;
+    if (!ws) return fail(MOE_EWORKSPACE, "%s: workspace is NULL (need %zu bytes)", fn, need);
+    if (!aligned16(ws)) return fail(MOE_EALIGN, "%s: workspace is not 16-byte aligned", fn);
+    if (ws_bytes < need) return fail(MOE_EWORKSPACE, "%s: workspace has %zu bytes, needs %zu", fn, ws_bytes, need);
+    return MOE_OK;
+}
+
+moe_opts resolve_opts(const moe_opts *o) {
+    moe_opts r{1, 1.0f, 1e-6f, 0};
+    if (o) r = *o;
+    return r;
+}
+
+int check_opts(const char *fn, const moe_opts &o) {
+    if (o.force_path < 0 || o.force_path > 1)
+        return fail(MOE_EINVAL, "%s: force_path=%d (0 auto, 1 dequant-GEMV)", fn, o.force_path);
+    if (!(o.eps >= 0.0f)) return fail(MOE_EINVAL, "%s: eps must be >= 0", fn);
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+const char *moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+int moe_prepare_qmat(const uint32_t *q, const uint16_t *scale, const uint16_t *bias, int n_mat, int rows, int cols,
+                     uint32_t *q_out, uint32_t *sb_out, void *stream) {
+    const char *fn = "moe_prepare_qmat";
+    g_err.clear();
+    if (n_mat < 1 || rows < 32 || rows % 32 || cols < 64 || cols % 64 || rows > (1 << 20) || cols > kMaxDim)
+        return fail(MOE_EINVAL, "%s: need n_mat >= 1, rows %% 32 == 0, cols %% 64 == 0 (got %d, %d, %d)", fn, n_mat,
+                    rows, cols);
+    CHECK_PTR(q);
+    CHECK_PTR(scale);
+    CHECK_PTR(bias);
+    CHECK_PTR(q_out);
+    CHECK_PTR(sb_out);
+    cudaError_t e = moe::launch_prepare_qmat(q, scale, bias, n_mat, rows, cols, q_out, sb_out,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+size_t moe_workspace_size(const moe_layer_w *w, int T_max) {
+    if (check_dims("moe_workspace_size", w) || T_max < 0 || T_max > kMaxT) return 0;
+    return ws_layout(w, T_max).total;
+}
+
+int moe_router_logits(const moe_layer_w *w, const uint16_t *h, int T, double *logits, uint16_t *xe, void *stream) {
+    const char *fn = "moe_router_logits";
+    g_err.clear();
+    if (int rc = check_dims(fn, w)) return rc;
+    if (int rc = check_T(fn, T)) return rc;
+    if (int rc = check_router_ptrs(fn, w)) return rc;
+    CHECK_PTR(h);
+    CHECK_PTR(logits);
+    CHECK_OPT_PTR(xe);
+    if (T == 0) return MOE_OK;
+    cudaError_t e = moe::launch_router_logits(w, h, T, 1e-6f, logits, xe, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_router_topk(const double *logits, int T, int E, int k, const uint16_t *per_expert_scale, int32_t *idx,
+                    float *wts, void *stream) {
+    const char *fn = "moe_router_topk";
+    g_err.clear();
+    if (int rc = check_T(fn, T)) return rc;
+    if (E < 1 || E > moe::kMaxE) return fail(MOE_EINVAL, "%s: E=%d must be in [1, %d]", fn, E, moe::kMaxE);
+    if (k < 1 || k > E || k > moe::kMaxK) return fail(MOE_EINVAL, "%s: k=%d must be in [1, min(E, %d)]", fn, k, moe::kMaxK);
+    CHECK_PTR(logits);
+    CHECK_PTR(per_expert_scale);
+    CHECK_PTR(idx);
+    CHECK_PTR(wts);
+    if (T == 0) return MOE_OK;
+    cudaError_t e = moe::launch_router_topk(logits, T, E, k, per_expert_scale, idx, wts,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_router(const moe_layer_w *w, const uint16_t *h, int T, int32_t *idx, float *wts, uint16_t *xe, void *ws,
+               size_t ws_bytes, void *stream) {
+    const char *fn = "moe_router";
+    g_err.clear();
+    if (int rc = check_dims(fn, w)) return rc;
+    if (int rc = check_T(fn, T)) return rc;
+    if (int rc = check_router_ptrs(fn, w)) return rc;
+    CHECK_PTR(h);
+    CHECK_PTR(idx);
+    CHECK_PTR(wts);
+    CHECK_OPT_PTR(xe);
+    if (T == 0) return MOE_OK;
+    if (int rc = check_ws(fn, w, T, ws, ws_bytes)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(w, T);
+    double *logits = at<double>(ws, L.logits);
+    cudaError_t e = moe::launch_router_logits(w, h, T, 1e-6f, logits, xe, st);
+    if (e == cudaSuccess) e = moe::launch_router_topk(logits, T, w->E, w->k, w->per_expert_scale, idx, wts, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, int32_t *inv,
+               int32_t *active, void *stream) {
+    const char *fn = "moe_bucket";
+    g_err.clear();
+    if (int rc = check_T(fn, T)) return rc;
+    if (E < 1 || E > moe::kMaxE) return fail(MOE_EINVAL, "%s: E=%d must be in [1, %d]", fn, E, moe::kMaxE);
+    if (k < 1 || k > moe::kMaxK) return fail(MOE_EINVAL, "%s: k=%d must be in [1, %d]", fn, k, moe::kMaxK);
+    if ((long long)T * k > 65536) return fail(MOE_EINVAL, "%s: T*k=%lld exceeds 65536", fn, (long long)T * k);
+    CHECK_PTR(idx);
+    CHECK_PTR(offsets);
+    CHECK_PTR(perm);
+    CHECK_OPT_PTR(inv);
+    CHECK_OPT_PTR(active);
+    if (T == 0) return MOE_OK;
+    cudaError_t e = moe::launch_bucket(idx, T * k, E, offsets, perm, inv, active, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *idx, const float *wts,
+                   const int32_t *offsets, const int32_t *perm, const int32_t *active, int with_shared, float *m_out,
+                   void *ws, size_t ws_bytes, const moe_opts *opts, void *stream) {
+    const char *fn = "moe_expert_ffn";
+    g_err.clear();
+    if (int rc = check_dims(fn, w)) return rc;
+    if (int rc = check_T(fn, T)) return rc;
+    if ((long long)T * w->k > 65536) return fail(MOE_EINVAL, "%s: T*k exceeds 65536", fn);
+    if (int rc = check_expert_ptrs(fn, w, with_shared)) return rc;
+    const moe_opts o = resolve_opts(opts);
+    if (int rc = check_opts(fn, o)) return rc;
+    CHECK_PTR(xe);
+    CHECK_PTR(idx);
+    CHECK_PTR(wts);
+    CHECK_PTR(offsets);
+    CHECK_PTR(perm);
+    CHECK_PTR(active);
+    CHECK_PTR(m_out);
+    if (T == 0) return MOE_OK;
+    if (int rc = check_ws(fn, w, T, ws, ws_bytes)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(w, T);
+    moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
+    cudaError_t e = moe::launch_expert_gemv(w, xe, T, offsets, perm, active, with_shared, b, st);
+    if (e == cudaSuccess)
+        e = moe::launch_combine(b.y, b.sh, wts, T, w->H, w->k, with_shared, nullptr, m_out, nullptr, 0, 1.0f, 0.0f, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T, void *ws, size_t ws_bytes,
+                      const moe_opts *opts, void *stream) {
+    const char *fn = "moe_layer_forward";
+    g_err.clear();
+    if (int rc = check_dims(fn, w)) return rc;
+    if (int rc = check_T(fn, T)) return rc;
+    if ((long long)T * w->k > 65536) return fail(MOE_EINVAL, "%s: T*k exceeds 65536", fn);
+    if (int rc = check_router_ptrs(fn, w)) return rc;
+    if (int rc = check_expert_ptrs(fn, w, 1)) return rc;
+    const moe_opts o = resolve_opts(opts);
+    if (int rc = check_opts(fn, o)) return rc;
+    CHECK_PTR(h_in);
+    CHECK_PTR(h_out);
+    if (T > 0) {
+        const char *a = reinterpret_cast<const char *>(h_in), *b = reinterpret_cast<const char *>(h_out);
+        const size_t n = sizeof(uint16_t) * (size_t)T * w->H;
+        if (a < b + n && b < a + n) return fail(MOE_EINVAL, "%s: h_out overlaps h_in", fn);
+    }
+    if (T == 0) return MOE_OK;
+    if (int rc = check_ws(fn, w, T, ws, ws_bytes)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(w, T);
+    double *logits = at<double>(ws, L.logits);
+    int32_t *idx = at<int32_t>(ws, L.idx);
+    float *wts = at<float>(ws, L.wts);
+    uint16_t *xe = at<uint16_t>(ws, L.xe);
+    int32_t *offsets = at<int32_t>(ws, L.offsets), *perm = at<int32_t>(ws, L.perm), *inv = at<int32_t>(ws, L.inv);
+    int32_t *active = at<int32_t>(ws, L.active);
+    moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
+    cudaError_t e = moe::launch_router_logits(w, h_in, T, o.eps, logits, xe, st);
+    if (e == cudaSuccess) e = moe::launch_router_topk(logits, T, w->E, w->k, w->per_expert_scale, idx, wts, st);
+    if (e == cudaSuccess) e = moe::launch_bucket(idx, T * w->k, w->E, offsets, perm, inv, active, st);
+    if (e == cudaSuccess) e = moe::launch_expert_gemv(w, xe, T, offsets, perm, active, 1, b, st);
+    if (e == cudaSuccess)
+        e = moe::launch_combine(b.y, b.sh, wts, T, w->H, w->k, 1, h_in, nullptr, h_out, o.post_norm, o.layer_scalar,
+                                o.eps, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// moe_internal.h -- launchers shared between the kernel files and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/moe_api.h"
+
+namespace moe {
+
+// Raise a kernel's dynamic shared memory limit once (per process) to at
+// least `bytes`.  A no-op below 48 KiB.
+cudaError_t ensure_smem(const void *kernel, size_t bytes);
+
+size_t router_logits_smem(int H);
+cudaError_t launch_router_logits(const moe_layer_w *w, const uint16_t *h, int T, float eps, double *logits,
+                                 uint16_t *xe, cudaStream_t st);
+cudaError_t launch_router_topk(const double *logits, int T, int E, int k, const uint16_t *pes, int32_t *idx,
+                               float *wts, cudaStream_t st);
+cudaError_t launch_bucket(const int32_t *idx, int n_pairs, int E, int32_t *offsets, int32_t *perm, int32_t *inv,
+                          int32_t *active, cudaStream_t st);
+cudaError_t launch_prepare_qmat(const uint32_t *q, const uint16_t *s, const uint16_t *b, int n_mat, int rows,
+                                int cols, uint32_t *q_out, uint32_t *sb_out, cudaStream_t st);
+
+// Intermediate buffers of the expert part (all device, from the workspace).
+struct FfnBuffers {
+    float *a_routed;  // [T*k, I]  SwiGLU output, by bucketed position
+    float *a_shared;  // [T, Is]
+    float *y;         // [T*k, H]  routed expert outputs, by pair id t*k+s
+    float *sh;        // [T, H]    shared expert output
+};
+
+size_t gemv_smem_bytes(int cols, int nt);
+cudaError_t launch_expert_gemv(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
+                               const int32_t *perm, const int32_t *active, int with_shared, const FfnBuffers &b,
+                               cudaStream_t st);
+// mode 0: m_out[t] = sum_s w y + sh ; mode 1: h_out = bf16((h + rmsnorm(m)) * scalar) (or no norm)
+cudaError_t launch_combine(const float *y, const float *sh, const float *wts, int T, int H, int k, int with_shared,
+                           const uint16_t *h_in, float *m_out, uint16_t *h_out, int post_norm, float layer_scalar,
+                           float eps, cudaStream_t st);
+
+}  // namespace moe

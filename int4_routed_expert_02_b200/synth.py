@@ -202,7 +202,7 @@ def gen_hidden(cfg: MoEConfig, cfg_id: int, stream: int, T: int, seed: int = 0, 
 
 
 def gen_zipf_hidden(cfg: MoEConfig, cfg_id: int, layer: int, step: int, router_codes: torch.Tensor,
-                    seed: int = 0) -> tuple[torch.Tensor, torch.Tensor]:
+                    seed: int = 0, T: int | None = None) -> tuple[torch.Tensor, torch.Tensor]:
     """Router inputs whose selected experts follow a Zipf(cfg.zipf) popularity.
 
     Per layer a random permutation assigns popularity ranks to experts; per
@@ -217,7 +217,8 @@ def gen_zipf_hidden(cfg: MoEConfig, cfg_id: int, layer: int, step: int, router_c
     router_codes: the layer's `router_codes` from gen_layer ([E, H] uint8).
     Returns (hidden [T, H] bf16, target expert ids [T, k] int64).
     """
-    E, k, T = cfg.E, cfg.k, cfg.T
+    E, k = cfg.E, cfg.k
+    T = cfg.T if T is None else T
     gp = _gen("cpu", tensor_seed(seed, cfg_id, layer, "zipf_perm"))
     perm = torch.randperm(E, generator=gp)            # perm[e] = popularity rank of expert e (0 = top)
     logp = -cfg.zipf * torch.log(perm.double() + 1.0)
