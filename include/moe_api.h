@@ -179,6 +179,39 @@ MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, cons
 MOE_API int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T, void *ws,
                       size_t ws_bytes, const moe_opts *opts, void *stream);
 
+/*
+ * moe_layer_forward for callers that cannot allocate device memory.  (The
+ * pages have no counterpart: this is a deployment convenience.)
+ *
+ * Some callers cannot call cudaMalloc on this path: code that runs while a
+ * stream is being captured into a CUDA graph in the global capture mode
+ * (allocation is forbidden there), latency-critical serving loops where an
+ * allocation may synchronise the device, and plugins that run inside a host
+ * framework that owns all device memory.  This entry point takes the same
+ * arguments as moe_layer_forward minus the workspace, and uses instead a
+ * scratch array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) that the library
+ * defines in device memory; every GPU that loads the library holds that array
+ * until the process exits.  It calls no cudaMalloc, cudaFree or allocating
+ * library routine.
+ *   - Sizes whose workspace (moe_workspace_size) exceeds the scratch are
+ *     rejected with MOE_EWORKSPACE and a message naming both sizes; decode
+ *     batches fit (about 140 KiB per token at hidden 2816, 128 experts, top-8).
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.  The device is the stream's device
+ *     (the current device for the NULL stream).
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; nothing in it needs to start at zero.  Calls whose
+ *     kernels overlap on the GPU (different streams, or several host threads)
+ *     race on the scratch: serialise them.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+MOE_API size_t moe_noalloc_scratch_bytes(void);
+
+MOE_API int moe_layer_forward_noalloc(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T,
+                                      const moe_opts *opts, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -161,6 +161,10 @@ int check_opts(const char *fn, const moe_opts &o) {
 
 }  // namespace
 
+namespace moe {
+int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace moe
+
 extern "C" {
 
 const char *moe_last_error(void) { return g_err.c_str(); }

@@ -9,6 +9,9 @@
 
 namespace moe {
 
+// Record `msg` as this host thread's moe_last_error() text; returns `code`.
+int set_last_error(int code, const char *msg);
+
 // Raise a kernel's dynamic shared memory limit once (per process) to at
 // least `bytes`.  A no-op below 48 KiB.
 cudaError_t ensure_smem(const void *kernel, size_t bytes);

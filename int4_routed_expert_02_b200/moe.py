@@ -21,7 +21,8 @@ _lib = C.CDLL(LIB_PATH)
 
 MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_ECUDA = 0, -1, -2, -3, -4
 EXPORTED = ("moe_last_error", "moe_version", "moe_prepare_qmat", "moe_workspace_size", "moe_router_logits",
-            "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward")
+            "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward",
+            "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc")
 
 
 class MoEError(RuntimeError):
@@ -58,6 +59,8 @@ _lib.moe_router.argtypes = [_P, _P, _I, _P, _P, _P, _P, C.c_size_t, _P]
 _lib.moe_bucket.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
 _lib.moe_expert_ffn.argtypes = [_P, _P, _I, _P, _P, _P, _P, _P, _I, _P, _P, C.c_size_t, _P, _P]
 _lib.moe_layer_forward.argtypes = [_P, _P, _P, _I, _P, C.c_size_t, _P, _P]
+_lib.moe_noalloc_scratch_bytes.restype = C.c_size_t
+_lib.moe_layer_forward_noalloc.argtypes = [_P, _P, _P, _I, _P, _P]
 
 
 def lib():
@@ -198,6 +201,17 @@ def moe_layer_forward(layer, h_in, h_out, T, ws, opts=None, stream=None):
     o = opts if opts is not None else _opts()
     _check(_lib.moe_layer_forward(layer.ptr(), _ptr(h_in), _ptr(h_out), T, _ptr(ws),
                                   ws.numel() if ws is not None else 0, C.byref(o), _stream(stream)))
+
+
+def moe_layer_forward_noalloc(layer, h_in, h_out, T, opts=None, stream=None):
+    """moe_layer_forward without a workspace: the library's static scratch
+    (moe_noalloc_scratch_bytes()) is used instead; see include/moe_api.h."""
+    o = opts if opts is not None else _opts()
+    _check(_lib.moe_layer_forward_noalloc(layer.ptr(), _ptr(h_in), _ptr(h_out), T, C.byref(o), _stream(stream)))
+
+
+def moe_noalloc_scratch_bytes() -> int:
+    return int(_lib.moe_noalloc_scratch_bytes())
 
 
 def make_opts(post_norm=True, layer_scalar=1.0, eps=1e-6, force_path=0) -> Opts:
