@@ -123,7 +123,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     cfg = synth.CONFIGS[args.config]
     T = args.tokens or cfg.T
-    st = MoEStack(cfg, args.config, T=T, device=dev, keep_router_codes=cfg.zipf > 0)
+    st = MoEStack(cfg, args.config, T=T, layers=args.layers or None, device=dev, keep_router_codes=cfg.zipf > 0)
     K, W = args.steps, args.warmup
 
     # one fresh input per step, generated up front (device-resident)
@@ -375,6 +375,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: the config's)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: build this many layers instead of the config's (not a bench line)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
