@@ -52,6 +52,7 @@ extern "C" {
 #define MOE_EALIGN (-2)     /* a pointer is not 16-byte aligned */
 #define MOE_EWORKSPACE (-3) /* workspace missing or smaller than moe_workspace_size() */
 #define MOE_ECUDA (-4)      /* a CUDA launch failed; the CUDA error string is in moe_last_error() */
+#define MOE_EDEVICE (-5)    /* a kernel recorded an error (a bounded wait ran out); see moe_decode_stack_status */
 
 /*
  * Quantised matrix set in the kernel ("tiled") layout, produced once per
@@ -178,6 +179,34 @@ MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, cons
  */
 MOE_API int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T, void *ws,
                       size_t ws_bytes, const moe_opts *opts, void *stream);
+
+/*
+ * Decode step through a stack of L layers (the per-token layer loop of the
+ * TurboFieldfare page, section "TurboFieldfare's expert streaming structure",
+ * last paragraph) in ONE persistent cooperative kernel, one CTA per SM.  Per
+ * layer it computes exactly what moe_layer_forward computes.
+ *   layers [L]  : HOST array of L layer descriptors, all with the same shape
+ *                 (its contents are copied into the launch; L <= 64).
+ *   h_in        : chained != 0: [T, H], the input of layer 0;
+ *                 chained == 0: [L, T, H], layer l's own input.
+ *   h_out [L,T,H]: every layer's output (chained: layer l's output is layer
+ *                 l+1's input).
+ *   1 <= T <= 8, H <= 4096, T * H <= 24576.  Needs cooperative launch.
+ * The workspace (moe_decode_stack_workspace_size) must stay untouched until
+ * the kernel finishes; its first bytes are reset by every call.  Every wait in
+ * the kernel is bounded (~1 s); if one runs out the kernel records a code in
+ * the workspace and returns early (outputs are then invalid) -- read it with
+ * moe_decode_stack_status.
+ */
+MOE_API size_t moe_decode_stack_workspace_size(const moe_layer_w *w, int T);
+
+MOE_API int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained, uint16_t *h_out,
+                             int T, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream);
+
+/* Synchronous: reads the device error code a moe_decode_stack call left in
+ * `ws` (after waiting for the device).  MOE_OK, or MOE_EDEVICE with the reason
+ * in moe_last_error(). */
+MOE_API int moe_decode_stack_status(const void *ws);
 
 /*
  * moe_layer_forward for callers that cannot allocate device memory.  (The

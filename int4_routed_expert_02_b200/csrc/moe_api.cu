@@ -331,4 +331,82 @@ int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_ou
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
 }
 
+size_t moe_decode_stack_workspace_size(const moe_layer_w *w, int T) {
+    if (check_dims("moe_decode_stack_workspace_size", w) || T < 1 || T > moe::decode_stack_max_tokens()) return 0;
+    return moe::decode_stack_ws_bytes(w, T);
+}
+
+int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained, uint16_t *h_out, int T,
+                     void *ws, size_t ws_bytes, const moe_opts *opts, void *stream) {
+    const char *fn = "moe_decode_stack";
+    g_err.clear();
+    if (!layers) return fail(MOE_EINVAL, "%s: layers is NULL", fn);
+    if (L < 1 || L > moe::decode_stack_max_layers())
+        return fail(MOE_EINVAL, "%s: L=%d must be in [1, %d]", fn, L, moe::decode_stack_max_layers());
+    if (T < 0 || T > moe::decode_stack_max_tokens())
+        return fail(MOE_EINVAL, "%s: T=%d must be in [0, %d]", fn, T, moe::decode_stack_max_tokens());
+    const moe_layer_w &w0 = layers[0];
+    for (int l = 0; l < L; ++l) {
+        const moe_layer_w *w = &layers[l];
+        if (int rc = check_dims(fn, w)) return rc;
+        if (w->H != w0.H || w->E != w0.E || w->k != w0.k || w->I != w0.I || w->Is != w0.Is)
+            return fail(MOE_EINVAL, "%s: layer %d has a different shape from layer 0", fn, l);
+        if (int rc = check_router_ptrs(fn, w)) return rc;
+        if (int rc = check_expert_ptrs(fn, w, 1)) return rc;
+    }
+    if (w0.H > 4096) return fail(MOE_EINVAL, "%s: H=%d exceeds 4096", fn, w0.H);
+    if (T * w0.H > moe::decode_stack_stage_floats())
+        return fail(MOE_EINVAL, "%s: T*H=%d exceeds %d", fn, T * w0.H, moe::decode_stack_stage_floats());
+    const moe_opts o = resolve_opts(opts);
+    if (int rc = check_opts(fn, o)) return rc;
+    CHECK_PTR(h_in);
+    CHECK_PTR(h_out);
+    if (T == 0) return MOE_OK;
+    const size_t need = moe::decode_stack_ws_bytes(&w0, T);
+    if (!ws) return fail(MOE_EWORKSPACE, "%s: workspace is NULL (need %zu bytes)", fn, need);
+    if (!aligned16(ws)) return fail(MOE_EALIGN, "%s: workspace is not 16-byte aligned", fn);
+    if (ws_bytes < need) return fail(MOE_EWORKSPACE, "%s: workspace has %zu bytes, needs %zu", fn, ws_bytes, need);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    cudaError_t e = st ? cudaStreamGetDevice(st, &dev) : cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    static std::mutex mu;
+    static int grids[64] = {0};
+    int grid = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 0 || dev >= 64) return fail(MOE_EINVAL, "%s: device %d out of range", fn, dev);
+        if (grids[dev] == 0) {
+            int coop = 0;
+            e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+            if (e != cudaSuccess) return cuda_fail(e, fn);
+            if (!coop) return fail(MOE_EINVAL, "%s: device %d has no cooperative launch", fn, dev);
+            e = moe::decode_stack_grid(dev, &grids[dev]);
+            if (e != cudaSuccess) return cuda_fail(e, fn);
+            if (grids[dev] <= 0) return fail(MOE_EINVAL, "%s: the decode kernel does not fit on an SM", fn);
+        }
+        grid = grids[dev];
+    }
+    if (!moe::decode_stack_fits(&w0, T, grid))
+        return fail(MOE_EINVAL, "%s: T=%d with H=%d, E=%d does not fit the kernel's shared memory", fn, T, w0.H, w0.E);
+    e = moe::launch_decode_stack(layers, L, h_in, chained, h_out, T, ws, o, grid, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_decode_stack_status(const void *ws) {
+    const char *fn = "moe_decode_stack_status";
+    g_err.clear();
+    if (!ws) return fail(MOE_EINVAL, "%s: workspace is NULL", fn);
+    int code = 0;
+    cudaError_t e = cudaMemcpy(&code, static_cast<const char *>(ws) + moe::decode_stack_status_offset(), sizeof code,
+                               cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    if (code != 0) {
+        static const char *what[] = {"", "grid barrier timed out", "wait for weights timed out",
+                                     "wait for a free ring slot timed out"};
+        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 4) ? what[code] : "?");
+    }
+    return MOE_OK;
+}
+
 }  // extern "C"

@@ -37,6 +37,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
+// fp32 -> bf16 bits, round to nearest even, with integer operations only
+// (keeps the conversion off the special-function pipe).  Finite inputs.
+__device__ __forceinline__ uint32_t f32_to_bf16_bits_alu(float x) {
+    const uint32_t u = __float_as_uint(x);
+    return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
+}
+
 template <typename T>
 __device__ __forceinline__ T warp_sum(T v) {
 #pragma unroll
@@ -58,20 +65,43 @@ __device__ __forceinline__ T block_sum(T v, T *red) {
 }
 
 // ---------------------------------------------------------------------------
-// 4-bit code decoding for the dequant-GEMV.
+// 4-bit code decoding for the dequant-GEMV ("subnormal" decode).
 //
-// For a packed word holding codes q_0..q_7 (q_j in bits 4j..4j+3), build for
-// each j the fp32 value f_j = 1 + q_j * c_j, exactly, by OR-ing the code into
-// the fraction of 1.0f at bits 16..19 (c = 2^-7) or 12..15 (c = 2^-11).  With
-// the input pre-scaled as x'_j = x_j / c_j,
-//     sum_j f_j * x'_j = sum_j x'_j + sum_j q_j * x_j,
-// so one FMA per code accumulates q*x, and the per-chunk constant sum_j x'_j
-// is subtracted once.  c_j depends only on j = column % 8:
-//     j : 0     1      2     3      4     5      6     7
-//     c : 2^-7  2^-11  2^-7  2^-11  2^-7  2^-11  2^-7  2^-7
+// A packed word holds codes q_0..q_7, q_j in bits 4j..4j+3.  With every other
+// bit cleared, the word read as an fp32 is exactly q_j * 2^(4j - 149): a
+// subnormal for j <= 4, and for j = 5 still q * 2^-129 because the code's top
+// bit then lands in the exponent's lowest bit, where the smallest normal
+// numbers continue the subnormal spacing (2^-126 + f * 2^-149).  Codes 6 and 7
+// would land in the exponent proper, so they are first shifted down by 12
+// bits, to the positions of codes 3 and 4.  One AND per code (plus one shift
+// per word) therefore yields an fp32 proportional to the code, and with the
+// input pre-scaled by 2^(100 - 4p) (p = the position the code is read at) the
+// product with the code is exactly q * x * 2^-49 -- no offset, no
+// cancellation.  Accumulated sums are multiplied back by 2^49 once per group.
+// fp32 subnormals are handled at full speed by FFMA (no flush-to-zero: the
+// library is built without fast-math).
 // ---------------------------------------------------------------------------
+constexpr float kCodeUnscale = 0x1p49f;
+
+__host__ __device__ constexpr int code_pos(int j) { return j < 6 ? j : j - 3; }
+
 __host__ __device__ constexpr float code_prescale(int j) {
-    return (j == 1 || j == 3 || j == 5) ? 2048.0f : 128.0f;
+    return code_pos(j) == 0 ? 0x1p100f
+         : code_pos(j) == 1 ? 0x1p96f
+         : code_pos(j) == 2 ? 0x1p92f
+         : code_pos(j) == 3 ? 0x1p88f
+         : code_pos(j) == 4 ? 0x1p84f
+                            : 0x1p80f;
+}
+
+// 1 / code_prescale(j), exact (a power of two).
+__host__ __device__ constexpr float code_unprescale(int j) {
+    return code_pos(j) == 0 ? 0x1p-100f
+         : code_pos(j) == 1 ? 0x1p-96f
+         : code_pos(j) == 2 ? 0x1p-92f
+         : code_pos(j) == 3 ? 0x1p-88f
+         : code_pos(j) == 4 ? 0x1p-84f
+                            : 0x1p-80f;
 }
 
 struct Decoded8 {
@@ -79,45 +109,38 @@ struct Decoded8 {
 };
 
 __device__ __forceinline__ Decoded8 decode_word(uint32_t w) {
-    constexpr uint32_t kOne = 0x3f800000u;
-    const uint32_t w8 = w << 8, w16 = w << 16, v8 = w >> 8, v12 = w >> 12;
+    const uint32_t v = w >> 12;
     Decoded8 d;
-    d.f[0] = __uint_as_float((w16 & 0x000f0000u) | kOne);
-    d.f[1] = __uint_as_float((w8 & 0x0000f000u) | kOne);
-    d.f[2] = __uint_as_float((w8 & 0x000f0000u) | kOne);
-    d.f[3] = __uint_as_float((w & 0x0000f000u) | kOne);
-    d.f[4] = __uint_as_float((w & 0x000f0000u) | kOne);
-    d.f[5] = __uint_as_float((v8 & 0x0000f000u) | kOne);
-    d.f[6] = __uint_as_float((v8 & 0x000f0000u) | kOne);
-    d.f[7] = __uint_as_float((v12 & 0x000f0000u) | kOne);
+    d.f[0] = __uint_as_float(w & 0x0000000fu);
+    d.f[1] = __uint_as_float(w & 0x000000f0u);
+    d.f[2] = __uint_as_float(w & 0x00000f00u);
+    d.f[3] = __uint_as_float(w & 0x0000f000u);
+    d.f[4] = __uint_as_float(w & 0x000f0000u);
+    d.f[5] = __uint_as_float(w & 0x00f00000u);
+    d.f[6] = __uint_as_float(v & 0x0000f000u);
+    d.f[7] = __uint_as_float(v & 0x000f0000u);
     return d;
 }
 
 // Two fp32 FMAs in one packed instruction (sm_100): (a.x*b.x + c.x, a.y*b.y + c.y).
+// The register pairs are formed inside the asm so the compiler can allocate
+// them as pairs.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    unsigned long long ra, rb, rc, rd;
-    ra = (unsigned long long)__float_as_uint(a.x) | ((unsigned long long)__float_as_uint(a.y) << 32);
-    rb = (unsigned long long)__float_as_uint(b.x) | ((unsigned long long)__float_as_uint(b.y) << 32);
-    rc = (unsigned long long)__float_as_uint(c.x) | ((unsigned long long)__float_as_uint(c.y) << 32);
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
-    return make_float2(__uint_as_float((uint32_t)rd), __uint_as_float((uint32_t)(rd >> 32)));
+    asm("{\n .reg .b64 ra, rb, rc;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%0, %1};\n"
+        " fma.rn.f32x2 rc, ra, rb, rc;\n mov.b64 {%0, %1}, rc;\n}"
+        : "+f"(c.x), "+f"(c.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return c;
 }
 
-// 16 bytes = 32 codes of one row against 32 pre-scaled inputs (two float4 x
-// 4).  Returns sum_j f_j * x'_j accumulated as two interleaved partial sums.
-__device__ __forceinline__ float dot_chunk(const uint4 q, const float4 *xp) {
-    float2 acc = make_float2(0.f, 0.f);
-    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const Decoded8 d = decode_word(words[i]);
-        const float4 xa = xp[2 * i], xb = xp[2 * i + 1];
-        acc = ffma2(make_float2(d.f[0], d.f[1]), make_float2(xa.x, xa.y), acc);
-        acc = ffma2(make_float2(d.f[2], d.f[3]), make_float2(xa.z, xa.w), acc);
-        acc = ffma2(make_float2(d.f[4], d.f[5]), make_float2(xb.x, xb.y), acc);
-        acc = ffma2(make_float2(d.f[6], d.f[7]), make_float2(xb.z, xb.w), acc);
-    }
-    return acc.x + acc.y;
+// One word (8 codes) against 8 pre-scaled inputs, into two packed accumulators.
+__device__ __forceinline__ void dot_word(uint32_t w, const float *xp, float2 &a0, float2 &a1) {
+    const Decoded8 d = decode_word(w);
+    const float4 xa = reinterpret_cast<const float4 *>(xp)[0], xb = reinterpret_cast<const float4 *>(xp)[1];
+    a0 = ffma2(make_float2(d.f[0], d.f[1]), make_float2(xa.x, xa.y), a0);
+    a1 = ffma2(make_float2(d.f[2], d.f[3]), make_float2(xa.z, xa.w), a1);
+    a0 = ffma2(make_float2(d.f[4], d.f[5]), make_float2(xb.x, xb.y), a0);
+    a1 = ffma2(make_float2(d.f[6], d.f[7]), make_float2(xb.z, xb.w), a1);
 }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const uint32_t *p) {

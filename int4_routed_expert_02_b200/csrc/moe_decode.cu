@@ -1,0 +1,1266 @@
+// moe_decode.cu -- persistent decode kernel: a stack of MoE layers for a small
+// token batch (T <= 8) in ONE cooperative launch, one CTA per SM.
+//
+// Per layer (TurboFieldfare introduction page, discuss.pytorch.kr, section
+// "TurboFieldfare's expert streaming structure": router -> routed experts +
+// shared expert -> weighted combine -> normalisation, residual, layer scalar;
+// weights MLX affine, section "How TurboFieldfare saves memory"):
+//
+//   P0  finish the previous layer: m = sum_s w_s y_s + shared, post-norm,
+//       residual, layer scalar (every CTA, redundantly; CTA 0 writes it out),
+//       and the RMS the router needs
+//   P1  router logits in fp64 for this CTA's share of the E experts; its
+//       router rows and router_scale were bulk-copied into shared memory at
+//       the start of the layer, overlapping P0
+//   --- grid barrier ---
+//   P2  top-k + softmax * per_expert_scale and bucketing, by rank counting
+//       (every CTA, redundantly, so no barrier is needed before the experts),
+//       and this CTA's job tables for the two expert phases
+//   P2' gate/up dequant-GEMV jobs (32 rows x one K part of <= 16 groups of
+//       both matrices, streamed in stages of <= 8 groups), partial sums to
+//       global
+//   --- grid barrier ---
+//   P3  down dequant-GEMV jobs (32 rows x <= 16 groups); each CTA forms the
+//       SwiGLU input a = silu(sum g) * (sum u) it needs
+//   --- grid barrier ---
+//
+// Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
+// into a ring of mbarrier-guarded slots, issued by one producer thread ahead
+// of 16 consumer warps.  Once the top-k is known each CTA also asks L2 to
+// prefetch the down-projection weights of its later jobs, and during the down
+// phase its share of the next layer's shared-expert weights, so HBM keeps
+// streaming across the grid barriers.  The dot products use the subnormal
+// code decode of moe_common.cuh (one AND + one FMA per code).  Loops keep the
+// special-function pipe idle: no runtime integer division, conversion or
+// reciprocal per element (job tables are built once per layer, the ring
+// position is advanced incrementally, bf16 rounding uses integer arithmetic).
+//
+// Every wait is bounded (grid barrier and mbarriers: ~1 s of globaltimer); on
+// a timeout the kernel records an error code in the workspace, stops taking
+// work, lets its own bulk copies land and returns.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace dec {
+
+constexpr int kCWarps = 16;                   // consumer warps
+constexpr int kWarps = kCWarps + 1;           // + the producer warp
+constexpr int kThreads = kWarps * 32;
+constexpr int kProducerWarp = kCWarps;
+constexpr int kMaxStages = 9;                 // ring slots: as many as fit beside the input stage
+constexpr int kStageGroups = 8;               // gate/up stage: <= 8 groups of each of the two matrices
+constexpr int kGuPartGroups = 16;             // gate/up job: one K part of <= 16 groups
+constexpr int kDnGroups = 16;                 // down job: <= 16 groups, one stage
+constexpr int kCodeBytesPerGroup = 1024;      // 32 rows x 64 codes x 4 bits
+constexpr int kSbBytesPerGroup = 128;         // 32 rows x (scale, bias)
+constexpr int kSlotBytes = 16 * (kCodeBytesPerGroup + kSbBytesPerGroup);  // 18432
+constexpr int kMaxT = 8;
+constexpr int kStageFloats = 24576;           // largest input stage (T * H)
+constexpr int kPoolBytes = 4 * kSlotBytes + kStageFloats * 4;  // ring + input stage share this pool
+constexpr int kMaxXs = 768;
+constexpr int kMaxLayers = 64;
+constexpr int kMaxPairs = kMaxT * kMaxK;
+constexpr int kMaxJobs = 128;                 // per CTA and phase
+constexpr int kRed = 16 * kMaxT * 32;         // one reduction buffer: [16 warps][kMaxT][32]
+constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
+
+constexpr int kErrGridBarrier = 1, kErrFull = 2, kErrEmpty = 3;
+
+struct Params {
+    moe_layer_w layers[kMaxLayers];
+    const uint16_t *h_in;  // [T,H] (chained) or [L,T,H]
+    uint16_t *h_out;       // [L,T,H]: every layer's output
+    int L, T, chained, post_norm;
+    float layer_scalar, eps;
+    int H, E, k, I, Is, Kmax, R;
+    int nkp, ndp_r, ndp_s;
+    int nslots;      // ring slots (the rest of the pool is the input stage)
+    int stage_all;   // 1: the down phase stages every slot's SwiGLU input at once
+    unsigned *bar;
+    int *err;
+    double *logits;  // [T,E]
+    float *gu_part;  // [nkp][R][2][Kmax]: gate (0) and up (1) partial sums per K part
+    float *y;        // [ndp_r][T*k][H]
+    float *sh;       // [ndp_s][T][H]
+};
+
+// One job of an expert phase: 32 rows (row block rb) x groups [g0, g1) of the
+// shared expert (slot 0) or of routed expert e (slot >= 1), for n tokens
+// starting at bucketed position seg0.
+struct JobDesc {
+    int16_t slot, rb, part, g0, g1, n;
+    int32_t seg0, e;
+};
+
+struct Smem {
+    alignas(128) unsigned char pool[kPoolBytes];  // ring slots, then the input stage
+    alignas(8) unsigned long long full[kMaxStages];
+    alignas(8) unsigned long long empty[kMaxStages];
+    alignas(8) unsigned long long rbar;  // router copies of the current layer
+    float *stage;                        // input stage (inside the pool, after the ring)
+    alignas(16) float xs[kMaxXs];        // sum of x per 32-column chunk
+    alignas(16) float red[2][kRed];
+    JobDesc gujob[kMaxJobs], dnjob[kMaxJobs];
+    int ngu, ndn, gu_stages;
+    double selv[kMaxPairs];
+    double pe[kMaxPairs];
+    float wts[kMaxPairs];
+    int idx[kMaxPairs];
+    int perm[kMaxPairs];
+    int poff[kMaxPairs], pcnt[kMaxPairs];
+    unsigned char first[kMaxPairs];
+    int act_e[kMaxPairs], act_off[kMaxPairs], act_n[kMaxPairs];
+    int tokrow[kMaxPairs];  // bucketed position j -> row offset (token * H) of its input
+    int tokrow_sh[kMaxT];   // shared expert: token t -> t * H
+    int rsoff[kMaxT + kMaxPairs + 1];  // stage-all: start of each rowset's SwiGLU input in the stage
+    int nact;
+    double rpart[128];
+    float rms[kMaxT];
+    float rinv[kMaxT];
+    int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
+    int flag;
+};
+
+// Position in the ring: stage sequence number q, its slot s and phase parity ph.
+struct Ring {
+    unsigned q;
+    int s;
+    unsigned ph;
+};
+
+__device__ __forceinline__ void ring_next(Ring &r, int ns) {
+    ++r.q;
+    if (++r.s == ns) {
+        r.s = 0;
+        r.ph ^= 1u;
+    }
+}
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long *b, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long *b, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(unsigned long long *b, unsigned parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ int ldcg_int(const int *p) { return __ldcg(p); }
+
+// Bounded wait for the phase with `parity` of mbarrier `b` to complete.
+__device__ bool mbar_wait(unsigned long long *b, unsigned parity, int *err, int code) {
+    if (mbar_test(b, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (unsigned it = 1;; ++it) {
+        if (mbar_test(b, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (ldcg_int(err) != 0) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                atomicCAS(err, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait used only when draining: ignores the error flag.
+__device__ void mbar_drain(unsigned long long *b, unsigned parity) {
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_test(b, parity)) {
+        if (globaltimer() - t0 > kWaitNs) return;
+    }
+}
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes, unsigned long long *b) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(b))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *src, unsigned bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Prefetch [p, p + bytes) into L2 in pieces of at most 64 KiB (16-byte units).
+__device__ __forceinline__ void prefetch_range(const void *p, size_t bytes) {
+    const char *c = static_cast<const char *>(p);
+    while (bytes >= 16) {
+        const unsigned n = (unsigned)(bytes > 65536 ? 65536 : (bytes & ~(size_t)15));
+        prefetch_l2(c, n);
+        c += n;
+        bytes -= n;
+    }
+}
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCWarps * 32) : "memory"); }
+
+// Grid-wide barrier number `nth` (1, 2, ...) on a monotonically increasing
+// counter; bounded.  Returns false (in every thread of the CTA alike) if any
+// CTA recorded an error.
+__device__ bool grid_sync(const Params &P, unsigned nth, int *verdict) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(P.bar, 1u);
+        const unsigned target = nth * gridDim.x;
+        const unsigned long long t0 = globaltimer();
+        for (unsigned it = 0;; ++it) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(P.bar) : "memory");
+            if (v >= target) break;
+            if ((it & 63u) == 63u) {
+                if (ldcg_int(P.err) != 0) break;
+                if (globaltimer() - t0 > kWaitNs) {
+                    atomicCAS(P.err, 0, kErrGridBarrier);
+                    break;
+                }
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+        *verdict = ldcg_int(P.err) == 0;
+    }
+    __syncthreads();
+    return *verdict != 0;
+}
+
+// ------------------------------------------------------------------ jobs
+
+// Job j of the gate/up phase (all divisions happen here, once per job).
+__device__ JobDesc make_gu_job(const Params &P, const Smem &S, int j) {
+    JobDesc J;
+    const int GH = P.H / 64;
+    const int A = (P.Is / 32) * P.nkp;
+    int part;
+    if (j < A) {
+        J.slot = 0;
+        J.rb = (int16_t)(j / P.nkp);
+        part = j - J.rb * P.nkp;
+        J.n = (int16_t)P.T;
+        J.seg0 = 0;
+        J.e = -1;
+    } else {
+        const int B = (P.I / 32) * P.nkp;
+        const int jj = j - A;
+        const int i = jj / B;
+        const int r = jj - i * B;
+        J.slot = (int16_t)(1 + i);
+        J.rb = (int16_t)(r / P.nkp);
+        part = r - J.rb * P.nkp;
+        J.seg0 = S.act_off[i];
+        J.n = (int16_t)S.act_n[i];
+        J.e = S.act_e[i];
+    }
+    J.part = (int16_t)part;
+    J.g0 = (int16_t)(GH * part / P.nkp);
+    J.g1 = (int16_t)(GH * (part + 1) / P.nkp);
+    return J;
+}
+
+// Job j of the down phase.
+__device__ JobDesc make_dn_job(const Params &P, const Smem &S, int j) {
+    JobDesc J;
+    const int RBH = P.H / 32;
+    const int A = P.ndp_s * RBH;
+    if (j < A) {
+        const int part = j / RBH;
+        J.slot = 0;
+        J.part = (int16_t)part;
+        J.rb = (int16_t)(j - part * RBH);
+        J.n = (int16_t)P.T;
+        J.seg0 = 0;
+        J.e = -1;
+        const int G = P.Is / 64;
+        J.g0 = (int16_t)(G * part / P.ndp_s);
+        J.g1 = (int16_t)(G * (part + 1) / P.ndp_s);
+    } else {
+        const int B = P.ndp_r * RBH;
+        const int jj = j - A;
+        const int i = jj / B;
+        const int r = jj - i * B;
+        const int part = r / RBH;
+        J.slot = (int16_t)(1 + i);
+        J.part = (int16_t)part;
+        J.rb = (int16_t)(r - part * RBH);
+        J.seg0 = S.act_off[i];
+        J.n = (int16_t)S.act_n[i];
+        J.e = S.act_e[i];
+        const int G = P.I / 64;
+        J.g0 = (int16_t)(G * part / P.ndp_r);
+        J.g1 = (int16_t)(G * (part + 1) / P.ndp_r);
+    }
+    return J;
+}
+
+// Weight pointers of a gate/up job (matrix 0 = gate, 1 = up).
+__device__ __forceinline__ void gu_ptrs(const Params &P, const moe_layer_w &W, const JobDesc &J, const uint32_t *(&q)[2],
+                                        const uint32_t *(&sb)[2]) {
+    const size_t CH = P.H / 32, GH = P.H / 64;
+    if (J.slot == 0) {
+        q[0] = W.sh_gate.q + (size_t)J.rb * CH * 128;
+        q[1] = W.sh_up.q + (size_t)J.rb * CH * 128;
+        sb[0] = W.sh_gate.sb + (size_t)J.rb * GH * 32;
+        sb[1] = W.sh_up.sb + (size_t)J.rb * GH * 32;
+    } else {
+        const size_t mrb = (size_t)J.e * (P.I / 32) + J.rb;
+        q[0] = W.gate.q + mrb * CH * 128;
+        q[1] = W.up.q + mrb * CH * 128;
+        sb[0] = W.gate.sb + mrb * GH * 32;
+        sb[1] = W.up.sb + mrb * GH * 32;
+    }
+}
+
+// Weight pointers of a down job.
+__device__ __forceinline__ void dn_ptrs(const Params &P, const moe_layer_w &W, const JobDesc &J, const uint32_t *&q,
+                                        const uint32_t *&sb) {
+    if (J.slot == 0) {
+        q = W.sh_down.q + (size_t)J.rb * (P.Is / 32) * 128;
+        sb = W.sh_down.sb + (size_t)J.rb * (P.Is / 64) * 32;
+    } else {
+        const size_t mrb = (size_t)J.e * (P.H / 32) + J.rb;
+        q = W.down.q + mrb * (P.I / 32) * 128;
+        sb = W.down.sb + mrb * (P.I / 64) * 32;
+    }
+}
+
+// rowset of the tt-th token of a job (shared: the token; routed: T + bucketed position)
+__device__ __forceinline__ int job_rowset(const Params &P, const JobDesc &J, int tt) {
+    return J.slot == 0 ? tt : P.T + J.seg0 + tt;
+}
+
+// Producer: the copies that fill ring slot s with groups [g0, g1) of nmat matrices.
+// Layout in the slot: codes of matrix 0 (ng KiB), codes of matrix 1, then the
+// (scale, bias) words of matrix 0 (ng * 128 B), of matrix 1.
+__device__ __forceinline__ void issue_stage(Smem &S, int s, const uint32_t *const *q, const uint32_t *const *sb,
+                                            int nmat, int g0, int g1) {
+    const int ng = g1 - g0;
+    const unsigned cb = (unsigned)ng * kCodeBytesPerGroup, sbb = (unsigned)ng * kSbBytesPerGroup;
+    unsigned char *slot = S.pool + (size_t)s * kSlotBytes;
+    mbar_expect_tx(&S.full[s], nmat * (cb + sbb));
+    for (int m = 0; m < nmat; ++m) {
+        bulk_g2s(slot + m * cb, q[m] + (size_t)g0 * 256, cb, &S.full[s]);
+        bulk_g2s(slot + nmat * cb + m * sbb, sb[m] + (size_t)g0 * 32, sbb, &S.full[s]);
+    }
+}
+
+__device__ __forceinline__ void prefetch_dn_jobs(const Params &P, const Smem &S, const moe_layer_w &W) {
+    for (int d = 0; d < S.ndn; ++d) {
+        const JobDesc D = S.dnjob[d];
+        const uint32_t *dq, *dsb;
+        dn_ptrs(P, W, D, dq, dsb);
+        const int ng = D.g1 - D.g0;
+        prefetch_l2(dq + (size_t)D.g0 * 256, (unsigned)ng * kCodeBytesPerGroup);
+        prefetch_l2(dsb + (size_t)D.g0 * 32, (unsigned)ng * kSbBytesPerGroup);
+    }
+}
+
+// ------------------------------------------------------------------ dot products
+
+// One (matrix, group) of a job for tokens [t0, t0 + n), n <= NT <= 2: lanes
+// are the 32 rows.  w: this lane's 64 codes of the group; s (already times
+// 2^49) and b: its scale and bias.  The input of token tt starts at
+// x + off(tt), its chunk sums at xsum + off(tt) / 32, where off(tt) =
+// tokrow[tt] (gathered tokens) or tt * stride (when tokrow is null).
+template <int NT>
+__device__ __forceinline__ void group_dot(const uint32_t (&w)[8], float s, float b, const float *x,
+                                          const float *xsum, const int *tokrow, int stride, int t0, int n,
+                                          float (&acc)[4]) {
+    constexpr int NA = NT == 1 ? 2 : 1;  // packed accumulators per token: 2 for ILP when alone
+    float2 a[NT][NA];
+    int xo[NT];
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) {
+#pragma unroll
+        for (int z = 0; z < NA; ++z) a[tt][z] = make_float2(0.f, 0.f);
+        xo[tt] = tt < n ? (tokrow ? tokrow[t0 + tt] : (t0 + tt) * stride) : 0;
+    }
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+        const Decoded8 f = decode_word(w[wi]);
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+            if (tt < n) {
+                const float4 *x4 = reinterpret_cast<const float4 *>(x + xo[tt] + wi * 8);
+                const float4 xa = x4[0], xb = x4[1];
+                a[tt][0] = ffma2(make_float2(f.f[0], f.f[1]), make_float2(xa.x, xa.y), a[tt][0]);
+                a[tt][NA - 1] = ffma2(make_float2(f.f[2], f.f[3]), make_float2(xa.z, xa.w), a[tt][NA - 1]);
+                a[tt][0] = ffma2(make_float2(f.f[4], f.f[5]), make_float2(xb.x, xb.y), a[tt][0]);
+                a[tt][NA - 1] = ffma2(make_float2(f.f[6], f.f[7]), make_float2(xb.z, xb.w), a[tt][NA - 1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) {
+        if (tt < n) {
+            float d = a[tt][0].x + a[tt][0].y;
+            if (NA == 2) d += a[tt][NA - 1].x + a[tt][NA - 1].y;
+            const int c = xo[tt] >> 5;
+            acc[tt] = fmaf(s, d, fmaf(b, xsum[c] + xsum[c + 1], acc[tt]));
+        }
+    }
+}
+
+// One (matrix, group) for the n <= 8 tokens of a job, in calls of at most two
+// tokens (codes are decoded once per call); acc[0] holds tokens 0-3, acc[1] 4-7.
+__device__ __forceinline__ void group_dot_n(const unsigned char *codes, uint32_t sbw, const float *x,
+                                            const float *xsum, const int *tokrow, int stride, int n,
+                                            float (&acc)[2][4], int lane) {
+    const uint4 c0 = reinterpret_cast<const uint4 *>(codes)[lane];
+    const uint4 c1 = reinterpret_cast<const uint4 *>(codes + 512)[lane];
+    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const float s = bf16_bits_to_float(sbw & 0xffffu) * kCodeUnscale, b = bf16_bits_to_float(sbw >> 16);
+    if (n == 1) {
+        group_dot<1>(w, s, b, x, xsum, tokrow, stride, 0, 1, acc[0]);
+        return;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (4 * h < n) {
+            float p0[4] = {acc[h][0], acc[h][1], 0.f, 0.f}, p1[4] = {acc[h][2], acc[h][3], 0.f, 0.f};
+            group_dot<2>(w, s, b, x, xsum, tokrow, stride, 4 * h, min(2, n - 4 * h), p0);
+            if (4 * h + 2 < n) group_dot<2>(w, s, b, x, xsum, tokrow, stride, 4 * h + 2, min(2, n - 4 * h - 2), p1);
+            acc[h][0] = p0[0];
+            acc[h][1] = p0[1];
+            acc[h][2] = p1[0];
+            acc[h][3] = p1[1];
+        }
+    }
+}
+
+// ------------------------------------------------------------------ phases
+
+// Input rows of a layer straight from global memory (bf16) into S.stage, and their RMS.
+__device__ __noinline__ void load_input(const Params &P, Smem &S, const uint16_t *h) {
+    const int T = P.T, H = P.H, H2 = H / 2;
+    float *stage = S.stage;
+    for (int t = 0; t < T; ++t) {
+        float ss = 0.f;
+        for (int i = threadIdx.x; i < H2; i += blockDim.x) {
+            const uint32_t v = __ldcg(reinterpret_cast<const unsigned int *>(h + (size_t)t * H) + i);
+            const float a = bf16_bits_to_float(v & 0xffffu), b = bf16_bits_to_float(v >> 16);
+            stage[(size_t)t * H + 2 * i] = a;
+            stage[(size_t)t * H + 2 * i + 1] = b;
+            ss = fmaf(a, a, fmaf(b, b, ss));
+        }
+        ss = block_sum(ss, S.red[0]);
+        if (threadIdx.x == 0) {
+            S.rms[t] = sqrtf(ss / (float)H + P.eps);
+            S.rinv[t] = 1.0f / S.rms[t];
+        }
+    }
+    __syncthreads();
+}
+
+// P0: output of layer lp (m from its y/sh parts, post-norm, residual, scalar)
+// into S.stage as floats, with its RMS; CTA 0 also writes it to h_out[lp].
+// All global loads of a token are issued before they are used; H/4 <= 1024 <
+// 2 * blockDim, so two float4 per thread cover a row.
+__device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
+    const int T = P.T, H = P.H, k = P.k, Tk = T * k, H4 = H / 4, ndp_r = P.ndp_r, ndp_s = P.ndp_s;
+    const float *y = P.y, *shp = P.sh;
+    const uint16_t *hprev = (P.chained && lp > 0) ? P.h_out + (size_t)(lp - 1) * T * H
+                                                  : (P.chained ? P.h_in : P.h_in + (size_t)lp * T * H);
+    uint16_t *out = P.h_out + (size_t)lp * T * H;
+    float *stage = S.stage;
+    const float scalar = P.layer_scalar;
+    for (int t = 0; t < T; ++t) {
+        float4 mreg[2];
+        uint2 hreg[2];
+        float ss = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i4 = threadIdx.x + r * blockDim.x;
+            mreg[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            hreg[r] = make_uint2(0u, 0u);
+            if (i4 < H4) {
+                hreg[r] = __ldcg(reinterpret_cast<const uint2 *>(hprev + (size_t)t * H) + i4);
+                float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+                // routed slots, 8 loads in flight at a time; each slot's K parts summed, then weighted
+                for (int b0 = 0; b0 < k; b0 += 8) {
+                    float4 v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        v[u] = b0 + u < k ? __ldcg(reinterpret_cast<const float4 *>(y + ((size_t)t * k + b0 + u) * H) + i4)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int dp = 1; dp < ndp_r; ++dp) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (b0 + u < k) {
+                                const float4 vv = __ldcg(reinterpret_cast<const float4 *>(
+                                                             y + ((size_t)dp * Tk + t * k + b0 + u) * H) + i4);
+                                v[u].x += vv.x;
+                                v[u].y += vv.y;
+                                v[u].z += vv.z;
+                                v[u].w += vv.w;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float w = b0 + u < k ? S.wts[t * k + b0 + u] : 0.f;
+                        m.x = fmaf(w, v[u].x, m.x);
+                        m.y = fmaf(w, v[u].y, m.y);
+                        m.z = fmaf(w, v[u].z, m.z);
+                        m.w = fmaf(w, v[u].w, m.w);
+                    }
+                }
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    v[u] = u < ndp_s ? __ldcg(reinterpret_cast<const float4 *>(shp + ((size_t)u * T + t) * H) + i4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int u = 4; u < ndp_s; ++u) {
+                    const float4 vv = __ldcg(reinterpret_cast<const float4 *>(shp + ((size_t)u * T + t) * H) + i4);
+                    m.x += vv.x;
+                    m.y += vv.y;
+                    m.z += vv.z;
+                    m.w += vv.w;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    m.x += v[u].x;
+                    m.y += v[u].y;
+                    m.z += v[u].z;
+                    m.w += v[u].w;
+                }
+                mreg[r] = m;
+                ss += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
+            }
+        }
+        ss = block_sum(ss, S.red[0]);
+        const float inv = P.post_norm ? 1.0f / sqrtf(ss / (float)H + P.eps) : 1.0f;
+        float ss2 = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i4 = threadIdx.x + r * blockDim.x;
+            if (i4 < H4) {
+                const float mv[4] = {mreg[r].x, mreg[r].y, mreg[r].z, mreg[r].w};
+                const uint32_t hv[2] = {hreg[r].x, hreg[r].y};
+                uint32_t o[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float hp = bf16_bits_to_float((hv[c >> 1] >> (16 * (c & 1))) & 0xffffu);
+                    o[c] = f32_to_bf16_bits_alu((hp + mv[c] * inv) * scalar);
+                    const float of = bf16_bits_to_float(o[c]);
+                    stage[(size_t)t * H + 4 * i4 + c] = of;
+                    ss2 = fmaf(of, of, ss2);
+                }
+                if (blockIdx.x == 0)
+                    reinterpret_cast<uint2 *>(out + (size_t)t * H)[i4] = make_uint2(o[0] | (o[1] << 16), o[2] | (o[3] << 16));
+            }
+        }
+        ss2 = block_sum(ss2, S.red[0]);
+        if (threadIdx.x == 0) {
+            S.rms[t] = sqrtf(ss2 / (float)H + P.eps);
+            S.rinv[t] = 1.0f / S.rms[t];
+        }
+    }
+    __syncthreads();
+}
+
+// Producer, at the start of layer l: router_scale, this CTA's router rows
+// [e0, e1) and a 16-byte-aligned superset of their scales and biases, into
+// the ring (idle until the top-k), completing on S.rbar (one phase per layer).
+__device__ void issue_router_copies(const Params &P, Smem &S, const moe_layer_w &W) {
+    const int E = P.E, H = P.H, G = H / 64;
+    const int e0 = (int)((long long)E * blockIdx.x / gridDim.x), e1 = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);
+    const int nrows = e1 - e0;
+    unsigned char *base = S.pool;
+    const unsigned rs_bytes = (unsigned)H * 2, rows_bytes = (unsigned)nrows * H;
+    const unsigned sb_lo = (unsigned)((size_t)e0 * G * 2) & ~15u;
+    const unsigned sb_hi = ((unsigned)((size_t)e1 * G * 2) + 15u) & ~15u;
+    const unsigned sb_bytes = nrows > 0 ? sb_hi - sb_lo : 0u;
+    S.rcopy[0] = e0;
+    S.rcopy[1] = nrows;
+    S.rcopy[2] = (int)sb_lo;
+    mbar_expect_tx(&S.rbar, rs_bytes + rows_bytes + 2 * sb_bytes);
+    // layout: [router_scale (H*2)] [rows (nrows*H)] [scales (sb_bytes)] [biases (sb_bytes)]
+    bulk_g2s(base, W.router_scale, rs_bytes, &S.rbar);
+    if (nrows > 0) {
+        bulk_g2s(base + rs_bytes, W.router_q + (size_t)e0 * (H / 4), rows_bytes, &S.rbar);
+        bulk_g2s(base + rs_bytes + rows_bytes, reinterpret_cast<const char *>(W.router_s) + sb_lo, sb_bytes, &S.rbar);
+        bulk_g2s(base + rs_bytes + rows_bytes + sb_bytes, reinterpret_cast<const char *>(W.router_b) + sb_lo, sb_bytes,
+                 &S.rbar);
+    }
+}
+
+// P1: router logits of this CTA's experts for every token, from the copies in
+// the ring.  The dot products accumulate in fp64 so that the top-k order does
+// not depend on summation order; the common factor 1 / (rms * sqrt(H)) of a
+// token's logits is applied last (it cannot change their order).
+__device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
+    const int T = P.T, H = P.H, E = P.E, G = H / 64, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    __syncthreads();  // S.rcopy written by the producer thread
+    const int e0 = S.rcopy[0], nrows = S.rcopy[1], sb_lo = S.rcopy[2];
+    const int items = nrows * T;
+    // every thread waits for the copies (they are issued even when nrows == 0);
+    // the verdict is made uniform before the barriers below
+    const bool got = __syncthreads_and(mbar_wait(&S.rbar, (unsigned)(l & 1), P.err, kErrFull)) != 0;
+    const unsigned char *base = S.pool;
+    const uint16_t *rsc = reinterpret_cast<const uint16_t *>(base);
+    const unsigned rows_bytes = (unsigned)nrows * H;
+    const unsigned sb_hi = ((unsigned)((size_t)(e0 + nrows) * G * 2) + 15u) & ~15u;
+    const unsigned sb_bytes = nrows > 0 ? sb_hi - (unsigned)sb_lo : 0u;
+    const unsigned char *rows = base + H * 2;
+    const int sb_skip = (int)((size_t)e0 * G * 2) - sb_lo;
+    const uint16_t *scs = reinterpret_cast<const uint16_t *>(rows + rows_bytes + sb_skip);
+    const uint16_t *bis = reinterpret_cast<const uint16_t *>(rows + rows_bytes + sb_bytes + sb_skip);
+    if (items > 0 && got) {
+        const int parts = items >= kWarps ? 1 : kWarps / items;
+        const int units = items * parts;
+        const int nch = H / 16;
+        const float *stage = S.stage;
+        for (int u = wid; u < units; u += kWarps) {
+            const int item = u / parts, part = u - item * parts;
+            const int er = item / T, t = item - er * T;
+            const int c0 = nch * part / parts, c1 = nch * (part + 1) / parts;
+            const float *h = stage + (size_t)t * H;
+            double acc = 0.0;
+            for (int c = c0 + lane; c < c1; c += 32) {
+                const uint4 q = reinterpret_cast<const uint4 *>(rows + (size_t)er * H)[c];
+                const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+                double dots[4] = {0.0, 0.0, 0.0, 0.0}, zss[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+                    for (int bi = 0; bi < 4; ++bi) {
+                        const int i = c * 16 + wi * 4 + bi;
+                        // h * router_scale is exact in fp32 (two bf16 values)
+                        const double z = (double)(h[i] * bf16_bits_to_float(rsc[i]));
+                        // the 8-bit code as a double: 2^52 + q read as fp64, minus 2^52 (exact)
+                        const double qd =
+                            __hiloint2double(0x43300000, (int)((words[wi] >> (8 * bi)) & 0xffu)) - 4503599627370496.0;
+                        dots[bi] = fma(qd, z, dots[bi]);
+                        zss[bi] += z;
+                    }
+                }
+                const double dot = (dots[0] + dots[1]) + (dots[2] + dots[3]);
+                const double zs = (zss[0] + zss[1]) + (zss[2] + zss[3]);
+                const int g = c >> 2;
+                acc += (double)bf16_bits_to_float(scs[er * G + g]) * dot + (double)bf16_bits_to_float(bis[er * G + g]) * zs;
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) S.rpart[u] = acc;
+        }
+        __syncthreads();
+        const double sqrt_h = sqrt((double)H);
+        for (int item = threadIdx.x; item < items; item += blockDim.x) {
+            double a = 0.0;
+            for (int p = 0; p < parts; ++p) a += S.rpart[item * parts + p];
+            const int er = item / T, t = item - er * T;
+            P.logits[(size_t)t * E + e0 + er] = a / ((double)S.rms[t] * sqrt_h);
+        }
+    }
+    __syncthreads();
+}
+
+// P2: top-k by rank counting (a logit's rank = how many logits beat it: larger,
+// or equal with a lower expert index), softmax * per_expert_scale, the
+// bucketing of the T*k pairs by rank counting too, and this CTA's job tables.
+// Every CTA.
+__device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_layer_w &W) {
+    const int T = P.T, E = P.E, k = P.k, n = T * k, H = P.H;
+    double *lg = reinterpret_cast<double *>(S.pool);  // ring is idle here: T*E doubles
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = __ldcg(P.logits + i);
+    __syncthreads();
+    for (int t = 0; t < T; ++t) {
+        const double2 *row = reinterpret_cast<const double2 *>(lg + (size_t)t * E);
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const double v = lg[(size_t)t * E + e];
+            int rank = 0;
+#pragma unroll 8
+            for (int j = 0; j < E / 2; ++j) {  // E is a multiple of 8
+                const double2 o = row[j];
+                rank += (o.x > v) | ((o.x == v) & (2 * j < e));
+                rank += (o.y > v) | ((o.y == v) & (2 * j + 1 < e));
+            }
+            if (rank < k) {
+                S.idx[t * k + rank] = e;
+                S.selv[t * k + rank] = v;
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < n) {
+        const int t = threadIdx.x / k;
+        S.pe[threadIdx.x] = exp(S.selv[threadIdx.x] - S.selv[t * k]);  // selv[t*k] is the token's maximum
+    }
+    __syncthreads();
+    if (threadIdx.x < n) {
+        const int p = threadIdx.x, t = p / k;
+        double z = 0.0;
+        for (int s = 0; s < k; ++s) z += S.pe[t * k + s];
+        const int e = S.idx[p];
+        S.wts[p] = (float)(S.pe[p] / z * (double)bf16_bits_to_float(W.per_expert_scale[e]));
+        // position of pair p among all pairs ordered by (expert, pair id)
+        int less = 0, eqb = 0, cnt = 0;
+        for (int q = 0; q < n; ++q) {
+            const int f = S.idx[q];
+            less += f < e;
+            eqb += (f == e) & (q < p);
+            cnt += f == e;
+        }
+        S.perm[less + eqb] = p;
+        S.tokrow[less + eqb] = t * H;
+        S.first[p] = eqb == 0;
+        S.poff[p] = less;
+        S.pcnt[p] = cnt;
+    }
+    if (threadIdx.x < T) S.tokrow_sh[threadIdx.x] = threadIdx.x * H;
+    __syncthreads();
+    if (threadIdx.x < n) {
+        const int p = threadIdx.x, e = S.idx[p];
+        int slot = 0, nact = 0;
+        for (int q = 0; q < n; ++q) {
+            slot += S.first[q] & (S.idx[q] < e);
+            nact += S.first[q];
+        }
+        if (S.first[p]) {  // one slot per distinct expert, ascending expert id
+            S.act_e[slot] = e;
+            S.act_off[slot] = S.poff[p];
+            S.act_n[slot] = S.pcnt[p];
+        }
+        if (p == 0) S.nact = nact;
+    }
+    __syncthreads();
+    // job tables of this CTA: gate/up jobs round-robin (every CTA mixes shared-
+    // expert jobs, already in L2, with routed ones from HBM); down jobs
+    // round-robin when every SwiGLU input is staged at once, else in blocks
+    const int na = S.nact, G = gridDim.x, c = blockIdx.x;
+    const int J2 = (P.Is / 32 + na * (P.I / 32)) * P.nkp;
+    const int J3 = (P.ndp_s + na * P.ndp_r) * (P.H / 32);
+    const int n2 = J2 > c ? (J2 - 1 - c) / G + 1 : 0;
+    int d0, dstep, n3;
+    if (P.stage_all) {
+        d0 = c;
+        dstep = G;
+        n3 = J3 > c ? (J3 - 1 - c) / G + 1 : 0;
+    } else {
+        d0 = (int)((long long)J3 * c / G);
+        dstep = 1;
+        n3 = (int)((long long)J3 * (c + 1) / G) - d0;
+    }
+    for (int i = threadIdx.x; i < n2 && i < kMaxJobs; i += blockDim.x) S.gujob[i] = make_gu_job(P, S, c + i * G);
+    for (int i = threadIdx.x; i < n3 && i < kMaxJobs; i += blockDim.x) S.dnjob[i] = make_dn_job(P, S, d0 + i * dstep);
+    if (threadIdx.x == 0) {
+        S.ngu = n2 < kMaxJobs ? n2 : kMaxJobs;
+        S.ndn = n3 < kMaxJobs ? n3 : kMaxJobs;
+        // stage-all: where each rowset's SwiGLU input starts (shared tokens first)
+        int off = 0;
+        for (int r = 0; r < T + n; ++r) {
+            S.rsoff[r] = off;
+            off += r < T ? P.Is : P.I;
+        }
+        S.rsoff[T + n] = off;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int st = 0;
+        for (int i = 0; i < S.ngu; ++i) st += (S.gujob[i].g1 - S.gujob[i].g0 + kStageGroups - 1) / kStageGroups;
+        S.gu_stages = st;
+    }
+    // the ring was written with generic stores above; order them before the
+    // bulk copies (async proxy) that refill it next
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+}
+
+// x' = bf16(rmsnorm_no_scale(h)) pre-scaled for the code decode, and its chunk
+// sums, in S.stage.  One thread per 32-column chunk; element m of chunk c is
+// visited in the order (m + c) % 32 so that a warp's threads hit distinct banks.
+__device__ __noinline__ void stage_x(const Params &P, Smem &S) {
+    const int T = P.T, H = P.H, nch = H / 32;
+    float *stage = S.stage;
+    for (int t = 0; t < T; ++t) {
+        const float r = S.rinv[t];
+        for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+            const int i = t * nch + c;
+            float *row = stage + (size_t)i * 32;
+            float sx = 0.f;
+#pragma unroll 8
+            for (int mm = 0; mm < 32; ++mm) {
+                const int m = (mm + c) & 31;
+                const float x = bf16_bits_to_float(f32_to_bf16_bits_alu(row[m] * r));
+                row[m] = x * code_prescale(m & 7);
+                sx += x;
+            }
+            S.xs[i] = sx;
+        }
+    }
+    __syncthreads();
+}
+
+// ------------------------------------------------------------------ streaming loops
+// (each its own function, so that its register allocation is its own)
+
+// Producer of the gate/up phase: bulk copies of the stages of its jobs, and,
+// once the ring is primed, an L2 prefetch of its down-phase jobs.
+__device__ __noinline__ bool gu_producer(const Params &P, Smem &S, const moe_layer_w &W, Ring ring,
+                                         unsigned &issued) {
+    bool ok = true, prefetched = false;
+    int nis = 0;
+    const int ns = P.nslots, ngu = S.ngu;
+    for (int i = 0; i < ngu && ok; ++i) {
+        const JobDesc J = S.gujob[i];
+        const uint32_t *q[2], *sb[2];
+        gu_ptrs(P, W, J, q, sb);
+        for (int g = J.g0; g < J.g1 && ok; g += kStageGroups) {
+            if (ring.q >= (unsigned)ns && !mbar_wait(&S.empty[ring.s], ring.ph ^ 1u, P.err, kErrEmpty)) {
+                ok = false;
+                break;
+            }
+            issue_stage(S, ring.s, q, sb, 2, g, min(g + kStageGroups, (int)J.g1));
+            issued = ring.q + 1;
+            ring_next(ring, ns);
+            if (++nis == ns && !prefetched) {
+                prefetched = true;
+                prefetch_dn_jobs(P, S, W);
+            }
+        }
+    }
+    if (ok && !prefetched) prefetch_dn_jobs(P, S, W);
+    return ok;
+}
+
+__device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, Ring ring) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
+    bool ok = true;
+    int buf = 0;
+    const int m = wid >> 3, gi = wid & 7;  // warps 0-7: gate, 8-15: up; gi = group within a stage
+    const int ns = P.nslots, ngu = S.ngu, Kmax = P.Kmax, R = P.R;
+    const float *stage = S.stage;
+    for (int i = 0; i < ngu; ++i) {
+        const JobDesc J = S.gujob[i];
+        const int n = J.n;
+        // the job's tokens: input rows gathered by token id
+        const int *tokrow = J.slot == 0 ? S.tokrow_sh : S.tokrow + J.seg0;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int g = J.g0; g < J.g1; g += kStageGroups) {
+            const int ngs = min(kStageGroups, (int)J.g1 - g);
+            const bool got = mbar_wait(&S.full[ring.s], ring.ph, P.err, kErrFull);
+            if (got && gi < ngs) {
+                const unsigned char *slot = S.pool + (size_t)ring.s * kSlotBytes;
+                const unsigned char *codes = slot + (m * ngs + gi) * kCodeBytesPerGroup;
+                const uint32_t sbw = reinterpret_cast<const uint32_t *>(
+                    slot + 2 * ngs * kCodeBytesPerGroup + (m * ngs + gi) * kSbBytesPerGroup)[lane];
+                const int gcol = (g + gi) * 64;
+                group_dot_n(codes, sbw, stage + gcol, S.xs + gcol / 32, tokrow, 0, n, acc, lane);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.empty[ring.s]);
+            if (!got) ok = false;
+            ring_next(ring, ns);
+        }
+        float *Rb = S.red[buf];
+#pragma unroll
+        for (int tt = 0; tt < kMaxT; ++tt)
+            if (tt < n) Rb[(wid * kMaxT + tt) * 32 + lane] = acc[tt >> 2][tt & 3];
+        consumer_sync();
+        // reduce the 8 warps of each matrix -> this K part's partial sums
+        for (int r = ctid; r < 2 * n * 32; r += kCWarps * 32) {
+            const int mm = (r >> 5) >= n ? 1 : 0, tt = (r >> 5) - mm * n, ln = r & 31;
+            float v = 0.f;
+#pragma unroll
+            for (int w8 = 0; w8 < 8; ++w8) v += Rb[((mm * 8 + w8) * kMaxT + tt) * 32 + ln];
+            const int rs = job_rowset(P, J, tt);
+            P.gu_part[(((size_t)J.part * R + rs) * 2 + mm) * Kmax + J.rb * 32 + ln] = v;
+        }
+        buf ^= 1;  // the next job reduces in the other buffer: no second barrier
+    }
+    return ok;
+}
+
+__device__ __noinline__ bool dn_producer(const Params &P, Smem &S, const moe_layer_w &W, Ring ring, int l,
+                                         unsigned &issued) {
+    const int G = gridDim.x;
+    bool ok = true;
+    int nis = 0;
+    const int ns = P.nslots, ndn = S.ndn;
+    for (int i = 0; i < ndn && ok; ++i) {
+        if (ring.q >= (unsigned)ns && !mbar_wait(&S.empty[ring.s], ring.ph ^ 1u, P.err, kErrEmpty)) {
+            ok = false;
+            break;
+        }
+        const JobDesc J = S.dnjob[i];
+        const uint32_t *q[1], *sb[1];
+        dn_ptrs(P, W, J, q[0], sb[0]);
+        issue_stage(S, ring.s, q, sb, 1, J.g0, J.g1);
+        issued = ring.q + 1;
+        ring_next(ring, ns);
+        if (++nis == ns && l + 1 < P.L) {
+            // this CTA's share of the next layer's shared-expert weights
+            const moe_layer_w &N = P.layers[l + 1];
+            const size_t shq = (size_t)P.Is * P.H / 2, shsb = (size_t)P.Is * (P.H / 64) * 4;
+            const void *ptrs[6] = {N.sh_gate.q, N.sh_up.q, N.sh_down.q, N.sh_gate.sb, N.sh_up.sb, N.sh_down.sb};
+            const size_t sizes[6] = {shq, shq, shq, shsb, shsb, shsb};
+            for (int a = 0; a < 6; ++a) {
+                const size_t per = ((sizes[a] / G) + 15) & ~(size_t)15;
+                const size_t off = per * blockIdx.x;
+                if (off < sizes[a])
+                    prefetch_range(static_cast<const char *>(ptrs[a]) + off,
+                                   (off + per <= sizes[a] ? per : sizes[a] - off) & ~(size_t)15);
+            }
+        }
+    }
+    return ok;
+}
+
+// SwiGLU input of one rowset and column: a = silu(sum of gate parts) * (sum of up parts).
+__device__ __forceinline__ float swiglu_in(const float *gu_part, size_t pstride, int nkp, int Kmax, int rs, int col) {
+    const size_t base = (size_t)rs * 2 * Kmax + col;
+    float g = 0.f, u = 0.f;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        if (p < nkp) {
+            g += __ldcg(&gu_part[p * pstride + base]);
+            u += __ldcg(&gu_part[p * pstride + base + Kmax]);
+        }
+    }
+    return silu_mul(g, u);
+}
+
+// Chunk sums (sum of the unscaled values) of nchunks 32-float chunks of the
+// stage, one consumer thread per chunk, bank-rotated.
+__device__ __forceinline__ void chunk_sums(Smem &S, int nchunks) {
+    const float *stage = S.stage;
+    for (int i = threadIdx.x; i < nchunks; i += kCWarps * 32) {
+        const float *row = stage + (size_t)i * 32;
+        float sx = 0.f;
+#pragma unroll 8
+        for (int mm = 0; mm < 32; ++mm) {
+            const int m = (mm + i) & 31;
+            sx = fmaf(row[m], code_unprescale(m & 7), sx);
+        }
+        S.xs[i] = sx;
+    }
+}
+
+__device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
+    bool ok = true;
+    int buf = 0;
+    const int T = P.T, Is = P.Is, I = P.I, ns = P.nslots, ndn = S.ndn, nkp = P.nkp, Kmax = P.Kmax;
+    const size_t pstride = (size_t)P.R * 2 * Kmax;
+    const float *gu_part = P.gu_part;
+    float *stage = S.stage;
+    if (P.stage_all) {
+        // every rowset's SwiGLU input, rowset r at S.rsoff[r] (shared tokens, then routed positions)
+        const int nrs = T + T * P.k, F = S.rsoff[nrs];
+        for (int b0 = ctid; b0 < F; b0 += 4 * kCWarps * 32) {
+            float a[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int i = b0 + v * kCWarps * 32;
+                a[v] = 0.f;
+                if (i < F) {
+                    int rs = 0;
+                    while (S.rsoff[rs + 1] <= i) ++rs;  // short scan, no division
+                    a[v] = swiglu_in(gu_part, pstride, nkp, Kmax, rs, i - S.rsoff[rs]);
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int i = b0 + v * kCWarps * 32;
+                if (i < F) stage[i] = a[v] * code_prescale(i & 7);  // rowset starts are multiples of 64
+            }
+        }
+        consumer_sync();
+        chunk_sums(S, F / 32);
+        consumer_sync();
+    }
+    int staged_slot = -1, staged_part = -1;
+    for (int i = 0; i < ndn; ++i) {
+        const JobDesc J = S.dnjob[i];
+        const int ng = J.g1 - J.g0, n = J.n;
+        const float *xb;
+        const float *xsb;
+        int stride;
+        if (P.stage_all) {
+            const int off = S.rsoff[J.slot == 0 ? 0 : T + J.seg0] + J.g0 * 64;
+            xb = stage + off;
+            xsb = S.xs + off / 32;
+            stride = J.slot == 0 ? Is : I;
+        } else {
+            const int ld = ng * 64;
+            if (J.slot != staged_slot || J.part != staged_part) {
+                // this slot's tokens, columns [g0*64, g1*64) only: row tt at tt * ld
+                for (int tt = 0; tt < n; ++tt) {
+                    const int rs = job_rowset(P, J, tt);
+                    for (int c = ctid; c < ld; c += kCWarps * 32)
+                        stage[tt * ld + c] = swiglu_in(gu_part, pstride, nkp, Kmax, rs, J.g0 * 64 + c) *
+                                             code_prescale(c & 7);
+                }
+                consumer_sync();
+                chunk_sums(S, n * 2 * ng);
+                staged_slot = J.slot;
+                staged_part = J.part;
+                consumer_sync();
+            }
+            xb = stage;
+            xsb = S.xs;
+            stride = ld;
+        }
+        const bool got = mbar_wait(&S.full[ring.s], ring.ph, P.err, kErrFull);
+        float *Rb = S.red[buf];
+        if (got && wid < ng) {
+            const int gi = wid;
+            const unsigned char *slot = S.pool + (size_t)ring.s * kSlotBytes;
+            const unsigned char *codes = slot + gi * kCodeBytesPerGroup;
+            const uint32_t sbw =
+                reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane];
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            // token tt's row at tt * stride, its chunk sums at tt * stride / 32
+            group_dot_n(codes, sbw, xb + gi * 64, xsb + 2 * gi, nullptr, stride, n, acc, lane);
+#pragma unroll
+            for (int tt = 0; tt < kMaxT; ++tt)
+                if (tt < n) Rb[(gi * kMaxT + tt) * 32 + lane] = acc[tt >> 2][tt & 3];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[ring.s]);
+        if (!got) ok = false;
+        ring_next(ring, ns);
+        consumer_sync();
+        for (int r = ctid; r < n * 32; r += kCWarps * 32) {
+            const int tt = r >> 5, ln = r & 31;
+            float v = 0.f;
+            for (int g2 = 0; g2 < ng; ++g2) v += Rb[(g2 * kMaxT + tt) * 32 + ln];
+            const int row = J.rb * 32 + ln;
+            if (J.slot == 0)
+                P.sh[((size_t)J.part * T + tt) * P.H + row] = v;
+            else
+                P.y[((size_t)J.part * T * P.k + S.perm[J.seg0 + tt]) * P.H + row] = v;
+        }
+        buf ^= 1;
+    }
+    return ok;
+}
+
+// ------------------------------------------------------------------ kernel
+
+__global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_constant__ Params P) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>(smem_raw);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const bool producer = (wid == kProducerWarp && lane == 0);
+    const bool consumer = wid < kCWarps;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMaxStages; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], kCWarps);
+        }
+        mbar_init(&S.rbar, 1);
+        S.stage = reinterpret_cast<float *>(S.pool + (size_t)P.nslots * kSlotBytes);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    Ring ring{0u, 0, 0u};  // position of the next job stage (the same in every thread)
+    unsigned issued = 0;   // producer: stages whose copies were actually issued
+    unsigned rissued = 0;  // producer: router copy batches issued (one per layer)
+    unsigned nbar = 0;     // grid barriers passed
+    bool ok = true;
+    const int ns = P.nslots;
+
+    for (int l = 0; l < P.L && ok; ++l) {
+        const moe_layer_w &W = P.layers[l];
+        if (producer) {
+            issue_router_copies(P, S, W);
+            ++rissued;
+        }
+        if (l == 0) {
+            load_input(P, S, P.h_in);
+        } else {
+            finish_layer(P, S, l - 1);
+            if (!P.chained) load_input(P, S, P.h_in + (size_t)l * P.T * P.H);
+        }
+        router_phase(P, S, l);
+        ok = grid_sync(P, ++nbar, &S.flag);
+        if (!ok) break;
+        topk_phase(P, S, W);
+        stage_x(P, S);
+
+        // ---------------- gate/up jobs
+        if (producer)
+            gu_producer(P, S, W, ring, issued);
+        else if (consumer)
+            gu_consumer(P, S, ring);
+        for (int st = S.gu_stages; st > 0; --st) ring_next(ring, ns);
+        ok = grid_sync(P, ++nbar, &S.flag);
+        if (!ok) break;
+
+        // ---------------- down jobs
+        if (producer)
+            dn_producer(P, S, W, ring, l, issued);
+        else if (consumer)
+            dn_consumer(P, S, ring);
+        for (int st = S.ndn; st > 0; --st) ring_next(ring, ns);
+        ok = grid_sync(P, ++nbar, &S.flag);
+    }
+    if (ok) finish_layer(P, S, P.L - 1);  // ok is uniform across the CTA here
+
+    // let this CTA's own bulk copies land before it exits (bounded)
+    __syncthreads();
+    if (producer) {
+        const unsigned first = issued > (unsigned)ns ? issued - ns : 0u;
+        for (unsigned q = first; q < issued; ++q) mbar_drain(&S.full[q % ns], (q / ns) & 1);
+        if (rissued > 0) mbar_drain(&S.rbar, (rissued - 1) & 1);
+    }
+}
+
+}  // namespace dec
+
+size_t decode_stack_smem() { return sizeof(dec::Smem); }
+
+static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exceeds 227 KiB");
+static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
+
+struct DecodeWs {
+    size_t bar, logits, gu_part, y, sh, total, zero_bytes;
+};
+
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static DecodeWs decode_ws(const moe_layer_w *w, int T) {
+    DecodeWs d;
+    const int Kmax = w->I > w->Is ? w->I : w->Is;
+    const int R = T + T * w->k;
+    const int nkp = (w->H / 64 + dec::kGuPartGroups - 1) / dec::kGuPartGroups;
+    const int ndp_r = (w->I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
+    const int ndp_s = (w->Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
+    size_t off = 0;
+    auto take = [&](size_t b) {
+        const size_t o = off;
+        off += al256(b);
+        return o;
+    };
+    d.bar = take(256);
+    d.zero_bytes = off;
+    d.logits = take(sizeof(double) * (size_t)T * w->E);
+    d.gu_part = take(sizeof(float) * (size_t)nkp * R * 2 * Kmax);
+    d.y = take(sizeof(float) * (size_t)ndp_r * T * w->k * w->H);
+    d.sh = take(sizeof(float) * (size_t)ndp_s * T * w->H);
+    d.total = off;
+    return d;
+}
+
+size_t decode_stack_ws_bytes(const moe_layer_w *w, int T) { return decode_ws(w, T).total; }
+
+size_t decode_stack_status_offset() { return sizeof(unsigned); }
+
+// Split of the shared-memory pool between the ring and the input stage for
+// calls of T tokens on layers shaped like w; false if the shape does not fit.
+static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots, int *stage_all) {
+    const long all = (long)T * w.Is + (long)T * w.k * w.I;  // every rowset's SwiGLU input
+    const long th = (long)T * w.H;
+    for (int sa = 1; sa >= 0; --sa) {
+        if (sa && (all > dec::kStageFloats || all / 32 > dec::kMaxXs)) continue;
+        long stage = th > (sa ? all : (long)T * dec::kDnGroups * 64) ? th : (sa ? all : (long)T * dec::kDnGroups * 64);
+        if (stage > dec::kStageFloats) return false;
+        stage = (stage + 31) & ~31L;  // keep the stage 128-byte aligned
+        long ns = (dec::kPoolBytes - stage * 4) / dec::kSlotBytes;
+        if (ns > dec::kMaxStages) ns = dec::kMaxStages;
+        const long ring = ns * dec::kSlotBytes;
+        const long rows = grid > 0 ? (w.E + grid - 1) / grid : w.E;
+        const long rcopy = 2L * w.H + rows * w.H + 2 * (rows * (w.H / 64) * 2 + 32);
+        if (ns < 3 || (long)T * w.E * 8 > ring || rcopy > ring) continue;
+        *nslots = (int)ns;
+        *stage_all = sa;
+        return true;
+    }
+    return false;
+}
+
+bool decode_stack_fits(const moe_layer_w *w, int T, int grid) {
+    int a, b;
+    return decode_layout(*w, T, grid, &a, &b);
+}
+
+int decode_stack_max_tokens() { return dec::kMaxT; }
+int decode_stack_max_layers() { return dec::kMaxLayers; }
+int decode_stack_stage_floats() { return dec::kStageFloats; }
+
+cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained,
+                                uint16_t *h_out, int T, void *ws, const moe_opts &o, int grid, cudaStream_t st) {
+    const moe_layer_w &w = layers[0];
+    const DecodeWs d = decode_ws(&w, T);
+    dec::Params P;  // ~10 KiB, passed by value (kernel parameters up to 32 KiB)
+    for (int l = 0; l < L; ++l) P.layers[l] = layers[l];
+    P.h_in = h_in;
+    P.h_out = h_out;
+    P.L = L;
+    P.T = T;
+    P.chained = chained;
+    P.post_norm = o.post_norm;
+    P.layer_scalar = o.layer_scalar;
+    P.eps = o.eps;
+    P.H = w.H;
+    P.E = w.E;
+    P.k = w.k;
+    P.I = w.I;
+    P.Is = w.Is;
+    P.Kmax = w.I > w.Is ? w.I : w.Is;
+    P.R = T + T * w.k;
+    P.nkp = (w.H / 64 + dec::kGuPartGroups - 1) / dec::kGuPartGroups;
+    P.ndp_r = (w.I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
+    P.ndp_s = (w.Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
+    if (!decode_layout(w, T, grid, &P.nslots, &P.stage_all)) return cudaErrorInvalidValue;
+    char *base = static_cast<char *>(ws);
+    P.bar = reinterpret_cast<unsigned *>(base + d.bar);
+    P.err = reinterpret_cast<int *>(base + d.bar + sizeof(unsigned));
+    P.logits = reinterpret_cast<double *>(base + d.logits);
+    P.gu_part = reinterpret_cast<float *>(base + d.gu_part);
+    P.y = reinterpret_cast<float *>(base + d.y);
+    P.sh = reinterpret_cast<float *>(base + d.sh);
+
+    const size_t smem = sizeof(dec::Smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(dec::decode_stack_kernel), smem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(ws, 0, d.zero_bytes, st);
+    if (e != cudaSuccess) return e;
+    void *args[] = {&P};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(dec::decode_stack_kernel), dim3(grid),
+                                    dim3(dec::kThreads), args, smem, st);
+    return e;
+}
+
+cudaError_t decode_stack_grid(int device, int *grid) {
+    int sms = 0, per = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+    if (e != cudaSuccess) return e;
+    e = ensure_smem(reinterpret_cast<const void *>(dec::decode_stack_kernel), sizeof(dec::Smem));
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, dec::decode_stack_kernel, dec::kThreads,
+                                                      sizeof(dec::Smem));
+    if (e != cudaSuccess) return e;
+    *grid = per >= 1 ? sms : 0;
+    return cudaSuccess;
+}
+
+}  // namespace moe

@@ -16,8 +16,8 @@
 //    the tokens of one expert segment; its warps split the input dimension by
 //    whole groups and are reduced through shared memory in a fixed order.
 //  * The input vector is broadcast from shared memory, pre-scaled so that a
-//    single FMA per code accumulates q*x (see decode_word); the affine part is
-//    applied per group as  s * sum(q x) + b * sum(x).
+//    single FMA per code accumulates q*x exactly (see decode_word); the affine
+//    part is applied per group as  s * sum(q x) + b * sum(x).
 //  * The shared expert's row blocks come first in the grid; routed blocks for
 //    slots beyond the number of experts actually used exit at once.
 #include "moe_common.cuh"
@@ -72,10 +72,10 @@ cudaError_t launch_prepare_qmat(const uint32_t *q, const uint16_t *s, const uint
 // ------------------------------------------------------------ GEMV core
 
 // Shared-memory staging of the inputs of one pass of up to NT tokens:
-//   xp[NT][cols]  pre-scaled inputs x' = x * code_prescale(col % 8)
-//   Xp[NT][cols/32], Xs[NT][cols/32]  per 32-column chunk: sum x', sum x
+//   xp[NT][cols]      pre-scaled inputs x' = x * code_prescale(col % 8)
+//   Xs[NT][cols/32]   sum of x over each 32-column chunk (for the bias term)
 struct Stage {
-    float *xp, *Xp, *Xs;
+    float *xp, *Xs;
     int cols, nchunk;
 };
 
@@ -86,18 +86,14 @@ __device__ __forceinline__ void stage_chunk_sums(const Stage &S, int nw) {
     for (int i = w; i < NT * S.nchunk; i += nw) {
         const int tt = i / S.nchunk, c = i - tt * S.nchunk;
         const float v = S.xp[(size_t)tt * S.cols + c * kChunkCols + lane];
-        const float sp = warp_sum(v);
         const float sx = warp_sum(v * inv_scale);
-        if (lane == 0) {
-            S.Xp[i] = sp;
-            S.Xs[i] = sx;
-        }
+        if (lane == 0) S.Xs[i] = sx;
     }
 }
 
 // Accumulate, for NMAT matrices whose 32-row block starts at q[m] / sb[m],
 // the dot products of this lane's row with the staged inputs over the groups
-// [g0, g1).  acc[m][tt] receives  sum_groups  s*(sum f x' - sum x') + b*sum x.
+// [g0, g1).  acc[m][tt] receives  sum_groups  s * sum(q x) + b * sum(x).
 template <int NT, int NMAT>
 __device__ __forceinline__ void gemv_slice(const uint32_t *const (&q)[NMAT], const uint32_t *const (&sb)[NMAT],
                                            const Stage &S, int nt, int g0, int g1, float (&acc)[NMAT][NT]) {
@@ -123,37 +119,19 @@ __device__ __forceinline__ void gemv_slice(const uint32_t *const (&q)[NMAT], con
         }
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-            const float s = bf16_bits_to_float(csb[m] & 0xffffu);
+            const float s = bf16_bits_to_float(csb[m] & 0xffffu) * kCodeUnscale;
             const float b = bf16_bits_to_float(csb[m] >> 16);
+            const uint32_t words[8] = {cur[m][0].x, cur[m][0].y, cur[m][0].z, cur[m][0].w,
+                                       cur[m][1].x, cur[m][1].y, cur[m][1].z, cur[m][1].w};
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c = 2 * g + h;
-                const uint32_t words[4] = {cur[m][h].x, cur[m][h].y, cur[m][h].z, cur[m][h].w};
-                float2 d2[NT];
+            for (int tt = 0; tt < NT; ++tt) {
+                if (tt < nt) {
+                    const float *xp = S.xp + (size_t)tt * S.cols + g * kGroup;
+                    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt) d2[tt] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-                    const Decoded8 d = decode_word(words[wi]);
-#pragma unroll
-                    for (int tt = 0; tt < NT; ++tt) {
-                        if (tt < nt) {
-                            const float4 *x4 =
-                                reinterpret_cast<const float4 *>(S.xp + (size_t)tt * S.cols + c * kChunkCols + wi * 8);
-                            const float4 xa = x4[0], xb = x4[1];
-                            d2[tt] = ffma2(make_float2(d.f[0], d.f[1]), make_float2(xa.x, xa.y), d2[tt]);
-                            d2[tt] = ffma2(make_float2(d.f[2], d.f[3]), make_float2(xa.z, xa.w), d2[tt]);
-                            d2[tt] = ffma2(make_float2(d.f[4], d.f[5]), make_float2(xb.x, xb.y), d2[tt]);
-                            d2[tt] = ffma2(make_float2(d.f[6], d.f[7]), make_float2(xb.z, xb.w), d2[tt]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int tt = 0; tt < NT; ++tt) {
-                    if (tt < nt) {
-                        const int ci = tt * S.nchunk + c;
-                        acc[m][tt] = fmaf(s, (d2[tt].x + d2[tt].y) - S.Xp[ci], fmaf(b, S.Xs[ci], acc[m][tt]));
-                    }
+                    for (int wi = 0; wi < 8; ++wi) dot_word(words[wi], xp + wi * 8, a0, a1);
+                    const int ci = tt * S.nchunk + 2 * g;
+                    acc[m][tt] = fmaf(s, (a0.x + a0.y) + (a1.x + a1.y), fmaf(b, S.Xs[ci] + S.Xs[ci + 1], acc[m][tt]));
                 }
             }
         }
@@ -221,7 +199,7 @@ gateup_kernel(const ExpertParams P) {
     Unit u;
     if (!decode_unit(P, P.Is / kRowBlock, P.I / kRowBlock, u)) return;
     const int H = P.H, C = H / kChunkCols, G = H / kGroup;
-    Stage S{smem_f, smem_f + (size_t)NT * H, smem_f + (size_t)NT * H + NT * C, H, C};
+    Stage S{smem_f, smem_f + (size_t)NT * H, H, C};
     float *red = S.Xs + NT * C;  // [2][NW][NT][32]
     const int rows = u.shared ? P.Is : P.I;
     const size_t mrb = u.shared ? (size_t)u.rb : (size_t)u.e * (rows / kRowBlock) + u.rb;
@@ -280,7 +258,7 @@ down_kernel(const ExpertParams P) {
     if (!decode_unit(P, P.H / kRowBlock, P.H / kRowBlock, u)) return;
     const int K = u.shared ? P.Is : P.I;  // input dimension of this matrix
     const int C = K / kChunkCols, G = K / kGroup;
-    Stage S{smem_f, smem_f + (size_t)NT * K, smem_f + (size_t)NT * K + NT * C, K, C};
+    Stage S{smem_f, smem_f + (size_t)NT * K, K, C};
     float *red = S.Xs + NT * C;  // [NW][NT][32]
     const size_t mrb = u.shared ? (size_t)u.rb : (size_t)u.e * (P.H / kRowBlock) + u.rb;
     const uint32_t *q[1] = {(u.shared ? P.sdq : P.dq) + mrb * C * 128};
@@ -329,7 +307,7 @@ constexpr int kGateUpWarps = 8;
 constexpr int kDownWarps = 4;
 
 static size_t stage_bytes(int cols, int nt, int nred) {
-    return sizeof(float) * ((size_t)nt * cols + 2 * (size_t)nt * (cols / kChunkCols) + (size_t)nred * nt * 32);
+    return sizeof(float) * ((size_t)nt * cols + (size_t)nt * (cols / kChunkCols) + (size_t)nred * nt * 32);
 }
 
 size_t gemv_smem_bytes(int cols, int nt) { return stage_bytes(cols, nt, 2 * kGateUpWarps); }

@@ -43,4 +43,16 @@ cudaError_t launch_combine(const float *y, const float *sh, const float *wts, in
                            const uint16_t *h_in, float *m_out, uint16_t *h_out, int post_norm, float layer_scalar,
                            float eps, cudaStream_t st);
 
+// Persistent decode kernel over a stack of layers (moe_decode.cu).
+size_t decode_stack_smem();
+size_t decode_stack_ws_bytes(const moe_layer_w *w, int T);
+size_t decode_stack_status_offset();
+int decode_stack_max_tokens();
+bool decode_stack_fits(const moe_layer_w *w, int T, int grid);
+int decode_stack_max_layers();
+int decode_stack_stage_floats();
+cudaError_t decode_stack_grid(int device, int *grid);
+cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained,
+                                uint16_t *h_out, int T, void *ws, const moe_opts &o, int grid, cudaStream_t st);
+
 }  // namespace moe

@@ -19,10 +19,11 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"libmoe.so not built ({LIB_PATH}); run `python -m int4_routed_expert_02_b200.build`")
 _lib = C.CDLL(LIB_PATH)
 
-MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_ECUDA = 0, -1, -2, -3, -4
+MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_ECUDA, MOE_EDEVICE = 0, -1, -2, -3, -4, -5
 EXPORTED = ("moe_last_error", "moe_version", "moe_prepare_qmat", "moe_workspace_size", "moe_router_logits",
             "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward",
-            "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc")
+            "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc", "moe_decode_stack_workspace_size",
+            "moe_decode_stack", "moe_decode_stack_status")
 
 
 class MoEError(RuntimeError):
@@ -60,6 +61,10 @@ _lib.moe_bucket.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
 _lib.moe_expert_ffn.argtypes = [_P, _P, _I, _P, _P, _P, _P, _P, _I, _P, _P, C.c_size_t, _P, _P]
 _lib.moe_layer_forward.argtypes = [_P, _P, _P, _I, _P, C.c_size_t, _P, _P]
 _lib.moe_noalloc_scratch_bytes.restype = C.c_size_t
+_lib.moe_decode_stack_workspace_size.argtypes = [_P, _I]
+_lib.moe_decode_stack_workspace_size.restype = C.c_size_t
+_lib.moe_decode_stack.argtypes = [_P, _I, _P, _I, _P, _I, _P, C.c_size_t, _P, _P]
+_lib.moe_decode_stack_status.argtypes = [_P]
 _lib.moe_layer_forward_noalloc.argtypes = [_P, _P, _P, _I, _P, _P]
 
 
@@ -208,6 +213,28 @@ def moe_layer_forward_noalloc(layer, h_in, h_out, T, opts=None, stream=None):
     (moe_noalloc_scratch_bytes()) is used instead; see include/moe_api.h."""
     o = opts if opts is not None else _opts()
     _check(_lib.moe_layer_forward_noalloc(layer.ptr(), _ptr(h_in), _ptr(h_out), T, C.byref(o), _stream(stream)))
+
+
+def layer_array(layers):
+    """A contiguous host array of moe_layer_w for moe_decode_stack."""
+    arr = (LayerW * len(layers))()
+    for i, l in enumerate(layers):
+        arr[i] = l.struct
+    return arr
+
+
+def moe_decode_stack_workspace_size(layer, T: int) -> int:
+    return int(_lib.moe_decode_stack_workspace_size(layer.ptr(), T))
+
+
+def moe_decode_stack(layer_arr, L, h_in, chained, h_out, T, ws, opts=None, stream=None):
+    o = opts if opts is not None else _opts()
+    _check(_lib.moe_decode_stack(C.addressof(layer_arr), L, _ptr(h_in), int(chained), _ptr(h_out), T, _ptr(ws),
+                                 ws.numel() if ws is not None else 0, C.byref(o), _stream(stream)))
+
+
+def moe_decode_stack_status(ws):
+    _check(_lib.moe_decode_stack_status(_ptr(ws)))
 
 
 def moe_noalloc_scratch_bytes() -> int:

@@ -17,7 +17,7 @@ from . import moe, synth
 
 class MoEStack:
     def __init__(self, cfg: synth.MoEConfig, cfg_id: int, T: int | None = None, layers: int | None = None,
-                 seed: int = 0, device="cuda", keep_router_codes: bool = False):
+                 seed: int = 0, device="cuda", keep_router_codes: bool = False, persistent: bool | None = None):
         self.cfg, self.cfg_id, self.seed = cfg, cfg_id, seed
         self.T = cfg.T if T is None else T
         self.L = cfg.layers if layers is None else layers
@@ -31,9 +31,22 @@ class MoEStack:
             self.layers.append(moe.DeviceLayer.from_config(w, cfg, device=self.device))
             del w
         H = cfg.H
-        # chained: buf[l] is layer l's input, buf[l+1] its output
-        # unchained: inp[l] -> out[l]
-        if cfg.chained:
+        fits = self.T <= 8 and H <= 4096 and self.T * H <= 24576
+        self.persistent = fits if persistent is None else persistent
+        if self.persistent:
+            # one cooperative kernel per step: every layer's output in h_out[l]
+            self.larr = moe.layer_array(self.layers)
+            self.ws_dec = torch.empty(moe.moe_decode_stack_workspace_size(self.layers[0], self.T), dtype=torch.uint8,
+                                      device=self.device)
+            self.h_out = torch.zeros(self.L, self.T, H, dtype=torch.bfloat16, device=self.device)
+            if cfg.chained:
+                self.buf = torch.zeros(1, self.T, H, dtype=torch.bfloat16, device=self.device)
+                self.inputs = [self.buf[0]] + [self.h_out[l] for l in range(self.L - 1)]
+            else:
+                self.inp = torch.zeros(self.L, self.T, H, dtype=torch.bfloat16, device=self.device)
+                self.inputs = [self.inp[l] for l in range(self.L)]
+            self.outputs = [self.h_out[l] for l in range(self.L)]
+        elif cfg.chained:
             self.buf = torch.zeros(self.L + 1, self.T, H, dtype=torch.bfloat16, device=self.device)
             self.inputs = [self.buf[l] for l in range(self.L)]
             self.outputs = [self.buf[l + 1] for l in range(self.L)]
@@ -42,7 +55,7 @@ class MoEStack:
             self.out = torch.zeros(self.L, self.T, H, dtype=torch.bfloat16, device=self.device)
             self.inputs = [self.inp[l] for l in range(self.L)]
             self.outputs = [self.out[l] for l in range(self.L)]
-        self.ws = moe.workspace(self.layers[0], self.T, device=self.device)
+        self.ws = moe.workspace(self.layers[0], self.T, device=self.device)  # per-layer calls
         self.opts = moe.make_opts()
         self.graph = None
 
@@ -59,14 +72,33 @@ class MoEStack:
     def final_output(self) -> torch.Tensor:
         return self.outputs[-1]
 
+    def launches_per_step(self) -> int:
+        """Kernels of the library launched per step."""
+        return 1 if self.persistent else 6 * self.L
+
     def enqueue(self, stream=None):
         """Enqueue one step (all L layers) on `stream` (default: torch's current stream)."""
+        if self.persistent:
+            h_in = self.buf[0] if self.cfg.chained else self.inp
+            moe.moe_decode_stack(self.larr, self.L, h_in, self.cfg.chained, self.h_out, self.T, self.ws_dec,
+                                 self.opts, stream=stream)
+            return
         for l in range(self.L):
             moe.moe_layer_forward(self.layers[l], self.inputs[l], self.outputs[l], self.T, self.ws, self.opts,
                                   stream=stream)
 
+    def status(self):
+        """Raise if the persistent kernel recorded a device-side error (synchronises)."""
+        if self.persistent:
+            moe.moe_decode_stack_status(self.ws_dec)
+
     def capture(self):
-        """Capture one step in a CUDA graph (replayed by run())."""
+        """Capture one step in a CUDA graph (replayed by run()).  The persistent
+        kernel is a single launch per step and is not captured."""
+        if self.persistent:
+            self.enqueue()
+            torch.cuda.synchronize(self.device)
+            return None
         s = torch.cuda.Stream(device=self.device)
         s.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(s):

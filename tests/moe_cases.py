@@ -55,3 +55,21 @@ def max_err_vs_rms(got: np.ndarray, ref: np.ndarray) -> float:
 
 def bf16_host(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().float().double().numpy()
+
+
+def assert_same_up_to_one_rounding(a: torch.Tensor, b: torch.Tensor, max_frac=0.10):
+    """Two bf16 results of the same fp32-accumulated computation along
+    different kernel paths: every element within one bf16 ulp of the other at
+    its magnitude, or within 1e-3 * rms (near zero, where ulps are tiny); and
+    few elements differing at all (rounding flips only)."""
+    a64 = a.detach().cpu().double()
+    b64 = b.detach().cpu().double()
+    rms = float(b64.pow(2).mean().sqrt())
+    mag = torch.maximum(a64.abs(), b64.abs()).clamp_min(1e-30)
+    ulp = torch.pow(2.0, torch.floor(torch.log2(mag)) - 7)      # bf16: 8 significant bits
+    tol = torch.maximum(ulp, torch.full_like(ulp, 1e-3 * rms))
+    diff = (a64 - b64).abs()
+    worst = float((diff / tol).max())
+    assert worst <= 1.0 + 1e-9, f"difference {worst:.2f} x (one ulp or 1e-3 rms)"
+    frac = float((diff > 0).double().mean())
+    assert frac <= max_frac, f"{frac:.2%} of elements differ"

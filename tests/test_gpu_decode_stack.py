@@ -1,0 +1,88 @@
+"""The persistent decode kernel (moe_decode_stack) against the per-layer path
+(moe_layer_forward) and the fp64 oracle.  Each layer is checked teacher-forced:
+on exactly the bf16 input the kernel gave it."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int4_routed_expert_02_b200 import synth
+from tests.moe_cases import (OUT_TOL, assert_same_up_to_one_rounding, bf16_host, host, max_err_vs_rms,
+                             oracle_layer)
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from int4_routed_expert_02_b200 import build
+    build.build()
+    from int4_routed_expert_02_b200 import moe
+    from int4_routed_expert_02_b200.stack import MoEStack
+
+
+def _check_stack(st, cfg, cfg_id, oracle_layers=(0,), tol=OUT_TOL):
+    st.status()
+    ws = moe.workspace(st.layers[0], st.T)
+    for l in range(st.L):
+        h_in = st.inputs[l]
+        ref = torch.empty_like(h_in)
+        moe.moe_layer_forward(st.layers[l], h_in, ref, st.T, ws)
+        torch.cuda.synchronize()
+        assert_same_up_to_one_rounding(st.outputs[l], ref)
+    for l in oracle_layers:
+        w = host(synth.gen_layer(cfg, cfg_id, l, device="cuda"))
+        OL = oracle_layer(w, cfg)
+        ref = oracle.layer_forward(OL, st.inputs[l].cpu())
+        err = max_err_vs_rms(bf16_host(st.outputs[l]), ref["out_f64"])
+        assert err <= tol, f"layer {l}: {err:.3e} vs the oracle"
+
+
+@pytest.mark.parametrize("cfg_id,T,L", [(0, 4, 3), (0, 1, 2), (1, 1, 4), (1, 8, 2), (2, 4, 3), (2, 8, 2)])
+def test_decode_stack_matches_per_layer_path_and_oracle(cfg_id, T, L):
+    cfg = synth.CONFIGS[cfg_id]
+    st = MoEStack(cfg, cfg_id, T=T, layers=L)
+    assert st.persistent
+    for step in range(2):   # second call reuses the workspace and the ring state
+        st.set_input(synth.gen_hidden(cfg, cfg_id, 500 + step, T).cuda())
+        st.run()
+        torch.cuda.synchronize()
+        _check_stack(st, cfg, cfg_id, oracle_layers=(0, L - 1) if step == 1 else ())
+
+
+def test_decode_stack_unchained_zipf_inputs():
+    cfg = synth.CONFIGS[3]
+    L, T = 3, 2
+    st = MoEStack(cfg, 3, T=T, layers=L, keep_router_codes=True)
+    h = torch.stack([synth.gen_zipf_hidden(cfg, 3, l, 0, st.router_codes[l], T=T)[0] for l in range(L)])
+    st.set_input(h.cuda())
+    st.run()
+    torch.cuda.synchronize()
+    _check_stack(st, cfg, 3, oracle_layers=(1,))
+
+
+@pytest.mark.parametrize("dims", [
+    dict(H=64, E=8, k=8, I=64, Is=64, T=3),           # k = E: every token uses every expert
+    dict(H=320, E=24, k=5, I=192, Is=1088, T=5),      # ragged groups, 2 shared down parts
+    dict(H=4096, E=32, k=2, I=1088, Is=128, T=2),     # widest hidden, 2 routed down parts
+])
+def test_decode_stack_edge_shapes(dims):
+    T = dims.pop("T")
+    cfg = synth.MoEConfig("edge", layers=2, T=T, **dims)
+    st = MoEStack(cfg, 98, T=T)
+    st.set_input(synth.gen_hidden(cfg, 98, 1, T).cuda())
+    st.run()
+    torch.cuda.synchronize()
+    _check_stack(st, cfg, 98, oracle_layers=(0,))
+
+
+def test_decode_stack_is_deterministic_and_rejects_bad_sizes():
+    cfg = synth.CONFIGS[1]
+    st = MoEStack(cfg, 1, T=1, layers=2)
+    st.set_input(synth.gen_hidden(cfg, 1, 3, 1).cuda())
+    st.run()
+    a = st.h_out.clone()
+    st.run()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), st.h_out.view(torch.int16))
+    assert moe.moe_decode_stack_workspace_size(st.layers[0], 9) == 0
+    with pytest.raises(moe.MoEError):
+        moe.moe_decode_stack(st.larr, 2, st.buf[0], 1, st.h_out, 9, st.ws_dec)

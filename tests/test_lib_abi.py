@@ -120,3 +120,23 @@ def test_other_entry_points_validate():
     assert L.moe_router(C.addressof(st), FAKE, 4, FAKE, FAKE, None, FAKE, 16, None) == moe.MOE_EWORKSPACE
     assert L.moe_expert_ffn(C.addressof(st), FAKE, 4, FAKE, FAKE, FAKE, FAKE, None, 1, FAKE, FAKE, 1 << 40,
                             None, None) == moe.MOE_EINVAL
+
+
+def _stack(layers, L, T, ws_bytes=1 << 40, h_in=FAKE, h_out=FAKE * 4):
+    arr = (moe.LayerW * len(layers))(*layers)
+    return moe.lib().moe_decode_stack(C.addressof(arr), L, h_in, 1, h_out, T, FAKE * 8, ws_bytes,
+                                      C.byref(moe.make_opts()), None)
+
+
+def test_decode_stack_validation():
+    a = fake_layer()
+    assert _stack([a], 0, 1) == moe.MOE_EINVAL
+    assert _stack([a] * 65, 65, 1) == moe.MOE_EINVAL
+    assert _stack([a], 1, 9) == moe.MOE_EINVAL and "T=9" in moe.last_error()
+    assert _stack([a, fake_layer(I=192)], 2, 1) == moe.MOE_EINVAL and "different shape" in moe.last_error()
+    assert _stack([fake_layer(H=8192)], 1, 1) == moe.MOE_EINVAL
+    assert _stack([fake_layer(H=4096)], 1, 8) == moe.MOE_EINVAL and "T*H" in moe.last_error()
+    assert _stack([a], 1, 0) == moe.MOE_OK
+    assert _stack([a], 1, 2, ws_bytes=16) == moe.MOE_EWORKSPACE
+    assert moe.lib().moe_decode_stack_workspace_size(C.addressof(a), 9) == 0
+    assert moe.lib().moe_decode_stack_workspace_size(C.addressof(a), 8) > 0
