@@ -52,7 +52,7 @@ extern "C" {
 #define MOE_EALIGN (-2)     /* a pointer is not 16-byte aligned */
 #define MOE_EWORKSPACE (-3) /* workspace missing or smaller than moe_workspace_size() */
 #define MOE_ECUDA (-4)      /* a CUDA launch failed; the CUDA error string is in moe_last_error() */
-#define MOE_EDEVICE (-5)    /* a kernel recorded an error (a bounded wait ran out); see moe_decode_stack_status */
+#define MOE_EDEVICE (-5)    /* a kernel recorded an error (a bounded wait ran out); see moe_workspace_status */
 
 /*
  * Quantised matrix set in the kernel ("tiled") layout, produced once per
@@ -98,7 +98,8 @@ typedef struct {
     int post_norm;      /* 1: out = (h + rmsnorm_no_scale(m)) * layer_scalar; 0: (h + m) * layer_scalar */
     float layer_scalar; /* default 1.0 */
     float eps;          /* default 1e-6, inside every RMS */
-    int force_path;     /* 0 auto, 1 CUDA-core dequant-GEMV, 2 tensor-core grouped GEMM */
+    int force_path;     /* 0 auto (tensor-core grouped GEMM from T >= 32 on, else dequant-GEMV),
+                           1 CUDA-core dequant-GEMV, 2 tensor-core (tcgen05) grouped GEMM */
 } moe_opts;
 
 /* Text of the last error on this host thread ("" if none). */
@@ -123,6 +124,16 @@ MOE_API int moe_prepare_qmat(const uint32_t *q, const uint16_t *scale, const uin
  * Returns 0 on invalid arguments.
  */
 MOE_API size_t moe_workspace_size(const moe_layer_w *w, int T_max);
+
+/*
+ * Synchronous: waits for the device, then reads the status word that the
+ * last moe_expert_ffn / moe_layer_forward call on the tensor-core path left in
+ * `ws` (its first bytes; reset by every such call).  The grouped-GEMM kernels
+ * bound every wait (~1 s); if one runs out they record a code there and stop
+ * early (outputs are then invalid).  MOE_OK, or MOE_EDEVICE with the reason in
+ * moe_last_error().  Also reads a moe_decode_stack workspace.
+ */
+MOE_API int moe_workspace_status(const void *ws);
 
 /*
  * Router logits only (the first three lines of the router pseudo-code):

@@ -103,10 +103,16 @@ int check_T(const char *fn, int T) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace carve-up for calls of up to T tokens.
+// Workspace carve-up for calls of up to T tokens.  The first 256 bytes hold
+// the device status word (byte offset 4, as in the decode-stack workspace).
+// The SwiGLU buffers of the GEMV path and the token / SwiGLU matrices of the
+// tensor-core path share one region (a call uses one path).
 struct WsLayout {
-    size_t logits, idx, wts, xe, offsets, perm, inv, active, a_routed, a_shared, y, sh, total;
+    size_t status, logits, idx, wts, xe, offsets, perm, inv, active, a_routed, a_shared, xg, act, y, sh, total;
 };
+
+constexpr size_t kStatusOffset = 4;
+constexpr int kMmaMinT = 32;  // auto path: tensor-core grouped GEMM from this many tokens on
 
 WsLayout ws_layout(const moe_layer_w *w, int T) {
     WsLayout L;
@@ -117,6 +123,7 @@ WsLayout ws_layout(const moe_layer_w *w, int T) {
         return o;
     };
     const size_t Tk = (size_t)T * w->k;
+    L.status = take(256);
     L.logits = take(sizeof(double) * T * w->E);
     L.idx = take(sizeof(int32_t) * Tk);
     L.wts = take(sizeof(float) * Tk);
@@ -125,8 +132,15 @@ WsLayout ws_layout(const moe_layer_w *w, int T) {
     L.perm = take(sizeof(int32_t) * Tk);
     L.inv = take(sizeof(int32_t) * Tk);
     L.active = take(sizeof(int32_t) * (w->E + 1));
-    L.a_routed = take(sizeof(float) * Tk * w->I);
-    L.a_shared = take(sizeof(float) * T * w->Is);
+    {
+        const size_t gemv_a = align256(sizeof(float) * Tk * w->I), gemv_s = align256(sizeof(float) * T * w->Is);
+        const size_t mma_x = align256(moe::mma_xg_bytes(w, T)), mma_a = align256(moe::mma_act_bytes(w, T));
+        const size_t region = take(gemv_a + gemv_s > mma_x + mma_a ? gemv_a + gemv_s : mma_x + mma_a);
+        L.a_routed = region;
+        L.a_shared = region + gemv_a;
+        L.xg = region;
+        L.act = region + mma_x;
+    }
     L.y = take(sizeof(float) * Tk * w->H);
     L.sh = take(sizeof(float) * T * w->H);
     L.total = off;
@@ -153,10 +167,28 @@ moe_opts resolve_opts(const moe_opts *o) {
 }
 
 int check_opts(const char *fn, const moe_opts &o) {
-    if (o.force_path < 0 || o.force_path > 1)
-        return fail(MOE_EINVAL, "%s: force_path=%d (0 auto, 1 dequant-GEMV)", fn, o.force_path);
+    if (o.force_path < 0 || o.force_path > 2)
+        return fail(MOE_EINVAL, "%s: force_path=%d (0 auto, 1 dequant-GEMV, 2 tensor-core GEMM)", fn, o.force_path);
     if (!(o.eps >= 0.0f)) return fail(MOE_EINVAL, "%s: eps must be >= 0", fn);
     return MOE_OK;
+}
+
+bool use_mma(const moe_opts &o, int T) { return o.force_path == 2 || (o.force_path == 0 && T >= kMmaMinT); }
+
+// Expert part of a call: the SwiGLU FFNs of the routed and shared experts into
+// y / sh, by the tensor-core grouped GEMM or the CUDA-core dequant-GEMV.
+cudaError_t run_experts(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets, const int32_t *perm,
+                        const int32_t *active, int with_shared, void *ws, const WsLayout &L, const moe_opts &o,
+                        cudaStream_t st) {
+    if (use_mma(o, T)) {
+        int *err = at<int>(ws, L.status + kStatusOffset);
+        cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
+        if (e != cudaSuccess) return e;
+        moe::MmaBuffers b{at<uint16_t>(ws, L.xg), at<uint16_t>(ws, L.act), at<float>(ws, L.y), at<float>(ws, L.sh), err};
+        return moe::launch_expert_mma(w, xe, T, offsets, perm, active, with_shared, b, st);
+    }
+    moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
+    return moe::launch_expert_gemv(w, xe, T, offsets, perm, active, with_shared, b, st);
 }
 
 }  // namespace
@@ -285,10 +317,10 @@ int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_
     if (int rc = check_ws(fn, w, T, ws, ws_bytes)) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const WsLayout L = ws_layout(w, T);
-    moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
-    cudaError_t e = moe::launch_expert_gemv(w, xe, T, offsets, perm, active, with_shared, b, st);
+    cudaError_t e = run_experts(w, xe, T, offsets, perm, active, with_shared, ws, L, o, st);
     if (e == cudaSuccess)
-        e = moe::launch_combine(b.y, b.sh, wts, T, w->H, w->k, with_shared, nullptr, m_out, nullptr, 0, 1.0f, 0.0f, st);
+        e = moe::launch_combine(at<float>(ws, L.y), at<float>(ws, L.sh), wts, T, w->H, w->k, with_shared, nullptr,
+                                m_out, nullptr, 0, 1.0f, 0.0f, st);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
 }
 
@@ -320,13 +352,12 @@ int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_ou
     uint16_t *xe = at<uint16_t>(ws, L.xe);
     int32_t *offsets = at<int32_t>(ws, L.offsets), *perm = at<int32_t>(ws, L.perm), *inv = at<int32_t>(ws, L.inv);
     int32_t *active = at<int32_t>(ws, L.active);
-    moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
     cudaError_t e = moe::launch_router_logits(w, h_in, T, o.eps, logits, xe, st);
     if (e == cudaSuccess) e = moe::launch_router_topk(logits, T, w->E, w->k, w->per_expert_scale, idx, wts, st);
     if (e == cudaSuccess) e = moe::launch_bucket(idx, T * w->k, w->E, offsets, perm, inv, active, st);
-    if (e == cudaSuccess) e = moe::launch_expert_gemv(w, xe, T, offsets, perm, active, 1, b, st);
+    if (e == cudaSuccess) e = run_experts(w, xe, T, offsets, perm, active, 1, ws, L, o, st);
     if (e == cudaSuccess)
-        e = moe::launch_combine(b.y, b.sh, wts, T, w->H, w->k, 1, h_in, nullptr, h_out, o.post_norm, o.layer_scalar,
+        e = moe::launch_combine(at<float>(ws, L.y), at<float>(ws, L.sh), wts, T, w->H, w->k, 1, h_in, nullptr, h_out, o.post_norm, o.layer_scalar,
                                 o.eps, st);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
 }
@@ -391,6 +422,23 @@ int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int
         return fail(MOE_EINVAL, "%s: T=%d with H=%d, E=%d does not fit the kernel's shared memory", fn, T, w0.H, w0.E);
     e = moe::launch_decode_stack(layers, L, h_in, chained, h_out, T, ws, o, grid, st);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_workspace_status(const void *ws) {
+    const char *fn = "moe_workspace_status";
+    g_err.clear();
+    if (!ws) return fail(MOE_EINVAL, "%s: workspace is NULL", fn);
+    int code = 0;
+    cudaError_t e = cudaMemcpy(&code, static_cast<const char *>(ws) + kStatusOffset, sizeof code, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    if (code != 0) {
+        static const char *what[] = {"", "wait for weights timed out", "wait for a free weight slot timed out",
+                                     "wait for a weight tile timed out", "wait for a free weight tile timed out",
+                                     "wait for a token tile timed out", "wait for a free token tile timed out",
+                                     "wait for the accumulator timed out", "wait for the epilogue timed out"};
+        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 9) ? what[code] : "?");
+    }
+    return MOE_OK;
 }
 
 int moe_decode_stack_status(const void *ws) {

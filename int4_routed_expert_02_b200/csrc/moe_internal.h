@@ -38,6 +38,20 @@ size_t gemv_smem_bytes(int cols, int nt);
 cudaError_t launch_expert_gemv(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
                                const int32_t *perm, const int32_t *active, int with_shared, const FfnBuffers &b,
                                cudaStream_t st);
+// Tensor-core grouped GEMM path (moe_mma.cu).
+struct MmaBuffers {
+    uint16_t *xg;   // [T + T*k, H]    FP16 token rows (shared, then bucketed pairs), chunk-permuted
+    uint16_t *act;  // [T + T*k, Kmax] FP16 SwiGLU rows, chunk-permuted, Kmax = max(I, Is)
+    float *y;       // [T*k, H]  routed expert outputs, by pair id t*k+s
+    float *sh;      // [T, H]    shared expert output
+    int *err;       // device error word (0 = ok)
+};
+size_t mma_xg_bytes(const moe_layer_w *w, int T);
+size_t mma_act_bytes(const moe_layer_w *w, int T);
+cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
+                              const int32_t *perm, const int32_t *active, int with_shared, const MmaBuffers &b,
+                              cudaStream_t st);
+
 // mode 0: m_out[t] = sum_s w y + sh ; mode 1: h_out = bf16((h + rmsnorm(m)) * scalar) (or no norm)
 cudaError_t launch_combine(const float *y, const float *sh, const float *wts, int T, int H, int k, int with_shared,
                            const uint16_t *h_in, float *m_out, uint16_t *h_out, int post_norm, float layer_scalar,

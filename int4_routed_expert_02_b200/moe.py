@@ -23,7 +23,7 @@ MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_ECUDA, MOE_EDEVICE = 0, -1, 
 EXPORTED = ("moe_last_error", "moe_version", "moe_prepare_qmat", "moe_workspace_size", "moe_router_logits",
             "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward",
             "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc", "moe_decode_stack_workspace_size",
-            "moe_decode_stack", "moe_decode_stack_status")
+            "moe_decode_stack", "moe_decode_stack_status", "moe_workspace_status")
 
 
 class MoEError(RuntimeError):
@@ -65,6 +65,7 @@ _lib.moe_decode_stack_workspace_size.argtypes = [_P, _I]
 _lib.moe_decode_stack_workspace_size.restype = C.c_size_t
 _lib.moe_decode_stack.argtypes = [_P, _I, _P, _I, _P, _I, _P, C.c_size_t, _P, _P]
 _lib.moe_decode_stack_status.argtypes = [_P]
+_lib.moe_workspace_status.argtypes = [_P]
 _lib.moe_layer_forward_noalloc.argtypes = [_P, _P, _P, _I, _P, _P]
 
 
@@ -235,6 +236,10 @@ def moe_decode_stack(layer_arr, L, h_in, chained, h_out, T, ws, opts=None, strea
 
 def moe_decode_stack_status(ws):
     _check(_lib.moe_decode_stack_status(_ptr(ws)))
+
+
+def moe_workspace_status(ws):
+    _check(_lib.moe_workspace_status(_ptr(ws)))
 
 
 def moe_noalloc_scratch_bytes() -> int:

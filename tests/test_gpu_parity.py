@@ -166,8 +166,9 @@ def test_expert_ffn_matches_oracle(cfg_id, T, sample):
     rows = list(rows)
     m_ref = oracle.expert_ffn(OL, xe[rows], idx[rows], wr[rows].astype(np.float32).astype(np.float64))
     assert max_err_vs_rms(m[rows], m_ref) <= OUT_TOL
-    # the decode GEMV is far tighter than the bar; keep it that way
-    assert max_err_vs_rms(m[rows], m_ref) <= 1e-3
+    # the decode GEMV (T < 32 takes it) is far tighter than the bar; keep it that way
+    if T < 32:
+        assert max_err_vs_rms(m[rows], m_ref) <= 1e-3
 
 
 def test_expert_ffn_without_shared_and_dense_equivalence():
