@@ -18,10 +18,13 @@
 //       and this CTA's job tables for the two expert phases
 //   P2' gate/up dequant-GEMV jobs (32 rows x one K part of <= 16 groups of
 //       both matrices, streamed in stages of <= 8 groups), partial sums to
-//       global
+//       global; the last K part of a (slot, row block) to finish -- found
+//       with an atomic counter -- forms a = silu(g) * u for those rows
 //   --- grid barrier ---
-//   P3  down dequant-GEMV jobs (32 rows x <= 16 groups); each CTA forms the
-//       SwiGLU input a = silu(sum g) * (sum u) it needs
+//   P3  down dequant-GEMV jobs (32 rows x <= 16 groups of one slot), in
+//       contiguous blocks per CTA so that a CTA stages each slot's a once;
+//       the last job of a row block to finish forms the combine
+//       m = sum_s w_s y_s + shared for those rows
 //   --- grid barrier ---
 //
 // Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
@@ -76,13 +79,16 @@ struct Params {
     int H, E, k, I, Is, Kmax, R;
     int nkp, ndp_r, ndp_s;
     int nslots;      // ring slots (the rest of the pool is the input stage)
-    int stage_all;   // 1: the down phase stages every slot's SwiGLU input at once
     unsigned *bar;
     int *err;
+    unsigned *cnt_gu;  // [1 + T*k][Kmax/32]: K parts done per (slot, row block); reset by the last
+    unsigned *cnt_dn;  // [H/32]: down jobs done per row block; reset by the last
     double *logits;  // [T,E]
     float *gu_part;  // [nkp][R][2][Kmax]: gate (0) and up (1) partial sums per K part
+    float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs)
     float *y;        // [ndp_r][T*k][H]
     float *sh;       // [ndp_s][T][H]
+    float *m;        // [T][H]: the combine m of the current layer
 };
 
 // One job of an expert phase: 32 rows (row block rb) x groups [g0, g1) of the
@@ -113,13 +119,13 @@ struct Smem {
     int act_e[kMaxPairs], act_off[kMaxPairs], act_n[kMaxPairs];
     int tokrow[kMaxPairs];  // bucketed position j -> row offset (token * H) of its input
     int tokrow_sh[kMaxT];   // shared expert: token t -> t * H
-    int rsoff[kMaxT + kMaxPairs + 1];  // stage-all: start of each rowset's SwiGLU input in the stage
     int nact;
     double rpart[128];
     float rms[kMaxT];
     float rinv[kMaxT];
     int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
     int flag;
+    int last;      // consumer broadcast: this CTA finished the last job of a row block
 };
 
 // Position in the ring: stage sequence number q, its slot s and phase parity ph.
@@ -477,13 +483,11 @@ __device__ __noinline__ void load_input(const Params &P, Smem &S, const uint16_t
     __syncthreads();
 }
 
-// P0: output of layer lp (m from its y/sh parts, post-norm, residual, scalar)
-// into S.stage as floats, with its RMS; CTA 0 also writes it to h_out[lp].
-// All global loads of a token are issued before they are used; H/4 <= 1024 <
-// 2 * blockDim, so two float4 per thread cover a row.
+// P0: output of layer lp (its combine m, post-norm, residual, scalar) into
+// S.stage as floats, with its RMS; CTA 0 also writes it to h_out[lp].
+// H/4 <= 1024 < 2 * blockDim, so two float4 per thread cover a row.
 __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
-    const int T = P.T, H = P.H, k = P.k, Tk = T * k, H4 = H / 4, ndp_r = P.ndp_r, ndp_s = P.ndp_s;
-    const float *y = P.y, *shp = P.sh;
+    const int T = P.T, H = P.H, H4 = H / 4;
     const uint16_t *hprev = (P.chained && lp > 0) ? P.h_out + (size_t)(lp - 1) * T * H
                                                   : (P.chained ? P.h_in : P.h_in + (size_t)lp * T * H);
     uint16_t *out = P.h_out + (size_t)lp * T * H;
@@ -500,59 +504,12 @@ __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
             hreg[r] = make_uint2(0u, 0u);
             if (i4 < H4) {
                 hreg[r] = __ldcg(reinterpret_cast<const uint2 *>(hprev + (size_t)t * H) + i4);
-                float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
-                // routed slots, 8 loads in flight at a time; each slot's K parts summed, then weighted
-                for (int b0 = 0; b0 < k; b0 += 8) {
-                    float4 v[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        v[u] = b0 + u < k ? __ldcg(reinterpret_cast<const float4 *>(y + ((size_t)t * k + b0 + u) * H) + i4)
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int dp = 1; dp < ndp_r; ++dp) {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            if (b0 + u < k) {
-                                const float4 vv = __ldcg(reinterpret_cast<const float4 *>(
-                                                             y + ((size_t)dp * Tk + t * k + b0 + u) * H) + i4);
-                                v[u].x += vv.x;
-                                v[u].y += vv.y;
-                                v[u].z += vv.z;
-                                v[u].w += vv.w;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const float w = b0 + u < k ? S.wts[t * k + b0 + u] : 0.f;
-                        m.x = fmaf(w, v[u].x, m.x);
-                        m.y = fmaf(w, v[u].y, m.y);
-                        m.z = fmaf(w, v[u].z, m.z);
-                        m.w = fmaf(w, v[u].w, m.w);
-                    }
-                }
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    v[u] = u < ndp_s ? __ldcg(reinterpret_cast<const float4 *>(shp + ((size_t)u * T + t) * H) + i4)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int u = 4; u < ndp_s; ++u) {
-                    const float4 vv = __ldcg(reinterpret_cast<const float4 *>(shp + ((size_t)u * T + t) * H) + i4);
-                    m.x += vv.x;
-                    m.y += vv.y;
-                    m.z += vv.z;
-                    m.w += vv.w;
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    m.x += v[u].x;
-                    m.y += v[u].y;
-                    m.z += v[u].z;
-                    m.w += v[u].w;
-                }
-                mreg[r] = m;
-                ss += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
+                mreg[r] = __ldcg(reinterpret_cast<const float4 *>(P.m + (size_t)t * H) + i4);
             }
         }
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            ss += mreg[r].x * mreg[r].x + mreg[r].y * mreg[r].y + mreg[r].z * mreg[r].z + mreg[r].w * mreg[r].w;
         ss = block_sum(ss, S.red[0]);
         const float inv = P.post_norm ? 1.0f / sqrtf(ss / (float)H + P.eps) : 1.0f;
         float ss2 = 0.f;
@@ -750,34 +707,19 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     }
     __syncthreads();
     // job tables of this CTA: gate/up jobs round-robin (every CTA mixes shared-
-    // expert jobs, already in L2, with routed ones from HBM); down jobs
-    // round-robin when every SwiGLU input is staged at once, else in blocks
+    // expert jobs, already in L2, with routed ones from HBM); down jobs in
+    // contiguous blocks, so that a CTA's jobs share a slot and stage its input once
     const int na = S.nact, G = gridDim.x, c = blockIdx.x;
     const int J2 = (P.Is / 32 + na * (P.I / 32)) * P.nkp;
     const int J3 = (P.ndp_s + na * P.ndp_r) * (P.H / 32);
     const int n2 = J2 > c ? (J2 - 1 - c) / G + 1 : 0;
-    int d0, dstep, n3;
-    if (P.stage_all) {
-        d0 = c;
-        dstep = G;
-        n3 = J3 > c ? (J3 - 1 - c) / G + 1 : 0;
-    } else {
-        d0 = (int)((long long)J3 * c / G);
-        dstep = 1;
-        n3 = (int)((long long)J3 * (c + 1) / G) - d0;
-    }
+    const int d0 = (int)((long long)J3 * c / G), dstep = 1;
+    const int n3 = (int)((long long)J3 * (c + 1) / G) - d0;
     for (int i = threadIdx.x; i < n2 && i < kMaxJobs; i += blockDim.x) S.gujob[i] = make_gu_job(P, S, c + i * G);
     for (int i = threadIdx.x; i < n3 && i < kMaxJobs; i += blockDim.x) S.dnjob[i] = make_dn_job(P, S, d0 + i * dstep);
     if (threadIdx.x == 0) {
         S.ngu = n2 < kMaxJobs ? n2 : kMaxJobs;
         S.ndn = n3 < kMaxJobs ? n3 : kMaxJobs;
-        // stage-all: where each rowset's SwiGLU input starts (shared tokens first)
-        int off = 0;
-        for (int r = 0; r < T + n; ++r) {
-            S.rsoff[r] = off;
-            off += r < T ? P.Is : P.I;
-        }
-        S.rsoff[T + n] = off;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -792,26 +734,17 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
 }
 
 // x' = bf16(rmsnorm_no_scale(h)) pre-scaled for the code decode, and its chunk
-// sums, in S.stage.  One thread per 32-column chunk; element m of chunk c is
-// visited in the order (m + c) % 32 so that a warp's threads hit distinct banks.
+// sums, in S.stage.  One warp per 32-column chunk, a lane per column.
 __device__ __noinline__ void stage_x(const Params &P, Smem &S) {
-    const int T = P.T, H = P.H, nch = H / 32;
+    const int T = P.T, nch = P.H / 32, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     float *stage = S.stage;
-    for (int t = 0; t < T; ++t) {
-        const float r = S.rinv[t];
-        for (int c = threadIdx.x; c < nch; c += blockDim.x) {
-            const int i = t * nch + c;
-            float *row = stage + (size_t)i * 32;
-            float sx = 0.f;
-#pragma unroll 8
-            for (int mm = 0; mm < 32; ++mm) {
-                const int m = (mm + c) & 31;
-                const float x = bf16_bits_to_float(f32_to_bf16_bits_alu(row[m] * r));
-                row[m] = x * code_prescale(m & 7);
-                sx += x;
-            }
-            S.xs[i] = sx;
-        }
+    const float pre = code_prescale(lane & 7);
+    for (int i = wid; i < T * nch; i += kWarps) {
+        const int t = i / nch;
+        const float x = bf16_bits_to_float(f32_to_bf16_bits_alu(stage[(size_t)i * 32 + lane] * S.rinv[t]));
+        stage[(size_t)i * 32 + lane] = x * pre;
+        const float sx = warp_sum(x);
+        if (lane == 0) S.xs[i] = sx;
     }
     __syncthreads();
 }
@@ -891,7 +824,31 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, Ring ring) {
             const int rs = job_rowset(P, J, tt);
             P.gu_part[(((size_t)J.part * R + rs) * 2 + mm) * Kmax + J.rb * 32 + ln] = v;
         }
-        buf ^= 1;  // the next job reduces in the other buffer: no second barrier
+        // the last K part of (slot, row block) to finish forms a = silu(g) * u
+        // for its rows (partials ordered before the count by the fences)
+        __threadfence();
+        consumer_sync();
+        if (ctid == 0) {
+            const unsigned old = atomicAdd(&P.cnt_gu[J.slot * (Kmax / 32) + J.rb], 1u);
+            S.last = old == (unsigned)(P.nkp - 1);
+        }
+        consumer_sync();
+        if (S.last) {
+            __threadfence();
+            const size_t pstride = (size_t)R * 2 * Kmax;
+            for (int r = ctid; r < n * 32; r += kCWarps * 32) {
+                const int tt = r >> 5, ln = r & 31;
+                const size_t base = (size_t)job_rowset(P, J, tt) * 2 * Kmax + J.rb * 32 + ln;
+                float g = 0.f, u = 0.f;
+                for (int p = 0; p < P.nkp; ++p) {
+                    g += __ldcg(&P.gu_part[p * pstride + base]);
+                    u += __ldcg(&P.gu_part[p * pstride + base + Kmax]);
+                }
+                P.act[(size_t)job_rowset(P, J, tt) * Kmax + J.rb * 32 + ln] = silu_mul(g, u);
+            }
+            if (ctid == 0) P.cnt_gu[J.slot * (Kmax / 32) + J.rb] = 0u;
+        }
+        buf ^= 1;  // the next job reduces in the other buffer
     }
     return ok;
 }
@@ -931,20 +888,6 @@ __device__ __noinline__ bool dn_producer(const Params &P, Smem &S, const moe_lay
     return ok;
 }
 
-// SwiGLU input of one rowset and column: a = silu(sum of gate parts) * (sum of up parts).
-__device__ __forceinline__ float swiglu_in(const float *gu_part, size_t pstride, int nkp, int Kmax, int rs, int col) {
-    const size_t base = (size_t)rs * 2 * Kmax + col;
-    float g = 0.f, u = 0.f;
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        if (p < nkp) {
-            g += __ldcg(&gu_part[p * pstride + base]);
-            u += __ldcg(&gu_part[p * pstride + base + Kmax]);
-        }
-    }
-    return silu_mul(g, u);
-}
-
 // Chunk sums (sum of the unscaled values) of nchunks 32-float chunks of the
 // stage, one consumer thread per chunk, bank-rotated.
 __device__ __forceinline__ void chunk_sums(Smem &S, int nchunks) {
@@ -965,66 +908,34 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
     bool ok = true;
     int buf = 0;
-    const int T = P.T, Is = P.Is, I = P.I, ns = P.nslots, ndn = S.ndn, nkp = P.nkp, Kmax = P.Kmax;
-    const size_t pstride = (size_t)P.R * 2 * Kmax;
-    const float *gu_part = P.gu_part;
+    const int T = P.T, k = P.k, H = P.H, ns = P.nslots, ndn = S.ndn, Kmax = P.Kmax;
+    // down jobs per row block in this layer: every part of the shared expert and of each active slot
+    const unsigned dn_per_rb = (unsigned)(P.ndp_s + S.nact * P.ndp_r);
     float *stage = S.stage;
-    if (P.stage_all) {
-        // every rowset's SwiGLU input, rowset r at S.rsoff[r] (shared tokens, then routed positions)
-        const int nrs = T + T * P.k, F = S.rsoff[nrs];
-        for (int b0 = ctid; b0 < F; b0 += 4 * kCWarps * 32) {
-            float a[4];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const int i = b0 + v * kCWarps * 32;
-                a[v] = 0.f;
-                if (i < F) {
-                    int rs = 0;
-                    while (S.rsoff[rs + 1] <= i) ++rs;  // short scan, no division
-                    a[v] = swiglu_in(gu_part, pstride, nkp, Kmax, rs, i - S.rsoff[rs]);
-                }
-            }
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const int i = b0 + v * kCWarps * 32;
-                if (i < F) stage[i] = a[v] * code_prescale(i & 7);  // rowset starts are multiples of 64
-            }
-        }
-        consumer_sync();
-        chunk_sums(S, F / 32);
-        consumer_sync();
-    }
     int staged_slot = -1, staged_part = -1;
     for (int i = 0; i < ndn; ++i) {
         const JobDesc J = S.dnjob[i];
-        const int ng = J.g1 - J.g0, n = J.n;
-        const float *xb;
-        const float *xsb;
-        int stride;
-        if (P.stage_all) {
-            const int off = S.rsoff[J.slot == 0 ? 0 : T + J.seg0] + J.g0 * 64;
-            xb = stage + off;
-            xsb = S.xs + off / 32;
-            stride = J.slot == 0 ? Is : I;
-        } else {
-            const int ld = ng * 64;
-            if (J.slot != staged_slot || J.part != staged_part) {
-                // this slot's tokens, columns [g0*64, g1*64) only: row tt at tt * ld
-                for (int tt = 0; tt < n; ++tt) {
-                    const int rs = job_rowset(P, J, tt);
-                    for (int c = ctid; c < ld; c += kCWarps * 32)
-                        stage[tt * ld + c] = swiglu_in(gu_part, pstride, nkp, Kmax, rs, J.g0 * 64 + c) *
-                                             code_prescale(c & 7);
-                }
-                consumer_sync();
-                chunk_sums(S, n * 2 * ng);
-                staged_slot = J.slot;
-                staged_part = J.part;
-                consumer_sync();
+        const int ng = J.g1 - J.g0, n = J.n, ld = ng * 64;
+        if (J.slot != staged_slot || J.part != staged_part) {
+            // this slot's SwiGLU rows, columns [g0*64, g1*64): token tt at tt * ld
+            const int q4 = ld / 4;
+            for (int e = ctid; e < n * q4; e += kCWarps * 32) {
+                const int tt = e / q4, c4 = e - tt * q4;
+                const float4 a = __ldcg(reinterpret_cast<const float4 *>(
+                                            P.act + (size_t)job_rowset(P, J, tt) * Kmax + J.g0 * 64) + c4);
+                const int c = 4 * c4;  // c % 8 is 0 or 4
+                float4 v;
+                v.x = a.x * code_prescale(c & 7);
+                v.y = a.y * code_prescale((c + 1) & 7);
+                v.z = a.z * code_prescale((c + 2) & 7);
+                v.w = a.w * code_prescale((c + 3) & 7);
+                reinterpret_cast<float4 *>(stage + (size_t)tt * ld)[c4] = v;
             }
-            xb = stage;
-            xsb = S.xs;
-            stride = ld;
+            consumer_sync();
+            chunk_sums(S, n * 2 * ng);
+            staged_slot = J.slot;
+            staged_part = J.part;
+            consumer_sync();
         }
         const bool got = mbar_wait(&S.full[ring.s], ring.ph, P.err, kErrFull);
         float *Rb = S.red[buf];
@@ -1035,8 +946,8 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
             const uint32_t sbw =
                 reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane];
             float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            // token tt's row at tt * stride, its chunk sums at tt * stride / 32
-            group_dot_n(codes, sbw, xb + gi * 64, xsb + 2 * gi, nullptr, stride, n, acc, lane);
+            // token tt's row at tt * ld, its chunk sums at tt * ld / 32
+            group_dot_n(codes, sbw, stage + gi * 64, S.xs + 2 * gi, nullptr, ld, n, acc, lane);
 #pragma unroll
             for (int tt = 0; tt < kMaxT; ++tt)
                 if (tt < n) Rb[(gi * kMaxT + tt) * 32 + lane] = acc[tt >> 2][tt & 3];
@@ -1052,9 +963,32 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
             for (int g2 = 0; g2 < ng; ++g2) v += Rb[(g2 * kMaxT + tt) * 32 + ln];
             const int row = J.rb * 32 + ln;
             if (J.slot == 0)
-                P.sh[((size_t)J.part * T + tt) * P.H + row] = v;
+                P.sh[((size_t)J.part * T + tt) * H + row] = v;
             else
-                P.y[((size_t)J.part * T * P.k + S.perm[J.seg0 + tt]) * P.H + row] = v;
+                P.y[((size_t)J.part * T * k + S.perm[J.seg0 + tt]) * H + row] = v;
+        }
+        // the last job of this row block to finish forms the combine for its rows
+        __threadfence();
+        consumer_sync();
+        if (ctid == 0) {
+            const unsigned old = atomicAdd(&P.cnt_dn[J.rb], 1u);
+            S.last = old == dn_per_rb - 1u;
+        }
+        consumer_sync();
+        if (S.last) {
+            __threadfence();
+            for (int r = ctid; r < T * 32; r += kCWarps * 32) {
+                const int t = r >> 5, row = J.rb * 32 + (r & 31);
+                float mv = 0.f;
+                for (int s2 = 0; s2 < k; ++s2) {
+                    float yv = 0.f;
+                    for (int dp = 0; dp < P.ndp_r; ++dp) yv += __ldcg(&P.y[((size_t)dp * T * k + t * k + s2) * H + row]);
+                    mv = fmaf(S.wts[t * k + s2], yv, mv);
+                }
+                for (int dp = 0; dp < P.ndp_s; ++dp) mv += __ldcg(&P.sh[((size_t)dp * T + t) * H + row]);
+                P.m[(size_t)t * H + row] = mv;
+            }
+            if (ctid == 0) P.cnt_dn[J.rb] = 0u;
         }
         buf ^= 1;
     }
@@ -1142,7 +1076,7 @@ static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exce
 static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
 
 struct DecodeWs {
-    size_t bar, logits, gu_part, y, sh, total, zero_bytes;
+    size_t bar, cnt_gu, cnt_dn, logits, gu_part, act, y, sh, m, total, zero_bytes;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1161,11 +1095,15 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
         return o;
     };
     d.bar = take(256);
+    d.cnt_gu = take(sizeof(unsigned) * (size_t)R * (Kmax / 32));
+    d.cnt_dn = take(sizeof(unsigned) * (size_t)(w->H / 32));
     d.zero_bytes = off;
     d.logits = take(sizeof(double) * (size_t)T * w->E);
     d.gu_part = take(sizeof(float) * (size_t)nkp * R * 2 * Kmax);
+    d.act = take(sizeof(float) * (size_t)R * Kmax);
     d.y = take(sizeof(float) * (size_t)ndp_r * T * w->k * w->H);
     d.sh = take(sizeof(float) * (size_t)ndp_s * T * w->H);
+    d.m = take(sizeof(float) * (size_t)T * w->H);
     d.total = off;
     return d;
 }
@@ -1176,30 +1114,24 @@ size_t decode_stack_status_offset() { return sizeof(unsigned); }
 
 // Split of the shared-memory pool between the ring and the input stage for
 // calls of T tokens on layers shaped like w; false if the shape does not fit.
-static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots, int *stage_all) {
-    const long all = (long)T * w.Is + (long)T * w.k * w.I;  // every rowset's SwiGLU input
-    const long th = (long)T * w.H;
-    for (int sa = 1; sa >= 0; --sa) {
-        if (sa && (all > dec::kStageFloats || all / 32 > dec::kMaxXs)) continue;
-        long stage = th > (sa ? all : (long)T * dec::kDnGroups * 64) ? th : (sa ? all : (long)T * dec::kDnGroups * 64);
-        if (stage > dec::kStageFloats) return false;
-        stage = (stage + 31) & ~31L;  // keep the stage 128-byte aligned
-        long ns = (dec::kPoolBytes - stage * 4) / dec::kSlotBytes;
-        if (ns > dec::kMaxStages) ns = dec::kMaxStages;
-        const long ring = ns * dec::kSlotBytes;
-        const long rows = grid > 0 ? (w.E + grid - 1) / grid : w.E;
-        const long rcopy = 2L * w.H + rows * w.H + 2 * (rows * (w.H / 64) * 2 + 32);
-        if (ns < 3 || (long)T * w.E * 8 > ring || rcopy > ring) continue;
-        *nslots = (int)ns;
-        *stage_all = sa;
-        return true;
-    }
-    return false;
+static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots) {
+    const long th = (long)T * w.H, tdn = (long)T * dec::kDnGroups * 64;
+    long stage = th > tdn ? th : tdn;
+    if (stage > dec::kStageFloats || stage / 32 > dec::kMaxXs) return false;
+    stage = (stage + 31) & ~31L;  // keep the stage 128-byte aligned
+    long ns = (dec::kPoolBytes - stage * 4) / dec::kSlotBytes;
+    if (ns > dec::kMaxStages) ns = dec::kMaxStages;
+    const long ring = ns * dec::kSlotBytes;
+    const long rows = grid > 0 ? (w.E + grid - 1) / grid : w.E;
+    const long rcopy = 2L * w.H + rows * w.H + 2 * (rows * (w.H / 64) * 2 + 32);
+    if (ns < 3 || (long)T * w.E * 8 > ring || rcopy > ring) return false;
+    *nslots = (int)ns;
+    return true;
 }
 
 bool decode_stack_fits(const moe_layer_w *w, int T, int grid) {
-    int a, b;
-    return decode_layout(*w, T, grid, &a, &b);
+    int a;
+    return decode_layout(*w, T, grid, &a);
 }
 
 int decode_stack_max_tokens() { return dec::kMaxT; }
@@ -1230,14 +1162,18 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.nkp = (w.H / 64 + dec::kGuPartGroups - 1) / dec::kGuPartGroups;
     P.ndp_r = (w.I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
     P.ndp_s = (w.Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
-    if (!decode_layout(w, T, grid, &P.nslots, &P.stage_all)) return cudaErrorInvalidValue;
+    if (!decode_layout(w, T, grid, &P.nslots)) return cudaErrorInvalidValue;
     char *base = static_cast<char *>(ws);
     P.bar = reinterpret_cast<unsigned *>(base + d.bar);
     P.err = reinterpret_cast<int *>(base + d.bar + sizeof(unsigned));
     P.logits = reinterpret_cast<double *>(base + d.logits);
+    P.cnt_gu = reinterpret_cast<unsigned *>(base + d.cnt_gu);
+    P.cnt_dn = reinterpret_cast<unsigned *>(base + d.cnt_dn);
     P.gu_part = reinterpret_cast<float *>(base + d.gu_part);
+    P.act = reinterpret_cast<float *>(base + d.act);
     P.y = reinterpret_cast<float *>(base + d.y);
     P.sh = reinterpret_cast<float *>(base + d.sh);
+    P.m = reinterpret_cast<float *>(base + d.m);
 
     const size_t smem = sizeof(dec::Smem);
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(dec::decode_stack_kernel), smem);

@@ -64,14 +64,14 @@ constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // input columns per k-block
 constexpr int kKS = 2;            // k-blocks per code stage
 constexpr int kCodeSlots = 4;     // code stages in flight
-constexpr int kABufs = 2;         // BF16 weight tiles (per k-block)
-constexpr int kBBufs = 3;         // token tiles (per k-block)
+constexpr int kABufs = 3;         // FP16 weight stages (32 KiB each)
+constexpr int kBBufs = 3;         // token slots of 16 KiB: 128 / N k-blocks of an N-token tile each
 constexpr int kMaxN = 128;        // tokens per tile
 constexpr int kBoxRows = 16;      // rows of one TMA box of the token matrix
-constexpr int kDqWarps = 8;
-constexpr int kProdWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 10 * 32;
+constexpr int kDqWarps = 16;      // dequant (and epilogue) warps: one 32-code record per thread per stage
+constexpr int kProdWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 18 * 32;
 constexpr int kTmemCols = 256;
 constexpr int kATileBytes = kBM * kBK * 2;       // 16 KiB
 constexpr int kBBufBytes = kMaxN * kBK * 2;      // 16 KiB
@@ -80,12 +80,17 @@ constexpr unsigned long long kWaitNs = 1000000000ull;
 
 enum { kErrCodeFull = 1, kErrCodeEmpty, kErrAFull, kErrAEmpty, kErrBFull, kErrBEmpty, kErrAccFull, kErrAccEmpty };
 
+// Shared-memory plan of the kernel for NMAT weight matrices per tile (2:
+// gate and up, 1: down).  A weight stage holds kAK k-blocks of every matrix
+// (NMAT * kAK = 2 tiles of 128 x 64 FP16), so that each of the 512 dequant
+// threads converts exactly one 32-code record per stage.
 template <int NMAT>
 struct Lay {
+    static constexpr int kAK = 2 / NMAT;
     static constexpr int kCodeBytes = NMAT * 4 * kKS * 1024;
     static constexpr int kSbBytes = NMAT * 4 * kKS * 128;
     static constexpr int kSlotBytes = kCodeBytes + kSbBytes;
-    static constexpr int kABytes = NMAT * kATileBytes;
+    static constexpr int kABytes = NMAT * kAK * kATileBytes;
     static constexpr int kAOff = 0;
     static constexpr int kBOff = kAOff + kABufs * kABytes;
     static constexpr int kCodeOff = kBOff + kBBufs * kBBufBytes;
@@ -96,6 +101,8 @@ struct Lay {
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
 };
 static_assert(Lay<2>::kAlloc <= 227 * 1024, "gate/up tile buffers exceed shared memory");
+static_assert(kDqWarps * 32 == 2 * 2 * kBM, "one record (row, 32 codes) per dequant thread and stage");
+static_assert(kKS % Lay<1>::kAK == 0 && kKS % Lay<2>::kAK == 0, "a code stage holds whole weight stages");
 
 struct Params {
     const uint32_t *q[2], *sb[2];    // routed matrices (tiled layout), stacked over experts
@@ -243,8 +250,18 @@ __device__ __forceinline__ uint32_t f16x2_from_bf16x2(uint32_t v) {
 }
 
 // 8 codes of one word -> 8 FP16 weights s*q + b, in the chunk order
-// (0,4,1,5,2,6,3,7).  0x6400 | q is the FP16 number 1024 + q, so subtracting
-// 1024 gives q exactly; the FMA with the group's scale and bias then rounds once.
+// (0,4,1,5,2,6,3,7).  A code moved to mantissa bits 6..9 of an FP16 half with
+// a zero exponent is the subnormal q * 2^-18, so one FMA with the scale
+// pre-multiplied by 2^18 (s2) and the bias gives s*q + b with a single
+// rounding.  Valid while s * 2^18 fits FP16 (|s| < 0.25).
+__device__ __forceinline__ uint4 dequant_word_sub(uint32_t w, uint32_t s2, uint32_t b2) {
+    constexpr uint32_t kM = 0x03C003C0u;
+    return make_uint4(h2_fma((w << 6) & kM, s2, b2), h2_fma((w << 2) & kM, s2, b2), h2_fma((w >> 2) & kM, s2, b2),
+                      h2_fma((w >> 6) & kM, s2, b2));
+}
+
+// The same for any scale: 0x6400 | q is the FP16 number 1024 + q, so
+// subtracting 1024 gives q exactly before the FMA with the scale and bias.
 __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t b2) {
     constexpr uint32_t kM = 0x000F000Fu, kMagic = 0x64006400u, kOne = 0x3C003C00u, kNeg1024 = 0xE400E400u;
     const uint32_t p0 = h2_fma((w & kM) | kMagic, kOne, kNeg1024);
@@ -377,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                     qb[m] = (t.e < 0 ? P.sq[m] : P.q[m]) + mrb * C * 128;
                     sbb[m] = (t.e < 0 ? P.ssb[m] : P.sb[m]) + mrb * G * 32;
                 }
-                const int nbox = t.N / kBoxRows;
+                const int nbox = t.N / kBoxRows, bkb = kMaxN / t.N;  // k-blocks per token slot
                 for (int kb = 0; kb < nkb && ok; ++kb) {
                     if (kb % kKS == 0) {
                         const int s = cs % kCodeSlots;
@@ -398,16 +415,20 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                             }
                         ++cs;
                     }
-                    const int b = kbc % kBBufs;
-                    if (kbc >= kBBufs && !mbar_wait(b_empty(b), ((kbc / kBBufs) & 1) ^ 1, P.err, kErrBEmpty)) {
-                        ok = false;
-                        break;
+                    if (kb % bkb == 0) {  // a new token slot: this and the next bkb - 1 k-blocks
+                        const int b = kbc % kBBufs;
+                        if (kbc >= kBBufs && !mbar_wait(b_empty(b), ((kbc / kBBufs) & 1) ^ 1, P.err, kErrBEmpty)) {
+                            ok = false;
+                            break;
+                        }
+                        const int nk = min(bkb, nkb - kb);
+                        mbar_expect_tx(b_full(b), (unsigned)(nk * nbox * kBoxBytes));
+                        for (int i = 0; i < nk; ++i)
+                            for (int j = 0; j < nbox; ++j)
+                                tma_load_2d(sB + (uint32_t)b * kBBufBytes + (uint32_t)((i * nbox + j) * kBoxBytes), &tmB,
+                                            (kb + i) * kBK, t.brow + j * kBoxRows, b_full(b));
+                        ++kbc;
                     }
-                    mbar_expect_tx(b_full(b), (unsigned)(nbox * kBoxBytes));
-                    for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(sB + (uint32_t)b * kBBufBytes + (uint32_t)j * kBoxBytes, &tmB, kb * kBK,
-                                    t.brow + j * kBoxRows, b_full(b));
-                    ++kbc;
                 }
             }
             // let this CTA's own copies land before it stops (bounded)
@@ -419,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t kbc = 0, ic = 0;
+            uint32_t asc = 0, kbc = 0, ic = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
                 Tile t;
@@ -429,26 +450,38 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                     tc_fence_after();
                 }
                 const uint32_t idesc = idesc_f16(t.N);
-                const int nkb = t.K / kBK;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const int a = kbc % kABufs, b = kbc % kBBufs;
-                    if (!mbar_wait(a_full(a), (kbc / kABufs) & 1, P.err, kErrAFull) ||
-                        !mbar_wait(b_full(b), (kbc / kBBufs) & 1, P.err, kErrBFull)) {
+                const int nkb = t.K / kBK, bkb = kMaxN / t.N;
+                for (int ks = 0; ks < nkb && ok; ks += L::kAK) {
+                    const int a = asc % kABufs;
+                    if (!mbar_wait(a_full(a), (asc / kABufs) & 1, P.err, kErrAFull)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t abase = sA + (uint32_t)a * L::kABytes, bbase = sB + (uint32_t)b * kBBufBytes;
+                    const uint32_t abase = sA + (uint32_t)a * L::kABytes;
+                    for (int kbi = 0; kbi < L::kAK && ks + kbi < nkb; ++kbi) {
+                        const int kb = ks + kbi, b = kbc % kBBufs;
+                        if (kb % bkb == 0 && !mbar_wait(b_full(b), (kbc / kBBufs) & 1, P.err, kErrBFull)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t bbase = sB + (uint32_t)b * kBBufBytes + (uint32_t)((kb % bkb) * t.N * kBK * 2);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
 #pragma unroll
-                        for (int m = 0; m < NMAT; ++m)
-                            mma_f16(tmem + (uint32_t)(m * t.N), sw128_desc(abase + m * kATileBytes + kk * 32),
-                                     sw128_desc(bbase + kk * 32), idesc, (kb | kk) != 0);
+                            for (int m = 0; m < NMAT; ++m)
+                                mma_f16(tmem + (uint32_t)(m * t.N),
+                                        sw128_desc(abase + (m * L::kAK + kbi) * kATileBytes + kk * 32),
+                                        sw128_desc(bbase + kk * 32), idesc, ((ks + kbi) | kk) != 0);
+                        }
+                        if (kb % bkb == bkb - 1 || kb == nkb - 1) {  // last k-block of this token slot
+                            mma_commit(b_empty(b));
+                            ++kbc;
+                        }
                     }
+                    if (!ok) break;
                     mma_commit(a_empty(a));
-                    mma_commit(b_empty(b));
-                    ++kbc;
+                    ++asc;
                 }
                 if (!ok) break;
                 mma_commit(acc_full);
@@ -460,99 +493,102 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
         }
     } else {
         // ---------------------------------------------------------- dequant + epilogue
-        const int r = threadIdx.x & (kBM - 1), half = threadIdx.x >> 7;
+        // thread -> one record per weight stage: tile row r, matrix m, k-block kbi of the stage, 32-code half
+        const int r = threadIdx.x & (kBM - 1), j4 = threadIdx.x >> 7;
+        const int m = NMAT == 2 ? (j4 >> 1) : 0, kbi = NMAT == 2 ? 0 : (j4 >> 1), half = j4 & 1;
         const int rbl = r >> 5, rl = r & 31;
-        uint32_t cs = 0, kbc = 0, ic = 0;
+        uint32_t cs = 0, asc = 0, ic = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
             Tile t;
             if (!get_tile(P, it, t)) continue;
             const int nkb = t.K / kBK;
-            const bool valid = r < t.rv;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int kbs = kb % kKS, s = cs % kCodeSlots;
-                if (kbs == 0 && !__all_sync(0xffffffffu, mbar_wait(code_full(s), (cs / kCodeSlots) & 1, P.err,
-                                                                    kErrCodeFull))) {
+            for (int ks = 0; ks < nkb; ks += L::kAK) {
+                const int s = cs % kCodeSlots, kbs = ks % kKS + kbi;
+                if (ks % kKS == 0 && !__all_sync(0xffffffffu, mbar_wait(code_full(s), (cs / kCodeSlots) & 1, P.err,
+                                                                          kErrCodeFull))) {
                     ok = false;
                     break;
                 }
                 const unsigned char *slot = gbase + L::kCodeOff + (size_t)s * L::kSlotBytes;
-                uint4 c[NMAT];
-                uint32_t sbw[NMAT];
+                const bool valid = r < t.rv && ks + kbi < nkb;
+                uint4 c = make_uint4(0u, 0u, 0u, 0u);
+                uint32_t sbw = 0;
                 if (valid) {
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        c[m] = *reinterpret_cast<const uint4 *>(slot + ((((m * 4 + rbl) * kKS + kbs) * 2 + half) * 512) +
-                                                                rl * 16);
-                        sbw[m] = *reinterpret_cast<const uint32_t *>(slot + L::kCodeBytes +
-                                                                     (((m * 4 + rbl) * kKS + kbs) * 32 + rl) * 4);
-                    }
+                    c = *reinterpret_cast<const uint4 *>(slot + ((((m * 4 + rbl) * kKS + kbs) * 2 + half) * 512) + rl * 16);
+                    sbw = *reinterpret_cast<const uint32_t *>(slot + L::kCodeBytes + (((m * 4 + rbl) * kKS + kbs) * 32 + rl) * 4);
                 }
-                if (kbs == kKS - 1 || kb == nkb - 1) {
+                if ((ks + L::kAK) % kKS == 0 || ks + L::kAK >= nkb) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(code_empty(s));
                     ++cs;
                 }
-                const int a = kbc % kABufs;
-                if (kbc >= kABufs &&
-                    !__all_sync(0xffffffffu, mbar_wait(a_empty(a), ((kbc / kABufs) & 1) ^ 1, P.err, kErrAEmpty))) {
+                const int a = asc % kABufs;
+                if (asc >= kABufs &&
+                    !__all_sync(0xffffffffu, mbar_wait(a_empty(a), ((asc / kABufs) & 1) ^ 1, P.err, kErrAEmpty))) {
                     ok = false;
                     break;
                 }
                 if (valid) {
-                    unsigned char *arow = gbase + L::kAOff + (size_t)a * L::kABytes + r * 128;
+                    unsigned char *arow =
+                        gbase + L::kAOff + (size_t)a * L::kABytes + (size_t)(m * L::kAK + kbi) * kATileBytes + r * 128;
+                    const float sf = __uint_as_float(sbw << 16), bf = __uint_as_float(sbw & 0xffff0000u);
+                    const uint32_t b2 = f16x2_from_f32(bf, bf);
+                    const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+                    uint4 o[4];
+                    if (fabsf(sf) < 0.25f) {
+                        const uint32_t s2 = f16x2_from_f32(sf * 262144.0f, sf * 262144.0f);
 #pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        const float sf = __uint_as_float(sbw[m] << 16), bf = __uint_as_float(sbw[m] & 0xffff0000u);
-                        const uint32_t s2 = f16x2_from_f32(sf, sf), b2 = f16x2_from_f32(bf, bf);
-                        const uint32_t wv[4] = {c[m].x, c[m].y, c[m].z, c[m].w};
+                        for (int wi = 0; wi < 4; ++wi) o[wi] = dequant_word_sub(wv[wi], s2, b2);
+                    } else {
+                        const uint32_t s2 = f16x2_from_f32(sf, sf);
 #pragma unroll
-                        for (int wi = 0; wi < 4; ++wi) {
-                            const int ch = (4 * half + wi) ^ (r & 7);
-                            *reinterpret_cast<uint4 *>(arow + m * kATileBytes + ch * 16) = dequant_word(wv[wi], s2, b2);
-                        }
+                        for (int wi = 0; wi < 4; ++wi) o[wi] = dequant_word(wv[wi], s2, b2);
                     }
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi)
+                        *reinterpret_cast<uint4 *>(arow + (((4 * half + wi) ^ (r & 7)) << 4)) = o[wi];
                 }
                 // generic-proxy stores -> visible to the tensor core (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(a_full(a));
-                ++kbc;
+                ++asc;
             }
             if (!ok) break;
-            // epilogue: warp w reads TMEM lanes 32*(w%4).. (tile rows), columns of chunks c with c%2 == w/4
+            // epilogue: warp w reads TMEM lanes 32*(w%4).. (tile rows), chunks of 8 columns c with c%4 == w/4
             if (!__all_sync(0xffffffffu, mbar_wait(acc_full, ic & 1, P.err, kErrAccFull))) break;
             tc_fence_after();
-            const int q4 = warp & 3, hsel = warp >> 2;
+            const int q4 = warp & 3, cg = warp >> 2;
             const int row = t.mt * kBM + q4 * 32 + lane;
             const bool rvalid = q4 * 32 < t.rv;  // warp-uniform
             const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16);
             if (rvalid) {
-                for (int ch = hsel; ch < t.N / 8; ch += 2) {
+                for (int ch = cg; ch < t.N / 8; ch += 4) {
                     if (NMAT == 2) {
                         float g[8], u[8];
                         tmem_ld8(taddr + ch * 8, g);
                         tmem_ld8(taddr + t.N + ch * 8, u);
                         const int col = (row & ~7) | chunk_pos(row & 7);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int n = ch * 8 + j;
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int n = ch * 8 + jj;
                             if (n < t.n) {
-                                const float a = fminf(fmaxf(silu_mul(g[j], u[j]), -65504.f), 65504.f);
-                                P.act[(size_t)(t.brow + n) * P.act_ld + col] = __half_as_ushort(__float2half_rn(a));
+                                const float av = fminf(fmaxf(silu_mul(g[jj], u[jj]), -65504.f), 65504.f);
+                                P.act[(size_t)(t.brow + n) * P.act_ld + col] = __half_as_ushort(__float2half_rn(av));
                             }
                         }
                     } else {
                         float v[8];
                         tmem_ld8(taddr + ch * 8, v);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int n = ch * 8 + j;
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int n = ch * 8 + jj;
                             if (n < t.n) {
                                 if (t.e < 0)
-                                    P.sh[(size_t)(t.seg0 + n) * P.H + row] = v[j];
+                                    P.sh[(size_t)(t.seg0 + n) * P.H + row] = v[jj];
                                 else
-                                    P.y[(size_t)__ldg(P.perm + t.seg0 + n) * P.H + row] = v[j];
+                                    P.y[(size_t)__ldg(P.perm + t.seg0 + n) * P.H + row] = v[jj];
                             }
                         }
                     }

@@ -43,12 +43,15 @@ router_logits_kernel(const uint32_t *__restrict__ rq, const uint16_t *__restrict
         ss += v * v;
     }
     ss = block_sum(ss, red);
-    const double r = sqrt(ss / (double)H + (double)eps);
-    const double sqrt_h = sqrt((double)H);
+    // one division per CTA: x / r is taken as x * (1 / r), which differs from
+    // the quotient by at most an ulp of fp64 -- far below what moves a logit
+    // gap or a BF16 rounding
+    const double rinv = 1.0 / sqrt(ss / (double)H + (double)eps);
+    const double inv_sqrt_h = 1.0 / sqrt((double)H);
     const bool write_xe = (xe != nullptr) && blockIdx.x == 0;
     for (int i = threadIdx.x; i < H; i += blockDim.x) {
-        const double xn = (double)bf16_bits_to_float(ht[i]) / r;
-        const double xs = xn * (double)bf16_bits_to_float(router_scale[i]) / sqrt_h;
+        const double xn = (double)bf16_bits_to_float(ht[i]) * rinv;
+        const double xs = xn * (double)bf16_bits_to_float(router_scale[i]) * inv_sqrt_h;
         xsT[(i & 15) * ld + (i >> 4)] = xs;
         if (write_xe) xe[(size_t)t * H + i] = f64_to_bf16_bits(xn);
     }
