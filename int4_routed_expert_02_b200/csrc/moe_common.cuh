@@ -85,23 +85,27 @@ constexpr float kCodeUnscale = 0x1p49f;
 
 __host__ __device__ constexpr int code_pos(int j) { return j < 6 ? j : j - 3; }
 
-__host__ __device__ constexpr float code_prescale(int j) {
-    return code_pos(j) == 0 ? 0x1p100f
-         : code_pos(j) == 1 ? 0x1p96f
-         : code_pos(j) == 2 ? 0x1p92f
-         : code_pos(j) == 3 ? 0x1p88f
-         : code_pos(j) == 4 ? 0x1p84f
-                            : 0x1p80f;
+// 2^(100 - 4 * code_pos(j)): built from its exponent field, so that a
+// runtime j costs a few integer operations and no table or branch.
+__host__ __device__ inline float code_prescale(int j) {
+    const unsigned e = 127u + 100u - 4u * (unsigned)code_pos(j & 7);
+#ifdef __CUDA_ARCH__
+    return __uint_as_float(e << 23);
+#else
+    union { unsigned u; float f; } v{e << 23};
+    return v.f;
+#endif
 }
 
-// 1 / code_prescale(j), exact (a power of two).
-__host__ __device__ constexpr float code_unprescale(int j) {
-    return code_pos(j) == 0 ? 0x1p-100f
-         : code_pos(j) == 1 ? 0x1p-96f
-         : code_pos(j) == 2 ? 0x1p-92f
-         : code_pos(j) == 3 ? 0x1p-88f
-         : code_pos(j) == 4 ? 0x1p-84f
-                            : 0x1p-80f;
+// 1 / code_prescale(j) = 2^(4 * code_pos(j) - 100), exact.
+__host__ __device__ inline float code_unprescale(int j) {
+    const unsigned e = 127u - 100u + 4u * (unsigned)code_pos(j & 7);
+#ifdef __CUDA_ARCH__
+    return __uint_as_float(e << 23);
+#else
+    union { unsigned u; float f; } v{e << 23};
+    return v.f;
+#endif
 }
 
 struct Decoded8 {

@@ -16,15 +16,15 @@
 //   P2  top-k + softmax * per_expert_scale and bucketing, by rank counting
 //       (every CTA, redundantly, so no barrier is needed before the experts),
 //       and this CTA's job tables for the two expert phases
-//   P2' gate/up dequant-GEMV jobs (32 rows x one K part of <= 16 groups of
-//       both matrices, streamed in stages of <= 8 groups), partial sums to
-//       global; the last K part of a (slot, row block) to finish -- found
-//       with an atomic counter -- forms a = silu(g) * u for those rows
+//   P2' gate/up dequant-GEMV jobs (32 rows of both matrices over the whole
+//       input, streamed in stages of <= 8 groups); each job forms
+//       a = silu(g) * u for its rows
 //   --- grid barrier ---
 //   P3  down dequant-GEMV jobs (32 rows x <= 16 groups of one slot), in
 //       contiguous blocks per CTA so that a CTA stages each slot's a once;
-//       the last job of a row block to finish forms the combine
-//       m = sum_s w_s y_s + shared for those rows
+//       the last job of a row block to finish (an atomic count, read one
+//       job later) forms the combine m = sum_s w_s y_s + shared for those
+//       rows at the end of the phase
 //   --- grid barrier ---
 //
 // Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
@@ -53,7 +53,6 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kProducerWarp = kCWarps;
 constexpr int kMaxStages = 9;                 // ring slots: as many as fit beside the input stage
 constexpr int kStageGroups = 8;               // gate/up stage: <= 8 groups of each of the two matrices
-constexpr int kGuPartGroups = 16;             // gate/up job: one K part of <= 16 groups
 constexpr int kDnGroups = 16;                 // down job: <= 16 groups, one stage
 constexpr int kCodeBytesPerGroup = 1024;      // 32 rows x 64 codes x 4 bits
 constexpr int kSbBytesPerGroup = 128;         // 32 rows x (scale, bias)
@@ -77,14 +76,12 @@ struct Params {
     int L, T, chained, post_norm;
     float layer_scalar, eps;
     int H, E, k, I, Is, Kmax, R;
-    int nkp, ndp_r, ndp_s;
+    int ndp_r, ndp_s;
     int nslots;      // ring slots (the rest of the pool is the input stage)
     unsigned *bar;
     int *err;
-    unsigned *cnt_gu;  // [1 + T*k][Kmax/32]: K parts done per (slot, row block); reset by the last
     unsigned *cnt_dn;  // [H/32]: down jobs done per row block; reset by the last
     double *logits;  // [T,E]
-    float *gu_part;  // [nkp][R][2][Kmax]: gate (0) and up (1) partial sums per K part
     float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs)
     float *y;        // [ndp_r][T*k][H]
     float *sh;       // [ndp_s][T][H]
@@ -125,7 +122,8 @@ struct Smem {
     float rinv[kMaxT];
     int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
     int flag;
-    int last;      // consumer broadcast: this CTA finished the last job of a row block
+    int nlast;                 // row blocks whose combine this CTA forms at the end of the down phase
+    int16_t last_rb[kMaxJobs];
 };
 
 // Position in the ring: stage sequence number q, its slot s and phase parity ph.
@@ -178,7 +176,7 @@ __device__ __forceinline__ bool mbar_test(unsigned long long *b, unsigned parity
 __device__ __forceinline__ int ldcg_int(const int *p) { return __ldcg(p); }
 
 // Bounded wait for the phase with `parity` of mbarrier `b` to complete.
-__device__ bool mbar_wait(unsigned long long *b, unsigned parity, int *err, int code) {
+__device__ __noinline__ bool mbar_wait(unsigned long long *b, unsigned parity, int *err, int code) {
     if (mbar_test(b, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (unsigned it = 1;; ++it) {
@@ -194,7 +192,7 @@ __device__ bool mbar_wait(unsigned long long *b, unsigned parity, int *err, int 
 }
 
 // Bounded wait used only when draining: ignores the error flag.
-__device__ void mbar_drain(unsigned long long *b, unsigned parity) {
+__device__ __noinline__ void mbar_drain(unsigned long long *b, unsigned parity) {
     const unsigned long long t0 = globaltimer();
     while (!mbar_test(b, parity)) {
         if (globaltimer() - t0 > kWaitNs) return;
@@ -229,7 +227,7 @@ __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;"
 // Grid-wide barrier number `nth` (1, 2, ...) on a monotonically increasing
 // counter; bounded.  Returns false (in every thread of the CTA alike) if any
 // CTA recorded an error.
-__device__ bool grid_sync(const Params &P, unsigned nth, int *verdict) {
+__device__ __noinline__ bool grid_sync(const Params &P, unsigned nth, int *verdict) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -258,39 +256,35 @@ __device__ bool grid_sync(const Params &P, unsigned nth, int *verdict) {
 
 // ------------------------------------------------------------------ jobs
 
-// Job j of the gate/up phase (all divisions happen here, once per job).
-__device__ JobDesc make_gu_job(const Params &P, const Smem &S, int j) {
+// Job j of the gate/up phase: 32 rows of both matrices over the whole input
+// (all divisions happen here, once per job).
+__device__ __noinline__ JobDesc make_gu_job(const Params &P, const Smem &S, int j) {
     JobDesc J;
-    const int GH = P.H / 64;
-    const int A = (P.Is / 32) * P.nkp;
-    int part;
+    const int A = P.Is / 32;
     if (j < A) {
         J.slot = 0;
-        J.rb = (int16_t)(j / P.nkp);
-        part = j - J.rb * P.nkp;
+        J.rb = (int16_t)j;
         J.n = (int16_t)P.T;
         J.seg0 = 0;
         J.e = -1;
     } else {
-        const int B = (P.I / 32) * P.nkp;
+        const int B = P.I / 32;
         const int jj = j - A;
         const int i = jj / B;
-        const int r = jj - i * B;
         J.slot = (int16_t)(1 + i);
-        J.rb = (int16_t)(r / P.nkp);
-        part = r - J.rb * P.nkp;
+        J.rb = (int16_t)(jj - i * B);
         J.seg0 = S.act_off[i];
         J.n = (int16_t)S.act_n[i];
         J.e = S.act_e[i];
     }
-    J.part = (int16_t)part;
-    J.g0 = (int16_t)(GH * part / P.nkp);
-    J.g1 = (int16_t)(GH * (part + 1) / P.nkp);
+    J.part = 0;
+    J.g0 = 0;
+    J.g1 = (int16_t)(P.H / 64);
     return J;
 }
 
 // Job j of the down phase.
-__device__ JobDesc make_dn_job(const Params &P, const Smem &S, int j) {
+__device__ __noinline__ JobDesc make_dn_job(const Params &P, const Smem &S, int j) {
     JobDesc J;
     const int RBH = P.H / 32;
     const int A = P.ndp_s * RBH;
@@ -375,7 +369,7 @@ __device__ __forceinline__ void issue_stage(Smem &S, int s, const uint32_t *cons
     }
 }
 
-__device__ __forceinline__ void prefetch_dn_jobs(const Params &P, const Smem &S, const moe_layer_w &W) {
+__device__ __noinline__ void prefetch_dn_jobs(const Params &P, const Smem &S, const moe_layer_w &W) {
     for (int d = 0; d < S.ndn; ++d) {
         const JobDesc D = S.dnjob[d];
         const uint32_t *dq, *dsb;
@@ -432,29 +426,29 @@ __device__ __forceinline__ void group_dot(const uint32_t (&w)[8], float s, float
     }
 }
 
-// One (matrix, group) for the n <= 8 tokens of a job, in calls of at most two
-// tokens (codes are decoded once per call); acc[0] holds tokens 0-3, acc[1] 4-7.
+// One (matrix, group) for the n <= NT tokens of a job, in calls of at most two
+// tokens (codes are decoded once per call); acc[tt] is token tt's sum.
+template <int NT>
 __device__ __forceinline__ void group_dot_n(const unsigned char *codes, uint32_t sbw, const float *x,
                                             const float *xsum, const int *tokrow, int stride, int n,
-                                            float (&acc)[2][4], int lane) {
+                                            float (&acc)[NT], int lane) {
     const uint4 c0 = reinterpret_cast<const uint4 *>(codes)[lane];
     const uint4 c1 = reinterpret_cast<const uint4 *>(codes + 512)[lane];
     const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
     const float s = bf16_bits_to_float(sbw & 0xffffu) * kCodeUnscale, b = bf16_bits_to_float(sbw >> 16);
-    if (n == 1) {
-        group_dot<1>(w, s, b, x, xsum, tokrow, stride, 0, 1, acc[0]);
+    if (NT == 1) {
+        float a4[4] = {acc[0], 0.f, 0.f, 0.f};
+        group_dot<1>(w, s, b, x, xsum, tokrow, stride, 0, 1, a4);
+        acc[0] = a4[0];
         return;
     }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (4 * h < n) {
-            float p0[4] = {acc[h][0], acc[h][1], 0.f, 0.f}, p1[4] = {acc[h][2], acc[h][3], 0.f, 0.f};
-            group_dot<2>(w, s, b, x, xsum, tokrow, stride, 4 * h, min(2, n - 4 * h), p0);
-            if (4 * h + 2 < n) group_dot<2>(w, s, b, x, xsum, tokrow, stride, 4 * h + 2, min(2, n - 4 * h - 2), p1);
-            acc[h][0] = p0[0];
-            acc[h][1] = p0[1];
-            acc[h][2] = p1[0];
-            acc[h][3] = p1[1];
+    for (int t0 = 0; t0 < NT; t0 += 2) {
+        if (t0 < n) {
+            float p[4] = {acc[t0], t0 + 1 < NT ? acc[t0 + 1 < NT ? t0 + 1 : 0] : 0.f, 0.f, 0.f};
+            group_dot<2>(w, s, b, x, xsum, tokrow, stride, t0, min(2, n - t0), p);
+            acc[t0] = p[0];
+            if (t0 + 1 < NT) acc[t0 + 1 < NT ? t0 + 1 : 0] = p[1];
         }
     }
 }
@@ -465,8 +459,10 @@ __device__ __forceinline__ void group_dot_n(const unsigned char *codes, uint32_t
 __device__ __noinline__ void load_input(const Params &P, Smem &S, const uint16_t *h) {
     const int T = P.T, H = P.H, H2 = H / 2;
     float *stage = S.stage;
+#pragma unroll 1
     for (int t = 0; t < T; ++t) {
         float ss = 0.f;
+#pragma unroll 1
         for (int i = threadIdx.x; i < H2; i += blockDim.x) {
             const uint32_t v = __ldcg(reinterpret_cast<const unsigned int *>(h + (size_t)t * H) + i);
             const float a = bf16_bits_to_float(v & 0xffffu), b = bf16_bits_to_float(v >> 16);
@@ -493,6 +489,7 @@ __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
     uint16_t *out = P.h_out + (size_t)lp * T * H;
     float *stage = S.stage;
     const float scalar = P.layer_scalar;
+#pragma unroll 1
     for (int t = 0; t < T; ++t) {
         float4 mreg[2];
         uint2 hreg[2];
@@ -544,7 +541,7 @@ __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
 // Producer, at the start of layer l: router_scale, this CTA's router rows
 // [e0, e1) and a 16-byte-aligned superset of their scales and biases, into
 // the ring (idle until the top-k), completing on S.rbar (one phase per layer).
-__device__ void issue_router_copies(const Params &P, Smem &S, const moe_layer_w &W) {
+__device__ __noinline__ void issue_router_copies(const Params &P, Smem &S, const moe_layer_w &W) {
     const int E = P.E, H = P.H, G = H / 64;
     const int e0 = (int)((long long)E * blockIdx.x / gridDim.x), e1 = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);
     const int nrows = e1 - e0;
@@ -593,12 +590,14 @@ __device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
         const int units = items * parts;
         const int nch = H / 16;
         const float *stage = S.stage;
+#pragma unroll 1
         for (int u = wid; u < units; u += kWarps) {
             const int item = u / parts, part = u - item * parts;
             const int er = item / T, t = item - er * T;
             const int c0 = nch * part / parts, c1 = nch * (part + 1) / parts;
             const float *h = stage + (size_t)t * H;
             double acc = 0.0;
+#pragma unroll 1
             for (int c = c0 + lane; c < c1; c += 32) {
                 const uint4 q = reinterpret_cast<const uint4 *>(rows + (size_t)er * H)[c];
                 const uint32_t words[4] = {q.x, q.y, q.z, q.w};
@@ -627,6 +626,7 @@ __device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
         }
         __syncthreads();
         const double sqrt_h = sqrt((double)H);
+#pragma unroll 1
         for (int item = threadIdx.x; item < items; item += blockDim.x) {
             double a = 0.0;
             for (int p = 0; p < parts; ++p) a += S.rpart[item * parts + p];
@@ -644,14 +644,17 @@ __device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
 __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_layer_w &W) {
     const int T = P.T, E = P.E, k = P.k, n = T * k, H = P.H;
     double *lg = reinterpret_cast<double *>(S.pool);  // ring is idle here: T*E doubles
+#pragma unroll 1
     for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = __ldcg(P.logits + i);
     __syncthreads();
+#pragma unroll 1
     for (int t = 0; t < T; ++t) {
         const double2 *row = reinterpret_cast<const double2 *>(lg + (size_t)t * E);
+#pragma unroll 1
         for (int e = threadIdx.x; e < E; e += blockDim.x) {
             const double v = lg[(size_t)t * E + e];
             int rank = 0;
-#pragma unroll 8
+#pragma unroll 2
             for (int j = 0; j < E / 2; ++j) {  // E is a multiple of 8
                 const double2 o = row[j];
                 rank += (o.x > v) | ((o.x == v) & (2 * j < e));
@@ -672,11 +675,13 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     if (threadIdx.x < n) {
         const int p = threadIdx.x, t = p / k;
         double z = 0.0;
+#pragma unroll 1
         for (int s = 0; s < k; ++s) z += S.pe[t * k + s];
         const int e = S.idx[p];
         S.wts[p] = (float)(S.pe[p] / z * (double)bf16_bits_to_float(W.per_expert_scale[e]));
         // position of pair p among all pairs ordered by (expert, pair id)
         int less = 0, eqb = 0, cnt = 0;
+#pragma unroll 1
         for (int q = 0; q < n; ++q) {
             const int f = S.idx[q];
             less += f < e;
@@ -694,6 +699,7 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     if (threadIdx.x < n) {
         const int p = threadIdx.x, e = S.idx[p];
         int slot = 0, nact = 0;
+#pragma unroll 1
         for (int q = 0; q < n; ++q) {
             slot += S.first[q] & (S.idx[q] < e);
             nact += S.first[q];
@@ -710,12 +716,14 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     // expert jobs, already in L2, with routed ones from HBM); down jobs in
     // contiguous blocks, so that a CTA's jobs share a slot and stage its input once
     const int na = S.nact, G = gridDim.x, c = blockIdx.x;
-    const int J2 = (P.Is / 32 + na * (P.I / 32)) * P.nkp;
+    const int J2 = P.Is / 32 + na * (P.I / 32);
     const int J3 = (P.ndp_s + na * P.ndp_r) * (P.H / 32);
     const int n2 = J2 > c ? (J2 - 1 - c) / G + 1 : 0;
     const int d0 = (int)((long long)J3 * c / G), dstep = 1;
     const int n3 = (int)((long long)J3 * (c + 1) / G) - d0;
+#pragma unroll 1
     for (int i = threadIdx.x; i < n2 && i < kMaxJobs; i += blockDim.x) S.gujob[i] = make_gu_job(P, S, c + i * G);
+#pragma unroll 1
     for (int i = threadIdx.x; i < n3 && i < kMaxJobs; i += blockDim.x) S.dnjob[i] = make_dn_job(P, S, d0 + i * dstep);
     if (threadIdx.x == 0) {
         S.ngu = n2 < kMaxJobs ? n2 : kMaxJobs;
@@ -724,6 +732,7 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     __syncthreads();
     if (threadIdx.x == 0) {
         int st = 0;
+#pragma unroll 1
         for (int i = 0; i < S.ngu; ++i) st += (S.gujob[i].g1 - S.gujob[i].g0 + kStageGroups - 1) / kStageGroups;
         S.gu_stages = st;
     }
@@ -739,6 +748,7 @@ __device__ __noinline__ void stage_x(const Params &P, Smem &S) {
     const int T = P.T, nch = P.H / 32, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     float *stage = S.stage;
     const float pre = code_prescale(lane & 7);
+#pragma unroll 1
     for (int i = wid; i < T * nch; i += kWarps) {
         const int t = i / nch;
         const float x = bf16_bits_to_float(f32_to_bf16_bits_alu(stage[(size_t)i * 32 + lane] * S.rinv[t]));
@@ -759,10 +769,12 @@ __device__ __noinline__ bool gu_producer(const Params &P, Smem &S, const moe_lay
     bool ok = true, prefetched = false;
     int nis = 0;
     const int ns = P.nslots, ngu = S.ngu;
+#pragma unroll 1
     for (int i = 0; i < ngu && ok; ++i) {
         const JobDesc J = S.gujob[i];
         const uint32_t *q[2], *sb[2];
         gu_ptrs(P, W, J, q, sb);
+#pragma unroll 1
         for (int g = J.g0; g < J.g1 && ok; g += kStageGroups) {
             if (ring.q >= (unsigned)ns && !mbar_wait(&S.empty[ring.s], ring.ph ^ 1u, P.err, kErrEmpty)) {
                 ok = false;
@@ -781,19 +793,23 @@ __device__ __noinline__ bool gu_producer(const Params &P, Smem &S, const moe_lay
     return ok;
 }
 
+template <int NT>
 __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, Ring ring) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
     bool ok = true;
     int buf = 0;
     const int m = wid >> 3, gi = wid & 7;  // warps 0-7: gate, 8-15: up; gi = group within a stage
-    const int ns = P.nslots, ngu = S.ngu, Kmax = P.Kmax, R = P.R;
-    const float *stage = S.stage;
+    const int ns = P.nslots, ngu = S.ngu;
+#pragma unroll 1
     for (int i = 0; i < ngu; ++i) {
         const JobDesc J = S.gujob[i];
         const int n = J.n;
         // the job's tokens: input rows gathered by token id
         const int *tokrow = J.slot == 0 ? S.tokrow_sh : S.tokrow + J.seg0;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float acc[NT];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
+#pragma unroll 1
         for (int g = J.g0; g < J.g1; g += kStageGroups) {
             const int ngs = min(kStageGroups, (int)J.g1 - g);
             const bool got = mbar_wait(&S.full[ring.s], ring.ph, P.err, kErrFull);
@@ -803,7 +819,7 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, Ring ring) {
                 const uint32_t sbw = reinterpret_cast<const uint32_t *>(
                     slot + 2 * ngs * kCodeBytesPerGroup + (m * ngs + gi) * kSbBytesPerGroup)[lane];
                 const int gcol = (g + gi) * 64;
-                group_dot_n(codes, sbw, stage + gcol, S.xs + gcol / 32, tokrow, 0, n, acc, lane);
+                group_dot_n<NT>(codes, sbw, S.stage + gcol, S.xs + gcol / 32, tokrow, 0, n, acc, lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.empty[ring.s]);
@@ -812,41 +828,20 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, Ring ring) {
         }
         float *Rb = S.red[buf];
 #pragma unroll
-        for (int tt = 0; tt < kMaxT; ++tt)
-            if (tt < n) Rb[(wid * kMaxT + tt) * 32 + lane] = acc[tt >> 2][tt & 3];
+        for (int tt = 0; tt < NT; ++tt)
+            if (tt < n) Rb[(wid * kMaxT + tt) * 32 + lane] = acc[tt];
         consumer_sync();
-        // reduce the 8 warps of each matrix -> this K part's partial sums
-        for (int r = ctid; r < 2 * n * 32; r += kCWarps * 32) {
-            const int mm = (r >> 5) >= n ? 1 : 0, tt = (r >> 5) - mm * n, ln = r & 31;
-            float v = 0.f;
+        // reduce the 8 warps of each matrix and form a = silu(g) * u for the job's rows
+#pragma unroll 1
+        for (int r = ctid; r < n * 32; r += kCWarps * 32) {
+            const int tt = r >> 5, ln = r & 31;
+            float gs = 0.f, us = 0.f;
 #pragma unroll
-            for (int w8 = 0; w8 < 8; ++w8) v += Rb[((mm * 8 + w8) * kMaxT + tt) * 32 + ln];
-            const int rs = job_rowset(P, J, tt);
-            P.gu_part[(((size_t)J.part * R + rs) * 2 + mm) * Kmax + J.rb * 32 + ln] = v;
-        }
-        // the last K part of (slot, row block) to finish forms a = silu(g) * u
-        // for its rows (partials ordered before the count by the fences)
-        __threadfence();
-        consumer_sync();
-        if (ctid == 0) {
-            const unsigned old = atomicAdd(&P.cnt_gu[J.slot * (Kmax / 32) + J.rb], 1u);
-            S.last = old == (unsigned)(P.nkp - 1);
-        }
-        consumer_sync();
-        if (S.last) {
-            __threadfence();
-            const size_t pstride = (size_t)R * 2 * Kmax;
-            for (int r = ctid; r < n * 32; r += kCWarps * 32) {
-                const int tt = r >> 5, ln = r & 31;
-                const size_t base = (size_t)job_rowset(P, J, tt) * 2 * Kmax + J.rb * 32 + ln;
-                float g = 0.f, u = 0.f;
-                for (int p = 0; p < P.nkp; ++p) {
-                    g += __ldcg(&P.gu_part[p * pstride + base]);
-                    u += __ldcg(&P.gu_part[p * pstride + base + Kmax]);
-                }
-                P.act[(size_t)job_rowset(P, J, tt) * Kmax + J.rb * 32 + ln] = silu_mul(g, u);
+            for (int w8 = 0; w8 < 8; ++w8) {
+                gs += Rb[(w8 * kMaxT + tt) * 32 + ln];
+                us += Rb[((8 + w8) * kMaxT + tt) * 32 + ln];
             }
-            if (ctid == 0) P.cnt_gu[J.slot * (Kmax / 32) + J.rb] = 0u;
+            P.act[(size_t)job_rowset(P, J, tt) * P.Kmax + J.rb * 32 + ln] = silu_mul(gs, us);
         }
         buf ^= 1;  // the next job reduces in the other buffer
     }
@@ -859,6 +854,7 @@ __device__ __noinline__ bool dn_producer(const Params &P, Smem &S, const moe_lay
     bool ok = true;
     int nis = 0;
     const int ns = P.nslots, ndn = S.ndn;
+#pragma unroll 1
     for (int i = 0; i < ndn && ok; ++i) {
         if (ring.q >= (unsigned)ns && !mbar_wait(&S.empty[ring.s], ring.ph ^ 1u, P.err, kErrEmpty)) {
             ok = false;
@@ -876,6 +872,7 @@ __device__ __noinline__ bool dn_producer(const Params &P, Smem &S, const moe_lay
             const size_t shq = (size_t)P.Is * P.H / 2, shsb = (size_t)P.Is * (P.H / 64) * 4;
             const void *ptrs[6] = {N.sh_gate.q, N.sh_up.q, N.sh_down.q, N.sh_gate.sb, N.sh_up.sb, N.sh_down.sb};
             const size_t sizes[6] = {shq, shq, shq, shsb, shsb, shsb};
+#pragma unroll 1
             for (int a = 0; a < 6; ++a) {
                 const size_t per = ((sizes[a] / G) + 15) & ~(size_t)15;
                 const size_t off = per * blockIdx.x;
@@ -890,12 +887,13 @@ __device__ __noinline__ bool dn_producer(const Params &P, Smem &S, const moe_lay
 
 // Chunk sums (sum of the unscaled values) of nchunks 32-float chunks of the
 // stage, one consumer thread per chunk, bank-rotated.
-__device__ __forceinline__ void chunk_sums(Smem &S, int nchunks) {
+__device__ __noinline__ void chunk_sums(Smem &S, int nchunks) {
     const float *stage = S.stage;
+#pragma unroll 1
     for (int i = threadIdx.x; i < nchunks; i += kCWarps * 32) {
         const float *row = stage + (size_t)i * 32;
         float sx = 0.f;
-#pragma unroll 8
+#pragma unroll 4
         for (int mm = 0; mm < 32; ++mm) {
             const int m = (mm + i) & 31;
             sx = fmaf(row[m], code_unprescale(m & 7), sx);
@@ -904,6 +902,45 @@ __device__ __forceinline__ void chunk_sums(Smem &S, int nchunks) {
     }
 }
 
+__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned *p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// The combine m[t][rows of rb] = sum_s w[t,s] * y[t,s] + shared, in a fixed
+// order; the loads of a batch are issued before any is used.
+__device__ __noinline__ void combine_rows(const Params &P, const Smem &S, int rb, int t, int ln) {
+    const int T = P.T, k = P.k, H = P.H, row = rb * 32 + ln;
+    const size_t ystride = (size_t)T * k * H;
+    float mv = 0.f;
+    for (int s0 = 0; s0 < k; s0 += 8) {
+        float yv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) yv[u] = s0 + u < k ? __ldcg(&P.y[(size_t)(t * k + s0 + u) * H + row]) : 0.f;
+        for (int dp = 1; dp < P.ndp_r; ++dp) {
+            float yd[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                yd[u] = s0 + u < k ? __ldcg(&P.y[dp * ystride + (size_t)(t * k + s0 + u) * H + row]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) yv[u] += yd[u];
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (s0 + u < k) mv = fmaf(S.wts[t * k + s0 + u], yv[u], mv);
+    }
+    for (int d0 = 0; d0 < P.ndp_s; d0 += 4) {
+        float sv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) sv[u] = d0 + u < P.ndp_s ? __ldcg(&P.sh[((size_t)(d0 + u) * T + t) * H + row]) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mv += sv[u];
+    }
+    P.m[(size_t)t * H + row] = mv;
+}
+
+template <int NT>
 __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
     bool ok = true;
@@ -913,12 +950,18 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
     const unsigned dn_per_rb = (unsigned)(P.ndp_s + S.nact * P.ndp_r);
     float *stage = S.stage;
     int staged_slot = -1, staged_part = -1;
+    // thread 0 counts each finished job; the count returned for job i is examined one job later
+    unsigned pend_old = 0u;
+    int pend_rb = -1;
+    if (ctid == 0) S.nlast = 0;
+#pragma unroll 1
     for (int i = 0; i < ndn; ++i) {
         const JobDesc J = S.dnjob[i];
         const int ng = J.g1 - J.g0, n = J.n, ld = ng * 64;
         if (J.slot != staged_slot || J.part != staged_part) {
             // this slot's SwiGLU rows, columns [g0*64, g1*64): token tt at tt * ld
             const int q4 = ld / 4;
+#pragma unroll 1
             for (int e = ctid; e < n * q4; e += kCWarps * 32) {
                 const int tt = e / q4, c4 = e - tt * q4;
                 const float4 a = __ldcg(reinterpret_cast<const float4 *>(
@@ -945,21 +988,25 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
             const unsigned char *codes = slot + gi * kCodeBytesPerGroup;
             const uint32_t sbw =
                 reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane];
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            // token tt's row at tt * ld, its chunk sums at tt * ld / 32
-            group_dot_n(codes, sbw, stage + gi * 64, S.xs + 2 * gi, nullptr, ld, n, acc, lane);
+            float acc[NT];
 #pragma unroll
-            for (int tt = 0; tt < kMaxT; ++tt)
-                if (tt < n) Rb[(gi * kMaxT + tt) * 32 + lane] = acc[tt >> 2][tt & 3];
+            for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
+            // token tt's row at tt * ld, its chunk sums at tt * ld / 32
+            group_dot_n<NT>(codes, sbw, stage + gi * 64, S.xs + 2 * gi, nullptr, ld, n, acc, lane);
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt)
+                if (tt < n) Rb[(gi * kMaxT + tt) * 32 + lane] = acc[tt];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[ring.s]);
         if (!got) ok = false;
         ring_next(ring, ns);
         consumer_sync();
+#pragma unroll 1
         for (int r = ctid; r < n * 32; r += kCWarps * 32) {
             const int tt = r >> 5, ln = r & 31;
             float v = 0.f;
+#pragma unroll 4
             for (int g2 = 0; g2 < ng; ++g2) v += Rb[(g2 * kMaxT + tt) * 32 + ln];
             const int row = J.rb * 32 + ln;
             if (J.slot == 0)
@@ -967,31 +1014,32 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
             else
                 P.y[((size_t)J.part * T * k + S.perm[J.seg0 + tt]) * H + row] = v;
         }
-        // the last job of this row block to finish forms the combine for its rows
-        __threadfence();
+        // count this job for its row block (release: the y rows above, ordered
+        // by the barrier, become visible before the count); the previous
+        // job's count has long returned by now
         consumer_sync();
         if (ctid == 0) {
-            const unsigned old = atomicAdd(&P.cnt_dn[J.rb], 1u);
-            S.last = old == dn_per_rb - 1u;
-        }
-        consumer_sync();
-        if (S.last) {
-            __threadfence();
-            for (int r = ctid; r < T * 32; r += kCWarps * 32) {
-                const int t = r >> 5, row = J.rb * 32 + (r & 31);
-                float mv = 0.f;
-                for (int s2 = 0; s2 < k; ++s2) {
-                    float yv = 0.f;
-                    for (int dp = 0; dp < P.ndp_r; ++dp) yv += __ldcg(&P.y[((size_t)dp * T * k + t * k + s2) * H + row]);
-                    mv = fmaf(S.wts[t * k + s2], yv, mv);
-                }
-                for (int dp = 0; dp < P.ndp_s; ++dp) mv += __ldcg(&P.sh[((size_t)dp * T + t) * H + row]);
-                P.m[(size_t)t * H + row] = mv;
-            }
-            if (ctid == 0) P.cnt_dn[J.rb] = 0u;
+            if (pend_rb >= 0 && pend_old == dn_per_rb - 1u) S.last_rb[S.nlast++] = (int16_t)pend_rb;
+            pend_old = atom_add_release_gpu(&P.cnt_dn[J.rb], 1u);
+            pend_rb = J.rb;
         }
         buf ^= 1;
     }
+    if (ctid == 0) {
+        if (pend_rb >= 0 && pend_old == dn_per_rb - 1u) S.last_rb[S.nlast++] = (int16_t)pend_rb;
+        if (S.nlast > 0) __threadfence();  // acquire the other jobs' rows
+    }
+    consumer_sync();
+    // the combine of the row blocks this CTA finished last
+    const int nl = S.nlast;
+#pragma unroll 1
+    for (int r = ctid; r < nl * T * 32; r += kCWarps * 32) {
+        const int li = r / (T * 32), rem = r - li * T * 32;
+        const int rb = S.last_rb[li];
+        combine_rows(P, S, rb, rem >> 5, rem & 31);
+    }
+    consumer_sync();
+    if (ctid < nl) P.cnt_dn[S.last_rb[ctid]] = 0u;
     return ok;
 }
 
@@ -1044,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         if (producer)
             gu_producer(P, S, W, ring, issued);
         else if (consumer)
-            gu_consumer(P, S, ring);
+            P.T == 1 ? gu_consumer<1>(P, S, ring) : gu_consumer<kMaxT>(P, S, ring);
         for (int st = S.gu_stages; st > 0; --st) ring_next(ring, ns);
         ok = grid_sync(P, ++nbar, &S.flag);
         if (!ok) break;
@@ -1053,7 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         if (producer)
             dn_producer(P, S, W, ring, l, issued);
         else if (consumer)
-            dn_consumer(P, S, ring);
+            P.T == 1 ? dn_consumer<1>(P, S, ring) : dn_consumer<kMaxT>(P, S, ring);
         for (int st = S.ndn; st > 0; --st) ring_next(ring, ns);
         ok = grid_sync(P, ++nbar, &S.flag);
     }
@@ -1076,7 +1124,7 @@ static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exce
 static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
 
 struct DecodeWs {
-    size_t bar, cnt_gu, cnt_dn, logits, gu_part, act, y, sh, m, total, zero_bytes;
+    size_t bar, cnt_dn, logits, act, y, sh, m, total, zero_bytes;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1085,7 +1133,6 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
     DecodeWs d;
     const int Kmax = w->I > w->Is ? w->I : w->Is;
     const int R = T + T * w->k;
-    const int nkp = (w->H / 64 + dec::kGuPartGroups - 1) / dec::kGuPartGroups;
     const int ndp_r = (w->I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
     const int ndp_s = (w->Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
     size_t off = 0;
@@ -1095,11 +1142,9 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
         return o;
     };
     d.bar = take(256);
-    d.cnt_gu = take(sizeof(unsigned) * (size_t)R * (Kmax / 32));
     d.cnt_dn = take(sizeof(unsigned) * (size_t)(w->H / 32));
     d.zero_bytes = off;
     d.logits = take(sizeof(double) * (size_t)T * w->E);
-    d.gu_part = take(sizeof(float) * (size_t)nkp * R * 2 * Kmax);
     d.act = take(sizeof(float) * (size_t)R * Kmax);
     d.y = take(sizeof(float) * (size_t)ndp_r * T * w->k * w->H);
     d.sh = take(sizeof(float) * (size_t)ndp_s * T * w->H);
@@ -1159,7 +1204,6 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.Is = w.Is;
     P.Kmax = w.I > w.Is ? w.I : w.Is;
     P.R = T + T * w.k;
-    P.nkp = (w.H / 64 + dec::kGuPartGroups - 1) / dec::kGuPartGroups;
     P.ndp_r = (w.I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
     P.ndp_s = (w.Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
     if (!decode_layout(w, T, grid, &P.nslots)) return cudaErrorInvalidValue;
@@ -1167,9 +1211,7 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.bar = reinterpret_cast<unsigned *>(base + d.bar);
     P.err = reinterpret_cast<int *>(base + d.bar + sizeof(unsigned));
     P.logits = reinterpret_cast<double *>(base + d.logits);
-    P.cnt_gu = reinterpret_cast<unsigned *>(base + d.cnt_gu);
     P.cnt_dn = reinterpret_cast<unsigned *>(base + d.cnt_dn);
-    P.gu_part = reinterpret_cast<float *>(base + d.gu_part);
     P.act = reinterpret_cast<float *>(base + d.act);
     P.y = reinterpret_cast<float *>(base + d.y);
     P.sh = reinterpret_cast<float *>(base + d.sh);
