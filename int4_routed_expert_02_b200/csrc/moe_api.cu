@@ -451,8 +451,8 @@ int moe_decode_stack_status(const void *ws) {
     if (e != cudaSuccess) return cuda_fail(e, fn);
     if (code != 0) {
         static const char *what[] = {"", "grid barrier timed out", "wait for weights timed out",
-                                     "wait for a free ring slot timed out"};
-        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 4) ? what[code] : "?");
+                                     "wait for a free ring slot timed out", "wait for a job buffer timed out"};
+        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 5) ? what[code] : "?");
     }
     return MOE_OK;
 }

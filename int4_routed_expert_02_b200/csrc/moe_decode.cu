@@ -16,20 +16,26 @@
 //   P2  top-k + softmax * per_expert_scale and bucketing, by rank counting
 //       (every CTA, redundantly, so no barrier is needed before the experts),
 //       and this CTA's job tables for the two expert phases
-//   P2' gate/up dequant-GEMV jobs (32 rows of both matrices over the whole
-//       input, streamed in stages of <= 8 groups); each job forms
-//       a = silu(g) * u for its rows
+//   P2' gate/up: a job (32 rows: a row block of one slot) is split into
+//       tasks of <= 16 quantisation groups of one matrix; tasks are dealt
+//       round-robin to the CTAs and taken by their warps independently; each
+//       task's partial sums go to global memory, and the warp that finishes a
+//       job's last task (an atomic count per job) sums the parts in a fixed
+//       order and forms a = silu(g) * u for the job's rows
 //   --- grid barrier ---
-//   P3  down dequant-GEMV jobs (32 rows x <= 16 groups of one slot), in
-//       contiguous blocks per CTA so that a CTA stages each slot's a once;
-//       the last job of a row block to finish (an atomic count, read one
-//       job later) forms the combine m = sum_s w_s y_s + shared for those
-//       rows at the end of the phase
+//   P3  down: tasks of 32 rows x <= 16 groups of one slot, in contiguous
+//       blocks per CTA so that a CTA stages each slot's a once; a warp
+//       writes its task's rows, and the warp that finishes the last task of
+//       a row block (an atomic count per row block) forms the combine
+//       m = sum_s w_s y_s + shared for those rows
 //   --- grid barrier ---
 //
 // Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
-// into a ring of mbarrier-guarded slots, issued by one producer thread ahead
-// of 16 consumer warps.  Once the top-k is known each CTA also asks L2 to
+// into a ring of mbarrier-guarded slots, one slot per task, issued by one
+// producer thread ahead of 16 consumer warps that never wait for one another
+// inside a phase.  The down tasks' weights do not depend on the gate/up
+// results, so the producer already fills the slots freed during the gate/up
+// phase with them.  Once the top-k is known each CTA also asks L2 to
 // prefetch the down-projection weights of its later jobs, and during the down
 // phase its share of the next layer's shared-expert weights, so HBM keeps
 // streaming across the grid barriers.  The dot products use the subnormal
@@ -51,20 +57,20 @@ constexpr int kCWarps = 16;                   // consumer warps
 constexpr int kWarps = kCWarps + 1;           // + the producer warp
 constexpr int kThreads = kWarps * 32;
 constexpr int kProducerWarp = kCWarps;
-constexpr int kMaxStages = 9;                 // ring slots: as many as fit beside the input stage
-constexpr int kStageGroups = 8;               // gate/up stage: <= 8 groups of each of the two matrices
-constexpr int kDnGroups = 16;                 // down job: <= 16 groups, one stage
+constexpr int kMaxStages = 11;                // ring slots: as many as fit beside the input stage
+constexpr int kTaskGroups = 16;               // groups per task (one ring slot)
 constexpr int kCodeBytesPerGroup = 1024;      // 32 rows x 64 codes x 4 bits
 constexpr int kSbBytesPerGroup = 128;         // 32 rows x (scale, bias)
 constexpr int kSlotBytes = 16 * (kCodeBytesPerGroup + kSbBytesPerGroup);  // 18432
 constexpr int kMaxT = 8;
 constexpr int kStageFloats = 24576;           // largest input stage (T * H)
-constexpr int kPoolBytes = 4 * kSlotBytes + kStageFloats * 4;  // ring + input stage share this pool
+constexpr int kPoolBytes = 11 * kSlotBytes;   // ring + input stage share this pool
 constexpr int kMaxXs = 768;
 constexpr int kMaxLayers = 64;
 constexpr int kMaxPairs = kMaxT * kMaxK;
-constexpr int kMaxJobs = 128;                 // per CTA and phase
-constexpr int kRed = 16 * kMaxT * 32;         // one reduction buffer: [16 warps][kMaxT][32]
+constexpr int kMaxTasks = 160;                // per CTA and phase
+constexpr int kMaxPG = 4;                     // gate/up parts per job (H <= 4096)
+constexpr int kMaxSegs = 16;                  // down: staged (slot, part) inputs per CTA
 constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
 
 constexpr int kErrGridBarrier = 1, kErrFull = 2, kErrEmpty = 3;
@@ -78,9 +84,12 @@ struct Params {
     int H, E, k, I, Is, Kmax, R;
     int ndp_r, ndp_s;
     int nslots;      // ring slots (the rest of the pool is the input stage)
+    int stage_floats;  // floats in the input stage
     unsigned *bar;
     int *err;
-    unsigned *cnt_dn;  // [H/32]: down jobs done per row block; reset by the last
+    unsigned *cnt_dn;  // [H/32]: down tasks done per row block; reset by the last
+    unsigned *cnt_gu;  // [jobs]: gate/up tasks done per job; reset by the last
+    float *gpart;      // [jobs][2][pg][T][32]: gate/up partial sums per task
     double *logits;  // [T,E]
     float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs)
     float *y;        // [ndp_r][T*k][H]
@@ -88,12 +97,20 @@ struct Params {
     float *m;        // [T][H]: the combine m of the current layer
 };
 
-// One job of an expert phase: 32 rows (row block rb) x groups [g0, g1) of the
-// shared expert (slot 0) or of routed expert e (slot >= 1), for n tokens
-// starting at bucketed position seg0.
-struct JobDesc {
-    int16_t slot, rb, part, g0, g1, n;
-    int32_t seg0, e;
+// One task of an expert phase: 32 rows (row block rb) x groups [g0, g1) of
+// matrix mat (gate/up: 0 gate, 1 up; down: 0) of the shared expert (slot 0)
+// or of routed expert e (slot >= 1), for n tokens starting at bucketed
+// position seg0.  job: gate/up, the CTA-local job; seg: down, the staged input.
+struct TaskDesc {
+    int16_t slot, rb, mat, part, g0, g1, n, seg;
+    int32_t seg0, e, job;
+};
+
+// A staged down-phase input: the SwiGLU rows of one (slot, part), columns
+// [g0*64, g0*64 + ld), token tt at stage offset off + tt * ld.
+struct SegDesc {
+    int16_t slot, part, n, g0, ld, pad;
+    int32_t seg0, off;
 };
 
 struct Smem {
@@ -101,11 +118,13 @@ struct Smem {
     alignas(8) unsigned long long full[kMaxStages];
     alignas(8) unsigned long long empty[kMaxStages];
     alignas(8) unsigned long long rbar;  // router copies of the current layer
+    unsigned slot_task[kMaxStages];      // ring sequence number of the task a slot currently holds
     float *stage;                        // input stage (inside the pool, after the ring)
     alignas(16) float xs[kMaxXs];        // sum of x per 32-column chunk
-    alignas(16) float red[2][kRed];
-    JobDesc gujob[kMaxJobs], dnjob[kMaxJobs];
-    int ngu, ndn, gu_stages;
+    float bred[32];  // block reductions
+    TaskDesc gut[kMaxTasks], dnt[kMaxTasks];
+    SegDesc seg[kMaxSegs];
+    int ngt, ndt, pg, nseg, seg_rounds;
     double selv[kMaxPairs];
     double pe[kMaxPairs];
     float wts[kMaxPairs];
@@ -122,24 +141,7 @@ struct Smem {
     float rinv[kMaxT];
     int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
     int flag;
-    int nlast;                 // row blocks whose combine this CTA forms at the end of the down phase
-    int16_t last_rb[kMaxJobs];
 };
-
-// Position in the ring: stage sequence number q, its slot s and phase parity ph.
-struct Ring {
-    unsigned q;
-    int s;
-    unsigned ph;
-};
-
-__device__ __forceinline__ void ring_next(Ring &r, int ns) {
-    ++r.q;
-    if (++r.s == ns) {
-        r.s = 0;
-        r.ph ^= 1u;
-    }
-}
 
 // ------------------------------------------------------------------ PTX helpers
 
@@ -256,128 +258,111 @@ __device__ __noinline__ bool grid_sync(const Params &P, unsigned nth, int *verdi
 
 // ------------------------------------------------------------------ jobs
 
-// Job j of the gate/up phase: 32 rows of both matrices over the whole input
-// (all divisions happen here, once per job).
-__device__ __noinline__ JobDesc make_gu_job(const Params &P, const Smem &S, int j) {
-    JobDesc J;
+// Task gt (grid-wide index; this CTA takes gt = c, c + G, ...) of the gate/up
+// phase.  Job j = gt / (2 pg) is 32 rows of the shared expert or of one
+// active slot; its 2 pg tasks are part p of gate and of up, p = 0..pg-1.
+// All divisions happen here, once per task.
+__device__ __noinline__ TaskDesc make_gu_task(const Params &P, const Smem &S, int gt) {
+    TaskDesc t;
+    const int pg = S.pg, j = gt / (2 * pg), r = gt - j * 2 * pg;
     const int A = P.Is / 32;
     if (j < A) {
-        J.slot = 0;
-        J.rb = (int16_t)j;
-        J.n = (int16_t)P.T;
-        J.seg0 = 0;
-        J.e = -1;
+        t.slot = 0;
+        t.rb = (int16_t)j;
+        t.n = (int16_t)P.T;
+        t.seg0 = 0;
+        t.e = -1;
     } else {
-        const int B = P.I / 32;
-        const int jj = j - A;
-        const int i = jj / B;
-        J.slot = (int16_t)(1 + i);
-        J.rb = (int16_t)(jj - i * B);
-        J.seg0 = S.act_off[i];
-        J.n = (int16_t)S.act_n[i];
-        J.e = S.act_e[i];
+        const int B = P.I / 32, jj = j - A, a = jj / B;
+        t.slot = (int16_t)(1 + a);
+        t.rb = (int16_t)(jj - a * B);
+        t.seg0 = S.act_off[a];
+        t.n = (int16_t)S.act_n[a];
+        t.e = S.act_e[a];
     }
-    J.part = 0;
-    J.g0 = 0;
-    J.g1 = (int16_t)(P.H / 64);
-    return J;
+    const int GH = P.H / 64;
+    t.mat = (int16_t)(r & 1);
+    t.part = (int16_t)(r >> 1);
+    t.g0 = (int16_t)(GH * t.part / pg);
+    t.g1 = (int16_t)(GH * (t.part + 1) / pg);
+    t.job = j;
+    t.seg = 0;
+    return t;
 }
 
-// Job j of the down phase.
-__device__ __noinline__ JobDesc make_dn_job(const Params &P, const Smem &S, int j) {
-    JobDesc J;
-    const int RBH = P.H / 32;
-    const int A = P.ndp_s * RBH;
-    if (j < A) {
-        const int part = j / RBH;
-        J.slot = 0;
-        J.part = (int16_t)part;
-        J.rb = (int16_t)(j - part * RBH);
-        J.n = (int16_t)P.T;
-        J.seg0 = 0;
-        J.e = -1;
-        const int G = P.Is / 64;
-        J.g0 = (int16_t)(G * part / P.ndp_s);
-        J.g1 = (int16_t)(G * (part + 1) / P.ndp_s);
+// (slot, part) number sp of the down phase: the shared expert's parts first,
+// then each active slot's.
+__device__ __forceinline__ void dn_slot_part(const Params &P, int sp, int &slot, int &part) {
+    if (sp < P.ndp_s) {
+        slot = 0;
+        part = sp;
     } else {
-        const int B = P.ndp_r * RBH;
-        const int jj = j - A;
-        const int i = jj / B;
-        const int r = jj - i * B;
-        const int part = r / RBH;
-        J.slot = (int16_t)(1 + i);
-        J.part = (int16_t)part;
-        J.rb = (int16_t)(r - part * RBH);
-        J.seg0 = S.act_off[i];
-        J.n = (int16_t)S.act_n[i];
-        J.e = S.act_e[i];
-        const int G = P.I / 64;
-        J.g0 = (int16_t)(G * part / P.ndp_r);
-        J.g1 = (int16_t)(G * (part + 1) / P.ndp_r);
-    }
-    return J;
-}
-
-// Weight pointers of a gate/up job (matrix 0 = gate, 1 = up).
-__device__ __forceinline__ void gu_ptrs(const Params &P, const moe_layer_w &W, const JobDesc &J, const uint32_t *(&q)[2],
-                                        const uint32_t *(&sb)[2]) {
-    const size_t CH = P.H / 32, GH = P.H / 64;
-    if (J.slot == 0) {
-        q[0] = W.sh_gate.q + (size_t)J.rb * CH * 128;
-        q[1] = W.sh_up.q + (size_t)J.rb * CH * 128;
-        sb[0] = W.sh_gate.sb + (size_t)J.rb * GH * 32;
-        sb[1] = W.sh_up.sb + (size_t)J.rb * GH * 32;
-    } else {
-        const size_t mrb = (size_t)J.e * (P.I / 32) + J.rb;
-        q[0] = W.gate.q + mrb * CH * 128;
-        q[1] = W.up.q + mrb * CH * 128;
-        sb[0] = W.gate.sb + mrb * GH * 32;
-        sb[1] = W.up.sb + mrb * GH * 32;
+        const int a = (sp - P.ndp_s) / P.ndp_r;
+        slot = 1 + a;
+        part = sp - P.ndp_s - a * P.ndp_r;
     }
 }
 
-// Weight pointers of a down job.
-__device__ __forceinline__ void dn_ptrs(const Params &P, const moe_layer_w &W, const JobDesc &J, const uint32_t *&q,
-                                        const uint32_t *&sb) {
-    if (J.slot == 0) {
-        q = W.sh_down.q + (size_t)J.rb * (P.Is / 32) * 128;
-        sb = W.sh_down.sb + (size_t)J.rb * (P.Is / 64) * 32;
+// Task d (grid-wide index) of the down phase: (slot, part) d / (H/32), row block d % (H/32).
+__device__ __noinline__ TaskDesc make_dn_task(const Params &P, const Smem &S, int d, int sp0) {
+    TaskDesc t;
+    const int RBH = P.H / 32, sp = d / RBH;
+    int slot, part;
+    dn_slot_part(P, sp, slot, part);
+    t.slot = (int16_t)slot;
+    t.part = (int16_t)part;
+    t.rb = (int16_t)(d - sp * RBH);
+    t.mat = 0;
+    const int G = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
+    t.g0 = (int16_t)(G * part / nd);
+    t.g1 = (int16_t)(G * (part + 1) / nd);
+    if (slot == 0) {
+        t.n = (int16_t)P.T;
+        t.seg0 = 0;
+        t.e = -1;
     } else {
-        const size_t mrb = (size_t)J.e * (P.H / 32) + J.rb;
+        t.seg0 = S.act_off[slot - 1];
+        t.n = (int16_t)S.act_n[slot - 1];
+        t.e = S.act_e[slot - 1];
+    }
+    t.job = 0;
+    t.seg = (int16_t)(sp - sp0);
+    return t;
+}
+
+// Weight pointers (codes, scale/bias words) of a task's row block.
+__device__ __forceinline__ void task_ptrs(const Params &P, const moe_layer_w &W, const TaskDesc &t, bool down,
+                                          const uint32_t *&q, const uint32_t *&sb) {
+    if (!down) {
+        const size_t CH = P.H / 32, GH = P.H / 64;
+        const moe_qmat &M = t.slot == 0 ? (t.mat ? W.sh_up : W.sh_gate) : (t.mat ? W.up : W.gate);
+        const size_t mrb = t.slot == 0 ? (size_t)t.rb : (size_t)t.e * (P.I / 32) + t.rb;
+        q = M.q + mrb * CH * 128;
+        sb = M.sb + mrb * GH * 32;
+    } else if (t.slot == 0) {
+        q = W.sh_down.q + (size_t)t.rb * (P.Is / 32) * 128;
+        sb = W.sh_down.sb + (size_t)t.rb * (P.Is / 64) * 32;
+    } else {
+        const size_t mrb = (size_t)t.e * (P.H / 32) + t.rb;
         q = W.down.q + mrb * (P.I / 32) * 128;
         sb = W.down.sb + mrb * (P.I / 64) * 32;
     }
 }
 
-// rowset of the tt-th token of a job (shared: the token; routed: T + bucketed position)
-__device__ __forceinline__ int job_rowset(const Params &P, const JobDesc &J, int tt) {
-    return J.slot == 0 ? tt : P.T + J.seg0 + tt;
+// rowset of the tt-th token of a task (shared: the token; routed: T + bucketed position)
+__device__ __forceinline__ int task_rowset(const Params &P, const TaskDesc &t, int tt) {
+    return t.slot == 0 ? tt : P.T + t.seg0 + tt;
 }
 
-// Producer: the copies that fill ring slot s with groups [g0, g1) of nmat matrices.
-// Layout in the slot: codes of matrix 0 (ng KiB), codes of matrix 1, then the
-// (scale, bias) words of matrix 0 (ng * 128 B), of matrix 1.
-__device__ __forceinline__ void issue_stage(Smem &S, int s, const uint32_t *const *q, const uint32_t *const *sb,
-                                            int nmat, int g0, int g1) {
+// Producer: the copies that fill ring slot s with groups [g0, g1) of one
+// matrix: codes (ng KiB), then the (scale, bias) words (ng * 128 B).
+__device__ __forceinline__ void issue_task(Smem &S, int s, const uint32_t *q, const uint32_t *sb, int g0, int g1) {
     const int ng = g1 - g0;
     const unsigned cb = (unsigned)ng * kCodeBytesPerGroup, sbb = (unsigned)ng * kSbBytesPerGroup;
     unsigned char *slot = S.pool + (size_t)s * kSlotBytes;
-    mbar_expect_tx(&S.full[s], nmat * (cb + sbb));
-    for (int m = 0; m < nmat; ++m) {
-        bulk_g2s(slot + m * cb, q[m] + (size_t)g0 * 256, cb, &S.full[s]);
-        bulk_g2s(slot + nmat * cb + m * sbb, sb[m] + (size_t)g0 * 32, sbb, &S.full[s]);
-    }
-}
-
-__device__ __noinline__ void prefetch_dn_jobs(const Params &P, const Smem &S, const moe_layer_w &W) {
-    for (int d = 0; d < S.ndn; ++d) {
-        const JobDesc D = S.dnjob[d];
-        const uint32_t *dq, *dsb;
-        dn_ptrs(P, W, D, dq, dsb);
-        const int ng = D.g1 - D.g0;
-        prefetch_l2(dq + (size_t)D.g0 * 256, (unsigned)ng * kCodeBytesPerGroup);
-        prefetch_l2(dsb + (size_t)D.g0 * 32, (unsigned)ng * kSbBytesPerGroup);
-    }
+    mbar_expect_tx(&S.full[s], cb + sbb);
+    bulk_g2s(slot, q + (size_t)g0 * 256, cb, &S.full[s]);
+    bulk_g2s(slot + cb, sb + (size_t)g0 * 32, sbb, &S.full[s]);
 }
 
 // ------------------------------------------------------------------ dot products
@@ -470,7 +455,7 @@ __device__ __noinline__ void load_input(const Params &P, Smem &S, const uint16_t
             stage[(size_t)t * H + 2 * i + 1] = b;
             ss = fmaf(a, a, fmaf(b, b, ss));
         }
-        ss = block_sum(ss, S.red[0]);
+        ss = block_sum(ss, S.bred);
         if (threadIdx.x == 0) {
             S.rms[t] = sqrtf(ss / (float)H + P.eps);
             S.rinv[t] = 1.0f / S.rms[t];
@@ -507,7 +492,7 @@ __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
 #pragma unroll
         for (int r = 0; r < 2; ++r)
             ss += mreg[r].x * mreg[r].x + mreg[r].y * mreg[r].y + mreg[r].z * mreg[r].z + mreg[r].w * mreg[r].w;
-        ss = block_sum(ss, S.red[0]);
+        ss = block_sum(ss, S.bred);
         const float inv = P.post_norm ? 1.0f / sqrtf(ss / (float)H + P.eps) : 1.0f;
         float ss2 = 0.f;
 #pragma unroll
@@ -529,7 +514,7 @@ __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
                     reinterpret_cast<uint2 *>(out + (size_t)t * H)[i4] = make_uint2(o[0] | (o[1] << 16), o[2] | (o[3] << 16));
             }
         }
-        ss2 = block_sum(ss2, S.red[0]);
+        ss2 = block_sum(ss2, S.bred);
         if (threadIdx.x == 0) {
             S.rms[t] = sqrtf(ss2 / (float)H + P.eps);
             S.rinv[t] = 1.0f / S.rms[t];
@@ -712,30 +697,51 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
         if (p == 0) S.nact = nact;
     }
     __syncthreads();
-    // job tables of this CTA: gate/up jobs round-robin (every CTA mixes shared-
-    // expert jobs, already in L2, with routed ones from HBM); down jobs in
-    // contiguous blocks, so that a CTA's jobs share a slot and stage its input once
+    // task tables of this CTA.  Gate/up jobs are dealt round-robin (every CTA
+    // mixes shared-expert jobs with routed ones); down tasks go in contiguous
+    // blocks, so that a CTA's tasks share few (slot, part) inputs.
     const int na = S.nact, G = gridDim.x, c = blockIdx.x;
-    const int J2 = P.Is / 32 + na * (P.I / 32);
-    const int J3 = (P.ndp_s + na * P.ndp_r) * (P.H / 32);
-    const int n2 = J2 > c ? (J2 - 1 - c) / G + 1 : 0;
-    const int d0 = (int)((long long)J3 * c / G), dstep = 1;
-    const int n3 = (int)((long long)J3 * (c + 1) / G) - d0;
-#pragma unroll 1
-    for (int i = threadIdx.x; i < n2 && i < kMaxJobs; i += blockDim.x) S.gujob[i] = make_gu_job(P, S, c + i * G);
-#pragma unroll 1
-    for (int i = threadIdx.x; i < n3 && i < kMaxJobs; i += blockDim.x) S.dnjob[i] = make_dn_job(P, S, d0 + i * dstep);
+    const int pg = (P.H / 64 + kTaskGroups - 1) / kTaskGroups;
+    const int NT2 = (P.Is / 32 + na * (P.I / 32)) * 2 * pg;  // gate/up tasks of the grid
+    const int n2 = NT2 > c ? (NT2 - 1 - c) / G + 1 : 0;
+    const int RBH = P.H / 32;
+    const int J3 = (P.ndp_s + na * P.ndp_r) * RBH;
+    const int d0 = (int)((long long)J3 * c / G), d1 = (int)((long long)J3 * (c + 1) / G);
+    const int sp0 = d0 / RBH;
     if (threadIdx.x == 0) {
-        S.ngu = n2 < kMaxJobs ? n2 : kMaxJobs;
-        S.ndn = n3 < kMaxJobs ? n3 : kMaxJobs;
+        S.pg = pg;
+        S.ngt = min(n2, kMaxTasks);
+        S.ndt = min(d1 - d0, kMaxTasks);
+        // staged down inputs: the (slot, part) of the CTA's tasks, consecutive
+        int nseg = d1 > d0 ? (d1 - 1) / RBH - sp0 + 1 : 0, off = 0;
+        nseg = min(nseg, kMaxSegs);
+        for (int k2 = 0; k2 < nseg; ++k2) {
+            int slot, part;
+            dn_slot_part(P, sp0 + k2, slot, part);
+            const int Gs = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
+            SegDesc &sg = S.seg[k2];
+            sg.slot = (int16_t)slot;
+            sg.part = (int16_t)part;
+            sg.g0 = (int16_t)(Gs * part / nd);
+            sg.ld = (int16_t)((Gs * (part + 1) / nd - sg.g0) * 64);
+            sg.n = (int16_t)(slot == 0 ? P.T : S.act_n[slot - 1]);
+            sg.seg0 = slot == 0 ? 0 : S.act_off[slot - 1];
+            sg.off = off;
+            sg.pad = 0;
+            off += sg.n * sg.ld;
+        }
+        S.nseg = nseg;
+        // all inputs at once if they fit the stage (and its chunk sums), else one
+        // (slot, part) at a time, each from the start of the stage
+        S.seg_rounds = off <= min(P.stage_floats, kMaxXs * 32) ? 1 : nseg;
+        if (S.seg_rounds > 1)
+            for (int k2 = 0; k2 < nseg; ++k2) S.seg[k2].off = 0;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int st = 0;
 #pragma unroll 1
-        for (int i = 0; i < S.ngu; ++i) st += (S.gujob[i].g1 - S.gujob[i].g0 + kStageGroups - 1) / kStageGroups;
-        S.gu_stages = st;
-    }
+    for (int i = threadIdx.x; i < S.ngt; i += blockDim.x) S.gut[i] = make_gu_task(P, S, c + i * G);
+#pragma unroll 1
+    for (int i = threadIdx.x; i < S.ndt; i += blockDim.x) S.dnt[i] = make_dn_task(P, S, d0 + i, sp0);
     // the ring was written with generic stores above; order them before the
     // bulk copies (async proxy) that refill it next
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -762,135 +768,186 @@ __device__ __noinline__ void stage_x(const Params &P, Smem &S) {
 // ------------------------------------------------------------------ streaming loops
 // (each its own function, so that its register allocation is its own)
 
-// Producer of the gate/up phase: bulk copies of the stages of its jobs, and,
-// once the ring is primed, an L2 prefetch of its down-phase jobs.
-__device__ __noinline__ bool gu_producer(const Params &P, Smem &S, const moe_layer_w &W, Ring ring,
-                                         unsigned &issued) {
-    bool ok = true, prefetched = false;
-    int nis = 0;
-    const int ns = P.nslots, ngu = S.ngu;
-#pragma unroll 1
-    for (int i = 0; i < ngu && ok; ++i) {
-        const JobDesc J = S.gujob[i];
-        const uint32_t *q[2], *sb[2];
-        gu_ptrs(P, W, J, q, sb);
-#pragma unroll 1
-        for (int g = J.g0; g < J.g1 && ok; g += kStageGroups) {
-            if (ring.q >= (unsigned)ns && !mbar_wait(&S.empty[ring.s], ring.ph ^ 1u, P.err, kErrEmpty)) {
-                ok = false;
-                break;
-            }
-            issue_stage(S, ring.s, q, sb, 2, g, min(g + kStageGroups, (int)J.g1));
-            issued = ring.q + 1;
-            ring_next(ring, ns);
-            if (++nis == ns && !prefetched) {
-                prefetched = true;
-                prefetch_dn_jobs(P, S, W);
-            }
-        }
-    }
-    if (ok && !prefetched) prefetch_dn_jobs(P, S, W);
-    return ok;
+// Ring position of task i of a phase that starts at ring sequence number rq.
+__device__ __forceinline__ void ring_pos(unsigned rq, int i, int ns, int &s, unsigned &ph) {
+    const unsigned q = rq + (unsigned)i;
+    s = (int)(q % (unsigned)ns);
+    ph = (q / (unsigned)ns) & 1u;
 }
 
-template <int NT>
-__device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, Ring ring) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
+// Producer of an expert phase: one ring slot per task, in task order.  The
+// ring runs through the gate/up tasks [0, ngt) and on into the down tasks
+// [ngt, ngt + ndt) (sequence numbers from the gate/up phase's rq).  In the
+// gate/up phase it issues every gate/up task and then the down tasks whose
+// slot was last used by a gate/up task (those slots are freed within the
+// phase); the down phase issues the rest.  Once the ring is primed, an L2
+// prefetch of what comes next (gate/up: the down tasks that do not fit the
+// ring; down: this CTA's share of the next layer's shared expert).
+__device__ __noinline__ bool task_producer(const Params &P, Smem &S, const moe_layer_w &W, bool down, unsigned rq,
+                                           int l, unsigned &issued) {
+    const int ns = P.nslots, ngt = S.ngt, ndt = S.ndt;
+    // ring positions [i0, i1) relative to the gate/up phase's first task
+    const int pre = min(ndt, ns);  // down tasks issued during the gate/up phase
+    const int i0 = down ? ngt + pre : 0, i1 = down ? ngt + ndt : ngt + pre;
+    const unsigned rq0 = down ? rq - (unsigned)ngt : rq;
     bool ok = true;
-    int buf = 0;
-    const int m = wid >> 3, gi = wid & 7;  // warps 0-7: gate, 8-15: up; gi = group within a stage
-    const int ns = P.nslots, ngu = S.ngu;
 #pragma unroll 1
-    for (int i = 0; i < ngu; ++i) {
-        const JobDesc J = S.gujob[i];
-        const int n = J.n;
-        // the job's tokens: input rows gathered by token id
-        const int *tokrow = J.slot == 0 ? S.tokrow_sh : S.tokrow + J.seg0;
-        float acc[NT];
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
-#pragma unroll 1
-        for (int g = J.g0; g < J.g1; g += kStageGroups) {
-            const int ngs = min(kStageGroups, (int)J.g1 - g);
-            const bool got = mbar_wait(&S.full[ring.s], ring.ph, P.err, kErrFull);
-            if (got && gi < ngs) {
-                const unsigned char *slot = S.pool + (size_t)ring.s * kSlotBytes;
-                const unsigned char *codes = slot + (m * ngs + gi) * kCodeBytesPerGroup;
-                const uint32_t sbw = reinterpret_cast<const uint32_t *>(
-                    slot + 2 * ngs * kCodeBytesPerGroup + (m * ngs + gi) * kSbBytesPerGroup)[lane];
-                const int gcol = (g + gi) * 64;
-                group_dot_n<NT>(codes, sbw, S.stage + gcol, S.xs + gcol / 32, tokrow, 0, n, acc, lane);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.empty[ring.s]);
-            if (!got) ok = false;
-            ring_next(ring, ns);
-        }
-        float *Rb = S.red[buf];
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt)
-            if (tt < n) Rb[(wid * kMaxT + tt) * 32 + lane] = acc[tt];
-        consumer_sync();
-        // reduce the 8 warps of each matrix and form a = silu(g) * u for the job's rows
-#pragma unroll 1
-        for (int r = ctid; r < n * 32; r += kCWarps * 32) {
-            const int tt = r >> 5, ln = r & 31;
-            float gs = 0.f, us = 0.f;
-#pragma unroll
-            for (int w8 = 0; w8 < 8; ++w8) {
-                gs += Rb[(w8 * kMaxT + tt) * 32 + ln];
-                us += Rb[((8 + w8) * kMaxT + tt) * 32 + ln];
-            }
-            P.act[(size_t)job_rowset(P, J, tt) * P.Kmax + J.rb * 32 + ln] = silu_mul(gs, us);
-        }
-        buf ^= 1;  // the next job reduces in the other buffer
-    }
-    return ok;
-}
-
-__device__ __noinline__ bool dn_producer(const Params &P, Smem &S, const moe_layer_w &W, Ring ring, int l,
-                                         unsigned &issued) {
-    const int G = gridDim.x;
-    bool ok = true;
-    int nis = 0;
-    const int ns = P.nslots, ndn = S.ndn;
-#pragma unroll 1
-    for (int i = 0; i < ndn && ok; ++i) {
-        if (ring.q >= (unsigned)ns && !mbar_wait(&S.empty[ring.s], ring.ph ^ 1u, P.err, kErrEmpty)) {
+    for (int i = i0; i < i1; ++i) {
+        int s;
+        unsigned ph;
+        ring_pos(rq0, i, ns, s, ph);
+        if (rq0 + (unsigned)i >= (unsigned)ns && !mbar_wait(&S.empty[s], ph ^ 1u, P.err, kErrEmpty)) {
             ok = false;
             break;
         }
-        const JobDesc J = S.dnjob[i];
-        const uint32_t *q[1], *sb[1];
-        dn_ptrs(P, W, J, q[0], sb[0]);
-        issue_stage(S, ring.s, q, sb, 1, J.g0, J.g1);
-        issued = ring.q + 1;
-        ring_next(ring, ns);
-        if (++nis == ns && l + 1 < P.L) {
-            // this CTA's share of the next layer's shared-expert weights
-            const moe_layer_w &N = P.layers[l + 1];
-            const size_t shq = (size_t)P.Is * P.H / 2, shsb = (size_t)P.Is * (P.H / 64) * 4;
-            const void *ptrs[6] = {N.sh_gate.q, N.sh_up.q, N.sh_down.q, N.sh_gate.sb, N.sh_up.sb, N.sh_down.sb};
-            const size_t sizes[6] = {shq, shq, shq, shsb, shsb, shsb};
+        const bool dn = i >= ngt;
+        const TaskDesc t = dn ? S.dnt[i - ngt] : S.gut[i];
+        const uint32_t *q, *sb;
+        task_ptrs(P, W, t, dn, q, sb);
+        // the slot now belongs to this task (its previous task has been consumed)
+        *reinterpret_cast<volatile unsigned *>(&S.slot_task[s]) = rq0 + (unsigned)i;
+        issue_task(S, s, q, sb, t.g0, t.g1);
+        issued = rq0 + (unsigned)i + 1u;
+        if (!down && i == min(ns, ngt) - 1) {
+            // the down tasks beyond the ring: into L2 for now
 #pragma unroll 1
-            for (int a = 0; a < 6; ++a) {
-                const size_t per = ((sizes[a] / G) + 15) & ~(size_t)15;
-                const size_t off = per * blockIdx.x;
-                if (off < sizes[a])
-                    prefetch_range(static_cast<const char *>(ptrs[a]) + off,
-                                   (off + per <= sizes[a] ? per : sizes[a] - off) & ~(size_t)15);
+            for (int d = pre; d < ndt; ++d) {
+                const TaskDesc u = S.dnt[d];
+                const uint32_t *uq, *usb;
+                task_ptrs(P, W, u, true, uq, usb);
+                const int ng = u.g1 - u.g0;
+                prefetch_l2(uq + (size_t)u.g0 * 256, (unsigned)ng * kCodeBytesPerGroup);
+                prefetch_l2(usb + (size_t)u.g0 * 32, (unsigned)ng * kSbBytesPerGroup);
             }
+        }
+    }
+    if (ok && down && l + 1 < P.L) {
+        // this CTA's share of the next layer's shared-expert weights
+        const moe_layer_w &N = P.layers[l + 1];
+        const size_t shq = (size_t)P.Is * P.H / 2, shsb = (size_t)P.Is * (P.H / 64) * 4;
+        const void *ptrs[6] = {N.sh_gate.q, N.sh_up.q, N.sh_down.q, N.sh_gate.sb, N.sh_up.sb, N.sh_down.sb};
+        const size_t sizes[6] = {shq, shq, shq, shsb, shsb, shsb};
+#pragma unroll 1
+        for (int a = 0; a < 6; ++a) {
+            const size_t per = ((sizes[a] / gridDim.x) + 15) & ~(size_t)15;
+            const size_t off = per * blockIdx.x;
+            if (off < sizes[a])
+                prefetch_range(static_cast<const char *>(ptrs[a]) + off,
+                               (off + per <= sizes[a] ? per : sizes[a] - off) & ~(size_t)15);
         }
     }
     return ok;
 }
 
-// Chunk sums (sum of the unscaled values) of nchunks 32-float chunks of the
-// stage, one consumer thread per chunk, bank-rotated.
-__device__ __noinline__ void chunk_sums(Smem &S, int nchunks) {
+// A warp's share of a task: lanes are the task's 32 rows; acc[tt] receives
+// the dot product of the row's groups [g0, g1) with token tt's input.
+template <int NT>
+__device__ __forceinline__ void task_dot(const unsigned char *slot, int ng, const float *x, const float *xsum,
+                                         const int *tokrow, int stride, int n, float (&acc)[NT], int lane) {
+#pragma unroll 1
+    for (int gi = 0; gi < ng; ++gi)
+        group_dot_n<NT>(slot + gi * kCodeBytesPerGroup,
+                        reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane],
+                        x + gi * 64, xsum + 2 * gi, tokrow, stride, n, acc, lane);
+}
+
+// A consumer warp's wait for task q in ring slot s: first until the producer
+// has handed the slot to q (the slot's previous task is done, so its full
+// barrier is in q's phase), then for the phase itself.  Warps take tasks out
+// of ring order, so without the first wait a warp could test a phase two
+// ahead of the barrier's, which the parity test cannot tell apart.
+__device__ __noinline__ bool wait_task(Smem &S, unsigned q, int s, unsigned ph, int *err) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) {
+        const volatile unsigned *own = &S.slot_task[s];
+        if (*own != q) {
+            const unsigned long long t0 = globaltimer();
+            while (*own != q) {
+                if (globaltimer() - t0 > kWaitNs || ldcg_int(err) != 0) {
+                    atomicCAS(err, 0, kErrFull);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+    }
+    __syncwarp();
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    return ok && mbar_wait(&S.full[s], ph, err, kErrFull);
+}
+
+__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned *p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+template <int NT>
+__device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int T = P.T, ns = P.nslots, nt = S.ngt, pg = S.pg, tpj = 2 * pg;
+    bool ok = true;
+#pragma unroll 1
+    for (int i = wid; i < nt; i += kCWarps) {
+        const TaskDesc t = S.gut[i];
+        int s;
+        unsigned ph;
+        ring_pos(rq, i, ns, s, ph);
+        const int n = t.n, ng = t.g1 - t.g0;
+        float acc[NT];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
+        const bool got = wait_task(S, rq + (unsigned)i, s, ph, P.err);
+        if (got) {
+            const int *tokrow = t.slot == 0 ? S.tokrow_sh : S.tokrow + t.seg0;
+            const int col = t.g0 * 64;
+            task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, S.stage + col, S.xs + col / 32, tokrow, 0, n, acc, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[s]);
+        if (!got) {
+            ok = false;
+            continue;
+        }
+        // this task's partial sums, then its count for the job (release: the
+        // warp's stores, ordered by __syncwarp, become visible first)
+        float *gp = P.gpart + (((size_t)t.job * 2 + t.mat) * pg + t.part) * T * 32;
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt)
+            if (tt < n) gp[tt * 32 + lane] = acc[tt];
+        __syncwarp();
+        unsigned old = 0u;
+        if (lane == 0) old = atom_add_release_gpu(&P.cnt_gu[t.job], 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == (unsigned)(tpj - 1)) {
+            // the job's last task: sum the parts in a fixed order, form a = silu(g) * u
+            if (lane == 0) __threadfence();
+            __syncwarp();
+            const float *jp = P.gpart + (size_t)t.job * 2 * pg * T * 32;
+#pragma unroll 1
+            for (int tt = 0; tt < n; ++tt) {
+                float gs = 0.f, us = 0.f;
+#pragma unroll
+                for (int p2 = 0; p2 < kMaxPG; ++p2) {
+                    if (p2 < pg) {
+                        gs += __ldcg(&jp[((size_t)p2 * T + tt) * 32 + lane]);
+                        us += __ldcg(&jp[((size_t)(pg + p2) * T + tt) * 32 + lane]);
+                    }
+                }
+                P.act[(size_t)task_rowset(P, t, tt) * P.Kmax + t.rb * 32 + lane] = silu_mul(gs, us);
+            }
+            __syncwarp();
+            if (lane == 0) P.cnt_gu[t.job] = 0u;
+        }
+    }
+    return ok;
+}
+
+// Chunk sums (sum of the unscaled values) of chunks [c0, c1) of the stage, bank-rotated.
+__device__ __noinline__ void chunk_sums(Smem &S, int c0, int c1) {
     const float *stage = S.stage;
 #pragma unroll 1
-    for (int i = threadIdx.x; i < nchunks; i += kCWarps * 32) {
+    for (int i = c0 + threadIdx.x; i < c1; i += kCWarps * 32) {
         const float *row = stage + (size_t)i * 32;
         float sx = 0.f;
 #pragma unroll 4
@@ -902,144 +959,131 @@ __device__ __noinline__ void chunk_sums(Smem &S, int nchunks) {
     }
 }
 
-__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned *p, unsigned v) {
-    unsigned old;
-    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+// Stage the down inputs of segments [k0, k1): a pre-scaled for the code
+// decode, and the chunk sums.  Consumer threads only.
+__device__ __noinline__ void stage_segments(const Params &P, Smem &S, int k0, int k1) {
+    const int ctid = threadIdx.x;
+#pragma unroll 1
+    for (int k2 = k0; k2 < k1; ++k2) {
+        const SegDesc sg = S.seg[k2];
+        const int q4 = sg.ld / 4;
+        const int rs0 = sg.slot == 0 ? 0 : P.T + sg.seg0;
+#pragma unroll 1
+        for (int e = ctid; e < sg.n * q4; e += kCWarps * 32) {
+            const int tt = e / q4, c4 = e - tt * q4;
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(P.act + (size_t)(rs0 + tt) * P.Kmax + sg.g0 * 64) + c4);
+            const int c = 4 * c4;
+            float4 v;
+            v.x = a.x * code_prescale(c & 7);
+            v.y = a.y * code_prescale((c + 1) & 7);
+            v.z = a.z * code_prescale((c + 2) & 7);
+            v.w = a.w * code_prescale((c + 3) & 7);
+            reinterpret_cast<float4 *>(S.stage + sg.off + (size_t)tt * sg.ld)[c4] = v;
+        }
+    }
+    consumer_sync();
+    if (k1 > k0) {
+        const SegDesc &a = S.seg[k0], &b = S.seg[k1 - 1];
+        chunk_sums(S, a.off / 32, (b.off + b.n * b.ld) / 32);
+    }
+    consumer_sync();
 }
 
-// The combine m[t][rows of rb] = sum_s w[t,s] * y[t,s] + shared, in a fixed
-// order; the loads of a batch are issued before any is used.
-__device__ __noinline__ void combine_rows(const Params &P, const Smem &S, int rb, int t, int ln) {
-    const int T = P.T, k = P.k, H = P.H, row = rb * 32 + ln;
+
+// The combine m[t][row] = sum_s w[t,s] * y[t,s] + shared, in a fixed order;
+// the loads of a batch are issued before any is used.
+__device__ __noinline__ void combine_row(const Params &P, const Smem &S, int row) {
+    const int T = P.T, k = P.k, H = P.H;
     const size_t ystride = (size_t)T * k * H;
-    float mv = 0.f;
-    for (int s0 = 0; s0 < k; s0 += 8) {
-        float yv[8];
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        float mv = 0.f;
+#pragma unroll 1
+        for (int s0 = 0; s0 < k; s0 += 8) {
+            float yv[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) yv[u] = s0 + u < k ? __ldcg(&P.y[(size_t)(t * k + s0 + u) * H + row]) : 0.f;
-        for (int dp = 1; dp < P.ndp_r; ++dp) {
-            float yd[8];
+            for (int u = 0; u < 8; ++u) yv[u] = s0 + u < k ? __ldcg(&P.y[(size_t)(t * k + s0 + u) * H + row]) : 0.f;
+#pragma unroll 1
+            for (int dp = 1; dp < P.ndp_r; ++dp) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u < k) yv[u] += __ldcg(&P.y[dp * ystride + (size_t)(t * k + s0 + u) * H + row]);
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                yd[u] = s0 + u < k ? __ldcg(&P.y[dp * ystride + (size_t)(t * k + s0 + u) * H + row]) : 0.f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) yv[u] += yd[u];
+                if (s0 + u < k) mv = fmaf(S.wts[t * k + s0 + u], yv[u], mv);
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (s0 + u < k) mv = fmaf(S.wts[t * k + s0 + u], yv[u], mv);
-    }
-    for (int d0 = 0; d0 < P.ndp_s; d0 += 4) {
         float sv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) sv[u] = d0 + u < P.ndp_s ? __ldcg(&P.sh[((size_t)(d0 + u) * T + t) * H + row]) : 0.f;
+        for (int u = 0; u < 4; ++u) sv[u] = u < P.ndp_s ? __ldcg(&P.sh[((size_t)u * T + t) * H + row]) : 0.f;
+#pragma unroll 1
+        for (int u = 4; u < P.ndp_s; ++u) mv += __ldcg(&P.sh[((size_t)u * T + t) * H + row]);
 #pragma unroll
         for (int u = 0; u < 4; ++u) mv += sv[u];
+        P.m[(size_t)t * H + row] = mv;
     }
-    P.m[(size_t)t * H + row] = mv;
 }
 
 template <int NT>
-__device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, Ring ring) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, ctid = threadIdx.x;
-    bool ok = true;
-    int buf = 0;
-    const int T = P.T, k = P.k, H = P.H, ns = P.nslots, ndn = S.ndn, Kmax = P.Kmax;
-    // down jobs per row block in this layer: every part of the shared expert and of each active slot
+__device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int T = P.T, k = P.k, H = P.H, ns = P.nslots, nt = S.ndt;
+    // down tasks per row block in this layer: every part of the shared expert and of each active slot
     const unsigned dn_per_rb = (unsigned)(P.ndp_s + S.nact * P.ndp_r);
-    float *stage = S.stage;
-    int staged_slot = -1, staged_part = -1;
-    // thread 0 counts each finished job; the count returned for job i is examined one job later
-    unsigned pend_old = 0u;
-    int pend_rb = -1;
-    if (ctid == 0) S.nlast = 0;
+    const int rounds = S.seg_rounds;
+    bool ok = true;
 #pragma unroll 1
-    for (int i = 0; i < ndn; ++i) {
-        const JobDesc J = S.dnjob[i];
-        const int ng = J.g1 - J.g0, n = J.n, ld = ng * 64;
-        if (J.slot != staged_slot || J.part != staged_part) {
-            // this slot's SwiGLU rows, columns [g0*64, g1*64): token tt at tt * ld
-            const int q4 = ld / 4;
+    for (int r = 0; r < rounds; ++r) {
+        const int k0 = rounds == 1 ? 0 : r, k1 = rounds == 1 ? S.nseg : r + 1;
+        stage_segments(P, S, k0, k1);
 #pragma unroll 1
-            for (int e = ctid; e < n * q4; e += kCWarps * 32) {
-                const int tt = e / q4, c4 = e - tt * q4;
-                const float4 a = __ldcg(reinterpret_cast<const float4 *>(
-                                            P.act + (size_t)job_rowset(P, J, tt) * Kmax + J.g0 * 64) + c4);
-                const int c = 4 * c4;  // c % 8 is 0 or 4
-                float4 v;
-                v.x = a.x * code_prescale(c & 7);
-                v.y = a.y * code_prescale((c + 1) & 7);
-                v.z = a.z * code_prescale((c + 2) & 7);
-                v.w = a.w * code_prescale((c + 3) & 7);
-                reinterpret_cast<float4 *>(stage + (size_t)tt * ld)[c4] = v;
-            }
-            consumer_sync();
-            chunk_sums(S, n * 2 * ng);
-            staged_slot = J.slot;
-            staged_part = J.part;
-            consumer_sync();
-        }
-        const bool got = mbar_wait(&S.full[ring.s], ring.ph, P.err, kErrFull);
-        float *Rb = S.red[buf];
-        if (got && wid < ng) {
-            const int gi = wid;
-            const unsigned char *slot = S.pool + (size_t)ring.s * kSlotBytes;
-            const unsigned char *codes = slot + gi * kCodeBytesPerGroup;
-            const uint32_t sbw =
-                reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane];
+        for (int i = wid; i < nt; i += kCWarps) {
+            const TaskDesc t = S.dnt[i];
+            if (t.seg < k0 || t.seg >= k1) continue;
+            int s;
+            unsigned ph;
+            ring_pos(rq, i, ns, s, ph);
+            const SegDesc sg = S.seg[t.seg];
+            const int n = t.n, ng = t.g1 - t.g0;
             float acc[NT];
 #pragma unroll
             for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
-            // token tt's row at tt * ld, its chunk sums at tt * ld / 32
-            group_dot_n<NT>(codes, sbw, stage + gi * 64, S.xs + 2 * gi, nullptr, ld, n, acc, lane);
+            const bool got = wait_task(S, rq + (unsigned)i, s, ph, P.err);
+            if (got)  // token tt's row at off + tt * ld, its chunk sums at (off + tt * ld) / 32
+                task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, S.stage + sg.off, S.xs + sg.off / 32, nullptr,
+                             sg.ld, n, acc, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.empty[s]);
+            if (!got) {
+                ok = false;
+                continue;
+            }
+            const int row = t.rb * 32 + lane;
 #pragma unroll
-            for (int tt = 0; tt < NT; ++tt)
-                if (tt < n) Rb[(gi * kMaxT + tt) * 32 + lane] = acc[tt];
+            for (int tt = 0; tt < NT; ++tt) {
+                if (tt < n) {
+                    if (t.slot == 0)
+                        P.sh[((size_t)t.part * T + tt) * H + row] = acc[tt];
+                    else
+                        P.y[((size_t)t.part * T * k + S.perm[t.seg0 + tt]) * H + row] = acc[tt];
+                }
+            }
+            // count this task for its row block (release: the warp's rows, ordered
+            // by __syncwarp, become visible first); the last one forms the combine
+            __syncwarp();
+            unsigned old = 0u;
+            if (lane == 0) old = atom_add_release_gpu(&P.cnt_dn[t.rb], 1u);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old == dn_per_rb - 1u) {
+                if (lane == 0) __threadfence();
+                __syncwarp();
+                combine_row(P, S, row);
+                __syncwarp();
+                if (lane == 0) P.cnt_dn[t.rb] = 0u;
+            }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[ring.s]);
-        if (!got) ok = false;
-        ring_next(ring, ns);
-        consumer_sync();
-#pragma unroll 1
-        for (int r = ctid; r < n * 32; r += kCWarps * 32) {
-            const int tt = r >> 5, ln = r & 31;
-            float v = 0.f;
-#pragma unroll 4
-            for (int g2 = 0; g2 < ng; ++g2) v += Rb[(g2 * kMaxT + tt) * 32 + ln];
-            const int row = J.rb * 32 + ln;
-            if (J.slot == 0)
-                P.sh[((size_t)J.part * T + tt) * H + row] = v;
-            else
-                P.y[((size_t)J.part * T * k + S.perm[J.seg0 + tt]) * H + row] = v;
-        }
-        // count this job for its row block (release: the y rows above, ordered
-        // by the barrier, become visible before the count); the previous
-        // job's count has long returned by now
-        consumer_sync();
-        if (ctid == 0) {
-            if (pend_rb >= 0 && pend_old == dn_per_rb - 1u) S.last_rb[S.nlast++] = (int16_t)pend_rb;
-            pend_old = atom_add_release_gpu(&P.cnt_dn[J.rb], 1u);
-            pend_rb = J.rb;
-        }
-        buf ^= 1;
+        if (rounds > 1) consumer_sync();
     }
-    if (ctid == 0) {
-        if (pend_rb >= 0 && pend_old == dn_per_rb - 1u) S.last_rb[S.nlast++] = (int16_t)pend_rb;
-        if (S.nlast > 0) __threadfence();  // acquire the other jobs' rows
-    }
-    consumer_sync();
-    // the combine of the row blocks this CTA finished last
-    const int nl = S.nlast;
-#pragma unroll 1
-    for (int r = ctid; r < nl * T * 32; r += kCWarps * 32) {
-        const int li = r / (T * 32), rem = r - li * T * 32;
-        const int rb = S.last_rb[li];
-        combine_rows(P, S, rb, rem >> 5, rem & 31);
-    }
-    consumer_sync();
-    if (ctid < nl) P.cnt_dn[S.last_rb[ctid]] = 0u;
     return ok;
 }
 
@@ -1055,16 +1099,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], kCWarps);
+            mbar_init(&S.empty[s], 1);  // one consumer warp per task
         }
         mbar_init(&S.rbar, 1);
+        for (int s = 0; s < kMaxStages; ++s) S.slot_task[s] = 0xffffffffu;
         S.stage = reinterpret_cast<float *>(S.pool + (size_t)P.nslots * kSlotBytes);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
-    Ring ring{0u, 0, 0u};  // position of the next job stage (the same in every thread)
-    unsigned issued = 0;   // producer: stages whose copies were actually issued
+    unsigned rq = 0;       // ring sequence number of the next task (the same in every thread)
+    unsigned issued = 0;   // producer: tasks whose copies were actually issued
     unsigned rissued = 0;  // producer: router copy batches issued (one per layer)
     unsigned nbar = 0;     // grid barriers passed
     bool ok = true;
@@ -1088,21 +1133,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         topk_phase(P, S, W);
         stage_x(P, S);
 
-        // ---------------- gate/up jobs
+        // ---------------- gate/up tasks
         if (producer)
-            gu_producer(P, S, W, ring, issued);
+            task_producer(P, S, W, false, rq, l, issued);
         else if (consumer)
-            P.T == 1 ? gu_consumer<1>(P, S, ring) : gu_consumer<kMaxT>(P, S, ring);
-        for (int st = S.gu_stages; st > 0; --st) ring_next(ring, ns);
+            P.T == 1 ? gu_consumer<1>(P, S, rq) : gu_consumer<kMaxT>(P, S, rq);
+        rq += (unsigned)S.ngt;
         ok = grid_sync(P, ++nbar, &S.flag);
         if (!ok) break;
 
-        // ---------------- down jobs
+        // ---------------- down tasks
         if (producer)
-            dn_producer(P, S, W, ring, l, issued);
+            task_producer(P, S, W, true, rq, l, issued);
         else if (consumer)
-            P.T == 1 ? dn_consumer<1>(P, S, ring) : dn_consumer<kMaxT>(P, S, ring);
-        for (int st = S.ndn; st > 0; --st) ring_next(ring, ns);
+            P.T == 1 ? dn_consumer<1>(P, S, rq) : dn_consumer<kMaxT>(P, S, rq);
+        rq += (unsigned)S.ndt;
         ok = grid_sync(P, ++nbar, &S.flag);
     }
     if (ok) finish_layer(P, S, P.L - 1);  // ok is uniform across the CTA here
@@ -1124,7 +1169,7 @@ static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exce
 static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
 
 struct DecodeWs {
-    size_t bar, cnt_dn, logits, act, y, sh, m, total, zero_bytes;
+    size_t bar, cnt_dn, cnt_gu, logits, gpart, act, y, sh, m, total, zero_bytes;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1133,8 +1178,8 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
     DecodeWs d;
     const int Kmax = w->I > w->Is ? w->I : w->Is;
     const int R = T + T * w->k;
-    const int ndp_r = (w->I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
-    const int ndp_s = (w->Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
+    const int ndp_r = (w->I / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
+    const int ndp_s = (w->Is / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
     size_t off = 0;
     auto take = [&](size_t b) {
         const size_t o = off;
@@ -1142,8 +1187,13 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
         return o;
     };
     d.bar = take(256);
+    const size_t pairs = (size_t)T * w->k < (size_t)w->E ? (size_t)T * w->k : (size_t)w->E;
+    const size_t jobs = (size_t)w->Is / 32 + pairs * (w->I / 32);
+    const size_t pg = (w->H / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
     d.cnt_dn = take(sizeof(unsigned) * (size_t)(w->H / 32));
+    d.cnt_gu = take(sizeof(unsigned) * jobs);
     d.zero_bytes = off;
+    d.gpart = take(sizeof(float) * jobs * 2 * pg * T * 32);
     d.logits = take(sizeof(double) * (size_t)T * w->E);
     d.act = take(sizeof(float) * (size_t)R * Kmax);
     d.y = take(sizeof(float) * (size_t)ndp_r * T * w->k * w->H);
@@ -1159,8 +1209,8 @@ size_t decode_stack_status_offset() { return sizeof(unsigned); }
 
 // Split of the shared-memory pool between the ring and the input stage for
 // calls of T tokens on layers shaped like w; false if the shape does not fit.
-static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots) {
-    const long th = (long)T * w.H, tdn = (long)T * dec::kDnGroups * 64;
+static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots, int *stage_floats) {
+    const long th = (long)T * w.H, tdn = (long)T * dec::kTaskGroups * 64;
     long stage = th > tdn ? th : tdn;
     if (stage > dec::kStageFloats || stage / 32 > dec::kMaxXs) return false;
     stage = (stage + 31) & ~31L;  // keep the stage 128-byte aligned
@@ -1169,14 +1219,26 @@ static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots) {
     const long ring = ns * dec::kSlotBytes;
     const long rows = grid > 0 ? (w.E + grid - 1) / grid : w.E;
     const long rcopy = 2L * w.H + rows * w.H + 2 * (rows * (w.H / 64) * 2 + 32);
-    if (ns < 3 || (long)T * w.E * 8 > ring || rcopy > ring) return false;
+    if (ns < 3 || (long)T * w.E * 8 > ring || rcopy > ring || grid <= 0) return false;
+    // task tables of the busiest CTA, for the most distinct experts a call can route to
+    const long pairs = (long)T * w.k < w.E ? (long)T * w.k : w.E;
+    const long pg = (w.H / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
+    const long j2 = w.Is / 32 + pairs * (w.I / 32);
+    const long ndp_r = (w.I / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
+    const long ndp_s = (w.Is / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
+    const long rbh = w.H / 32, j3 = (ndp_s + pairs * ndp_r) * rbh;
+    const long gu_tasks = (j2 * 2 * pg + grid - 1) / grid, dn_tasks = (j3 + grid - 1) / grid;
+    if (pg > dec::kMaxPG || gu_tasks > dec::kMaxTasks || dn_tasks > dec::kMaxTasks ||
+        (dn_tasks + rbh - 1) / rbh + 1 > dec::kMaxSegs)
+        return false;
     *nslots = (int)ns;
+    *stage_floats = (int)((dec::kPoolBytes - ring) / 4);
     return true;
 }
 
 bool decode_stack_fits(const moe_layer_w *w, int T, int grid) {
-    int a;
-    return decode_layout(*w, T, grid, &a);
+    int a, b;
+    return decode_layout(*w, T, grid, &a, &b);
 }
 
 int decode_stack_max_tokens() { return dec::kMaxT; }
@@ -1204,14 +1266,16 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.Is = w.Is;
     P.Kmax = w.I > w.Is ? w.I : w.Is;
     P.R = T + T * w.k;
-    P.ndp_r = (w.I / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
-    P.ndp_s = (w.Is / 64 + dec::kDnGroups - 1) / dec::kDnGroups;
-    if (!decode_layout(w, T, grid, &P.nslots)) return cudaErrorInvalidValue;
+    P.ndp_r = (w.I / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
+    P.ndp_s = (w.Is / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
+    if (!decode_layout(w, T, grid, &P.nslots, &P.stage_floats)) return cudaErrorInvalidValue;
     char *base = static_cast<char *>(ws);
     P.bar = reinterpret_cast<unsigned *>(base + d.bar);
     P.err = reinterpret_cast<int *>(base + d.bar + sizeof(unsigned));
     P.logits = reinterpret_cast<double *>(base + d.logits);
     P.cnt_dn = reinterpret_cast<unsigned *>(base + d.cnt_dn);
+    P.cnt_gu = reinterpret_cast<unsigned *>(base + d.cnt_gu);
+    P.gpart = reinterpret_cast<float *>(base + d.gpart);
     P.act = reinterpret_cast<float *>(base + d.act);
     P.y = reinterpret_cast<float *>(base + d.y);
     P.sh = reinterpret_cast<float *>(base + d.sh);
