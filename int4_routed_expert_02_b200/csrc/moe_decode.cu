@@ -91,7 +91,9 @@ struct Params {
     unsigned *cnt_gu;  // [jobs]: gate/up tasks done per job; reset by the last
     float *gpart;      // [jobs][2][pg][T][32]: gate/up partial sums per task
     double *logits;  // [T,E]
-    float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs)
+    float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs),
+                     // pre-scaled for the code decode
+    float *act_cs;   // [R][Kmax/32]: sums of a over 32-column chunks
     float *y;        // [ndp_r][T*k][H]
     float *sh;       // [ndp_s][T][H]
     float *m;        // [T][H]: the combine m of the current layer
@@ -126,13 +128,12 @@ struct Smem {
     SegDesc seg[kMaxSegs];
     int ngt, ndt, pg, nseg, seg_rounds;
     double selv[kMaxPairs];
-    double pe[kMaxPairs];
     float wts[kMaxPairs];
     int idx[kMaxPairs];
     int perm[kMaxPairs];
+    int act_e[kMaxPairs], act_off[kMaxPairs], act_n[kMaxPairs];
     int poff[kMaxPairs], pcnt[kMaxPairs];
     unsigned char first[kMaxPairs];
-    int act_e[kMaxPairs], act_off[kMaxPairs], act_n[kMaxPairs];
     int tokrow[kMaxPairs];  // bucketed position j -> row offset (token * H) of its input
     int tokrow_sh[kMaxT];   // shared expert: token t -> t * H
     int nact;
@@ -262,9 +263,9 @@ __device__ __noinline__ bool grid_sync(const Params &P, unsigned nth, int *verdi
 // phase.  Job j = gt / (2 pg) is 32 rows of the shared expert or of one
 // active slot; its 2 pg tasks are part p of gate and of up, p = 0..pg-1.
 // All divisions happen here, once per task.
-__device__ __noinline__ TaskDesc make_gu_task(const Params &P, const Smem &S, int gt) {
+__device__ __forceinline__ TaskDesc make_gu_task(const Params &P, const Smem &S, int gt, int pg) {
     TaskDesc t;
-    const int pg = S.pg, j = gt / (2 * pg), r = gt - j * 2 * pg;
+    const int j = gt / (2 * pg), r = gt - j * 2 * pg;
     const int A = P.Is / 32;
     if (j < A) {
         t.slot = 0;
@@ -304,7 +305,7 @@ __device__ __forceinline__ void dn_slot_part(const Params &P, int sp, int &slot,
 }
 
 // Task d (grid-wide index) of the down phase: (slot, part) d / (H/32), row block d % (H/32).
-__device__ __noinline__ TaskDesc make_dn_task(const Params &P, const Smem &S, int d, int sp0) {
+__device__ __forceinline__ TaskDesc make_dn_task(const Params &P, const Smem &S, int d, int sp0) {
     TaskDesc t;
     const int RBH = P.H / 32, sp = d / RBH;
     int slot, part;
@@ -628,74 +629,118 @@ __device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
 // Every CTA.
 __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_layer_w &W) {
     const int T = P.T, E = P.E, k = P.k, n = T * k, H = P.H;
-    double *lg = reinterpret_cast<double *>(S.pool);  // ring is idle here: T*E doubles
+    // the logits as order-preserving unsigned keys (larger logit <=> larger
+    // key, exactly): a compare of two keys is integer work, not fp64
+    unsigned long long *lk = reinterpret_cast<unsigned long long *>(S.pool);  // ring is idle here: T*E keys
 #pragma unroll 1
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = __ldcg(P.logits + i);
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+        unsigned long long b = (unsigned long long)__double_as_longlong(__ldcg(P.logits + i));
+        if (b == 0x8000000000000000ull) b = 0ull;  // -0 and +0 are the same logit
+        lk[i] = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+    }
     __syncthreads();
+    // F adjacent lanes share one (token, expert): each counts over a quarter
+    // (F = 4) of the other experts, and the counts are summed by shuffles
+    const int F = T * E * 4 <= (int)blockDim.x ? 4 : 1, items = T * E * F, Ej = E / (2 * F);
 #pragma unroll 1
-    for (int t = 0; t < T; ++t) {
-        const double2 *row = reinterpret_cast<const double2 *>(lg + (size_t)t * E);
-#pragma unroll 1
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            const double v = lg[(size_t)t * E + e];
-            int rank = 0;
-#pragma unroll 2
-            for (int j = 0; j < E / 2; ++j) {  // E is a multiple of 8
-                const double2 o = row[j];
-                rank += (o.x > v) | ((o.x == v) & (2 * j < e));
-                rank += (o.y > v) | ((o.y == v) & (2 * j + 1 < e));
+    for (int it0 = 0; it0 < items; it0 += blockDim.x) {
+        const int it = it0 + threadIdx.x;
+        const int te = it / F, f = it - te * F;
+        int rank = 0;
+        unsigned long long v = 0ull;
+        int t = 0, e = 0;
+        if (it < items) {
+            t = te / E;
+            e = te - t * E;
+            v = lk[(size_t)t * E + e];
+            const ulonglong2 *row = reinterpret_cast<const ulonglong2 *>(lk + (size_t)t * E) + f * Ej;
+            const int jb = 2 * f * Ej;
+#pragma unroll 4
+            for (int j = 0; j < Ej; ++j) {  // E is a multiple of 8
+                const ulonglong2 o = row[j];
+                rank += (o.x > v) | ((o.x == v) & (jb + 2 * j < e));
+                rank += (o.y > v) | ((o.y == v) & (jb + 2 * j + 1 < e));
             }
-            if (rank < k) {
-                S.idx[t * k + rank] = e;
-                S.selv[t * k + rank] = v;
-            }
+        }
+        if (F == 4) {
+            rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+            rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+        }
+        if (it < items && f == 0 && rank < k) {
+            S.idx[t * k + rank] = e;
+            // back from the key to the logit
+            const unsigned long long b = (v >> 63) ? (v & 0x7fffffffffffffffull) : ~v;
+            S.selv[t * k + rank] = __longlong_as_double((long long)b);
         }
     }
     __syncthreads();
-    if (threadIdx.x < n) {
-        const int t = threadIdx.x / k;
-        S.pe[threadIdx.x] = exp(S.selv[threadIdx.x] - S.selv[t * k]);  // selv[t*k] is the token's maximum
-    }
-    __syncthreads();
-    if (threadIdx.x < n) {
-        const int p = threadIdx.x, t = p / k;
-        double z = 0.0;
-#pragma unroll 1
-        for (int s = 0; s < k; ++s) z += S.pe[t * k + s];
-        const int e = S.idx[p];
-        S.wts[p] = (float)(S.pe[p] / z * (double)bf16_bits_to_float(W.per_expert_scale[e]));
-        // position of pair p among all pairs ordered by (expert, pair id)
-        int less = 0, eqb = 0, cnt = 0;
-#pragma unroll 1
-        for (int q = 0; q < n; ++q) {
-            const int f = S.idx[q];
-            less += f < e;
-            eqb += (f == e) & (q < p);
-            cnt += f == e;
+    // bucketing: pair p's position among all pairs ordered by (expert, pair
+    // id), and the slot of its expert among the distinct experts (ascending).
+    // Few pairs: one pass that also finds first occurrences by rescanning;
+    // many pairs: first occurrences in a pass of their own.
+    if (n <= 16) {
+        int id[16];  // every pair's expert, in registers
+#pragma unroll
+        for (int q = 0; q < 16; ++q) id[q] = q < n ? S.idx[q] : 0x7fffffff;
+        if (threadIdx.x < n) {
+            const int p = threadIdx.x, t = p / k, e = S.idx[p];
+            int less = 0, eqb = 0, cnt = 0, slot = 0, nact = 0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int f = id[q];
+                bool firstq = q < n;
+#pragma unroll
+                for (int r = 0; r < q; ++r) firstq &= id[r] != f;
+                less += f < e;
+                eqb += (f == e) & (q < p);
+                cnt += f == e;
+                slot += firstq & (f < e);
+                nact += firstq;
+            }
+            S.perm[less + eqb] = p;
+            S.tokrow[less + eqb] = t * H;
+            if (eqb == 0) {
+                S.act_e[slot] = e;
+                S.act_off[slot] = less;
+                S.act_n[slot] = cnt;
+            }
+            if (p == 0) S.nact = nact;
         }
-        S.perm[less + eqb] = p;
-        S.tokrow[less + eqb] = t * H;
-        S.first[p] = eqb == 0;
-        S.poff[p] = less;
-        S.pcnt[p] = cnt;
+    } else {
+        if (threadIdx.x < n) {
+            const int p = threadIdx.x, t = p / k, e = S.idx[p];
+            int less = 0, eqb = 0, cnt = 0;
+#pragma unroll 1
+            for (int q = 0; q < n; ++q) {
+                const int f = S.idx[q];
+                less += f < e;
+                eqb += (f == e) & (q < p);
+                cnt += f == e;
+            }
+            S.perm[less + eqb] = p;
+            S.tokrow[less + eqb] = t * H;
+            S.first[p] = eqb == 0;
+            S.poff[p] = less;
+            S.pcnt[p] = cnt;
+        }
+        __syncthreads();
+        if (threadIdx.x < n) {
+            const int p = threadIdx.x, e = S.idx[p];
+            int slot = 0, nact = 0;
+#pragma unroll 1
+            for (int q = 0; q < n; ++q) {
+                slot += S.first[q] & (S.idx[q] < e);
+                nact += S.first[q];
+            }
+            if (S.first[p]) {
+                S.act_e[slot] = e;
+                S.act_off[slot] = S.poff[p];
+                S.act_n[slot] = S.pcnt[p];
+            }
+            if (p == 0) S.nact = nact;
+        }
     }
     if (threadIdx.x < T) S.tokrow_sh[threadIdx.x] = threadIdx.x * H;
-    __syncthreads();
-    if (threadIdx.x < n) {
-        const int p = threadIdx.x, e = S.idx[p];
-        int slot = 0, nact = 0;
-#pragma unroll 1
-        for (int q = 0; q < n; ++q) {
-            slot += S.first[q] & (S.idx[q] < e);
-            nact += S.first[q];
-        }
-        if (S.first[p]) {  // one slot per distinct expert, ascending expert id
-            S.act_e[slot] = e;
-            S.act_off[slot] = S.poff[p];
-            S.act_n[slot] = S.pcnt[p];
-        }
-        if (p == 0) S.nact = nact;
-    }
     __syncthreads();
     // task tables of this CTA.  Gate/up jobs are dealt round-robin (every CTA
     // mixes shared-expert jobs with routed ones); down tasks go in contiguous
@@ -708,59 +753,107 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     const int J3 = (P.ndp_s + na * P.ndp_r) * RBH;
     const int d0 = (int)((long long)J3 * c / G), d1 = (int)((long long)J3 * (c + 1) / G);
     const int sp0 = d0 / RBH;
+    // staged down inputs: the (slot, part) of the CTA's tasks, consecutive; one
+    // thread per input, each adding up the sizes of the ones before it
+    const int nseg = min(d1 > d0 ? (d1 - 1) / RBH - sp0 + 1 : 0, kMaxSegs);
+    const int ngt = min(n2, kMaxTasks), ndt = min(d1 - d0, kMaxTasks);
+    if (threadIdx.x < nseg) {
+        const int k2 = threadIdx.x;
+        int off = 0, slot = 0, part = 0;
+#pragma unroll 1
+        for (int q = 0; q <= k2; ++q) {
+            dn_slot_part(P, sp0 + q, slot, part);
+            const int Gs = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
+            const int ld = (Gs * (part + 1) / nd - Gs * part / nd) * 64;
+            const int nn = slot == 0 ? P.T : S.act_n[slot - 1];
+            if (q < k2) off += nn * ld;
+        }
+        const int Gs = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
+        SegDesc &sg = S.seg[k2];
+        sg.slot = (int16_t)slot;
+        sg.part = (int16_t)part;
+        sg.g0 = (int16_t)(Gs * part / nd);
+        sg.ld = (int16_t)((Gs * (part + 1) / nd - sg.g0) * 64);
+        sg.n = (int16_t)(slot == 0 ? P.T : S.act_n[slot - 1]);
+        sg.seg0 = slot == 0 ? 0 : S.act_off[slot - 1];
+        sg.off = off;
+        sg.pad = 0;
+        if (k2 == nseg - 1) {
+            // all inputs at once if they fit the stage (and its chunk sums), else one
+            // (slot, part) at a time, each from the start of the stage
+            S.seg_rounds = off + sg.n * sg.ld <= min(P.stage_floats, kMaxXs * 32) ? 1 : nseg;
+        }
+    }
     if (threadIdx.x == 0) {
         S.pg = pg;
-        S.ngt = min(n2, kMaxTasks);
-        S.ndt = min(d1 - d0, kMaxTasks);
-        // staged down inputs: the (slot, part) of the CTA's tasks, consecutive
-        int nseg = d1 > d0 ? (d1 - 1) / RBH - sp0 + 1 : 0, off = 0;
-        nseg = min(nseg, kMaxSegs);
-        for (int k2 = 0; k2 < nseg; ++k2) {
-            int slot, part;
-            dn_slot_part(P, sp0 + k2, slot, part);
-            const int Gs = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
-            SegDesc &sg = S.seg[k2];
-            sg.slot = (int16_t)slot;
-            sg.part = (int16_t)part;
-            sg.g0 = (int16_t)(Gs * part / nd);
-            sg.ld = (int16_t)((Gs * (part + 1) / nd - sg.g0) * 64);
-            sg.n = (int16_t)(slot == 0 ? P.T : S.act_n[slot - 1]);
-            sg.seg0 = slot == 0 ? 0 : S.act_off[slot - 1];
-            sg.off = off;
-            sg.pad = 0;
-            off += sg.n * sg.ld;
-        }
+        S.ngt = ngt;
+        S.ndt = ndt;
         S.nseg = nseg;
-        // all inputs at once if they fit the stage (and its chunk sums), else one
-        // (slot, part) at a time, each from the start of the stage
-        S.seg_rounds = off <= min(P.stage_floats, kMaxXs * 32) ? 1 : nseg;
-        if (S.seg_rounds > 1)
-            for (int k2 = 0; k2 < nseg; ++k2) S.seg[k2].off = 0;
+        if (nseg == 0) S.seg_rounds = 1;
+    }
+    // gate/up tables on the first 256 threads, down tables on the rest
+    const int half = blockDim.x / 2;
+    if ((int)threadIdx.x < half) {
+#pragma unroll 1
+        for (int i = threadIdx.x; i < ngt; i += half) S.gut[i] = make_gu_task(P, S, c + i * G, pg);
+    } else {
+#pragma unroll 1
+        for (int i = threadIdx.x - half; i < ndt; i += (int)blockDim.x - half) S.dnt[i] = make_dn_task(P, S, d0 + i, sp0);
     }
     __syncthreads();
-#pragma unroll 1
-    for (int i = threadIdx.x; i < S.ngt; i += blockDim.x) S.gut[i] = make_gu_task(P, S, c + i * G);
-#pragma unroll 1
-    for (int i = threadIdx.x; i < S.ndt; i += blockDim.x) S.dnt[i] = make_dn_task(P, S, d0 + i, sp0);
+    if (S.seg_rounds > 1 && (int)threadIdx.x < nseg) S.seg[threadIdx.x].off = 0;
     // the ring was written with generic stores above; order them before the
     // bulk copies (async proxy) that refill it next
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
 }
 
-// x' = bf16(rmsnorm_no_scale(h)) pre-scaled for the code decode, and its chunk
-// sums, in S.stage.  One warp per 32-column chunk, a lane per column.
-__device__ __noinline__ void stage_x(const Params &P, Smem &S) {
-    const int T = P.T, nch = P.H / 32, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    float *stage = S.stage;
-    const float pre = code_prescale(lane & 7);
+// Gate weights w = softmax(logits[top-k]) * per_expert_scale[top-k], in fp64;
+// selv[t*k] is token t's largest selected logit.  One warp, off the critical
+// path (they are first needed by the combine in the down phase).
+__device__ __noinline__ void gate_weights(const Params &P, Smem &S, const moe_layer_w &W) {
+    const int k = P.k, n = P.T * k;
 #pragma unroll 1
-    for (int i = wid; i < T * nch; i += kWarps) {
-        const int t = i / nch;
-        const float x = bf16_bits_to_float(f32_to_bf16_bits_alu(stage[(size_t)i * 32 + lane] * S.rinv[t]));
-        stage[(size_t)i * 32 + lane] = x * pre;
-        const float sx = warp_sum(x);
-        if (lane == 0) S.xs[i] = sx;
+    for (int p = threadIdx.x & 31; p < n; p += 32) {
+        const int t = p / k;
+        const double mx = S.selv[t * k];
+        double z = 0.0;
+#pragma unroll 1
+        for (int s2 = 0; s2 < k; ++s2) z += exp(S.selv[t * k + s2] - mx);
+        S.wts[p] = (float)(exp(S.selv[p] - mx) / z * (double)bf16_bits_to_float(W.per_expert_scale[S.idx[p]]));
+    }
+}
+
+// x' = bf16(rmsnorm_no_scale(h)) pre-scaled for the code decode, and its chunk
+// sums, in S.stage.  A thread per 4 columns; the 8 threads of a 32-column
+// chunk are adjacent lanes and sum it with three shuffles.
+__device__ __noinline__ void stage_x(const Params &P, Smem &S) {
+    const int T = P.T, H4 = P.H / 4, lane = threadIdx.x & 31;
+    const int n4 = T * H4, rounds = (n4 + (int)blockDim.x - 1) / (int)blockDim.x;
+#pragma unroll 1
+    for (int r = 0; r < rounds; ++r) {  // every thread runs every round: the shuffles need whole warps
+        const int i = r * blockDim.x + threadIdx.x;
+        float sx = 0.f;
+        if (i < n4) {
+            const int t = i / H4;
+            float4 v = reinterpret_cast<float4 *>(S.stage)[i];
+            const float ri = S.rinv[t];
+            const float x0 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.x * ri));
+            const float x1 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.y * ri));
+            const float x2 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.z * ri));
+            const float x3 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.w * ri));
+            const int c = (4 * i) & 7;  // 0 or 4
+            v.x = x0 * code_prescale(c);
+            v.y = x1 * code_prescale(c + 1);
+            v.z = x2 * code_prescale(c + 2);
+            v.w = x3 * code_prescale(c + 3);
+            reinterpret_cast<float4 *>(S.stage)[i] = v;
+            sx = (x0 + x1) + (x2 + x3);
+        }
+        sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 4);
+        if (i < n4 && (lane & 7) == 0) S.xs[i >> 3] = sx;
     }
     __syncthreads();
 }
@@ -934,7 +1027,11 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
                         us += __ldcg(&jp[((size_t)(pg + p2) * T + tt) * 32 + lane]);
                     }
                 }
-                P.act[(size_t)task_rowset(P, t, tt) * P.Kmax + t.rb * 32 + lane] = silu_mul(gs, us);
+                const float a = silu_mul(gs, us);
+                const size_t rs = (size_t)task_rowset(P, t, tt);
+                P.act[rs * P.Kmax + t.rb * 32 + lane] = a * code_prescale(lane & 7);
+                const float cs = warp_sum(a);  // the job's 32 rows are one 32-column chunk of the down input
+                if (lane == 0) P.act_cs[rs * (P.Kmax / 32) + t.rb] = cs;
             }
             __syncwarp();
             if (lane == 0) P.cnt_gu[t.job] = 0u;
@@ -943,52 +1040,29 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
     return ok;
 }
 
-// Chunk sums (sum of the unscaled values) of chunks [c0, c1) of the stage, bank-rotated.
-__device__ __noinline__ void chunk_sums(Smem &S, int c0, int c1) {
-    const float *stage = S.stage;
-#pragma unroll 1
-    for (int i = c0 + threadIdx.x; i < c1; i += kCWarps * 32) {
-        const float *row = stage + (size_t)i * 32;
-        float sx = 0.f;
-#pragma unroll 4
-        for (int mm = 0; mm < 32; ++mm) {
-            const int m = (mm + i) & 31;
-            sx = fmaf(row[m], code_unprescale(m & 7), sx);
-        }
-        S.xs[i] = sx;
-    }
-}
-
-// Stage the down inputs of segments [k0, k1): a pre-scaled for the code
-// decode, and the chunk sums.  Consumer threads only.
+// Stage the down inputs of segments [k0, k1): a (already pre-scaled for the
+// code decode) and its chunk sums.  Consumer threads only.
 __device__ __noinline__ void stage_segments(const Params &P, Smem &S, int k0, int k1) {
-    const int ctid = threadIdx.x;
+    const int ctid = threadIdx.x, KC = P.Kmax / 32;
 #pragma unroll 1
     for (int k2 = k0; k2 < k1; ++k2) {
         const SegDesc sg = S.seg[k2];
-        const int q4 = sg.ld / 4;
+        const int q4 = sg.ld / 4, nc = sg.ld / 32;
         const int rs0 = sg.slot == 0 ? 0 : P.T + sg.seg0;
 #pragma unroll 1
         for (int e = ctid; e < sg.n * q4; e += kCWarps * 32) {
             const int tt = e / q4, c4 = e - tt * q4;
-            const float4 a = __ldcg(reinterpret_cast<const float4 *>(P.act + (size_t)(rs0 + tt) * P.Kmax + sg.g0 * 64) + c4);
-            const int c = 4 * c4;
-            float4 v;
-            v.x = a.x * code_prescale(c & 7);
-            v.y = a.y * code_prescale((c + 1) & 7);
-            v.z = a.z * code_prescale((c + 2) & 7);
-            v.w = a.w * code_prescale((c + 3) & 7);
-            reinterpret_cast<float4 *>(S.stage + sg.off + (size_t)tt * sg.ld)[c4] = v;
+            reinterpret_cast<float4 *>(S.stage + sg.off + (size_t)tt * sg.ld)[c4] =
+                __ldcg(reinterpret_cast<const float4 *>(P.act + (size_t)(rs0 + tt) * P.Kmax + sg.g0 * 64) + c4);
+        }
+#pragma unroll 1
+        for (int e = ctid; e < sg.n * nc; e += kCWarps * 32) {
+            const int tt = e / nc, c = e - tt * nc;
+            S.xs[(sg.off + tt * sg.ld) / 32 + c] = __ldcg(&P.act_cs[(size_t)(rs0 + tt) * KC + sg.g0 * 2 + c]);
         }
     }
     consumer_sync();
-    if (k1 > k0) {
-        const SegDesc &a = S.seg[k0], &b = S.seg[k1 - 1];
-        chunk_sums(S, a.off / 32, (b.off + b.n * b.ld) / 32);
-    }
-    consumer_sync();
 }
-
 
 // The combine m[t][row] = sum_s w[t,s] * y[t,s] + shared, in a fixed order;
 // the loads of a batch are issued before any is used.
@@ -1136,8 +1210,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         // ---------------- gate/up tasks
         if (producer)
             task_producer(P, S, W, false, rq, l, issued);
-        else if (consumer)
+        else if (consumer) {
             P.T == 1 ? gu_consumer<1>(P, S, rq) : gu_consumer<kMaxT>(P, S, rq);
+            if (wid == kCWarps - 1) gate_weights(P, S, W);
+        }
         rq += (unsigned)S.ngt;
         ok = grid_sync(P, ++nbar, &S.flag);
         if (!ok) break;
@@ -1169,7 +1245,7 @@ static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exce
 static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
 
 struct DecodeWs {
-    size_t bar, cnt_dn, cnt_gu, logits, gpart, act, y, sh, m, total, zero_bytes;
+    size_t bar, cnt_dn, cnt_gu, logits, gpart, act, act_cs, y, sh, m, total, zero_bytes;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1196,6 +1272,7 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
     d.gpart = take(sizeof(float) * jobs * 2 * pg * T * 32);
     d.logits = take(sizeof(double) * (size_t)T * w->E);
     d.act = take(sizeof(float) * (size_t)R * Kmax);
+    d.act_cs = take(sizeof(float) * (size_t)R * (Kmax / 32));
     d.y = take(sizeof(float) * (size_t)ndp_r * T * w->k * w->H);
     d.sh = take(sizeof(float) * (size_t)ndp_s * T * w->H);
     d.m = take(sizeof(float) * (size_t)T * w->H);
@@ -1277,6 +1354,7 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.cnt_gu = reinterpret_cast<unsigned *>(base + d.cnt_gu);
     P.gpart = reinterpret_cast<float *>(base + d.gpart);
     P.act = reinterpret_cast<float *>(base + d.act);
+    P.act_cs = reinterpret_cast<float *>(base + d.act_cs);
     P.y = reinterpret_cast<float *>(base + d.y);
     P.sh = reinterpret_cast<float *>(base + d.sh);
     P.m = reinterpret_cast<float *>(base + d.m);

@@ -15,9 +15,12 @@
 // (the MMA's M) by the n <= 128 tokens of one expert (the MMA's N, padded to a
 // multiple of 16), over the whole input dimension in k-blocks of 64 (one
 // quantisation group, one 128-byte swizzle row of FP16):
-//   producer thread  bulk-copies the tiled 4-bit codes and (scale, bias) words
-//                    of the tile into a ring, and loads the tokens' FP16 rows
-//                    with TMA tensor copies (128-byte swizzle);
+//   weight producer  loads the tiled 4-bit codes and (scale, bias) words of
+//                    the tile into a ring with 3-D TMA tensor copies (one box
+//                    of 4 row blocks x a code stage per matrix);
+//   token producer   loads the tokens' FP16 rows with 2-D TMA tensor copies
+//                    (128-byte swizzle), in a warp of its own so that neither
+//                    producer waits behind the other;
 //   8 dequant warps  turn each k-block of codes into FP16 weights
 //                    w = s*q + b (exact q, one rounding) in the swizzled
 //                    K-major layout the tensor core reads;
@@ -69,9 +72,10 @@ constexpr int kBBufs = 3;         // token slots of 16 KiB: 128 / N k-blocks of 
 constexpr int kMaxN = 128;        // tokens per tile
 constexpr int kBoxRows = 16;      // rows of one TMA box of the token matrix
 constexpr int kDqWarps = 16;      // dequant (and epilogue) warps: one 32-code record per thread per stage
-constexpr int kProdWarp = 16;
+constexpr int kProdWarp = 16;   // weight codes
 constexpr int kMmaWarp = 17;
-constexpr int kThreads = 18 * 32;
+constexpr int kTokWarp = 18;    // token tiles
+constexpr int kThreads = 19 * 32;
 constexpr int kTmemCols = 256;
 constexpr int kATileBytes = kBM * kBK * 2;       // 16 KiB
 constexpr int kBBufBytes = kMaxN * kBK * 2;      // 16 KiB
@@ -117,6 +121,14 @@ struct Params {
     float *sh;  // down output, shared: [T, H]
     int H;
     int *err;
+};
+
+// TMA tensor maps of one launch: the token matrix (B operand) and the tiled
+// codes / (scale, bias) words of the routed matrices (q, sb) and of the
+// shared expert's (sq, ssb), each viewed as [row blocks][chunks or groups][32 lanes x words].
+struct Maps {
+    CUtensorMap tok;
+    CUtensorMap q[2], sb[2], sq[2], ssb[2];
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -180,6 +192,15 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
+}
+
+// 3-D tiled TMA load (no multicast): box at (x, y, z) of the tensor map.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
 }
 
 // 2-D tiled TMA load (no multicast): box at (x = column, y = row) of the tensor map.
@@ -330,7 +351,8 @@ __device__ __forceinline__ bool get_tile(const Params &P, int it, Tile &t) {
 
 template <int NMAT>
 __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_constant__ Params P,
-                                                                 const __grid_constant__ CUtensorMap tmB) {
+                                                                 const __grid_constant__ Maps M) {
+    const CUtensorMap &tmB = M.tok;
     using L = Lay<NMAT>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -379,61 +401,63 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kProdWarp) {
-        // ---------------------------------------------------------- producer
+        // ---------------------------------------------------------- weight producer
         if (lane == 0) {
-            uint32_t cs = 0, kbc = 0;
+            uint32_t cs = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
                 Tile t;
                 if (!get_tile(P, it, t)) continue;
-                const int C = t.K / 32, G = t.K / 64, nkb = t.K / kBK, nrb = t.rv / 32;
-                const uint32_t *qb[NMAT], *sbb[NMAT];
+                const int nkb = t.K / kBK;
+                const int mrb0 = (t.e < 0 ? 0 : t.e * (P.rows_r / 32)) + t.mt * 4;  // first row block of the tile
+                for (int kb = 0; kb < nkb; kb += kKS) {
+                    const int s = cs % kCodeSlots;
+                    if (cs >= kCodeSlots &&
+                        !mbar_wait(code_empty(s), ((cs / kCodeSlots) & 1) ^ 1, P.err, kErrCodeEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    // whole boxes always land (out-of-range rows and chunks are zero-filled)
+                    mbar_expect_tx(code_full(s), (unsigned)L::kSlotBytes);
+                    const uint32_t slot = sC + (uint32_t)s * L::kSlotBytes;
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m) {
-                    const size_t mrb = (t.e < 0 ? (size_t)0 : (size_t)t.e * (P.rows_r / 32)) + (size_t)t.mt * 4;
-                    qb[m] = (t.e < 0 ? P.sq[m] : P.q[m]) + mrb * C * 128;
-                    sbb[m] = (t.e < 0 ? P.ssb[m] : P.sb[m]) + mrb * G * 32;
-                }
-                const int nbox = t.N / kBoxRows, bkb = kMaxN / t.N;  // k-blocks per token slot
-                for (int kb = 0; kb < nkb && ok; ++kb) {
-                    if (kb % kKS == 0) {
-                        const int s = cs % kCodeSlots;
-                        if (cs >= kCodeSlots &&
-                            !mbar_wait(code_empty(s), ((cs / kCodeSlots) & 1) ^ 1, P.err, kErrCodeEmpty)) {
-                            ok = false;
-                            break;
-                        }
-                        const int nk = min(kKS, nkb - kb);
-                        mbar_expect_tx(code_full(s), (unsigned)(NMAT * nrb * nk * (1024 + 128)));
-                        const uint32_t slot = sC + (uint32_t)s * L::kSlotBytes;
-                        for (int m = 0; m < NMAT; ++m)
-                            for (int rbl = 0; rbl < nrb; ++rbl) {
-                                bulk_g2s(slot + (uint32_t)((m * 4 + rbl) * kKS) * 1024u,
-                                         qb[m] + ((size_t)rbl * C + 2 * kb) * 128, (unsigned)nk * 1024u, code_full(s));
-                                bulk_g2s(slot + L::kCodeBytes + (uint32_t)((m * 4 + rbl) * kKS) * 128u,
-                                         sbb[m] + ((size_t)rbl * G + kb) * 32, (unsigned)nk * 128u, code_full(s));
-                            }
-                        ++cs;
+                    for (int m = 0; m < NMAT; ++m) {
+                        tma_load_3d(slot + (uint32_t)(m * 4 * kKS) * 1024u, t.e < 0 ? &M.sq[m] : &M.q[m], 0, 2 * kb,
+                                    mrb0, code_full(s));
+                        tma_load_3d(slot + L::kCodeBytes + (uint32_t)(m * 4 * kKS) * 128u, t.e < 0 ? &M.ssb[m] : &M.sb[m],
+                                    0, kb, mrb0, code_full(s));
                     }
-                    if (kb % bkb == 0) {  // a new token slot: this and the next bkb - 1 k-blocks
-                        const int b = kbc % kBBufs;
-                        if (kbc >= kBBufs && !mbar_wait(b_empty(b), ((kbc / kBBufs) & 1) ^ 1, P.err, kErrBEmpty)) {
-                            ok = false;
-                            break;
-                        }
-                        const int nk = min(bkb, nkb - kb);
-                        mbar_expect_tx(b_full(b), (unsigned)(nk * nbox * kBoxBytes));
-                        for (int i = 0; i < nk; ++i)
-                            for (int j = 0; j < nbox; ++j)
-                                tma_load_2d(sB + (uint32_t)b * kBBufBytes + (uint32_t)((i * nbox + j) * kBoxBytes), &tmB,
-                                            (kb + i) * kBK, t.brow + j * kBoxRows, b_full(b));
-                        ++kbc;
-                    }
+                    ++cs;
                 }
             }
-            // let this CTA's own copies land before it stops (bounded)
+            // let this lane's copies land before the CTA stops (bounded)
             for (uint32_t c = cs > (uint32_t)kCodeSlots ? cs - kCodeSlots : 0u; c < cs; ++c)
                 mbar_drain(code_full(c % kCodeSlots), (c / kCodeSlots) & 1);
+        }
+    } else if (warp == kTokWarp) {
+        // ---------------------------------------------------------- token producer
+        if (lane == 0) {
+            uint32_t kbc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
+                Tile t;
+                if (!get_tile(P, it, t)) continue;
+                const int nkb = t.K / kBK, nbox = t.N / kBoxRows, bkb = kMaxN / t.N;  // k-blocks per token slot
+                for (int kb = 0; kb < nkb; kb += bkb) {
+                    const int b = kbc % kBBufs;
+                    if (kbc >= kBBufs && !mbar_wait(b_empty(b), ((kbc / kBBufs) & 1) ^ 1, P.err, kErrBEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    const int nk = min(bkb, nkb - kb);
+                    mbar_expect_tx(b_full(b), (unsigned)(nk * nbox * kBoxBytes));
+                    for (int i = 0; i < nk; ++i)
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(sB + (uint32_t)b * kBBufBytes + (uint32_t)((i * nbox + j) * kBoxBytes), &tmB,
+                                        (kb + i) * kBK, t.brow + j * kBoxRows, b_full(b));
+                    ++kbc;
+                }
+            }
             for (uint32_t c = kbc > (uint32_t)kBBufs ? kbc - kBBufs : 0u; c < kbc; ++c)
                 mbar_drain(b_full(c % kBBufs), (c / kBBufs) & 1);
         }
@@ -659,6 +683,33 @@ static cudaError_t make_map(CUtensorMap *m, const uint16_t *ptr, int rows, int c
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Tiled codes [n_rb][C][128 u32] or (scale, bias) words [n_rb][G][32 u32] of a
+// matrix set, boxes of 4 row blocks x `per` chunks (or groups) x all lanes.
+static cudaError_t make_qmap(CUtensorMap *m, const uint32_t *ptr, int n_rb, int per_rb, int words, int per) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)words, (cuuint64_t)per_rb, (cuuint64_t)n_rb};
+    const cuuint64_t strides[2] = {(cuuint64_t)words * 4, (cuuint64_t)words * 4 * per_rb};
+    const cuuint32_t box[3] = {(cuuint32_t)words, (cuuint32_t)per, 4};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Maps of the routed matrices q/sb[0..nmat) ([n_mat][rows][K] each) and of the shared ones ([rows_s][K_s]).
+static cudaError_t make_weight_maps(Maps &M, const Params &P, int nmat, int n_mat) {
+    for (int m = 0; m < nmat; ++m) {
+        cudaError_t e = make_qmap(&M.q[m], P.q[m], n_mat * P.rows_r / 32, P.K_r / 32, 128, 2 * kKS);
+        if (e == cudaSuccess) e = make_qmap(&M.sb[m], P.sb[m], n_mat * P.rows_r / 32, P.K_r / 64, 32, kKS);
+        if (e == cudaSuccess && P.with_shared) e = make_qmap(&M.sq[m], P.sq[m], P.rows_s / 32, P.K_s / 32, 128, 2 * kKS);
+        if (e == cudaSuccess && P.with_shared) e = make_qmap(&M.ssb[m], P.ssb[m], P.rows_s / 32, P.K_s / 64, 32, kKS);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 static int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -667,7 +718,7 @@ static int sm_count() {
 }
 
 template <int NMAT>
-static cudaError_t launch_mma(Params &P, const CUtensorMap &map, int max_items, cudaStream_t st) {
+static cudaError_t launch_mma(Params &P, const Maps &map, int max_items, cudaStream_t st) {
     using Lt = Lay<NMAT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(expert_mma_kernel<NMAT>), Lt::kAlloc);
     if (e != cudaSuccess) return e;
@@ -705,10 +756,10 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    CUtensorMap mx, ma;
-    cudaError_t e = make_map(&mx, b.xg, R, H, H);
+    static thread_local Maps mx, ma;  // large; kept off the stack
+    cudaError_t e = make_map(&mx.tok, b.xg, R, H, H);
     if (e != cudaSuccess) return e;
-    e = make_map(&ma, b.act, R, Kmax, Kmax);
+    e = make_map(&ma.tok, b.act, R, Kmax, Kmax);
     if (e != cudaSuccess) return e;
 
     Params P{};
@@ -744,6 +795,8 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
     {
         const int mt_s = (Is + kBM - 1) / kBM, mt_r = (I + kBM - 1) / kBM;
         const int items = (with_shared ? mt_s * P.nt_max : 0) + max_active * P.nt_max * mt_r;
+        e = make_weight_maps(mx, P, 2, w->E);
+        if (e != cudaSuccess) return e;
         e = launch_mma<2>(P, mx, items, st);
         if (e != cudaSuccess) return e;
     }
@@ -763,6 +816,8 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
     {
         const int mt = (H + kBM - 1) / kBM;
         const int items = (with_shared ? mt * P.nt_max : 0) + max_active * P.nt_max * mt;
+        e = make_weight_maps(ma, P, 1, w->E);
+        if (e != cudaSuccess) return e;
         e = launch_mma<1>(P, ma, items, st);
     }
     return e;
