@@ -44,6 +44,14 @@ def peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu
+# capture, per unit of work: decode_stack_kernel at the Gemma shape, T = 1,
+# per layer (2-layer capture halved); the two grouped-GEMM kernels of one
+# 128-token layer-chunk.  Reset to None whenever the kernel changes.
+DECODE_TRAFFIC_PER_LAYER = (74_528_768 + 1_682_688) / 2
+PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_850_432 + 6_467_072 + 147_067_136 + 9_365_248
+
+
 def expert_bytes(rows_cols: int) -> float:
     """Algorithmic bytes of an int4 matrix with rows*cols weights: 4 bits per
     code + a bf16 scale and a bf16 bias per 64 codes = 4.5 bits per weight."""
@@ -182,7 +190,9 @@ def run_ours(args, rank, world, local_rank):
         roof = {"kernel": "decode_stack_kernel (persistent: all layers of a step in one cooperative launch)",
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / hbm["hbm_gbs"], 4), "peak_source": hbm["source"] + " (burst copy)",
-                "traffic": None, "bytes_per_launch": int(step_bytes), "us_per_launch": round(ms_per_step * 1e3, 2)}
+                "traffic": (int(DECODE_TRAFFIC_PER_LAYER * st.L)
+                            if DECODE_TRAFFIC_PER_LAYER and args.config == 1 and T == 1 else None),
+                "bytes_per_launch": int(step_bytes), "us_per_launch": round(ms_per_step * 1e3, 2)}
     else:
         roof = _expert_roofline(st, moe, cfg, T, hbm, dev)
 
@@ -196,11 +206,17 @@ def run_ours(args, rank, world, local_rank):
         cpu = cpu_baseline(cfg, args.config, T, budget_s=args.cpu_budget)
 
     launches_per_step = st.launches_per_step()
+    n_layers = st.L
+    prefill = None
+    if args.prefill and world == 1 and args.config == 1 and not args.layers:
+        del st
+        torch.cuda.empty_cache()
+        prefill = prefill_measure(dev)
     res = {
         "metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 weights, bf16 activations, fp32 accumulate (router fp64)", "data": "synthetic",
-        "config": {"workload": workload_name(cfg, T), "config_id": args.config, "layers": st.L, "tokens_per_step": T,
+        "config": {"workload": workload_name(cfg, T), "config_id": args.config, "layers": n_layers, "tokens_per_step": T,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (13.2 GB of weights, 1.1 GB touched per step)"},
         "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm["hbm_gbs"], 4),
@@ -208,6 +224,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
+    if prefill is not None:
+        res["prefill"] = prefill
     return res
 
 
@@ -264,6 +282,51 @@ def _expert_roofline(st, moe, cfg, T, hbm, dev):
             "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / hbm["hbm_gbs"], 4), "peak_source": hbm["source"] + " (burst copy)",
             "traffic": None, "bytes_per_launch": int(nbytes), "us_per_launch": round(us, 3)}
+
+
+def expert_flops(cfg, T: int) -> float:
+    """Multiply-adds x 2 of the expert FFNs for T tokens: every token through
+    k routed experts and the shared expert, three matrices each."""
+    return 2.0 * T * (3.0 * cfg.I * cfg.H * cfg.k + 3.0 * cfg.Is * cfg.H)
+
+
+def prefill_measure(dev, chunks=8, layers=None):
+    """Chunked prefill at the Gemma shape: `chunks` chunks of 128 tokens, each
+    through every layer (chained), chunk after chunk; plus the per-launch
+    expert FFN (tensor-core grouped GEMM) against the tensor and HBM peaks."""
+    from int4_routed_expert_02_b200 import moe
+    from int4_routed_expert_02_b200.stack import MoEStack
+    cfg = synth.CONFIGS[4]
+    T = cfg.T
+    st = MoEStack(cfg, 4, T=T, layers=layers, device=dev)
+    inputs = [synth.gen_hidden(cfg, 4, 20_000 + c, T, device=dev) for c in range(chunks + 1)]
+    stream = torch.cuda.current_stream(dev)
+    st.set_input(inputs[0])
+    st.run()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for c in range(chunks):
+        st.set_input(inputs[1 + c])
+        st.run()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    st.status()
+    hbm = peaks()
+    roof = _expert_roofline(st, moe, cfg, T, hbm, dev)
+    fl = expert_flops(cfg, T)
+    tflops = fl / (roof["us_per_launch"] / 1e6) / 1e12
+    peak_t = hbm["bf16_tflops"]  # FP16 and BF16 share the dense tensor rate
+    return {"workload": workload_name(cfg, T) + f", {chunks} chunks chunk-major", "tok_s": round(chunks * T / (ms / 1e3), 1),
+            "ms_per_chunk": round(ms / chunks, 4),
+            "expert_ffn": {"kernel": "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
+                           "us_per_launch": roof["us_per_launch"], "flops_per_launch": fl,
+                           "tflops": round(tflops, 2), "tensor_peak_tflops": peak_t,
+                           "tensor_frac": round(tflops / peak_t, 4), "hbm_gbs": roof["achieved"],
+                           "hbm_frac": roof["frac"], "bytes_per_launch": roof["bytes_per_launch"],
+                           "traffic": PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK,
+                           "peak_source": hbm["source"] + " (bf16 dense burst; FP16 same rate; copy bandwidth)"}}
 
 
 def _e2e(st, cfg, T, K, W, inputs, dev):
@@ -388,6 +451,8 @@ def main():
                     help="profiling only: build this many layers instead of the config's (not a bench line)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", dest="prefill", action="store_false",
+                    help="skip the chunked-prefill measurement that the default line carries")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
