@@ -47,6 +47,8 @@
 // Every wait is bounded (grid barrier and mbarriers: ~1 s of globaltimer); on
 // a timeout the kernel records an error code in the workspace, stops taking
 // work, lets its own bulk copies land and returns.
+#include <cstdlib>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -86,6 +88,7 @@ struct Params {
     int nslots;      // ring slots (the rest of the pool is the input stage)
     int stage_floats;  // floats in the input stage
     unsigned *bar;
+    unsigned bar_extra;  // arrivals the grid barrier waits for beyond the grid (0; tests of the timeout path set 1)
     int *err;
     unsigned *cnt_dn;  // [H/32]: down tasks done per row block; reset by the last
     unsigned *cnt_gu;  // [jobs]: gate/up tasks done per job; reset by the last
@@ -235,7 +238,7 @@ __device__ __noinline__ bool grid_sync(const Params &P, unsigned nth, int *verdi
     if (threadIdx.x == 0) {
         __threadfence();
         atomicAdd(P.bar, 1u);
-        const unsigned target = nth * gridDim.x;
+        const unsigned target = nth * gridDim.x + P.bar_extra;
         const unsigned long long t0 = globaltimer();
         for (unsigned it = 0;; ++it) {
             unsigned v;
@@ -1348,6 +1351,11 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     if (!decode_layout(w, T, grid, &P.nslots, &P.stage_floats)) return cudaErrorInvalidValue;
     char *base = static_cast<char *>(ws);
     P.bar = reinterpret_cast<unsigned *>(base + d.bar);
+    // test hook: MOE_TEST_BARRIER_EXTRA=1 makes the first grid barrier wait for an
+    // arrival that never comes, so that its bounded wait runs out (about 1 s) and
+    // the kernel reports "grid barrier timed out" through the workspace status
+    const char *extra = getenv("MOE_TEST_BARRIER_EXTRA");
+    P.bar_extra = (extra && extra[0] == '1') ? 1u : 0u;
     P.err = reinterpret_cast<int *>(base + d.bar + sizeof(unsigned));
     P.logits = reinterpret_cast<double *>(base + d.logits);
     P.cnt_dn = reinterpret_cast<unsigned *>(base + d.cnt_dn);

@@ -86,3 +86,23 @@ def test_decode_stack_is_deterministic_and_rejects_bad_sizes():
     assert moe.moe_decode_stack_workspace_size(st.layers[0], 9) == 0
     with pytest.raises(moe.MoEError):
         moe.moe_decode_stack(st.larr, 2, st.buf[0], 1, st.h_out, 9, st.ws_dec)
+
+
+def test_barrier_timeout_is_reported_and_the_context_survives(monkeypatch):
+    """The grid barrier's bounded wait runs out (a test hook makes it wait for
+    one arrival more than the grid has): the kernel records the code, every CTA
+    returns, the status call reports MOE_EDEVICE, and the next call is fine."""
+    cfg = synth.CONFIGS[0]
+    st = MoEStack(cfg, 0, T=1, layers=1)
+    st.set_input(synth.gen_hidden(cfg, 0, 3, 1).cuda())
+    monkeypatch.setenv("MOE_TEST_BARRIER_EXTRA", "1")
+    st.run()
+    torch.cuda.synchronize()
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_decode_stack_status(st.ws_dec)
+    assert ei.value.code == moe.MOE_EDEVICE and "grid barrier timed out" in str(ei.value)
+    monkeypatch.delenv("MOE_TEST_BARRIER_EXTRA")
+    st.run()
+    torch.cuda.synchronize()
+    moe.moe_decode_stack_status(st.ws_dec)
+    assert torch.isfinite(st.final_output().float()).all()
