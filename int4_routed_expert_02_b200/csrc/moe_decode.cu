@@ -21,14 +21,18 @@
 //       round-robin to the CTAs and taken by their warps independently; each
 //       task's partial sums go to global memory, and the warp that finishes a
 //       job's last task (an atomic count per job) sums the parts in a fixed
-//       order and forms a = silu(g) * u for the job's rows
-//   --- grid barrier ---
+//       order and forms a = silu(g) * u for the job's rows, then counts the
+//       job done for its slot
+//   (no grid barrier: a CTA stages a slot's input once all of that slot's
+//   jobs are counted)
 //   P3  down: tasks of 32 rows x <= 16 groups of one slot, in contiguous
 //       blocks per CTA so that a CTA stages each slot's a once; a warp
 //       writes its task's rows, and the warp that finishes the last task of
 //       a row block (an atomic count per row block) forms the combine
-//       m = sum_s w_s y_s + shared for those rows
-//   --- grid barrier ---
+//       m = sum_s w_s y_s + shared for those rows, then counts the row block
+//       done
+//   (no grid barrier: the next layer's P0 waits until every row block of m
+//   is counted)
 //
 // Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
 // into a ring of mbarrier-guarded slots, one slot per task, issued by one
@@ -75,7 +79,7 @@ constexpr int kMaxPG = 4;                     // gate/up parts per job (H <= 409
 constexpr int kMaxSegs = 16;                  // down: staged (slot, part) inputs per CTA
 constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
 
-constexpr int kErrGridBarrier = 1, kErrFull = 2, kErrEmpty = 3;
+constexpr int kErrGridBarrier = 1, kErrFull = 2, kErrEmpty = 3, kErrReady = 4;
 
 struct Params {
     moe_layer_w layers[kMaxLayers];
@@ -92,6 +96,8 @@ struct Params {
     int *err;
     unsigned *cnt_dn;  // [H/32]: down tasks done per row block; reset by the last
     unsigned *cnt_gu;  // [jobs]: gate/up tasks done per job; reset by the last
+    unsigned *act_done;   // [1 + T*k]: gate/up jobs done per slot, over all layers so far
+    unsigned *rows_done;  // row blocks of m combined, over all layers so far
     float *gpart;      // [jobs][2][pg][T][32]: gate/up partial sums per task
     double *logits;  // [T,E]
     float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs),
@@ -130,6 +136,7 @@ struct Smem {
     TaskDesc gut[kMaxTasks], dnt[kMaxTasks];
     SegDesc seg[kMaxSegs];
     int ngt, ndt, pg, nseg, seg_rounds;
+    unsigned act_expect[kMaxPairs + 1];  // act_done per slot once this layer's gate/up jobs are all done
     double selv[kMaxPairs];
     float wts[kMaxPairs];
     int idx[kMaxPairs];
@@ -145,6 +152,7 @@ struct Smem {
     float rinv[kMaxT];
     int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
     int flag;
+    int flag2;  // consumer-only verdicts
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -745,6 +753,8 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     }
     if (threadIdx.x < T) S.tokrow_sh[threadIdx.x] = threadIdx.x * H;
     __syncthreads();
+    // this layer's gate/up jobs per slot: the shared expert's Is/32, each active slot's I/32
+    if ((int)threadIdx.x <= S.nact) S.act_expect[threadIdx.x] += threadIdx.x == 0 ? P.Is / 32 : P.I / 32;
     // task tables of this CTA.  Gate/up jobs are dealt round-robin (every CTA
     // mixes shared-expert jobs with routed ones); down tasks go in contiguous
     // blocks, so that a CTA's tasks share few (slot, part) inputs.
@@ -978,6 +988,25 @@ __device__ __forceinline__ unsigned atom_add_release_gpu(unsigned *p, unsigned v
     return old;
 }
 
+// Bounded wait of one thread until a global count reaches `target` (acquire);
+// false (with an error recorded) on a timeout or another CTA's error.
+__device__ __noinline__ bool wait_count(const Params &P, const unsigned *ctr, unsigned target) {
+    const unsigned long long t0 = globaltimer();
+    for (unsigned it = 0;; ++it) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        if ((it & 63u) == 63u) {
+            if (ldcg_int(P.err) != 0) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                atomicCAS(P.err, 0, kErrReady);
+                return false;
+            }
+        }
+        __nanosleep(32);
+    }
+}
+
 template <int NT>
 __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -1037,7 +1066,10 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
                 if (lane == 0) P.act_cs[rs * (P.Kmax / 32) + t.rb] = cs;
             }
             __syncwarp();
-            if (lane == 0) P.cnt_gu[t.job] = 0u;
+            if (lane == 0) {
+                P.cnt_gu[t.job] = 0u;
+                atom_add_release_gpu(&P.act_done[t.slot], 1u);  // the job's rows of a are written
+            }
         }
     }
     return ok;
@@ -1045,8 +1077,19 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
 
 // Stage the down inputs of segments [k0, k1): a (already pre-scaled for the
 // code decode) and its chunk sums.  Consumer threads only.
-__device__ __noinline__ void stage_segments(const Params &P, Smem &S, int k0, int k1) {
+__device__ __noinline__ bool stage_segments(const Params &P, Smem &S, int k0, int k1) {
     const int ctid = threadIdx.x, KC = P.Kmax / 32;
+    // every consumer warp is past its gate/up tasks (the stage still held their
+    // input); then wait until each staged slot's SwiGLU rows are all written
+    consumer_sync();
+    if (ctid == 0) {
+        bool ok = true;
+        for (int k2 = k0; k2 < k1 && ok; ++k2) ok = wait_count(P, &P.act_done[S.seg[k2].slot], S.act_expect[S.seg[k2].slot]);
+        __threadfence();
+        S.flag2 = ok;
+    }
+    consumer_sync();
+    if (!S.flag2) return false;
 #pragma unroll 1
     for (int k2 = k0; k2 < k1; ++k2) {
         const SegDesc sg = S.seg[k2];
@@ -1065,6 +1108,7 @@ __device__ __noinline__ void stage_segments(const Params &P, Smem &S, int k0, in
         }
     }
     consumer_sync();
+    return true;
 }
 
 // The combine m[t][row] = sum_s w[t,s] * y[t,s] + shared, in a fixed order;
@@ -1112,7 +1156,7 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) 
 #pragma unroll 1
     for (int r = 0; r < rounds; ++r) {
         const int k0 = rounds == 1 ? 0 : r, k1 = rounds == 1 ? S.nseg : r + 1;
-        stage_segments(P, S, k0, k1);
+        if (!stage_segments(P, S, k0, k1)) return false;
 #pragma unroll 1
         for (int i = wid; i < nt; i += kCWarps) {
             const TaskDesc t = S.dnt[i];
@@ -1156,12 +1200,27 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) 
                 __syncwarp();
                 combine_row(P, S, row);
                 __syncwarp();
-                if (lane == 0) P.cnt_dn[t.rb] = 0u;
+                if (lane == 0) {
+                    P.cnt_dn[t.rb] = 0u;
+                    atom_add_release_gpu(P.rows_done, 1u);  // these 32 rows of m are written
+                }
             }
         }
         if (rounds > 1) consumer_sync();
     }
     return ok;
+}
+
+// All threads: wait until `target` row blocks of m are combined (over all layers so far).
+__device__ __noinline__ bool wait_rows(const Params &P, Smem &S, unsigned target) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const bool ok = wait_count(P, P.rows_done, target);
+        __threadfence();
+        S.flag = ok && ldcg_int(P.err) == 0;
+    }
+    __syncthreads();
+    return S.flag != 0;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -1180,6 +1239,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         }
         mbar_init(&S.rbar, 1);
         for (int s = 0; s < kMaxStages; ++s) S.slot_task[s] = 0xffffffffu;
+        for (int s = 0; s <= kMaxPairs; ++s) S.act_expect[s] = 0u;
         S.stage = reinterpret_cast<float *>(S.pool + (size_t)P.nslots * kSlotBytes);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1201,6 +1261,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         if (l == 0) {
             load_input(P, S, P.h_in);
         } else {
+            // every row block of the previous layer's m is combined
+            ok = wait_rows(P, S, (unsigned)l * (unsigned)(P.H / 32));
+            if (!ok) break;
             finish_layer(P, S, l - 1);
             if (!P.chained) load_input(P, S, P.h_in + (size_t)l * P.T * P.H);
         }
@@ -1218,17 +1281,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
             if (wid == kCWarps - 1) gate_weights(P, S, W);
         }
         rq += (unsigned)S.ngt;
-        ok = grid_sync(P, ++nbar, &S.flag);
-        if (!ok) break;
 
-        // ---------------- down tasks
+        // ---------------- down tasks (each CTA as soon as its own gate/up tasks are done)
         if (producer)
             task_producer(P, S, W, true, rq, l, issued);
         else if (consumer)
             P.T == 1 ? dn_consumer<1>(P, S, rq) : dn_consumer<kMaxT>(P, S, rq);
         rq += (unsigned)S.ndt;
-        ok = grid_sync(P, ++nbar, &S.flag);
+        __syncthreads();
+        if (threadIdx.x == 0) S.flag = ldcg_int(P.err) == 0;
+        __syncthreads();
+        ok = S.flag != 0;
     }
+    if (ok) ok = wait_rows(P, S, (unsigned)P.L * (unsigned)(P.H / 32));
     if (ok) finish_layer(P, S, P.L - 1);  // ok is uniform across the CTA here
 
     // let this CTA's own bulk copies land before it exits (bounded)
@@ -1248,7 +1313,7 @@ static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exce
 static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
 
 struct DecodeWs {
-    size_t bar, cnt_dn, cnt_gu, logits, gpart, act, act_cs, y, sh, m, total, zero_bytes;
+    size_t bar, cnt_dn, cnt_gu, act_done, logits, gpart, act, act_cs, y, sh, m, total, zero_bytes;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1271,6 +1336,7 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
     const size_t pg = (w->H / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
     d.cnt_dn = take(sizeof(unsigned) * (size_t)(w->H / 32));
     d.cnt_gu = take(sizeof(unsigned) * jobs);
+    d.act_done = take(sizeof(unsigned) * (R + 1));  // per slot, then rows_done
     d.zero_bytes = off;
     d.gpart = take(sizeof(float) * jobs * 2 * pg * T * 32);
     d.logits = take(sizeof(double) * (size_t)T * w->E);
@@ -1360,6 +1426,8 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.logits = reinterpret_cast<double *>(base + d.logits);
     P.cnt_dn = reinterpret_cast<unsigned *>(base + d.cnt_dn);
     P.cnt_gu = reinterpret_cast<unsigned *>(base + d.cnt_gu);
+    P.act_done = reinterpret_cast<unsigned *>(base + d.act_done);
+    P.rows_done = P.act_done + (T + T * w.k);
     P.gpart = reinterpret_cast<float *>(base + d.gpart);
     P.act = reinterpret_cast<float *>(base + d.act);
     P.act_cs = reinterpret_cast<float *>(base + d.act_cs);
