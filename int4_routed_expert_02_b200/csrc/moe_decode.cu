@@ -18,17 +18,18 @@
 //       and this CTA's job tables for the two expert phases
 //   P2' gate/up: a job (32 rows: a row block of one slot) is split into
 //       tasks of <= 16 quantisation groups of one matrix; tasks are dealt
-//       round-robin to the CTAs and taken by their warps independently; each
-//       task's partial sums go to global memory, and the warp that finishes a
-//       job's last task (an atomic count per job) sums the parts in a fixed
-//       order and forms a = silu(g) * u for the job's rows, then counts the
-//       job done for its slot
+//       round-robin to the CTAs and taken by teams of kWPT warps (every
+//       kWPT-th group each) independently; each warp's partial sums go to
+//       global memory, and the warp that
+//       finishes a job's last share (an atomic count per job) sums the parts
+//       in a fixed order and forms a = silu(g) * u for the job's rows, then
+//       counts the job done for its slot
 //   (no grid barrier: a CTA stages a slot's input once all of that slot's
 //   jobs are counted)
 //   P3  down: tasks of 32 rows x <= 16 groups of one slot, in contiguous
-//       blocks per CTA so that a CTA stages each slot's a once; a warp
-//       writes its task's rows, and the warp that finishes the last task of
-//       a row block (an atomic count per row block) forms the combine
+//       blocks per CTA so that a CTA stages each slot's a once; each warp of
+//       a task's team writes its partial rows, and the warp that finishes the
+//       last share of a row block (an atomic count per row block) forms the combine
 //       m = sum_s w_s y_s + shared for those rows, then counts the row block
 //       done
 //   (no grid barrier: the next layer's P0 waits until every row block of m
@@ -36,8 +37,8 @@
 //
 // Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
 // into a ring of mbarrier-guarded slots, one slot per task, issued by one
-// producer thread ahead of 16 consumer warps that never wait for one another
-// inside a phase.  The down tasks' weights do not depend on the gate/up
+// producer thread ahead of 15 consumer warps (teams of kWPT = 1) that never
+// wait for one another inside a phase.  The down tasks' weights do not depend on the gate/up
 // results, so the producer already fills the slots freed during the gate/up
 // phase with them.  Once the top-k is known each CTA also asks L2 to
 // prefetch the down-projection weights of its later jobs, and during the down
@@ -59,7 +60,10 @@
 namespace moe {
 namespace dec {
 
-constexpr int kCWarps = 16;                   // consumer warps
+constexpr int kCWarps = 15;                   // consumer warps: with the producer 16 warps, 4 per SM sub-partition,
+                                              // so a thread may hold 128 registers (no spills)
+constexpr int kWPT = 1;                       // consumer warps per task (a team; more than one measured slower)
+constexpr int kTeams = kCWarps / kWPT;
 constexpr int kWarps = kCWarps + 1;           // + the producer warp
 constexpr int kThreads = kWarps * 32;
 constexpr int kProducerWarp = kCWarps;
@@ -81,8 +85,10 @@ constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
 
 constexpr int kErrGridBarrier = 1, kErrFull = 2, kErrEmpty = 3, kErrReady = 4;
 
-struct Params {
-    moe_layer_w layers[kMaxLayers];
+// Sizes, options and workspace pointers of a launch.  The kernel copies them
+// into shared memory once, so that every phase reads them at shared-memory
+// latency instead of through the kernel-parameter space.
+struct Cfg {
     const uint16_t *h_in;  // [T,H] (chained) or [L,T,H]
     uint16_t *h_out;       // [L,T,H]: every layer's output
     int L, T, chained, post_norm;
@@ -98,14 +104,19 @@ struct Params {
     unsigned *cnt_gu;  // [jobs]: gate/up tasks done per job; reset by the last
     unsigned *act_done;   // [1 + T*k]: gate/up jobs done per slot, over all layers so far
     unsigned *rows_done;  // row blocks of m combined, over all layers so far
-    float *gpart;      // [jobs][2][pg][T][32]: gate/up partial sums per task
+    float *gpart;      // [jobs][2][pg][kWPT][T][32]: gate/up partial sums per task member
     double *logits;  // [T,E]
     float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs),
                      // pre-scaled for the code decode
     float *act_cs;   // [R][Kmax/32]: sums of a over 32-column chunks
-    float *y;        // [ndp_r][T*k][H]
-    float *sh;       // [ndp_s][T][H]
+    float *y;        // [ndp_r * kWPT][T*k][H]: down partial sums per task member
+    float *sh;       // [ndp_s * kWPT][T][H]
     float *m;        // [T][H]: the combine m of the current layer
+};
+
+struct Params {
+    Cfg c;
+    moe_layer_w layers[kMaxLayers];
 };
 
 // One task of an expert phase: 32 rows (row block rb) x groups [g0, g1) of
@@ -153,11 +164,19 @@ struct Smem {
     int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
     int flag;
     int flag2;  // consumer-only verdicts
+    Cfg c;          // the launch's Cfg
+    moe_layer_w w;  // the current layer's weights
 };
 
 // ------------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Block-cooperative copy of a 4-byte-aligned struct (no barrier).
+__device__ __forceinline__ void copy_words(void *dst, const void *src, size_t bytes) {
+    for (int i = threadIdx.x; i < (int)(bytes / 4); i += blockDim.x)
+        static_cast<unsigned *>(dst)[i] = static_cast<const unsigned *>(src)[i];
+}
 
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
@@ -241,7 +260,7 @@ __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;"
 // Grid-wide barrier number `nth` (1, 2, ...) on a monotonically increasing
 // counter; bounded.  Returns false (in every thread of the CTA alike) if any
 // CTA recorded an error.
-__device__ __noinline__ bool grid_sync(const Params &P, unsigned nth, int *verdict) {
+__device__ __noinline__ bool grid_sync(const Cfg &P, unsigned nth, int *verdict) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -274,7 +293,7 @@ __device__ __noinline__ bool grid_sync(const Params &P, unsigned nth, int *verdi
 // phase.  Job j = gt / (2 pg) is 32 rows of the shared expert or of one
 // active slot; its 2 pg tasks are part p of gate and of up, p = 0..pg-1.
 // All divisions happen here, once per task.
-__device__ __forceinline__ TaskDesc make_gu_task(const Params &P, const Smem &S, int gt, int pg) {
+__device__ __forceinline__ TaskDesc make_gu_task(const Cfg &P, const Smem &S, int gt, int pg) {
     TaskDesc t;
     const int j = gt / (2 * pg), r = gt - j * 2 * pg;
     const int A = P.Is / 32;
@@ -304,7 +323,7 @@ __device__ __forceinline__ TaskDesc make_gu_task(const Params &P, const Smem &S,
 
 // (slot, part) number sp of the down phase: the shared expert's parts first,
 // then each active slot's.
-__device__ __forceinline__ void dn_slot_part(const Params &P, int sp, int &slot, int &part) {
+__device__ __forceinline__ void dn_slot_part(const Cfg &P, int sp, int &slot, int &part) {
     if (sp < P.ndp_s) {
         slot = 0;
         part = sp;
@@ -316,7 +335,7 @@ __device__ __forceinline__ void dn_slot_part(const Params &P, int sp, int &slot,
 }
 
 // Task d (grid-wide index) of the down phase: (slot, part) d / (H/32), row block d % (H/32).
-__device__ __forceinline__ TaskDesc make_dn_task(const Params &P, const Smem &S, int d, int sp0) {
+__device__ __forceinline__ TaskDesc make_dn_task(const Cfg &P, const Smem &S, int d, int sp0) {
     TaskDesc t;
     const int RBH = P.H / 32, sp = d / RBH;
     int slot, part;
@@ -343,7 +362,7 @@ __device__ __forceinline__ TaskDesc make_dn_task(const Params &P, const Smem &S,
 }
 
 // Weight pointers (codes, scale/bias words) of a task's row block.
-__device__ __forceinline__ void task_ptrs(const Params &P, const moe_layer_w &W, const TaskDesc &t, bool down,
+__device__ __forceinline__ void task_ptrs(const Cfg &P, const moe_layer_w &W, const TaskDesc &t, bool down,
                                           const uint32_t *&q, const uint32_t *&sb) {
     if (!down) {
         const size_t CH = P.H / 32, GH = P.H / 64;
@@ -362,7 +381,7 @@ __device__ __forceinline__ void task_ptrs(const Params &P, const moe_layer_w &W,
 }
 
 // rowset of the tt-th token of a task (shared: the token; routed: T + bucketed position)
-__device__ __forceinline__ int task_rowset(const Params &P, const TaskDesc &t, int tt) {
+__device__ __forceinline__ int task_rowset(const Cfg &P, const TaskDesc &t, int tt) {
     return t.slot == 0 ? tt : P.T + t.seg0 + tt;
 }
 
@@ -453,7 +472,7 @@ __device__ __forceinline__ void group_dot_n(const unsigned char *codes, uint32_t
 // ------------------------------------------------------------------ phases
 
 // Input rows of a layer straight from global memory (bf16) into S.stage, and their RMS.
-__device__ __noinline__ void load_input(const Params &P, Smem &S, const uint16_t *h) {
+__device__ __noinline__ void load_input(const Cfg &P, Smem &S, const uint16_t *h) {
     const int T = P.T, H = P.H, H2 = H / 2;
     float *stage = S.stage;
 #pragma unroll 1
@@ -479,7 +498,7 @@ __device__ __noinline__ void load_input(const Params &P, Smem &S, const uint16_t
 // P0: output of layer lp (its combine m, post-norm, residual, scalar) into
 // S.stage as floats, with its RMS; CTA 0 also writes it to h_out[lp].
 // H/4 <= 1024 < 2 * blockDim, so two float4 per thread cover a row.
-__device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
+__device__ __noinline__ void finish_layer(const Cfg &P, Smem &S, int lp) {
     const int T = P.T, H = P.H, H4 = H / 4;
     const uint16_t *hprev = (P.chained && lp > 0) ? P.h_out + (size_t)(lp - 1) * T * H
                                                   : (P.chained ? P.h_in : P.h_in + (size_t)lp * T * H);
@@ -538,7 +557,7 @@ __device__ __noinline__ void finish_layer(const Params &P, Smem &S, int lp) {
 // Producer, at the start of layer l: router_scale, this CTA's router rows
 // [e0, e1) and a 16-byte-aligned superset of their scales and biases, into
 // the ring (idle until the top-k), completing on S.rbar (one phase per layer).
-__device__ __noinline__ void issue_router_copies(const Params &P, Smem &S, const moe_layer_w &W) {
+__device__ __noinline__ void issue_router_copies(const Cfg &P, Smem &S, const moe_layer_w &W) {
     const int E = P.E, H = P.H, G = H / 64;
     const int e0 = (int)((long long)E * blockIdx.x / gridDim.x), e1 = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);
     const int nrows = e1 - e0;
@@ -565,7 +584,7 @@ __device__ __noinline__ void issue_router_copies(const Params &P, Smem &S, const
 // the ring.  The dot products accumulate in fp64 so that the top-k order does
 // not depend on summation order; the common factor 1 / (rms * sqrt(H)) of a
 // token's logits is applied last (it cannot change their order).
-__device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
+__device__ __noinline__ void router_phase(const Cfg &P, Smem &S, int l) {
     const int T = P.T, H = P.H, E = P.E, G = H / 64, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     __syncthreads();  // S.rcopy written by the producer thread
     const int e0 = S.rcopy[0], nrows = S.rcopy[1], sb_lo = S.rcopy[2];
@@ -638,50 +657,79 @@ __device__ __noinline__ void router_phase(const Params &P, Smem &S, int l) {
 // or equal with a lower expert index), softmax * per_expert_scale, the
 // bucketing of the T*k pairs by rank counting too, and this CTA's job tables.
 // Every CTA.
-__device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_layer_w &W) {
+__device__ __noinline__ void topk_phase(const Cfg &P, Smem &S, const moe_layer_w &W) {
     const int T = P.T, E = P.E, k = P.k, n = T * k, H = P.H;
     // the logits as order-preserving unsigned keys (larger logit <=> larger
-    // key, exactly): a compare of two keys is integer work, not fp64
-    unsigned long long *lk = reinterpret_cast<unsigned long long *>(S.pool);  // ring is idle here: T*E keys
+    // key, exactly): lk[t][e], and their high words kh, in F segments of SL
+    // experts per token; a segment takes SS = SL + 4 words (zero padding,
+    // below every key), so the F segments that a warp reads at once start in
+    // different banks
+    unsigned long long *lk = reinterpret_cast<unsigned long long *>(S.pool);  // ring is idle here
+    const int F = (E >= 32 && T * E * 4 <= (int)blockDim.x) ? 4 : 1;
+    const int SL = ((E + F - 1) / F + 3) & ~3, SS = SL + 4, RS = F * SS;
+    uint32_t *kh = reinterpret_cast<uint32_t *>(S.pool + (((size_t)T * E * 8 + 15) & ~(size_t)15));
 #pragma unroll 1
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
-        unsigned long long b = (unsigned long long)__double_as_longlong(__ldcg(P.logits + i));
-        if (b == 0x8000000000000000ull) b = 0ull;  // -0 and +0 are the same logit
-        lk[i] = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+    for (int i = threadIdx.x; i < T * RS; i += blockDim.x) {
+        const int t = i / RS, r = i - t * RS, q = r / SS, o = r - q * SS, e = q * SL + o;
+        uint32_t hi = 0u;
+        if (o < SL && e < E) {
+            unsigned long long b = (unsigned long long)__double_as_longlong(__ldcg(P.logits + (size_t)t * E + e));
+            if (b == 0x8000000000000000ull) b = 0ull;  // -0 and +0 are the same logit
+            b = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+            lk[(size_t)t * E + e] = b;
+            hi = (uint32_t)(b >> 32);
+        }
+        kh[i] = hi;
     }
     __syncthreads();
-    // F adjacent lanes share one (token, expert): each counts over a quarter
-    // (F = 4) of the other experts, and the counts are summed by shuffles
-    const int F = T * E * 4 <= (int)blockDim.x ? 4 : 1, items = T * E * F, Ej = E / (2 * F);
+    // rank of (t, e) = keys larger than its key, plus equal keys of lower
+    // index.  F adjacent lanes share one (t, e), each counting over one
+    // segment of high words: how many are larger and how many equal (its own
+    // included).  With no other key sharing its high word, the count of
+    // larger high words is the rank; otherwise it is counted again on the
+    // full keys.
+    const int items = T * E * F;
 #pragma unroll 1
     for (int it0 = 0; it0 < items; it0 += blockDim.x) {
         const int it = it0 + threadIdx.x;
-        const int te = it / F, f = it - te * F;
-        int rank = 0;
+        const int te = F == 4 ? it >> 2 : it, f = it - te * F;
+        int gt = 0, eq = 0, t = 0, e = 0;
         unsigned long long v = 0ull;
-        int t = 0, e = 0;
         if (it < items) {
             t = te / E;
             e = te - t * E;
             v = lk[(size_t)t * E + e];
-            const ulonglong2 *row = reinterpret_cast<const ulonglong2 *>(lk + (size_t)t * E) + f * Ej;
-            const int jb = 2 * f * Ej;
+            const uint32_t hv = (uint32_t)(v >> 32);
+            const uint4 *seg = reinterpret_cast<const uint4 *>(kh + (size_t)t * RS + f * SS);
 #pragma unroll 4
-            for (int j = 0; j < Ej; ++j) {  // E is a multiple of 8
-                const ulonglong2 o = row[j];
-                rank += (o.x > v) | ((o.x == v) & (jb + 2 * j < e));
-                rank += (o.y > v) | ((o.y == v) & (jb + 2 * j + 1 < e));
+            for (int j = 0; j < SL / 4; ++j) {
+                const uint4 h = seg[j];
+                gt += (h.x > hv) + (h.y > hv) + (h.z > hv) + (h.w > hv);
+                eq += (h.x == hv) + (h.y == hv) + (h.z == hv) + (h.w == hv);
             }
         }
         if (F == 4) {
-            rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-            rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+            gt += __shfl_xor_sync(0xffffffffu, gt, 1);
+            gt += __shfl_xor_sync(0xffffffffu, gt, 2);
+            eq += __shfl_xor_sync(0xffffffffu, eq, 1);
+            eq += __shfl_xor_sync(0xffffffffu, eq, 2);
         }
-        if (it < items && f == 0 && rank < k) {
-            S.idx[t * k + rank] = e;
-            // back from the key to the logit
-            const unsigned long long b = (v >> 63) ? (v & 0x7fffffffffffffffull) : ~v;
-            S.selv[t * k + rank] = __longlong_as_double((long long)b);
+        if (it < items && f == 0) {
+            int rank = gt;
+            if (eq > 1) {
+                rank = 0;
+#pragma unroll 1
+                for (int j = 0; j < E; ++j) {
+                    const unsigned long long o = lk[(size_t)t * E + j];
+                    rank += (o > v) | ((o == v) & (j < e));
+                }
+            }
+            if (rank < k) {
+                S.idx[t * k + rank] = e;
+                // back from the key to the logit
+                const unsigned long long b = (v >> 63) ? (v & 0x7fffffffffffffffull) : ~v;
+                S.selv[t * k + rank] = __longlong_as_double((long long)b);
+            }
         }
     }
     __syncthreads();
@@ -689,7 +737,22 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
     // id), and the slot of its expert among the distinct experts (ascending).
     // Few pairs: one pass that also finds first occurrences by rescanning;
     // many pairs: first occurrences in a pass of their own.
-    if (n <= 16) {
+    if (T == 1) {
+        // one token: its k experts are distinct, so every pair is its expert's
+        // only one and the slots are the experts in ascending order
+        if (threadIdx.x < n) {
+            const int p = threadIdx.x, e = S.idx[p];
+            int less = 0;
+#pragma unroll 1
+            for (int q = 0; q < n; ++q) less += S.idx[q] < e;
+            S.perm[less] = p;
+            S.tokrow[less] = 0;
+            S.act_e[less] = e;
+            S.act_off[less] = less;
+            S.act_n[less] = 1;
+            if (p == 0) S.nact = n;
+        }
+    } else if (n <= 16) {
         int id[16];  // every pair's expert, in registers
 #pragma unroll
         for (int q = 0; q < 16; ++q) id[q] = q < n ? S.idx[q] : 0x7fffffff;
@@ -824,7 +887,7 @@ __device__ __noinline__ void topk_phase(const Params &P, Smem &S, const moe_laye
 // Gate weights w = softmax(logits[top-k]) * per_expert_scale[top-k], in fp64;
 // selv[t*k] is token t's largest selected logit.  One warp, off the critical
 // path (they are first needed by the combine in the down phase).
-__device__ __noinline__ void gate_weights(const Params &P, Smem &S, const moe_layer_w &W) {
+__device__ __noinline__ void gate_weights(const Cfg &P, Smem &S, const moe_layer_w &W) {
     const int k = P.k, n = P.T * k;
 #pragma unroll 1
     for (int p = threadIdx.x & 31; p < n; p += 32) {
@@ -840,7 +903,7 @@ __device__ __noinline__ void gate_weights(const Params &P, Smem &S, const moe_la
 // x' = bf16(rmsnorm_no_scale(h)) pre-scaled for the code decode, and its chunk
 // sums, in S.stage.  A thread per 4 columns; the 8 threads of a 32-column
 // chunk are adjacent lanes and sum it with three shuffles.
-__device__ __noinline__ void stage_x(const Params &P, Smem &S) {
+__device__ __noinline__ void stage_x(const Cfg &P, Smem &S) {
     const int T = P.T, H4 = P.H / 4, lane = threadIdx.x & 31;
     const int n4 = T * H4, rounds = (n4 + (int)blockDim.x - 1) / (int)blockDim.x;
 #pragma unroll 1
@@ -889,8 +952,8 @@ __device__ __forceinline__ void ring_pos(unsigned rq, int i, int ns, int &s, uns
 // phase); the down phase issues the rest.  Once the ring is primed, an L2
 // prefetch of what comes next (gate/up: the down tasks that do not fit the
 // ring; down: this CTA's share of the next layer's shared expert).
-__device__ __noinline__ bool task_producer(const Params &P, Smem &S, const moe_layer_w &W, bool down, unsigned rq,
-                                           int l, unsigned &issued) {
+__device__ __noinline__ bool task_producer(const Cfg &P, Smem &S, const moe_layer_w &W, bool down, unsigned rq,
+                                           const moe_layer_w *next, unsigned &issued) {
     const int ns = P.nslots, ngt = S.ngt, ndt = S.ndt;
     // ring positions [i0, i1) relative to the gate/up phase's first task
     const int pre = min(ndt, ns);  // down tasks issued during the gate/up phase
@@ -927,9 +990,9 @@ __device__ __noinline__ bool task_producer(const Params &P, Smem &S, const moe_l
             }
         }
     }
-    if (ok && down && l + 1 < P.L) {
+    if (ok && down && next != nullptr) {
         // this CTA's share of the next layer's shared-expert weights
-        const moe_layer_w &N = P.layers[l + 1];
+        const moe_layer_w &N = *next;
         const size_t shq = (size_t)P.Is * P.H / 2, shsb = (size_t)P.Is * (P.H / 64) * 4;
         const void *ptrs[6] = {N.sh_gate.q, N.sh_up.q, N.sh_down.q, N.sh_gate.sb, N.sh_up.sb, N.sh_down.sb};
         const size_t sizes[6] = {shq, shq, shq, shsb, shsb, shsb};
@@ -945,13 +1008,14 @@ __device__ __noinline__ bool task_producer(const Params &P, Smem &S, const moe_l
     return ok;
 }
 
-// A warp's share of a task: lanes are the task's 32 rows; acc[tt] receives
-// the dot product of the row's groups [g0, g1) with token tt's input.
+// A team member's share of a task: lanes are the task's 32 rows; acc[tt]
+// receives the dot product of the row's groups gi0, gi0 + kWPT, ... (< ng,
+// relative to the task's first group) with token tt's input.
 template <int NT>
-__device__ __forceinline__ void task_dot(const unsigned char *slot, int ng, const float *x, const float *xsum,
+__device__ __forceinline__ void task_dot(const unsigned char *slot, int ng, int gi0, const float *x, const float *xsum,
                                          const int *tokrow, int stride, int n, float (&acc)[NT], int lane) {
 #pragma unroll 1
-    for (int gi = 0; gi < ng; ++gi)
+    for (int gi = gi0; gi < ng; gi += kWPT)
         group_dot_n<NT>(slot + gi * kCodeBytesPerGroup,
                         reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane],
                         x + gi * 64, xsum + 2 * gi, tokrow, stride, n, acc, lane);
@@ -990,7 +1054,7 @@ __device__ __forceinline__ unsigned atom_add_release_gpu(unsigned *p, unsigned v
 
 // Bounded wait of one thread until a global count reaches `target` (acquire);
 // false (with an error recorded) on a timeout or another CTA's error.
-__device__ __noinline__ bool wait_count(const Params &P, const unsigned *ctr, unsigned target) {
+__device__ __noinline__ bool wait_count(const Cfg &P, const unsigned *ctr, unsigned target) {
     const unsigned long long t0 = globaltimer();
     for (unsigned it = 0;; ++it) {
         unsigned v;
@@ -1008,12 +1072,12 @@ __device__ __noinline__ bool wait_count(const Params &P, const unsigned *ctr, un
 }
 
 template <int NT>
-__device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int T = P.T, ns = P.nslots, nt = S.ngt, pg = S.pg, tpj = 2 * pg;
+__device__ __noinline__ bool gu_consumer(const Cfg &P, Smem &S, unsigned rq) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, team = wid / kWPT, mb = wid - team * kWPT;
+    const int T = P.T, ns = P.nslots, nt = S.ngt, pg = S.pg, pw = pg * kWPT, tpj = 2 * pw;
     bool ok = true;
 #pragma unroll 1
-    for (int i = wid; i < nt; i += kCWarps) {
+    for (int i = team; i < nt; i += kTeams) {
         const TaskDesc t = S.gut[i];
         int s;
         unsigned ph;
@@ -1026,7 +1090,8 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
         if (got) {
             const int *tokrow = t.slot == 0 ? S.tokrow_sh : S.tokrow + t.seg0;
             const int col = t.g0 * 64;
-            task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, S.stage + col, S.xs + col / 32, tokrow, 0, n, acc, lane);
+            task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, mb, S.stage + col, S.xs + col / 32, tokrow, 0, n, acc,
+                         lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[s]);
@@ -1034,9 +1099,9 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
             ok = false;
             continue;
         }
-        // this task's partial sums, then its count for the job (release: the
+        // this member's partial sums, then its count for the job (release: the
         // warp's stores, ordered by __syncwarp, become visible first)
-        float *gp = P.gpart + (((size_t)t.job * 2 + t.mat) * pg + t.part) * T * 32;
+        float *gp = P.gpart + ((((size_t)t.job * 2 + t.mat) * pg + t.part) * kWPT + mb) * T * 32;
 #pragma unroll
         for (int tt = 0; tt < NT; ++tt)
             if (tt < n) gp[tt * 32 + lane] = acc[tt];
@@ -1048,15 +1113,15 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
             // the job's last task: sum the parts in a fixed order, form a = silu(g) * u
             if (lane == 0) __threadfence();
             __syncwarp();
-            const float *jp = P.gpart + (size_t)t.job * 2 * pg * T * 32;
+            const float *jp = P.gpart + (size_t)t.job * 2 * pw * T * 32;
 #pragma unroll 1
             for (int tt = 0; tt < n; ++tt) {
                 float gs = 0.f, us = 0.f;
 #pragma unroll
-                for (int p2 = 0; p2 < kMaxPG; ++p2) {
-                    if (p2 < pg) {
+                for (int p2 = 0; p2 < kMaxPG * kWPT; ++p2) {
+                    if (p2 < pw) {
                         gs += __ldcg(&jp[((size_t)p2 * T + tt) * 32 + lane]);
-                        us += __ldcg(&jp[((size_t)(pg + p2) * T + tt) * 32 + lane]);
+                        us += __ldcg(&jp[((size_t)(pw + p2) * T + tt) * 32 + lane]);
                     }
                 }
                 const float a = silu_mul(gs, us);
@@ -1077,7 +1142,7 @@ __device__ __noinline__ bool gu_consumer(const Params &P, Smem &S, unsigned rq) 
 
 // Stage the down inputs of segments [k0, k1): a (already pre-scaled for the
 // code decode) and its chunk sums.  Consumer threads only.
-__device__ __noinline__ bool stage_segments(const Params &P, Smem &S, int k0, int k1) {
+__device__ __noinline__ bool stage_segments(const Cfg &P, Smem &S, int k0, int k1) {
     const int ctid = threadIdx.x, KC = P.Kmax / 32;
     // every consumer warp is past its gate/up tasks (the stage still held their
     // input); then wait until each staged slot's SwiGLU rows are all written
@@ -1111,10 +1176,11 @@ __device__ __noinline__ bool stage_segments(const Params &P, Smem &S, int k0, in
     return true;
 }
 
-// The combine m[t][row] = sum_s w[t,s] * y[t,s] + shared, in a fixed order;
-// the loads of a batch are issued before any is used.
-__device__ __noinline__ void combine_row(const Params &P, const Smem &S, int row) {
-    const int T = P.T, k = P.k, H = P.H;
+// The combine m[t][row] = sum_s w[t,s] * y[t,s] + shared, in a fixed order.
+// y and the shared output are sums of kWPT * ndp parts; the loads of up to
+// 2 parts x 8 routed slots (or 8 shared parts) are issued before any is used.
+__device__ __noinline__ void combine_row(const Cfg &P, const Smem &S, int row) {
+    const int T = P.T, k = P.k, H = P.H, ny = P.ndp_r * kWPT, nsh = P.ndp_s * kWPT;
     const size_t ystride = (size_t)T * k * H;
 #pragma unroll 1
     for (int t = 0; t < T; ++t) {
@@ -1123,34 +1189,44 @@ __device__ __noinline__ void combine_row(const Params &P, const Smem &S, int row
         for (int s0 = 0; s0 < k; s0 += 8) {
             float yv[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) yv[u] = s0 + u < k ? __ldcg(&P.y[(size_t)(t * k + s0 + u) * H + row]) : 0.f;
+            for (int u = 0; u < 8; ++u) yv[u] = 0.f;
 #pragma unroll 1
-            for (int dp = 1; dp < P.ndp_r; ++dp) {
+            for (int d0 = 0; d0 < ny; d0 += 2) {
+                float pv[2][8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (s0 + u < k) yv[u] += __ldcg(&P.y[dp * ystride + (size_t)(t * k + s0 + u) * H + row]);
+                for (int d = 0; d < 2; ++d)
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        pv[d][u] = (d0 + d < ny && s0 + u < k)
+                                       ? __ldcg(&P.y[(d0 + d) * ystride + (size_t)(t * k + s0 + u) * H + row])
+                                       : 0.f;
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) yv[u] += pv[d][u];
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 if (s0 + u < k) mv = fmaf(S.wts[t * k + s0 + u], yv[u], mv);
         }
-        float sv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) sv[u] = u < P.ndp_s ? __ldcg(&P.sh[((size_t)u * T + t) * H + row]) : 0.f;
 #pragma unroll 1
-        for (int u = 4; u < P.ndp_s; ++u) mv += __ldcg(&P.sh[((size_t)u * T + t) * H + row]);
+        for (int u0 = 0; u0 < nsh; u0 += 8) {
+            float sv[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) mv += sv[u];
+            for (int u = 0; u < 8; ++u) sv[u] = u0 + u < nsh ? __ldcg(&P.sh[((size_t)(u0 + u) * T + t) * H + row]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mv += sv[u];
+        }
         P.m[(size_t)t * H + row] = mv;
     }
 }
 
 template <int NT>
-__device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+__device__ __noinline__ bool dn_consumer(const Cfg &P, Smem &S, unsigned rq) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, team = wid / kWPT, mb = wid - team * kWPT;
     const int T = P.T, k = P.k, H = P.H, ns = P.nslots, nt = S.ndt;
-    // down tasks per row block in this layer: every part of the shared expert and of each active slot
-    const unsigned dn_per_rb = (unsigned)(P.ndp_s + S.nact * P.ndp_r);
+    // member results per row block in this layer: every part of the shared expert and of each active slot
+    const unsigned dn_per_rb = (unsigned)((P.ndp_s + S.nact * P.ndp_r) * kWPT);
     const int rounds = S.seg_rounds;
     bool ok = true;
 #pragma unroll 1
@@ -1158,7 +1234,7 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) 
         const int k0 = rounds == 1 ? 0 : r, k1 = rounds == 1 ? S.nseg : r + 1;
         if (!stage_segments(P, S, k0, k1)) return false;
 #pragma unroll 1
-        for (int i = wid; i < nt; i += kCWarps) {
+        for (int i = team; i < nt; i += kTeams) {
             const TaskDesc t = S.dnt[i];
             if (t.seg < k0 || t.seg >= k1) continue;
             int s;
@@ -1171,7 +1247,7 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) 
             for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
             const bool got = wait_task(S, rq + (unsigned)i, s, ph, P.err);
             if (got)  // token tt's row at off + tt * ld, its chunk sums at (off + tt * ld) / 32
-                task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, S.stage + sg.off, S.xs + sg.off / 32, nullptr,
+                task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, mb, S.stage + sg.off, S.xs + sg.off / 32, nullptr,
                              sg.ld, n, acc, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.empty[s]);
@@ -1179,14 +1255,14 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) 
                 ok = false;
                 continue;
             }
-            const int row = t.rb * 32 + lane;
+            const int row = t.rb * 32 + lane, pm = t.part * kWPT + mb;
 #pragma unroll
             for (int tt = 0; tt < NT; ++tt) {
                 if (tt < n) {
                     if (t.slot == 0)
-                        P.sh[((size_t)t.part * T + tt) * H + row] = acc[tt];
+                        P.sh[((size_t)pm * T + tt) * H + row] = acc[tt];
                     else
-                        P.y[((size_t)t.part * T * k + S.perm[t.seg0 + tt]) * H + row] = acc[tt];
+                        P.y[((size_t)pm * T * k + S.perm[t.seg0 + tt]) * H + row] = acc[tt];
                 }
             }
             // count this task for its row block (release: the warp's rows, ordered
@@ -1212,7 +1288,7 @@ __device__ __noinline__ bool dn_consumer(const Params &P, Smem &S, unsigned rq) 
 }
 
 // All threads: wait until `target` row blocks of m are combined (over all layers so far).
-__device__ __noinline__ bool wait_rows(const Params &P, Smem &S, unsigned target) {
+__device__ __noinline__ bool wait_rows(const Cfg &P, Smem &S, unsigned target) {
     __syncthreads();
     if (threadIdx.x == 0) {
         const bool ok = wait_count(P, P.rows_done, target);
@@ -1225,9 +1301,10 @@ __device__ __noinline__ bool wait_rows(const Params &P, Smem &S, unsigned target
 
 // ------------------------------------------------------------------ kernel
 
-__global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_constant__ Params Pk) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem &S = *reinterpret_cast<Smem *>(smem_raw);
+    const Cfg &P = S.c;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const bool producer = (wid == kProducerWarp && lane == 0);
     const bool consumer = wid < kCWarps;
@@ -1235,14 +1312,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 1);  // one consumer warp per task
+            mbar_init(&S.empty[s], kWPT);  // every warp of the task's team
         }
         mbar_init(&S.rbar, 1);
         for (int s = 0; s < kMaxStages; ++s) S.slot_task[s] = 0xffffffffu;
         for (int s = 0; s <= kMaxPairs; ++s) S.act_expect[s] = 0u;
-        S.stage = reinterpret_cast<float *>(S.pool + (size_t)P.nslots * kSlotBytes);
+        S.stage = reinterpret_cast<float *>(S.pool + (size_t)Pk.c.nslots * kSlotBytes);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    copy_words(&S.c, &Pk.c, sizeof(Cfg));
+    copy_words(&S.w, &Pk.layers[0], sizeof(moe_layer_w));
     __syncthreads();
 
     unsigned rq = 0;       // ring sequence number of the next task (the same in every thread)
@@ -1253,7 +1332,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     const int ns = P.nslots;
 
     for (int l = 0; l < P.L && ok; ++l) {
-        const moe_layer_w &W = P.layers[l];
+        const moe_layer_w &W = S.w;
+        const moe_layer_w *next = l + 1 < P.L ? &Pk.layers[l + 1] : nullptr;
         if (producer) {
             issue_router_copies(P, S, W);
             ++rissued;
@@ -1275,7 +1355,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 
         // ---------------- gate/up tasks
         if (producer)
-            task_producer(P, S, W, false, rq, l, issued);
+            task_producer(P, S, W, false, rq, next, issued);
         else if (consumer) {
             P.T == 1 ? gu_consumer<1>(P, S, rq) : gu_consumer<kMaxT>(P, S, rq);
             if (wid == kCWarps - 1) gate_weights(P, S, W);
@@ -1284,12 +1364,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 
         // ---------------- down tasks (each CTA as soon as its own gate/up tasks are done)
         if (producer)
-            task_producer(P, S, W, true, rq, l, issued);
+            task_producer(P, S, W, true, rq, next, issued);
         else if (consumer)
             P.T == 1 ? dn_consumer<1>(P, S, rq) : dn_consumer<kMaxT>(P, S, rq);
         rq += (unsigned)S.ndt;
         __syncthreads();
         if (threadIdx.x == 0) S.flag = ldcg_int(P.err) == 0;
+        if (next != nullptr) copy_words(&S.w, next, sizeof(moe_layer_w));  // every use of this layer's is done
         __syncthreads();
         ok = S.flag != 0;
     }
@@ -1311,6 +1392,7 @@ size_t decode_stack_smem() { return sizeof(dec::Smem); }
 
 static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exceeds 227 KiB");
 static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
+static_assert(sizeof(dec::Cfg) % 4 == 0 && sizeof(moe_layer_w) % 4 == 0, "copied word by word");
 
 struct DecodeWs {
     size_t bar, cnt_dn, cnt_gu, act_done, logits, gpart, act, act_cs, y, sh, m, total, zero_bytes;
@@ -1338,12 +1420,12 @@ static DecodeWs decode_ws(const moe_layer_w *w, int T) {
     d.cnt_gu = take(sizeof(unsigned) * jobs);
     d.act_done = take(sizeof(unsigned) * (R + 1));  // per slot, then rows_done
     d.zero_bytes = off;
-    d.gpart = take(sizeof(float) * jobs * 2 * pg * T * 32);
+    d.gpart = take(sizeof(float) * jobs * 2 * pg * dec::kWPT * T * 32);
     d.logits = take(sizeof(double) * (size_t)T * w->E);
     d.act = take(sizeof(float) * (size_t)R * Kmax);
     d.act_cs = take(sizeof(float) * (size_t)R * (Kmax / 32));
-    d.y = take(sizeof(float) * (size_t)ndp_r * T * w->k * w->H);
-    d.sh = take(sizeof(float) * (size_t)ndp_s * T * w->H);
+    d.y = take(sizeof(float) * (size_t)ndp_r * dec::kWPT * T * w->k * w->H);
+    d.sh = take(sizeof(float) * (size_t)ndp_s * dec::kWPT * T * w->H);
     d.m = take(sizeof(float) * (size_t)T * w->H);
     d.total = off;
     return d;
@@ -1365,7 +1447,8 @@ static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots, in
     const long ring = ns * dec::kSlotBytes;
     const long rows = grid > 0 ? (w.E + grid - 1) / grid : w.E;
     const long rcopy = 2L * w.H + rows * w.H + 2 * (rows * (w.H / 64) * 2 + 32);
-    if (ns < 3 || (long)T * w.E * 8 > ring || rcopy > ring || grid <= 0) return false;
+    const long topk_keys = (long)T * w.E * 8 + 16 + (long)T * (w.E + 28) * 4;  // keys and padded high words
+    if (ns < 3 || topk_keys > ring || rcopy > ring || grid <= 0) return false;
     // task tables of the busiest CTA, for the most distinct experts a call can route to
     const long pairs = (long)T * w.k < w.E ? (long)T * w.k : w.E;
     const long pg = (w.H / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
@@ -1395,8 +1478,9 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
                                 uint16_t *h_out, int T, void *ws, const moe_opts &o, int grid, cudaStream_t st) {
     const moe_layer_w &w = layers[0];
     const DecodeWs d = decode_ws(&w, T);
-    dec::Params P;  // ~10 KiB, passed by value (kernel parameters up to 32 KiB)
-    for (int l = 0; l < L; ++l) P.layers[l] = layers[l];
+    dec::Params Pk;  // ~10 KiB, passed by value (kernel parameters up to 32 KiB)
+    dec::Cfg &P = Pk.c;
+    for (int l = 0; l < L; ++l) Pk.layers[l] = layers[l];
     P.h_in = h_in;
     P.h_out = h_out;
     P.L = L;
@@ -1440,7 +1524,7 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(ws, 0, d.zero_bytes, st);
     if (e != cudaSuccess) return e;
-    void *args[] = {&P};
+    void *args[] = {&Pk};
     e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(dec::decode_stack_kernel), dim3(grid),
                                     dim3(dec::kThreads), args, smem, st);
     return e;

@@ -21,10 +21,15 @@
 //   token producer   loads the tokens' FP16 rows with 2-D TMA tensor copies
 //                    (128-byte swizzle), in a warp of its own so that neither
 //                    producer waits behind the other;
-//   8 dequant warps  turn each k-block of codes into FP16 weights
-//                    w = s*q + b (exact q, one rounding) in the swizzled
-//                    K-major layout the tensor core reads;
-//   MMA thread       issues tcgen05.mma kind::f16 (FP16 x FP16 -> FP32 in TMEM)
+//   16 dequant warps turn each k-block of codes into FP16 weights
+//                    w = s*q + b (exact q, one rounding) and store them into
+//                    tensor memory (tcgen05.st: TMEM lane = tile row, two
+//                    weights per 32-bit column), where the MMA reads its A
+//                    operand -- so the FP16 weights never pass through shared
+//                    memory, whose bandwidth an MMA with few tokens (small N)
+//                    would otherwise spend mostly on re-reading A;
+//   MMA thread       issues tcgen05.mma kind::f16 with A in TMEM and B (the
+//                    tokens) in shared memory (FP16 x FP16 -> FP32 in TMEM)
 //                    and signals buffers free with tcgen05.commit;
 //   epilogue         (the dequant warps) reads the accumulators with
 //                    tcgen05.ld: gate/up tiles hold 128 gate rows in TMEM
@@ -66,8 +71,8 @@ namespace mma {
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // input columns per k-block
 constexpr int kKS = 2;            // k-blocks per code stage
-constexpr int kCodeSlots = 4;     // code stages in flight
-constexpr int kABufs = 3;         // FP16 weight stages (32 KiB each)
+constexpr int kCodeSlots = 8;     // code stages in flight
+constexpr int kABufs = 4;         // FP16 weight stages in TMEM (64 columns each)
 constexpr int kBBufs = 3;         // token slots of 16 KiB: 128 / N k-blocks of an N-token tile each
 constexpr int kMaxN = 128;        // tokens per tile
 constexpr int kBoxRows = 16;      // rows of one TMA box of the token matrix
@@ -76,8 +81,9 @@ constexpr int kProdWarp = 16;   // weight codes
 constexpr int kMmaWarp = 17;
 constexpr int kTokWarp = 18;    // token tiles
 constexpr int kThreads = 19 * 32;
-constexpr int kTmemCols = 256;
-constexpr int kATileBytes = kBM * kBK * 2;       // 16 KiB
+constexpr int kTmemCols = 512;   // accumulators in columns [0, 256), weight stages in [256, 512)
+constexpr int kAccCols = 256;
+constexpr int kAStageCols = 64;   // 2 tiles of 128 x 64 FP16 (32 columns each)
 constexpr int kBBufBytes = kMaxN * kBK * 2;      // 16 KiB
 constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 2 KiB
 constexpr unsigned long long kWaitNs = 1000000000ull;
@@ -85,18 +91,16 @@ constexpr unsigned long long kWaitNs = 1000000000ull;
 enum { kErrCodeFull = 1, kErrCodeEmpty, kErrAFull, kErrAEmpty, kErrBFull, kErrBEmpty, kErrAccFull, kErrAccEmpty };
 
 // Shared-memory plan of the kernel for NMAT weight matrices per tile (2:
-// gate and up, 1: down).  A weight stage holds kAK k-blocks of every matrix
-// (NMAT * kAK = 2 tiles of 128 x 64 FP16), so that each of the 512 dequant
-// threads converts exactly one 32-code record per stage.
+// gate and up, 1: down).  A weight stage (in TMEM) holds kAK k-blocks of
+// every matrix (NMAT * kAK = 2 tiles of 128 x 64 FP16), so that each of the
+// 512 dequant threads converts exactly one 32-code record per stage.
 template <int NMAT>
 struct Lay {
     static constexpr int kAK = 2 / NMAT;
     static constexpr int kCodeBytes = NMAT * 4 * kKS * 1024;
     static constexpr int kSbBytes = NMAT * 4 * kKS * 128;
     static constexpr int kSlotBytes = kCodeBytes + kSbBytes;
-    static constexpr int kABytes = NMAT * kAK * kATileBytes;
-    static constexpr int kAOff = 0;
-    static constexpr int kBOff = kAOff + kABufs * kABytes;
+    static constexpr int kBOff = 0;
     static constexpr int kCodeOff = kBOff + kBBufs * kBBufBytes;
     static constexpr int kBarOff = kCodeOff + kCodeSlots * kSlotBytes;
     static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 3;
@@ -105,6 +109,7 @@ struct Lay {
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
 };
 static_assert(Lay<2>::kAlloc <= 227 * 1024, "gate/up tile buffers exceed shared memory");
+static_assert(kAccCols + kABufs * kAStageCols <= kTmemCols && 2 * kMaxN <= kAccCols, "tensor memory plan");
 static_assert(kDqWarps * 32 == 2 * 2 * kBM, "one record (row, 32 codes) per dequant thread and stage");
 static_assert(kKS % Lay<1>::kAK == 0 && kKS % Lay<2>::kAK == 0, "a code stage holds whole weight stages");
 
@@ -238,6 +243,27 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
         : "memory");
 }
 
+// The same with A read from tensor memory at a_tmem (lane 0 = row 0 of the
+// 128-row operand, 16 K-elements in 8 consecutive 32-bit columns).
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, int acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// One thread's 16 consecutive 32-bit columns of its TMEM lane (a warp stores
+// its 32 lanes; the address's lane field must be the warp's lane quarter).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint4 (&v)[4]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w), "r"(v[1].x), "r"(v[1].y), "r"(v[1].z), "r"(v[1].w),
+        "r"(v[2].x), "r"(v[2].y), "r"(v[2].z), "r"(v[2].w), "r"(v[3].x), "r"(v[3].y), "r"(v[3].z), "r"(v[3].w)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -358,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *gbase = smem_raw + (base - raw);
-    const uint32_t sA = base + L::kAOff, sB = base + L::kBOff, sC = base + L::kCodeOff;
+    const uint32_t sB = base + L::kBOff, sC = base + L::kCodeOff;
     const uint32_t bars = base + L::kBarOff;
     auto code_full = [&](int i) { return bars + 8u * i; };
     auto code_empty = [&](int i) { return bars + 8u * (kCodeSlots + i); };
@@ -481,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                         ok = false;
                         break;
                     }
-                    const uint32_t abase = sA + (uint32_t)a * L::kABytes;
+                    const uint32_t abase = tmem + (uint32_t)(kAccCols + a * kAStageCols);
                     for (int kbi = 0; kbi < L::kAK && ks + kbi < nkb; ++kbi) {
                         const int kb = ks + kbi, b = kbc % kBBufs;
                         if (kb % bkb == 0 && !mbar_wait(b_full(b), (kbc / kBBufs) & 1, P.err, kErrBFull)) {
@@ -494,9 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                         for (int kk = 0; kk < kBK / 16; ++kk) {
 #pragma unroll
                             for (int m = 0; m < NMAT; ++m)
-                                mma_f16(tmem + (uint32_t)(m * t.N),
-                                        sw128_desc(abase + (m * L::kAK + kbi) * kATileBytes + kk * 32),
-                                        sw128_desc(bbase + kk * 32), idesc, ((ks + kbi) | kk) != 0);
+                                mma_f16_tmem_a(tmem + (uint32_t)(m * t.N), abase + (uint32_t)((m * L::kAK + kbi) * 32 + kk * 8),
+                                               sw128_desc(bbase + kk * 32), idesc, ((ks + kbi) | kk) != 0);
                         }
                         if (kb % bkb == bkb - 1 || kb == nkb - 1) {  // last k-block of this token slot
                             mma_commit(b_empty(b));
@@ -553,9 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                     ok = false;
                     break;
                 }
-                if (valid) {
-                    unsigned char *arow =
-                        gbase + L::kAOff + (size_t)a * L::kABytes + (size_t)(m * L::kAK + kbi) * kATileBytes + r * 128;
+                tc_fence_after();  // the MMAs that read this stage's columns have completed
+                if (valid) {  // warp-uniform: rv is a multiple of 32, kbi is the warp's
                     const float sf = __uint_as_float(sbw << 16), bf = __uint_as_float(sbw & 0xffff0000u);
                     const uint32_t b2 = f16x2_from_f32(bf, bf);
                     const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
@@ -569,12 +593,13 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
 #pragma unroll
                         for (int wi = 0; wi < 4; ++wi) o[wi] = dequant_word(wv[wi], s2, b2);
                     }
-#pragma unroll
-                    for (int wi = 0; wi < 4; ++wi)
-                        *reinterpret_cast<uint4 *>(arow + (((4 * half + wi) ^ (r & 7)) << 4)) = o[wi];
+                    // columns: stage a, tile (m, kbi), this half's 16 columns; lane field: this warp's rows
+                    tmem_st16(tmem + ((uint32_t)(r & ~31) << 16) +
+                                  (uint32_t)(kAccCols + a * kAStageCols + (m * L::kAK + kbi) * 32 + half * 16),
+                              o);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 }
-                // generic-proxy stores -> visible to the tensor core (async proxy)
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(a_full(a));
                 ++asc;
