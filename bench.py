@@ -48,8 +48,8 @@ def peaks():
 # capture, per unit of work: decode_stack_kernel at the Gemma shape, T = 1,
 # per layer (2-layer capture halved); the two grouped-GEMM kernels of one
 # 128-token layer-chunk.  Reset to None whenever the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = None  # re-capture after the last kernel change
-PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_850_432 + 6_467_072 + 147_067_136 + 9_365_248
+DECODE_TRAFFIC_PER_LAYER = (74_531_072 + 2_422_784) // 2
+PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_847_616 + 4_750_080 + 147_008_512 + 8_972_288
 
 
 def expert_bytes(rows_cols: int) -> float:
