@@ -49,7 +49,7 @@ def peaks():
 # per layer (2-layer capture halved); the two grouped-GEMM kernels of one
 # 128-token layer-chunk.  Reset to None whenever the kernel changes.
 DECODE_TRAFFIC_PER_LAYER = (74_531_072 + 2_422_784) // 2
-PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_847_616 + 4_750_080 + 147_008_512 + 8_972_288
+PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_960_000 + 5_408_000 + 147_004_672 + 8_862_720
 
 
 def expert_bytes(rows_cols: int) -> float:

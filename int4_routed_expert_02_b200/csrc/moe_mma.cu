@@ -31,12 +31,16 @@
 //   MMA thread       issues tcgen05.mma kind::f16 with A in TMEM and B (the
 //                    tokens) in shared memory (FP16 x FP16 -> FP32 in TMEM)
 //                    and signals buffers free with tcgen05.commit;
-//   epilogue         (the dequant warps) reads the accumulators with
-//                    tcgen05.ld: gate/up tiles hold 128 gate rows in TMEM
-//                    columns [0, N) and the same 128 up rows in [N, 2N), so each
-//                    thread forms a = silu(g) * u for its row and writes it as
-//                    FP16 -- the down GEMM's B operand; down tiles write fp32
-//                    y rows for the combine.
+//   4 epilogue warps read the accumulators with tcgen05.ld (warp w: TMEM
+//                    lanes 32 (w % 4) ..): gate/up tiles hold 128 gate rows in
+//                    accumulator columns [0, N) and the same 128 up rows in
+//                    [N, 2N), so each thread forms a = silu(g) * u for its row
+//                    and writes it as FP16 -- the down GEMM's B operand; down
+//                    tiles write fp32 y rows for the combine.  The accumulator
+//                    is double-buffered (two 128-column buffers, tiles wider
+//                    than 128 columns take both), so the MMAs of the next tile
+//                    run while the epilogue drains this one, and the dequant
+//                    warps never wait for an epilogue.
 //
 // Operand precision.  The tensor cores take FP16 or BF16 at the same rate and
 // the same bytes.  FP16 is used: its 11-bit significand keeps the rounding of
@@ -76,13 +80,15 @@ constexpr int kABufs = 4;         // FP16 weight stages in TMEM (64 columns each
 constexpr int kBBufs = 3;         // token slots of 16 KiB: 128 / N k-blocks of an N-token tile each
 constexpr int kMaxN = 128;        // tokens per tile
 constexpr int kBoxRows = 16;      // rows of one TMA box of the token matrix
-constexpr int kDqWarps = 16;      // dequant (and epilogue) warps: one 32-code record per thread per stage
+constexpr int kDqWarps = 16;      // dequant warps: one 32-code record per thread per stage
 constexpr int kProdWarp = 16;   // weight codes
 constexpr int kMmaWarp = 17;
 constexpr int kTokWarp = 18;    // token tiles
-constexpr int kThreads = 19 * 32;
+constexpr int kEpiWarp0 = 19;   // 4 epilogue warps: warp w reads TMEM lanes 32 * (w % 4) ..
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;   // accumulators in columns [0, 256), weight stages in [256, 512)
-constexpr int kAccCols = 256;
+constexpr int kAccCols = 256;     // two accumulator buffers of 128 columns; a tile wider than 128 takes both
 constexpr int kAStageCols = 64;   // 2 tiles of 128 x 64 FP16 (32 columns each)
 constexpr int kBBufBytes = kMaxN * kBK * 2;      // 16 KiB
 constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 2 KiB
@@ -103,7 +109,7 @@ struct Lay {
     static constexpr int kBOff = 0;
     static constexpr int kCodeOff = kBOff + kBBufs * kBBufBytes;
     static constexpr int kBarOff = kCodeOff + kCodeSlots * kSlotBytes;
-    static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 3;
+    static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 5;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kTmemSlotOff + 16;
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
@@ -169,11 +175,14 @@ __device__ __forceinline__ bool mbar_test(uint32_t b, unsigned parity) {
 }
 
 // Bounded wait for the phase with `parity` to complete; false on a timeout or
-// when another thread has recorded an error.
-__device__ bool mbar_wait(uint32_t b, unsigned parity, int *err, int code) {
+// when another thread has recorded an error.  sleep_ns > 0 backs off between
+// tests: the producers, which run ahead, then leave the issue slots of their
+// SM sub-partition to the dequantising warps that share it.
+__device__ bool mbar_wait(uint32_t b, unsigned parity, int *err, int code, unsigned sleep_ns = 0) {
     if (mbar_test(b, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (unsigned it = 1;; ++it) {
+        if (sleep_ns) __nanosleep(sleep_ns);
         if (mbar_test(b, parity)) return true;
         if ((it & 63u) == 0) {
             if (__ldcg(err) != 0) return false;
@@ -392,8 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
     auto a_empty = [&](int i) { return bars + 8u * (2 * kCodeSlots + kABufs + i); };
     auto b_full = [&](int i) { return bars + 8u * (2 * kCodeSlots + 2 * kABufs + i); };
     auto b_empty = [&](int i) { return bars + 8u * (2 * kCodeSlots + 2 * kABufs + kBBufs + i); };
-    const uint32_t acc_full = bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs);
-    const uint32_t acc_empty = acc_full + 8u, drain = acc_full + 16u;
+    // accumulator buffer i (columns [128 i, 128 i + 128)): full (MMAs done) and empty (epilogue done)
+    auto acc_full = [&](int i) { return bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + i); };
+    auto acc_empty = [&](int i) { return bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 2 + i); };
+    const uint32_t drain = bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::kTmemSlotOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -410,8 +421,10 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
             mbar_init(b_full(i), 1);
             mbar_init(b_empty(i), 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kDqWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(acc_full(i), 1);
+            mbar_init(acc_empty(i), kEpiWarps);
+        }
         mbar_init(drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -439,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                 for (int kb = 0; kb < nkb; kb += kKS) {
                     const int s = cs % kCodeSlots;
                     if (cs >= kCodeSlots &&
-                        !mbar_wait(code_empty(s), ((cs / kCodeSlots) & 1) ^ 1, P.err, kErrCodeEmpty)) {
+                        !mbar_wait(code_empty(s), ((cs / kCodeSlots) & 1) ^ 1, P.err, kErrCodeEmpty, 256)) {
                         ok = false;
                         break;
                     }
@@ -471,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                 const int nkb = t.K / kBK, nbox = t.N / kBoxRows, bkb = kMaxN / t.N;  // k-blocks per token slot
                 for (int kb = 0; kb < nkb; kb += bkb) {
                     const int b = kbc % kBBufs;
-                    if (kbc >= kBBufs && !mbar_wait(b_empty(b), ((kbc / kBBufs) & 1) ^ 1, P.err, kErrBEmpty)) {
+                    if (kbc >= kBBufs && !mbar_wait(b_empty(b), ((kbc / kBBufs) & 1) ^ 1, P.err, kErrBEmpty, 256)) {
                         ok = false;
                         break;
                     }
@@ -491,16 +504,28 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             uint32_t asc = 0, kbc = 0, ic = 0;
-            bool ok = true;
+            bool ok = true, prev_wide = false;
             for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
                 Tile t;
                 if (!get_tile(P, it, t)) continue;
-                if (ic > 0) {
-                    if (!mbar_wait(acc_empty, (ic - 1) & 1, P.err, kErrAccEmpty)) break;
+                // tile ic accumulates in buffer ic % 2, or in both when wider than one;
+                // wait until the epilogue has drained the last tile whose columns it
+                // overwrites (tiles are drained in order, so tile j's count implies
+                // every earlier one's)
+                const bool wide = NMAT * t.N > kAccCols / 2;
+                const int need = (wide || prev_wide) ? (int)ic - 1 : (int)ic - 2;
+                prev_wide = wide;
+                if (need >= 0) {
+                    if (!mbar_wait(acc_empty(need & 1), (need >> 1) & 1, P.err, kErrAccEmpty)) break;
                     tc_fence_after();
                 }
+                const uint32_t dacc = tmem + (wide ? 0u : (ic & 1u) * (uint32_t)(kAccCols / 2));
                 const uint32_t idesc = idesc_f16(t.N);
                 const int nkb = t.K / kBK, bkb = kMaxN / t.N;
+                const uint32_t bstep = (uint32_t)t.N * kBK * 2;  // bytes of one k-block of the tile's tokens
+                int kin = 0;                                      // k-block inside the current token slot
+                // one issuing thread: keep the per-MMA work to adds (descriptors and
+                // addresses advance by constants, no division in the loop)
                 for (int ks = 0; ks < nkb && ok; ks += L::kAK) {
                     const int a = asc % kABufs;
                     if (!mbar_wait(a_full(a), (asc / kABufs) & 1, P.err, kErrAFull)) {
@@ -510,22 +535,24 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                     const uint32_t abase = tmem + (uint32_t)(kAccCols + a * kAStageCols);
                     for (int kbi = 0; kbi < L::kAK && ks + kbi < nkb; ++kbi) {
                         const int kb = ks + kbi, b = kbc % kBBufs;
-                        if (kb % bkb == 0 && !mbar_wait(b_full(b), (kbc / kBBufs) & 1, P.err, kErrBFull)) {
+                        if (kin == 0 && !mbar_wait(b_full(b), (kbc / kBBufs) & 1, P.err, kErrBFull)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t bbase = sB + (uint32_t)b * kBBufBytes + (uint32_t)((kb % bkb) * t.N * kBK * 2);
+                        const uint64_t bdesc = sw128_desc(sB + (uint32_t)b * kBBufBytes + (uint32_t)kin * bstep);
+                        const uint32_t a0 = abase + (uint32_t)(kbi * 32);
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk) {
 #pragma unroll
-                            for (int m = 0; m < NMAT; ++m)
-                                mma_f16_tmem_a(tmem + (uint32_t)(m * t.N), abase + (uint32_t)((m * L::kAK + kbi) * 32 + kk * 8),
-                                               sw128_desc(bbase + kk * 32), idesc, ((ks + kbi) | kk) != 0);
+                            for (int m = 0; m < NMAT; ++m)  // +32 bytes of K: +2 in the descriptor's address field
+                                mma_f16_tmem_a(dacc + (uint32_t)(m * t.N), a0 + (uint32_t)(m * L::kAK * 32 + kk * 8),
+                                               bdesc + (uint64_t)(2 * kk), idesc, (kb | kk) != 0);
                         }
-                        if (kb % bkb == bkb - 1 || kb == nkb - 1) {  // last k-block of this token slot
+                        if (++kin == bkb || kb == nkb - 1) {  // last k-block of this token slot
                             mma_commit(b_empty(b));
                             ++kbc;
+                            kin = 0;
                         }
                     }
                     if (!ok) break;
@@ -533,20 +560,20 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                     ++asc;
                 }
                 if (!ok) break;
-                mma_commit(acc_full);
+                mma_commit(acc_full(ic & 1));
                 ++ic;
             }
             // every MMA this thread issued has completed once `drain` fires
             mma_commit(drain);
             mbar_drain(drain, 0);
         }
-    } else {
-        // ---------------------------------------------------------- dequant + epilogue
+    } else if (warp < kDqWarps) {
+        // ---------------------------------------------------------- dequant
         // thread -> one record per weight stage: tile row r, matrix m, k-block kbi of the stage, 32-code half
         const int r = threadIdx.x & (kBM - 1), j4 = threadIdx.x >> 7;
         const int m = NMAT == 2 ? (j4 >> 1) : 0, kbi = NMAT == 2 ? 0 : (j4 >> 1), half = j4 & 1;
         const int rbl = r >> 5, rl = r & 31;
-        uint32_t cs = 0, asc = 0, ic = 0;
+        uint32_t cs = 0, asc = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
             Tile t;
@@ -604,16 +631,24 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                 if (lane == 0) mbar_arrive(a_full(a));
                 ++asc;
             }
-            if (!ok) break;
-            // epilogue: warp w reads TMEM lanes 32*(w%4).. (tile rows), chunks of 8 columns c with c%4 == w/4
-            if (!__all_sync(0xffffffffu, mbar_wait(acc_full, ic & 1, P.err, kErrAccFull))) break;
+        }
+    } else if (warp >= kEpiWarp0) {
+        // ---------------------------------------------------------- epilogue
+        // warp w reads TMEM lanes 32*(w%4).. (tile rows); tiles in order, buffers alternating
+        const int q4 = warp & 3;
+        uint32_t ic = 0;
+        for (int it = blockIdx.x; it < P.n_items; it += gridDim.x) {
+            Tile t;
+            if (!get_tile(P, it, t)) continue;
+            const int ab = (int)(ic & 1u);
+            if (!__all_sync(0xffffffffu, mbar_wait(acc_full(ab), (ic >> 1) & 1, P.err, kErrAccFull))) break;
             tc_fence_after();
-            const int q4 = warp & 3, cg = warp >> 2;
+            const bool wide = NMAT * t.N > kAccCols / 2;
             const int row = t.mt * kBM + q4 * 32 + lane;
             const bool rvalid = q4 * 32 < t.rv;  // warp-uniform
-            const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16);
+            const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + (wide ? 0u : (uint32_t)ab * (kAccCols / 2));
             if (rvalid) {
-                for (int ch = cg; ch < t.N / 8; ch += 4) {
+                for (int ch = 0; ch < t.N / 8; ++ch) {
                     if (NMAT == 2) {
                         float g[8], u[8];
                         tmem_ld8(taddr + ch * 8, g);
@@ -645,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
+            if (lane == 0) mbar_arrive(acc_empty(ab));
             ++ic;
         }
     }
