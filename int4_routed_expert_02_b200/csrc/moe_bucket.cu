@@ -13,18 +13,38 @@
 namespace moe {
 
 constexpr int kBucketThreads = 256;
+constexpr int kBucketWarps = kBucketThreads / kWarp;
 
+// Warp w owns a contiguous block of the pairs.  Counting per (warp, expert)
+// and an exclusive sum over the warps give each warp the first position of
+// its block's pairs inside every expert's segment, so the 8 warps scatter at
+// once and the result is the same stable order (by expert, then pair id) as
+// one pass over all pairs.
 __global__ void __launch_bounds__(kBucketThreads)
 bucket_kernel(const int32_t *__restrict__ idx, int n, int E, int32_t *__restrict__ offsets,
               int32_t *__restrict__ perm, int32_t *__restrict__ inv, int32_t *__restrict__ active) {
     __shared__ int cnt[kMaxE];
     __shared__ int cursor[kMaxE];
+    __shared__ int wpos[kBucketWarps][kMaxE];  // per warp and expert: its count, then its first position
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+    for (int e = tid; e < E; e += blockDim.x)
+        for (int w = 0; w < kBucketWarps; ++w) wpos[w][e] = 0;
     __syncthreads();
-    for (int p = tid; p < n; p += blockDim.x) {
+    const int B = ((n + kBucketWarps - 1) / kBucketWarps + kWarp - 1) & ~(kWarp - 1);
+    const int p0 = min(n, wid * B), p1 = min(n, p0 + B);
+    for (int p = p0 + lane; p < p1; p += kWarp) {
         const int e = idx[p];
-        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);  // integer counts: order does not matter
+        if (e >= 0 && e < E) atomicAdd(&wpos[wid][e], 1);  // integer counts: order does not matter
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int w = 0; w < kBucketWarps; ++w) {
+            const int c = wpos[w][e];
+            wpos[w][e] = run;
+            run += c;
+        }
+        cnt[e] = run;
     }
     __syncthreads();
     if (wid == 0) {
@@ -52,25 +72,24 @@ bucket_kernel(const int32_t *__restrict__ idx, int n, int E, int32_t *__restrict
             offsets[E] = run;
             if (active) active[0] = nact;
         }
-        __syncwarp();
-        // stable scatter, 32 pairs at a time in ascending pair order
-        for (int base = 0; base < n; base += kWarp) {
-            const int p = base + lane;
-            int e = p < n ? idx[p] : -1;
-            const bool ok = e >= 0 && e < E;
-            if (!ok) e = -2 - lane;  // unique key: never matches a real expert
-            const unsigned peers = __match_any_sync(0xffffffffu, e);
-            const int rank = __popc(peers & ((1u << lane) - 1u));
-            int pos = 0;
-            if (ok) {
-                pos = cursor[e] + rank;
-                perm[pos] = p;
-                if (inv) inv[p] = pos;
-            }
-            __syncwarp();
-            if (ok && rank == 0) cursor[e] += __popc(peers);
-            __syncwarp();
+    }
+    __syncthreads();
+    // stable scatter of this warp's block, 32 pairs at a time in ascending pair order
+    for (int base = p0; base < p1; base += kWarp) {
+        const int p = base + lane;
+        int e = p < p1 ? idx[p] : -1;
+        const bool ok = e >= 0 && e < E;
+        if (!ok) e = -2 - lane;  // unique key: never matches a real expert
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        if (ok) {
+            const int pos = cursor[e] + wpos[wid][e] + rank;
+            perm[pos] = p;
+            if (inv) inv[p] = pos;
         }
+        __syncwarp();
+        if (ok && rank == 0) wpos[wid][e] += __popc(peers);
+        __syncwarp();
     }
 }
 

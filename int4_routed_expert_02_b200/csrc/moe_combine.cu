@@ -13,31 +13,56 @@
 
 namespace moe {
 
-constexpr int kCombineThreads = 256;
+constexpr int kCombineMaxThreads = 1024;  // one thread per 4 columns up to H = 4096
 
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineMaxThreads)
 combine_kernel(const float *__restrict__ y, const float *__restrict__ sh, const float *__restrict__ wts, int H, int k,
                int with_shared, const uint16_t *__restrict__ h_in, float *__restrict__ m_out,
                uint16_t *__restrict__ h_out, int post_norm, float layer_scalar, float eps) {
-    extern __shared__ float msh[];  // [H]
-    __shared__ float red[kCombineThreads / 32];
-    const int t = blockIdx.x;
-    float wk[kMaxK];
-#pragma unroll
-    for (int s = 0; s < kMaxK; ++s) wk[s] = s < k ? wts[(size_t)t * k + s] : 0.f;
+    extern __shared__ float4 msh4[];  // [H / 4]
+    __shared__ float red[kCombineMaxThreads / 32];
+    __shared__ float wk[kMaxK];
+    const int t = blockIdx.x, H4 = H / 4;
+    if (threadIdx.x < k) wk[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
+    __syncthreads();
+    const float4 *y4 = reinterpret_cast<const float4 *>(y) + (size_t)t * k * H4;
     float ss = 0.f;
-    for (int i = threadIdx.x; i < H; i += blockDim.x) {
-        float m = 0.f;
-#pragma unroll 8
-        for (int s = 0; s < k; ++s) m = fmaf(wk[s], y[((size_t)t * k + s) * H + i], m);
-        if (with_shared) m += sh[(size_t)t * H + i];
-        if (m_out) m_out[(size_t)t * H + i] = m;
-        msh[i] = m;
-        ss = fmaf(m, m, ss);
+    // four columns per thread and step; the loads of 8 routed slots (and the
+    // shared row) are issued before any is used; per column the sum runs over
+    // s = 0, 1, ... in order, then adds the shared branch
+    for (int i = threadIdx.x; i < H4; i += blockDim.x) {
+        float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < k; s0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = s0 + u < k ? __ldg(y4 + (size_t)(s0 + u) * H4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (s0 + u < k) {
+                    const float w = wk[s0 + u];
+                    m.x = fmaf(w, v[u].x, m.x);
+                    m.y = fmaf(w, v[u].y, m.y);
+                    m.z = fmaf(w, v[u].z, m.z);
+                    m.w = fmaf(w, v[u].w, m.w);
+                }
+            }
+        }
+        if (with_shared) {
+            const float4 sv = __ldg(reinterpret_cast<const float4 *>(sh) + (size_t)t * H4 + i);
+            m.x += sv.x;
+            m.y += sv.y;
+            m.z += sv.z;
+            m.w += sv.w;
+        }
+        if (m_out) reinterpret_cast<float4 *>(m_out)[(size_t)t * H4 + i] = m;
+        msh4[i] = m;
+        ss = fmaf(m.x, m.x, fmaf(m.y, m.y, fmaf(m.z, m.z, fmaf(m.w, m.w, ss))));
     }
     if (!h_out) return;
     ss = block_sum(ss, red);
     const float inv = post_norm ? 1.0f / sqrtf(ss / (float)H + eps) : 1.0f;
+    const float *msh = reinterpret_cast<const float *>(msh4);
     for (int i = threadIdx.x; i < H; i += blockDim.x) {
         const float v = (bf16_bits_to_float(h_in[(size_t)t * H + i]) + msh[i] * inv) * layer_scalar;
         h_out[(size_t)t * H + i] = f32_to_bf16_bits(v);
@@ -50,7 +75,8 @@ cudaError_t launch_combine(const float *y, const float *sh, const float *wts, in
     const size_t smem = sizeof(float) * (size_t)H;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(combine_kernel), smem);
     if (e != cudaSuccess) return e;
-    combine_kernel<<<T, kCombineThreads, smem, st>>>(y, sh, wts, H, k, with_shared, h_in, m_out, h_out, post_norm,
+    const int threads = min(kCombineMaxThreads, ((H / 4 + 31) / 32) * 32);
+    combine_kernel<<<T, threads, smem, st>>>(y, sh, wts, H, k, with_shared, h_in, m_out, h_out, post_norm,
                                                      layer_scalar, eps);
     return cudaGetLastError();
 }

@@ -15,7 +15,7 @@
 
 namespace moe {
 
-constexpr int kRouterThreads = 256;                   // 8 warps = 8 experts per CTA
+constexpr int kRouterThreads = 256;                   // 8 warps, each `epw` experts
 constexpr int kRouterRows = kRouterThreads / kWarp;
 
 // Dynamic shared memory: xsT[16][ld] (xs transposed so that lane c of a warp
@@ -25,7 +25,7 @@ constexpr int kRouterRows = kRouterThreads / kWarp;
 __global__ void __launch_bounds__(kRouterThreads)
 router_logits_kernel(const uint32_t *__restrict__ rq, const uint16_t *__restrict__ rs,
                      const uint16_t *__restrict__ rb, const uint16_t *__restrict__ router_scale,
-                     const uint16_t *__restrict__ h, int H, int E, float eps, double *__restrict__ logits,
+                     const uint16_t *__restrict__ h, int H, int E, int epw, float eps, double *__restrict__ logits,
                      uint16_t *__restrict__ xe) {
     extern __shared__ double smem_d[];
     const int nchunk = H / 16;
@@ -64,31 +64,39 @@ router_logits_kernel(const uint32_t *__restrict__ rq, const uint16_t *__restrict
     }
     __syncthreads();
 
+    // warp w takes experts blockIdx.x * 8 * epw + j * 8 + w, j < epw (the
+    // norm above is shared by all of them)
     const int lane = threadIdx.x & 31;
-    const int e = blockIdx.x * kRouterRows + (threadIdx.x >> 5);
-    if (e >= E) return;
     const int G = H / kGroup;
-    const uint32_t *row = rq + (size_t)e * (H / 4);
-    double acc = 0.0;
-    for (int c = lane; c < nchunk; c += kWarp) {
-        const uint4 q = ldg_nc_v4(row + 4 * c);
-        const int g = c >> 2;  // four 16-code chunks per group of 64
-        const double s = (double)bf16_bits_to_float(rs[(size_t)e * G + g]);
-        const double b = (double)bf16_bits_to_float(rb[(size_t)e * G + g]);
-        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-        double dot = 0.0;
+    for (int j = 0; j < epw; ++j) {
+        const int e = (blockIdx.x * epw + j) * kRouterRows + (threadIdx.x >> 5);
+        if (e >= E) break;
+        const uint32_t *row = rq + (size_t)e * (H / 4);
+        double acc = 0.0;
+        for (int c = lane; c < nchunk; c += kWarp) {
+            const uint4 q = ldg_nc_v4(row + 4 * c);
+            const int g = c >> 2;  // four 16-code chunks per group of 64
+            const double s = (double)bf16_bits_to_float(rs[(size_t)e * G + g]);
+            const double b = (double)bf16_bits_to_float(rb[(size_t)e * G + g]);
+            const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+            double dot = 0.0;
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
+            for (int wi = 0; wi < 4; ++wi) {
 #pragma unroll
-            for (int bi = 0; bi < 4; ++bi) {
-                const int m = wi * 4 + bi;
-                dot += (double)((words[wi] >> (8 * bi)) & 0xffu) * xsT[m * ld + c];
+                for (int bi = 0; bi < 4; ++bi) {
+                    const int m = wi * 4 + bi;
+                    // the 8-bit code as a double: 2^52 + q read as fp64, minus 2^52 (exact,
+                    // and an add instead of an integer-to-double conversion)
+                    const double qd =
+                        __hiloint2double(0x43300000, (int)((words[wi] >> (8 * bi)) & 0xffu)) - 4503599627370496.0;
+                    dot += qd * xsT[m * ld + c];
+                }
             }
+            acc += s * dot + b * csum[c];
         }
-        acc += s * dot + b * csum[c];
+        acc = warp_sum(acc);
+        if (lane == 0) logits[(size_t)t * E + e] = acc;
     }
-    acc = warp_sum(acc);
-    if (lane == 0) logits[(size_t)t * E + e] = acc;
 }
 
 // One warp per token.  k rounds of a warp-wide argmax over the logits not yet
@@ -153,9 +161,12 @@ cudaError_t launch_router_logits(const moe_layer_w *w, const uint16_t *h, int T,
     const size_t smem = router_logits_smem(w->H);
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(router_logits_kernel), smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((w->E + kRouterRows - 1) / kRouterRows, T);
+    // many tokens: one CTA covers 32 experts (the token's norm is computed
+    // once for them); few tokens: 8, so that more CTAs share the work
+    const int epw = T >= 16 ? 4 : 1;
+    dim3 grid((w->E + kRouterRows * epw - 1) / (kRouterRows * epw), T);
     router_logits_kernel<<<grid, kRouterThreads, smem, st>>>(w->router_q, w->router_s, w->router_b,
-                                                             w->router_scale, h, w->H, w->E, eps, logits, xe);
+                                                             w->router_scale, h, w->H, w->E, epw, eps, logits, xe);
     return cudaGetLastError();
 }
 
