@@ -17,19 +17,25 @@ from . import moe, synth
 
 class MoEStack:
     def __init__(self, cfg: synth.MoEConfig, cfg_id: int, T: int | None = None, layers: int | None = None,
-                 seed: int = 0, device="cuda", keep_router_codes: bool = False, persistent: bool | None = None):
+                 seed: int = 0, device="cuda", keep_router_codes: bool = False, persistent: bool | None = None,
+                 device_layers: list | None = None):
+        """device_layers: the weights of another stack of the same configuration
+        to share (they are not regenerated)."""
         self.cfg, self.cfg_id, self.seed = cfg, cfg_id, seed
         self.T = cfg.T if T is None else T
         self.L = cfg.layers if layers is None else layers
         self.device = torch.device(device)
         self.layers = []
         self.router_codes = []
-        for l in range(self.L):
+        for l in range(self.L if device_layers is None else 0):
             w = synth.gen_layer(cfg, cfg_id, l, seed=seed, device=self.device)
             if keep_router_codes and "router_codes" in w:
                 self.router_codes.append(w["router_codes"].cpu())
             self.layers.append(moe.DeviceLayer.from_config(w, cfg, device=self.device))
             del w
+        if device_layers is not None:
+            assert len(device_layers) >= self.L
+            self.layers = list(device_layers[:self.L])
         H = cfg.H
         fits = self.T <= 8 and H <= 4096 and self.T * H <= 24576
         self.persistent = fits if persistent is None else persistent

@@ -141,3 +141,29 @@ def test_prefill_chunk_layer_auto_path_is_deterministic():
     rows = [3, 64, 100]
     ref = oracle.layer_forward(OL, h[rows])
     assert max_err_vs_rms(bf16_host(outs[0])[rows], ref["out_f64"]) <= OUT_TOL
+
+
+def test_prefill_rows_of_eight_chunks_in_one_call():
+    """The rows of 8 chunks of 128 through a Gemma-shaped layer in ONE call
+    (T = 1024, ~64 rows per expert tile): sampled rows match the oracle, and
+    every row matches the same rows run as 8 separate 128-token chunks."""
+    cfg = synth.CONFIGS[4]
+    w, D, OL = _layer(synth.CONFIGS[1], 1, layer=5)
+    T = 1024
+    h = synth.gen_hidden(cfg, 4, 7, T)
+    hd = h.cuda()
+    out = torch.empty_like(hd)
+    ws = moe.workspace(D, T)
+    moe.moe_layer_forward(D, hd, out, T, ws)
+    torch.cuda.synchronize()
+    moe.moe_workspace_status(ws)
+    rows = [0, 127, 128, 555, 1023]
+    ref = oracle.layer_forward(OL, h[rows])
+    assert max_err_vs_rms(bf16_host(out)[rows], ref["out_f64"]) <= OUT_TOL
+    ws128 = moe.workspace(D, 128)
+    chunked = torch.empty_like(hd)
+    for c in range(8):
+        moe.moe_layer_forward(D, hd[c * 128:(c + 1) * 128], chunked[c * 128:(c + 1) * 128], 128, ws128)
+    torch.cuda.synchronize()
+    moe.moe_workspace_status(ws128)
+    assert max_err_vs_rms(bf16_host(out), bf16_host(chunked)) <= 5e-3
