@@ -49,6 +49,7 @@ def peaks():
 # per layer (2-layer capture halved); the two grouped-GEMM kernels of one
 # 128-token layer-chunk.  Reset to None whenever the kernel changes.
 DECODE_TRAFFIC_PER_LAYER = (74_531_072 + 2_422_784) // 2
+HEAD_TRAFFIC_PER_CALL = 415_259_392 + 3_848_192  # moe_qmat_gemv over the 262,144 x 2816 head, one token
 PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER = 369_931_520 + 15_747_328 + 162_025_216 + 65_058_816  # one 1024-token layer call
 PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_960_000 + 5_408_000 + 147_004_672 + 8_862_720
 
@@ -208,13 +209,15 @@ def run_ours(args, rank, world, local_rank):
 
     launches_per_step = st.launches_per_step()
     n_layers = st.L
-    prefill = prefill_fused = None
+    prefill = prefill_fused = head = None
     if args.prefill and world == 1 and args.config == 1 and not args.layers:
         del st
         torch.cuda.empty_cache()
         prefill, pst = prefill_measure(dev)
         prefill_fused, _ = prefill_measure(dev, chunks=2, T=1024, share=pst)
         del pst
+        torch.cuda.empty_cache()
+        head = head_measure(dev)
     res = {
         "metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -230,6 +233,7 @@ def run_ours(args, rank, world, local_rank):
     if prefill is not None:
         res["prefill"] = prefill
         res["prefill_fused"] = prefill_fused
+        res["output_head"] = head
     return res
 
 
@@ -338,6 +342,43 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None):
                            "hbm_frac": roof["frac"], "bytes_per_launch": roof["bytes_per_launch"],
                            "traffic": traffic,
                            "peak_source": hbm["source"] + " (bf16 dense burst; FP16 same rate; copy bandwidth)"}}, st
+
+
+HEAD_ROWS = 262_144  # vocabulary rows of the output head (synthetic: the pages give no vocabulary size)
+
+
+def head_measure(dev, reps=50, warmup=5):
+    """The output head that shares the embedding's quantised weights: one
+    4-bit [262,144 x 2816] matrix times one token (moe_qmat_gemv), against the
+    HBM roofline (4.5 bits per weight, every byte read once per call)."""
+    from int4_routed_expert_02_b200 import moe
+    cfg = synth.CONFIGS[1]
+    V, H = HEAD_ROWS, cfg.H
+    w = synth.gen_vocab_head(cfg, 1, V, device=dev)
+    qt, sbt = moe.prepare_qmat(w["head_q"], w["head_s"], w["head_b"], 1, V, H)
+    del w
+    x = synth.gen_hidden(cfg, 1, 30_000, 1, device=dev)
+    y = torch.empty(1, V, dtype=torch.float32, device=dev)
+    ws = moe.qmat_gemv_workspace(device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        moe.moe_qmat_gemv(qt, sbt, V, H, x, 1, y, ws)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        moe.moe_qmat_gemv(qt, sbt, V, H, x, 1, y, ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = int(expert_bytes(V * H) + V * 4 + H * 2)  # weights + fp32 output + bf16 input
+    hbm = peaks()
+    gbs = nbytes / (us / 1e6) / 1e9
+    return {"workload": f"output head sharing the embedding's 4-bit weights: {V} x {H}, 1 token per call",
+            "kernel": "qmat_gemv_kernel (dequant-GEMV, one 32-row block per warp at a time)",
+            "us_per_call": round(us, 2), "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm["hbm_gbs"],
+            "unit": "GB/s", "frac": round(gbs / hbm["hbm_gbs"], 4), "bytes_per_call": nbytes,
+            "traffic": HEAD_TRAFFIC_PER_CALL, "peak_source": hbm["source"] + " (burst copy)"}
 
 
 def _e2e(st, cfg, T, K, W, inputs, dev):
@@ -462,6 +503,8 @@ def main():
                     help="profiling only: build this many layers instead of the config's (not a bench line)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head-only", action="store_true",
+                    help="profiling only: time the output-head GEMV alone and print its object")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false",
                     help="skip the chunked-prefill measurement that the default line carries")
     args = ap.parse_args()
@@ -479,6 +522,10 @@ def main():
     try:
         if args.impl == "reference":
             res = run_reference(args, rank, world)
+        elif args.head_only:
+            from int4_routed_expert_02_b200 import build
+            build.build()
+            res = {"output_head": head_measure(torch.device("cuda", local_rank))} if rank == 0 else None
         else:
             res = run_ours(args, rank, world, local_rank)
         if rank == 0 and res is not None:

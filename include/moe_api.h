@@ -220,6 +220,29 @@ MOE_API int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h
 MOE_API int moe_decode_stack_status(const void *ws);
 
 /*
+ * y[t][r] = sum_c W[r][c] * x[t][c] for ONE 4-bit MLX-affine matrix W
+ * [rows, cols] in the tiled layout (moe_prepare_qmat with n_mat = 1), e.g. the
+ * vocabulary-sized output head that shares the embedding's quantised weights
+ * (TurboFieldfare introduction page, section "How TurboFieldfare saves
+ * memory": embedding and language-model head share one quantised weight; the
+ * decode-time table there lists that head at 14.2 ms of a 162.8 ms step).
+ *   w        : device pointers q (codes) and sb (scale | bias << 16 words).
+ *   rows     : a positive multiple of 32 (the vocabulary size for a head).
+ *   cols     : a multiple of 64 in [64, 8192] (the hidden size).
+ *   x [T, cols] bf16, y [T, rows] fp32, 1 <= T <= 8, all device, 16-byte aligned.
+ *   ws       : moe_qmat_gemv_workspace_size() bytes of device memory, 16-byte
+ *              aligned; the call resets it (a work counter); calls that overlap
+ *              on the GPU need workspaces of their own.
+ * Each weight group's products are exact (the code times the pre-scaled input)
+ * and accumulate in fp32.  Asynchronous on `stream`; MOE_EINVAL / MOE_EALIGN /
+ * MOE_EWORKSPACE on bad arguments, MOE_ECUDA on a launch failure.
+ */
+MOE_API size_t moe_qmat_gemv_workspace_size(void);
+
+MOE_API int moe_qmat_gemv(const moe_qmat *w, int rows, int cols, const uint16_t *x, int T, float *y, void *ws,
+                          size_t ws_bytes, void *stream);
+
+/*
  * moe_layer_forward for callers that cannot allocate device memory.  (The
  * pages have no counterpart: this is a deployment convenience.)
  *

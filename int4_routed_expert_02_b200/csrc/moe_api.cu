@@ -424,6 +424,31 @@ int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
 }
 
+size_t moe_qmat_gemv_workspace_size(void) { return 256; }
+
+int moe_qmat_gemv(const moe_qmat *w, int rows, int cols, const uint16_t *x, int T, float *y, void *ws,
+                  size_t ws_bytes, void *stream) {
+    const char *fn = "moe_qmat_gemv";
+    g_err.clear();
+    if (!w) return fail(MOE_EINVAL, "%s: matrix is NULL", fn);
+    if (rows < 32 || rows % 32) return fail(MOE_EINVAL, "%s: rows=%d must be a positive multiple of 32", fn, rows);
+    if (cols < 64 || cols % 64 || cols > kMaxDim)
+        return fail(MOE_EINVAL, "%s: cols=%d must be a multiple of 64 in [64, %d]", fn, cols, kMaxDim);
+    if (T < 1 || T > 8) return fail(MOE_EINVAL, "%s: T=%d must be in [1, 8]", fn, T);
+    if (moe::qmat_gemv_smem(cols, T) > (size_t)200 * 1024)
+        return fail(MOE_EINVAL, "%s: T=%d rows of %d columns do not fit the shared-memory stage", fn, T, cols);
+    CHECK_PTR(w->q);
+    CHECK_PTR(w->sb);
+    CHECK_PTR(x);
+    CHECK_PTR(y);
+    CHECK_PTR(ws);
+    if (ws_bytes < moe_qmat_gemv_workspace_size())
+        return fail(MOE_EWORKSPACE, "%s: workspace of %zu bytes, need %zu", fn, ws_bytes, moe_qmat_gemv_workspace_size());
+    cudaError_t e = moe::launch_qmat_gemv(*w, rows, cols, x, T, y, static_cast<unsigned *>(ws),
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
 int moe_workspace_status(const void *ws) {
     const char *fn = "moe_workspace_status";
     g_err.clear();

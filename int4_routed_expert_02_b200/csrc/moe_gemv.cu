@@ -330,6 +330,83 @@ static cudaError_t launch_ffn_nt(const ExpertParams &P, int max_active, cudaStre
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ one large matrix
+// y[t][r] = sum_c W[r][c] x[t][c] for a single tiled 4-bit matrix W [rows,
+// cols], e.g. the vocabulary-sized output head that shares the embedding's
+// quantised weights (TurboFieldfare introduction page, section "How
+// TurboFieldfare saves memory": the embedding and the language-model head
+// share the same quantised weights; the decode-time table there puts that
+// head at 14.2 ms of a 162.8 ms step).  Pure streaming: every byte of W is
+// read once, so the kernel is HBM-bound.  Each CTA stages x once; its warps
+// then take 32-row blocks one at a time from a global counter (all rows of a
+// block, every column), so no warp idles while another still streams.
+constexpr int kQgWarps = 8;
+
+template <int NT>
+__global__ void __launch_bounds__(kQgWarps * 32)
+qmat_gemv_kernel(const uint32_t *__restrict__ q, const uint32_t *__restrict__ sb, int rows, int cols,
+                 const uint16_t *__restrict__ x, int T, float *__restrict__ y, unsigned *__restrict__ ctr) {
+    extern __shared__ __align__(16) float smem_f[];
+    const int C = cols / kChunkCols, G = cols / kGroup, nrb = rows / kRowBlock;
+    Stage S{smem_f, smem_f + (size_t)NT * cols, cols, C};
+    for (int i = threadIdx.x; i < NT * cols; i += blockDim.x) {
+        const int tt = i / cols, col = i - tt * cols;
+        const float v = tt < T ? bf16_bits_to_float(x[(size_t)tt * cols + col]) : 0.f;
+        S.xp[i] = v * code_prescale(col & 7);
+    }
+    __syncthreads();
+    stage_chunk_sums<NT>(S, kQgWarps);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (;;) {
+        int rb = 0;
+        if (lane == 0) rb = (int)atomicAdd(ctr, 1u);
+        rb = __shfl_sync(0xffffffffu, rb, 0);
+        if (rb >= nrb) break;
+        const uint32_t *qq[1] = {q + (size_t)rb * C * 128};
+        const uint32_t *ss[1] = {sb + (size_t)rb * G * 32};
+        float acc[1][NT];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) acc[0][tt] = 0.f;
+        gemv_slice<NT, 1>(qq, ss, S, T, 0, G, acc);
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt)
+            if (tt < T) y[(size_t)tt * rows + (size_t)rb * kRowBlock + lane] = acc[0][tt];
+    }
+}
+
+size_t qmat_gemv_smem(int cols, int T) {
+    const int nt = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
+    return stage_bytes(cols, nt, 0);
+}
+
+template <int NT>
+static cudaError_t launch_qmat_gemv_nt(const moe_qmat &w, int rows, int cols, const uint16_t *x, int T, float *y,
+                                       unsigned *ctr, cudaStream_t st) {
+    const size_t smem = stage_bytes(cols, NT, 0);
+    const void *fn = reinterpret_cast<const void *>(qmat_gemv_kernel<NT>);
+    cudaError_t e = ensure_smem(fn, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kQgWarps * 32, smem)) != cudaSuccess) return e;
+    const int nrb = rows / kRowBlock;
+    int grid = sms * (per > 0 ? per : 1);
+    if (grid * kQgWarps > nrb) grid = (nrb + kQgWarps - 1) / kQgWarps;
+    if ((e = cudaMemsetAsync(ctr, 0, sizeof(unsigned), st)) != cudaSuccess) return e;
+    qmat_gemv_kernel<NT><<<grid, kQgWarps * 32, smem, st>>>(w.q, w.sb, rows, cols, x, T, y, ctr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qmat_gemv(const moe_qmat &w, int rows, int cols, const uint16_t *x, int T, float *y,
+                             unsigned *ctr, cudaStream_t st) {
+    if (T <= 1) return launch_qmat_gemv_nt<1>(w, rows, cols, x, T, y, ctr, st);
+    if (T <= 2) return launch_qmat_gemv_nt<2>(w, rows, cols, x, T, y, ctr, st);
+    if (T <= 4) return launch_qmat_gemv_nt<4>(w, rows, cols, x, T, y, ctr, st);
+    return launch_qmat_gemv_nt<8>(w, rows, cols, x, T, y, ctr, st);
+}
+
 cudaError_t launch_expert_gemv(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
                                const int32_t *perm, const int32_t *active, int with_shared, const FfnBuffers &b,
                                cudaStream_t st) {

@@ -38,6 +38,10 @@ size_t gemv_smem_bytes(int cols, int nt);
 cudaError_t launch_expert_gemv(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
                                const int32_t *perm, const int32_t *active, int with_shared, const FfnBuffers &b,
                                cudaStream_t st);
+// One tiled 4-bit matrix times up to 8 bf16 rows (moe_gemv.cu); ctr: a device word (reset by the launch).
+size_t qmat_gemv_smem(int cols, int T);
+cudaError_t launch_qmat_gemv(const moe_qmat &w, int rows, int cols, const uint16_t *x, int T, float *y,
+                             unsigned *ctr, cudaStream_t st);
 // Tensor-core grouped GEMM path (moe_mma.cu).
 struct MmaBuffers {
     uint16_t *xg;   // [T + T*k, H]    FP16 token rows (shared, then bucketed pairs), chunk-permuted

@@ -23,7 +23,8 @@ MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_ECUDA, MOE_EDEVICE = 0, -1, 
 EXPORTED = ("moe_last_error", "moe_version", "moe_prepare_qmat", "moe_workspace_size", "moe_router_logits",
             "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward",
             "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc", "moe_decode_stack_workspace_size",
-            "moe_decode_stack", "moe_decode_stack_status", "moe_workspace_status")
+            "moe_decode_stack", "moe_decode_stack_status", "moe_workspace_status", "moe_qmat_gemv_workspace_size",
+            "moe_qmat_gemv")
 
 
 class MoEError(RuntimeError):
@@ -67,6 +68,8 @@ _lib.moe_decode_stack.argtypes = [_P, _I, _P, _I, _P, _I, _P, C.c_size_t, _P, _P
 _lib.moe_decode_stack_status.argtypes = [_P]
 _lib.moe_workspace_status.argtypes = [_P]
 _lib.moe_layer_forward_noalloc.argtypes = [_P, _P, _P, _I, _P, _P]
+_lib.moe_qmat_gemv_workspace_size.restype = C.c_size_t
+_lib.moe_qmat_gemv.argtypes = [_P, _I, _I, _P, _I, _P, _P, C.c_size_t, _P]
 
 
 def lib():
@@ -189,6 +192,17 @@ def moe_router_topk(logits, T, E, k, per_expert_scale, idx, wts, stream=None):
 def moe_router(layer, h, T, idx, wts, xe, ws, stream=None):
     _check(_lib.moe_router(layer.ptr(), _ptr(h), T, _ptr(idx), _ptr(wts), _ptr(xe), _ptr(ws),
                            ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+def moe_qmat_gemv(q_tiled, sb_tiled, rows, cols, x, T, y, ws, stream=None):
+    """y[T, rows] (fp32) = W x for one tiled 4-bit matrix (prepare_qmat with n_mat = 1)."""
+    m = QMat(q_tiled.data_ptr(), sb_tiled.data_ptr())
+    _check(_lib.moe_qmat_gemv(C.byref(m), rows, cols, _ptr(x), T, _ptr(y), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def qmat_gemv_workspace(device="cuda") -> torch.Tensor:
+    return torch.empty(int(_lib.moe_qmat_gemv_workspace_size()), dtype=torch.uint8, device=device)
 
 
 def moe_bucket(idx, T, k, E, offsets, perm, inv=None, active=None, stream=None):

@@ -68,6 +68,7 @@ _TENSOR_IDS = {
     "sh_up_q": 23, "sh_up_s": 24, "sh_up_b": 25,
     "sh_down_q": 26, "sh_down_s": 27, "sh_down_b": 28,
     "hidden": 40, "zipf_perm": 41, "zipf_gumbel": 42,
+    "head_q": 50, "head_s": 51, "head_b": 52,
 }
 
 _MASK64 = (1 << 64) - 1
@@ -184,6 +185,14 @@ def gen_experts(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="
         out[name + "_q"], out[name + "_s"], out[name + "_b"] = _qmat(name, 1, rows, cols, 4, cfg_id, layer,
                                                                       seed, device, lead=False)
     return out
+
+
+def gen_vocab_head(cfg: MoEConfig, cfg_id: int, V: int, seed: int = 0, device="cpu") -> dict:
+    """A vocabulary-sized 4-bit matrix [V, H] (MLX layout), drawn like the
+    expert matrices: the output head that shares the embedding's quantised
+    weights.  head_q [V, H/8], head_s / head_b [V, H/64]."""
+    q, s, b = _qmat("head", 1, V, cfg.H, 4, cfg_id, 0, seed, device, lead=False)
+    return {"head_q": q, "head_s": s, "head_b": b}
 
 
 def gen_layer(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="cpu") -> dict:

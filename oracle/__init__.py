@@ -57,6 +57,7 @@ def lib():
             L.oracle_double_to_bf16.restype = C.c_uint16
             L.oracle_double_to_bf16.argtypes = [C.c_double]
             L.oracle_dequant.argtypes = [P, P, P, I, I, I, P]
+            L.oracle_qmat_gemv.argtypes = [P, P, P, I, I, I, P, I, P]
             L.oracle_rmsnorm_no_scale.argtypes = [P, I, C.c_double, P]
             L.oracle_rmsnorm_no_scale.restype = None
             L.oracle_topk.argtypes = [P, I, I, P]
@@ -131,6 +132,16 @@ def dequant(q, s, b, rows, cols, bits) -> np.ndarray:
     rc = lib().oracle_dequant(_p(qa), _p(sa), _p(ba), rows, cols, bits, _p(out))
     assert rc == 0
     return out
+
+
+def qmat_gemv(q, s, b, rows, cols, x, bits=4) -> np.ndarray:
+    """Y [T, rows] = dequant(W) x for x [T, cols] (fp64), one matrix in MLX layout."""
+    xa = np.ascontiguousarray(np.atleast_2d(x), np.float64)
+    qa, sa, ba = _np(q, np.uint32), _np(s, np.uint16), _np(b, np.uint16)
+    y = np.empty((xa.shape[0], rows), np.float64)
+    rc = lib().oracle_qmat_gemv(_p(qa), _p(sa), _p(ba), rows, cols, bits, _p(xa), xa.shape[0], _p(y))
+    assert rc == 0
+    return y
 
 
 def rmsnorm_no_scale(h, eps=EPS) -> np.ndarray:

@@ -125,6 +125,18 @@ static void qmatvec(const uint32_t *q, const uint16_t *s, const uint16_t *b, int
     }
 }
 
+/* Y[t][r] = sum_c deq(W[r, c]) * X[t][c] for T input rows: one quantised
+ * matrix applied to T vectors, e.g. the vocabulary-sized output head that
+ * shares the embedding's quantised weights (TurboFieldfare page, "How
+ * TurboFieldfare saves memory"). */
+int oracle_qmat_gemv(const uint32_t *q, const uint16_t *s, const uint16_t *b, int rows, int cols, int bits,
+                     const double *x, int T, double *y)
+{
+    if (cols % 64 || (bits != 4 && bits != 8) || rows < 0 || T < 0) return ORACLE_EINVAL;
+    for (int t = 0; t < T; ++t) qmatvec(q, s, b, rows, cols, bits, x + (size_t)t * cols, y + (size_t)t * rows);
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------ router */
 
 /* rmsnorm_no_scale (router pseudo-code, first line): xn = h / sqrt(mean(h^2) + eps).

@@ -98,6 +98,53 @@ def test_dequant_matches_packed_codes():
         assert np.array_equal(oracle.dequant(q, s, b, 3, 192, bits), want)
 
 
+# ------------------------------------------------------- one quantised matrix
+
+@pytest.mark.parametrize("row", _golden_rows(), ids=lambda r: f"{r[0]}bit-{r[1]:#010x}")
+def test_qmat_gemv_worked_example(row):
+    """One row of the worked example times x = (1, 2, 3, ...): the hand-computed
+    values weighted by their column number (the rest of the group is the bias)."""
+    bits, word, s, b, codes, vals = row
+    per = 32 // bits
+    q = np.zeros((1, 64 * bits // 32), np.uint32)
+    q[0, 0] = word
+    x = np.arange(1, 65, dtype=np.float64)
+    want = sum(v * (c + 1) for c, v in enumerate(vals)) + b * sum(range(per + 1, 65))
+    assert oracle.qmat_gemv(q, bf16([s]), bf16([b]), 1, 64, x, bits=bits)[0, 0] == want
+
+
+def test_qmat_gemv_unit_vectors_give_the_columns():
+    rng = np.random.default_rng(4)
+    rows, cols = 5, 128
+    codes = rng.integers(0, 16, size=(rows, cols))
+    q = synth.pack_codes(torch.from_numpy(codes), 4).numpy().view(np.uint32)
+    s = bf16(rng.uniform(0.01, 0.05, size=rows * 2))
+    b = bf16(rng.uniform(-0.5, 0.5, size=rows * 2))
+    sd, bd = oracle.bf16_to_f64(s).reshape(rows, 2), oracle.bf16_to_f64(b).reshape(rows, 2)
+    for j in (0, 63, 64, 127):
+        e = np.zeros(cols)
+        e[j] = 1.0
+        y = oracle.qmat_gemv(q, s, b, rows, cols, e)[0]
+        assert np.array_equal(y, sd[:, j // 64] * codes[:, j] + bd[:, j // 64])
+
+
+def test_qmat_gemv_bias_only_and_linearity():
+    rows, cols = 3, 192
+    q = np.zeros((rows, cols // 8), np.uint32)   # every code 0: W = bias of each group
+    b = bf16([1.0, -2.0, 0.5, 4.0, 0.25, -1.0, 3.0, 2.0, -0.5])
+    s = bf16([0.125] * 9)
+    x = np.arange(cols, dtype=np.float64)
+    gsum = x.reshape(3, 64).sum(axis=1)
+    bd = oracle.bf16_to_f64(b).reshape(rows, 3)
+    assert np.array_equal(oracle.qmat_gemv(q, s, b, rows, cols, x)[0], bd @ gsum)
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 16, size=(rows, cols))
+    q = synth.pack_codes(torch.from_numpy(codes), 4).numpy().view(np.uint32)
+    x1, x2 = rng.standard_normal(cols), rng.standard_normal(cols)
+    y = oracle.qmat_gemv(q, s, b, rows, cols, np.stack([x1, x2, 2.0 * x1 - 3.0 * x2]))
+    assert np.allclose(y[2], 2.0 * y[0] - 3.0 * y[1], rtol=1e-12, atol=1e-12)
+
+
 # ----------------------------------------------------------------- rmsnorm
 
 def test_rmsnorm_constant_vector_closed_form():
