@@ -140,3 +140,24 @@ def test_decode_stack_validation():
     assert _stack([a], 1, 2, ws_bytes=16) == moe.MOE_EWORKSPACE
     assert moe.lib().moe_decode_stack_workspace_size(C.addressof(a), 9) == 0
     assert moe.lib().moe_decode_stack_workspace_size(C.addressof(a), 8) > 0
+
+
+def test_qmat_gemv_validation():
+    L = moe.lib()
+    ws = L.moe_qmat_gemv_workspace_size()
+    assert ws >= 4
+    m = moe.QMat(FAKE, FAKE)
+
+    def call(rows, cols, T, x=FAKE, y=FAKE, wsp=FAKE, wsb=ws, mat=m):
+        return L.moe_qmat_gemv(C.byref(mat) if mat is not None else None, rows, cols, x, T, y, wsp, wsb, None)
+
+    assert call(48, 64, 1) == moe.MOE_EINVAL                     # rows not a multiple of 32
+    assert call(64, 96, 1) == moe.MOE_EINVAL                     # cols not a multiple of 64
+    assert call(64, 16384, 1) == moe.MOE_EINVAL                  # cols above the limit
+    assert call(64, 64, 0) == moe.MOE_EINVAL and call(64, 64, 9) == moe.MOE_EINVAL
+    assert call(64, 8192, 8) == moe.MOE_EINVAL and "shared-memory" in moe.last_error()
+    assert call(64, 64, 1, mat=None) == moe.MOE_EINVAL
+    assert call(64, 64, 1, mat=moe.QMat(FAKE + 4, FAKE)) == moe.MOE_EALIGN
+    assert call(64, 64, 1, x=FAKE + 2) == moe.MOE_EALIGN
+    assert call(64, 64, 1, y=None) == moe.MOE_EINVAL
+    assert call(64, 64, 1, wsb=ws - 1) == moe.MOE_EWORKSPACE
