@@ -1,18 +1,28 @@
 """Benchmark of the int4 routed-expert MoE layer stack on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C] [--tokens T]
 
-Workload (default, config 1): Gemma-4-26B-A4B-shaped decode -- 30 stacked MoE
+Headline workload (config 1): Gemma-4-26B-A4B-shaped decode -- 30 stacked MoE
 layers, H=2816, E=128 experts, top-8, expert intermediate 704, shared expert
 intermediate 2112, one token per step, a fresh N(0,1) hidden row per step,
 random weights drawn as the tiny configuration (synthetic, seeded).  One step
 = one token through all layers (router, bucketing, routed + shared experts,
-combine) replayed as one CUDA graph.  Weights (13.2 GB) are far larger than
-L2 and each step touches 1.1 GB of them, so no step finds its weights in L2.
+combine, post-norm, residual) in one persistent kernel launch.  Weights
+(13.2 GB) are far larger than L2 and each step touches 1.1 GB of them, so no
+step finds its weights in L2.
 
-Prints one JSON line.  `value` is tokens/s over all ranks (each rank runs an
-independent replica: the layer fits one GPU, so multi-GPU is replicas only).
-`--impl reference` times the fp64 CPU oracle on the host cores instead.
+The default line also carries every other configuration of the workload set,
+each with its own roofline, end-to-end number and oracle baseline:
+  configs.tiny_T4            hidden 256, 16 experts, top-4, 4 tokens (latency; L2-resident)
+  configs.qwen35b_T1/T4/T8   40 layers, H=2048, 256 experts, top-8, decode batches of 1, 4, 8
+  configs.qwen80b_zipf_T1    48 layers, H=2048, 512 experts, top-10, Zipf(1.1) expert popularity
+  prefill                    8 chunks of 128 tokens through the 30 Gemma-shaped layers
+  prefill_fused              the same 1024 rows through each layer in one call
+  prefill_batch64            64-token decode batches on the Gemma shape
+  output_head                the 262,144 x 2816 4-bit head GEMV
+`value` is tokens/s over all ranks (each rank runs an independent replica:
+the layer fits one GPU, so multi-GPU is replicas only).  `--impl reference`
+times the fp64 CPU oracle on the host cores instead.
 """
 from __future__ import annotations
 
@@ -33,6 +43,7 @@ sys.path.insert(0, ROOT)
 from int4_routed_expert_02_b200 import synth  # noqa: E402
 
 METRIC = "MoE-layer decode tok/s + HBM GB/s vs peak; prefill-chunk TFLOP/s vs peak"
+TINY_REDRAWS = os.path.join(ROOT, "tests", "golden", "tiny_redraws.txt")
 
 
 def peaks():
@@ -45,10 +56,9 @@ def peaks():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu
-# capture, per unit of work: decode_stack_kernel at the Gemma shape, T = 1,
-# per layer (2-layer capture halved); the two grouped-GEMM kernels of one
-# 128-token layer-chunk.  Reset to None whenever the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = (74_531_072 + 2_422_784) // 2
+# capture, per unit of work; None where no capture of the current kernel
+# exists.  Reset to None whenever the kernel changes.
+DECODE_TRAFFIC_PER_LAYER = None   # decode_stack_kernel, Gemma shape, T = 1, per layer
 HEAD_TRAFFIC_PER_CALL = 415_259_392 + 3_848_192  # moe_qmat_gemv over the 262,144 x 2816 head, one token
 PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER = 369_931_520 + 15_747_328 + 162_025_216 + 65_058_816  # one 1024-token layer call
 PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_960_000 + 5_408_000 + 147_004_672 + 8_862_720
@@ -60,7 +70,7 @@ def expert_bytes(rows_cols: int) -> float:
     return rows_cols * 0.5 + rows_cols / 64 * 4
 
 
-def layer_bytes(cfg, distinct_experts: int) -> dict:
+def layer_bytes(cfg, distinct_experts: float) -> dict:
     H, E, I, Is = cfg.H, cfg.E, cfg.I, cfg.Is
     routed = distinct_experts * expert_bytes(3 * I * H)
     shared = expert_bytes(3 * Is * H)
@@ -68,9 +78,23 @@ def layer_bytes(cfg, distinct_experts: int) -> dict:
     return dict(routed=routed, shared=shared, router=router, total=routed + shared + router)
 
 
-def workload_name(cfg, T):
-    return (f"{cfg.name}: {cfg.layers} MoE layers, H={cfg.H}, E={cfg.E}, top-{cfg.k}, I={cfg.I}, "
-            f"shared I={cfg.Is}, T={T} token(s) per step")
+def pool_bytes(cfg) -> float:
+    return cfg.layers * layer_bytes(cfg, cfg.E)["total"]
+
+
+def workload_name(cfg, T, layers=None):
+    L = cfg.layers if layers is None else layers
+    extra = ", Zipf(%.1f) expert popularity" % cfg.zipf if cfg.zipf else ""
+    return (f"{cfg.name}: {L} MoE layers, H={cfg.H}, E={cfg.E}, top-{cfg.k}, I={cfg.I}, "
+            f"shared I={cfg.Is}, T={T} token(s) per step{extra}")
+
+
+def l2_note(cfg, step_bytes):
+    pool = pool_bytes(cfg)
+    if pool < 100e6:
+        return f"weights ({pool / 1e6:.2f} MB) fit in L2: a latency figure, no HBM roofline claim"
+    return (f"inputs larger than L2 ({pool / 1e9:.1f} GB of weights, {step_bytes / 1e9:.2f} GB touched per step; "
+            f"each layer's weights are revisited only a whole stack later)")
 
 
 class ClockSampler:
@@ -118,140 +142,48 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
-# --------------------------------------------------------------------------- ours
+# --------------------------------------------------------------------------- inputs
 
-def run_ours(args, rank, world, local_rank):
-    from int4_routed_expert_02_b200 import build
-    if rank == 0 or not os.path.exists(build.LIB):
-        build.build()
-    if world > 1:
-        torch.distributed.barrier()
-    from int4_routed_expert_02_b200 import moe
-    from int4_routed_expert_02_b200.stack import MoEStack
+class Inputs:
+    """Device-resident inputs of every step of a decode run (generated up front)."""
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    cfg = synth.CONFIGS[args.config]
-    T = args.tokens or cfg.T
-    st = MoEStack(cfg, args.config, T=T, layers=args.layers or None, device=dev, keep_router_codes=cfg.zipf > 0)
-    K, W = args.steps, args.warmup
-
-    # one fresh input per step, generated up front (device-resident)
-    def make_input(step):
+    def __init__(self, cfg, cfg_id, st, T, n_steps, rank, dev):
+        self.cfg = cfg
         if cfg.zipf > 0:
-            rows = [synth.gen_zipf_hidden(cfg, args.config, l, step, st.router_codes[l], T=T)[0]
-                    for l in range(st.L)]
-            return torch.stack(rows).to(dev)
-        return synth.gen_hidden(cfg, args.config, 10_000 + step + rank * 1_000_000, T, device=dev)
+            centred = [c.to(torch.float64) - 128.0 for c in st.router_codes]
+            self.h = [torch.stack([synth.gen_zipf_hidden(cfg, cfg_id, l, s, st.router_codes[l], T=T,
+                                                         centred=centred[l])[0] for l in range(st.L)]).to(dev)
+                      for s in range(n_steps)]
+        elif cfg_id == 0:
+            red = synth.load_redraws(TINY_REDRAWS)
+            self.h = [synth.gen_hidden_redrawn(cfg, 0, 10_000 + s, T, red, device=dev) for s in range(n_steps)]
+        else:
+            self.h = [synth.gen_hidden(cfg, cfg_id, 10_000 + s + rank * 1_000_000, T, device=dev)
+                      for s in range(n_steps)]
 
-    inputs = [make_input(s) for s in range(W + K)]
-    stream = torch.cuda.current_stream(dev)
-    st.capture()
+    def __getitem__(self, i):
+        return self.h[i]
 
-    def step(i):
-        st.set_input(inputs[i])
-        st.run()
 
-    for i in range(W):
-        step(i)
-    torch.cuda.synchronize(dev)
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    if rank == 0:
-        clocks.start()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(K):
-        step(W + i)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop() if rank == 0 else None
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    ms_per_step = ms / K
-    tok_s = world * T * K / (ms / 1e3)
-
-    # algorithmic bytes: distinct experts actually selected, per layer, per step
-    distinct = T * cfg.k if T == 1 else _distinct_experts(st, moe, cfg, T)
-    step_bytes = st.L * layer_bytes(cfg, distinct)["total"]
-    hbm = peaks()
-    gbs = step_bytes / (ms_per_step / 1e3) / 1e9
-
-    st.status()
-    # dominant kernel: the persistent decode kernel is the whole step (one
-    # launch); otherwise the expert GEMVs, timed per launch on the same inputs
-    if st.persistent:
-        achieved = step_bytes / (ms_per_step / 1e3) / 1e9
-        roof = {"kernel": "decode_stack_kernel (persistent: all layers of a step in one cooperative launch)",
-                "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / hbm["hbm_gbs"], 4), "peak_source": hbm["source"] + " (burst copy)",
-                "traffic": (int(DECODE_TRAFFIC_PER_LAYER * st.L)
-                            if DECODE_TRAFFIC_PER_LAYER and args.config == 1 and T == 1 else None),
-                "bytes_per_launch": int(step_bytes), "us_per_launch": round(ms_per_step * 1e3, 2)}
-    else:
-        roof = _expert_roofline(st, moe, cfg, T, hbm, dev)
-
-    # end to end through the C ABI with host buffers: pinned input -> device,
-    # all layers, result -> pinned host buffer, every step
-    e2e = _e2e(st, cfg, T, K, W, inputs, dev)
-
-    # cpu baseline (oracle) on rank 0 at N = 1 only
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(cfg, args.config, T, budget_s=args.cpu_budget)
-
-    launches_per_step = st.launches_per_step()
-    n_layers = st.L
-    prefill = prefill_fused = head = None
-    if args.prefill and world == 1 and args.config == 1 and not args.layers:
-        del st
-        torch.cuda.empty_cache()
-        prefill, pst = prefill_measure(dev)
-        prefill_fused, _ = prefill_measure(dev, chunks=2, T=1024, share=pst)
-        del pst
-        torch.cuda.empty_cache()
-        head = head_measure(dev)
-    res = {
-        "metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights, bf16 activations, fp32 accumulate (router fp64)", "data": "synthetic",
-        "config": {"workload": workload_name(cfg, T), "config_id": args.config, "layers": n_layers, "tokens_per_step": T,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (13.2 GB of weights, 1.1 GB touched per step)"},
-        "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm["hbm_gbs"], 4),
-        "bytes_per_step": int(step_bytes),
-        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
-        "clocks": clk,
-    }
-    if prefill is not None:
-        res["prefill"] = prefill
-        res["prefill_fused"] = prefill_fused
-        res["output_head"] = head
-    return res
-
+# --------------------------------------------------------------------------- ours
 
 def _distinct_experts(st, moe, cfg, T):
     """Mean number of distinct experts per layer for the last step's routing."""
-    ws = st.ws
+    if T == 1:
+        return float(cfg.k)
     tot = 0
     for l in range(st.L):
         idx = torch.empty(T, cfg.k, dtype=torch.int32, device=st.device)
         wts = torch.empty(T, cfg.k, dtype=torch.float32, device=st.device)
-        moe.moe_router(st.layers[l], st.inputs[l], T, idx, wts, None, ws)
+        moe.moe_router(st.layers[l], st.inputs[l], T, idx, wts, None, st.ws)
         tot += int(torch.unique(idx).numel())
     return tot / st.L
 
 
 def _expert_roofline(st, moe, cfg, T, hbm, dev):
-    """Per-launch time of the expert part (gate/up GEMV + down GEMV + weighted
-    sum: three launches of moe_expert_ffn) on each layer's real input."""
+    """Per-launch time of the expert part (moe_expert_ffn: gate/up + down +
+    weighted sum) on each layer's real input, against the HBM roofline of
+    the distinct experts it reads."""
     L = st.L
     bufs = []
     for l in range(L):
@@ -278,18 +210,118 @@ def _expert_roofline(st, moe, cfg, T, hbm, dev):
             moe.moe_expert_ffn(st.layers[l], xe, T, idx, wts, offsets, perm, active, 1, m, ws2)
             b.record(stream)
     torch.cuda.synchronize(dev)
+    moe.moe_workspace_status(ws2)
     times = [a.elapsed_time(b) for a, b in evs[L:]]  # drop the first (warm) repetition
     us = statistics.mean(times) * 1e3
-    if T == 1:
-        nbytes = cfg.k * expert_bytes(3 * cfg.I * cfg.H) + expert_bytes(3 * cfg.Is * cfg.H)
-    else:
-        d = statistics.mean(int(torch.unique(bufs[l][1]).numel()) for l in range(L))
-        nbytes = d * expert_bytes(3 * cfg.I * cfg.H) + expert_bytes(3 * cfg.Is * cfg.H)
+    d = statistics.mean(int(torch.unique(bufs[l][1]).numel()) for l in range(L))
+    nbytes = d * expert_bytes(3 * cfg.I * cfg.H) + expert_bytes(3 * cfg.Is * cfg.H)
     achieved = nbytes / (us / 1e6) / 1e9
-    return {"kernel": "expert FFN: gate/up dequant-GEMV + down dequant-GEMV + weighted sum (moe_expert_ffn)",
-            "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / hbm["hbm_gbs"], 4), "peak_source": hbm["source"] + " (burst copy)",
-            "traffic": None, "bytes_per_launch": int(nbytes), "us_per_launch": round(us, 3)}
+    return {"kernel": "expert FFN per layer call (moe_expert_ffn)", "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": hbm["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / hbm["hbm_gbs"], 4),
+            "peak_source": hbm["source"] + " (burst copy)", "traffic": None, "bytes_per_launch": int(nbytes),
+            "us_per_launch": round(us, 3), "distinct_experts": round(d, 2)}
+
+
+def _e2e(st, cfg, T, K, W, inputs, dev):
+    """The same steps through the C ABI with host buffers: the step's input
+    from pinned host memory to the device, all layers, the last layer's output
+    back to pinned host memory, every step."""
+    h_host = [inputs[i].cpu().pin_memory() for i in range(W + K)]
+    out_host = torch.empty_like(st.final_output(), device="cpu").pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    target = st.buf[0] if cfg.chained else st.inp
+
+    def step(i):
+        target.copy_(h_host[i], non_blocking=True)
+        st.run()
+        out_host.copy_(st.final_output(), non_blocking=True)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i in range(K):
+        step(W + i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    return {"value": round(T * K / (ms / 1e3), 2), "unit": "tok/s",
+            "h2d_bytes_per_step": int(h_host[0].numel() * h_host[0].element_size()),
+            "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())}
+
+
+def decode_measure(cfg_id, T, K, W, dev, rank=0, world=1, clocks=False, cpu_budget=3.0, layers=None,
+                   share=None, want_cpu=True):
+    """One decode configuration: K timed steps of T tokens through the whole
+    stack (device-resident inputs), its HBM roofline, the end-to-end number
+    and the oracle on the host cores.  Returns (result, stack)."""
+    from int4_routed_expert_02_b200 import moe
+    from int4_routed_expert_02_b200.stack import MoEStack
+    cfg = synth.CONFIGS[cfg_id]
+    st = MoEStack(cfg, cfg_id, T=T, layers=layers, device=dev, keep_router_codes=cfg.zipf > 0,
+                  device_layers=None if share is None else share.layers)
+    inputs = Inputs(cfg, cfg_id, st, T, W + K, rank, dev)
+    stream = torch.cuda.current_stream(dev)
+    st.capture()
+
+    def step(i):
+        st.set_input(inputs[i])
+        st.run()
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(dev.index if dev.index is not None else 0)
+    if clocks:
+        clk.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        step(W + i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk_res = clk.stop() if clocks else None
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    st.status()
+    ms_per_step = ms / K
+    tok_s = world * T * K / (ms / 1e3)
+    distinct = _distinct_experts(st, moe, cfg, T)
+    step_bytes = st.L * layer_bytes(cfg, distinct)["total"]
+    hbm = peaks()
+    gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    if st.persistent:
+        traffic = (int(DECODE_TRAFFIC_PER_LAYER * st.L)
+                   if DECODE_TRAFFIC_PER_LAYER and cfg_id == 1 and T == 1 and layers is None else None)
+        roof = {"kernel": "decode_stack_kernel (persistent: all layers of a step in one cooperative launch)",
+                "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / hbm["hbm_gbs"], 4), "peak_source": hbm["source"] + " (burst copy)",
+                "traffic": traffic, "bytes_per_launch": int(step_bytes), "us_per_launch": round(ms_per_step * 1e3, 2),
+                "distinct_experts_per_layer": round(distinct, 2)}
+    else:
+        roof = _expert_roofline(st, moe, cfg, T, hbm, dev)
+    res = {"workload": workload_name(cfg, T, st.L), "config_id": cfg_id, "tokens_per_step": T, "layers": st.L,
+           "value": round(tok_s, 2), "unit": "tok/s", "ms_per_step": round(ms_per_step, 5), "steps": K, "warmup": W,
+           "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm["hbm_gbs"], 4), "bytes_per_step": int(step_bytes),
+           "roofline": roof, "l2": l2_note(cfg, step_bytes),
+           "path": "persistent decode kernel" if st.persistent else "per-layer calls (CUDA graph)",
+           "gpu_launches_per_step": st.launches_per_step()}
+    res["e2e"] = _e2e(st, cfg, T, K, W, inputs, dev)
+    if clocks:
+        res["clocks"] = clk_res
+    if want_cpu and rank == 0 and world == 1 and cpu_budget > 0:
+        res["cpu_baseline"] = cpu_baseline(cfg, cfg_id, T, budget_s=cpu_budget)
+    del inputs
+    return res, st
 
 
 def expert_flops(cfg, T: int) -> float:
@@ -333,6 +365,7 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None):
     traffic = PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER if fused else PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK
     name = (workload_name(cfg, T) + ", the rows of 8 chunks of 128 through each layer in one call") if fused else \
         (workload_name(cfg, T) + f", {chunks} chunks chunk-major")
+    bound_us = max(roof["bytes_per_launch"] / (hbm["hbm_gbs"] * 1e3), fl / (peak_t * 1e6))
     return {"workload": name, "tok_s": round(chunks * T / (ms / 1e3), 1),
             "ms_per_chunk": round(ms / chunks, 4),
             "expert_ffn": {"kernel": "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
@@ -340,6 +373,7 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None):
                            "tflops": round(tflops, 2), "tensor_peak_tflops": peak_t,
                            "tensor_frac": round(tflops / peak_t, 4), "hbm_gbs": roof["achieved"],
                            "hbm_frac": roof["frac"], "bytes_per_launch": roof["bytes_per_launch"],
+                           "binding_roof_frac": round(bound_us / roof["us_per_launch"], 4),
                            "traffic": traffic,
                            "peak_source": hbm["source"] + " (bf16 dense burst; FP16 same rate; copy bandwidth)"}}, st
 
@@ -381,114 +415,166 @@ def head_measure(dev, reps=50, warmup=5):
             "traffic": HEAD_TRAFFIC_PER_CALL, "peak_source": hbm["source"] + " (burst copy)"}
 
 
-def _e2e(st, cfg, T, K, W, inputs, dev):
-    from int4_routed_expert_02_b200 import moe  # noqa: F401
-    h_host = [inp.cpu().pin_memory() for inp in inputs]
-    out_host = torch.empty_like(st.final_output(), device="cpu").pin_memory()
-    stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    target = st.buf[0] if cfg.chained else st.inp
-
-    def step(i):
-        target.copy_(h_host[i], non_blocking=True)
-        st.run()
-        out_host.copy_(st.final_output(), non_blocking=True)
-
-    for i in range(W):
-        step(i)
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for i in range(K):
-        step(W + i)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    return {"value": round(T * K / (ms / 1e3), 2), "unit": "tok/s",
-            "h2d_bytes_per_step": int(h_host[0].numel() * h_host[0].element_size()),
-            "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())}
-
-
 # --------------------------------------------------------------------------- oracle
 
-class OracleSample:
-    """The fp64 CPU oracle as it stands (plain C, one thread) on host copies
-    of the first few layers of a configuration."""
-
-    def __init__(self, cfg, cfg_id, n_layers):
-        import oracle
-        self.oracle = oracle
-        self.cfg, self.cfg_id = cfg, cfg_id
-        dev = "cuda" if torch.cuda.is_available() else "cpu"
-        self.layers = []
-        self.router_codes = []
-        for l in range(n_layers):
-            w = {k: v.cpu() for k, v in synth.gen_layer(cfg, cfg_id, l, device=dev).items()}
-            self.router_codes.append(w.get("router_codes"))
-            self.layers.append(oracle.OracleLayer.from_config(w, cfg))
-
-    def hidden(self, layer, step):
-        if self.cfg.zipf > 0:
-            return synth.gen_zipf_hidden(self.cfg, self.cfg_id, layer, step, self.router_codes[layer], T=1)[0]
-        return synth.gen_hidden(self.cfg, self.cfg_id, 10_000 + step, 1)
-
-    def time_layer(self, layer, h):
-        t0 = time.perf_counter()
-        r = self.oracle.layer_forward(self.layers[layer], h)
-        dt = time.perf_counter() - t0
-        return dt, torch.from_numpy(r["out_bf16"].view("int16")).view(torch.bfloat16)
+def _oracle_layer_input(cfg, cfg_id, layer, w, T):
+    if cfg.zipf > 0:
+        return synth.gen_zipf_hidden(cfg, cfg_id, layer, 0, w["router_codes"], T=T)[0]
+    if cfg_id == 0:
+        return synth.gen_hidden_redrawn(cfg, 0, 10_000, T, synth.load_redraws(TINY_REDRAWS))
+    return synth.gen_hidden(cfg, cfg_id, 10_000, T)
 
 
-def cpu_baseline(cfg, cfg_id, T, budget_s=15.0):
-    """Oracle tok/s on a bounded sample: one token through consecutive layers
-    until the time budget is spent, scaled to the full layer stack."""
+def cpu_baseline(cfg, cfg_id, T, budget_s=15.0, threads=None):
+    """The fp64 oracle as it stands on a bounded sample of the workload: a few
+    tokens (min(T, 4)) through consecutive layers of the stack (chained where
+    the configuration chains) until the budget is spent, timed on one thread
+    and on every host core (its row loops split over OpenMP threads; the same
+    arithmetic, the same bits); tok/s scaled to T tokens and the full stack."""
     import oracle
+    cores = threads or os.cpu_count() or 1
+    Ts = min(T, 4)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    spent, n, h = 0.0, 0, None
-    while n < cfg.layers and spent < budget_s:
-        w = {k: v.cpu() for k, v in synth.gen_layer(cfg, cfg_id, n, device=dev).items()}
-        OL = oracle.OracleLayer.from_config(w, cfg)
-        if h is None or not cfg.chained:
-            h = (synth.gen_zipf_hidden(cfg, cfg_id, n, 0, w["router_codes"], T=1)[0] if cfg.zipf > 0
-                 else synth.gen_hidden(cfg, cfg_id, 0, 1))
-        t0 = time.perf_counter()
-        r = oracle.layer_forward(OL, h)
-        spent += time.perf_counter() - t0
-        h = torch.from_numpy(r["out_bf16"].view("int16")).view(torch.bfloat16)
-        n += 1
-        del w, OL
-    tok_s = (n / cfg.layers) / spent
-    return {"value": round(tok_s, 6), "unit": "tok/s", "cores": 1, "kind": "oracle",
-            "sample": f"1 token through {n} of {cfg.layers} layers (fp64 C oracle, 1 thread, {spent:.1f} s); "
-                      f"tok/s scaled to the full {cfg.layers}-layer stack"}
+    s1 = sall = 0.0
+    n, h, used = 0, None, 1
+    try:
+        while n < cfg.layers and (n == 0 or s1 < budget_s):
+            w = {k: v.cpu() for k, v in synth.gen_layer(cfg, cfg_id, n, device=dev).items()}
+            OL = oracle.OracleLayer.from_config(w, cfg)
+            if h is None or not cfg.chained:
+                h = _oracle_layer_input(cfg, cfg_id, n, w, Ts)
+            oracle.set_threads(1)
+            t0 = time.perf_counter()
+            r = oracle.layer_forward(OL, h)
+            s1 += time.perf_counter() - t0
+            used = oracle.set_threads(cores)
+            t0 = time.perf_counter()
+            oracle.layer_forward(OL, h)
+            sall += time.perf_counter() - t0
+            h = torch.from_numpy(r["out_bf16"].view("int16")).view(torch.bfloat16)
+            n += 1
+            del w, OL
+    finally:
+        oracle.set_threads(1)
+    v1 = Ts * (n / cfg.layers) / s1
+    vall = Ts * (n / cfg.layers) / sall
+    cpu_model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    cpu_model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"value": round(vall, 6), "unit": "tok/s", "cores": used, "kind": "oracle",
+            "value_1_thread": round(v1, 6), "cpu_model": cpu_model,
+            "sample": f"{Ts} token(s) through {n} of {cfg.layers} layers, fp64 C oracle: {sall:.2f} s on {used} "
+                      f"threads, {s1:.2f} s on 1 thread; tok/s scaled to the full stack"}
 
 
 def run_reference(args, rank, world):
-    """The reference arm: the fp64 CPU oracle on the host cores.  Each step is
-    a bounded sample: one fresh token through one layer (cycling over the
-    first two layers); tok/s is scaled to the full layer stack."""
+    """The reference arm: the fp64 CPU oracle on the host cores (OpenMP over
+    its row loops).  Each step is a bounded sample: T fresh tokens through one
+    layer (cycling over the first two layers); tok/s is scaled to the full
+    layer stack."""
+    import oracle
     cfg = synth.CONFIGS[args.config]
     T = args.tokens or cfg.T
     if rank != 0:
         return None
-    smp = OracleSample(cfg, args.config, min(2, cfg.layers))
+    cores = os.cpu_count() or 1
+    used = oracle.set_threads(cores)
+    layers, hs = [], []
+    for l in range(min(2, cfg.layers)):
+        w = {k: v.cpu() for k, v in synth.gen_layer(cfg, args.config, l, device="cpu").items()}
+        layers.append(oracle.OracleLayer.from_config(w, cfg))
+        hs.append(w)
     times = []
-    for s in range(args.warmup + args.steps):
-        l = s % len(smp.layers)
-        dt, _ = smp.time_layer(l, smp.hidden(l, s))
-        if s >= args.warmup:
-            times.append(dt)
+    try:
+        for s in range(args.warmup + args.steps):
+            l = s % len(layers)
+            if cfg.zipf > 0:
+                h = synth.gen_zipf_hidden(cfg, args.config, l, s, hs[l]["router_codes"], T=T)[0]
+            elif args.config == 0:
+                h = synth.gen_hidden_redrawn(cfg, 0, 10_000 + s, T, synth.load_redraws(TINY_REDRAWS))
+            else:
+                h = synth.gen_hidden(cfg, args.config, 10_000 + s, T)
+            t0 = time.perf_counter()
+            oracle.layer_forward(layers[l], h)
+            dt = time.perf_counter() - t0
+            if s >= args.warmup:
+                times.append(dt)
+    finally:
+        oracle.set_threads(1)
     per_layer = statistics.mean(times)
-    v = 1.0 / (per_layer * cfg.layers)
-    cpu = {"value": round(v, 6), "unit": "tok/s", "cores": 1, "kind": "oracle",
-           "sample": f"{args.steps} steps of 1 token through 1 layer (fp64 C oracle, 1 thread, "
+    v = T / (per_layer * cfg.layers)
+    cpu = {"value": round(v, 6), "unit": "tok/s", "cores": used, "kind": "oracle",
+           "sample": f"{args.steps} steps of {T} token(s) through 1 layer (fp64 C oracle, {used} threads, "
                      f"{per_layer * 1e3:.1f} ms/layer); tok/s scaled to {cfg.layers} layers"}
     return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_layer * cfg.layers * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_name(cfg, T), "config_id": args.config, "layers": cfg.layers,
-                       "tokens_per_step": 1, "parallelism": "host CPU, 1 thread"},
+                       "tokens_per_step": T, "parallelism": f"host CPU, {used} threads",
+                       "l2": l2_note(cfg, cfg.layers * layer_bytes(cfg, cfg.k * T)["total"])},
             "cpu_baseline": cpu, "e2e": {"value": round(v, 6), "unit": "tok/s", "h2d_bytes_per_step": 0,
                                          "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------- main
+
+OTHER_DECODE = [("tiny_T4", 0, 4), ("qwen35b_T1", 2, 1), ("qwen35b_T4", 2, 4), ("qwen35b_T8", 2, 8),
+                ("qwen80b_zipf_T1", 3, 1)]
+
+
+def run_ours(args, rank, world, local_rank):
+    from int4_routed_expert_02_b200 import build
+    if rank == 0 or not os.path.exists(build.LIB):
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    T = args.tokens or synth.CONFIGS[args.config].T
+    K, W = args.steps, args.warmup
+    head_res, st = decode_measure(args.config, T, K, W, dev, rank, world, clocks=(rank == 0),
+                                  cpu_budget=0 if args.no_cpu_baseline else args.cpu_budget,
+                                  layers=args.layers or None)
+    cfg = synth.CONFIGS[args.config]
+    res = {
+        "metric": METRIC, "value": head_res["value"], "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": head_res["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights, bf16 activations, fp32 accumulate (router fp64)", "data": "synthetic",
+        "config": {"workload": head_res["workload"], "config_id": args.config, "layers": head_res["layers"],
+                   "tokens_per_step": T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "l2": head_res["l2"]},
+        "hbm_gbs": head_res["hbm_gbs"], "hbm_frac": head_res["hbm_frac"], "bytes_per_step": head_res["bytes_per_step"],
+        "roofline": head_res["roofline"], "cpu_baseline": head_res.get("cpu_baseline"), "e2e": head_res["e2e"],
+        "gpu_launches": head_res["gpu_launches_per_step"] * K, "clocks": head_res.get("clocks"),
+    }
+    if not args.all_configs or world > 1 or args.layers or args.tokens or args.config != 1:
+        return res
+    # the rest of the workload set, each on its own weights (freed in turn)
+    del st
+    torch.cuda.empty_cache()
+    res["configs"] = {}
+    for name, cid, t in OTHER_DECODE:
+        k2 = K if t == 1 else max(64, K // 4)
+        r, s2 = decode_measure(cid, t, k2, W, dev, cpu_budget=args.sub_cpu_budget)
+        res["configs"][name] = r
+        del s2
+        torch.cuda.empty_cache()
+    prefill, pst = prefill_measure(dev)
+    res["prefill"] = prefill
+    res["prefill_fused"], _ = prefill_measure(dev, chunks=2, T=1024, share=pst)
+    r64, s64 = decode_measure(4, 64, 32, W, dev, cpu_budget=args.sub_cpu_budget, share=pst)
+    r64["workload"] += " (64-token decode batches on the Gemma shape)"
+    res["prefill_batch64"] = r64
+    del pst, s64
+    torch.cuda.empty_cache()
+    res["output_head"] = head_measure(dev)
+    return res
 
 
 def main():
@@ -501,12 +587,13 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: the config's)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: build this many layers instead of the config's (not a bench line)")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="oracle seconds per leg for the headline")
+    ap.add_argument("--sub-cpu-budget", type=float, default=3.0, help="oracle seconds per leg for the other configs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--head-only", action="store_true",
                     help="profiling only: time the output-head GEMV alone and print its object")
-    ap.add_argument("--no-prefill", dest="prefill", action="store_false",
-                    help="skip the chunked-prefill measurement that the default line carries")
+    ap.add_argument("--headline-only", dest="all_configs", action="store_false",
+                    help="only the headline configuration (skip the other configurations of the line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

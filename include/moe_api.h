@@ -121,7 +121,11 @@ MOE_API int moe_prepare_qmat(const uint32_t *q, const uint16_t *scale, const uin
 /*
  * Bytes of workspace that moe_router / moe_expert_ffn / moe_layer_forward
  * need for calls with up to T_max tokens on layers shaped like `w`.
- * Returns 0 on invalid arguments.
+ * Returns 0 on invalid arguments.  (The pages define no workspace: it is this
+ * library's ownership rule -- the caller allocates every buffer, the calls
+ * never allocate, so that they can be enqueued from code that may not
+ * allocate.)  Layout and contents are private to the library; the first 16
+ * bytes hold the status word that moe_workspace_status reads.
  */
 MOE_API size_t moe_workspace_size(const moe_layer_w *w, int T_max);
 
@@ -161,7 +165,11 @@ MOE_API int moe_router(const moe_layer_w *w, const uint16_t *h, int T, int32_t *
                void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Token -> expert bucketing of the T*k (token, slot) pairs:
+ * Token -> expert bucketing of the T*k (token, slot) pairs (TurboFieldfare
+ * introduction page, section "TurboFieldfare's expert streaming structure",
+ * last paragraph: prefill runs in chunks of up to 128 tokens so that several
+ * rows share one read of an expert; grouping the pairs by expert is what
+ * lets an expert's weights be read once for all of its rows):
  *   offsets [E+1]: exclusive prefix sum of pairs per expert;
  *   perm [T*k]   : pair ids p = t*k + s grouped by expert, ascending p inside
  *                  an expert (stable);
@@ -177,6 +185,18 @@ MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets
  * Expert part of the layer: m [T, H] fp32 = sum_s wts[t,s] * FFN_idx[t,s](xe_t)
  * (+ FFN_shared(xe_t) when with_shared).  Inputs: xe [T, H] bf16, idx/wts
  * [T, k], and the bucketing of idx (offsets, perm, active from moe_bucket).
+ * (TurboFieldfare introduction page, section "TurboFieldfare's expert
+ * streaming structure": the routed experts' outputs are summed with the
+ * router's weights and the shared expert's output is added without one;
+ * weights are MLX affine 4-bit, groups of 64, a BF16 scale and bias per
+ * group, section "How TurboFieldfare saves memory".)
+ * Path: force_path 1, or T < 32 in auto mode, is the CUDA-core dequant-GEMV
+ * (fp32 sums of exact products).  force_path 2, or T >= 32, is the tcgen05
+ * grouped GEMM on FP16 operands: it needs every weight s*q + b and every
+ * SwiGLU value within the FP16 range (|v| <= 65504).  A layer outside that
+ * range is not computed approximately: the kernel records MOE_EDEVICE
+ * ("outside the FP16 range") in the workspace status word (read it with
+ * moe_workspace_status) and its outputs are invalid; use force_path 1 there.
  */
 MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *idx, const float *wts,
                    const int32_t *offsets, const int32_t *perm, const int32_t *active, int with_shared,
@@ -184,12 +204,45 @@ MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, cons
 
 /*
  * One whole MoE layer: router -> bucketing -> routed + shared experts ->
- * weighted combine -> normalisation, residual, layer scalar.
+ * weighted combine -> normalisation, residual, layer scalar (TurboFieldfare
+ * introduction page, section "TurboFieldfare's expert streaming structure":
+ * the router pseudo-code, then the three phases of a layer, the last of which
+ * combines the routed branches with the router's weights, adds the shared
+ * branch and applies normalisation, residual and the layer scalar).
  *   h_in [T, H] bf16 -> h_out [T, H] bf16 (h_out may not alias h_in).
- * opts may be NULL (post_norm 1, layer_scalar 1, eps 1e-6, auto path).
+ * opts may be NULL (post_norm 1, layer_scalar 1, eps 1e-6, auto path).  The
+ * expert part follows the path rules of moe_expert_ffn.
  */
 MOE_API int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T, void *ws,
                       size_t ws_bytes, const moe_opts *opts, void *stream);
+
+/*
+ * Expert-parallel split of a layer over G devices (no counterpart in the
+ * pages, which run one device; the split is this library's multi-GPU form of
+ * the same arithmetic).  A rank owns the routed experts [e_lo, e_hi) --
+ * contiguous blocks, e.g. [E*r/G, E*(r+1)/G) -- and, when with_shared != 0,
+ * the shared expert (one rank per layer).  Every rank runs the whole router
+ * (it is small) and computes
+ *   m_out [T, H] fp32 = sum over its pairs of w_s * FFN_idx_s(xe)  (+ FFN_shared(xe)),
+ * so that the sum of every rank's m_out is moe_expert_ffn's m for the layer
+ * (up to fp32 summation order).  The caller adds the ranks' m_out (an
+ * all-reduce, e.g. NCCL over NVLink) and finishes the layer with moe_combine.
+ *   h_in [T, H] bf16; ws: moe_workspace_size(w, T) bytes.  Asynchronous; the
+ *   expert part follows the path rules of moe_expert_ffn.
+ */
+MOE_API int moe_layer_partial(const moe_layer_w *w, const uint16_t *h_in, int T, int e_lo, int e_hi, int with_shared,
+                              float *m_out, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream);
+
+/*
+ * The end of a layer (TurboFieldfare introduction page, section
+ * "TurboFieldfare's expert streaming structure": after the weighted combine,
+ * normalisation, residual and layer scalar):
+ *   h_out [T, H] bf16 = bf16((h_in + rmsnorm_no_scale(m)) * layer_scalar)   (post_norm, else h_in + m)
+ * m [T, H] fp32 is the combine (e.g. the all-reduced sum of moe_layer_partial
+ * outputs).  H a multiple of 64, <= 8192.  Asynchronous.
+ */
+MOE_API int moe_combine(const uint16_t *h_in, const float *m, uint16_t *h_out, int T, int H, const moe_opts *opts,
+                        void *stream);
 
 /*
  * Decode step through a stack of L layers (the per-token layer loop of the
@@ -213,6 +266,12 @@ MOE_API size_t moe_decode_stack_workspace_size(const moe_layer_w *w, int T);
 
 MOE_API int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained, uint16_t *h_out,
                              int T, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream);
+
+/* 1 if moe_decode_stack can run layers shaped like `w` with T tokens on the
+ * stream's device (NULL: the current device) -- its plan of shared memory
+ * and work per CTA fits one CTA per SM -- else 0 (also on bad arguments).
+ * Callers fall back to moe_layer_forward per layer when it returns 0. */
+MOE_API int moe_decode_stack_fits(const moe_layer_w *w, int T, void *stream);
 
 /* Synchronous: reads the device error code a moe_decode_stack call left in
  * `ws` (after waiting for the device).  MOE_OK, or MOE_EDEVICE with the reason
@@ -267,6 +326,11 @@ MOE_API int moe_qmat_gemv(const moe_qmat *w, int rows, int cols, const uint16_t 
  *     call's contents; nothing in it needs to start at zero.  Calls whose
  *     kernels overlap on the GPU (different streams, or several host threads)
  *     race on the scratch: serialise them.
+ *   - The looked-up address is kept for the life of the process.  It does not
+ *     survive cudaDeviceReset (or any other teardown of the device's primary
+ *     context): do not call this entry point after one.
+ *   - The tensor-core path (T >= 32, or force_path 2) leaves its status words
+ *     in the scratch; moe_noalloc_status reads them.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 
@@ -274,6 +338,16 @@ MOE_API size_t moe_noalloc_scratch_bytes(void);
 
 MOE_API int moe_layer_forward_noalloc(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_out, int T,
                                       const moe_opts *opts, void *stream);
+
+/*
+ * Synchronous: waits for `stream` (the NULL stream: the current device), then
+ * reads the status words that the last moe_layer_forward_noalloc call on the
+ * stream's device left in the static scratch -- what moe_workspace_status
+ * reads for a caller-provided workspace: MOE_OK, or MOE_EDEVICE with the
+ * reason (a bounded wait that ran out, or a value outside the FP16 range of
+ * the tensor-core path) in moe_last_error().  Allocates nothing.
+ */
+MOE_API int moe_noalloc_status(void *stream);
 
 #ifdef __cplusplus
 }

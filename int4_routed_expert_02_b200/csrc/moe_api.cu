@@ -108,7 +108,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // The SwiGLU buffers of the GEMV path and the token / SwiGLU matrices of the
 // tensor-core path share one region (a call uses one path).
 struct WsLayout {
-    size_t status, logits, idx, wts, xe, offsets, perm, inv, active, a_routed, a_shared, xg, act, y, sh, total;
+    size_t status, logits, idx, wts, xe, offsets, perm, inv, active, wts_ep, active_ep, a_routed, a_shared, xg, act, y,
+        sh, total;
 };
 
 constexpr size_t kStatusOffset = 4;
@@ -132,6 +133,8 @@ WsLayout ws_layout(const moe_layer_w *w, int T) {
     L.perm = take(sizeof(int32_t) * Tk);
     L.inv = take(sizeof(int32_t) * Tk);
     L.active = take(sizeof(int32_t) * (w->E + 1));
+    L.wts_ep = take(sizeof(float) * Tk);
+    L.active_ep = take(sizeof(int32_t) * (w->E + 1));
     {
         const size_t gemv_a = align256(sizeof(float) * Tk * w->I), gemv_s = align256(sizeof(float) * T * w->Is);
         const size_t mma_x = align256(moe::mma_xg_bytes(w, T)), mma_a = align256(moe::mma_act_bytes(w, T));
@@ -182,9 +185,10 @@ cudaError_t run_experts(const moe_layer_w *w, const uint16_t *xe, int T, const i
                         cudaStream_t st) {
     if (use_mma(o, T)) {
         int *err = at<int>(ws, L.status + kStatusOffset);
-        cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
+        cudaError_t e = cudaMemsetAsync(err, 0, 2 * sizeof(int), st);  // timeout word, FP16-range word
         if (e != cudaSuccess) return e;
-        moe::MmaBuffers b{at<uint16_t>(ws, L.xg), at<uint16_t>(ws, L.act), at<float>(ws, L.y), at<float>(ws, L.sh), err};
+        moe::MmaBuffers b{at<uint16_t>(ws, L.xg), at<uint16_t>(ws, L.act), at<float>(ws, L.y), at<float>(ws, L.sh), err,
+                          err + 1};
         return moe::launch_expert_mma(w, xe, T, offsets, perm, active, with_shared, b, st);
     }
     moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
@@ -362,9 +366,95 @@ int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16_t *h_ou
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
 }
 
+int moe_layer_partial(const moe_layer_w *w, const uint16_t *h_in, int T, int e_lo, int e_hi, int with_shared,
+                      float *m_out, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream) {
+    const char *fn = "moe_layer_partial";
+    g_err.clear();
+    if (int rc = check_dims(fn, w)) return rc;
+    if (int rc = check_T(fn, T)) return rc;
+    if ((long long)T * w->k > 65536) return fail(MOE_EINVAL, "%s: T*k exceeds 65536", fn);
+    if (e_lo < 0 || e_hi > w->E || e_lo > e_hi)
+        return fail(MOE_EINVAL, "%s: expert range [%d, %d) outside [0, %d]", fn, e_lo, e_hi, w->E);
+    if (int rc = check_router_ptrs(fn, w)) return rc;
+    if (int rc = check_expert_ptrs(fn, w, with_shared)) return rc;
+    const moe_opts o = resolve_opts(opts);
+    if (int rc = check_opts(fn, o)) return rc;
+    CHECK_PTR(h_in);
+    CHECK_PTR(m_out);
+    if (T == 0) return MOE_OK;
+    if (int rc = check_ws(fn, w, T, ws, ws_bytes)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(w, T);
+    double *logits = at<double>(ws, L.logits);
+    int32_t *idx = at<int32_t>(ws, L.idx);
+    float *wts = at<float>(ws, L.wts), *wts_ep = at<float>(ws, L.wts_ep);
+    uint16_t *xe = at<uint16_t>(ws, L.xe);
+    int32_t *offsets = at<int32_t>(ws, L.offsets), *perm = at<int32_t>(ws, L.perm), *inv = at<int32_t>(ws, L.inv);
+    int32_t *active = at<int32_t>(ws, L.active), *active_ep = at<int32_t>(ws, L.active_ep);
+    cudaError_t e = moe::launch_router_logits(w, h_in, T, o.eps, logits, xe, st);
+    if (e == cudaSuccess) e = moe::launch_router_topk(logits, T, w->E, w->k, w->per_expert_scale, idx, wts, st);
+    if (e == cudaSuccess) e = moe::launch_bucket(idx, T * w->k, w->E, offsets, perm, inv, active, st);
+    if (e == cudaSuccess) e = moe::launch_ep_select(idx, wts, active, T * w->k, e_lo, e_hi, wts_ep, active_ep, st);
+    if (e == cudaSuccess) e = run_experts(w, xe, T, offsets, perm, active_ep, with_shared, ws, L, o, st);
+    if (e == cudaSuccess)
+        e = moe::launch_combine(at<float>(ws, L.y), at<float>(ws, L.sh), wts_ep, T, w->H, w->k, with_shared, nullptr,
+                                m_out, nullptr, 0, 1.0f, o.eps, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_combine(const uint16_t *h_in, const float *m, uint16_t *h_out, int T, int H, const moe_opts *opts,
+                void *stream) {
+    const char *fn = "moe_combine";
+    g_err.clear();
+    if (H < 64 || H % 64 || H > 8192) return fail(MOE_EINVAL, "%s: H=%d must be a multiple of 64 in [64, 8192]", fn, H);
+    if (int rc = check_T(fn, T)) return rc;
+    const moe_opts o = resolve_opts(opts);
+    if (int rc = check_opts(fn, o)) return rc;
+    CHECK_PTR(h_in);
+    CHECK_PTR(m);
+    CHECK_PTR(h_out);
+    if (T == 0) return MOE_OK;
+    cudaError_t e = moe::launch_combine(nullptr, m, nullptr, T, H, 0, 1, h_in, nullptr, h_out, o.post_norm,
+                                        o.layer_scalar, o.eps, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
 size_t moe_decode_stack_workspace_size(const moe_layer_w *w, int T) {
     if (check_dims("moe_decode_stack_workspace_size", w) || T < 1 || T > moe::decode_stack_max_tokens()) return 0;
     return moe::decode_stack_ws_bytes(w, T);
+}
+
+// Grid of the persistent decode kernel on `dev` (one CTA per SM), cached.
+static cudaError_t decode_grid_of(int dev, int *grid) {
+    static std::mutex mu;
+    static int grids[64] = {0};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (grids[dev] == 0) {
+        int coop = 0;
+        cudaError_t e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+        if (e != cudaSuccess) return e;
+        if (!coop) {
+            grids[dev] = -1;
+        } else {
+            e = moe::decode_stack_grid(dev, &grids[dev]);
+            if (e != cudaSuccess) return e;
+            if (grids[dev] <= 0) grids[dev] = -1;
+        }
+    }
+    *grid = grids[dev];
+    return cudaSuccess;
+}
+
+int moe_decode_stack_fits(const moe_layer_w *w, int T, void *stream) {
+    g_err.clear();
+    if (!w || check_dims("moe_decode_stack_fits", w) || T < 1 || T > moe::decode_stack_max_tokens()) return 0;
+    if (w->H > 4096 || T * w->H > moe::decode_stack_stage_floats()) return 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0, grid = 0;
+    if ((st ? cudaStreamGetDevice(st, &dev) : cudaGetDevice(&dev)) != cudaSuccess) return 0;
+    if (decode_grid_of(dev, &grid) != cudaSuccess || grid <= 0) return 0;
+    return moe::decode_stack_fits(w, T, grid) ? 1 : 0;
 }
 
 int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained, uint16_t *h_out, int T,
@@ -401,23 +491,12 @@ int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int
     int dev = 0;
     cudaError_t e = st ? cudaStreamGetDevice(st, &dev) : cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, fn);
-    static std::mutex mu;
-    static int grids[64] = {0};
+    if (dev < 0 || dev >= 64) return fail(MOE_EINVAL, "%s: device %d out of range", fn, dev);
     int grid = 0;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        if (dev < 0 || dev >= 64) return fail(MOE_EINVAL, "%s: device %d out of range", fn, dev);
-        if (grids[dev] == 0) {
-            int coop = 0;
-            e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
-            if (e != cudaSuccess) return cuda_fail(e, fn);
-            if (!coop) return fail(MOE_EINVAL, "%s: device %d has no cooperative launch", fn, dev);
-            e = moe::decode_stack_grid(dev, &grids[dev]);
-            if (e != cudaSuccess) return cuda_fail(e, fn);
-            if (grids[dev] <= 0) return fail(MOE_EINVAL, "%s: the decode kernel does not fit on an SM", fn);
-        }
-        grid = grids[dev];
-    }
+    if ((e = decode_grid_of(dev, &grid)) != cudaSuccess) return cuda_fail(e, fn);
+    if (grid <= 0)
+        return fail(MOE_EINVAL, "%s: device %d cannot run the decode kernel (cooperative launch, one CTA per SM)", fn,
+                    dev);
     if (!moe::decode_stack_fits(&w0, T, grid))
         return fail(MOE_EINVAL, "%s: T=%d with H=%d, E=%d does not fit the kernel's shared memory", fn, T, w0.H, w0.E);
     e = moe::launch_decode_stack(layers, L, h_in, chained, h_out, T, ws, o, grid, st);
@@ -453,16 +532,21 @@ int moe_workspace_status(const void *ws) {
     const char *fn = "moe_workspace_status";
     g_err.clear();
     if (!ws) return fail(MOE_EINVAL, "%s: workspace is NULL", fn);
-    int code = 0;
-    cudaError_t e = cudaMemcpy(&code, static_cast<const char *>(ws) + kStatusOffset, sizeof code, cudaMemcpyDeviceToHost);
+    int code[2] = {0, 0};
+    cudaError_t e = cudaMemcpy(code, static_cast<const char *>(ws) + kStatusOffset, sizeof code, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, fn);
-    if (code != 0) {
+    if (code[0] != 0) {
         static const char *what[] = {"", "wait for weights timed out", "wait for a free weight slot timed out",
                                      "wait for a weight tile timed out", "wait for a free weight tile timed out",
                                      "wait for a token tile timed out", "wait for a free token tile timed out",
                                      "wait for the accumulator timed out", "wait for the epilogue timed out"};
-        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 9) ? what[code] : "?");
+        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code[0],
+                    (code[0] > 0 && code[0] < 9) ? what[code[0]] : "?");
     }
+    if (code[1] != 0)
+        return fail(MOE_EDEVICE, "%s: %s outside the FP16 range of the tensor-core path; outputs are invalid "
+                    "(force_path 1 computes this layer)", fn,
+                    code[1] == 1 ? "a weight s*q + b" : "a SwiGLU value silu(g)*u");
     return MOE_OK;
 }
 
@@ -476,8 +560,12 @@ int moe_decode_stack_status(const void *ws) {
     if (e != cudaSuccess) return cuda_fail(e, fn);
     if (code != 0) {
         static const char *what[] = {"", "grid barrier timed out", "wait for weights timed out",
-                                     "wait for a free ring slot timed out", "wait for a job buffer timed out"};
-        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 5) ? what[code] : "?");
+                                     "wait for a free ring slot timed out",
+                                     "wait for another CTA's gate/up units timed out",
+                                     "wait for a ring slot's hand-over timed out",
+                                     "wait for the routing tables timed out",
+                                     "wait for a staged down-projection input timed out"};
+        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 8) ? what[code] : "?");
     }
     return MOE_OK;
 }

@@ -39,7 +39,9 @@ combine_kernel(const float *__restrict__ y, const float *__restrict__ sh, const 
                 v[u] = s0 + u < k ? __ldg(y4 + (size_t)(s0 + u) * H4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                if (s0 + u < k) {
+                // a zero weight adds nothing (0 * y = 0 for finite y); skipping it lets a
+                // rank of an expert-parallel split leave the y rows of pairs it does not own unset
+                if (s0 + u < k && wk[s0 + u] != 0.f) {
                     const float w = wk[s0 + u];
                     m.x = fmaf(w, v[u].x, m.x);
                     m.y = fmaf(w, v[u].y, m.y);
@@ -78,6 +80,33 @@ cudaError_t launch_combine(const float *y, const float *sh, const float *wts, in
     const int threads = min(kCombineMaxThreads, ((H / 4 + 31) / 32) * 32);
     combine_kernel<<<T, threads, smem, st>>>(y, sh, wts, H, k, with_shared, h_in, m_out, h_out, post_norm,
                                                      layer_scalar, eps);
+    return cudaGetLastError();
+}
+
+// Expert-parallel selection (no counterpart in the pages, which run on one
+// device): the pairs whose expert lies in [e_lo, e_hi) keep their gate
+// weight, the others get 0; the active list keeps the experts in range.
+__global__ void __launch_bounds__(256) ep_select_kernel(const int32_t *__restrict__ idx, const float *__restrict__ wts,
+                                                        const int32_t *__restrict__ active, int n, int e_lo, int e_hi,
+                                                        float *__restrict__ wts_out, int32_t *__restrict__ active_out) {
+    for (int p = threadIdx.x; p < n; p += blockDim.x) {
+        const int e = idx[p];
+        wts_out[p] = (e >= e_lo && e < e_hi) ? wts[p] : 0.f;
+    }
+    if (threadIdx.x == 0) {
+        const int na = active[0];
+        int cnt = 0;
+        for (int i = 0; i < na; ++i) {
+            const int e = active[1 + i];
+            if (e >= e_lo && e < e_hi) active_out[1 + cnt++] = e;
+        }
+        active_out[0] = cnt;
+    }
+}
+
+cudaError_t launch_ep_select(const int32_t *idx, const float *wts, const int32_t *active, int n, int e_lo, int e_hi,
+                             float *wts_out, int32_t *active_out, cudaStream_t st) {
+    ep_select_kernel<<<1, 256, 0, st>>>(idx, wts, active, n, e_lo, e_hi, wts_out, active_out);
     return cudaGetLastError();
 }
 

@@ -48,7 +48,8 @@ struct MmaBuffers {
     uint16_t *act;  // [T + T*k, Kmax] FP16 SwiGLU rows, chunk-permuted, Kmax = max(I, Is)
     float *y;       // [T*k, H]  routed expert outputs, by pair id t*k+s
     float *sh;      // [T, H]    shared expert output
-    int *err;       // device error word (0 = ok)
+    int *err;       // device error word (0 = ok): a bounded wait ran out
+    int *range_err; // device word (0 = ok): a weight or SwiGLU value outside the FP16 range
 };
 size_t mma_xg_bytes(const moe_layer_w *w, int T);
 size_t mma_act_bytes(const moe_layer_w *w, int T);
@@ -60,6 +61,10 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
 cudaError_t launch_combine(const float *y, const float *sh, const float *wts, int T, int H, int k, int with_shared,
                            const uint16_t *h_in, float *m_out, uint16_t *h_out, int post_norm, float layer_scalar,
                            float eps, cudaStream_t st);
+
+// Expert-parallel selection: gate weights of pairs outside [e_lo, e_hi) set to 0, active list filtered.
+cudaError_t launch_ep_select(const int32_t *idx, const float *wts, const int32_t *active, int n, int e_lo, int e_hi,
+                             float *wts_out, int32_t *active_out, cudaStream_t st);
 
 // Persistent decode kernel over a stack of layers (moe_decode.cu).
 size_t decode_stack_smem();

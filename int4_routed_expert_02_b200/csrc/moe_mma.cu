@@ -47,8 +47,13 @@
 // w = s*q + b and of the SwiGLU output 8x finer than BF16's 8 bits (BF16
 // operands cost up to ~2e-2 * rms of the layer output, the whole error budget;
 // FP16 ~1e-3).  The activations convert exactly (a BF16 value of the
-// normalised input has 8 significant bits and |x| <= sqrt(H)); the SwiGLU
-// output is saturated to +-65504, the FP16 range.
+// normalised input has 8 significant bits and |x| <= sqrt(H)).  FP16's range
+// is the price: a weight s*q + b or a SwiGLU output beyond +-65504 cannot be
+// represented.  The dequant warps test every group's extremes (q = 0 and
+// q = 15) and the epilogue every SwiGLU value; the first value out of range
+// is recorded in a status word of its own (range_err), which no wait polls,
+// so the kernels run to their end and the call reports the layer as outside
+// this path's domain instead of returning a silently saturated result.
 //
 // K order inside a chunk of 8.  The dequantisation makes BF16 pairs from
 // nibbles j and j+4 of a word (one mask per pair), so the 8 weights of a
@@ -131,7 +136,8 @@ struct Params {
     float *y;   // down output, routed: [T*k, H] by pair id
     float *sh;  // down output, shared: [T, H]
     int H;
-    int *err;
+    int *err;        // bounded-wait timeouts (every wait polls it and stops)
+    int *range_err;  // a weight or SwiGLU value outside the FP16 range (no wait polls it)
 };
 
 // TMA tensor maps of one launch: the token matrix (B operand) and the tiled
@@ -608,6 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                 tc_fence_after();  // the MMAs that read this stage's columns have completed
                 if (valid) {  // warp-uniform: rv is a multiple of 32, kbi is the warp's
                     const float sf = __uint_as_float(sbw << 16), bf = __uint_as_float(sbw & 0xffff0000u);
+                    // s*q + b is linear in q: its extremes over the group are at q = 0 and q = 15
+                    if (!(fmaxf(fabsf(bf), fabsf(fmaf(15.0f, sf, bf))) <= 65504.0f)) atomicCAS(P.range_err, 0, 1);
                     const uint32_t b2 = f16x2_from_f32(bf, bf);
                     const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
                     uint4 o[4];
@@ -658,7 +666,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
                         for (int jj = 0; jj < 8; ++jj) {
                             const int n = ch * 8 + jj;
                             if (n < t.n) {
-                                const float av = fminf(fmaxf(silu_mul(g[jj], u[jj]), -65504.f), 65504.f);
+                                float av = silu_mul(g[jj], u[jj]);
+                                if (!(fabsf(av) <= 65504.f)) {
+                                    atomicCAS(P.range_err, 0, 2);
+                                    av = 0.f;  // the call is reported as outside this path's domain
+                                }
                                 P.act[(size_t)(t.brow + n) * P.act_ld + col] = __half_as_ushort(__float2half_rn(av));
                             }
                         }
@@ -836,6 +848,7 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
     P.sh = b.sh;
     P.H = H;
     P.err = b.err;
+    P.range_err = b.range_err;
     const long long pairs = (long long)T * k;
     const int max_active = (int)(pairs < w->E ? pairs : w->E);
 

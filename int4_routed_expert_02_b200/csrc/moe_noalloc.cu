@@ -78,4 +78,22 @@ int moe_layer_forward_noalloc(const moe_layer_w *w, const uint16_t *h_in, uint16
     return moe_layer_forward(w, h_in, h_out, T, scratch, kStaticScratchBytes, opts, stream);
 }
 
+int moe_noalloc_status(void *stream) {
+    int dev = 0;
+    cudaError_t e = stream ? cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &dev) : cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "moe_noalloc_status: cannot tell the stream's device: %s", cudaGetErrorString(e));
+        return moe::set_last_error(MOE_ECUDA, msg);
+    }
+    void *scratch = nullptr;
+    if (int rc = scratch_on(dev, &scratch)) return rc;
+    if (stream && (e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "moe_noalloc_status: %s", cudaGetErrorString(e));
+        return moe::set_last_error(MOE_ECUDA, msg);
+    }
+    return moe_workspace_status(scratch);
+}
+
 }  // extern "C"

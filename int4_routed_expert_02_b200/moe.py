@@ -24,7 +24,7 @@ EXPORTED = ("moe_last_error", "moe_version", "moe_prepare_qmat", "moe_workspace_
             "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward",
             "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc", "moe_decode_stack_workspace_size",
             "moe_decode_stack", "moe_decode_stack_status", "moe_workspace_status", "moe_qmat_gemv_workspace_size",
-            "moe_qmat_gemv")
+            "moe_qmat_gemv", "moe_noalloc_status", "moe_decode_stack_fits", "moe_layer_partial", "moe_combine")
 
 
 class MoEError(RuntimeError):
@@ -66,8 +66,12 @@ _lib.moe_decode_stack_workspace_size.argtypes = [_P, _I]
 _lib.moe_decode_stack_workspace_size.restype = C.c_size_t
 _lib.moe_decode_stack.argtypes = [_P, _I, _P, _I, _P, _I, _P, C.c_size_t, _P, _P]
 _lib.moe_decode_stack_status.argtypes = [_P]
+_lib.moe_decode_stack_fits.argtypes = [_P, _I, _P]
+_lib.moe_layer_partial.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, C.c_size_t, _P, _P]
+_lib.moe_combine.argtypes = [_P, _P, _P, _I, _I, _P, _P]
 _lib.moe_workspace_status.argtypes = [_P]
 _lib.moe_layer_forward_noalloc.argtypes = [_P, _P, _P, _I, _P, _P]
+_lib.moe_noalloc_status.argtypes = [_P]
 _lib.moe_qmat_gemv_workspace_size.restype = C.c_size_t
 _lib.moe_qmat_gemv.argtypes = [_P, _I, _I, _P, _I, _P, _P, C.c_size_t, _P]
 
@@ -252,12 +256,38 @@ def moe_decode_stack_status(ws):
     _check(_lib.moe_decode_stack_status(_ptr(ws)))
 
 
+def moe_layer_partial(layer, h_in, T, e_lo, e_hi, with_shared, m_out, ws, opts=None, stream=None):
+    """This rank's part of an expert-parallel layer: m_out = the weighted sum
+    over its routed experts [e_lo, e_hi) (+ the shared expert)."""
+    o = opts if opts is not None else _opts()
+    _check(_lib.moe_layer_partial(layer.ptr(), _ptr(h_in), T, e_lo, e_hi, int(with_shared), _ptr(m_out), _ptr(ws),
+                                  ws.numel() if ws is not None else 0, C.byref(o), _stream(stream)))
+
+
+def moe_combine(h_in, m, h_out, T, H, opts=None, stream=None):
+    """h_out = bf16((h_in + rmsnorm_no_scale(m)) * layer_scalar)."""
+    o = opts if opts is not None else _opts()
+    _check(_lib.moe_combine(_ptr(h_in), _ptr(m), _ptr(h_out), T, H, C.byref(o), _stream(stream)))
+
+
+def moe_decode_stack_fits(layer, T, stream=None) -> bool:
+    """True if the persistent decode kernel can run layers shaped like
+    `layer` with T tokens on the stream's device."""
+    return bool(_lib.moe_decode_stack_fits(layer.ptr(), T, _stream(stream)))
+
+
 def moe_workspace_status(ws):
     _check(_lib.moe_workspace_status(_ptr(ws)))
 
 
 def moe_noalloc_scratch_bytes() -> int:
     return int(_lib.moe_noalloc_scratch_bytes())
+
+
+def moe_noalloc_status(stream=None):
+    """Raise if the last moe_layer_forward_noalloc call on the stream's device
+    left a device-side error in the static scratch (synchronises the stream)."""
+    _check(_lib.moe_noalloc_status(_stream(stream)))
 
 
 def make_opts(post_norm=True, layer_scalar=1.0, eps=1e-6, force_path=0) -> Opts:

@@ -37,8 +37,9 @@ class MoEStack:
             assert len(device_layers) >= self.L
             self.layers = list(device_layers[:self.L])
         H = cfg.H
-        fits = self.T <= 8 and H <= 4096 and self.T * H <= 24576
-        self.persistent = fits if persistent is None else persistent
+        if persistent is None:
+            persistent = moe.moe_decode_stack_fits(self.layers[0], self.T, torch.cuda.current_stream(self.device))
+        self.persistent = persistent
         if self.persistent:
             # one cooperative kernel per step: every layer's output in h_out[l]
             self.larr = moe.layer_array(self.layers)

@@ -32,7 +32,7 @@ import torch
 
 __all__ = [
     "MoEConfig", "CONFIGS", "tensor_seed", "gen_layer", "gen_router", "gen_experts", "gen_hidden",
-    "gen_zipf_hidden", "pack_codes", "bf16_bits", "from_bf16_bits",
+    "gen_zipf_hidden", "load_redraws", "gen_hidden_redrawn", "pack_codes", "bf16_bits", "from_bf16_bits",
 ]
 
 
@@ -125,9 +125,9 @@ def _words(shape, device, seed):
                          generator=_gen(device, seed))
 
 
-def _scales(shape, device, seed):
+def _scales(shape, device, seed, std=0.02):
     n = torch.randn(shape, dtype=torch.float32, device=device, generator=_gen(device, seed))
-    return (n * 0.02).abs().to(torch.bfloat16)
+    return (n * std).abs().to(torch.bfloat16)
 
 
 def _biases(scale_bf16, mid, device, seed):
@@ -140,12 +140,12 @@ def _uniform(shape, lo, hi, device, seed):
     return (lo + (hi - lo) * u).to(torch.bfloat16)
 
 
-def _qmat(prefix, n_mat, rows, cols, bits, cfg_id, layer, seed, device, lead=True):
+def _qmat(prefix, n_mat, rows, cols, bits, cfg_id, layer, seed, device, lead=True, scale_std=0.02):
     shape_w = (n_mat, rows, cols * bits // 32) if lead else (rows, cols * bits // 32)
     shape_g = (n_mat, rows, cols // 64) if lead else (rows, cols // 64)
     mid = 1 << (bits - 1)
     q = _words(shape_w, device, tensor_seed(seed, cfg_id, layer, prefix + "_q"))
-    s = _scales(shape_g, device, tensor_seed(seed, cfg_id, layer, prefix + "_s"))
+    s = _scales(shape_g, device, tensor_seed(seed, cfg_id, layer, prefix + "_s"), scale_std)
     b = _biases(s, mid, device, tensor_seed(seed, cfg_id, layer, prefix + "_b"))
     return q, s, b
 
@@ -171,19 +171,23 @@ def gen_router(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="c
     return out
 
 
-def gen_experts(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="cpu") -> dict:
+def gen_experts(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="cpu",
+                scale_std: float = 0.02) -> dict:
     """Routed + shared expert matrices of one layer (MLX layout):
       gate_q, up_q [E, I, H/8]   gate_s/b, up_s/b [E, I, H/64]
       down_q [E, H, I/8]         down_s/b [E, H, I/64]
-      sh_gate_q, sh_up_q [Is, H/8] (+ s/b [Is, H/64]);  sh_down_q [H, Is/8] (+ s/b [H, Is/64])"""
+      sh_gate_q, sh_up_q [Is, H/8] (+ s/b [Is, H/64]);  sh_down_q [H, Is/8] (+ s/b [H, Is/64])
+    scale_std: the group scales are |N(0, scale_std)| (0.02 in every workload;
+    tests widen it to reach large scales)."""
     H, E, I, Is = cfg.H, cfg.E, cfg.I, cfg.Is
     out = {}
     for name, rows, cols in (("gate", I, H), ("up", I, H), ("down", H, I)):
         out[name + "_q"], out[name + "_s"], out[name + "_b"] = _qmat(name, E, rows, cols, 4, cfg_id, layer,
-                                                                      seed, device)
+                                                                      seed, device, scale_std=scale_std)
     for name, rows, cols in (("sh_gate", Is, H), ("sh_up", Is, H), ("sh_down", H, Is)):
         out[name + "_q"], out[name + "_s"], out[name + "_b"] = _qmat(name, 1, rows, cols, 4, cfg_id, layer,
-                                                                      seed, device, lead=False)
+                                                                      seed, device, lead=False,
+                                                                      scale_std=scale_std)
     return out
 
 
@@ -195,10 +199,11 @@ def gen_vocab_head(cfg: MoEConfig, cfg_id: int, V: int, seed: int = 0, device="c
     return {"head_q": q, "head_s": s, "head_b": b}
 
 
-def gen_layer(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="cpu") -> dict:
+def gen_layer(cfg: MoEConfig, cfg_id: int, layer: int, seed: int = 0, device="cpu",
+              expert_scale_std: float = 0.02) -> dict:
     """All weights of one MoE layer in MLX layout (gen_router + gen_experts)."""
     out = gen_router(cfg, cfg_id, layer, seed, device)
-    out.update(gen_experts(cfg, cfg_id, layer, seed, device))
+    out.update(gen_experts(cfg, cfg_id, layer, seed, device, scale_std=expert_scale_std))
     return out
 
 
@@ -210,8 +215,34 @@ def gen_hidden(cfg: MoEConfig, cfg_id: int, stream: int, T: int, seed: int = 0, 
     return torch.randn((T, cfg.H), dtype=torch.float32, device=device, generator=g).to(torch.bfloat16)
 
 
+def load_redraws(path: str) -> dict:
+    """A stored table of redrawn rows ({(stream, token): draw}), as written by
+    tests/golden/make_tiny_redraws.py (lines 'stream token draw'; '#' comments)."""
+    table = {}
+    with open(path) as f:
+        for ln in f:
+            ln = ln.strip()
+            if ln and not ln.startswith("#"):
+                stream, tok, draw = (int(v) for v in ln.split())
+                table[(stream, tok)] = draw
+    return table
+
+
+def gen_hidden_redrawn(cfg: MoEConfig, cfg_id: int, stream: int, T: int, redraws: dict, seed: int = 0,
+                       device="cpu") -> torch.Tensor:
+    """gen_hidden with the rows that a stored redraw table names replaced by
+    their redraws (draw d of token t: gen_hidden(..., draw=d * 65536 + t + 1))."""
+    h = gen_hidden(cfg, cfg_id, stream, T, seed=seed)
+    for t in range(T):
+        d = redraws.get((stream, t), 0)
+        if d:
+            h[t] = gen_hidden(cfg, cfg_id, stream, 1, seed=seed, draw=d * 65536 + t + 1)[0]
+    return h.to(device)
+
+
 def gen_zipf_hidden(cfg: MoEConfig, cfg_id: int, layer: int, step: int, router_codes: torch.Tensor,
-                    seed: int = 0, T: int | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+                    seed: int = 0, T: int | None = None, centred: torch.Tensor | None = None
+                    ) -> tuple[torch.Tensor, torch.Tensor]:
     """Router inputs whose selected experts follow a Zipf(cfg.zipf) popularity.
 
     Per layer a random permutation assigns popularity ranks to experts; per
@@ -224,6 +255,8 @@ def gen_zipf_hidden(cfg: MoEConfig, cfg_id: int, layer: int, step: int, router_c
     selects them; the test-side oracle confirms this per draw.
 
     router_codes: the layer's `router_codes` from gen_layer ([E, H] uint8).
+    centred: optionally, router_codes - 128 as fp64 ([E, H], on the CPU),
+    when the caller draws many steps of one layer.
     Returns (hidden [T, H] bf16, target expert ids [T, k] int64).
     """
     E, k = cfg.E, cfg.k
@@ -235,6 +268,7 @@ def gen_zipf_hidden(cfg: MoEConfig, cfg_id: int, layer: int, step: int, router_c
     u = torch.rand((T, E), dtype=torch.float64, generator=gg).clamp_min(1e-300)
     keys = logp[None, :] - torch.log(-torch.log(u))
     target = torch.topk(keys, k, dim=1).indices      # [T, k]
-    centred = router_codes.cpu().to(torch.float64) - 128.0  # [E, H]
+    if centred is None:
+        centred = router_codes.cpu().to(torch.float64) - 128.0  # [E, H]
     h = centred[target].sum(1) / math.sqrt(k * (256.0 ** 2 - 1.0) / 12.0)
     return h.to(torch.bfloat16), target

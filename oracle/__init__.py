@@ -28,7 +28,7 @@ def build_oracle(force: bool = False) -> str:
     """Compile moe_oracle.c into libmoe_oracle.so with gcc (plain C, -O2)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-std=c99", "-O2", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", "-std=c99", "-O2", "-fPIC", "-fopenmp", "-shared", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -70,12 +70,21 @@ def lib():
             L.oracle_combine.argtypes = [P, P, I, I, I, C.c_double, C.c_double, P, P]
             L.oracle_combine.restype = None
             L.oracle_layer_forward.argtypes = [P, P, I, C.c_double, I, C.c_double, P, P, P, P, P]
+            L.oracle_set_threads.argtypes = [I]
+            L.oracle_set_threads.restype = I
+            L.oracle_set_threads(1)  # the plain sequential oracle unless a caller asks for more
             _lib = L
     return _lib
 
 
 def _p(a):
     return None if a is None else a.ctypes.data
+
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's row loops (1: sequential); returns the count in
+    effect.  Results do not depend on it."""
+    return int(lib().oracle_set_threads(int(n)))
 
 
 def _np(t, dtype):

@@ -40,8 +40,26 @@
 #include <stdlib.h>
 #include <string.h>
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
 #define ORACLE_OK 0
 #define ORACLE_EINVAL -1
+
+/* Threads of the row loops (1 = the plain sequential oracle).  Returns the
+ * count in effect: 1 when the library was built without OpenMP. */
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n < 1) n = 1;
+    omp_set_num_threads(n);
+    return n;
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* ---------------------------------------------------------------- bf16 */
 
@@ -114,10 +132,17 @@ int oracle_dequant(const uint32_t *q, const uint16_t *s, const uint16_t *b, int 
     return ORACLE_OK;
 }
 
-/* y[r] = sum_c deq(W[r, c]) * x[c] : the affine-quantised projection. */
+/* y[r] = sum_c deq(W[r, c]) * x[c] : the affine-quantised projection.
+ * Rows are independent and each row's sum runs in the same order whatever
+ * the thread count, so the OpenMP split (when the library is built with it
+ * and oracle_set_threads asks for more than one thread) changes nothing in
+ * the result. */
 static void qmatvec(const uint32_t *q, const uint16_t *s, const uint16_t *b, int rows, int cols, int bits,
                     const double *x, double *y)
 {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static) if ((long)rows * cols >= 65536)
+#endif
     for (int r = 0; r < rows; ++r) {
         double acc = 0.0;
         for (int c = 0; c < cols; ++c) acc += deq(q, s, b, cols, bits, r, c) * x[c];

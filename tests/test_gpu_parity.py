@@ -265,8 +265,9 @@ def test_empty_call_and_output_canaries_and_determinism():
 
 def test_full_decode_stack_teacher_forced_on_sampled_layers():
     """The benchmark's workload (Gemma-shaped, 30 layers, T = 1) in the same
-    launch configuration (one CUDA graph per step); each sampled layer is
-    checked against the oracle on exactly the bf16 input the GPU gave it."""
+    launch configuration (one persistent decode launch per step); each
+    sampled layer is checked against the oracle on exactly the bf16 input the
+    GPU gave it."""
     from int4_routed_expert_02_b200.stack import MoEStack
     cfg = synth.CONFIGS[1]
     st = MoEStack(cfg, 1)

@@ -421,3 +421,46 @@ def test_zipf_planted_experts_are_the_ones_the_router_selects():
         assert sorted(idx[0]) == sorted(target[0].tolist())
         gap = np.sort(logits[0])[::-1]
         assert gap[cfg.k - 1] - gap[cfg.k] > 1.0
+
+
+def test_threaded_oracle_gives_the_same_bits():
+    """The all-cores oracle (the row loops split over OpenMP threads) is the
+    same computation: every row's sum runs in the same order, so the layer's
+    outputs are bit-identical to the sequential oracle's."""
+    cfg = synth.CONFIGS[2]
+    w = synth.gen_layer(cfg, 2, 0)
+    L = oracle.OracleLayer.from_config(w, cfg)
+    h = synth.gen_hidden(cfg, 2, 0, 2)
+    try:
+        oracle.set_threads(1)
+        a = oracle.layer_forward(L, h)
+        oracle.set_threads(4)
+        b = oracle.layer_forward(L, h)
+    finally:
+        oracle.set_threads(1)
+    for key in ("idx", "w", "m", "out_f64", "out_bf16"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_stored_tiny_redraws_are_the_oracles():
+    """The benchmark's tiny-configuration inputs follow a stored redraw table;
+    recompute the first 120 steps with the oracle and compare."""
+    import importlib.util
+    import os
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_tiny_redraws", os.path.join(here, "make_tiny_redraws.py"))
+    mk = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mk)
+    table = synth.load_redraws(os.path.join(here, "tiny_redraws.txt"))
+    cfg = synth.CONFIGS[0]
+    w = {n: v.cpu() for n, v in synth.gen_layer(cfg, 0, 0).items()}
+    L = oracle.OracleLayer(w, cfg.H, cfg.E, cfg.k, cfg.I, cfg.Is)
+    for step in range(120):
+        stream = mk.FIRST_STREAM + step
+        h = synth.gen_hidden_redrawn(cfg, 0, stream, cfg.T, table)
+        logits = oracle.router(L, h)[0]
+        for t in range(cfg.T):
+            assert mk.min_gap(logits[t], cfg.k) >= mk.GAP, (stream, t)
+            if (stream, t) in table:   # a listed row's first draw was below the gap
+                first = synth.gen_hidden(cfg, 0, stream, cfg.T)[t:t + 1]
+                assert mk.min_gap(oracle.router(L, first)[0][0], cfg.k) < mk.GAP

@@ -7,7 +7,11 @@ a workspace.  For them the library keeps a fixed scratch array in device
 memory.  This test calls that entry point through the C ABI and checks its
 output against moe_layer_forward with a caller-provided workspace, on two
 calls in a row (the scratch keeps the first call's contents when the second
-one starts).  It lives in its own file, collected last.
+one starts).  Both run the same kernels on the same inputs, so the outputs
+must be bit-identical.  The cases cover the CUDA-core path (T < 32) and the
+tensor-core path (T >= 32 in auto mode, and force_path 2), whose status words
+live in the static scratch and are read back with moe_noalloc_status.  It
+lives in its own file, collected last.
 """
 import ctypes as C
 
@@ -16,13 +20,12 @@ import pytest
 import torch
 
 from int4_routed_expert_02_b200 import synth
-from tests.moe_cases import OUT_TOL, max_err_vs_rms
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("cfg_id,T", [(0, 4), (1, 1), (2, 8)])
-def test_noalloc_matches_the_workspace_entry_point(cfg_id, T):
+@pytest.mark.parametrize("cfg_id,T,force_path", [(0, 4, 0), (1, 1, 0), (2, 8, 0), (2, 32, 0), (0, 4, 2)])
+def test_noalloc_matches_the_workspace_entry_point(cfg_id, T, force_path):
     from int4_routed_expert_02_b200 import build
     build.build()
     from int4_routed_expert_02_b200 import moe
@@ -30,8 +33,9 @@ def test_noalloc_matches_the_workspace_entry_point(cfg_id, T):
     cfg = synth.CONFIGS[cfg_id]
     w = synth.gen_layer(cfg, cfg_id, 0, device="cuda")
     D = moe.DeviceLayer.from_config(w, cfg)
+    assert moe.moe_workspace_size(D, T) <= moe.moe_noalloc_scratch_bytes()
     ws = moe.workspace(D, T)
-    opts = moe.make_opts()
+    opts = moe.make_opts(force_path=force_path)
     lib = moe.lib()
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
@@ -39,11 +43,12 @@ def test_noalloc_matches_the_workspace_entry_point(cfg_id, T):
         ref = torch.empty_like(h)
         got = torch.full_like(h, float("nan"))
         moe.moe_layer_forward(D, h, ref, T, ws, opts)
+        moe.moe_workspace_status(ws)
         rc = lib.moe_layer_forward_noalloc(D.ptr(), h.data_ptr(), got.data_ptr(), T, C.byref(opts), stream)
         assert rc == moe.MOE_OK, moe.last_error()
+        assert lib.moe_noalloc_status(stream) == moe.MOE_OK, moe.last_error()
         torch.cuda.synchronize()
-        err = max_err_vs_rms(got.cpu().double().numpy(), ref.cpu().double().numpy())
-        assert err <= OUT_TOL, f"call {call}: max|err|/rms = {err:.3e}"
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), f"call {call}: outputs differ"
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
