@@ -415,6 +415,77 @@ def head_measure(dev, reps=50, warmup=5):
             "traffic": HEAD_TRAFFIC_PER_CALL, "peak_source": hbm["source"] + " (burst copy)"}
 
 
+def residency_measure(dev, slots=16, K=48, W=8, T=1):
+    """Tiered expert residency on the Gemma-shaped decode: every layer's
+    routed experts in pinned host memory, a device cache of `slots` experts
+    per layer (the pages' 16-slot LFU), decisions and copies on the GPU
+    (moe_layer_forward_cached, one layer call after another).  Reports tok/s,
+    the hit rate and the bytes that crossed the host bus per token."""
+    from int4_routed_expert_02_b200.residency import CachedStack
+    cfg = synth.CONFIGS[1]
+    cs = CachedStack(cfg, 1, T, slots=slots, device=dev)
+    inputs = [synth.gen_hidden(cfg, 1, 10_000 + s, T, device=dev) for s in range(W + K)]
+    stream = torch.cuda.current_stream(dev)
+    for i in range(W):
+        cs.set_input(inputs[i])
+        cs.run()
+    torch.cuda.synchronize(dev)
+    s0 = cs.stats()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        cs.set_input(inputs[W + i])
+        cs.run()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    s1 = cs.stats()
+    hits, misses = s1["hits"] - s0["hits"], s1["misses"] - s0["misses"]
+    per_expert = expert_bytes(3 * cfg.I * cfg.H)
+    host_bytes = misses * per_expert / K
+    res = {"workload": workload_name(cfg, T) + f", routed experts in pinned host memory, {slots}-slot device "
+                                               "cache per layer (LFU, recency ties)",
+           "value": round(T * K / (ms / 1e3), 2), "unit": "tok/s", "ms_per_step": round(ms / K, 4),
+           "hit_rate": round(hits / max(hits + misses, 1), 4), "host_bytes_per_token": int(host_bytes),
+           "host_gbs": round(host_bytes * K / (ms / 1e3) / 1e9, 2), "steps": K, "warmup": W,
+           "resident_bytes": int(sum(sum(t.numel() * t.element_size() for t in l.cache.values()) +
+                                     l.dl.nbytes() for l in cs.layers)),
+           "launches_per_step": 7 * cs.L}
+    del cs
+    torch.cuda.empty_cache()
+    return res
+
+
+def ep_measure(dev, rank, world, T=1024, K=4, W=2):
+    """Expert-parallel prefill over the world's GPUs: the Gemma-shaped stack's
+    experts split in contiguous blocks, one all-reduce (NCCL) of each layer's
+    fp32 partial combine, T rows per call through every layer.  The total
+    work is fixed (strong scaling): tok/s = T * K / the slowest rank's time."""
+    from int4_routed_expert_02_b200.ep import EPStack
+    cfg = synth.CONFIGS[4]
+    ep = EPStack(cfg, 4, T, rank, world, device=dev)
+    inputs = [synth.gen_hidden(cfg, 4, 20_000 + c, T, device=dev) for c in range(W + K)]
+    stream = torch.cuda.current_stream(dev)
+    for i in range(W):
+        ep.set_input(inputs[i])
+        ep.run()
+    torch.cuda.synchronize(dev)
+    torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        ep.set_input(inputs[W + i])
+        ep.run()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = torch.tensor([e0.elapsed_time(e1)], device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"workload": workload_name(cfg, T) + f", experts split over {world} GPUs, one NCCL all-reduce per layer",
+            "value": round(T * K / (ms / 1e3), 1), "unit": "tok/s", "ms_per_call": round(ms / K, 3),
+            "scaling": "strong", "n_gpus": world}
+
+
 # --------------------------------------------------------------------------- oracle
 
 def _oracle_layer_input(cfg, cfg_id, layer, w, T):
@@ -553,6 +624,14 @@ def run_ours(args, rank, world, local_rank):
         "roofline": head_res["roofline"], "cpu_baseline": head_res.get("cpu_baseline"), "e2e": head_res["e2e"],
         "gpu_launches": head_res["gpu_launches_per_step"] * K, "clocks": head_res.get("clocks"),
     }
+    if world > 1 and args.all_configs and not (args.layers or args.tokens) and args.config == 1:
+        del st
+        torch.cuda.empty_cache()
+        try:
+            res["ep_prefill"] = ep_measure(dev, rank, world)
+        except Exception as exc:  # noqa: BLE001 -- report, keep the headline
+            res["ep_prefill"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        return res
     if not args.all_configs or world > 1 or args.layers or args.tokens or args.config != 1:
         return res
     # the rest of the workload set, each on its own weights (freed in turn)
@@ -574,6 +653,7 @@ def run_ours(args, rank, world, local_rank):
     del pst, s64
     torch.cuda.empty_cache()
     res["output_head"] = head_measure(dev)
+    res["residency"] = residency_measure(dev)
     return res
 
 

@@ -217,6 +217,50 @@ MOE_API int moe_layer_forward(const moe_layer_w *w, const uint16_t *h_in, uint16
                       size_t ws_bytes, const moe_opts *opts, void *stream);
 
 /*
+ * Tiered expert residency: a layer whose routed experts live in a pool in
+ * host memory, with a cache of `slots` experts in device memory
+ * (TurboFieldfare introduction page, section "TurboFieldfare's expert
+ * streaming structure": a 16-slot LFU cache of experts per layer, and only
+ * the misses are read; Swiftlet article, section "why the same model runs in
+ * so little memory": an LFU + recency cache pool).  The pool is the routed
+ * gate/up/down matrices of all E experts in the tiled layout (as in
+ * moe_layer_w), in pinned host memory that the GPU can address (cudaHostAlloc,
+ * or torch's pin_memory); the cache has the same layout for `slots` experts
+ * in device memory.  The bookkeeping arrays are device memory owned by the
+ * caller and set up once by moe_expert_cache_reset.
+ */
+typedef struct {
+    int slots;                              /* C >= the distinct experts one call can select: min(E, T*k) */
+    moe_qmat gate, up, down;                /* device cache, C experts */
+    moe_qmat pool_gate, pool_up, pool_down; /* host pool, E experts (device-addressable pinned memory) */
+    int32_t *slot_of;                       /* [E]: cache slot of expert e, -1 when not resident */
+    int32_t *expert_of;                     /* [C]: expert in slot s, -1 when empty */
+    uint32_t *uses;                         /* [C]: uses of the slot's expert since it was loaded */
+    uint32_t *last;                         /* [C]: the call that last used the slot */
+    uint32_t *ctl;                          /* [4]: calls, hits, misses (cumulative; distinct experts per call), spare */
+} moe_expert_cache;
+
+/* Empties the cache (every slot free, counters 0).  E: the layer's routed experts. */
+MOE_API int moe_expert_cache_reset(const moe_expert_cache *c, int E, void *stream);
+
+/*
+ * moe_layer_forward with the routed experts served from a cache.  w supplies
+ * the router, the per-expert scales and the shared expert (resident); its
+ * routed gate/up/down pointers are not used.  Per call, on the GPU: the
+ * router; then, for the distinct experts selected, in ascending expert
+ * order: a resident expert counts a use; a missing one takes the slot with
+ * the fewest uses among those this call does not need (an empty slot first;
+ * ties: least recently used, then the lowest slot) and is copied from the
+ * pool over the bus; then bucketing, the experts (on the cache, by slot) and
+ * the combine.  The result equals moe_layer_forward's on the same weights.
+ * Workspace: moe_workspace_size(w, T).  Asynchronous; MOE_EINVAL when
+ * slots < min(E, T*k).
+ */
+MOE_API int moe_layer_forward_cached(const moe_layer_w *w, const moe_expert_cache *c, const uint16_t *h_in,
+                                     uint16_t *h_out, int T, void *ws, size_t ws_bytes, const moe_opts *opts,
+                                     void *stream);
+
+/*
  * Expert-parallel split of a layer over G devices (no counterpart in the
  * pages, which run one device; the split is this library's multi-GPU form of
  * the same arithmetic).  A rank owns the routed experts [e_lo, e_hi) --
@@ -256,6 +300,13 @@ MOE_API int moe_combine(const uint16_t *h_in, const float *m, uint16_t *h_out, i
  *   h_out [L,T,H]: every layer's output (chained: layer l's output is layer
  *                 l+1's input).
  *   1 <= T <= 8, H <= 4096, T * H <= 24576.  Needs cooperative launch.
+ * opts->force_path picks how the experts' dot products run: 1 CUDA-core FMAs
+ * (exact products, fp32 sums), 2 the warp-level tensor cores (BF16 operands:
+ * codes as exact 128 + q, expert inputs as BF16 -- exact for gate/up, a
+ * high + low pair for down -- fp32 accumulation), 0 automatic: CUDA cores for
+ * T = 1, tensor cores for T >= 2 (the FMA work grows with T, the MMA's does not).
+ * The first call with a given layer array encodes TMA descriptors on the host
+ * (cached), and every call copies them into the workspace before the kernel.
  * The workspace (moe_decode_stack_workspace_size) must stay untouched until
  * the kernel finishes; its first bytes are reset by every call.  Every wait in
  * the kernel is bounded (~1 s); if one runs out the kernel records a code in
@@ -268,9 +319,11 @@ MOE_API int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h
                              int T, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream);
 
 /* 1 if moe_decode_stack can run layers shaped like `w` with T tokens on the
- * stream's device (NULL: the current device) -- its plan of shared memory
- * and work per CTA fits one CTA per SM -- else 0 (also on bad arguments).
- * Callers fall back to moe_layer_forward per layer when it returns 0. */
+ * stream's device (NULL: the current device) with the automatic path -- its
+ * plan of shared memory and work per CTA fits one CTA per SM -- else 0 (also
+ * on bad arguments).  Callers fall back to moe_layer_forward per layer when
+ * it returns 0.  (A forced path that does not fit makes moe_decode_stack
+ * return MOE_EINVAL.) */
 MOE_API int moe_decode_stack_fits(const moe_layer_w *w, int T, void *stream);
 
 /* Synchronous: reads the device error code a moe_decode_stack call left in

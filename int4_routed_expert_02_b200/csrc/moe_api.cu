@@ -108,8 +108,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // The SwiGLU buffers of the GEMV path and the token / SwiGLU matrices of the
 // tensor-core path share one region (a call uses one path).
 struct WsLayout {
-    size_t status, logits, idx, wts, xe, offsets, perm, inv, active, wts_ep, active_ep, a_routed, a_shared, xg, act, y,
-        sh, total;
+    size_t status, logits, idx, wts, xe, offsets, perm, inv, active, wts_ep, active_ep, idx_c, miss, a_routed,
+        a_shared, xg, act, y, sh, total;
 };
 
 constexpr size_t kStatusOffset = 4;
@@ -135,6 +135,8 @@ WsLayout ws_layout(const moe_layer_w *w, int T) {
     L.active = take(sizeof(int32_t) * (w->E + 1));
     L.wts_ep = take(sizeof(float) * Tk);
     L.active_ep = take(sizeof(int32_t) * (w->E + 1));
+    L.idx_c = take(sizeof(int32_t) * Tk);
+    L.miss = take(sizeof(int32_t) * (2 * (size_t)w->E + 1));
     {
         const size_t gemv_a = align256(sizeof(float) * Tk * w->I), gemv_s = align256(sizeof(float) * T * w->Is);
         const size_t mma_x = align256(moe::mma_xg_bytes(w, T)), mma_a = align256(moe::mma_act_bytes(w, T));
@@ -402,6 +404,80 @@ int moe_layer_partial(const moe_layer_w *w, const uint16_t *h_in, int T, int e_l
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
 }
 
+int moe_expert_cache_reset(const moe_expert_cache *c, int E, void *stream) {
+    const char *fn = "moe_expert_cache_reset";
+    g_err.clear();
+    if (!c) return fail(MOE_EINVAL, "%s: cache is NULL", fn);
+    if (E < 1 || c->slots < 1) return fail(MOE_EINVAL, "%s: E=%d, slots=%d", fn, E, c->slots);
+    CHECK_PTR(c->slot_of);
+    CHECK_PTR(c->expert_of);
+    CHECK_PTR(c->uses);
+    CHECK_PTR(c->last);
+    CHECK_PTR(c->ctl);
+    cudaError_t e = moe::launch_cache_reset(E, c->slots, c->slot_of, c->expert_of, c->uses, c->last, c->ctl,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
+int moe_layer_forward_cached(const moe_layer_w *w, const moe_expert_cache *c, const uint16_t *h_in, uint16_t *h_out,
+                             int T, void *ws, size_t ws_bytes, const moe_opts *opts, void *stream) {
+    const char *fn = "moe_layer_forward_cached";
+    g_err.clear();
+    if (!c) return fail(MOE_EINVAL, "%s: cache is NULL", fn);
+    if (int rc = check_dims(fn, w)) return rc;
+    if (int rc = check_T(fn, T)) return rc;
+    if ((long long)T * w->k > 65536) return fail(MOE_EINVAL, "%s: T*k exceeds 65536", fn);
+    const long long need = (long long)T * w->k < w->E ? (long long)T * w->k : w->E;
+    if (c->slots < need || c->slots > w->E)
+        return fail(MOE_EINVAL, "%s: slots=%d must be in [min(E, T*k)=%lld, E=%d]", fn, c->slots, need, w->E);
+    if (int rc = check_router_ptrs(fn, w)) return rc;
+    // the shared expert is resident; the routed experts come from the cache
+    moe_layer_w wc = *w;
+    wc.E = c->slots;
+    wc.gate = c->gate;
+    wc.up = c->up;
+    wc.down = c->down;
+    if (int rc = check_expert_ptrs(fn, &wc, 1)) return rc;
+    CHECK_PTR(c->pool_gate.q);
+    CHECK_PTR(c->pool_gate.sb);
+    CHECK_PTR(c->pool_up.q);
+    CHECK_PTR(c->pool_up.sb);
+    CHECK_PTR(c->pool_down.q);
+    CHECK_PTR(c->pool_down.sb);
+    CHECK_PTR(c->slot_of);
+    CHECK_PTR(c->expert_of);
+    CHECK_PTR(c->uses);
+    CHECK_PTR(c->last);
+    CHECK_PTR(c->ctl);
+    const moe_opts o = resolve_opts(opts);
+    if (int rc = check_opts(fn, o)) return rc;
+    CHECK_PTR(h_in);
+    CHECK_PTR(h_out);
+    if (T == 0) return MOE_OK;
+    if (int rc = check_ws(fn, w, T, ws, ws_bytes)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(w, T);
+    double *logits = at<double>(ws, L.logits);
+    int32_t *idx = at<int32_t>(ws, L.idx), *idx_c = at<int32_t>(ws, L.idx_c), *miss = at<int32_t>(ws, L.miss);
+    float *wts = at<float>(ws, L.wts);
+    uint16_t *xe = at<uint16_t>(ws, L.xe);
+    int32_t *offsets = at<int32_t>(ws, L.offsets), *perm = at<int32_t>(ws, L.perm), *inv = at<int32_t>(ws, L.inv);
+    int32_t *active = at<int32_t>(ws, L.active);
+    const moe_qmat pool[3] = {c->pool_gate, c->pool_up, c->pool_down}, cache[3] = {c->gate, c->up, c->down};
+    cudaError_t e = moe::launch_router_logits(w, h_in, T, o.eps, logits, xe, st);
+    if (e == cudaSuccess) e = moe::launch_router_topk(logits, T, w->E, w->k, w->per_expert_scale, idx, wts, st);
+    if (e == cudaSuccess)
+        e = moe::launch_residency(idx, T * w->k, w->E, c->slots, c->slot_of, c->expert_of, c->uses, c->last, c->ctl,
+                                  miss, idx_c, st);
+    if (e == cudaSuccess) e = moe::launch_fill(w, pool, cache, miss, st);
+    if (e == cudaSuccess) e = moe::launch_bucket(idx_c, T * w->k, c->slots, offsets, perm, inv, active, st);
+    if (e == cudaSuccess) e = run_experts(&wc, xe, T, offsets, perm, active, 1, ws, L, o, st);
+    if (e == cudaSuccess)
+        e = moe::launch_combine(at<float>(ws, L.y), at<float>(ws, L.sh), wts, T, w->H, w->k, 1, h_in, nullptr, h_out,
+                                o.post_norm, o.layer_scalar, o.eps, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
+}
+
 int moe_combine(const uint16_t *h_in, const float *m, uint16_t *h_out, int T, int H, const moe_opts *opts,
                 void *stream) {
     const char *fn = "moe_combine";
@@ -454,7 +530,7 @@ int moe_decode_stack_fits(const moe_layer_w *w, int T, void *stream) {
     int dev = 0, grid = 0;
     if ((st ? cudaStreamGetDevice(st, &dev) : cudaGetDevice(&dev)) != cudaSuccess) return 0;
     if (decode_grid_of(dev, &grid) != cudaSuccess || grid <= 0) return 0;
-    return moe::decode_stack_fits(w, T, grid) ? 1 : 0;
+    return moe::decode_stack_fits(w, T, grid, 0) ? 1 : 0;
 }
 
 int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained, uint16_t *h_out, int T,
@@ -497,7 +573,7 @@ int moe_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int
     if (grid <= 0)
         return fail(MOE_EINVAL, "%s: device %d cannot run the decode kernel (cooperative launch, one CTA per SM)", fn,
                     dev);
-    if (!moe::decode_stack_fits(&w0, T, grid))
+    if (!moe::decode_stack_fits(&w0, T, grid, o.force_path))
         return fail(MOE_EINVAL, "%s: T=%d with H=%d, E=%d does not fit the kernel's shared memory", fn, T, w0.H, w0.E);
     e = moe::launch_decode_stack(layers, L, h_in, chained, h_out, T, ws, o, grid, st);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, fn);
@@ -564,8 +640,9 @@ int moe_decode_stack_status(const void *ws) {
                                      "wait for another CTA's gate/up units timed out",
                                      "wait for a ring slot's hand-over timed out",
                                      "wait for the routing tables timed out",
-                                     "wait for a staged down-projection input timed out"};
-        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 8) ? what[code] : "?");
+                                     "wait for a staged down-projection input timed out",
+                                     "wait for another CTA's router logits timed out"};
+        return fail(MOE_EDEVICE, "%s: device error %d (%s)", fn, code, (code > 0 && code < 9) ? what[code] : "?");
     }
     return MOE_OK;
 }

@@ -4,55 +4,56 @@
 // Per layer (TurboFieldfare introduction page, discuss.pytorch.kr, section
 // "TurboFieldfare's expert streaming structure": router -> routed experts +
 // shared expert -> weighted combine -> normalisation, residual, layer scalar;
-// weights MLX affine, section "How TurboFieldfare saves memory"):
+// weights MLX affine, section "How TurboFieldfare saves memory"), one layer is
+// a chain of three grid-wide exchanges and the weight streams between them:
 //
-//   P0  finish the previous layer: m = sum_s w_s y_s + shared, post-norm,
-//       residual, layer scalar (every CTA, redundantly; CTA 0 writes it out),
-//       and the RMS the router needs
-//   P1  router logits in fp64 for this CTA's share of the E experts; its
-//       router rows and router_scale were bulk-copied into shared memory at
-//       the start of the layer, overlapping P0
-//   --- grid barrier ---
-//   P2  top-k + softmax * per_expert_scale and bucketing, by rank counting
-//       (every CTA, redundantly, so no barrier is needed before the experts),
-//       and this CTA's job tables for the two expert phases
-//   P2' gate/up: a job (32 rows: a row block of one slot) is split into
-//       tasks of <= 16 quantisation groups of one matrix; tasks are dealt
-//       round-robin to the CTAs and taken by teams of kWPT warps (every
-//       kWPT-th group each) independently; each warp's partial sums go to
-//       global memory, and the warp that
-//       finishes a job's last share (an atomic count per job) sums the parts
-//       in a fixed order and forms a = silu(g) * u for the job's rows, then
-//       counts the job done for its slot
-//   (no grid barrier: a CTA stages a slot's input once all of that slot's
-//   jobs are counted)
-//   P3  down: tasks of 32 rows x <= 16 groups of one slot, in contiguous
-//       blocks per CTA so that a CTA stages each slot's a once; each warp of
-//       a task's team writes its partial rows, and the warp that finishes the
-//       last share of a row block (an atomic count per row block) forms the combine
-//       m = sum_s w_s y_s + shared for those rows, then counts the row block
-//       done
-//   (no grid barrier: the next layer's P0 waits until every row block of m
-//   is counted)
+//   F  every CTA reads the previous layer's combine m (all rows), finishes that
+//      layer (post-norm, residual, layer scalar; CTA c writes its slice of the
+//      bf16 output) and forms this layer's expert input xe = bf16(rmsnorm(h)),
+//      pre-scaled for the code decode
+//   R  router logits in fp64 for this CTA's share of the experts, into global
+//      memory as flag-in-data words (each carries the layer's tag)
+//   S  the shared expert's gate/up rows of this CTA (they need only xe): each
+//      8-row unit is 8 one-row pieces, one warp each; a piece forms the row's
+//      g and u over the whole input and a = silu(g) * u, stored in global
+//      memory; the last piece of a unit counts the unit done (release)
+//   K  read every logit, polling each until it carries this layer's tag (no
+//      barrier); top-k (ties to the lower index) and
+//      softmax * per_expert_scale, redundantly on every CTA, and the
+//      bucketing of the T*k pairs into distinct experts ("slots")
+//   G  routed gate/up units (slot, 8 rows), dealt round-robin over the grid
+//      in slot order, so that early slots complete early; pieces as in S
+//   D  down projection of this CTA's output rows (8-row blocks): per slot, as
+//      soon as that slot's a is complete everywhere (its unit count), the
+//      first warp stages a into the slot's ring slot and the block tasks run
+//      -- so the down of early slots overlaps the gate/up of later ones
+//   then the CTA sums its rows' routed outputs with the gate weights and the
+//      shared output in a fixed order (deterministic), writes m, and arrives
+//      at the next layer's barrier.
 //
-// Weights stream HBM -> shared memory with 1-D bulk copies (cp.async.bulk)
-// into a ring of mbarrier-guarded slots, one slot per task, issued by one
-// producer thread ahead of 15 consumer warps (teams of kWPT = 1) that never
-// wait for one another inside a phase.  The down tasks' weights do not depend on the gate/up
-// results, so the producer already fills the slots freed during the gate/up
-// phase with them.  Once the top-k is known each CTA also asks L2 to
-// prefetch the down-projection weights of its later jobs, and during the down
-// phase its share of the next layer's shared-expert weights, so HBM keeps
-// streaming across the grid barriers.  The dot products use the subnormal
-// code decode of moe_common.cuh (one AND + one FMA per code).  Loops keep the
-// special-function pipe idle: no runtime integer division, conversion or
-// reciprocal per element (job tables are built once per layer, the ring
-// position is advanced incrementally, bf16 rounding uses integer arithmetic).
+// Weights move HBM -> shared memory by TMA tensor copies (no multicast) into a
+// ring of fixed-size slots, issued by one producer thread ahead of 15
+// consumer warps.  Once the top-k is known the producer asks L2 to prefetch
+// every routed byte this CTA will need (and, after the routed units, the next
+// layer's router and shared-expert units), so HBM streams across the
+// exchanges while the ring fills in order.  The 4-bit codes are decoded with
+// the subnormal trick of moe_common.cuh (one AND and half a packed FMA per
+// code against inputs pre-scaled per nibble position); products are exact and
+// sums fp32.  The router accumulates in fp64 so that the top-k does not depend
+// on the summation order.
 //
-// Every wait is bounded (grid barrier and mbarriers: ~1 s of globaltimer); on
-// a timeout the kernel records an error code in the workspace, stops taking
-// work, lets its own bulk copies land and returns.
+// Every wait (grid barriers, readiness counts, mbarriers, slot ownership) is
+// bounded by ~1 s of globaltimer; on a timeout the kernel records an error
+// code in the workspace, every CTA stops taking work, the producer lets its
+// own copies land, and the kernel returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
 #include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -60,58 +61,61 @@
 namespace moe {
 namespace dec {
 
-constexpr int kCWarps = 15;                   // consumer warps: with the producer 16 warps, 4 per SM sub-partition,
-                                              // so a thread may hold 128 registers (no spills)
-constexpr int kWPT = 1;                       // consumer warps per task (a team; more than one measured slower)
-constexpr int kTeams = kCWarps / kWPT;
-constexpr int kWarps = kCWarps + 1;           // + the producer warp
-constexpr int kThreads = kWarps * 32;
-constexpr int kProducerWarp = kCWarps;
-constexpr int kMaxStages = 11;                // ring slots: as many as fit beside the input stage
-constexpr int kTaskGroups = 16;               // groups per task (one ring slot)
-constexpr int kCodeBytesPerGroup = 1024;      // 32 rows x 64 codes x 4 bits
-constexpr int kSbBytesPerGroup = 128;         // 32 rows x (scale, bias)
-constexpr int kSlotBytes = 16 * (kCodeBytesPerGroup + kSbBytesPerGroup);  // 18432
+constexpr int kCW = 15;                       // consumer warps
+constexpr int kProdWarp = kCW;                // the producer warp (its lane 0 issues every copy)
+constexpr int kThreads = (kCW + 1) * 32;      // 512: 4 warps per SM sub-partition, 128 registers a thread
+constexpr int kCThreads = kCW * 32;
 constexpr int kMaxT = 8;
-constexpr int kStageFloats = 24576;           // largest input stage (T * H)
-constexpr int kPoolBytes = 11 * kSlotBytes;   // ring + input stage share this pool
-constexpr int kMaxXs = 768;
 constexpr int kMaxLayers = 64;
-constexpr int kMaxPairs = kMaxT * kMaxK;
-constexpr int kMaxTasks = 160;                // per CTA and phase
-constexpr int kMaxPG = 4;                     // gate/up parts per job (H <= 4096)
-constexpr int kMaxSegs = 16;                  // down: staged (slot, part) inputs per CTA
+constexpr int kMaxPairs = kMaxT * kMaxK;      // 256
+constexpr int kMaxSlots = 16;                 // ring slots
+constexpr int kMaps = 12;                     // TMA tensor maps per layer
+constexpr int kMaxBlk = 4;                    // 8-row output blocks per CTA (H <= 4096 on >= 128 SMs)
+constexpr int kMaxParts = 8;                  // K-parts of a down matrix
+constexpr int kPartChunks = 32;               // at most 32 chunks (1024 columns) per K-part
+constexpr int kBarCtrs = 8;                   // grid-barrier counters, 128 bytes apart
+constexpr int kMaxStageTH = 24576;            // largest T * H
+constexpr int kMaxCand = 512;                 // top-k candidates per token
 constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
 
-constexpr int kErrGridBarrier = 1, kErrFull = 2, kErrEmpty = 3, kErrReady = 4;
+enum { kErrBarrier = 1, kErrFull, kErrEmpty, kErrReady, kErrOwner, kErrTables, kErrStage, kErrLogits };
+enum {
+    kMapGateQ = 0, kMapUpQ, kMapGateSb, kMapUpSb,        // routed gate/up: codes, (scale, bias) words
+    kMapShGateQ, kMapShUpQ, kMapShGateSb, kMapShUpSb,    // shared gate/up
+    kMapDownQ, kMapDownSb, kMapShDownQ, kMapShDownSb     // routed and shared down
+};
 
-// Sizes, options and workspace pointers of a launch.  The kernel copies them
-// into shared memory once, so that every phase reads them at shared-memory
-// latency instead of through the kernel-parameter space.
+// Sizes, options, shared-memory plan and workspace pointers of a launch.
+// Copied into shared memory at the start, so phases read them at shared
+// latency instead of through the parameter space.
 struct Cfg {
-    const uint16_t *h_in;  // [T,H] (chained) or [L,T,H]
+    const uint16_t *h_in;  // chained: [T,H]; else [L,T,H]
     uint16_t *h_out;       // [L,T,H]: every layer's output
     int L, T, chained, post_norm;
     float layer_scalar, eps;
-    int H, E, k, I, Is, Kmax, R;
-    int ndp_r, ndp_s;
-    int nslots;      // ring slots (the rest of the pool is the input stage)
-    int stage_floats;  // floats in the input stage
-    unsigned *bar;
-    unsigned bar_extra;  // arrivals the grid barrier waits for beyond the grid (0; tests of the timeout path set 1)
-    int *err;
-    unsigned *cnt_dn;  // [H/32]: down tasks done per row block; reset by the last
-    unsigned *cnt_gu;  // [jobs]: gate/up tasks done per job; reset by the last
-    unsigned *act_done;   // [1 + T*k]: gate/up jobs done per slot, over all layers so far
-    unsigned *rows_done;  // row blocks of m combined, over all layers so far
-    float *gpart;      // [jobs][2][pg][kWPT][T][32]: gate/up partial sums per task member
-    double *logits;  // [T,E]
-    float *act;      // [R][Kmax]: SwiGLU output a per rowset (shared tokens, then bucketed pairs),
-                     // pre-scaled for the code decode
-    float *act_cs;   // [R][Kmax/32]: sums of a over 32-column chunks
-    float *y;        // [ndp_r * kWPT][T*k][H]: down partial sums per task member
-    float *sh;       // [ndp_s * kWPT][T][H]
-    float *m;        // [T][H]: the combine m of the current layer
+    int H, E, k, I, Is;
+    int CH, GH;                  // 32-column chunks and 64-column groups of H
+    int units_s, units_r;        // 8-row units of the shared / one routed gate (or up) matrix
+    int nrb8;                    // 8-row blocks of the output rows (H / 8)
+    int parts_s, pc_s;           // shared down: K-parts, chunks per part
+    int parts_r, pc_r;           // routed down
+    int ns, slot_bytes;          // ring slots and their size
+    int gcb;                     // bytes of one matrix's codes in a gate/up slot (1024-aligned)
+    int sbs;                     // bytes of one matrix's (scale, bias) words in a gate/up slot (128-aligned)
+    int dcb_s, dcb_r;            // bytes of one 8-row block's codes in a down slot (1024-aligned)
+    int sbd_s, sbd_r;            // bytes of one 8-row block's words in a down slot (128-aligned)
+    int maxc;                    // top-k candidate capacity per token
+    int off_ring, off_x, off_xs, off_h, off_y, off_cand, off_part;  // dynamic shared memory offsets
+    int yrows;                   // rows per ybuf entry (8 * kMaxBlk)
+    unsigned *bar;               // [kBarCtrs * 32] monotonic arrival counters
+    unsigned bar_extra;          // arrivals beyond the grid the barriers wait for (tests of the timeout path)
+    int *err;                    // device status word
+    unsigned *ready;             // [1 + kMaxPairs]: gate/up units done, shared then per routed slot
+    unsigned long long *logit_ll;  // [T,E][2]: each logit as two words (32 bits of it | layer tag << 32)
+    float *a_sh;                 // [T,Is]   SwiGLU output of the shared expert
+    float *a_r;                  // [T*k,I]  of the routed experts, by bucketed position
+    float *m;                    // [T,H]    combine of the current layer
+    const CUtensorMap *maps;     // [L][kMaps]
 };
 
 struct Params {
@@ -119,64 +123,36 @@ struct Params {
     moe_layer_w layers[kMaxLayers];
 };
 
-// One task of an expert phase: 32 rows (row block rb) x groups [g0, g1) of
-// matrix mat (gate/up: 0 gate, 1 up; down: 0) of the shared expert (slot 0)
-// or of routed expert e (slot >= 1), for n tokens starting at bucketed
-// position seg0.  job: gate/up, the CTA-local job; seg: down, the staged input.
-struct TaskDesc {
-    int16_t slot, rb, mat, part, g0, g1, n, seg;
-    int32_t seg0, e, job;
-};
-
-// A staged down-phase input: the SwiGLU rows of one (slot, part), columns
-// [g0*64, g0*64 + ld), token tt at stage offset off + tt * ld.
-struct SegDesc {
-    int16_t slot, part, n, g0, ld, pad;
-    int32_t seg0, off;
-};
-
-struct Smem {
-    alignas(128) unsigned char pool[kPoolBytes];  // ring slots, then the input stage
-    alignas(8) unsigned long long full[kMaxStages];
-    alignas(8) unsigned long long empty[kMaxStages];
-    alignas(8) unsigned long long rbar;  // router copies of the current layer
-    unsigned slot_task[kMaxStages];      // ring sequence number of the task a slot currently holds
-    float *stage;                        // input stage (inside the pool, after the ring)
-    alignas(16) float xs[kMaxXs];        // sum of x per 32-column chunk
-    float bred[32];  // block reductions
-    TaskDesc gut[kMaxTasks], dnt[kMaxTasks];
-    SegDesc seg[kMaxSegs];
-    int ngt, ndt, pg, nseg, seg_rounds;
-    unsigned act_expect[kMaxPairs + 1];  // act_done per slot once this layer's gate/up jobs are all done
-    double selv[kMaxPairs];
-    float wts[kMaxPairs];
-    int idx[kMaxPairs];
-    int perm[kMaxPairs];
-    int act_e[kMaxPairs], act_off[kMaxPairs], act_n[kMaxPairs];
-    int poff[kMaxPairs], pcnt[kMaxPairs];
-    unsigned char first[kMaxPairs];
-    int tokrow[kMaxPairs];  // bucketed position j -> row offset (token * H) of its input
-    int tokrow_sh[kMaxT];   // shared expert: token t -> t * H
-    int nact;
-    double rpart[128];
-    float rms[kMaxT];
-    float rinv[kMaxT];
-    int rcopy[3];  // router copies of this layer: first row, rows, byte offset of the scale/bias superset
-    int flag;
-    int flag2;  // consumer-only verdicts
-    Cfg c;          // the launch's Cfg
-    moe_layer_w w;  // the current layer's weights
+// Fixed part of the shared memory (at its 1024-aligned base).
+struct Shared {
+    unsigned long long full[kMaxSlots];    // ring slot filled (TMA completion)
+    unsigned long long empty[kMaxSlots];   // ring slot consumed
+    volatile unsigned owner[kMaxSlots];    // sequence number of the task a slot holds
+    int cnt[kMaxSlots];                    // pieces / block tasks of the slot's task that are done
+    volatile int astate[kMaxSlots];        // down slot: 0 a not staged, 1 staging, 2 staged
+    volatile int tables_layer;             // 1 + the layer whose routing tables are ready
+    volatile int verdict;                  // consumers: 1 while no error is recorded
+    int D;                                 // distinct experts of the current layer
+    int ccount[kMaxT];                     // top-k candidates per token
+    int slot_e[kMaxPairs], slot_off[kMaxPairs], slot_n[kMaxPairs];
+    int pos_tok[kMaxPairs];                // bucketed position -> token
+    int pos_pair[kMaxPairs];               // bucketed position -> pair id t*k + s
+    int pos_idx[kMaxPairs];                // 0, 1, 2, ...: bucketed positions (rows of the routed SwiGLU buffer)
+    int first[kMaxPairs];                  // pair is the first of its expert
+    int idx[kMaxPairs];                    // [t][s] selected expert
+    double selv[kMaxPairs];                // [t][s] its logit
+    float wts[kMaxPairs];                  // [t][s] gate weight
+    unsigned exp_ready[1 + kMaxPairs];     // readiness counts expected once this layer's units are done
+    float rms[kMaxT], rinv[kMaxT];
+    float red[32];
+    double rpart[kCW];                     // router partial sums (fewer items than warps)
+    int toks_sh[kMaxT];                    // 0, 1, ..., T-1
+    Cfg c;
 };
 
 // ------------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-// Block-cooperative copy of a 4-byte-aligned struct (no barrier).
-__device__ __forceinline__ void copy_words(void *dst, const void *src, size_t bytes) {
-    for (int i = threadIdx.x; i < (int)(bytes / 4); i += blockDim.x)
-        static_cast<unsigned *>(dst)[i] = static_cast<const unsigned *>(src)[i];
-}
 
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
@@ -208,7 +184,18 @@ __device__ __forceinline__ bool mbar_test(unsigned long long *b, unsigned parity
 
 __device__ __forceinline__ int ldcg_int(const int *p) { return __ldcg(p); }
 
-// Bounded wait for the phase with `parity` of mbarrier `b` to complete.
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait for the phase with `parity` of mbarrier `b`; false on a timeout
+// (recorded with `code`) or when an error is already recorded.
 __device__ __noinline__ bool mbar_wait(unsigned long long *b, unsigned parity, int *err, int code) {
     if (mbar_test(b, parity)) return true;
     const unsigned long long t0 = globaltimer();
@@ -224,7 +211,7 @@ __device__ __noinline__ bool mbar_wait(unsigned long long *b, unsigned parity, i
     }
 }
 
-// Bounded wait used only when draining: ignores the error flag.
+// Bounded wait used when stopping: ignores the error word.
 __device__ __noinline__ void mbar_drain(unsigned long long *b, unsigned parity) {
     const unsigned long long t0 = globaltimer();
     while (!mbar_test(b, parity)) {
@@ -244,374 +231,314 @@ __device__ __forceinline__ void prefetch_l2(const void *src, unsigned bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-// Prefetch [p, p + bytes) into L2 in pieces of at most 64 KiB (16-byte units).
-__device__ __forceinline__ void prefetch_range(const void *p, size_t bytes) {
-    const char *c = static_cast<const char *>(p);
-    while (bytes >= 16) {
-        const unsigned n = (unsigned)(bytes > 65536 ? 65536 : (bytes & ~(size_t)15));
-        prefetch_l2(c, n);
-        c += n;
-        bytes -= n;
-    }
+// 3-D tiled TMA load (no multicast) of the box at (x, y, z) of `map`.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z,
+                                            unsigned long long *b) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(b))
+        : "memory");
 }
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCWarps * 32) : "memory"); }
+// The same box into L2 only.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
+                 "r"(z)
+                 : "memory");
+}
 
-// Grid-wide barrier number `nth` (1, 2, ...) on a monotonically increasing
-// counter; bounded.  Returns false (in every thread of the CTA alike) if any
-// CTA recorded an error.
-__device__ __noinline__ bool grid_sync(const Cfg &P, unsigned nth, int *verdict) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(P.bar, 1u);
+// Named barrier of the 15 consumer warps.
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCThreads) : "memory"); }
+
+// ------------------------------------------------------------------ grid barrier (split phase)
+
+// Arrival of this CTA (thread 0 of the consumers, after a consumer barrier):
+// its global writes become visible before the count.
+__device__ __forceinline__ void grid_arrive(const Cfg &P) {
+    __threadfence();
+    red_release_add(P.bar + 32 * (blockIdx.x % kBarCtrs), 1u);
+}
+
+// Wait until every CTA has arrived `nth` times (sum of the counters); called
+// by all consumer threads.  False (uniformly) if an error is recorded.
+__device__ __noinline__ bool grid_wait(const Cfg &P, Shared &S, unsigned nth) {
+    consumer_sync();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
         const unsigned target = nth * gridDim.x + P.bar_extra;
         const unsigned long long t0 = globaltimer();
+        bool ok = true;
         for (unsigned it = 0;; ++it) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(P.bar) : "memory");
+            unsigned v = lane < kBarCtrs ? ld_acquire(P.bar + 32 * lane) : 0u;
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
             if (v >= target) break;
             if ((it & 63u) == 63u) {
-                if (ldcg_int(P.err) != 0) break;
-                if (globaltimer() - t0 > kWaitNs) {
-                    atomicCAS(P.err, 0, kErrGridBarrier);
+                int bad = 0;
+                if (lane == 0) {
+                    bad = ldcg_int(P.err) != 0;
+                    if (!bad && globaltimer() - t0 > kWaitNs) {
+                        atomicCAS(P.err, 0, kErrBarrier);
+                        bad = 1;
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, bad, 0)) {
+                    ok = false;
                     break;
                 }
             }
-            __nanosleep(32);
         }
         __threadfence();
-        *verdict = ldcg_int(P.err) == 0;
+        if (lane == 0) S.verdict = ok && ldcg_int(P.err) == 0;
     }
-    __syncthreads();
-    return *verdict != 0;
+    consumer_sync();
+    return S.verdict != 0;
 }
 
-// ------------------------------------------------------------------ jobs
-
-// Task gt (grid-wide index; this CTA takes gt = c, c + G, ...) of the gate/up
-// phase.  Job j = gt / (2 pg) is 32 rows of the shared expert or of one
-// active slot; its 2 pg tasks are part p of gate and of up, p = 0..pg-1.
-// All divisions happen here, once per task.
-__device__ __forceinline__ TaskDesc make_gu_task(const Cfg &P, const Smem &S, int gt, int pg) {
-    TaskDesc t;
-    const int j = gt / (2 * pg), r = gt - j * 2 * pg;
-    const int A = P.Is / 32;
-    if (j < A) {
-        t.slot = 0;
-        t.rb = (int16_t)j;
-        t.n = (int16_t)P.T;
-        t.seg0 = 0;
-        t.e = -1;
-    } else {
-        const int B = P.I / 32, jj = j - A, a = jj / B;
-        t.slot = (int16_t)(1 + a);
-        t.rb = (int16_t)(jj - a * B);
-        t.seg0 = S.act_off[a];
-        t.n = (int16_t)S.act_n[a];
-        t.e = S.act_e[a];
-    }
-    const int GH = P.H / 64;
-    t.mat = (int16_t)(r & 1);
-    t.part = (int16_t)(r >> 1);
-    t.g0 = (int16_t)(GH * t.part / pg);
-    t.g1 = (int16_t)(GH * (t.part + 1) / pg);
-    t.job = j;
-    t.seg = 0;
-    return t;
-}
-
-// (slot, part) number sp of the down phase: the shared expert's parts first,
-// then each active slot's.
-__device__ __forceinline__ void dn_slot_part(const Cfg &P, int sp, int &slot, int &part) {
-    if (sp < P.ndp_s) {
-        slot = 0;
-        part = sp;
-    } else {
-        const int a = (sp - P.ndp_s) / P.ndp_r;
-        slot = 1 + a;
-        part = sp - P.ndp_s - a * P.ndp_r;
+// Bounded wait of lane 0 until a global count reaches `target` (acquire).
+__device__ __noinline__ bool wait_count(const Cfg &P, const unsigned *ctr, unsigned target) {
+    const unsigned long long t0 = globaltimer();
+    for (unsigned it = 0;; ++it) {
+        if (ld_acquire(ctr) >= target) return true;
+        if ((it & 63u) == 63u) {
+            if (ldcg_int(P.err) != 0) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                atomicCAS(P.err, 0, kErrReady);
+                return false;
+            }
+        }
+        __nanosleep(32);
     }
 }
 
-// Task d (grid-wide index) of the down phase: (slot, part) d / (H/32), row block d % (H/32).
-__device__ __forceinline__ TaskDesc make_dn_task(const Cfg &P, const Smem &S, int d, int sp0) {
-    TaskDesc t;
-    const int RBH = P.H / 32, sp = d / RBH;
-    int slot, part;
-    dn_slot_part(P, sp, slot, part);
-    t.slot = (int16_t)slot;
-    t.part = (int16_t)part;
-    t.rb = (int16_t)(d - sp * RBH);
-    t.mat = 0;
-    const int G = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
-    t.g0 = (int16_t)(G * part / nd);
-    t.g1 = (int16_t)(G * (part + 1) / nd);
-    if (slot == 0) {
-        t.n = (int16_t)P.T;
-        t.seg0 = 0;
-        t.e = -1;
-    } else {
-        t.seg0 = S.act_off[slot - 1];
-        t.n = (int16_t)S.act_n[slot - 1];
-        t.e = S.act_e[slot - 1];
-    }
-    t.job = 0;
-    t.seg = (int16_t)(sp - sp0);
-    return t;
+// The logits exchange carries its own validity: a logit is written as two
+// 8-byte words, each holding 32 bits of it and the layer's tag (1 + layer)
+// above them.  An aligned 8-byte store is seen whole or not at all, so a
+// reader that finds the current tag in both words has the value, with no
+// barrier between the router and the top-k.  (Every CTA writes the next
+// layer's logits only after the layer-end barrier, which every reader has
+// passed.)  The workspace is zeroed per launch, and tags start at 1.
+__device__ __forceinline__ void put_logit(const Cfg &P, int t, int e, double v, unsigned tag) {
+    const unsigned long long b = (unsigned long long)__double_as_longlong(v);
+    unsigned long long *w = P.logit_ll + 2 * ((size_t)t * P.E + e);
+    const unsigned long long w0 = (b & 0xffffffffull) | ((unsigned long long)tag << 32);
+    const unsigned long long w1 = (b >> 32) | ((unsigned long long)tag << 32);
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(w), "l"(w0) : "memory");
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(w + 1), "l"(w1) : "memory");
 }
 
-// Weight pointers (codes, scale/bias words) of a task's row block.
-__device__ __forceinline__ void task_ptrs(const Cfg &P, const moe_layer_w &W, const TaskDesc &t, bool down,
-                                          const uint32_t *&q, const uint32_t *&sb) {
-    if (!down) {
-        const size_t CH = P.H / 32, GH = P.H / 64;
-        const moe_qmat &M = t.slot == 0 ? (t.mat ? W.sh_up : W.sh_gate) : (t.mat ? W.up : W.gate);
-        const size_t mrb = t.slot == 0 ? (size_t)t.rb : (size_t)t.e * (P.I / 32) + t.rb;
-        q = M.q + mrb * CH * 128;
-        sb = M.sb + mrb * GH * 32;
-    } else if (t.slot == 0) {
-        q = W.sh_down.q + (size_t)t.rb * (P.Is / 32) * 128;
-        sb = W.sh_down.sb + (size_t)t.rb * (P.Is / 64) * 32;
-    } else {
-        const size_t mrb = (size_t)t.e * (P.H / 32) + t.rb;
-        q = W.down.q + mrb * (P.I / 32) * 128;
-        sb = W.down.sb + mrb * (P.I / 64) * 32;
-    }
-}
-
-// rowset of the tt-th token of a task (shared: the token; routed: T + bucketed position)
-__device__ __forceinline__ int task_rowset(const Cfg &P, const TaskDesc &t, int tt) {
-    return t.slot == 0 ? tt : P.T + t.seg0 + tt;
-}
-
-// Producer: the copies that fill ring slot s with groups [g0, g1) of one
-// matrix: codes (ng KiB), then the (scale, bias) words (ng * 128 B).
-__device__ __forceinline__ void issue_task(Smem &S, int s, const uint32_t *q, const uint32_t *sb, int g0, int g1) {
-    const int ng = g1 - g0;
-    const unsigned cb = (unsigned)ng * kCodeBytesPerGroup, sbb = (unsigned)ng * kSbBytesPerGroup;
-    unsigned char *slot = S.pool + (size_t)s * kSlotBytes;
-    mbar_expect_tx(&S.full[s], cb + sbb);
-    bulk_g2s(slot, q + (size_t)g0 * 256, cb, &S.full[s]);
-    bulk_g2s(slot + cb, sb + (size_t)g0 * 32, sbb, &S.full[s]);
-}
-
-// ------------------------------------------------------------------ dot products
-
-// One (matrix, group) of a job for tokens [t0, t0 + n), n <= NT <= 2: lanes
-// are the 32 rows.  w: this lane's 64 codes of the group; s (already times
-// 2^49) and b: its scale and bias.  The input of token tt starts at
-// x + off(tt), its chunk sums at xsum + off(tt) / 32, where off(tt) =
-// tokrow[tt] (gathered tokens) or tt * stride (when tokrow is null).
-template <int NT>
-__device__ __forceinline__ void group_dot(const uint32_t (&w)[8], float s, float b, const float *x,
-                                          const float *xsum, const int *tokrow, int stride, int t0, int n,
-                                          float (&acc)[4]) {
-    constexpr int NA = NT == 1 ? 2 : 1;  // packed accumulators per token: 2 for ILP when alone
-    float2 a[NT][NA];
-    int xo[NT];
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt) {
-#pragma unroll
-        for (int z = 0; z < NA; ++z) a[tt][z] = make_float2(0.f, 0.f);
-        xo[tt] = tt < n ? (tokrow ? tokrow[t0 + tt] : (t0 + tt) * stride) : 0;
-    }
-#pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-        const Decoded8 f = decode_word(w[wi]);
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt) {
-            if (tt < n) {
-                const float4 *x4 = reinterpret_cast<const float4 *>(x + xo[tt] + wi * 8);
-                const float4 xa = x4[0], xb = x4[1];
-                a[tt][0] = ffma2(make_float2(f.f[0], f.f[1]), make_float2(xa.x, xa.y), a[tt][0]);
-                a[tt][NA - 1] = ffma2(make_float2(f.f[2], f.f[3]), make_float2(xa.z, xa.w), a[tt][NA - 1]);
-                a[tt][0] = ffma2(make_float2(f.f[4], f.f[5]), make_float2(xb.x, xb.y), a[tt][0]);
-                a[tt][NA - 1] = ffma2(make_float2(f.f[6], f.f[7]), make_float2(xb.z, xb.w), a[tt][NA - 1]);
+// Bounded poll for logit (t, e) of the layer with `tag`; false (error
+// recorded) when it does not arrive.
+__device__ __forceinline__ bool get_logit(const Cfg &P, int t, int e, unsigned tag, double &v) {
+    const unsigned long long *w = P.logit_ll + 2 * ((size_t)t * P.E + e);
+    unsigned long long w0, w1;
+    unsigned long long t0 = 0;
+    for (unsigned it = 0;; ++it) {
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w0) : "l"(w) : "memory");
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w1) : "l"(w + 1) : "memory");
+        if ((unsigned)(w0 >> 32) == tag && (unsigned)(w1 >> 32) == tag) break;
+        if ((it & 63u) == 63u) {
+            if (ldcg_int(P.err) != 0) return false;
+            if (t0 == 0) {
+                t0 = globaltimer();
+            } else if (globaltimer() - t0 > kWaitNs) {
+                atomicCAS(P.err, 0, kErrLogits);
+                return false;
             }
         }
     }
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt) {
-        if (tt < n) {
-            float d = a[tt][0].x + a[tt][0].y;
-            if (NA == 2) d += a[tt][NA - 1].x + a[tt][NA - 1].y;
-            const int c = xo[tt] >> 5;
-            acc[tt] = fmaf(s, d, fmaf(b, xsum[c] + xsum[c + 1], acc[tt]));
-        }
-    }
+    v = __longlong_as_double((long long)((w0 & 0xffffffffull) | (w1 << 32)));
+    return true;
 }
 
-// One (matrix, group) for the n <= NT tokens of a job, in calls of at most two
-// tokens (codes are decoded once per call); acc[tt] is token tt's sum.
-template <int NT>
-__device__ __forceinline__ void group_dot_n(const unsigned char *codes, uint32_t sbw, const float *x,
-                                            const float *xsum, const int *tokrow, int stride, int n,
-                                            float (&acc)[NT], int lane) {
-    const uint4 c0 = reinterpret_cast<const uint4 *>(codes)[lane];
-    const uint4 c1 = reinterpret_cast<const uint4 *>(codes + 512)[lane];
-    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const float s = bf16_bits_to_float(sbw & 0xffffu) * kCodeUnscale, b = bf16_bits_to_float(sbw >> 16);
-    if (NT == 1) {
-        float a4[4] = {acc[0], 0.f, 0.f, 0.f};
-        group_dot<1>(w, s, b, x, xsum, tokrow, stride, 0, 1, a4);
-        acc[0] = a4[0];
-        return;
-    }
-#pragma unroll
-    for (int t0 = 0; t0 < NT; t0 += 2) {
-        if (t0 < n) {
-            float p[4] = {acc[t0], t0 + 1 < NT ? acc[t0 + 1 < NT ? t0 + 1 : 0] : 0.f, 0.f, 0.f};
-            group_dot<2>(w, s, b, x, xsum, tokrow, stride, t0, min(2, n - t0), p);
-            acc[t0] = p[0];
-            if (t0 + 1 < NT) acc[t0 + 1 < NT ? t0 + 1 : 0] = p[1];
+// A consumer warp's wait for ring task `seq`: first until the producer has
+// handed the slot to it (the slot's previous task is consumed, so its full
+// barrier is in this task's phase), then for the bytes.  Warps take tasks out
+// of ring order; without the first wait a warp could test a phase two ahead of
+// the barrier's own, which the parity test cannot tell apart.
+__device__ __noinline__ bool wait_task(Shared &S, const Cfg &P, unsigned seq) {
+    const int s = (int)(seq % (unsigned)P.ns);
+    const unsigned ph = (seq / (unsigned)P.ns) & 1u;
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0 && S.owner[s] != seq) {
+        const unsigned long long t0 = globaltimer();
+        for (unsigned it = 0; S.owner[s] != seq; ++it) {
+            if ((it & 63u) == 63u) {
+                if (ldcg_int(P.err) != 0 || globaltimer() - t0 > kWaitNs) {
+                    atomicCAS(P.err, 0, kErrOwner);
+                    ok = 0;
+                    break;
+                }
+            }
         }
     }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    return ok && mbar_wait(&S.full[s], ph, P.err, kErrFull);
 }
 
 // ------------------------------------------------------------------ phases
 
-// Input rows of a layer straight from global memory (bf16) into S.stage, and their RMS.
-__device__ __noinline__ void load_input(const Cfg &P, Smem &S, const uint16_t *h) {
-    const int T = P.T, H = P.H, H2 = H / 2;
-    float *stage = S.stage;
+constexpr int kXStride = 36;  // floats per 32-column chunk of a staged input (padding spreads the banks)
+
+// Sum over the consumer threads, the same in every CTA (fixed order).
+__device__ __forceinline__ float consumer_sum(float v, float *red) {
+    v = warp_sum(v);
+    consumer_sync();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    consumer_sync();
+    float s = 0.f;
+#pragma unroll 1
+    for (int i = 0; i < kCW; ++i) s += red[i];
+    return s;
+}
+
+// Layer input rows (bf16) from global memory into the h stage.
+__device__ __noinline__ void load_h(const Cfg &P, uint16_t *hs, const uint16_t *src) {
+    const int n = P.T * P.H / 8;  // 16-byte units
+#pragma unroll 1
+    for (int i = threadIdx.x; i < n; i += kCThreads)
+        reinterpret_cast<uint4 *>(hs)[i] = __ldcg(reinterpret_cast<const uint4 *>(src) + i);
+    consumer_sync();
+}
+
+// Output of layer lp: m (every row, from global memory), post-norm,
+// residual, layer scalar.  Every CTA computes the whole output; CTA c writes
+// its slice of 4-column quads to h_out[lp]; chained stacks keep the output in
+// the h stage as the next layer's input.
+__device__ __noinline__ void finish_layer(const Cfg &P, Shared &S, uint16_t *hs, int lp) {
+    const int T = P.T, H = P.H, H4 = H / 4;
+    uint16_t *out = P.h_out + (size_t)lp * T * H;
+    const int q0 = (int)((long long)H4 * blockIdx.x / gridDim.x), q1 = (int)((long long)H4 * (blockIdx.x + 1) / gridDim.x);
+    const float scalar = P.layer_scalar;
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        float4 mr[3];
+        float ss = 0.f;
+#pragma unroll
+        for (int r = 0; r < 3; ++r) {
+            const int i4 = threadIdx.x + r * kCThreads;
+            mr[r] = i4 < H4 ? __ldcg(reinterpret_cast<const float4 *>(P.m + (size_t)t * H) + i4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            ss += mr[r].x * mr[r].x + mr[r].y * mr[r].y + mr[r].z * mr[r].z + mr[r].w * mr[r].w;
+        }
+        ss = consumer_sum(ss, S.red);
+        const float inv = P.post_norm ? 1.0f / sqrtf(ss / (float)H + P.eps) : 1.0f;
+#pragma unroll
+        for (int r = 0; r < 3; ++r) {
+            const int i4 = threadIdx.x + r * kCThreads;
+            if (i4 < H4) {
+                uint2 hv = reinterpret_cast<const uint2 *>(hs + (size_t)t * H)[i4];
+                const float mv[4] = {mr[r].x, mr[r].y, mr[r].z, mr[r].w};
+                const uint32_t hw[2] = {hv.x, hv.y};
+                uint32_t o[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float hp = bf16_bits_to_float((hw[c >> 1] >> (16 * (c & 1))) & 0xffffu);
+                    o[c] = f32_to_bf16_bits_alu((hp + mv[c] * inv) * scalar);
+                }
+                const uint2 ov = make_uint2(o[0] | (o[1] << 16), o[2] | (o[3] << 16));
+                if (i4 >= q0 && i4 < q1) reinterpret_cast<uint2 *>(out + (size_t)t * H)[i4] = ov;
+                if (P.chained) reinterpret_cast<uint2 *>(hs + (size_t)t * H)[i4] = ov;
+            }
+        }
+    }
+    consumer_sync();
+}
+
+// RMS of the layer input, xe = bf16(rmsnorm_no_scale(h)) pre-scaled for the
+// code decode into x ([T][CH][kXStride]), and the chunk sums of xe into xs.
+__device__ __noinline__ void stage_x(const Cfg &P, Shared &S, const uint16_t *hs, float *x, float *xs) {
+    const int T = P.T, H = P.H, H4 = H / 4, CH = P.CH, lane = threadIdx.x & 31;
 #pragma unroll 1
     for (int t = 0; t < T; ++t) {
         float ss = 0.f;
 #pragma unroll 1
-        for (int i = threadIdx.x; i < H2; i += blockDim.x) {
-            const uint32_t v = __ldcg(reinterpret_cast<const unsigned int *>(h + (size_t)t * H) + i);
+        for (int i = threadIdx.x; i < H / 2; i += kCThreads) {
+            const uint32_t v = reinterpret_cast<const uint32_t *>(hs + (size_t)t * H)[i];
             const float a = bf16_bits_to_float(v & 0xffffu), b = bf16_bits_to_float(v >> 16);
-            stage[(size_t)t * H + 2 * i] = a;
-            stage[(size_t)t * H + 2 * i + 1] = b;
             ss = fmaf(a, a, fmaf(b, b, ss));
         }
-        ss = block_sum(ss, S.bred);
+        ss = consumer_sum(ss, S.red);
         if (threadIdx.x == 0) {
             S.rms[t] = sqrtf(ss / (float)H + P.eps);
             S.rinv[t] = 1.0f / S.rms[t];
         }
     }
-    __syncthreads();
-}
-
-// P0: output of layer lp (its combine m, post-norm, residual, scalar) into
-// S.stage as floats, with its RMS; CTA 0 also writes it to h_out[lp].
-// H/4 <= 1024 < 2 * blockDim, so two float4 per thread cover a row.
-__device__ __noinline__ void finish_layer(const Cfg &P, Smem &S, int lp) {
-    const int T = P.T, H = P.H, H4 = H / 4;
-    const uint16_t *hprev = (P.chained && lp > 0) ? P.h_out + (size_t)(lp - 1) * T * H
-                                                  : (P.chained ? P.h_in : P.h_in + (size_t)lp * T * H);
-    uint16_t *out = P.h_out + (size_t)lp * T * H;
-    float *stage = S.stage;
-    const float scalar = P.layer_scalar;
+    consumer_sync();
+    const int n4 = T * H4, rounds = (n4 + kCThreads - 1) / kCThreads;
 #pragma unroll 1
-    for (int t = 0; t < T; ++t) {
-        float4 mreg[2];
-        uint2 hreg[2];
-        float ss = 0.f;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int i4 = threadIdx.x + r * blockDim.x;
-            mreg[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-            hreg[r] = make_uint2(0u, 0u);
-            if (i4 < H4) {
-                hreg[r] = __ldcg(reinterpret_cast<const uint2 *>(hprev + (size_t)t * H) + i4);
-                mreg[r] = __ldcg(reinterpret_cast<const float4 *>(P.m + (size_t)t * H) + i4);
-            }
+    for (int r = 0; r < rounds; ++r) {  // every consumer runs every round: the shuffles need whole warps
+        const int i = r * kCThreads + threadIdx.x;
+        float sx = 0.f;
+        if (i < n4) {
+            const int t = i / H4, col = 4 * (i - t * H4);
+            const uint2 hv = reinterpret_cast<const uint2 *>(hs)[i];
+            const float ri = S.rinv[t];
+            const float x0 = bf16_bits_to_float(f32_to_bf16_bits_alu(bf16_bits_to_float(hv.x & 0xffffu) * ri));
+            const float x1 = bf16_bits_to_float(f32_to_bf16_bits_alu(bf16_bits_to_float(hv.x >> 16) * ri));
+            const float x2 = bf16_bits_to_float(f32_to_bf16_bits_alu(bf16_bits_to_float(hv.y & 0xffffu) * ri));
+            const float x3 = bf16_bits_to_float(f32_to_bf16_bits_alu(bf16_bits_to_float(hv.y >> 16) * ri));
+            const int c = col & 7;  // 0 or 4
+            float4 v;
+            v.x = x0 * code_prescale(c);
+            v.y = x1 * code_prescale(c + 1);
+            v.z = x2 * code_prescale(c + 2);
+            v.w = x3 * code_prescale(c + 3);
+            *reinterpret_cast<float4 *>(x + ((size_t)t * CH + (col >> 5)) * kXStride + (col & 31)) = v;
+            sx = (x0 + x1) + (x2 + x3);
         }
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-            ss += mreg[r].x * mreg[r].x + mreg[r].y * mreg[r].y + mreg[r].z * mreg[r].z + mreg[r].w * mreg[r].w;
-        ss = block_sum(ss, S.bred);
-        const float inv = P.post_norm ? 1.0f / sqrtf(ss / (float)H + P.eps) : 1.0f;
-        float ss2 = 0.f;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int i4 = threadIdx.x + r * blockDim.x;
-            if (i4 < H4) {
-                const float mv[4] = {mreg[r].x, mreg[r].y, mreg[r].z, mreg[r].w};
-                const uint32_t hv[2] = {hreg[r].x, hreg[r].y};
-                uint32_t o[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float hp = bf16_bits_to_float((hv[c >> 1] >> (16 * (c & 1))) & 0xffffu);
-                    o[c] = f32_to_bf16_bits_alu((hp + mv[c] * inv) * scalar);
-                    const float of = bf16_bits_to_float(o[c]);
-                    stage[(size_t)t * H + 4 * i4 + c] = of;
-                    ss2 = fmaf(of, of, ss2);
-                }
-                if (blockIdx.x == 0)
-                    reinterpret_cast<uint2 *>(out + (size_t)t * H)[i4] = make_uint2(o[0] | (o[1] << 16), o[2] | (o[3] << 16));
-            }
-        }
-        ss2 = block_sum(ss2, S.bred);
-        if (threadIdx.x == 0) {
-            S.rms[t] = sqrtf(ss2 / (float)H + P.eps);
-            S.rinv[t] = 1.0f / S.rms[t];
-        }
+        sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 4);
+        if (i < n4 && (lane & 7) == 0) xs[i >> 3] = sx;  // 8 quads = one chunk: index t * CH + chunk
     }
-    __syncthreads();
+    consumer_sync();
 }
 
-// Producer, at the start of layer l: router_scale, this CTA's router rows
-// [e0, e1) and a 16-byte-aligned superset of their scales and biases, into
-// the ring (idle until the top-k), completing on S.rbar (one phase per layer).
-__device__ __noinline__ void issue_router_copies(const Cfg &P, Smem &S, const moe_layer_w &W) {
-    const int E = P.E, H = P.H, G = H / 64;
-    const int e0 = (int)((long long)E * blockIdx.x / gridDim.x), e1 = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);
-    const int nrows = e1 - e0;
-    unsigned char *base = S.pool;
-    const unsigned rs_bytes = (unsigned)H * 2, rows_bytes = (unsigned)nrows * H;
-    const unsigned sb_lo = (unsigned)((size_t)e0 * G * 2) & ~15u;
+// Router rows [e0, e1) of this CTA and the byte layout of their copy in a ring slot:
+// [router_scale: 2H][rows: nrows * H][scale superset: sbb][bias superset: sbb].
+struct RouterCopy {
+    int e0, nrows;
+    unsigned sb_lo, sbb;
+};
+
+__device__ __forceinline__ RouterCopy router_copy(const Cfg &P) {
+    RouterCopy r;
+    const int G = P.GH;
+    r.e0 = (int)((long long)P.E * blockIdx.x / gridDim.x);
+    const int e1 = (int)((long long)P.E * (blockIdx.x + 1) / gridDim.x);
+    r.nrows = e1 - r.e0;
+    r.sb_lo = (unsigned)((size_t)r.e0 * G * 2) & ~15u;
     const unsigned sb_hi = ((unsigned)((size_t)e1 * G * 2) + 15u) & ~15u;
-    const unsigned sb_bytes = nrows > 0 ? sb_hi - sb_lo : 0u;
-    S.rcopy[0] = e0;
-    S.rcopy[1] = nrows;
-    S.rcopy[2] = (int)sb_lo;
-    mbar_expect_tx(&S.rbar, rs_bytes + rows_bytes + 2 * sb_bytes);
-    // layout: [router_scale (H*2)] [rows (nrows*H)] [scales (sb_bytes)] [biases (sb_bytes)]
-    bulk_g2s(base, W.router_scale, rs_bytes, &S.rbar);
-    if (nrows > 0) {
-        bulk_g2s(base + rs_bytes, W.router_q + (size_t)e0 * (H / 4), rows_bytes, &S.rbar);
-        bulk_g2s(base + rs_bytes + rows_bytes, reinterpret_cast<const char *>(W.router_s) + sb_lo, sb_bytes, &S.rbar);
-        bulk_g2s(base + rs_bytes + rows_bytes + sb_bytes, reinterpret_cast<const char *>(W.router_b) + sb_lo, sb_bytes,
-                 &S.rbar);
-    }
+    r.sbb = r.nrows > 0 ? sb_hi - r.sb_lo : 0u;
+    return r;
 }
 
-// P1: router logits of this CTA's experts for every token, from the copies in
-// the ring.  The dot products accumulate in fp64 so that the top-k order does
-// not depend on summation order; the common factor 1 / (rms * sqrt(H)) of a
+// R: logits of this CTA's experts for every token.  The dot products run in
+// fp64 (h * router_scale is exact in fp32; the 8-bit code becomes a double by
+// the 2^52 exponent trick), and the common factor 1 / (rms * sqrt(H)) of a
 // token's logits is applied last (it cannot change their order).
-__device__ __noinline__ void router_phase(const Cfg &P, Smem &S, int l) {
-    const int T = P.T, H = P.H, E = P.E, G = H / 64, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    __syncthreads();  // S.rcopy written by the producer thread
-    const int e0 = S.rcopy[0], nrows = S.rcopy[1], sb_lo = S.rcopy[2];
-    const int items = nrows * T;
-    // every thread waits for the copies (they are issued even when nrows == 0);
-    // the verdict is made uniform before the barriers below
-    const bool got = __syncthreads_and(mbar_wait(&S.rbar, (unsigned)(l & 1), P.err, kErrFull)) != 0;
-    const unsigned char *base = S.pool;
-    const uint16_t *rsc = reinterpret_cast<const uint16_t *>(base);
-    const unsigned rows_bytes = (unsigned)nrows * H;
-    const unsigned sb_hi = ((unsigned)((size_t)(e0 + nrows) * G * 2) + 15u) & ~15u;
-    const unsigned sb_bytes = nrows > 0 ? sb_hi - (unsigned)sb_lo : 0u;
-    const unsigned char *rows = base + H * 2;
-    const int sb_skip = (int)((size_t)e0 * G * 2) - sb_lo;
-    const uint16_t *scs = reinterpret_cast<const uint16_t *>(rows + rows_bytes + sb_skip);
-    const uint16_t *bis = reinterpret_cast<const uint16_t *>(rows + rows_bytes + sb_bytes + sb_skip);
-    if (items > 0 && got) {
-        const int parts = items >= kWarps ? 1 : kWarps / items;
-        const int units = items * parts;
-        const int nch = H / 16;
-        const float *stage = S.stage;
+__device__ __noinline__ void router_compute(const Cfg &P, Shared &S, const unsigned char *slot, const uint16_t *hs,
+                                            double *rpart, bool got, unsigned tag) {
+    const int T = P.T, H = P.H, G = P.GH, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const RouterCopy rc = router_copy(P);
+    const int items = rc.nrows * T;
+    if (items > 0) {
+        const int parts = items >= kCW ? 1 : kCW / items, units = items * parts, nch = H / 16;
+        const uint16_t *rsc = reinterpret_cast<const uint16_t *>(slot);
+        const unsigned char *rows = slot + 2 * H;
+        const int sb_skip = (int)((size_t)rc.e0 * G * 2) - (int)rc.sb_lo;
+        const uint16_t *scs = reinterpret_cast<const uint16_t *>(rows + (size_t)rc.nrows * H + sb_skip);
+        const uint16_t *bis = reinterpret_cast<const uint16_t *>(rows + (size_t)rc.nrows * H + rc.sbb + sb_skip);
+        const double sqrt_h = sqrt((double)H);
 #pragma unroll 1
-        for (int u = wid; u < units; u += kWarps) {
+        for (int u = got ? wid : units; u < units; u += kCW) {
             const int item = u / parts, part = u - item * parts;
             const int er = item / T, t = item - er * T;
             const int c0 = nch * part / parts, c1 = nch * (part + 1) / parts;
-            const float *h = stage + (size_t)t * H;
+            const uint16_t *h = hs + (size_t)t * H;
             double acc = 0.0;
 #pragma unroll 1
             for (int c = c0 + lane; c < c1; c += 32) {
@@ -623,9 +550,7 @@ __device__ __noinline__ void router_phase(const Cfg &P, Smem &S, int l) {
 #pragma unroll
                     for (int bi = 0; bi < 4; ++bi) {
                         const int i = c * 16 + wi * 4 + bi;
-                        // h * router_scale is exact in fp32 (two bf16 values)
-                        const double z = (double)(h[i] * bf16_bits_to_float(rsc[i]));
-                        // the 8-bit code as a double: 2^52 + q read as fp64, minus 2^52 (exact)
+                        const double z = (double)(bf16_bits_to_float(h[i]) * bf16_bits_to_float(rsc[i]));
                         const double qd =
                             __hiloint2double(0x43300000, (int)((words[wi] >> (8 * bi)) & 0xffu)) - 4503599627370496.0;
                         dots[bi] = fma(qd, z, dots[bi]);
@@ -638,841 +563,1336 @@ __device__ __noinline__ void router_phase(const Cfg &P, Smem &S, int l) {
                 acc += (double)bf16_bits_to_float(scs[er * G + g]) * dot + (double)bf16_bits_to_float(bis[er * G + g]) * zs;
             }
             acc = warp_sum(acc);
-            if (lane == 0) S.rpart[u] = acc;
-        }
-        __syncthreads();
-        const double sqrt_h = sqrt((double)H);
-#pragma unroll 1
-        for (int item = threadIdx.x; item < items; item += blockDim.x) {
-            double a = 0.0;
-            for (int p = 0; p < parts; ++p) a += S.rpart[item * parts + p];
-            const int er = item / T, t = item - er * T;
-            P.logits[(size_t)t * E + e0 + er] = a / ((double)S.rms[t] * sqrt_h);
-        }
-    }
-    __syncthreads();
-}
-
-// P2: top-k by rank counting (a logit's rank = how many logits beat it: larger,
-// or equal with a lower expert index), softmax * per_expert_scale, the
-// bucketing of the T*k pairs by rank counting too, and this CTA's job tables.
-// Every CTA.
-__device__ __noinline__ void topk_phase(const Cfg &P, Smem &S, const moe_layer_w &W) {
-    const int T = P.T, E = P.E, k = P.k, n = T * k, H = P.H;
-    // the logits as order-preserving unsigned keys (larger logit <=> larger
-    // key, exactly): lk[t][e], and their high words kh, in F segments of SL
-    // experts per token; a segment takes SS = SL + 4 words (zero padding,
-    // below every key), so the F segments that a warp reads at once start in
-    // different banks
-    unsigned long long *lk = reinterpret_cast<unsigned long long *>(S.pool);  // ring is idle here
-    const int F = (E >= 32 && T * E * 4 <= (int)blockDim.x) ? 4 : 1;
-    const int SL = ((E + F - 1) / F + 3) & ~3, SS = SL + 4, RS = F * SS;
-    uint32_t *kh = reinterpret_cast<uint32_t *>(S.pool + (((size_t)T * E * 8 + 15) & ~(size_t)15));
-#pragma unroll 1
-    for (int i = threadIdx.x; i < T * RS; i += blockDim.x) {
-        const int t = i / RS, r = i - t * RS, q = r / SS, o = r - q * SS, e = q * SL + o;
-        uint32_t hi = 0u;
-        if (o < SL && e < E) {
-            unsigned long long b = (unsigned long long)__double_as_longlong(__ldcg(P.logits + (size_t)t * E + e));
-            if (b == 0x8000000000000000ull) b = 0ull;  // -0 and +0 are the same logit
-            b = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
-            lk[(size_t)t * E + e] = b;
-            hi = (uint32_t)(b >> 32);
-        }
-        kh[i] = hi;
-    }
-    __syncthreads();
-    // rank of (t, e) = keys larger than its key, plus equal keys of lower
-    // index.  F adjacent lanes share one (t, e), each counting over one
-    // segment of high words: how many are larger and how many equal (its own
-    // included).  With no other key sharing its high word, the count of
-    // larger high words is the rank; otherwise it is counted again on the
-    // full keys.
-    const int items = T * E * F;
-#pragma unroll 1
-    for (int it0 = 0; it0 < items; it0 += blockDim.x) {
-        const int it = it0 + threadIdx.x;
-        const int te = F == 4 ? it >> 2 : it, f = it - te * F;
-        int gt = 0, eq = 0, t = 0, e = 0;
-        unsigned long long v = 0ull;
-        if (it < items) {
-            t = te / E;
-            e = te - t * E;
-            v = lk[(size_t)t * E + e];
-            const uint32_t hv = (uint32_t)(v >> 32);
-            const uint4 *seg = reinterpret_cast<const uint4 *>(kh + (size_t)t * RS + f * SS);
-#pragma unroll 4
-            for (int j = 0; j < SL / 4; ++j) {
-                const uint4 h = seg[j];
-                gt += (h.x > hv) + (h.y > hv) + (h.z > hv) + (h.w > hv);
-                eq += (h.x == hv) + (h.y == hv) + (h.z == hv) + (h.w == hv);
+            if (lane == 0) {
+                if (parts == 1)
+                    put_logit(P, t, rc.e0 + er, acc / ((double)S.rms[t] * sqrt_h), tag);
+                else
+                    rpart[u] = acc;
             }
         }
-        if (F == 4) {
-            gt += __shfl_xor_sync(0xffffffffu, gt, 1);
-            gt += __shfl_xor_sync(0xffffffffu, gt, 2);
-            eq += __shfl_xor_sync(0xffffffffu, eq, 1);
-            eq += __shfl_xor_sync(0xffffffffu, eq, 2);
-        }
-        if (it < items && f == 0) {
-            int rank = gt;
-            if (eq > 1) {
-                rank = 0;
+        if (parts > 1) {
+            consumer_sync();  // every consumer, whatever its wait gave
 #pragma unroll 1
-                for (int j = 0; j < E; ++j) {
-                    const unsigned long long o = lk[(size_t)t * E + j];
-                    rank += (o > v) | ((o == v) & (j < e));
+            for (int item = got ? (int)threadIdx.x : items; item < items; item += kCThreads) {
+                double a = 0.0;
+                for (int p = 0; p < parts; ++p) a += rpart[item * parts + p];  // fixed order
+                const int er = item / T, t = item - er * T;
+                put_logit(P, t, rc.e0 + er, a / ((double)S.rms[t] * sqrt_h), tag);
+            }
+        }
+    }
+}
+
+// One row of a gate/up unit (slot layout: gate codes [CH][8 rows][16 B] with
+// the 128-byte swizzle at 0, up codes at gcb, gate (scale, bias) words
+// [GH][8 rows] at 2 gcb, up words after them) against the n <= NT tokens
+// toks[]: lanes are 32-column chunks.  g[tt], u[tt]: full sums in every lane.
+template <int NT>
+__device__ __forceinline__ void g_piece(const Cfg &P, const unsigned char *slot, int row, int n, const int (&tk)[NT],
+                                        const float *x, const float *xs, float (&g)[NT], float (&u)[NT]) {
+    const int lane = threadIdx.x & 31, CH = P.CH, gcb = P.gcb;
+    const unsigned char *sbb = slot + 2 * gcb;
+    const int sbs = P.sbs;
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) g[tt] = u[tt] = 0.f;
+#pragma unroll 1
+    for (int c = lane; c < CH; c += 32) {
+        const int sw = (row ^ (c & 7)) << 4;
+#pragma unroll
+        for (int mat = 0; mat < 2; ++mat) {
+            const uint4 q = *reinterpret_cast<const uint4 *>(slot + mat * gcb + c * 128 + sw);
+            const uint32_t sbw = *reinterpret_cast<const uint32_t *>(sbb + mat * sbs + (c >> 1) * 32 + row * 4);
+            const float s = bf16_bits_to_float(sbw & 0xffffu) * kCodeUnscale, b = bf16_bits_to_float(sbw >> 16);
+            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+            float2 a0[NT], a1[NT];
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) a0[tt] = a1[tt] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+                const Decoded8 d = decode_word(wv[wi]);
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt) {
+                    if (tt < n) {
+                        const float4 *xp =
+                            reinterpret_cast<const float4 *>(x + ((size_t)tk[tt] * CH + c) * kXStride + wi * 8);
+                        const float4 xa = xp[0], xb = xp[1];
+                        a0[tt] = ffma2(make_float2(d.f[0], d.f[1]), make_float2(xa.x, xa.y), a0[tt]);
+                        a1[tt] = ffma2(make_float2(d.f[2], d.f[3]), make_float2(xa.z, xa.w), a1[tt]);
+                        a0[tt] = ffma2(make_float2(d.f[4], d.f[5]), make_float2(xb.x, xb.y), a0[tt]);
+                        a1[tt] = ffma2(make_float2(d.f[6], d.f[7]), make_float2(xb.z, xb.w), a1[tt]);
+                    }
                 }
             }
-            if (rank < k) {
-                S.idx[t * k + rank] = e;
-                // back from the key to the logit
-                const unsigned long long b = (v >> 63) ? (v & 0x7fffffffffffffffull) : ~v;
-                S.selv[t * k + rank] = __longlong_as_double((long long)b);
-            }
-        }
-    }
-    __syncthreads();
-    // bucketing: pair p's position among all pairs ordered by (expert, pair
-    // id), and the slot of its expert among the distinct experts (ascending).
-    // Few pairs: one pass that also finds first occurrences by rescanning;
-    // many pairs: first occurrences in a pass of their own.
-    if (T == 1) {
-        // one token: its k experts are distinct, so every pair is its expert's
-        // only one and the slots are the experts in ascending order
-        if (threadIdx.x < n) {
-            const int p = threadIdx.x, e = S.idx[p];
-            int less = 0;
-#pragma unroll 1
-            for (int q = 0; q < n; ++q) less += S.idx[q] < e;
-            S.perm[less] = p;
-            S.tokrow[less] = 0;
-            S.act_e[less] = e;
-            S.act_off[less] = less;
-            S.act_n[less] = 1;
-            if (p == 0) S.nact = n;
-        }
-    } else if (n <= 16) {
-        int id[16];  // every pair's expert, in registers
 #pragma unroll
-        for (int q = 0; q < 16; ++q) id[q] = q < n ? S.idx[q] : 0x7fffffff;
-        if (threadIdx.x < n) {
-            const int p = threadIdx.x, t = p / k, e = S.idx[p];
-            int less = 0, eqb = 0, cnt = 0, slot = 0, nact = 0;
+            for (int tt = 0; tt < NT; ++tt) {
+                if (tt < n) {
+                    const float dsum = (a0[tt].x + a0[tt].y) + (a1[tt].x + a1[tt].y);
+                    float &acc = mat ? u[tt] : g[tt];
+                    acc = fmaf(s, dsum, fmaf(b, xs[tk[tt] * CH + c], acc));
+                }
+            }
+        }
+    }
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int f = id[q];
-                bool firstq = q < n;
-#pragma unroll
-                for (int r = 0; r < q; ++r) firstq &= id[r] != f;
-                less += f < e;
-                eqb += (f == e) & (q < p);
-                cnt += f == e;
-                slot += firstq & (f < e);
-                nact += firstq;
-            }
-            S.perm[less + eqb] = p;
-            S.tokrow[less + eqb] = t * H;
-            if (eqb == 0) {
-                S.act_e[slot] = e;
-                S.act_off[slot] = less;
-                S.act_n[slot] = cnt;
-            }
-            if (p == 0) S.nact = nact;
-        }
-    } else {
-        if (threadIdx.x < n) {
-            const int p = threadIdx.x, t = p / k, e = S.idx[p];
-            int less = 0, eqb = 0, cnt = 0;
-#pragma unroll 1
-            for (int q = 0; q < n; ++q) {
-                const int f = S.idx[q];
-                less += f < e;
-                eqb += (f == e) & (q < p);
-                cnt += f == e;
-            }
-            S.perm[less + eqb] = p;
-            S.tokrow[less + eqb] = t * H;
-            S.first[p] = eqb == 0;
-            S.poff[p] = less;
-            S.pcnt[p] = cnt;
-        }
-        __syncthreads();
-        if (threadIdx.x < n) {
-            const int p = threadIdx.x, e = S.idx[p];
-            int slot = 0, nact = 0;
-#pragma unroll 1
-            for (int q = 0; q < n; ++q) {
-                slot += S.first[q] & (S.idx[q] < e);
-                nact += S.first[q];
-            }
-            if (S.first[p]) {
-                S.act_e[slot] = e;
-                S.act_off[slot] = S.poff[p];
-                S.act_n[slot] = S.pcnt[p];
-            }
-            if (p == 0) S.nact = nact;
-        }
-    }
-    if (threadIdx.x < T) S.tokrow_sh[threadIdx.x] = threadIdx.x * H;
-    __syncthreads();
-    // this layer's gate/up jobs per slot: the shared expert's Is/32, each active slot's I/32
-    if ((int)threadIdx.x <= S.nact) S.act_expect[threadIdx.x] += threadIdx.x == 0 ? P.Is / 32 : P.I / 32;
-    // task tables of this CTA.  Gate/up jobs are dealt round-robin (every CTA
-    // mixes shared-expert jobs with routed ones); down tasks go in contiguous
-    // blocks, so that a CTA's tasks share few (slot, part) inputs.
-    const int na = S.nact, G = gridDim.x, c = blockIdx.x;
-    const int pg = (P.H / 64 + kTaskGroups - 1) / kTaskGroups;
-    const int NT2 = (P.Is / 32 + na * (P.I / 32)) * 2 * pg;  // gate/up tasks of the grid
-    const int n2 = NT2 > c ? (NT2 - 1 - c) / G + 1 : 0;
-    const int RBH = P.H / 32;
-    const int J3 = (P.ndp_s + na * P.ndp_r) * RBH;
-    const int d0 = (int)((long long)J3 * c / G), d1 = (int)((long long)J3 * (c + 1) / G);
-    const int sp0 = d0 / RBH;
-    // staged down inputs: the (slot, part) of the CTA's tasks, consecutive; one
-    // thread per input, each adding up the sizes of the ones before it
-    const int nseg = min(d1 > d0 ? (d1 - 1) / RBH - sp0 + 1 : 0, kMaxSegs);
-    const int ngt = min(n2, kMaxTasks), ndt = min(d1 - d0, kMaxTasks);
-    if (threadIdx.x < nseg) {
-        const int k2 = threadIdx.x;
-        int off = 0, slot = 0, part = 0;
-#pragma unroll 1
-        for (int q = 0; q <= k2; ++q) {
-            dn_slot_part(P, sp0 + q, slot, part);
-            const int Gs = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
-            const int ld = (Gs * (part + 1) / nd - Gs * part / nd) * 64;
-            const int nn = slot == 0 ? P.T : S.act_n[slot - 1];
-            if (q < k2) off += nn * ld;
-        }
-        const int Gs = slot == 0 ? P.Is / 64 : P.I / 64, nd = slot == 0 ? P.ndp_s : P.ndp_r;
-        SegDesc &sg = S.seg[k2];
-        sg.slot = (int16_t)slot;
-        sg.part = (int16_t)part;
-        sg.g0 = (int16_t)(Gs * part / nd);
-        sg.ld = (int16_t)((Gs * (part + 1) / nd - sg.g0) * 64);
-        sg.n = (int16_t)(slot == 0 ? P.T : S.act_n[slot - 1]);
-        sg.seg0 = slot == 0 ? 0 : S.act_off[slot - 1];
-        sg.off = off;
-        sg.pad = 0;
-        if (k2 == nseg - 1) {
-            // all inputs at once if they fit the stage (and its chunk sums), else one
-            // (slot, part) at a time, each from the start of the stage
-            S.seg_rounds = off + sg.n * sg.ld <= min(P.stage_floats, kMaxXs * 32) ? 1 : nseg;
-        }
-    }
-    if (threadIdx.x == 0) {
-        S.pg = pg;
-        S.ngt = ngt;
-        S.ndt = ndt;
-        S.nseg = nseg;
-        if (nseg == 0) S.seg_rounds = 1;
-    }
-    // gate/up tables on the first 256 threads, down tables on the rest
-    const int half = blockDim.x / 2;
-    if ((int)threadIdx.x < half) {
-#pragma unroll 1
-        for (int i = threadIdx.x; i < ngt; i += half) S.gut[i] = make_gu_task(P, S, c + i * G, pg);
-    } else {
-#pragma unroll 1
-        for (int i = threadIdx.x - half; i < ndt; i += (int)blockDim.x - half) S.dnt[i] = make_dn_task(P, S, d0 + i, sp0);
-    }
-    __syncthreads();
-    if (S.seg_rounds > 1 && (int)threadIdx.x < nseg) S.seg[threadIdx.x].off = 0;
-    // the ring was written with generic stores above; order them before the
-    // bulk copies (async proxy) that refill it next
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-}
-
-// Gate weights w = softmax(logits[top-k]) * per_expert_scale[top-k], in fp64;
-// selv[t*k] is token t's largest selected logit.  One warp, off the critical
-// path (they are first needed by the combine in the down phase).
-__device__ __noinline__ void gate_weights(const Cfg &P, Smem &S, const moe_layer_w &W) {
-    const int k = P.k, n = P.T * k;
-#pragma unroll 1
-    for (int p = threadIdx.x & 31; p < n; p += 32) {
-        const int t = p / k;
-        const double mx = S.selv[t * k];
-        double z = 0.0;
-#pragma unroll 1
-        for (int s2 = 0; s2 < k; ++s2) z += exp(S.selv[t * k + s2] - mx);
-        S.wts[p] = (float)(exp(S.selv[p] - mx) / z * (double)bf16_bits_to_float(W.per_expert_scale[S.idx[p]]));
+    for (int tt = 0; tt < NT; ++tt) {
+        g[tt] = warp_sum(g[tt]);
+        u[tt] = warp_sum(u[tt]);
     }
 }
 
-// x' = bf16(rmsnorm_no_scale(h)) pre-scaled for the code decode, and its chunk
-// sums, in S.stage.  A thread per 4 columns; the 8 threads of a 32-column
-// chunk are adjacent lanes and sum it with three shuffles.
-__device__ __noinline__ void stage_x(const Cfg &P, Smem &S) {
-    const int T = P.T, H4 = P.H / 4, lane = threadIdx.x & 31;
-    const int n4 = T * H4, rounds = (n4 + (int)blockDim.x - 1) / (int)blockDim.x;
+// One 8-row block of a down slot (codes [pc][8 rows][16 B], 128-byte swizzle;
+// words [pc/2][8 rows]) against the n <= NT staged inputs apre ([n][pc][kXStride],
+// pre-scaled) with chunk sums asum ([n][pc]): lanes are (row r = lane % 8,
+// chunk offset j = lane / 8), four chunks per step.  y[tt]: row r's sums in
+// lanes r (= lanes 0..7).
+template <int NT>
+__device__ __forceinline__ void d_block(const unsigned char *codes, const unsigned char *sbp, const float *apre,
+                                        const float *asum, int pc, int pcv, int n, float (&y)[NT]) {
+    const int lane = threadIdx.x & 31, r = lane & 7, j = lane >> 3;
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) y[tt] = 0.f;
 #pragma unroll 1
-    for (int r = 0; r < rounds; ++r) {  // every thread runs every round: the shuffles need whole warps
-        const int i = r * blockDim.x + threadIdx.x;
+    for (int c = j; c < pcv; c += 4) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(codes + c * 128 + ((r ^ (c & 7)) << 4));
+        const uint32_t sbw = *reinterpret_cast<const uint32_t *>(sbp + (c >> 1) * 32 + r * 4);
+        const float s = bf16_bits_to_float(sbw & 0xffffu) * kCodeUnscale, b = bf16_bits_to_float(sbw >> 16);
+        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+        float2 a0[NT], a1[NT];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) a0[tt] = a1[tt] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            const Decoded8 d = decode_word(wv[wi]);
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) {
+                if (tt < n) {
+                    const float4 *xp = reinterpret_cast<const float4 *>(apre + ((size_t)tt * pc + c) * kXStride + wi * 8);
+                    const float4 xa = xp[0], xb = xp[1];
+                    a0[tt] = ffma2(make_float2(d.f[0], d.f[1]), make_float2(xa.x, xa.y), a0[tt]);
+                    a1[tt] = ffma2(make_float2(d.f[2], d.f[3]), make_float2(xa.z, xa.w), a1[tt]);
+                    a0[tt] = ffma2(make_float2(d.f[4], d.f[5]), make_float2(xb.x, xb.y), a0[tt]);
+                    a1[tt] = ffma2(make_float2(d.f[6], d.f[7]), make_float2(xb.z, xb.w), a1[tt]);
+                }
+            }
+        }
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+            if (tt < n) {
+                const float dsum = (a0[tt].x + a0[tt].y) + (a1[tt].x + a1[tt].y);
+                y[tt] = fmaf(s, dsum, fmaf(b, asum[tt * pc + c], y[tt]));
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) {
+        y[tt] += __shfl_xor_sync(0xffffffffu, y[tt], 8);
+        y[tt] += __shfl_xor_sync(0xffffffffu, y[tt], 16);
+    }
+}
+
+// ------------------------------------------------------------------ tensor-core (mma.sync) variants
+//
+// For batches of 2 to 8 tokens the per-token FMA work of the CUDA-core decode
+// grows with T while the bytes do not; these variants use the warp-level
+// tensor-core MMA (m16n8k16, BF16 operands, FP32 accumulation), whose N = 8
+// columns hold up to 8 tokens at no extra cost.  Codes become exact BF16
+// values 128 + q with one mask-or per pair (0x4300 | q is 128 + q), so every
+// product is exact; per 64-column group the sum is rescaled:
+//     sum_k (s q_k + b) x_k = s * D + (b - 128 s) * sum_k x_k,   D = sum_k (128 + q_k) x_k.
+// K order inside a 32-column chunk: lane t of a quad takes word t of a row's
+// 16-byte record (columns 8t..8t+7); its two MMAs take the nibble pairs
+// (0,4), (1,5) and (2,6), (3,7).  The activations are staged in the same
+// order, so the dot products are unchanged.
+
+constexpr int kMaxPieces = 4;  // K-pieces of a gate/up unit on the MMA path
+
+// BF16 pairs (128 + q_j, 128 + q_{j+4}) of a word's nibble pairs j = 0..3.
+__device__ __forceinline__ void code_pairs(uint32_t w, uint32_t (&p)[4]) {
+    constexpr uint32_t kM = 0x000F000Fu, kB = 0x43004300u;
+    p[0] = (w & kM) | kB;
+    p[1] = ((w >> 4) & kM) | kB;
+    p[2] = ((w >> 8) & kM) | kB;
+    p[3] = ((w >> 12) & kM) | kB;
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bytes of one token's staged input on the MMA path: [CH][4 lanes][8 bf16] plus 16 bytes of padding,
+// so that the 8 tokens read by one load instruction fall in different banks
+__host__ __device__ __forceinline__ int xb_token_bytes(int CH) { return CH * 64 + 16; }
+
+// xe of every token as BF16 in the MMA order ([T][CH][t][8]: columns 8t + 0,4,1,5,2,6,3,7)
+// and its 64-column group sums xg ([T][GH], fp32).
+__device__ __noinline__ void stage_x_mma(const Cfg &P, Shared &S, const uint16_t *hs, unsigned char *xb, float *xg) {
+    const int T = P.T, H = P.H, CH = P.CH, GH = P.GH, lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        float ss = 0.f;
+#pragma unroll 1
+        for (int i = threadIdx.x; i < H / 2; i += kCThreads) {
+            const uint32_t v = reinterpret_cast<const uint32_t *>(hs + (size_t)t * H)[i];
+            const float a = bf16_bits_to_float(v & 0xffffu), b = bf16_bits_to_float(v >> 16);
+            ss = fmaf(a, a, fmaf(b, b, ss));
+        }
+        ss = consumer_sum(ss, S.red);
+        if (threadIdx.x == 0) {
+            S.rms[t] = sqrtf(ss / (float)H + P.eps);
+            S.rinv[t] = 1.0f / S.rms[t];
+        }
+    }
+    consumer_sync();
+    // one thread per 8 columns (a word t of a chunk): 4 threads of a quad make a chunk, 8 a group
+    const int n8 = T * H / 8, rounds = (n8 + kCThreads - 1) / kCThreads;
+#pragma unroll 1
+    for (int r = 0; r < rounds; ++r) {
+        const int i = r * kCThreads + threadIdx.x;
         float sx = 0.f;
-        if (i < n4) {
-            const int t = i / H4;
-            float4 v = reinterpret_cast<float4 *>(S.stage)[i];
+        if (i < n8) {
+            const int t = i / (H / 8), col = 8 * (i - t * (H / 8)), c = col >> 5, wq = (col >> 3) & 3;
+            const uint4 hv = *reinterpret_cast<const uint4 *>(hs + (size_t)t * H + col);
+            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
             const float ri = S.rinv[t];
-            const float x0 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.x * ri));
-            const float x1 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.y * ri));
-            const float x2 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.z * ri));
-            const float x3 = bf16_bits_to_float(f32_to_bf16_bits_alu(v.w * ri));
-            const int c = (4 * i) & 7;  // 0 or 4
-            v.x = x0 * code_prescale(c);
-            v.y = x1 * code_prescale(c + 1);
-            v.z = x2 * code_prescale(c + 2);
-            v.w = x3 * code_prescale(c + 3);
-            reinterpret_cast<float4 *>(S.stage)[i] = v;
-            sx = (x0 + x1) + (x2 + x3);
+            uint32_t xv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float h = bf16_bits_to_float((hw[j >> 1] >> (16 * (j & 1))) & 0xffffu);
+                xv[j] = f32_to_bf16_bits_alu(h * ri);
+                sx += bf16_bits_to_float(xv[j]);
+            }
+            // order 0,4,1,5,2,6,3,7 as four BF16 pairs
+            const uint4 o = make_uint4(xv[0] | (xv[4] << 16), xv[1] | (xv[5] << 16), xv[2] | (xv[6] << 16),
+                                       xv[3] | (xv[7] << 16));
+            *reinterpret_cast<uint4 *>(xb + (size_t)t * xb_token_bytes(CH) + (size_t)c * 64 + wq * 16) = o;
         }
         sx += __shfl_xor_sync(0xffffffffu, sx, 1);
         sx += __shfl_xor_sync(0xffffffffu, sx, 2);
         sx += __shfl_xor_sync(0xffffffffu, sx, 4);
-        if (i < n4 && (lane & 7) == 0) S.xs[i >> 3] = sx;
+        if (i < n8 && (lane & 7) == 0) xg[i >> 3] = sx;  // 8 threads = 64 columns: index t * GH + group
     }
-    __syncthreads();
+    (void)GH;
+    consumer_sync();
 }
 
-// ------------------------------------------------------------------ streaming loops
-// (each its own function, so that its register allocation is its own)
-
-// Ring position of task i of a phase that starts at ring sequence number rq.
-__device__ __forceinline__ void ring_pos(unsigned rq, int i, int ns, int &s, unsigned &ph) {
-    const unsigned q = rq + (unsigned)i;
-    s = (int)(q % (unsigned)ns);
-    ph = (q / (unsigned)ns) & 1u;
-}
-
-// Producer of an expert phase: one ring slot per task, in task order.  The
-// ring runs through the gate/up tasks [0, ngt) and on into the down tasks
-// [ngt, ngt + ndt) (sequence numbers from the gate/up phase's rq).  In the
-// gate/up phase it issues every gate/up task and then the down tasks whose
-// slot was last used by a gate/up task (those slots are freed within the
-// phase); the down phase issues the rest.  Once the ring is primed, an L2
-// prefetch of what comes next (gate/up: the down tasks that do not fit the
-// ring; down: this CTA's share of the next layer's shared expert).
-__device__ __noinline__ bool task_producer(const Cfg &P, Smem &S, const moe_layer_w &W, bool down, unsigned rq,
-                                           const moe_layer_w *next, unsigned &issued) {
-    const int ns = P.nslots, ngt = S.ngt, ndt = S.ndt;
-    // ring positions [i0, i1) relative to the gate/up phase's first task
-    const int pre = min(ndt, ns);  // down tasks issued during the gate/up phase
-    const int i0 = down ? ngt + pre : 0, i1 = down ? ngt + ndt : ngt + pre;
-    const unsigned rq0 = down ? rq - (unsigned)ngt : rq;
-    bool ok = true;
+// Chunks [c0, c1) (whole groups) of a gate/up unit against the n <= 8 tokens
+// toks[] on the tensor cores: A rows 0..7 the unit's gate rows, 8..15 its up
+// rows; B column j token toks[j].  acc (per lane g = lane / 4, t = lane % 4):
+// gate row g and up row g, for the tokens of columns 2t and 2t + 1.
+__device__ __forceinline__ void g_piece_mma(const Cfg &P, const unsigned char *slot, int c0, int c1, int n,
+                                            const int *toks, const unsigned char *xb, const float *xg,
+                                            float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3, gcb = P.gcb, GH = P.GH;
+    const int my_tok = g < n ? toks[g] : -1;
+    const int tok0 = 2 * t < n ? toks[2 * t] : -1, tok1 = 2 * t + 1 < n ? toks[2 * t + 1] : -1;
+    const unsigned char *xrow = xb + (size_t)(my_tok < 0 ? 0 : my_tok) * xb_token_bytes(P.CH);
+    const unsigned char *sbg = slot + 2 * gcb, *sbu = slot + 2 * gcb + P.sbs;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q] = 0.f;
 #pragma unroll 1
-    for (int i = i0; i < i1; ++i) {
-        int s;
-        unsigned ph;
-        ring_pos(rq0, i, ns, s, ph);
-        if (rq0 + (unsigned)i >= (unsigned)ns && !mbar_wait(&S.empty[s], ph ^ 1u, P.err, kErrEmpty)) {
-            ok = false;
-            break;
+    for (int c = c0; c < c1; c += 2) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int ch = c + cc;
+            const int off = ch * 128 + ((g ^ (ch & 7)) << 4) + 4 * t;
+            const uint32_t wg = *reinterpret_cast<const uint32_t *>(slot + off);
+            const uint32_t wu = *reinterpret_cast<const uint32_t *>(slot + gcb + off);
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (my_tok >= 0) xv = *reinterpret_cast<const uint4 *>(xrow + ch * 64 + t * 16);
+            uint32_t pg[4], pu[4];
+            code_pairs(wg, pg);
+            code_pairs(wu, pu);
+            mma_bf16(d, pg[0], pu[0], pg[1], pu[1], xv.x, xv.y);
+            mma_bf16(d, pg[2], pu[2], pg[3], pu[3], xv.z, xv.w);
         }
-        const bool dn = i >= ngt;
-        const TaskDesc t = dn ? S.dnt[i - ngt] : S.gut[i];
-        const uint32_t *q, *sb;
-        task_ptrs(P, W, t, dn, q, sb);
-        // the slot now belongs to this task (its previous task has been consumed)
-        *reinterpret_cast<volatile unsigned *>(&S.slot_task[s]) = rq0 + (unsigned)i;
-        issue_task(S, s, q, sb, t.g0, t.g1);
-        issued = rq0 + (unsigned)i + 1u;
-        if (!down && i == min(ns, ngt) - 1) {
-            // the down tasks beyond the ring: into L2 for now
+        const int grp = c >> 1;
+        const uint32_t wsg = *reinterpret_cast<const uint32_t *>(sbg + grp * 32 + g * 4);
+        const uint32_t wsu = *reinterpret_cast<const uint32_t *>(sbu + grp * 32 + g * 4);
+        const float sg = bf16_bits_to_float(wsg & 0xffffu), bg = fmaf(-128.f, sg, bf16_bits_to_float(wsg >> 16));
+        const float su = bf16_bits_to_float(wsu & 0xffffu), bu = fmaf(-128.f, su, bf16_bits_to_float(wsu >> 16));
+        const float x0 = tok0 >= 0 ? xg[tok0 * GH + grp] : 0.f, x1 = tok1 >= 0 ? xg[tok1 * GH + grp] : 0.f;
+        acc[0] = fmaf(sg, d[0], fmaf(bg, x0, acc[0]));
+        acc[1] = fmaf(sg, d[1], fmaf(bg, x1, acc[1]));
+        acc[2] = fmaf(su, d[2], fmaf(bu, x0, acc[2]));
+        acc[3] = fmaf(su, d[3], fmaf(bu, x1, acc[3]));
+    }
+}
+
+// bytes of one token's staged down input on the MMA path: [pc][4 lanes][16 bf16] (+16 padding)
+__host__ __device__ __forceinline__ int ahl_token_bytes(int pc) { return pc * 128 + 16; }
+
+// One 8-row block of a down slot on the tensor cores: A rows 0..7 the high
+// BF16 parts of the tokens' inputs (a = hi + lo), rows 8..15 the low parts;
+// B the block's 8 rows.  y[0], y[1] (lane g, t): token g, rows 2t and 2t + 1.
+__device__ __forceinline__ void d_block_mma(const unsigned char *codes, const unsigned char *sbp,
+                                            const unsigned char *ahl, const float *asg, int pc, int pcv, int n,
+                                            float (&y)[2]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const bool mine = g < n;
+    const unsigned char *arow = ahl + (size_t)(mine ? g : 0) * ahl_token_bytes(pc);
+    y[0] = y[1] = 0.f;
 #pragma unroll 1
-            for (int d = pre; d < ndt; ++d) {
-                const TaskDesc u = S.dnt[d];
-                const uint32_t *uq, *usb;
-                task_ptrs(P, W, u, true, uq, usb);
-                const int ng = u.g1 - u.g0;
-                prefetch_l2(uq + (size_t)u.g0 * 256, (unsigned)ng * kCodeBytesPerGroup);
-                prefetch_l2(usb + (size_t)u.g0 * 32, (unsigned)ng * kSbBytesPerGroup);
+    for (int c = 0; c < pcv; c += 2) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int ch = c + cc;
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(codes + ch * 128 + ((g ^ (ch & 7)) << 4) + 4 * t);
+            uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
+            if (mine) {
+                a0 = *reinterpret_cast<const uint4 *>(arow + ch * 128 + t * 32);
+                a1 = *reinterpret_cast<const uint4 *>(arow + ch * 128 + t * 32 + 16);
+            }
+            uint32_t pw[4];
+            code_pairs(w, pw);
+            mma_bf16(d, a0.x, a0.y, a0.z, a0.w, pw[0], pw[1]);
+            mma_bf16(d, a1.x, a1.y, a1.z, a1.w, pw[2], pw[3]);
+        }
+        const int grp = c >> 1;
+        const uint2 sw = *reinterpret_cast<const uint2 *>(sbp + grp * 32 + 2 * t * 4);  // rows 2t, 2t + 1
+        const float s0 = bf16_bits_to_float(sw.x & 0xffffu), b0 = fmaf(-128.f, s0, bf16_bits_to_float(sw.x >> 16));
+        const float s1 = bf16_bits_to_float(sw.y & 0xffffu), b1 = fmaf(-128.f, s1, bf16_bits_to_float(sw.y >> 16));
+        const float as = mine ? asg[g * (pc / 2) + grp] : 0.f;
+        y[0] = fmaf(s0, d[0] + d[2], fmaf(b0, as, y[0]));
+        y[1] = fmaf(s1, d[1] + d[3], fmaf(b1, as, y[1]));
+    }
+}
+
+// The logit as an order-preserving 64-bit key (larger logit <=> larger key).
+__device__ __forceinline__ unsigned long long logit_key(double v) {
+    unsigned long long b = (unsigned long long)__double_as_longlong(v);
+    if (b == 0x8000000000000000ull) b = 0ull;  // -0 and +0 are the same logit
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ double key_logit(unsigned long long k) {
+    const unsigned long long b = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
+    return __longlong_as_double((long long)b);
+}
+
+struct Cand {
+    unsigned long long key;
+    int e, pad;
+};
+
+// K: top-k of every token (ties to the lower expert index; ordered by logit
+// desc, index asc), gate weights softmax(logits[top-k]) * per_expert_scale
+// in fp64, and the bucketing of the T*k pairs by expert (stable by pair id).
+// Every CTA computes the same result from the same logits.
+//   1. candidates: a warp ranks 32 experts of one token among themselves; only
+//      those ranked below k can be in the top k of all E, so the others are
+//      dropped;
+//   2. each candidate's rank among its token's candidates is its rank among
+//      all E logits (everything that beats a top-k logit is a candidate);
+//   3. weights and buckets by counting over the T*k pairs.
+__device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, const uint16_t *pes, unsigned tag) {
+    const int T = P.T, E = P.E, k = P.k, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nsl = (E + 31) / 32;
+    if (threadIdx.x < T) S.ccount[threadIdx.x] = 0;
+    consumer_sync();
+#pragma unroll 1
+    for (int item = wid; item < T * nsl; item += kCW) {
+        const int t = item / nsl, sl = item - t * nsl, e = sl * 32 + lane;
+        const bool valid = e < E;
+        double v = 0.0;
+        if (valid && !get_logit(P, t, e, tag, v)) v = 0.0;  // an error is recorded; the layer's result is void
+        const unsigned long long key = valid ? logit_key(v) : 0ull;
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
+            rank += (kj > key) | ((kj == key) & (j < lane));
+        }
+        if (valid && rank < k) {
+            const int pos = atomicAdd(&S.ccount[t], 1);
+            if (pos < P.maxc) cand[t * P.maxc + pos] = Cand{key, e, 0};
+        }
+    }
+    consumer_sync();
+#pragma unroll 1
+    for (int i = threadIdx.x; i < T * P.maxc; i += kCThreads) {
+        const int t = i / P.maxc, ci = i - t * P.maxc, nc = min(S.ccount[t], P.maxc);
+        if (ci < nc) {
+            const Cand me = cand[i];
+            int rank = 0;
+#pragma unroll 1
+            for (int j = 0; j < nc; ++j) {
+                const Cand o = cand[t * P.maxc + j];
+                rank += (o.key > me.key) | ((o.key == me.key) & (o.e < me.e));
+            }
+            if (rank < k) {
+                S.idx[t * k + rank] = me.e;
+                S.selv[t * k + rank] = key_logit(me.key);
             }
         }
     }
-    if (ok && down && next != nullptr) {
-        // this CTA's share of the next layer's shared-expert weights
-        const moe_layer_w &N = *next;
-        const size_t shq = (size_t)P.Is * P.H / 2, shsb = (size_t)P.Is * (P.H / 64) * 4;
-        const void *ptrs[6] = {N.sh_gate.q, N.sh_up.q, N.sh_down.q, N.sh_gate.sb, N.sh_up.sb, N.sh_down.sb};
-        const size_t sizes[6] = {shq, shq, shq, shsb, shsb, shsb};
+    consumer_sync();
+    const int n = T * k;
 #pragma unroll 1
-        for (int a = 0; a < 6; ++a) {
-            const size_t per = ((sizes[a] / gridDim.x) + 15) & ~(size_t)15;
-            const size_t off = per * blockIdx.x;
-            if (off < sizes[a])
-                prefetch_range(static_cast<const char *>(ptrs[a]) + off,
-                               (off + per <= sizes[a] ? per : sizes[a] - off) & ~(size_t)15);
+    for (int p = threadIdx.x; p < n; p += kCThreads) {
+        const int t = p / k, e = S.idx[p];
+        const double mx = S.selv[t * k];
+        double z = 0.0;
+#pragma unroll 1
+        for (int s2 = 0; s2 < k; ++s2) z += exp(S.selv[t * k + s2] - mx);
+        S.wts[p] = (float)(exp(S.selv[p] - mx) / z * (double)bf16_bits_to_float(pes[e]));
+        int less = 0, eqb = 0, cnt = 0;
+#pragma unroll 1
+        for (int q = 0; q < n; ++q) {
+            const int f = S.idx[q];
+            less += f < e;
+            eqb += (f == e) & (q < p);
+            cnt += f == e;
+        }
+        S.pos_pair[less + eqb] = p;
+        S.pos_tok[less + eqb] = t;
+        S.first[p] = eqb == 0;
+        S.slot_off[p] = less;  // scratch: moved to the slot's entry below
+        S.slot_n[p] = cnt;
+    }
+    consumer_sync();
+    int my_slot = -1, my_e = 0, my_off = 0, my_n = 0;
+    if (threadIdx.x < n && S.first[threadIdx.x]) {
+        const int p = threadIdx.x, e = S.idx[p];
+        int slot = 0;
+#pragma unroll 1
+        for (int q = 0; q < n; ++q) slot += S.first[q] & (S.idx[q] < e);
+        my_slot = slot;
+        my_e = e;
+        my_off = S.slot_off[p];
+        my_n = S.slot_n[p];
+    }
+    consumer_sync();
+    if (my_slot >= 0) {
+        S.slot_e[my_slot] = my_e;
+        S.slot_off[my_slot] = my_off;
+        S.slot_n[my_slot] = my_n;
+    }
+    if (threadIdx.x == 0) {
+        int d = 0;
+        for (int q = 0; q < n; ++q) d += S.first[q];
+        S.D = d;
+    }
+    consumer_sync();
+}
+
+// ------------------------------------------------------------------ work bookkeeping
+
+// A piece of a gate/up unit is done (its a row is stored): the last of the
+// unit's 8 pieces counts the unit done in global memory (release) and frees
+// the ring slot.  Stores of the other pieces are ordered before the count by
+// their fences and the shared-memory count (fence - atomic - atomic - fence).
+__device__ __forceinline__ void piece_done(Shared &S, const Cfg &P, unsigned tseq, unsigned *ready) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence();
+        const int s = (int)(tseq % (unsigned)P.ns);
+        if (atomicAdd(&S.cnt[s], 1) == 7) {
+            S.cnt[s] = 0;
+            __threadfence();
+            red_release_add(ready, 1u);
+            mbar_arrive(&S.empty[s]);
         }
     }
-    return ok;
 }
 
-// A team member's share of a task: lanes are the task's 32 rows; acc[tt]
-// receives the dot product of the row's groups gi0, gi0 + kWPT, ... (< ng,
-// relative to the task's first group) with token tt's input.
-template <int NT>
-__device__ __forceinline__ void task_dot(const unsigned char *slot, int ng, int gi0, const float *x, const float *xsum,
-                                         const int *tokrow, int stride, int n, float (&acc)[NT], int lane) {
-#pragma unroll 1
-    for (int gi = gi0; gi < ng; gi += kWPT)
-        group_dot_n<NT>(slot + gi * kCodeBytesPerGroup,
-                        reinterpret_cast<const uint32_t *>(slot + ng * kCodeBytesPerGroup + gi * kSbBytesPerGroup)[lane],
-                        x + gi * 64, xsum + 2 * gi, tokrow, stride, n, acc, lane);
-}
-
-// A consumer warp's wait for task q in ring slot s: first until the producer
-// has handed the slot to q (the slot's previous task is done, so its full
-// barrier is in q's phase), then for the phase itself.  Warps take tasks out
-// of ring order, so without the first wait a warp could test a phase two
-// ahead of the barrier's, which the parity test cannot tell apart.
-__device__ __noinline__ bool wait_task(Smem &S, unsigned q, int s, unsigned ph, int *err) {
-    bool ok = true;
+// A block task of a down group is done: the last of the group's nblk tasks
+// frees the ring slot (and its staged input).
+__device__ __forceinline__ void block_done(Shared &S, const Cfg &P, unsigned tseq, int nblk) {
+    __syncwarp();
     if ((threadIdx.x & 31) == 0) {
-        const volatile unsigned *own = &S.slot_task[s];
-        if (*own != q) {
-            const unsigned long long t0 = globaltimer();
-            while (*own != q) {
-                if (globaltimer() - t0 > kWaitNs || ldcg_int(err) != 0) {
-                    atomicCAS(err, 0, kErrFull);
-                    ok = false;
-                    break;
+        const int s = (int)(tseq % (unsigned)P.ns);
+        if (atomicAdd(&S.cnt[s], 1) == nblk - 1) {
+            S.cnt[s] = 0;
+            S.astate[s] = 0;
+            mbar_arrive(&S.empty[s]);
+        }
+    }
+}
+
+// The SwiGLU input of a down group, staged once per group in its ring slot:
+// the first warp to arrive waits until every gate/up unit of the slot (the
+// shared expert, or routed slot j) is counted done across the grid, then
+// copies the n token rows of K-part p, pre-scaled for the code decode
+// ([n][pc][kXStride]), with their 32-column sums ([n][pc]); the other warps
+// of the group wait for it.
+__device__ __noinline__ bool stage_a(Shared &S, const Cfg &P, int s, bool shd, int j, int p, int pc, int pcv, int n,
+                                     int off, float *apre, float *asum) {
+    const int lane = threadIdx.x & 31;
+    int mine = 0, ok = 1;
+    if (lane == 0) mine = atomicCAS(const_cast<int *>(&S.astate[s]), 0, 1) == 0;
+    mine = __shfl_sync(0xffffffffu, mine, 0);
+    if (mine) {
+        const int ri = shd ? 0 : 1 + j;
+        if (lane == 0) ok = wait_count(P, P.ready + ri, S.exp_ready[ri]);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        __syncwarp();  // the other lanes' loads below come after lane 0's acquire
+        if (!ok) return false;
+        const int K = shd ? P.Is : P.I;
+#pragma unroll 1
+        for (int tt = 0; tt < n; ++tt) {
+            const float *src = shd ? P.a_sh + (size_t)tt * P.Is : P.a_r + (size_t)(off + tt) * P.I;
+            for (int c = lane; c < pcv; c += 32) {
+                const int col = (p * pc + c) * 32;
+                const float4 *s4 = reinterpret_cast<const float4 *>(src + col);
+                float *dst = apre + ((size_t)tt * pc + c) * kXStride;
+                float sum = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float4 v = col + 4 * q < K ? __ldcg(s4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    sum += (v.x + v.y) + (v.z + v.w);
+                    const int c8 = (4 * q) & 7;  // 0 or 4
+                    v.x *= code_prescale(c8);
+                    v.y *= code_prescale(c8 + 1);
+                    v.z *= code_prescale(c8 + 2);
+                    v.w *= code_prescale(c8 + 3);
+                    reinterpret_cast<float4 *>(dst)[q] = v;
+                }
+                asum[tt * pc + c] = sum;
+            }
+        }
+        __syncwarp();
+        __threadfence_block();
+        if (lane == 0) S.astate[s] = 2;
+        return true;
+    }
+    if (lane == 0) {
+        const unsigned long long t0 = globaltimer();
+        for (unsigned it = 0; S.astate[s] != 2; ++it) {
+            if ((it & 63u) == 63u && (ldcg_int(P.err) != 0 || globaltimer() - t0 > kWaitNs)) {
+                atomicCAS(P.err, 0, kErrStage);
+                ok = 0;
+                break;
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __threadfence_block();
+    return ok != 0;
+}
+
+// This CTA's 8-row output blocks [b0, b1) and its shared-expert units.
+struct CtaWork {
+    int b0, nblk, nshg;
+};
+
+__device__ __forceinline__ CtaWork cta_work(const Cfg &P) {
+    CtaWork w;
+    const int G = gridDim.x, c = blockIdx.x;
+    w.b0 = (int)((long long)P.nrb8 * c / G);
+    w.nblk = (int)((long long)P.nrb8 * (c + 1) / G) - w.b0;
+    w.nshg = c < P.units_s ? (P.units_s - 1 - c) / G + 1 : 0;
+    return w;
+}
+
+// Down group gi of a layer: the shared expert's K-part p (gi < parts_s), or
+// routed slot j's K-part p.
+struct DGroup {
+    bool shd;
+    int j, p, pc, dcb, sbd, pcv;
+};
+
+__device__ __forceinline__ DGroup dgroup(const Cfg &P, int gi) {
+    DGroup d;
+    d.shd = gi < P.parts_s;
+    if (d.shd) {
+        d.j = -1;
+        d.p = gi;
+    } else {
+        d.j = (gi - P.parts_s) / P.parts_r;
+        d.p = gi - P.parts_s - d.j * P.parts_r;
+    }
+    d.pc = d.shd ? P.pc_s : P.pc_r;
+    d.dcb = d.shd ? P.dcb_s : P.dcb_r;
+    d.sbd = d.shd ? P.sbd_s : P.sbd_r;
+    const int CK = (d.shd ? P.Is : P.I) / 32;
+    d.pcv = min(d.pc, CK - d.p * d.pc);
+    return d;
+}
+
+// The MMA path's staging of a down group's input: for each of its n tokens,
+// a = hi + lo (two BF16 values, round to nearest each) in the MMA order
+// ([n][pc][t][16 bf16] + padding per token) and the 64-column sums of hi + lo
+// ([n][pc/2], fp32).  One lane per 32-column chunk; the first warp of the
+// group stages, the others wait (as stage_a).
+__device__ __noinline__ bool stage_a_mma(Shared &S, const Cfg &P, int s, bool shd, int j, int p, int pc, int pcv,
+                                         int n, int off, unsigned char *ahl, float *asg) {
+    const int lane = threadIdx.x & 31;
+    int mine = 0, ok = 1;
+    if (lane == 0) mine = atomicCAS(const_cast<int *>(&S.astate[s]), 0, 1) == 0;
+    mine = __shfl_sync(0xffffffffu, mine, 0);
+    if (mine) {
+        const int ri = shd ? 0 : 1 + j;
+        if (lane == 0) ok = wait_count(P, P.ready + ri, S.exp_ready[ri]);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        __syncwarp();  // the other lanes' loads below come after lane 0's acquire
+        if (!ok) return false;
+#pragma unroll 1
+        for (int tt = 0; tt < n; ++tt) {
+            const float *src = shd ? P.a_sh + (size_t)tt * P.Is : P.a_r + (size_t)(off + tt) * P.I;
+            const int c = lane;
+            float sum = 0.f;
+            if (c < pcv) {
+                const float4 *s4 = reinterpret_cast<const float4 *>(src + (p * pc + c) * 32);
+                unsigned char *dst = ahl + (size_t)tt * ahl_token_bytes(pc) + c * 128;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {  // columns 8w .. 8w + 7 of the chunk
+                    const float4 va = __ldcg(s4 + 2 * w), vb = __ldcg(s4 + 2 * w + 1);
+                    const float v[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+                    uint32_t hi[8], lo[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        hi[q] = f32_to_bf16_bits_alu(v[q]);
+                        lo[q] = f32_to_bf16_bits_alu(v[q] - bf16_bits_to_float(hi[q]));
+                        sum += bf16_bits_to_float(hi[q]) + bf16_bits_to_float(lo[q]);
+                    }
+                    const uint4 o0 = make_uint4(hi[0] | (hi[4] << 16), lo[0] | (lo[4] << 16), hi[1] | (hi[5] << 16),
+                                                lo[1] | (lo[5] << 16));
+                    const uint4 o1 = make_uint4(hi[2] | (hi[6] << 16), lo[2] | (lo[6] << 16), hi[3] | (hi[7] << 16),
+                                                lo[3] | (lo[7] << 16));
+                    reinterpret_cast<uint4 *>(dst + w * 32)[0] = o0;
+                    reinterpret_cast<uint4 *>(dst + w * 32)[1] = o1;
                 }
             }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);  // the two chunks of a group
+            if (c < pcv && (c & 1) == 0) asg[tt * (pc / 2) + (c >> 1)] = sum;
         }
+        __syncwarp();
+        __threadfence_block();
+        if (lane == 0) S.astate[s] = 2;
+        return true;
     }
-    __syncwarp();
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    return ok && mbar_wait(&S.full[s], ph, err, kErrFull);
-}
-
-__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned *p, unsigned v) {
-    unsigned old;
-    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-
-// Bounded wait of one thread until a global count reaches `target` (acquire);
-// false (with an error recorded) on a timeout or another CTA's error.
-__device__ __noinline__ bool wait_count(const Cfg &P, const unsigned *ctr, unsigned target) {
-    const unsigned long long t0 = globaltimer();
-    for (unsigned it = 0;; ++it) {
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-        if (v >= target) return true;
-        if ((it & 63u) == 63u) {
-            if (ldcg_int(P.err) != 0) return false;
-            if (globaltimer() - t0 > kWaitNs) {
-                atomicCAS(P.err, 0, kErrReady);
-                return false;
+    if (lane == 0) {
+        const unsigned long long t0 = globaltimer();
+        for (unsigned it = 0; S.astate[s] != 2; ++it) {
+            if ((it & 63u) == 63u && (ldcg_int(P.err) != 0 || globaltimer() - t0 > kWaitNs)) {
+                atomicCAS(P.err, 0, kErrStage);
+                ok = 0;
+                break;
             }
         }
-        __nanosleep(32);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __threadfence_block();
+    return ok != 0;
+}
+
+// MMA path: a K-piece of a gate/up unit is done (its partial sums are in
+// `part`); true (warp-uniform) for the warp that completes the unit, which
+// then owns the slot's partials.
+__device__ __forceinline__ bool piece_last(Shared &S, const Cfg &P, unsigned tseq, int npc) {
+    __syncwarp();
+    int last = 0;
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence_block();
+        const int s = (int)(tseq % (unsigned)P.ns);
+        last = atomicAdd(&S.cnt[s], 1) == npc - 1;
+        if (last) S.cnt[s] = 0;
+        __threadfence_block();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    __syncwarp();
+    return last != 0;
+}
+
+// The completing warp of a unit counts it done in global memory (release) and frees its ring slot.
+__device__ __forceinline__ void unit_release(Shared &S, const Cfg &P, unsigned tseq, unsigned *ready) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence();
+        red_release_add(ready, 1u);
+        mbar_arrive(&S.empty[tseq % (unsigned)P.ns]);
     }
 }
 
-template <int NT>
-__device__ __noinline__ bool gu_consumer(const Cfg &P, Smem &S, unsigned rq) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, team = wid / kWPT, mb = wid - team * kWPT;
-    const int T = P.T, ns = P.nslots, nt = S.ngt, pg = S.pg, pw = pg * kWPT, tpj = 2 * pw;
+// MMA path: one K-piece of a gate/up unit (8 rows) for the tokens toks[0..n);
+// the warp completing the unit sums the pieces' partials in order and stores
+// a = silu(g) * u for its 8 rows (row0 .. row0 + 7 of `a`, token tt of the
+// list at a + aidx[tt] * lda).
+__device__ __forceinline__ void unit_piece_mma(Shared &S, const Cfg &P, unsigned char *ring, float *part, unsigned tseq,
+                                               int pi, int npc, int n, const int *toks, const int *aidx, float *a,
+                                               int lda, int row0, const unsigned char *xb, const float *xg,
+                                               unsigned *ready) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int s = (int)(tseq % (unsigned)P.ns);
+    const int gpp = (P.GH + npc - 1) / npc;
+    const int c0 = min(P.CH, 2 * pi * gpp), c1 = min(P.CH, c0 + 2 * gpp);
+    float acc[4];
+    g_piece_mma(P, ring + (size_t)s * P.slot_bytes, c0, c1, n, toks, xb, xg, acc);
+    float *mine = part + ((size_t)s * kMaxPieces + pi) * 128 + lane * 4;
+    *reinterpret_cast<float4 *>(mine) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    if (!piece_last(S, P, tseq, npc)) return;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < npc; ++q) {  // fixed order
+        const float4 v = *reinterpret_cast<const float4 *>(part + ((size_t)s * kMaxPieces + q) * 128 + lane * 4);
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
+    }
+    if (2 * t < n) a[(size_t)aidx[2 * t] * lda + row0 + g] = silu_mul(sum.x, sum.z);
+    if (2 * t + 1 < n) a[(size_t)aidx[2 * t + 1] * lda + row0 + g] = silu_mul(sum.y, sum.w);
+    unit_release(S, P, tseq, ready);
+}
+
+// ------------------------------------------------------------------ consumers
+
+template <int NT, bool kMma>
+__device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned char *base) {
+    // kMma: the tensor-core (mma.sync) variants; otherwise CUDA-core FMAs for at most NT tokens
+    const Cfg &P = S.c;
+    const int T = P.T, H = P.H, G = gridDim.x, c = blockIdx.x, ns = P.ns;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    unsigned char *ring = base + P.off_ring;
+    float *x = reinterpret_cast<float *>(base + P.off_x);   // FFMA path: pre-scaled fp32 xe
+    unsigned char *xb = base + P.off_x;                    // MMA path: BF16 xe in the MMA order
+    float *xs = reinterpret_cast<float *>(base + P.off_xs); // chunk sums (FFMA) or group sums (MMA)
+    uint16_t *hs = reinterpret_cast<uint16_t *>(base + P.off_h);
+    float *ybuf = reinterpret_cast<float *>(base + P.off_y);
+    Cand *cand = reinterpret_cast<Cand *>(base + P.off_cand);
+    float *part = reinterpret_cast<float *>(base + P.off_part);
+    const CtaWork cw = cta_work(P);
+    unsigned seq = 0, nbar = 0;
     bool ok = true;
 #pragma unroll 1
-    for (int i = team; i < nt; i += kTeams) {
-        const TaskDesc t = S.gut[i];
-        int s;
-        unsigned ph;
-        ring_pos(rq, i, ns, s, ph);
-        const int n = t.n, ng = t.g1 - t.g0;
-        float acc[NT];
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
-        const bool got = wait_task(S, rq + (unsigned)i, s, ph, P.err);
-        if (got) {
-            const int *tokrow = t.slot == 0 ? S.tokrow_sh : S.tokrow + t.seg0;
-            const int col = t.g0 * 64;
-            task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, mb, S.stage + col, S.xs + col / 32, tokrow, 0, n, acc,
-                         lane);
+    for (int l = 0; l < P.L && ok; ++l) {
+        // ---------------------------------------------------------- F: the layer's input
+        if (l == 0) {
+            load_h(P, hs, P.h_in);
+        } else {
+            if (!(ok = grid_wait(P, S, ++nbar))) break;  // every CTA has written m of layer l-1
+            finish_layer(P, S, hs, l - 1);
+            if (!P.chained) load_h(P, hs, P.h_in + (size_t)l * T * H);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[s]);
-        if (!got) {
-            ok = false;
-            continue;
+        if (kMma)
+            stage_x_mma(P, S, hs, xb, xs);
+        else
+            stage_x(P, S, hs, x, xs);
+        // ---------------------------------------------------------- R: router rows of this CTA
+        {
+            const bool got = wait_task(S, P, seq);
+            router_compute(P, S, ring + (size_t)(seq % (unsigned)ns) * P.slot_bytes, hs, S.rpart, got,
+                           (unsigned)l + 1u);
+            consumer_sync();
+            if (threadIdx.x == 0) mbar_arrive(&S.empty[seq % (unsigned)ns]);
+            ++seq;
         }
-        // this member's partial sums, then its count for the job (release: the
-        // warp's stores, ordered by __syncwarp, become visible first)
-        float *gp = P.gpart + ((((size_t)t.job * 2 + t.mat) * pg + t.part) * kWPT + mb) * T * 32;
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt)
-            if (tt < n) gp[tt * 32 + lane] = acc[tt];
-        __syncwarp();
-        unsigned old = 0u;
-        if (lane == 0) old = atom_add_release_gpu(&P.cnt_gu[t.job], 1u);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old == (unsigned)(tpj - 1)) {
-            // the job's last task: sum the parts in a fixed order, form a = silu(g) * u
-            if (lane == 0) __threadfence();
-            __syncwarp();
-            const float *jp = P.gpart + (size_t)t.job * 2 * pw * T * 32;
+        // ---------------------------------------------------------- S: shared gate/up pieces
+        {
+            const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(cw.nshg, 1) - 1) / max(cw.nshg, 1))) : 8;
 #pragma unroll 1
-            for (int tt = 0; tt < n; ++tt) {
-                float gs = 0.f, us = 0.f;
+            for (int i = wid; i < cw.nshg * npc; i += kCW) {
+                const int ui = i / npc, pi = i - ui * npc;
+                const unsigned tseq = seq + (unsigned)ui;
+                if (!wait_task(S, P, tseq)) break;
+                const int row0 = (c + ui * G) * 8;  // first row of the unit in the shared gate/up matrices
+                if (kMma) {
+                    unit_piece_mma(S, P, ring, part, tseq, pi, npc, T, S.toks_sh, S.toks_sh, P.a_sh, P.Is, row0, xb,
+                                   xs, P.ready);
+                } else {
+                    int tk[NT];
 #pragma unroll
-                for (int p2 = 0; p2 < kMaxPG * kWPT; ++p2) {
-                    if (p2 < pw) {
-                        gs += __ldcg(&jp[((size_t)p2 * T + tt) * 32 + lane]);
-                        us += __ldcg(&jp[((size_t)(pw + p2) * T + tt) * 32 + lane]);
+                    for (int tt = 0; tt < NT; ++tt) tk[tt] = tt < T ? tt : 0;
+                    float g[NT], u[NT];
+                    g_piece<NT>(P, ring + (size_t)(tseq % (unsigned)ns) * P.slot_bytes, pi, T, tk, x, xs, g, u);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int tt = 0; tt < NT; ++tt)
+                            if (tt < T) P.a_sh[(size_t)tt * P.Is + row0 + pi] = silu_mul(g[tt], u[tt]);
+                    }
+                    piece_done(S, P, tseq, P.ready);
+                }
+            }
+            seq += (unsigned)cw.nshg;
+        }
+        // ---------------------------------------------------------- K: top-k and buckets
+        // (the logits carry the layer's tag: no barrier before reading them)
+        topk_bucket(P, S, cand, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
+        if (threadIdx.x == 0) S.verdict = ldcg_int(P.err) == 0;
+        consumer_sync();
+        if (!(ok = S.verdict != 0)) break;
+        if (threadIdx.x == 0) {
+            S.exp_ready[0] += (unsigned)P.units_s;
+            for (int j = 0; j < S.D; ++j) S.exp_ready[1 + j] += (unsigned)P.units_r;
+            __threadfence_block();
+            S.tables_layer = l + 1;  // the producer may issue this layer's routed copies
+        }
+        consumer_sync();
+        // ---------------------------------------------------------- G and D
+        const int D = S.D, nu = D * P.units_r;
+        const int nrg = c < nu ? (nu - 1 - c) / G + 1 : 0;
+        const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
+        const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(nrg, 1) - 1) / max(nrg, 1))) : 8;
+        const int nitems = nrg * npc + ngr * cw.nblk;
+#pragma unroll 1
+        for (int i = wid; i < nitems; i += kCW) {
+            if (i < nrg * npc) {
+                const int ui = i / npc, pi = i - ui * npc;
+                const unsigned tseq = seq + (unsigned)ui;
+                if (!wait_task(S, P, tseq)) break;
+                const int u = c + ui * G, j = u / P.units_r, sub = u - j * P.units_r;
+                const int n = S.slot_n[j], off = S.slot_off[j];
+                if (kMma) {
+                    unit_piece_mma(S, P, ring, part, tseq, pi, npc, n, S.pos_tok + off, S.pos_idx + off, P.a_r, P.I,
+                                   sub * 8, xb, xs, P.ready + 1 + j);
+                } else {
+                    int tk[NT];
+#pragma unroll
+                    for (int tt = 0; tt < NT; ++tt) tk[tt] = S.pos_tok[off + (tt < n ? tt : 0)];
+                    float g[NT], uu[NT];
+                    g_piece<NT>(P, ring + (size_t)(tseq % (unsigned)ns) * P.slot_bytes, pi, n, tk, x, xs, g, uu);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int tt = 0; tt < NT; ++tt)
+                            if (tt < n) P.a_r[(size_t)(off + tt) * P.I + sub * 8 + pi] = silu_mul(g[tt], uu[tt]);
+                    }
+                    piece_done(S, P, tseq, P.ready + 1 + j);
+                }
+            } else {
+                const int di = i - nrg * npc, gi = di / cw.nblk, bi = di - gi * cw.nblk;
+                const unsigned tseq = seq + (unsigned)(nrg + gi);
+                if (!wait_task(S, P, tseq)) break;
+                const DGroup dg = dgroup(P, gi);
+                const int n = dg.shd ? T : S.slot_n[dg.j], off = dg.shd ? 0 : S.slot_off[dg.j];
+                const int s = (int)(tseq % (unsigned)ns);
+                unsigned char *slot = ring + (size_t)s * P.slot_bytes;
+                unsigned char *area = slot + cw.nblk * (dg.dcb + dg.sbd);
+                const unsigned char *codes = slot + bi * dg.dcb, *sbp = slot + cw.nblk * dg.dcb + bi * dg.sbd;
+                if (kMma) {
+                    float *asg = reinterpret_cast<float *>(area + (size_t)n * ahl_token_bytes(dg.pc));
+                    if (!stage_a_mma(S, P, s, dg.shd, dg.j, dg.p, dg.pc, dg.pcv, n, off, area, asg)) break;
+                    float y[2];
+                    d_block_mma(codes, sbp, area, asg, dg.pc, dg.pcv, n, y);
+                    const int g8 = lane >> 2, t4 = lane & 3;
+                    if (g8 < n) {
+                        const int entry = dg.shd ? T * P.k * P.parts_r + dg.p * T + g8
+                                                 : S.pos_pair[off + g8] * P.parts_r + dg.p;
+                        ybuf[(size_t)entry * P.yrows + bi * 8 + 2 * t4] = y[0];
+                        ybuf[(size_t)entry * P.yrows + bi * 8 + 2 * t4 + 1] = y[1];
+                    }
+                } else {
+                    float *apre = reinterpret_cast<float *>(area);
+                    float *asum = apre + (size_t)n * dg.pc * kXStride;
+                    if (!stage_a(S, P, s, dg.shd, dg.j, dg.p, dg.pc, dg.pcv, n, off, apre, asum)) break;
+                    float y[NT];
+                    d_block<NT>(codes, sbp, apre, asum, dg.pc, dg.pcv, n, y);
+                    if (lane < 8) {
+                        const int row = bi * 8 + lane;
+#pragma unroll
+                        for (int tt = 0; tt < NT; ++tt) {
+                            if (tt < n) {
+                                const int entry = dg.shd ? T * P.k * P.parts_r + dg.p * T + tt
+                                                         : S.pos_pair[off + tt] * P.parts_r + dg.p;
+                                ybuf[(size_t)entry * P.yrows + row] = y[tt];
+                            }
+                        }
                     }
                 }
-                const float a = silu_mul(gs, us);
-                const size_t rs = (size_t)task_rowset(P, t, tt);
-                P.act[rs * P.Kmax + t.rb * 32 + lane] = a * code_prescale(lane & 7);
-                const float cs = warp_sum(a);  // the job's 32 rows are one 32-column chunk of the down input
-                if (lane == 0) P.act_cs[rs * (P.Kmax / 32) + t.rb] = cs;
-            }
-            __syncwarp();
-            if (lane == 0) {
-                P.cnt_gu[t.job] = 0u;
-                atom_add_release_gpu(&P.act_done[t.slot], 1u);  // the job's rows of a are written
+                block_done(S, P, tseq, cw.nblk);
             }
         }
+        seq += (unsigned)(nrg + ngr);
+        consumer_sync();
+        // ---------------------------------------------------------- the combine of this CTA's rows
+        if (cw.nblk > 0) {
+            const int nrows = cw.nblk * 8, r0 = cw.b0 * 8, k = P.k, pr = P.parts_r;
+#pragma unroll 1
+            for (int i = threadIdx.x; i < T * nrows; i += kCThreads) {
+                const int t = i / nrows, r = i - t * nrows;
+                float acc = 0.f;
+#pragma unroll 1
+                for (int s2 = 0; s2 < k; ++s2) {
+                    float ys = 0.f;
+                    for (int p = 0; p < pr; ++p) ys += ybuf[(size_t)((t * k + s2) * pr + p) * P.yrows + r];
+                    acc = fmaf(S.wts[t * k + s2], ys, acc);
+                }
+                float sh = 0.f;
+                for (int p = 0; p < P.parts_s; ++p) sh += ybuf[(size_t)(T * k * pr + p * T + t) * P.yrows + r];
+                P.m[(size_t)t * H + r0 + r] = acc + sh;
+            }
+        }
+        consumer_sync();
+        if (threadIdx.x == 0) grid_arrive(P);  // m rows written
     }
-    return ok;
+    if (ok && grid_wait(P, S, ++nbar)) finish_layer(P, S, hs, P.L - 1);
 }
 
-// Stage the down inputs of segments [k0, k1): a (already pre-scaled for the
-// code decode) and its chunk sums.  Consumer threads only.
-__device__ __noinline__ bool stage_segments(const Cfg &P, Smem &S, int k0, int k1) {
-    const int ctid = threadIdx.x, KC = P.Kmax / 32;
-    // every consumer warp is past its gate/up tasks (the stage still held their
-    // input); then wait until each staged slot's SwiGLU rows are all written
-    consumer_sync();
-    if (ctid == 0) {
-        bool ok = true;
-        for (int k2 = k0; k2 < k1 && ok; ++k2) ok = wait_count(P, &P.act_done[S.seg[k2].slot], S.act_expect[S.seg[k2].slot]);
-        __threadfence();
-        S.flag2 = ok;
-    }
-    consumer_sync();
-    if (!S.flag2) return false;
-#pragma unroll 1
-    for (int k2 = k0; k2 < k1; ++k2) {
-        const SegDesc sg = S.seg[k2];
-        const int q4 = sg.ld / 4, nc = sg.ld / 32;
-        const int rs0 = sg.slot == 0 ? 0 : P.T + sg.seg0;
-#pragma unroll 1
-        for (int e = ctid; e < sg.n * q4; e += kCWarps * 32) {
-            const int tt = e / q4, c4 = e - tt * q4;
-            reinterpret_cast<float4 *>(S.stage + sg.off + (size_t)tt * sg.ld)[c4] =
-                __ldcg(reinterpret_cast<const float4 *>(P.act + (size_t)(rs0 + tt) * P.Kmax + sg.g0 * 64) + c4);
+// ------------------------------------------------------------------ producer
+
+// Hand ring slot of task `sq` to the task and arm its full barrier for
+// `bytes`; null on a timeout or a recorded error.
+__device__ __forceinline__ unsigned char *claim(Shared &S, const Cfg &P, unsigned char *ring, unsigned sq,
+                                               unsigned bytes) {
+    const int s = (int)(sq % (unsigned)P.ns);
+    const unsigned q = sq / (unsigned)P.ns;
+    if (q > 0 && !mbar_wait(&S.empty[s], (q - 1u) & 1u, P.err, kErrEmpty)) return nullptr;
+    S.owner[s] = sq;
+    mbar_expect_tx(&S.full[s], bytes);
+    return ring + (size_t)s * P.slot_bytes;
+}
+
+__device__ __noinline__ bool issue_seg_a(Shared &S, const Cfg &P, const moe_layer_w &W, const CUtensorMap *mp,
+                                         unsigned char *ring, const CtaWork &cw, unsigned &seq) {
+    const int H = P.H, G = gridDim.x, c = blockIdx.x;
+    {
+        const RouterCopy rc = router_copy(P);
+        const unsigned rows_bytes = (unsigned)rc.nrows * H;
+        unsigned char *dst = claim(S, P, ring, seq, 2u * H + rows_bytes + 2u * rc.sbb);
+        if (!dst) return false;
+        unsigned long long *fb = &S.full[seq % (unsigned)P.ns];
+        bulk_g2s(dst, W.router_scale, 2u * H, fb);
+        if (rc.nrows > 0) {
+            bulk_g2s(dst + 2 * H, W.router_q + (size_t)rc.e0 * (H / 4), rows_bytes, fb);
+            bulk_g2s(dst + 2 * H + rows_bytes, reinterpret_cast<const char *>(W.router_s) + rc.sb_lo, rc.sbb, fb);
+            bulk_g2s(dst + 2 * H + rows_bytes + rc.sbb, reinterpret_cast<const char *>(W.router_b) + rc.sb_lo, rc.sbb,
+                     fb);
         }
-#pragma unroll 1
-        for (int e = ctid; e < sg.n * nc; e += kCWarps * 32) {
-            const int tt = e / nc, c = e - tt * nc;
-            S.xs[(sg.off + tt * sg.ld) / 32 + c] = __ldcg(&P.act_cs[(size_t)(rs0 + tt) * KC + sg.g0 * 2 + c]);
-        }
+        ++seq;
     }
-    consumer_sync();
+    const unsigned ubytes = 2u * P.CH * 128u + 2u * P.GH * 32u;
+#pragma unroll 1
+    for (int ui = 0; ui < cw.nshg; ++ui) {
+        const int u = c + ui * G, rb = u >> 2, x = u & 3;
+        unsigned char *dst = claim(S, P, ring, seq, ubytes);
+        if (!dst) return false;
+        unsigned long long *fb = &S.full[seq % (unsigned)P.ns];
+        tma_load_3d(dst, mp + kMapShGateQ, 32 * x, 0, rb, fb);
+        tma_load_3d(dst + P.gcb, mp + kMapShUpQ, 32 * x, 0, rb, fb);
+        tma_load_3d(dst + 2 * P.gcb, mp + kMapShGateSb, 8 * x, 0, rb, fb);
+        tma_load_3d(dst + 2 * P.gcb + P.sbs, mp + kMapShUpSb, 8 * x, 0, rb, fb);
+        ++seq;
+    }
     return true;
 }
 
-// The combine m[t][row] = sum_s w[t,s] * y[t,s] + shared, in a fixed order.
-// y and the shared output are sums of kWPT * ndp parts; the loads of up to
-// 2 parts x 8 routed slots (or 8 shared parts) are issued before any is used.
-__device__ __noinline__ void combine_row(const Cfg &P, const Smem &S, int row) {
-    const int T = P.T, k = P.k, H = P.H, ny = P.ndp_r * kWPT, nsh = P.ndp_s * kWPT;
-    const size_t ystride = (size_t)T * k * H;
+// The router rows and shared-expert units of a layer into L2 (no shared
+// memory): issued while the previous layer's routed weights stream, so that
+// the layer's first copies find their bytes in L2.
+__device__ __noinline__ void prefetch_seg_a(const Cfg &P, const moe_layer_w &W, const CUtensorMap *mp,
+                                            const CtaWork &cw) {
+    const int H = P.H, G = gridDim.x, c = blockIdx.x;
+    const RouterCopy rc = router_copy(P);
+    prefetch_l2(W.router_scale, 2u * H);
+    if (rc.nrows > 0) {
+        const char *rows = reinterpret_cast<const char *>(W.router_q + (size_t)rc.e0 * (H / 4));
+        for (unsigned o = 0, n = (unsigned)rc.nrows * H; o < n; o += 65536u) prefetch_l2(rows + o, min(65536u, n - o));
+        prefetch_l2(reinterpret_cast<const char *>(W.router_s) + rc.sb_lo, rc.sbb);
+        prefetch_l2(reinterpret_cast<const char *>(W.router_b) + rc.sb_lo, rc.sbb);
+    }
 #pragma unroll 1
-    for (int t = 0; t < T; ++t) {
-        float mv = 0.f;
-#pragma unroll 1
-        for (int s0 = 0; s0 < k; s0 += 8) {
-            float yv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) yv[u] = 0.f;
-#pragma unroll 1
-            for (int d0 = 0; d0 < ny; d0 += 2) {
-                float pv[2][8];
-#pragma unroll
-                for (int d = 0; d < 2; ++d)
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        pv[d][u] = (d0 + d < ny && s0 + u < k)
-                                       ? __ldcg(&P.y[(d0 + d) * ystride + (size_t)(t * k + s0 + u) * H + row])
-                                       : 0.f;
-#pragma unroll
-                for (int d = 0; d < 2; ++d)
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) yv[u] += pv[d][u];
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (s0 + u < k) mv = fmaf(S.wts[t * k + s0 + u], yv[u], mv);
-        }
-#pragma unroll 1
-        for (int u0 = 0; u0 < nsh; u0 += 8) {
-            float sv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) sv[u] = u0 + u < nsh ? __ldcg(&P.sh[((size_t)(u0 + u) * T + t) * H + row]) : 0.f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) mv += sv[u];
-        }
-        P.m[(size_t)t * H + row] = mv;
+    for (int ui = 0; ui < cw.nshg; ++ui) {
+        const int u = c + ui * G, rb = u >> 2, x = u & 3;
+        tma_prefetch_3d(mp + kMapShGateQ, 32 * x, 0, rb);
+        tma_prefetch_3d(mp + kMapShUpQ, 32 * x, 0, rb);
+        tma_prefetch_3d(mp + kMapShGateSb, 8 * x, 0, rb);
+        tma_prefetch_3d(mp + kMapShUpSb, 8 * x, 0, rb);
     }
 }
 
-template <int NT>
-__device__ __noinline__ bool dn_consumer(const Cfg &P, Smem &S, unsigned rq) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, team = wid / kWPT, mb = wid - team * kWPT;
-    const int T = P.T, k = P.k, H = P.H, ns = P.nslots, nt = S.ndt;
-    // member results per row block in this layer: every part of the shared expert and of each active slot
-    const unsigned dn_per_rb = (unsigned)((P.ndp_s + S.nact * P.ndp_r) * kWPT);
-    const int rounds = S.seg_rounds;
-    bool ok = true;
+// Coordinates of routed gate/up unit u (of the grid's D * units_r) of the layer.
+__device__ __forceinline__ void routed_unit(const Cfg &P, const Shared &S, int u, int &rb, int &x) {
+    const int j = u / P.units_r, sub = u - j * P.units_r;
+    rb = S.slot_e[j] * (P.I / 32) + (sub >> 2);
+    x = sub & 3;
+}
+
+// Row block of 8-row output block b of down group dg (routed: of slot j's expert).
+__device__ __forceinline__ int down_rb(const Cfg &P, const Shared &S, const DGroup &dg, int b) {
+    return (dg.shd ? 0 : S.slot_e[dg.j] * (P.H / 32)) + (b >> 2);
+}
+
+__device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned char *base) {
+    if ((threadIdx.x & 31) != 0) return;
+    const Cfg &P = S.c;
+    const int G = gridDim.x, c = blockIdx.x, ns = P.ns;
+    unsigned char *ring = base + P.off_ring;
+    const CtaWork cw = cta_work(P);
+    unsigned seq = 0;
+    bool ok = issue_seg_a(S, P, Pk.layers[0], P.maps, ring, cw, seq);
 #pragma unroll 1
-    for (int r = 0; r < rounds; ++r) {
-        const int k0 = rounds == 1 ? 0 : r, k1 = rounds == 1 ? S.nseg : r + 1;
-        if (!stage_segments(P, S, k0, k1)) return false;
+    for (int l = 0; l < P.L && ok; ++l) {
+        {  // this layer's routing tables
+            const unsigned long long t0 = globaltimer();
+            for (unsigned it = 0; S.tables_layer < l + 1; ++it) {
+                if ((it & 63u) == 63u && (ldcg_int(P.err) != 0 || globaltimer() - t0 > kWaitNs)) {
+                    atomicCAS(P.err, 0, kErrTables);
+                    ok = false;
+                    break;
+                }
+                __nanosleep(64);
+            }
+            if (!ok) break;
+            __threadfence_block();
+        }
+        const CUtensorMap *mp = P.maps + (size_t)l * kMaps;
+        const int D = S.D, nu = D * P.units_r;
+        const int nrg = c < nu ? (nu - 1 - c) / G + 1 : 0;
+        const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
+        // every routed byte this CTA needs beyond what the ring takes at once: into L2 now
 #pragma unroll 1
-        for (int i = team; i < nt; i += kTeams) {
-            const TaskDesc t = S.dnt[i];
-            if (t.seg < k0 || t.seg >= k1) continue;
-            int s;
-            unsigned ph;
-            ring_pos(rq, i, ns, s, ph);
-            const SegDesc sg = S.seg[t.seg];
-            const int n = t.n, ng = t.g1 - t.g0;
-            float acc[NT];
-#pragma unroll
-            for (int tt = 0; tt < NT; ++tt) acc[tt] = 0.f;
-            const bool got = wait_task(S, rq + (unsigned)i, s, ph, P.err);
-            if (got)  // token tt's row at off + tt * ld, its chunk sums at (off + tt * ld) / 32
-                task_dot<NT>(S.pool + (size_t)s * kSlotBytes, ng, mb, S.stage + sg.off, S.xs + sg.off / 32, nullptr,
-                             sg.ld, n, acc, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.empty[s]);
-            if (!got) {
+        for (int ui = ns; ui < nrg; ++ui) {
+            int rb, x;
+            routed_unit(P, S, c + ui * G, rb, x);
+            tma_prefetch_3d(mp + kMapGateQ, 32 * x, 0, rb);
+            tma_prefetch_3d(mp + kMapUpQ, 32 * x, 0, rb);
+            tma_prefetch_3d(mp + kMapGateSb, 8 * x, 0, rb);
+            tma_prefetch_3d(mp + kMapUpSb, 8 * x, 0, rb);
+        }
+#pragma unroll 1
+        for (int gi = 0; gi < ngr; ++gi) {
+            const DGroup dg = dgroup(P, gi);
+            for (int bi = 0; bi < cw.nblk; ++bi) {
+                const int b = cw.b0 + bi, rb = down_rb(P, S, dg, b);
+                tma_prefetch_3d(mp + (dg.shd ? kMapShDownQ : kMapDownQ), 32 * (b & 3), dg.p * dg.pc, rb);
+                tma_prefetch_3d(mp + (dg.shd ? kMapShDownSb : kMapDownSb), 8 * (b & 3), dg.p * (dg.pc / 2), rb);
+            }
+        }
+        // routed gate/up units, then the down groups, in ring order
+        const unsigned ubytes = 2u * P.CH * 128u + 2u * P.GH * 32u;
+#pragma unroll 1
+        for (int ui = 0; ui < nrg && ok; ++ui) {
+            int rb, x;
+            routed_unit(P, S, c + ui * G, rb, x);
+            unsigned char *dst = claim(S, P, ring, seq, ubytes);
+            if (!dst) {
                 ok = false;
-                continue;
+                break;
             }
-            const int row = t.rb * 32 + lane, pm = t.part * kWPT + mb;
-#pragma unroll
-            for (int tt = 0; tt < NT; ++tt) {
-                if (tt < n) {
-                    if (t.slot == 0)
-                        P.sh[((size_t)pm * T + tt) * H + row] = acc[tt];
-                    else
-                        P.y[((size_t)pm * T * k + S.perm[t.seg0 + tt]) * H + row] = acc[tt];
-                }
-            }
-            // count this task for its row block (release: the warp's rows, ordered
-            // by __syncwarp, become visible first); the last one forms the combine
-            __syncwarp();
-            unsigned old = 0u;
-            if (lane == 0) old = atom_add_release_gpu(&P.cnt_dn[t.rb], 1u);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if (old == dn_per_rb - 1u) {
-                if (lane == 0) __threadfence();
-                __syncwarp();
-                combine_row(P, S, row);
-                __syncwarp();
-                if (lane == 0) {
-                    P.cnt_dn[t.rb] = 0u;
-                    atom_add_release_gpu(P.rows_done, 1u);  // these 32 rows of m are written
-                }
-            }
+            unsigned long long *fb = &S.full[seq % (unsigned)ns];
+            tma_load_3d(dst, mp + kMapGateQ, 32 * x, 0, rb, fb);
+            tma_load_3d(dst + P.gcb, mp + kMapUpQ, 32 * x, 0, rb, fb);
+            tma_load_3d(dst + 2 * P.gcb, mp + kMapGateSb, 8 * x, 0, rb, fb);
+            tma_load_3d(dst + 2 * P.gcb + P.sbs, mp + kMapUpSb, 8 * x, 0, rb, fb);
+            ++seq;
         }
-        if (rounds > 1) consumer_sync();
+        if (ok && l + 1 < P.L) prefetch_seg_a(P, Pk.layers[l + 1], P.maps + (size_t)(l + 1) * kMaps, cw);
+#pragma unroll 1
+        for (int gi = 0; gi < ngr && ok; ++gi) {
+            const DGroup dg = dgroup(P, gi);
+            const unsigned gbytes = (unsigned)cw.nblk * (unsigned)(dg.pc * 128 + dg.pc * 16);
+            unsigned char *dst = claim(S, P, ring, seq, gbytes);
+            if (!dst) {
+                ok = false;
+                break;
+            }
+            unsigned long long *fb = &S.full[seq % (unsigned)ns];
+            for (int bi = 0; bi < cw.nblk; ++bi) {
+                const int b = cw.b0 + bi, rb = down_rb(P, S, dg, b);
+                tma_load_3d(dst + bi * dg.dcb, mp + (dg.shd ? kMapShDownQ : kMapDownQ), 32 * (b & 3), dg.p * dg.pc, rb,
+                            fb);
+                tma_load_3d(dst + cw.nblk * dg.dcb + bi * dg.sbd, mp + (dg.shd ? kMapShDownSb : kMapDownSb), 8 * (b & 3),
+                            dg.p * (dg.pc / 2), rb, fb);
+            }
+            ++seq;
+        }
+        if (ok && l + 1 < P.L) ok = issue_seg_a(S, P, Pk.layers[l + 1], P.maps + (size_t)(l + 1) * kMaps, ring, cw, seq);
     }
-    return ok;
-}
-
-// All threads: wait until `target` row blocks of m are combined (over all layers so far).
-__device__ __noinline__ bool wait_rows(const Cfg &P, Smem &S, unsigned target) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const bool ok = wait_count(P, P.rows_done, target);
-        __threadfence();
-        S.flag = ok && ldcg_int(P.err) == 0;
-    }
-    __syncthreads();
-    return S.flag != 0;
+    // let this thread's copies land before the CTA ends (bounded)
+    for (unsigned q = seq > (unsigned)ns ? seq - (unsigned)ns : 0u; q < seq; ++q)
+        mbar_drain(&S.full[q % (unsigned)ns], (q / (unsigned)ns) & 1u);
 }
 
 // ------------------------------------------------------------------ kernel
 
+template <int NT, bool MMA>
 __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_constant__ Params Pk) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem &S = *reinterpret_cast<Smem *>(smem_raw);
-    const Cfg &P = S.c;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const bool producer = (wid == kProducerWarp && lane == 0);
-    const bool consumer = wid < kCWarps;
-
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Shared &S = *reinterpret_cast<Shared *>(base);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], kWPT);  // every warp of the task's team
+        for (int i = 0; i < kMaxSlots; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], 1);
         }
-        mbar_init(&S.rbar, 1);
-        for (int s = 0; s < kMaxStages; ++s) S.slot_task[s] = 0xffffffffu;
-        for (int s = 0; s <= kMaxPairs; ++s) S.act_expect[s] = 0u;
-        S.stage = reinterpret_cast<float *>(S.pool + (size_t)Pk.c.nslots * kSlotBytes);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    copy_words(&S.c, &Pk.c, sizeof(Cfg));
-    copy_words(&S.w, &Pk.layers[0], sizeof(moe_layer_w));
-    __syncthreads();
-
-    unsigned rq = 0;       // ring sequence number of the next task (the same in every thread)
-    unsigned issued = 0;   // producer: tasks whose copies were actually issued
-    unsigned rissued = 0;  // producer: router copy batches issued (one per layer)
-    unsigned nbar = 0;     // grid barriers passed
-    bool ok = true;
-    const int ns = P.nslots;
-
-    for (int l = 0; l < P.L && ok; ++l) {
-        const moe_layer_w &W = S.w;
-        const moe_layer_w *next = l + 1 < P.L ? &Pk.layers[l + 1] : nullptr;
-        if (producer) {
-            issue_router_copies(P, S, W);
-            ++rissued;
-        }
-        if (l == 0) {
-            load_input(P, S, P.h_in);
-        } else {
-            // every row block of the previous layer's m is combined
-            ok = wait_rows(P, S, (unsigned)l * (unsigned)(P.H / 32));
-            if (!ok) break;
-            finish_layer(P, S, l - 1);
-            if (!P.chained) load_input(P, S, P.h_in + (size_t)l * P.T * P.H);
-        }
-        router_phase(P, S, l);
-        ok = grid_sync(P, ++nbar, &S.flag);
-        if (!ok) break;
-        topk_phase(P, S, W);
-        stage_x(P, S);
-
-        // ---------------- gate/up tasks
-        if (producer)
-            task_producer(P, S, W, false, rq, next, issued);
-        else if (consumer) {
-            P.T == 1 ? gu_consumer<1>(P, S, rq) : gu_consumer<kMaxT>(P, S, rq);
-            if (wid == kCWarps - 1) gate_weights(P, S, W);
-        }
-        rq += (unsigned)S.ngt;
-
-        // ---------------- down tasks (each CTA as soon as its own gate/up tasks are done)
-        if (producer)
-            task_producer(P, S, W, true, rq, next, issued);
-        else if (consumer)
-            P.T == 1 ? dn_consumer<1>(P, S, rq) : dn_consumer<kMaxT>(P, S, rq);
-        rq += (unsigned)S.ndt;
-        __syncthreads();
-        if (threadIdx.x == 0) S.flag = ldcg_int(P.err) == 0;
-        if (next != nullptr) copy_words(&S.w, next, sizeof(moe_layer_w));  // every use of this layer's is done
-        __syncthreads();
-        ok = S.flag != 0;
+    for (int i = threadIdx.x; i < (int)(sizeof(Cfg) / 4); i += blockDim.x)
+        reinterpret_cast<unsigned *>(&S.c)[i] = reinterpret_cast<const unsigned *>(&Pk.c)[i];
+    for (int i = threadIdx.x; i < kMaxSlots; i += blockDim.x) {
+        S.owner[i] = 0xffffffffu;
+        S.cnt[i] = 0;
+        S.astate[i] = 0;
     }
-    if (ok) ok = wait_rows(P, S, (unsigned)P.L * (unsigned)(P.H / 32));
-    if (ok) finish_layer(P, S, P.L - 1);  // ok is uniform across the CTA here
-
-    // let this CTA's own bulk copies land before it exits (bounded)
-    __syncthreads();
-    if (producer) {
-        const unsigned first = issued > (unsigned)ns ? issued - ns : 0u;
-        for (unsigned q = first; q < issued; ++q) mbar_drain(&S.full[q % ns], (q / ns) & 1);
-        if (rissued > 0) mbar_drain(&S.rbar, (rissued - 1) & 1);
+    for (int i = threadIdx.x; i < 1 + kMaxPairs; i += blockDim.x) S.exp_ready[i] = 0u;
+    for (int i = threadIdx.x; i < kMaxPairs; i += blockDim.x) S.pos_idx[i] = i;
+    for (int i = threadIdx.x; i < kMaxT; i += blockDim.x) S.toks_sh[i] = i;
+    if (threadIdx.x == 0) {
+        S.tables_layer = 0;
+        S.verdict = 1;
     }
+    __syncthreads();
+    if ((threadIdx.x >> 5) == kProdWarp)
+        producer_main(Pk, S, base);
+    else
+        consumer_main<NT, MMA>(Pk, S, base);
+    __syncthreads();
 }
 
 }  // namespace dec
 
-size_t decode_stack_smem() { return sizeof(dec::Smem); }
+// ------------------------------------------------------------------ host side
 
-static_assert(sizeof(dec::Smem) <= 227 * 1024, "decode kernel shared memory exceeds 227 KiB");
-static_assert(sizeof(dec::Params) <= 32000, "decode kernel parameters exceed the 32 KiB limit");
-static_assert(sizeof(dec::Cfg) % 4 == 0 && sizeof(moe_layer_w) % 4 == 0, "copied word by word");
+namespace {
+
+size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct DecodeWs {
-    size_t bar, cnt_dn, cnt_gu, act_done, logits, gpart, act, act_cs, y, sh, m, total, zero_bytes;
+    size_t ctl, ready, zero_bytes, logits, a_sh, a_r, m, maps, total;
 };
 
-static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-static DecodeWs decode_ws(const moe_layer_w *w, int T) {
+// Workspace: control words (barrier counters 128 bytes apart; the status word
+// at byte 4), readiness counts, logits, SwiGLU outputs, m, tensor maps.
+DecodeWs decode_ws(const moe_layer_w *w, int T) {
     DecodeWs d;
-    const int Kmax = w->I > w->Is ? w->I : w->Is;
-    const int R = T + T * w->k;
-    const int ndp_r = (w->I / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    const int ndp_s = (w->Is / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
     size_t off = 0;
-    auto take = [&](size_t b) {
+    auto take = [&](size_t b, size_t a = 256) {
+        off = al(off, a);
         const size_t o = off;
-        off += al256(b);
+        off += b;
         return o;
     };
-    d.bar = take(256);
-    const size_t pairs = (size_t)T * w->k < (size_t)w->E ? (size_t)T * w->k : (size_t)w->E;
-    const size_t jobs = (size_t)w->Is / 32 + pairs * (w->I / 32);
-    const size_t pg = (w->H / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    d.cnt_dn = take(sizeof(unsigned) * (size_t)(w->H / 32));
-    d.cnt_gu = take(sizeof(unsigned) * jobs);
-    d.act_done = take(sizeof(unsigned) * (R + 1));  // per slot, then rows_done
-    d.zero_bytes = off;
-    d.gpart = take(sizeof(float) * jobs * 2 * pg * dec::kWPT * T * 32);
-    d.logits = take(sizeof(double) * (size_t)T * w->E);
-    d.act = take(sizeof(float) * (size_t)R * Kmax);
-    d.act_cs = take(sizeof(float) * (size_t)R * (Kmax / 32));
-    d.y = take(sizeof(float) * (size_t)ndp_r * dec::kWPT * T * w->k * w->H);
-    d.sh = take(sizeof(float) * (size_t)ndp_s * dec::kWPT * T * w->H);
+    d.ctl = take(2048);
+    d.ready = take(sizeof(unsigned) * (1 + dec::kMaxPairs));
+    d.logits = take(2 * sizeof(unsigned long long) * (size_t)T * w->E);  // flag-in-data words: zeroed per launch
+    d.zero_bytes = al(off, 256);
+    d.a_sh = take(sizeof(float) * (size_t)T * w->Is);
+    d.a_r = take(sizeof(float) * (size_t)T * w->k * w->I);
     d.m = take(sizeof(float) * (size_t)T * w->H);
-    d.total = off;
+    d.maps = take(sizeof(CUtensorMap) * dec::kMaxLayers * dec::kMaps, 128);
+    d.total = al(off, 256);
     return d;
 }
+
+// K-parts of a down matrix with K input columns: parts of at most
+// kPartChunks chunks, an even number of chunks each (whole groups).
+void down_parts(int K, int *parts, int *pc) {
+    const int C = K / 32, Gk = K / 64;
+    int n = (C + dec::kPartChunks - 1) / dec::kPartChunks;
+    *parts = n;
+    *pc = 2 * ((Gk + n - 1) / n);
+}
+
+// The kernel's shared-memory plan for layers shaped like w, T tokens, a grid
+// of `grid` CTAs; false if it does not fit.
+bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, size_t *smem) {
+    if (grid <= 0 || T < 1 || T > dec::kMaxT || (long)T * w.H > dec::kMaxStageTH || w.H > 4096) return false;
+    if ((long)T * w.k > dec::kMaxPairs) return false;
+    P.H = w.H;
+    P.E = w.E;
+    P.k = w.k;
+    P.I = w.I;
+    P.Is = w.Is;
+    P.T = T;
+    P.CH = w.H / 32;
+    P.GH = w.H / 64;
+    P.units_s = w.Is / 8;
+    P.units_r = w.I / 8;
+    P.nrb8 = w.H / 8;
+    down_parts(w.Is, &P.parts_s, &P.pc_s);
+    down_parts(w.I, &P.parts_r, &P.pc_r);
+    if (P.parts_s > dec::kMaxParts || P.parts_r > dec::kMaxParts) return false;
+    const int nblk_max = (P.nrb8 + grid - 1) / grid;
+    if (nblk_max > dec::kMaxBlk) return false;
+    P.gcb = (int)al((size_t)P.CH * 128, 1024);
+    P.sbs = (int)al((size_t)P.GH * 32, 128);
+    P.dcb_s = (int)al((size_t)P.pc_s * 128, 1024);
+    P.dcb_r = (int)al((size_t)P.pc_r * 128, 1024);
+    P.sbd_s = (int)al((size_t)P.pc_s * 16, 128);
+    P.sbd_r = (int)al((size_t)P.pc_r * 16, 128);
+    const size_t g_slot = 2 * (size_t)P.gcb + 2 * (size_t)P.sbs;
+    auto d_slot = [&](int dcb, int sbd, int pc) {
+        const size_t area = mma ? (size_t)T * dec::ahl_token_bytes(pc) + (size_t)T * (pc / 2) * 4
+                                : (size_t)T * pc * (dec::kXStride + 1) * 4;
+        return (size_t)nblk_max * (dcb + sbd) + area;
+    };
+    const long nrows_r = (w.E + grid - 1) / grid;
+    const size_t r_slot = 2 * (size_t)w.H + nrows_r * w.H + 2 * al(nrows_r * P.GH * 2 + 32, 16);
+    size_t slot = g_slot;
+    slot = std::max(slot, d_slot(P.dcb_s, P.sbd_s, P.pc_s));
+    slot = std::max(slot, d_slot(P.dcb_r, P.sbd_r, P.pc_r));
+    slot = std::max(slot, r_slot);
+    P.slot_bytes = (int)al(slot, 1024);
+    const int nsl = (w.E + 31) / 32;
+    P.maxc = std::min(w.E, nsl * std::min(w.k, 32));
+    if (P.maxc > dec::kMaxCand) return false;
+    P.yrows = 8 * dec::kMaxBlk;
+    // after the fixed part: ring (1024-aligned), x, xs, h, ybuf, candidates
+    size_t off = al(sizeof(dec::Shared), 1024);
+    P.off_ring = (int)off;
+    const size_t x_bytes = mma ? (size_t)T * dec::xb_token_bytes(P.CH) : (size_t)T * P.CH * dec::kXStride * 4;
+    const size_t xs_bytes = mma ? (size_t)T * P.GH * 4 : (size_t)T * P.CH * 4;
+    const size_t part_per_slot = mma ? (size_t)dec::kMaxPieces * 128 * 4 : 0;
+    const size_t fixed_tail = al(x_bytes, 16) + al(xs_bytes, 16) + al((size_t)T * w.H * 2, 16) +
+                              al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16) +
+                              al((size_t)T * P.maxc * sizeof(dec::Cand), 16);
+    const size_t budget = 227 * 1024 - 1024;  // the base is aligned to 1024 bytes inside the allocation
+    if (off + fixed_tail + 3 * ((size_t)P.slot_bytes + part_per_slot) > budget) return false;
+    long ns = (long)((budget - off - fixed_tail) / ((size_t)P.slot_bytes + part_per_slot));
+    if (ns > dec::kMaxSlots) ns = dec::kMaxSlots;
+    P.ns = (int)ns;
+    off += (size_t)ns * P.slot_bytes;
+    P.off_x = (int)off;
+    off += al(x_bytes, 16);
+    P.off_xs = (int)off;
+    off += al(xs_bytes, 16);
+    P.off_h = (int)off;
+    off += al((size_t)T * w.H * 2, 16);
+    P.off_y = (int)off;
+    off += al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16);
+    P.off_cand = (int)off;
+    off += al((size_t)T * P.maxc * sizeof(dec::Cand), 16);
+    P.off_part = (int)off;
+    off += (size_t)ns * part_per_slot;
+    *smem = off + 1024;
+    return *smem <= 227 * 1024;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A tiled matrix set as a 3-D tensor of 32-bit words: [n_rb][per_rb][words],
+// boxes of {bx words, by, 1}.
+cudaError_t make_map(CUtensorMap *m, const uint32_t *ptr, int words, int per_rb, int n_rb, int bx, int by,
+                     bool swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)words, (cuuint64_t)per_rb, (cuuint64_t)n_rb};
+    const cuuint64_t strides[2] = {(cuuint64_t)words * 4, (cuuint64_t)words * 4 * per_rb};
+    const cuuint32_t box[3] = {(cuuint32_t)bx, (cuuint32_t)by, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The 12 tensor maps of one layer (see the kMap* enumeration).
+cudaError_t layer_maps(const moe_layer_w &w, const dec::Cfg &P, CUtensorMap *m) {
+    const int CH = w.H / 32, GH = w.H / 64, rr = w.E * w.I / 32, rs = w.Is / 32, rd = w.E * w.H / 32, rds = w.H / 32;
+    cudaError_t e;
+    if ((e = make_map(&m[dec::kMapGateQ], w.gate.q, 128, CH, rr, 32, CH, true)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapUpQ], w.up.q, 128, CH, rr, 32, CH, true)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapGateSb], w.gate.sb, 32, GH, rr, 8, GH, false)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapUpSb], w.up.sb, 32, GH, rr, 8, GH, false)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapShGateQ], w.sh_gate.q, 128, CH, rs, 32, CH, true)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapShUpQ], w.sh_up.q, 128, CH, rs, 32, CH, true)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapShGateSb], w.sh_gate.sb, 32, GH, rs, 8, GH, false)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapShUpSb], w.sh_up.sb, 32, GH, rs, 8, GH, false)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapDownQ], w.down.q, 128, w.I / 32, rd, 32, P.pc_r, true)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapDownSb], w.down.sb, 32, w.I / 64, rd, 8, P.pc_r / 2, false)) != cudaSuccess) return e;
+    if ((e = make_map(&m[dec::kMapShDownQ], w.sh_down.q, 128, w.Is / 32, rds, 32, P.pc_s, true)) != cudaSuccess)
+        return e;
+    return make_map(&m[dec::kMapShDownSb], w.sh_down.sb, 32, w.Is / 64, rds, 8, P.pc_s / 2, false);
+}
+
+// Host copies of the tensor maps of recent layer sets (a stack's maps are
+// encoded once and copied into the workspace on every launch).
+struct MapCache {
+    std::mutex mu;
+    struct Entry {
+        std::vector<moe_layer_w> key;
+        int pc_s = 0, pc_r = 0;
+        CUtensorMap *host = nullptr;  // pinned, L * kMaps maps
+        cudaEvent_t copied = nullptr;  // after the last copy out of `host`
+        unsigned long long used = 0;
+    };
+    Entry entries[8];
+    unsigned long long tick = 0;
+};
+MapCache g_maps;
+
+bool same_layers(const std::vector<moe_layer_w> &a, const moe_layer_w *b, int L) {
+    return (int)a.size() == L && std::memcmp(a.data(), b, sizeof(moe_layer_w) * L) == 0;
+}
+
+// Copies the maps of `layers` into the workspace (`dst`) on stream st,
+// encoding them first unless a recent launch used the same layer set.
+cudaError_t copy_maps(const moe_layer_w *layers, int L, const dec::Cfg &P, void *dst, cudaStream_t st) {
+    std::lock_guard<std::mutex> lock(g_maps.mu);
+    MapCache::Entry *hit = nullptr, *victim = &g_maps.entries[0];
+    for (auto &en : g_maps.entries) {
+        if (en.host && en.pc_s == P.pc_s && en.pc_r == P.pc_r && same_layers(en.key, layers, L)) hit = &en;
+        if (en.used < victim->used) victim = &en;
+    }
+    if (!hit) {
+        hit = victim;
+        if (!hit->host) {
+            cudaError_t e = cudaMallocHost(&hit->host, sizeof(CUtensorMap) * dec::kMaxLayers * dec::kMaps);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hit->copied, cudaEventDisableTiming);
+            if (e != cudaSuccess) {
+                if (hit->host) cudaFreeHost(hit->host);
+                hit->host = nullptr;
+                return e;
+            }
+        } else {
+            // an earlier launch may still be copying out of this entry
+            cudaError_t e = cudaEventSynchronize(hit->copied);
+            if (e != cudaSuccess) return e;
+        }
+        hit->key.assign(layers, layers + L);
+        hit->pc_s = P.pc_s;
+        hit->pc_r = P.pc_r;
+        for (int l = 0; l < L; ++l) {
+            cudaError_t e = layer_maps(layers[l], P, hit->host + (size_t)l * dec::kMaps);
+            if (e != cudaSuccess) {
+                hit->key.clear();
+                return e;
+            }
+        }
+    }
+    hit->used = ++g_maps.tick;
+    cudaError_t e = cudaMemcpyAsync(dst, hit->host, sizeof(CUtensorMap) * dec::kMaps * L, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaEventRecord(hit->copied, st);
+    return e;
+}
+
+template <int NT, bool MMA>
+const void *kernel_ptr() {
+    return reinterpret_cast<const void *>(dec::decode_stack_kernel<NT, MMA>);
+}
+
+// The tensor-core variants for T >= 2 (the CUDA cores' FMA work grows with T,
+// the MMA's does not), the CUDA-core FMAs for one token; force_path overrides.
+bool use_mma(int T, int force_path) { return force_path == 2 || (force_path == 0 && T >= 2); }
+
+const void *kernel_for(int T, bool mma) {
+    if (mma) return kernel_ptr<8, true>();
+    if (T <= 1) return kernel_ptr<1, false>();
+    if (T <= 2) return kernel_ptr<2, false>();
+    if (T <= 4) return kernel_ptr<4, false>();
+    return kernel_ptr<8, false>();
+}
+
+}  // namespace
 
 size_t decode_stack_ws_bytes(const moe_layer_w *w, int T) { return decode_ws(w, T).total; }
 
 size_t decode_stack_status_offset() { return sizeof(unsigned); }
 
-// Split of the shared-memory pool between the ring and the input stage for
-// calls of T tokens on layers shaped like w; false if the shape does not fit.
-static bool decode_layout(const moe_layer_w &w, int T, int grid, int *nslots, int *stage_floats) {
-    const long th = (long)T * w.H, tdn = (long)T * dec::kTaskGroups * 64;
-    long stage = th > tdn ? th : tdn;
-    if (stage > dec::kStageFloats || stage / 32 > dec::kMaxXs) return false;
-    stage = (stage + 31) & ~31L;  // keep the stage 128-byte aligned
-    long ns = (dec::kPoolBytes - stage * 4) / dec::kSlotBytes;
-    if (ns > dec::kMaxStages) ns = dec::kMaxStages;
-    const long ring = ns * dec::kSlotBytes;
-    const long rows = grid > 0 ? (w.E + grid - 1) / grid : w.E;
-    const long rcopy = 2L * w.H + rows * w.H + 2 * (rows * (w.H / 64) * 2 + 32);
-    const long topk_keys = (long)T * w.E * 8 + 16 + (long)T * (w.E + 28) * 4;  // keys and padded high words
-    if (ns < 3 || topk_keys > ring || rcopy > ring || grid <= 0) return false;
-    // task tables of the busiest CTA, for the most distinct experts a call can route to
-    const long pairs = (long)T * w.k < w.E ? (long)T * w.k : w.E;
-    const long pg = (w.H / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    const long j2 = w.Is / 32 + pairs * (w.I / 32);
-    const long ndp_r = (w.I / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    const long ndp_s = (w.Is / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    const long rbh = w.H / 32, j3 = (ndp_s + pairs * ndp_r) * rbh;
-    const long gu_tasks = (j2 * 2 * pg + grid - 1) / grid, dn_tasks = (j3 + grid - 1) / grid;
-    if (pg > dec::kMaxPG || gu_tasks > dec::kMaxTasks || dn_tasks > dec::kMaxTasks ||
-        (dn_tasks + rbh - 1) / rbh + 1 > dec::kMaxSegs)
-        return false;
-    *nslots = (int)ns;
-    *stage_floats = (int)((dec::kPoolBytes - ring) / 4);
-    return true;
-}
-
-bool decode_stack_fits(const moe_layer_w *w, int T, int grid) {
-    int a, b;
-    return decode_layout(*w, T, grid, &a, &b);
+bool decode_stack_fits(const moe_layer_w *w, int T, int grid, int force_path) {
+    dec::Cfg P{};
+    size_t smem = 0;
+    return decode_plan(*w, T, grid, use_mma(T, force_path), P, &smem);
 }
 
 int decode_stack_max_tokens() { return dec::kMaxT; }
 int decode_stack_max_layers() { return dec::kMaxLayers; }
-int decode_stack_stage_floats() { return dec::kStageFloats; }
+int decode_stack_stage_floats() { return dec::kMaxStageTH; }
 
 cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t *h_in, int chained,
                                 uint16_t *h_out, int T, void *ws, const moe_opts &o, int grid, cudaStream_t st) {
@@ -1480,67 +1900,63 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     const DecodeWs d = decode_ws(&w, T);
     dec::Params Pk;  // ~10 KiB, passed by value (kernel parameters up to 32 KiB)
     dec::Cfg &P = Pk.c;
+    std::memset(&P, 0, sizeof P);
+    size_t smem = 0;
+    const bool mma = use_mma(T, o.force_path);
+    if (!decode_plan(w, T, grid, mma, P, &smem)) return cudaErrorInvalidValue;
     for (int l = 0; l < L; ++l) Pk.layers[l] = layers[l];
     P.h_in = h_in;
     P.h_out = h_out;
     P.L = L;
-    P.T = T;
     P.chained = chained;
     P.post_norm = o.post_norm;
     P.layer_scalar = o.layer_scalar;
     P.eps = o.eps;
-    P.H = w.H;
-    P.E = w.E;
-    P.k = w.k;
-    P.I = w.I;
-    P.Is = w.Is;
-    P.Kmax = w.I > w.Is ? w.I : w.Is;
-    P.R = T + T * w.k;
-    P.ndp_r = (w.I / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    P.ndp_s = (w.Is / 64 + dec::kTaskGroups - 1) / dec::kTaskGroups;
-    if (!decode_layout(w, T, grid, &P.nslots, &P.stage_floats)) return cudaErrorInvalidValue;
     char *base = static_cast<char *>(ws);
-    P.bar = reinterpret_cast<unsigned *>(base + d.bar);
-    // test hook: MOE_TEST_BARRIER_EXTRA=1 makes the first grid barrier wait for an
-    // arrival that never comes, so that its bounded wait runs out (about 1 s) and
-    // the kernel reports "grid barrier timed out" through the workspace status
+    P.bar = reinterpret_cast<unsigned *>(base + d.ctl);
+    // test hook: MOE_TEST_BARRIER_EXTRA=1 makes the grid barriers wait for one
+    // arrival more than the grid has, so that the first one's bounded wait runs
+    // out (about 1 s) and the kernel reports "grid barrier timed out" through
+    // the workspace status
     const char *extra = getenv("MOE_TEST_BARRIER_EXTRA");
     P.bar_extra = (extra && extra[0] == '1') ? 1u : 0u;
-    P.err = reinterpret_cast<int *>(base + d.bar + sizeof(unsigned));
-    P.logits = reinterpret_cast<double *>(base + d.logits);
-    P.cnt_dn = reinterpret_cast<unsigned *>(base + d.cnt_dn);
-    P.cnt_gu = reinterpret_cast<unsigned *>(base + d.cnt_gu);
-    P.act_done = reinterpret_cast<unsigned *>(base + d.act_done);
-    P.rows_done = P.act_done + (T + T * w.k);
-    P.gpart = reinterpret_cast<float *>(base + d.gpart);
-    P.act = reinterpret_cast<float *>(base + d.act);
-    P.act_cs = reinterpret_cast<float *>(base + d.act_cs);
-    P.y = reinterpret_cast<float *>(base + d.y);
-    P.sh = reinterpret_cast<float *>(base + d.sh);
+    P.err = reinterpret_cast<int *>(base + d.ctl + sizeof(unsigned));
+    P.ready = reinterpret_cast<unsigned *>(base + d.ready);
+    P.logit_ll = reinterpret_cast<unsigned long long *>(base + d.logits);
+    P.a_sh = reinterpret_cast<float *>(base + d.a_sh);
+    P.a_r = reinterpret_cast<float *>(base + d.a_r);
     P.m = reinterpret_cast<float *>(base + d.m);
+    P.maps = reinterpret_cast<const CUtensorMap *>(base + d.maps);
 
-    const size_t smem = sizeof(dec::Smem);
-    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(dec::decode_stack_kernel), smem);
+    const void *fn = kernel_for(T, mma);
+    cudaError_t e = ensure_smem(fn, smem);
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(ws, 0, d.zero_bytes, st);
-    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(ws, 0, d.zero_bytes, st)) != cudaSuccess) return e;
+    if ((e = copy_maps(layers, L, P, base + d.maps, st)) != cudaSuccess) return e;
     void *args[] = {&Pk};
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(dec::decode_stack_kernel), dim3(grid),
-                                    dim3(dec::kThreads), args, smem, st);
-    return e;
+    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(dec::kThreads), args, smem, st);
 }
 
 cudaError_t decode_stack_grid(int device, int *grid) {
     int sms = 0, per = 0;
     cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
     if (e != cudaSuccess) return e;
-    e = ensure_smem(reinterpret_cast<const void *>(dec::decode_stack_kernel), sizeof(dec::Smem));
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, dec::decode_stack_kernel, dec::kThreads,
-                                                      sizeof(dec::Smem));
-    if (e != cudaSuccess) return e;
-    *grid = per >= 1 ? sms : 0;
+    // the largest plan any launch may use: one CTA per SM must fit
+    const size_t smem = 227 * 1024;
+    const void *fns[5] = {kernel_ptr<1, false>(), kernel_ptr<2, false>(), kernel_ptr<4, false>(), kernel_ptr<8, false>(),
+                          kernel_ptr<8, true>()};
+    for (const void *fn : fns) {
+        if ((e = ensure_smem(fn, smem)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, dec::kThreads, smem)) != cudaSuccess) return e;
+        if (per < 1) {
+            *grid = 0;
+            return cudaSuccess;
+        }
+    }
+    *grid = sms;
     return cudaSuccess;
 }
+
+size_t decode_stack_smem() { return 227 * 1024; }
 
 }  // namespace moe

@@ -66,12 +66,21 @@ cudaError_t launch_combine(const float *y, const float *sh, const float *wts, in
 cudaError_t launch_ep_select(const int32_t *idx, const float *wts, const int32_t *active, int n, int e_lo, int e_hi,
                              float *wts_out, int32_t *active_out, cudaStream_t st);
 
+// Tiered expert residency (moe_cache.cu).
+cudaError_t launch_residency(const int32_t *idx, int n, int E, int C, int32_t *slot_of, int32_t *expert_of,
+                             uint32_t *uses, uint32_t *last, uint32_t *ctl, int32_t *miss, int32_t *idx_c,
+                             cudaStream_t st);
+cudaError_t launch_fill(const moe_layer_w *w, const moe_qmat pool[3], const moe_qmat cache[3], const int32_t *miss,
+                        cudaStream_t st);
+cudaError_t launch_cache_reset(int E, int C, int32_t *slot_of, int32_t *expert_of, uint32_t *uses, uint32_t *last,
+                               uint32_t *ctl, cudaStream_t st);
+
 // Persistent decode kernel over a stack of layers (moe_decode.cu).
 size_t decode_stack_smem();
 size_t decode_stack_ws_bytes(const moe_layer_w *w, int T);
 size_t decode_stack_status_offset();
 int decode_stack_max_tokens();
-bool decode_stack_fits(const moe_layer_w *w, int T, int grid);
+bool decode_stack_fits(const moe_layer_w *w, int T, int grid, int force_path);
 int decode_stack_max_layers();
 int decode_stack_stage_floats();
 cudaError_t decode_stack_grid(int device, int *grid);

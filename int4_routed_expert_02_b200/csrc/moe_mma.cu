@@ -69,6 +69,7 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -114,7 +115,7 @@ struct Lay {
     static constexpr int kBOff = 0;
     static constexpr int kCodeOff = kBOff + kBBufs * kBBufBytes;
     static constexpr int kBarOff = kCodeOff + kCodeSlots * kSlotBytes;
-    static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 5;
+    static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 6;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kTmemSlotOff + 16;
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
@@ -138,6 +139,7 @@ struct Params {
     int H;
     int *err;        // bounded-wait timeouts (every wait polls it and stops)
     int *range_err;  // a weight or SwiGLU value outside the FP16 range (no wait polls it)
+    int test_stall;  // tests of the timeout path: the epilogue first waits on a barrier nothing arrives at
 };
 
 // TMA tensor maps of one launch: the token matrix (B operand) and the tiled
@@ -411,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
     auto acc_full = [&](int i) { return bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + i); };
     auto acc_empty = [&](int i) { return bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 2 + i); };
     const uint32_t drain = bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 4);
+    const uint32_t stall = bars + 8u * (2 * kCodeSlots + 2 * kABufs + 2 * kBBufs + 5);  // never arrived at
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::kTmemSlotOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -432,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
             mbar_init(acc_empty(i), kEpiWarps);
         }
         mbar_init(drain, 1);
+        mbar_init(stall, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kMmaWarp) {
@@ -645,7 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
         // warp w reads TMEM lanes 32*(w%4).. (tile rows); tiles in order, buffers alternating
         const int q4 = warp & 3;
         uint32_t ic = 0;
-        for (int it = blockIdx.x; it < P.n_items; it += gridDim.x) {
+        // test hook: a wait that runs out (about 1 s); every role then stops as on a real timeout
+        const bool stalled =
+            P.test_stall && !__all_sync(0xffffffffu, mbar_wait(stall, 0, P.err, kErrAccFull));
+        for (int it = stalled ? P.n_items : (int)blockIdx.x; it < P.n_items; it += gridDim.x) {
             Tile t;
             if (!get_tile(P, it, t)) continue;
             const int ab = (int)(ic & 1u);
@@ -849,6 +856,10 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
     P.H = H;
     P.err = b.err;
     P.range_err = b.range_err;
+    // test hook: MOE_TEST_MMA_STALL=1 makes the epilogue's first wait run out, so that the
+    // kernels' bounded waits and their report through the workspace status are exercised
+    const char *stall_env = getenv("MOE_TEST_MMA_STALL");
+    P.test_stall = (stall_env && stall_env[0] == '1') ? 1 : 0;
     const long long pairs = (long long)T * k;
     const int max_active = (int)(pairs < w->E ? pairs : w->E);
 

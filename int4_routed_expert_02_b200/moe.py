@@ -24,7 +24,8 @@ EXPORTED = ("moe_last_error", "moe_version", "moe_prepare_qmat", "moe_workspace_
             "moe_router_topk", "moe_router", "moe_bucket", "moe_expert_ffn", "moe_layer_forward",
             "moe_noalloc_scratch_bytes", "moe_layer_forward_noalloc", "moe_decode_stack_workspace_size",
             "moe_decode_stack", "moe_decode_stack_status", "moe_workspace_status", "moe_qmat_gemv_workspace_size",
-            "moe_qmat_gemv", "moe_noalloc_status", "moe_decode_stack_fits", "moe_layer_partial", "moe_combine")
+            "moe_qmat_gemv", "moe_noalloc_status", "moe_decode_stack_fits", "moe_layer_partial", "moe_combine",
+            "moe_expert_cache_reset", "moe_layer_forward_cached")
 
 
 class MoEError(RuntimeError):
@@ -43,6 +44,13 @@ class LayerW(C.Structure):
                 ("router_scale", C.c_void_p), ("per_expert_scale", C.c_void_p),
                 ("gate", QMat), ("up", QMat), ("down", QMat),
                 ("sh_gate", QMat), ("sh_up", QMat), ("sh_down", QMat)]
+
+
+class ExpertCache(C.Structure):
+    _fields_ = [("slots", C.c_int), ("gate", QMat), ("up", QMat), ("down", QMat),
+                ("pool_gate", QMat), ("pool_up", QMat), ("pool_down", QMat),
+                ("slot_of", C.c_void_p), ("expert_of", C.c_void_p), ("uses", C.c_void_p), ("last", C.c_void_p),
+                ("ctl", C.c_void_p)]
 
 
 class Opts(C.Structure):
@@ -69,6 +77,8 @@ _lib.moe_decode_stack_status.argtypes = [_P]
 _lib.moe_decode_stack_fits.argtypes = [_P, _I, _P]
 _lib.moe_layer_partial.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, C.c_size_t, _P, _P]
 _lib.moe_combine.argtypes = [_P, _P, _P, _I, _I, _P, _P]
+_lib.moe_expert_cache_reset.argtypes = [_P, _I, _P]
+_lib.moe_layer_forward_cached.argtypes = [_P, _P, _P, _P, _I, _P, C.c_size_t, _P, _P]
 _lib.moe_workspace_status.argtypes = [_P]
 _lib.moe_layer_forward_noalloc.argtypes = [_P, _P, _P, _I, _P, _P]
 _lib.moe_noalloc_status.argtypes = [_P]
@@ -268,6 +278,18 @@ def moe_combine(h_in, m, h_out, T, H, opts=None, stream=None):
     """h_out = bf16((h_in + rmsnorm_no_scale(m)) * layer_scalar)."""
     o = opts if opts is not None else _opts()
     _check(_lib.moe_combine(_ptr(h_in), _ptr(m), _ptr(h_out), T, H, C.byref(o), _stream(stream)))
+
+
+def moe_expert_cache_reset(cache, E, stream=None):
+    _check(_lib.moe_expert_cache_reset(C.addressof(cache), E, _stream(stream)))
+
+
+def moe_layer_forward_cached(layer, cache, h_in, h_out, T, ws, opts=None, stream=None):
+    """moe_layer_forward with the routed experts served from a device cache
+    filled from a host pool (see moe_layer_forward_cached in the header)."""
+    o = opts if opts is not None else _opts()
+    _check(_lib.moe_layer_forward_cached(layer.ptr(), C.addressof(cache), _ptr(h_in), _ptr(h_out), T, _ptr(ws),
+                                         ws.numel() if ws is not None else 0, C.byref(o), _stream(stream)))
 
 
 def moe_decode_stack_fits(layer, T, stream=None) -> bool:

@@ -18,7 +18,7 @@ from . import moe, synth
 class MoEStack:
     def __init__(self, cfg: synth.MoEConfig, cfg_id: int, T: int | None = None, layers: int | None = None,
                  seed: int = 0, device="cuda", keep_router_codes: bool = False, persistent: bool | None = None,
-                 device_layers: list | None = None):
+                 device_layers: list | None = None, opts=None):
         """device_layers: the weights of another stack of the same configuration
         to share (they are not regenerated)."""
         self.cfg, self.cfg_id, self.seed = cfg, cfg_id, seed
@@ -63,7 +63,7 @@ class MoEStack:
             self.inputs = [self.inp[l] for l in range(self.L)]
             self.outputs = [self.out[l] for l in range(self.L)]
         self.ws = moe.workspace(self.layers[0], self.T, device=self.device)  # per-layer calls
-        self.opts = moe.make_opts()
+        self.opts = opts if opts is not None else moe.make_opts()
         self.graph = None
 
     def weight_bytes(self) -> int:

@@ -36,10 +36,13 @@ def _check_stack(st, cfg, cfg_id, oracle_layers=(0,), tol=OUT_TOL):
         assert err <= tol, f"layer {l}: {err:.3e} vs the oracle"
 
 
-@pytest.mark.parametrize("cfg_id,T,L", [(0, 4, 3), (0, 1, 2), (1, 1, 4), (1, 8, 2), (2, 4, 3), (2, 8, 2)])
-def test_decode_stack_matches_per_layer_path_and_oracle(cfg_id, T, L):
+@pytest.mark.parametrize("cfg_id,T,L,path", [(0, 4, 3, 0), (0, 1, 2, 0), (1, 1, 4, 0), (1, 8, 2, 0), (2, 4, 3, 0),
+                                              (2, 8, 2, 0), (0, 4, 2, 1), (1, 1, 3, 2), (2, 2, 2, 1), (2, 3, 2, 2)])
+def test_decode_stack_matches_per_layer_path_and_oracle(cfg_id, T, L, path):
+    """path 0: automatic (CUDA-core FMAs for T = 1, tensor cores for T >= 2);
+    1 and 2 force the CUDA-core and the tensor-core variants."""
     cfg = synth.CONFIGS[cfg_id]
-    st = MoEStack(cfg, cfg_id, T=T, layers=L)
+    st = MoEStack(cfg, cfg_id, T=T, layers=L, opts=moe.make_opts(force_path=path))
     assert st.persistent
     for step in range(2):   # second call reuses the workspace and the ring state
         st.set_input(synth.gen_hidden(cfg, cfg_id, 500 + step, T).cuda())

@@ -167,3 +167,28 @@ def test_prefill_rows_of_eight_chunks_in_one_call():
     torch.cuda.synchronize()
     moe.moe_workspace_status(ws128)
     assert max_err_vs_rms(bf16_host(out), bf16_host(chunked)) <= 5e-3
+
+
+def test_grouped_gemm_wait_timeout_is_reported_and_the_next_call_is_fine(monkeypatch):
+    """A test hook makes the epilogue's first wait run out (about 1 s): every
+    role of both grouped-GEMM kernels stops as on a real timeout, the status
+    call reports MOE_EDEVICE, and the next call on the same context is right."""
+    cfg = synth.CONFIGS[0]
+    T = 32
+    w, D, OL = _layer(cfg, 0)
+    h = hidden_with_gap(cfg, 0, OL, 6, T)
+    hd = h.cuda()
+    out = torch.empty_like(hd)
+    ws = moe.workspace(D, T)
+    monkeypatch.setenv("MOE_TEST_MMA_STALL", "1")
+    moe.moe_layer_forward(D, hd, out, T, ws, moe.make_opts(force_path=MMA))
+    torch.cuda.synchronize()
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_workspace_status(ws)
+    assert ei.value.code == moe.MOE_EDEVICE and "timed out" in str(ei.value)
+    monkeypatch.delenv("MOE_TEST_MMA_STALL")
+    moe.moe_layer_forward(D, hd, out, T, ws, moe.make_opts(force_path=MMA))
+    torch.cuda.synchronize()
+    moe.moe_workspace_status(ws)
+    ref = oracle.layer_forward(OL, h)
+    assert max_err_vs_rms(bf16_host(out), ref["out_f64"]) <= OUT_TOL

@@ -161,3 +161,35 @@ def test_qmat_gemv_validation():
     assert call(64, 64, 1, x=FAKE + 2) == moe.MOE_EALIGN
     assert call(64, 64, 1, y=None) == moe.MOE_EINVAL
     assert call(64, 64, 1, wsb=ws - 1) == moe.MOE_EWORKSPACE
+
+
+def test_new_entry_points_reject_bad_arguments_before_any_launch():
+    st = fake_layer()
+    lib = moe.lib()
+    o = moe.make_opts()
+    # expert-parallel part: an empty or reversed expert range, an out-of-range end
+    for lo, hi in ((3, 2), (-1, 4), (0, 17)):
+        rc = lib.moe_layer_partial(C.addressof(st), FAKE, 4, lo, hi, 1, FAKE * 2, FAKE * 8, 1 << 40, C.byref(o), None)
+        assert rc == moe.MOE_EINVAL and "expert range" in moe.last_error()
+    # combine: hidden size not a multiple of 64, a null pointer, T = 0 enqueues nothing
+    assert lib.moe_combine(FAKE, FAKE * 2, FAKE * 4, 4, 100, C.byref(o), None) == moe.MOE_EINVAL
+    assert lib.moe_combine(None, FAKE * 2, FAKE * 4, 4, 256, C.byref(o), None) == moe.MOE_EINVAL
+    assert lib.moe_combine(FAKE, FAKE * 2, FAKE * 4, 0, 256, C.byref(o), None) == moe.MOE_OK
+    # expert cache: no slots; fewer slots than one call can select (T=4, k=4 -> 16 of E=16)
+    c = moe.ExpertCache(slots=0)
+    assert lib.moe_expert_cache_reset(C.addressof(c), 16, None) == moe.MOE_EINVAL
+    c = moe.ExpertCache(slots=8)
+    for n in ("gate", "up", "down", "pool_gate", "pool_up", "pool_down"):
+        setattr(c, n, moe.QMat(FAKE, FAKE))
+    c.slot_of = c.expert_of = c.uses = c.last = c.ctl = FAKE
+    rc = lib.moe_layer_forward_cached(C.addressof(st), C.addressof(c), FAKE, FAKE * 4, 4, FAKE * 8, 1 << 40,
+                                      C.byref(o), None)
+    assert rc == moe.MOE_EINVAL and "slots" in moe.last_error()
+    # T = 1 selects 4 experts: 8 slots pass the size check, and a null pool pointer is then caught
+    c.pool_down = moe.QMat(None, FAKE)
+    rc = lib.moe_layer_forward_cached(C.addressof(st), C.addressof(c), FAKE, FAKE * 4, 1, FAKE * 8, 1 << 40,
+                                      C.byref(o), None)
+    assert rc == moe.MOE_EINVAL
+    # the decode kernel's fit query answers 0 on bad sizes (and without a device)
+    assert lib.moe_decode_stack_fits(C.addressof(st), 9, None) == 0
+    assert lib.moe_decode_stack_fits(C.addressof(fake_layer(H=100)), 1, None) == 0
