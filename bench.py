@@ -180,7 +180,7 @@ def _distinct_experts(st, moe, cfg, T):
     return tot / st.L
 
 
-def _expert_roofline(st, moe, cfg, T, hbm, dev):
+def _expert_roofline(st, moe, cfg, T, hbm, dev, opts=None):
     """Per-launch time of the expert part (moe_expert_ffn: gate/up + down +
     weighted sum) on each layer's real input, against the HBM roofline of
     the distinct experts it reads."""
@@ -207,7 +207,7 @@ def _expert_roofline(st, moe, cfg, T, hbm, dev):
             xe, idx, wts, offsets, perm, active = bufs[l]
             a, b = evs[r * L + l]
             a.record(stream)
-            moe.moe_expert_ffn(st.layers[l], xe, T, idx, wts, offsets, perm, active, 1, m, ws2)
+            moe.moe_expert_ffn(st.layers[l], xe, T, idx, wts, offsets, perm, active, 1, m, ws2, opts)
             b.record(stream)
     torch.cuda.synchronize(dev)
     moe.moe_workspace_status(ws2)
@@ -330,18 +330,28 @@ def expert_flops(cfg, T: int) -> float:
     return 2.0 * T * (3.0 * cfg.I * cfg.H * cfg.k + 3.0 * cfg.Is * cfg.H)
 
 
-def prefill_measure(dev, chunks=8, layers=None, T=None, share=None):
+PREFILL_KERNELS = {
+    0: "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
+    2: "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
+    3: "gateup_kernel + down_kernel (weight-stationary warp MMA, exact FP16 codes) + gather + combine",
+}
+
+
+def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0):
     """Chunked prefill at the Gemma shape: `chunks` chunks of T tokens (128),
     each through every layer (chained), chunk after chunk; plus the per-launch
     expert FFN (tensor-core grouped GEMM) against the tensor and HBM peaks.
     With T = 1024, the 8 chunks' rows go through each layer in
     one call, so every expert's weights are read once for ~64 rows.  `share`:
-    a stack whose weights to reuse.  Returns (result, stack)."""
+    a stack whose weights to reuse; `force_path` the expert path (0 automatic).
+    Returns (result, stack)."""
     from int4_routed_expert_02_b200 import moe
     from int4_routed_expert_02_b200.stack import MoEStack
     cfg = synth.CONFIGS[4]
     T = cfg.T if T is None else T
-    st = MoEStack(cfg, 4, T=T, layers=layers, device=dev, device_layers=None if share is None else share.layers)
+    opts = moe.make_opts(force_path=force_path)
+    st = MoEStack(cfg, 4, T=T, layers=layers, device=dev, device_layers=None if share is None else share.layers,
+                  opts=opts)
     inputs = [synth.gen_hidden(cfg, 4, 20_000 + c, T, device=dev) for c in range(chunks + 1)]
     stream = torch.cuda.current_stream(dev)
     st.set_input(inputs[0])
@@ -357,18 +367,20 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None):
     ms = e0.elapsed_time(e1)
     st.status()
     hbm = peaks()
-    roof = _expert_roofline(st, moe, cfg, T, hbm, dev)
+    roof = _expert_roofline(st, moe, cfg, T, hbm, dev, opts)
     fl = expert_flops(cfg, T)
     tflops = fl / (roof["us_per_launch"] / 1e6) / 1e12
     peak_t = hbm["bf16_tflops"]  # FP16 and BF16 share the dense tensor rate
     fused = T != cfg.T
-    traffic = PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER if fused else PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK
+    traffic = (PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER if fused else PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK) \
+        if force_path in (0, 2) else None
     name = (workload_name(cfg, T) + ", the rows of 8 chunks of 128 through each layer in one call") if fused else \
         (workload_name(cfg, T) + f", {chunks} chunks chunk-major")
     bound_us = max(roof["bytes_per_launch"] / (hbm["hbm_gbs"] * 1e3), fl / (peak_t * 1e6))
     return {"workload": name, "tok_s": round(chunks * T / (ms / 1e3), 1),
             "ms_per_chunk": round(ms / chunks, 4),
-            "expert_ffn": {"kernel": "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
+            "force_path": force_path,
+            "expert_ffn": {"kernel": PREFILL_KERNELS[force_path],
                            "us_per_launch": roof["us_per_launch"], "flops_per_launch": fl,
                            "tflops": round(tflops, 2), "tensor_peak_tflops": peak_t,
                            "tensor_frac": round(tflops / peak_t, 4), "hbm_gbs": roof["achieved"],
@@ -647,6 +659,8 @@ def run_ours(args, rank, world, local_rank):
     prefill, pst = prefill_measure(dev)
     res["prefill"] = prefill
     res["prefill_fused"], _ = prefill_measure(dev, chunks=2, T=1024, share=pst)
+    res["prefill_ws"], _ = prefill_measure(dev, share=pst, force_path=3)
+    res["prefill_fused_ws"], _ = prefill_measure(dev, chunks=2, T=1024, share=pst, force_path=3)
     r64, s64 = decode_measure(4, 64, 32, W, dev, cpu_budget=args.sub_cpu_budget, share=pst)
     r64["workload"] += " (64-token decode batches on the Gemma shape)"
     res["prefill_batch64"] = r64

@@ -99,7 +99,8 @@ typedef struct {
     float layer_scalar; /* default 1.0 */
     float eps;          /* default 1e-6, inside every RMS */
     int force_path;     /* 0 auto (tensor-core grouped GEMM from T >= 32 on, else dequant-GEMV),
-                           1 CUDA-core dequant-GEMV, 2 tensor-core (tcgen05) grouped GEMM */
+                           1 CUDA-core dequant-GEMV, 2 tensor-core (tcgen05) grouped GEMM,
+                           3 weight-stationary warp-level MMA (exact codes, FP32 scale/bias) */
 } moe_opts;
 
 /* Text of the last error on this host thread ("" if none). */
@@ -197,6 +198,11 @@ MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets
  * range is not computed approximately: the kernel records MOE_EDEVICE
  * ("outside the FP16 range") in the workspace status word (read it with
  * moe_workspace_status) and its outputs are invalid; use force_path 1 there.
+ * force_path 3 runs the experts on the warp-level tensor cores with every
+ * weight read once per group of 8 (gate/up) or 16 (down) tokens of an expert:
+ * codes enter as exact FP16 values, scale and bias stay FP32, so only the
+ * token rows and SwiGLU outputs are FP16 (a SwiGLU value beyond 65504 is
+ * reported as above; weights have no range limit).  E <= 1024.
  */
 MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *idx, const float *wts,
                    const int32_t *offsets, const int32_t *perm, const int32_t *active, int with_shared,
@@ -303,8 +309,9 @@ MOE_API int moe_combine(const uint16_t *h_in, const float *m, uint16_t *h_out, i
  * opts->force_path picks how the experts' dot products run: 1 CUDA-core FMAs
  * (exact products, fp32 sums), 2 the warp-level tensor cores (BF16 operands:
  * codes as exact 128 + q, expert inputs as BF16 -- exact for gate/up, a
- * high + low pair for down -- fp32 accumulation), 0 automatic: CUDA cores for
- * T = 1, tensor cores for T >= 2 (the FMA work grows with T, the MMA's does not).
+ * high + low pair for down -- fp32 accumulation; 3 means the same here), 0
+ * automatic: CUDA cores for T = 1, tensor cores for T >= 2 (the FMA work grows
+ * with T, the MMA's does not).
  * The first call with a given layer array encodes TMA descriptors on the host
  * (cached), and every call copies them into the workspace before the kernel.
  * The workspace (moe_decode_stack_workspace_size) must stay untouched until

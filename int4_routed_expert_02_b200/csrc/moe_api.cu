@@ -172,25 +172,33 @@ moe_opts resolve_opts(const moe_opts *o) {
 }
 
 int check_opts(const char *fn, const moe_opts &o) {
-    if (o.force_path < 0 || o.force_path > 2)
-        return fail(MOE_EINVAL, "%s: force_path=%d (0 auto, 1 dequant-GEMV, 2 tensor-core GEMM)", fn, o.force_path);
+    if (o.force_path < 0 || o.force_path > 3)
+        return fail(MOE_EINVAL, "%s: force_path=%d (0 auto, 1 dequant-GEMV, 2 tcgen05 grouped GEMM, 3 warp-MMA "
+                    "weight-stationary)", fn, o.force_path);
     if (!(o.eps >= 0.0f)) return fail(MOE_EINVAL, "%s: eps must be >= 0", fn);
     return MOE_OK;
 }
 
-bool use_mma(const moe_opts &o, int T) { return o.force_path == 2 || (o.force_path == 0 && T >= kMmaMinT); }
+enum Path { kPathGemv = 1, kPathTc = 2, kPathWs = 3 };
+
+Path expert_path(const moe_opts &o, int T) {
+    if (o.force_path != 0) return static_cast<Path>(o.force_path);
+    return T >= kMmaMinT ? kPathTc : kPathGemv;
+}
 
 // Expert part of a call: the SwiGLU FFNs of the routed and shared experts into
 // y / sh, by the tensor-core grouped GEMM or the CUDA-core dequant-GEMV.
 cudaError_t run_experts(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets, const int32_t *perm,
                         const int32_t *active, int with_shared, void *ws, const WsLayout &L, const moe_opts &o,
                         cudaStream_t st) {
-    if (use_mma(o, T)) {
+    const Path path = expert_path(o, T);
+    if (path != kPathGemv) {
         int *err = at<int>(ws, L.status + kStatusOffset);
         cudaError_t e = cudaMemsetAsync(err, 0, 2 * sizeof(int), st);  // timeout word, FP16-range word
         if (e != cudaSuccess) return e;
         moe::MmaBuffers b{at<uint16_t>(ws, L.xg), at<uint16_t>(ws, L.act), at<float>(ws, L.y), at<float>(ws, L.sh), err,
                           err + 1};
+        if (path == kPathWs) return moe::launch_expert_wsmma(w, xe, T, offsets, perm, active, with_shared, b, st);
         return moe::launch_expert_mma(w, xe, T, offsets, perm, active, with_shared, b, st);
     }
     moe::FfnBuffers b{at<float>(ws, L.a_routed), at<float>(ws, L.a_shared), at<float>(ws, L.y), at<float>(ws, L.sh)};
@@ -621,8 +629,8 @@ int moe_workspace_status(const void *ws) {
     }
     if (code[1] != 0)
         return fail(MOE_EDEVICE, "%s: %s outside the FP16 range of the tensor-core path; outputs are invalid "
-                    "(force_path 1 computes this layer)", fn,
-                    code[1] == 1 ? "a weight s*q + b" : "a SwiGLU value silu(g)*u");
+                    "(%s)", fn, code[1] == 1 ? "a weight s*q + b" : "a SwiGLU value silu(g)*u",
+                    code[1] == 1 ? "force_path 1 or 3 computes this layer" : "force_path 1 computes this layer");
     return MOE_OK;
 }
 

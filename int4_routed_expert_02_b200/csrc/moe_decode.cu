@@ -271,9 +271,9 @@ __device__ __noinline__ bool grid_wait(const Cfg &P, Shared &S, unsigned nth) {
         bool ok = true;
         for (unsigned it = 0;; ++it) {
             unsigned v = lane < kBarCtrs ? ld_acquire(P.bar + 32 * lane) : 0u;
-            v += __shfl_xor_sync(0xffffffffu, v, 1);
-            v += __shfl_xor_sync(0xffffffffu, v, 2);
-            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            // the full butterfly: every lane holds the same sum, so all lanes leave the loop together
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             if (v >= target) break;
             if ((it & 63u) == 63u) {
                 int bad = 0;
@@ -375,7 +375,9 @@ __device__ __noinline__ bool wait_task(Shared &S, const Cfg &P, unsigned seq) {
         }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    return ok && mbar_wait(&S.full[s], ph, P.err, kErrFull);
+    // each lane waits for the bytes itself (its own acquire of the copies); the verdict is the warp's
+    const int got = ok && mbar_wait(&S.full[s], ph, P.err, kErrFull);
+    return __all_sync(0xffffffffu, got) != 0;
 }
 
 // ------------------------------------------------------------------ phases
@@ -1626,10 +1628,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         S.verdict = 1;
     }
     __syncthreads();
-    if ((threadIdx.x >> 5) == kProdWarp)
-        producer_main(Pk, S, base);
-    else
+    if ((threadIdx.x >> 5) == kProdWarp) {
+        producer_main(Pk, S, base);  // lane 0 works, the other lanes return at once
+        __syncwarp();
+    } else {
         consumer_main<NT, MMA>(Pk, S, base);
+    }
     __syncthreads();
 }
 
@@ -1868,7 +1872,7 @@ const void *kernel_ptr() {
 
 // The tensor-core variants for T >= 2 (the CUDA cores' FMA work grows with T,
 // the MMA's does not), the CUDA-core FMAs for one token; force_path overrides.
-bool use_mma(int T, int force_path) { return force_path == 2 || (force_path == 0 && T >= 2); }
+bool use_mma(int T, int force_path) { return force_path >= 2 || (force_path == 0 && T >= 2); }
 
 const void *kernel_for(int T, bool mma) {
     if (mma) return kernel_ptr<8, true>();

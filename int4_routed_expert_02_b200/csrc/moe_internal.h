@@ -52,6 +52,14 @@ struct MmaBuffers {
     int *range_err; // device word (0 = ok): a weight or SwiGLU value outside the FP16 range
 };
 size_t mma_xg_bytes(const moe_layer_w *w, int T);
+// FP16 token rows for the tensor-core paths: row r < T token r, row T + j the token of bucketed pair j.
+cudaError_t launch_gather_tokens(const uint16_t *xe, const int32_t *perm, int T, int k, int H, uint16_t *xg,
+                                 cudaStream_t st);
+// Weight-stationary warp-MMA expert FFN (moe_wsmma.cu): same buffers as launch_expert_mma.
+bool wsmma_supported(const moe_layer_w *w);
+cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
+                                const int32_t *perm, const int32_t *active, int with_shared, const MmaBuffers &b,
+                                cudaStream_t st);
 size_t mma_act_bytes(const moe_layer_w *w, int T);
 cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,
                               const int32_t *perm, const int32_t *active, int with_shared, const MmaBuffers &b,

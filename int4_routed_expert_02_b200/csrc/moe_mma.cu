@@ -812,6 +812,17 @@ static cudaError_t launch_mma(Params &P, const Maps &map, int max_items, cudaStr
 
 }  // namespace mma
 
+cudaError_t launch_gather_tokens(const uint16_t *xe, const int32_t *perm, int T, int k, int H, uint16_t *xg,
+                                 cudaStream_t st) {
+    const int R = T + T * k;
+    const long long chunks = (long long)R * (H / 8);
+    long long blocks = (chunks + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    if (blocks <= 0) return cudaSuccess;
+    mma::gather_kernel<<<(int)blocks, 256, 0, st>>>(xe, perm, T, k, H, R, xg);
+    return cudaGetLastError();
+}
+
 size_t mma_xg_bytes(const moe_layer_w *w, int T) {
     return sizeof(uint16_t) * ((size_t)T + (size_t)T * w->k) * w->H;
 }
@@ -828,11 +839,7 @@ cudaError_t launch_expert_mma(const moe_layer_w *w, const uint16_t *xe, int T, c
     const int Kmax = I > Is ? I : Is;
     const int R = T + T * k;
     {
-        const long long chunks = (long long)R * (H / 8);
-        long long blocks = (chunks + 255) / 256;
-        if (blocks > 4096) blocks = 4096;
-        gather_kernel<<<(int)blocks, 256, 0, st>>>(xe, perm, T, k, H, R, b.xg);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_gather_tokens(xe, perm, T, k, H, b.xg, st);
         if (e != cudaSuccess) return e;
     }
     static thread_local Maps mx, ma;  // large; kept off the stack

@@ -23,7 +23,7 @@ if torch.cuda.is_available():
     from int4_routed_expert_02_b200 import moe
 
 
-@pytest.mark.parametrize("cfg_id,T,path", [(0, 4, 0), (0, 64, 2), (1, 33, 0), (2, 8, 1)])
+@pytest.mark.parametrize("cfg_id,T,path", [(0, 4, 0), (0, 64, 2), (1, 33, 0), (2, 8, 1), (1, 40, 3)])
 def test_rank_parts_sum_to_the_layer(cfg_id, T, path):
     cfg = synth.CONFIGS[cfg_id]
     w = synth.gen_layer(cfg, cfg_id, 0, device="cuda")

@@ -30,7 +30,7 @@ def _selected(D, h, T, cfg, ws):
 
 
 @pytest.mark.parametrize("cfg_id,T,slots,path", [(0, 1, 6, 0), (0, 4, 16, 0), (1, 1, 16, 0), (2, 4, 40, 1),
-                                                 (0, 40, 16, 2)])
+                                                 (0, 40, 16, 2), (0, 24, 16, 3)])
 def test_cached_layer_matches_the_resident_layer_and_the_rule(cfg_id, T, slots, path):
     cfg = synth.CONFIGS[cfg_id]
     D = moe.DeviceLayer.from_config(synth.gen_layer(cfg, cfg_id, 0, device="cuda"), cfg)

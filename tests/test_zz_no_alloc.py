@@ -24,7 +24,8 @@ from int4_routed_expert_02_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("cfg_id,T,force_path", [(0, 4, 0), (1, 1, 0), (2, 8, 0), (2, 32, 0), (0, 4, 2)])
+@pytest.mark.parametrize("cfg_id,T,force_path", [(0, 4, 0), (1, 1, 0), (2, 8, 0), (2, 32, 0), (0, 4, 2),
+                                                        (0, 40, 3)])
 def test_noalloc_matches_the_workspace_entry_point(cfg_id, T, force_path):
     from int4_routed_expert_02_b200 import build
     build.build()
