@@ -686,6 +686,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--head-only", action="store_true",
                     help="profiling only: time the output-head GEMV alone and print its object")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="profiling only: the 128-token prefill chunks alone (with --layers, --expert-path)")
+    ap.add_argument("--expert-path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="with --prefill-only: force_path of the expert FFN (0 automatic)")
     ap.add_argument("--headline-only", dest="all_configs", action="store_false",
                     help="only the headline configuration (skip the other configurations of the line)")
     args = ap.parse_args()
@@ -703,6 +707,11 @@ def main():
     try:
         if args.impl == "reference":
             res = run_reference(args, rank, world)
+        elif args.prefill_only:
+            from int4_routed_expert_02_b200 import build
+            build.build()
+            res = {"prefill": prefill_measure(torch.device("cuda", local_rank), chunks=2, layers=args.layers or None,
+                                              force_path=args.expert_path)[0]} if rank == 0 else None
         elif args.head_only:
             from int4_routed_expert_02_b200 import build
             build.build()

@@ -192,10 +192,11 @@ cudaError_t run_experts(const moe_layer_w *w, const uint16_t *xe, int T, const i
                         const int32_t *active, int with_shared, void *ws, const WsLayout &L, const moe_opts &o,
                         cudaStream_t st) {
     const Path path = expert_path(o, T);
+    // the status words describe this call, whatever path it takes: timeout word, FP16-range word
+    int *err = at<int>(ws, L.status + kStatusOffset);
+    cudaError_t e = cudaMemsetAsync(err, 0, 2 * sizeof(int), st);
+    if (e != cudaSuccess) return e;
     if (path != kPathGemv) {
-        int *err = at<int>(ws, L.status + kStatusOffset);
-        cudaError_t e = cudaMemsetAsync(err, 0, 2 * sizeof(int), st);  // timeout word, FP16-range word
-        if (e != cudaSuccess) return e;
         moe::MmaBuffers b{at<uint16_t>(ws, L.xg), at<uint16_t>(ws, L.act), at<float>(ws, L.y), at<float>(ws, L.sh), err,
                           err + 1};
         if (path == kPathWs) return moe::launch_expert_wsmma(w, xe, T, offsets, perm, active, with_shared, b, st);

@@ -117,7 +117,7 @@ def test_ws_dense_mixture_with_and_without_shared_expert():
     dict(H=320, E=24, k=5, I=192, Is=320, T=33),      # 5 and 3 groups of K, 6 and 10 row blocks
     dict(H=256, E=8, k=8, I=128, Is=192, T=130),      # every expert holds 130 tokens: 17 / 9 token groups
     dict(H=512, E=16, k=2, I=256, Is=128, T=300),     # the shared expert over 38 / 19 token groups
-    dict(H=1024, E=4, k=1, I=1088, Is=64, T=9),       # 17 groups of K in down: warps take 3 or 2
+    dict(H=1024, E=8, k=1, I=1088, Is=64, T=9),       # 17 groups of K in down: warps take 3 or 2
 ])
 def test_ws_edge_shapes(dims):
     T = dims.pop("T")
@@ -136,13 +136,15 @@ def test_ws_edge_shapes(dims):
 
 
 def test_ws_large_scales_and_weights_beyond_fp16():
-    """Scales |N(0, 0.3)| and one shared-expert group with s = 8192 (weights up
-    to 122880, beyond FP16): the warp-MMA path keeps scale and bias in FP32,
-    so it computes the layer to the bar and reports nothing."""
+    """Scales |N(0, 0.3)| and one group of the shared expert's down matrix
+    with s = 8192, b = -65536 (weights from -65536 to 57344: beyond FP16,
+    which the tcgen05 path reports): the warp-MMA path keeps scale and bias in
+    FP32 and the down output is FP32, so it computes the layer to the bar and
+    reports nothing."""
     cfg = synth.CONFIGS[0]
     w = synth.gen_layer(cfg, 0, 0, device="cuda", expert_scale_std=0.3)
-    w["sh_gate_s"][3, 1] = 8192.0
-    w["sh_gate_b"][3, 1] = 0.0
+    w["sh_down_s"][5, 1] = 8192.0                                  # both exact in bf16
+    w["sh_down_b"][5, 1] = -65536.0
     D = moe.DeviceLayer.from_config(w, cfg)
     OL = oracle_layer(host(w), cfg)
     T = 32
@@ -151,6 +153,12 @@ def test_ws_large_scales_and_weights_beyond_fp16():
     m, _ = _ffn(cfg, D, xe_d, idx, wr, WS)                         # status read: no report
     ref = oracle.expert_ffn(OL, xe, idx, wr.astype(np.float32).astype(np.float64))
     assert max_err_vs_rms(m.cpu().double().numpy(), ref) <= 5e-3
+    rest = [r for r in range(cfg.H) if r != 5]                     # the other rows on their own scale
+    assert max_err_vs_rms(m.cpu().double().numpy()[:, rest], ref[:, rest]) <= 5e-3
+    _, ws = _ffn(cfg, D, xe_d, idx, wr, TC, check=False)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_workspace_status(ws)
+    assert "weight" in str(ei.value)
 
 
 def test_ws_swiglu_outside_fp16_range_is_reported():
