@@ -152,7 +152,9 @@ def test_ws_large_scales_and_weights_beyond_fp16():
     idx, wr, xe, xe_d = _routed(cfg, OL, h)
     m, _ = _ffn(cfg, D, xe_d, idx, wr, WS)                         # status read: no report
     ref = oracle.expert_ffn(OL, xe, idx, wr.astype(np.float32).astype(np.float64))
-    assert max_err_vs_rms(m.cpu().double().numpy(), ref) <= 5e-3
+    # row 5 sums terms up to 65536 * |a| that cancel to a much smaller value, so
+    # the FP16 rounding of the SwiGLU inputs a (2^-12 relative) weighs more there
+    assert max_err_vs_rms(m.cpu().double().numpy(), ref) <= OUT_TOL
     rest = [r for r in range(cfg.H) if r != 5]                     # the other rows on their own scale
     assert max_err_vs_rms(m.cpu().double().numpy()[:, rest], ref[:, rest]) <= 5e-3
     _, ws = _ffn(cfg, D, xe_d, idx, wr, TC, check=False)
