@@ -69,11 +69,12 @@ constexpr int kMaxT = 8;
 constexpr int kMaxLayers = 64;
 constexpr int kMaxPairs = kMaxT * kMaxK;      // 256
 constexpr int kMaxSlots = 16;                 // ring slots
+constexpr int kMaxA = 9;                      // the static region's tasks: router rows + up to 8 shared units
 constexpr int kMaps = 12;                     // TMA tensor maps per layer
 constexpr int kMaxBlk = 4;                    // 8-row output blocks per CTA (H <= 4096 on >= 128 SMs)
 constexpr int kMaxParts = 8;                  // K-parts of a down matrix
 constexpr int kPartChunks = 32;               // at most 32 chunks (1024 columns) per K-part
-constexpr int kBarCtrs = 8;                   // grid-barrier counters, 128 bytes apart
+constexpr int kBarCtrs = 1;                   // grid-barrier counters, 128 bytes apart (one polls fastest)
 constexpr int kMaxStageTH = 24576;            // largest T * H
 constexpr int kMaxCand = 512;                 // top-k candidates per token
 constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
@@ -99,13 +100,15 @@ struct Cfg {
     int nrb8;                    // 8-row blocks of the output rows (H / 8)
     int parts_s, pc_s;           // shared down: K-parts, chunks per part
     int parts_r, pc_r;           // routed down
-    int ns, slot_bytes;          // ring slots and their size
+    int ns, slot_bytes;          // ring slots and their size (routed gate/up units and down groups)
+    int a_rbytes, a_ubytes;      // static region: router part, one shared gate/up unit (1024-aligned)
+    int ua;                      // shared units a CTA keeps in the static region (the rest go through the ring)
     int gcb;                     // bytes of one matrix's codes in a gate/up slot (1024-aligned)
     int sbs;                     // bytes of one matrix's (scale, bias) words in a gate/up slot (128-aligned)
     int dcb_s, dcb_r;            // bytes of one 8-row block's codes in a down slot (1024-aligned)
     int sbd_s, sbd_r;            // bytes of one 8-row block's words in a down slot (128-aligned)
     int maxc;                    // top-k candidate capacity per token
-    int off_ring, off_x, off_xs, off_h, off_y, off_cand, off_part;  // dynamic shared memory offsets
+    int off_a, off_ring, off_x, off_xs, off_h, off_y, off_cand, off_part;  // dynamic shared memory offsets
     int yrows;                   // rows per ybuf entry (8 * kMaxBlk)
     unsigned *bar;               // [kBarCtrs * 32] monotonic arrival counters
     unsigned bar_extra;          // arrivals beyond the grid the barriers wait for (tests of the timeout path)
@@ -130,6 +133,9 @@ struct Shared {
     volatile unsigned owner[kMaxSlots];    // sequence number of the task a slot holds
     int cnt[kMaxSlots];                    // pieces / block tasks of the slot's task that are done
     volatile int astate[kMaxSlots];        // down slot: 0 a not staged, 1 staging, 2 staged
+    unsigned long long afull[kMaxA];       // static region task filled (phase = layer parity)
+    unsigned long long aempty;             // static region consumed (1 + shared units arrivals per layer)
+    int acnt[kMaxA];                       // pieces of a shared unit that are done
     volatile int tables_layer;             // 1 + the layer whose routing tables are ready
     volatile int verdict;                  // consumers: 1 while no error is recorded
     int D;                                 // distinct experts of the current layer
@@ -239,6 +245,11 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         "[%5];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(b))
         : "memory");
+}
+
+// The descriptor of a tensor map into the TMA unit's cache ahead of its first use.
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
 
 // The same box into L2 only.
@@ -377,6 +388,13 @@ __device__ __noinline__ bool wait_task(Shared &S, const Cfg &P, unsigned seq) {
     ok = __shfl_sync(0xffffffffu, ok, 0);
     // each lane waits for the bytes itself (its own acquire of the copies); the verdict is the warp's
     const int got = ok && mbar_wait(&S.full[s], ph, P.err, kErrFull);
+    return __all_sync(0xffffffffu, got) != 0;
+}
+
+// Wait of a whole warp for static-region task i of layer l (router rows: 0,
+// shared units: 1 + u); the verdict is the warp's.
+__device__ __noinline__ bool wait_a(Shared &S, const Cfg &P, int i, int l) {
+    const int got = mbar_wait(&S.afull[i], (unsigned)l & 1u, P.err, kErrFull);
     return __all_sync(0xffffffffu, got) != 0;
 }
 
@@ -546,13 +564,20 @@ __device__ __noinline__ void router_compute(const Cfg &P, Shared &S, const unsig
             for (int c = c0 + lane; c < c1; c += 32) {
                 const uint4 q = reinterpret_cast<const uint4 *>(rows + (size_t)er * H)[c];
                 const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+                // the chunk's 16 inputs and scales as 16-byte loads (bf16 pairs)
+                const uint4 ha = reinterpret_cast<const uint4 *>(h)[2 * c], hb = reinterpret_cast<const uint4 *>(h)[2 * c + 1];
+                const uint4 ra = reinterpret_cast<const uint4 *>(rsc)[2 * c], rb = reinterpret_cast<const uint4 *>(rsc)[2 * c + 1];
+                const uint32_t hw[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+                const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
                 double dots[4] = {0.0, 0.0, 0.0, 0.0}, zss[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
                 for (int wi = 0; wi < 4; ++wi) {
 #pragma unroll
                     for (int bi = 0; bi < 4; ++bi) {
-                        const int i = c * 16 + wi * 4 + bi;
-                        const double z = (double)(bf16_bits_to_float(h[i]) * bf16_bits_to_float(rsc[i]));
+                        const int i = wi * 4 + bi;  // element of the chunk
+                        const uint32_t hbits = (hw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+                        const uint32_t rbits = (rw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+                        const double z = (double)(bf16_bits_to_float(hbits) * bf16_bits_to_float(rbits));
                         const double qd =
                             __hiloint2double(0x43300000, (int)((words[wi] >> (8 * bi)) & 0xffu)) - 4503599627370496.0;
                         dots[bi] = fma(qd, z, dots[bi]);
@@ -885,46 +910,72 @@ struct Cand {
 // K: top-k of every token (ties to the lower expert index; ordered by logit
 // desc, index asc), gate weights softmax(logits[top-k]) * per_expert_scale
 // in fp64, and the bucketing of the T*k pairs by expert (stable by pair id).
-// Every CTA computes the same result from the same logits.
-//   1. candidates: a warp ranks 32 experts of one token among themselves; only
-//      those ranked below k can be in the top k of all E, so the others are
-//      dropped;
-//   2. each candidate's rank among its token's candidates is its rank among
-//      all E logits (everything that beats a top-k logit is a candidate);
-//   3. weights and buckets by counting over the T*k pairs.
+// Every CTA computes the same result from the same logits.  Warp t handles
+// token t alone, with no block-wide barrier until the bucketing:
+//   1. per group of 32 experts, each lane polls one logit and ranks it among
+//      the group by shuffles; only those ranked below k can be in the top k
+//      of all E, and they are appended (ballot order) to the warp's candidate
+//      list (everything that beats a top-k logit is itself a candidate);
+//   2. each candidate's rank among the candidates is its rank among all E;
+//   3. lanes r < k form the softmax weights (one exp per lane);
+// then, over the whole block, the buckets by counting over the T*k pairs.
 __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, const uint16_t *pes, unsigned tag) {
     const int T = P.T, E = P.E, k = P.k, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int nsl = (E + 31) / 32;
-    if (threadIdx.x < T) S.ccount[threadIdx.x] = 0;
-    consumer_sync();
+    if (wid < T) {
+        const int t = wid, nsl = (E + 31) / 32;
+        Cand *cw = cand + (size_t)t * P.maxc;
+        int nc = 0;
+        // the lane's logits in batches of 8 groups (one round trip per batch when they are all there)
+        constexpr int kPoll = 8;
 #pragma unroll 1
-    for (int item = wid; item < T * nsl; item += kCW) {
-        const int t = item / nsl, sl = item - t * nsl, e = sl * 32 + lane;
-        const bool valid = e < E;
-        double v = 0.0;
-        if (valid && !get_logit(P, t, e, tag, v)) v = 0.0;  // an error is recorded; the layer's result is void
-        const unsigned long long key = valid ? logit_key(v) : 0ull;
-        int rank = 0;
+        for (int sb = 0; sb < nsl; sb += kPoll) {
+            unsigned long long w0[kPoll], w1[kPoll];
+#pragma unroll
+            for (int q = 0; q < kPoll; ++q) {
+                const int e = (sb + q) * 32 + lane;
+                w0[q] = w1[q] = 0ull;
+                if (sb + q < nsl && e < E) {
+                    const unsigned long long *w = P.logit_ll + 2 * ((size_t)t * E + e);
+                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w0[q]) : "l"(w) : "memory");
+                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w1[q]) : "l"(w + 1) : "memory");
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < kPoll; ++q) {
+                const int sl = sb + q;
+                if (sl >= nsl) break;
+                const int e = sl * 32 + lane;
+                const bool valid = e < E;
+                double v = 0.0;
+                if (valid) {
+                    if ((unsigned)(w0[q] >> 32) == tag && (unsigned)(w1[q] >> 32) == tag)
+                        v = __longlong_as_double((long long)((w0[q] & 0xffffffffull) | (w1[q] << 32)));
+                    else if (!get_logit(P, t, e, tag, v))
+                        v = 0.0;  // an error is recorded; the layer's result is void
+                }
+                const unsigned long long key = valid ? logit_key(v) : 0ull;
+                int rank = 0;
 #pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-            const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
-            rank += (kj > key) | ((kj == key) & (j < lane));
+                for (int j = 0; j < 32; ++j) {
+                    const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
+                    rank += (kj > key) | ((kj == key) & (j < lane));
+                }
+                const bool cnd = valid && rank < k;
+                const unsigned mask = __ballot_sync(0xffffffffu, cnd);
+                const int pos = nc + __popc(mask & ((1u << lane) - 1u));
+                if (cnd && pos < P.maxc) cw[pos] = Cand{key, e, 0};
+                nc += __popc(mask);
+            }
         }
-        if (valid && rank < k) {
-            const int pos = atomicAdd(&S.ccount[t], 1);
-            if (pos < P.maxc) cand[t * P.maxc + pos] = Cand{key, e, 0};
-        }
-    }
-    consumer_sync();
+        nc = min(nc, P.maxc);
+        __syncwarp();
 #pragma unroll 1
-    for (int i = threadIdx.x; i < T * P.maxc; i += kCThreads) {
-        const int t = i / P.maxc, ci = i - t * P.maxc, nc = min(S.ccount[t], P.maxc);
-        if (ci < nc) {
-            const Cand me = cand[i];
+        for (int ci = lane; ci < nc; ci += 32) {
+            const Cand me = cw[ci];
             int rank = 0;
-#pragma unroll 1
+#pragma unroll 4
             for (int j = 0; j < nc; ++j) {
-                const Cand o = cand[t * P.maxc + j];
+                const Cand o = cw[j];
                 rank += (o.key > me.key) | ((o.key == me.key) & (o.e < me.e));
             }
             if (rank < k) {
@@ -932,17 +983,27 @@ __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, co
                 S.selv[t * k + rank] = key_logit(me.key);
             }
         }
+        __syncwarp();
+        // softmax over the k selected logits (rank 0 holds the largest), times per_expert_scale
+        const double mx = S.selv[t * k];
+        double z = 0.0, ex = 0.0;
+        for (int r = lane; r < k; r += 32) {
+            const double q = exp(S.selv[t * k + r] - mx);
+            if (r == lane) ex = q;
+            z += q;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        for (int r = lane; r < k; r += 32) {
+            const double q = r == lane ? ex : exp(S.selv[t * k + r] - mx);
+            S.wts[t * k + r] = (float)(q / z * (double)bf16_bits_to_float(pes[S.idx[t * k + r]]));
+        }
     }
     consumer_sync();
     const int n = T * k;
 #pragma unroll 1
     for (int p = threadIdx.x; p < n; p += kCThreads) {
         const int t = p / k, e = S.idx[p];
-        const double mx = S.selv[t * k];
-        double z = 0.0;
-#pragma unroll 1
-        for (int s2 = 0; s2 < k; ++s2) z += exp(S.selv[t * k + s2] - mx);
-        S.wts[p] = (float)(exp(S.selv[p] - mx) / z * (double)bf16_bits_to_float(pes[e]));
         int less = 0, eqb = 0, cnt = 0;
 #pragma unroll 1
         for (int q = 0; q < n; ++q) {
@@ -985,22 +1046,39 @@ __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, co
 
 // ------------------------------------------------------------------ work bookkeeping
 
-// A piece of a gate/up unit is done (its a row is stored): the last of the
-// unit's 8 pieces counts the unit done in global memory (release) and frees
-// the ring slot.  Stores of the other pieces are ordered before the count by
-// their fences and the shared-memory count (fence - atomic - atomic - fence).
-__device__ __forceinline__ void piece_done(Shared &S, const Cfg &P, unsigned tseq, unsigned *ready) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) {
-        __threadfence();
-        const int s = (int)(tseq % (unsigned)P.ns);
-        if (atomicAdd(&S.cnt[s], 1) == 7) {
-            S.cnt[s] = 0;
-            __threadfence();
+// CUDA-core path: piece pi (row row0 + pi) of an 8-row gate/up unit is done;
+// every lane holds the row's sums g, u for the n tokens.  The outputs
+// a = silu(g) * u wait in shared memory (`part`: [8][kMaxT]); lane 0 of the
+// warp that completes the unit writes all 8 rows of every token to global
+// memory itself and counts the unit done with one release (its own stores,
+// so no further fence), then frees the buffer.
+constexpr int kFfmaPart = 8 * kMaxT;  // floats of a unit's staging buffer
+template <int NT>
+__device__ __forceinline__ void piece_done_ffma(float *part, int *cnt, unsigned long long *empty, unsigned *ready,
+                                                int pi, int n, const float (&g)[NT], const float (&u)[NT], float *adst,
+                                                const int *ip, int lda, int row0) {
+    const int lane = threadIdx.x & 31;
+    int last = 0;
+    if (lane == 0) {
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt)
+            if (tt < n) part[pi * kMaxT + tt] = silu_mul(g[tt], u[tt]);
+        __threadfence_block();
+        last = atomicAdd(cnt, 1) == 7;
+        if (last) {
+            *cnt = 0;
+            __threadfence_block();
+#pragma unroll 1
+            for (int tt = 0; tt < n; ++tt) {
+                float *dst = adst + (size_t)ip[tt] * lda + row0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dst[q] = part[q * kMaxT + tt];
+            }
             red_release_add(ready, 1u);
-            mbar_arrive(&S.empty[s]);
+            mbar_arrive(empty);
         }
     }
+    __syncwarp();
 }
 
 // A block task of a down group is done: the last of the group's nblk tasks
@@ -1187,14 +1265,13 @@ __device__ __noinline__ bool stage_a_mma(Shared &S, const Cfg &P, int s, bool sh
 // MMA path: a K-piece of a gate/up unit is done (its partial sums are in
 // `part`); true (warp-uniform) for the warp that completes the unit, which
 // then owns the slot's partials.
-__device__ __forceinline__ bool piece_last(Shared &S, const Cfg &P, unsigned tseq, int npc) {
+__device__ __forceinline__ bool piece_last(int *cnt, int npc) {
     __syncwarp();
     int last = 0;
     if ((threadIdx.x & 31) == 0) {
         __threadfence_block();
-        const int s = (int)(tseq % (unsigned)P.ns);
-        last = atomicAdd(&S.cnt[s], 1) == npc - 1;
-        if (last) S.cnt[s] = 0;
+        last = atomicAdd(cnt, 1) == npc - 1;
+        if (last) *cnt = 0;
         __threadfence_block();
     }
     last = __shfl_sync(0xffffffffu, last, 0);
@@ -1202,13 +1279,13 @@ __device__ __forceinline__ bool piece_last(Shared &S, const Cfg &P, unsigned tse
     return last != 0;
 }
 
-// The completing warp of a unit counts it done in global memory (release) and frees its ring slot.
-__device__ __forceinline__ void unit_release(Shared &S, const Cfg &P, unsigned tseq, unsigned *ready) {
+// The completing warp of a unit counts it done in global memory (release) and frees its buffer.
+__device__ __forceinline__ void unit_release(unsigned long long *empty, unsigned *ready) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) {
         __threadfence();
         red_release_add(ready, 1u);
-        mbar_arrive(&S.empty[tseq % (unsigned)P.ns]);
+        mbar_arrive(empty);
     }
 }
 
@@ -1216,22 +1293,23 @@ __device__ __forceinline__ void unit_release(Shared &S, const Cfg &P, unsigned t
 // the warp completing the unit sums the pieces' partials in order and stores
 // a = silu(g) * u for its 8 rows (row0 .. row0 + 7 of `a`, token tt of the
 // list at a + aidx[tt] * lda).
-__device__ __forceinline__ void unit_piece_mma(Shared &S, const Cfg &P, unsigned char *ring, float *part, unsigned tseq,
-                                               int pi, int npc, int n, const int *toks, const int *aidx, float *a,
-                                               int lda, int row0, const unsigned char *xb, const float *xg,
-                                               unsigned *ready) {
+//   slot: the unit's bytes; part: its partial-sum buffer ([kMaxPieces][128] floats); cnt / empty: its
+//   piece counter and the barrier that frees its buffer.
+__device__ __forceinline__ void unit_piece_mma(const Cfg &P, const unsigned char *slot, float *part, int *cnt,
+                                               unsigned long long *empty, int pi, int npc, int n, const int *toks,
+                                               const int *aidx, float *a, int lda, int row0, const unsigned char *xb,
+                                               const float *xg, unsigned *ready) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int s = (int)(tseq % (unsigned)P.ns);
     const int gpp = (P.GH + npc - 1) / npc;
     const int c0 = min(P.CH, 2 * pi * gpp), c1 = min(P.CH, c0 + 2 * gpp);
     float acc[4];
-    g_piece_mma(P, ring + (size_t)s * P.slot_bytes, c0, c1, n, toks, xb, xg, acc);
-    float *mine = part + ((size_t)s * kMaxPieces + pi) * 128 + lane * 4;
+    g_piece_mma(P, slot, c0, c1, n, toks, xb, xg, acc);
+    float *mine = part + (size_t)pi * 128 + lane * 4;
     *reinterpret_cast<float4 *>(mine) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    if (!piece_last(S, P, tseq, npc)) return;
+    if (!piece_last(cnt, npc)) return;
     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int q = 0; q < npc; ++q) {  // fixed order
-        const float4 v = *reinterpret_cast<const float4 *>(part + ((size_t)s * kMaxPieces + q) * 128 + lane * 4);
+        const float4 v = *reinterpret_cast<const float4 *>(part + (size_t)q * 128 + lane * 4);
         sum.x += v.x;
         sum.y += v.y;
         sum.z += v.z;
@@ -1239,7 +1317,7 @@ __device__ __forceinline__ void unit_piece_mma(Shared &S, const Cfg &P, unsigned
     }
     if (2 * t < n) a[(size_t)aidx[2 * t] * lda + row0 + g] = silu_mul(sum.x, sum.z);
     if (2 * t + 1 < n) a[(size_t)aidx[2 * t + 1] * lda + row0 + g] = silu_mul(sum.y, sum.w);
-    unit_release(S, P, tseq, ready);
+    unit_release(empty, ready);
 }
 
 // ------------------------------------------------------------------ consumers
@@ -1251,6 +1329,7 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
     const int T = P.T, H = P.H, G = gridDim.x, c = blockIdx.x, ns = P.ns;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     unsigned char *ring = base + P.off_ring;
+    const unsigned char *abase = base + P.off_a;            // static region: router rows, shared units
     float *x = reinterpret_cast<float *>(base + P.off_x);   // FFMA path: pre-scaled fp32 xe
     unsigned char *xb = base + P.off_x;                    // MMA path: BF16 xe in the MMA order
     float *xs = reinterpret_cast<float *>(base + P.off_xs); // chunk sums (FFMA) or group sums (MMA)
@@ -1277,40 +1356,10 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
             stage_x(P, S, hs, x, xs);
         // ---------------------------------------------------------- R: router rows of this CTA
         {
-            const bool got = wait_task(S, P, seq);
-            router_compute(P, S, ring + (size_t)(seq % (unsigned)ns) * P.slot_bytes, hs, S.rpart, got,
-                           (unsigned)l + 1u);
+            const bool got = wait_a(S, P, 0, l);
+            router_compute(P, S, abase, hs, S.rpart, got, (unsigned)l + 1u);
             consumer_sync();
-            if (threadIdx.x == 0) mbar_arrive(&S.empty[seq % (unsigned)ns]);
-            ++seq;
-        }
-        // ---------------------------------------------------------- S: shared gate/up pieces
-        {
-            const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(cw.nshg, 1) - 1) / max(cw.nshg, 1))) : 8;
-#pragma unroll 1
-            for (int i = wid; i < cw.nshg * npc; i += kCW) {
-                const int ui = i / npc, pi = i - ui * npc;
-                const unsigned tseq = seq + (unsigned)ui;
-                if (!wait_task(S, P, tseq)) break;
-                const int row0 = (c + ui * G) * 8;  // first row of the unit in the shared gate/up matrices
-                if (kMma) {
-                    unit_piece_mma(S, P, ring, part, tseq, pi, npc, T, S.toks_sh, S.toks_sh, P.a_sh, P.Is, row0, xb,
-                                   xs, P.ready);
-                } else {
-                    int tk[NT];
-#pragma unroll
-                    for (int tt = 0; tt < NT; ++tt) tk[tt] = tt < T ? tt : 0;
-                    float g[NT], u[NT];
-                    g_piece<NT>(P, ring + (size_t)(tseq % (unsigned)ns) * P.slot_bytes, pi, T, tk, x, xs, g, u);
-                    if (lane == 0) {
-#pragma unroll
-                        for (int tt = 0; tt < NT; ++tt)
-                            if (tt < T) P.a_sh[(size_t)tt * P.Is + row0 + pi] = silu_mul(g[tt], u[tt]);
-                    }
-                    piece_done(S, P, tseq, P.ready);
-                }
-            }
-            seq += (unsigned)cw.nshg;
+            if (threadIdx.x == 0) mbar_arrive(&S.aempty);
         }
         // ---------------------------------------------------------- K: top-k and buckets
         // (the logits carry the layer's tag: no barrier before reading them)
@@ -1325,39 +1374,76 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
             S.tables_layer = l + 1;  // the producer may issue this layer's routed copies
         }
         consumer_sync();
-        // ---------------------------------------------------------- G and D
+        // ---------------------------------------------------------- S, G and D
+        // the shared units already in the static region first (they overlap the routed copies), then the
+        // gate/up units of the ring (routed, then shared ones that did not fit), then the down blocks
         const int D = S.D, nu = D * P.units_r;
         const int nrg = c < nu ? (nu - 1 - c) / G + 1 : 0;
         const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
-        const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(nrg, 1) - 1) / max(nrg, 1))) : 8;
-        const int nitems = nrg * npc + ngr * cw.nblk;
+        const int nss = min(cw.nshg, P.ua), ngu = nrg + (cw.nshg - nss);  // ring gate/up units: routed, shared
+        const int nun = nss + ngu;
+        const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(nun, 1) - 1) / max(nun, 1))) : 8;
+        const int nitems = nun * npc + ngr * cw.nblk;
 #pragma unroll 1
         for (int i = wid; i < nitems; i += kCW) {
-            if (i < nrg * npc) {
+            if (i < nss * npc) {
                 const int ui = i / npc, pi = i - ui * npc;
-                const unsigned tseq = seq + (unsigned)ui;
-                if (!wait_task(S, P, tseq)) break;
-                const int u = c + ui * G, j = u / P.units_r, sub = u - j * P.units_r;
-                const int n = S.slot_n[j], off = S.slot_off[j];
+                if (!wait_a(S, P, 1 + ui, l)) break;
+                const unsigned char *unit = abase + P.a_rbytes + (size_t)ui * P.a_ubytes;
+                const int row0 = (c + ui * G) * 8;  // first row of the unit in the shared gate/up matrices
                 if (kMma) {
-                    unit_piece_mma(S, P, ring, part, tseq, pi, npc, n, S.pos_tok + off, S.pos_idx + off, P.a_r, P.I,
-                                   sub * 8, xb, xs, P.ready + 1 + j);
+                    unit_piece_mma(P, unit, part + (size_t)(ns + ui) * kMaxPieces * 128, &S.acnt[1 + ui], &S.aempty,
+                                   pi, npc, T, S.toks_sh, S.toks_sh, P.a_sh, P.Is, row0, xb, xs, P.ready);
                 } else {
                     int tk[NT];
 #pragma unroll
-                    for (int tt = 0; tt < NT; ++tt) tk[tt] = S.pos_tok[off + (tt < n ? tt : 0)];
-                    float g[NT], uu[NT];
-                    g_piece<NT>(P, ring + (size_t)(tseq % (unsigned)ns) * P.slot_bytes, pi, n, tk, x, xs, g, uu);
-                    if (lane == 0) {
+                    for (int tt = 0; tt < NT; ++tt) tk[tt] = tt < T ? tt : 0;
+                    float g[NT], u[NT];
+                    g_piece<NT>(P, unit, pi, T, tk, x, xs, g, u);
+                    piece_done_ffma<NT>(part + (size_t)(ns + ui) * kFfmaPart, &S.acnt[1 + ui], &S.aempty, P.ready, pi,
+                                        T, g, u, P.a_sh, S.toks_sh, P.Is, row0);
+                }
+            } else if (i < nun * npc) {
+                const int ii = i - nss * npc, ui = ii / npc, pi = ii - ui * npc;
+                const unsigned tseq = seq + (unsigned)ui;
+                if (!wait_task(S, P, tseq)) break;
+                int n, row0, lda;
+                const int *tp, *ip;
+                float *adst;
+                unsigned *rdy;
+                if (ui < nrg) {  // routed unit: slot j's rows sub*8 .. sub*8+7
+                    const int u = c + ui * G, j = u / P.units_r, sub = u - j * P.units_r, off = S.slot_off[j];
+                    n = S.slot_n[j];
+                    tp = S.pos_tok + off;
+                    ip = S.pos_idx + off;
+                    adst = P.a_r;
+                    lda = P.I;
+                    row0 = sub * 8;
+                    rdy = P.ready + 1 + j;
+                } else {  // shared unit that did not fit the static region
+                    n = T;
+                    tp = ip = S.toks_sh;
+                    adst = P.a_sh;
+                    lda = P.Is;
+                    row0 = (c + (nss + ui - nrg) * G) * 8;
+                    rdy = P.ready;
+                }
+                const int s = (int)(tseq % (unsigned)ns);
+                if (kMma) {
+                    unit_piece_mma(P, ring + (size_t)s * P.slot_bytes, part + (size_t)s * kMaxPieces * 128, &S.cnt[s],
+                                   &S.empty[s], pi, npc, n, tp, ip, adst, lda, row0, xb, xs, rdy);
+                } else {
+                    int tk[NT];
 #pragma unroll
-                        for (int tt = 0; tt < NT; ++tt)
-                            if (tt < n) P.a_r[(size_t)(off + tt) * P.I + sub * 8 + pi] = silu_mul(g[tt], uu[tt]);
-                    }
-                    piece_done(S, P, tseq, P.ready + 1 + j);
+                    for (int tt = 0; tt < NT; ++tt) tk[tt] = tp[tt < n ? tt : 0];
+                    float g[NT], uu[NT];
+                    g_piece<NT>(P, ring + (size_t)s * P.slot_bytes, pi, n, tk, x, xs, g, uu);
+                    piece_done_ffma<NT>(part + (size_t)s * kFfmaPart, &S.cnt[s], &S.empty[s], rdy, pi, n, g, uu, adst,
+                                        ip, lda, row0);
                 }
             } else {
-                const int di = i - nrg * npc, gi = di / cw.nblk, bi = di - gi * cw.nblk;
-                const unsigned tseq = seq + (unsigned)(nrg + gi);
+                const int di = i - nun * npc, gi = di / cw.nblk, bi = di - gi * cw.nblk;
+                const unsigned tseq = seq + (unsigned)(ngu + gi);
                 if (!wait_task(S, P, tseq)) break;
                 const DGroup dg = dgroup(P, gi);
                 const int n = dg.shd ? T : S.slot_n[dg.j], off = dg.shd ? 0 : S.slot_off[dg.j];
@@ -1398,7 +1484,7 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                 block_done(S, P, tseq, cw.nblk);
             }
         }
-        seq += (unsigned)(nrg + ngr);
+        seq += (unsigned)(ngu + ngr);
         consumer_sync();
         // ---------------------------------------------------------- the combine of this CTA's rows
         if (cw.nblk > 0) {
@@ -1438,62 +1524,39 @@ __device__ __forceinline__ unsigned char *claim(Shared &S, const Cfg &P, unsigne
     return ring + (size_t)s * P.slot_bytes;
 }
 
+// The static part of layer l -- the router rows of this CTA and its shared
+// gate/up units, which do not depend on the routing -- into the static
+// region, once the previous layer's copy there is consumed.
 __device__ __noinline__ bool issue_seg_a(Shared &S, const Cfg &P, const moe_layer_w &W, const CUtensorMap *mp,
-                                         unsigned char *ring, const CtaWork &cw, unsigned &seq) {
+                                         unsigned char *abase, const CtaWork &cw, int l) {
     const int H = P.H, G = gridDim.x, c = blockIdx.x;
+    if (l > 0 && !mbar_wait(&S.aempty, (unsigned)(l - 1) & 1u, P.err, kErrEmpty)) return false;
     {
         const RouterCopy rc = router_copy(P);
         const unsigned rows_bytes = (unsigned)rc.nrows * H;
-        unsigned char *dst = claim(S, P, ring, seq, 2u * H + rows_bytes + 2u * rc.sbb);
-        if (!dst) return false;
-        unsigned long long *fb = &S.full[seq % (unsigned)P.ns];
-        bulk_g2s(dst, W.router_scale, 2u * H, fb);
+        unsigned long long *fb = &S.afull[0];
+        mbar_expect_tx(fb, 2u * H + rows_bytes + 2u * rc.sbb);
+        bulk_g2s(abase, W.router_scale, 2u * H, fb);
         if (rc.nrows > 0) {
-            bulk_g2s(dst + 2 * H, W.router_q + (size_t)rc.e0 * (H / 4), rows_bytes, fb);
-            bulk_g2s(dst + 2 * H + rows_bytes, reinterpret_cast<const char *>(W.router_s) + rc.sb_lo, rc.sbb, fb);
-            bulk_g2s(dst + 2 * H + rows_bytes + rc.sbb, reinterpret_cast<const char *>(W.router_b) + rc.sb_lo, rc.sbb,
-                     fb);
+            bulk_g2s(abase + 2 * H, W.router_q + (size_t)rc.e0 * (H / 4), rows_bytes, fb);
+            bulk_g2s(abase + 2 * H + rows_bytes, reinterpret_cast<const char *>(W.router_s) + rc.sb_lo, rc.sbb, fb);
+            bulk_g2s(abase + 2 * H + rows_bytes + rc.sbb, reinterpret_cast<const char *>(W.router_b) + rc.sb_lo,
+                     rc.sbb, fb);
         }
-        ++seq;
     }
     const unsigned ubytes = 2u * P.CH * 128u + 2u * P.GH * 32u;
 #pragma unroll 1
-    for (int ui = 0; ui < cw.nshg; ++ui) {
+    for (int ui = 0; ui < min(cw.nshg, P.ua); ++ui) {
         const int u = c + ui * G, rb = u >> 2, x = u & 3;
-        unsigned char *dst = claim(S, P, ring, seq, ubytes);
-        if (!dst) return false;
-        unsigned long long *fb = &S.full[seq % (unsigned)P.ns];
+        unsigned char *dst = abase + P.a_rbytes + (size_t)ui * P.a_ubytes;
+        unsigned long long *fb = &S.afull[1 + ui];
+        mbar_expect_tx(fb, ubytes);
         tma_load_3d(dst, mp + kMapShGateQ, 32 * x, 0, rb, fb);
         tma_load_3d(dst + P.gcb, mp + kMapShUpQ, 32 * x, 0, rb, fb);
         tma_load_3d(dst + 2 * P.gcb, mp + kMapShGateSb, 8 * x, 0, rb, fb);
         tma_load_3d(dst + 2 * P.gcb + P.sbs, mp + kMapShUpSb, 8 * x, 0, rb, fb);
-        ++seq;
     }
     return true;
-}
-
-// The router rows and shared-expert units of a layer into L2 (no shared
-// memory): issued while the previous layer's routed weights stream, so that
-// the layer's first copies find their bytes in L2.
-__device__ __noinline__ void prefetch_seg_a(const Cfg &P, const moe_layer_w &W, const CUtensorMap *mp,
-                                            const CtaWork &cw) {
-    const int H = P.H, G = gridDim.x, c = blockIdx.x;
-    const RouterCopy rc = router_copy(P);
-    prefetch_l2(W.router_scale, 2u * H);
-    if (rc.nrows > 0) {
-        const char *rows = reinterpret_cast<const char *>(W.router_q + (size_t)rc.e0 * (H / 4));
-        for (unsigned o = 0, n = (unsigned)rc.nrows * H; o < n; o += 65536u) prefetch_l2(rows + o, min(65536u, n - o));
-        prefetch_l2(reinterpret_cast<const char *>(W.router_s) + rc.sb_lo, rc.sbb);
-        prefetch_l2(reinterpret_cast<const char *>(W.router_b) + rc.sb_lo, rc.sbb);
-    }
-#pragma unroll 1
-    for (int ui = 0; ui < cw.nshg; ++ui) {
-        const int u = c + ui * G, rb = u >> 2, x = u & 3;
-        tma_prefetch_3d(mp + kMapShGateQ, 32 * x, 0, rb);
-        tma_prefetch_3d(mp + kMapShUpQ, 32 * x, 0, rb);
-        tma_prefetch_3d(mp + kMapShGateSb, 8 * x, 0, rb);
-        tma_prefetch_3d(mp + kMapShUpSb, 8 * x, 0, rb);
-    }
 }
 
 // Coordinates of routed gate/up unit u (of the grid's D * units_r) of the layer.
@@ -1513,11 +1576,17 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
     const Cfg &P = S.c;
     const int G = gridDim.x, c = blockIdx.x, ns = P.ns;
     unsigned char *ring = base + P.off_ring;
+    unsigned char *abase = base + P.off_a;
     const CtaWork cw = cta_work(P);
     unsigned seq = 0;
-    bool ok = issue_seg_a(S, P, Pk.layers[0], P.maps, ring, cw, seq);
+    int a_issued = 0;  // layers whose static part has been issued
+    for (int i = 0; i < kMaps * min(P.L, 2); ++i) prefetch_map(P.maps + i);
+    bool ok = issue_seg_a(S, P, Pk.layers[0], P.maps, abase, cw, 0);
+    if (ok) a_issued = 1;
 #pragma unroll 1
     for (int l = 0; l < P.L && ok; ++l) {
+        if (l + 2 < P.L)
+            for (int i = 0; i < kMaps; ++i) prefetch_map(P.maps + (size_t)(l + 2) * kMaps + i);
         {  // this layer's routing tables
             const unsigned long long t0 = globaltimer();
             for (unsigned it = 0; S.tables_layer < l + 1; ++it) {
@@ -1535,30 +1604,20 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
         const int D = S.D, nu = D * P.units_r;
         const int nrg = c < nu ? (nu - 1 - c) / G + 1 : 0;
         const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
-        // every routed byte this CTA needs beyond what the ring takes at once: into L2 now
-#pragma unroll 1
-        for (int ui = ns; ui < nrg; ++ui) {
-            int rb, x;
-            routed_unit(P, S, c + ui * G, rb, x);
-            tma_prefetch_3d(mp + kMapGateQ, 32 * x, 0, rb);
-            tma_prefetch_3d(mp + kMapUpQ, 32 * x, 0, rb);
-            tma_prefetch_3d(mp + kMapGateSb, 8 * x, 0, rb);
-            tma_prefetch_3d(mp + kMapUpSb, 8 * x, 0, rb);
-        }
-#pragma unroll 1
-        for (int gi = 0; gi < ngr; ++gi) {
-            const DGroup dg = dgroup(P, gi);
-            for (int bi = 0; bi < cw.nblk; ++bi) {
-                const int b = cw.b0 + bi, rb = down_rb(P, S, dg, b);
-                tma_prefetch_3d(mp + (dg.shd ? kMapShDownQ : kMapDownQ), 32 * (b & 3), dg.p * dg.pc, rb);
-                tma_prefetch_3d(mp + (dg.shd ? kMapShDownSb : kMapDownSb), 8 * (b & 3), dg.p * (dg.pc / 2), rb);
-            }
-        }
-        // routed gate/up units, then the down groups, in ring order
+        // routed gate/up units first (the layer's critical path); once the ring is full, the rest of them
+        // are asked into L2 before the loop waits for free slots
         const unsigned ubytes = 2u * P.CH * 128u + 2u * P.GH * 32u;
 #pragma unroll 1
         for (int ui = 0; ui < nrg && ok; ++ui) {
             int rb, x;
+            if (ui == ns) {
+#pragma unroll 1
+                for (int uj = ns; uj < nrg; ++uj) {
+                    routed_unit(P, S, c + uj * G, rb, x);
+                    tma_prefetch_3d(mp + kMapGateQ, 32 * x, 0, rb);
+                    tma_prefetch_3d(mp + kMapUpQ, 32 * x, 0, rb);
+                }
+            }
             routed_unit(P, S, c + ui * G, rb, x);
             unsigned char *dst = claim(S, P, ring, seq, ubytes);
             if (!dst) {
@@ -1572,7 +1631,28 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             tma_load_3d(dst + 2 * P.gcb + P.sbs, mp + kMapUpSb, 8 * x, 0, rb, fb);
             ++seq;
         }
-        if (ok && l + 1 < P.L) prefetch_seg_a(P, Pk.layers[l + 1], P.maps + (size_t)(l + 1) * kMaps, cw);
+        // shared units that did not fit the static region
+#pragma unroll 1
+        for (int ui = min(cw.nshg, P.ua); ui < cw.nshg && ok; ++ui) {
+            const int u = c + ui * G, rb = u >> 2, x = u & 3;
+            unsigned char *dst = claim(S, P, ring, seq, ubytes);
+            if (!dst) {
+                ok = false;
+                break;
+            }
+            unsigned long long *fb = &S.full[seq % (unsigned)ns];
+            tma_load_3d(dst, mp + kMapShGateQ, 32 * x, 0, rb, fb);
+            tma_load_3d(dst + P.gcb, mp + kMapShUpQ, 32 * x, 0, rb, fb);
+            tma_load_3d(dst + 2 * P.gcb, mp + kMapShGateSb, 8 * x, 0, rb, fb);
+            tma_load_3d(dst + 2 * P.gcb + P.sbs, mp + kMapShUpSb, 8 * x, 0, rb, fb);
+            ++seq;
+        }
+        // the next layer's static part: its region was consumed before this layer's top-k
+        if (ok && l + 1 < P.L) {
+            ok = issue_seg_a(S, P, Pk.layers[l + 1], P.maps + (size_t)(l + 1) * kMaps, abase, cw, l + 1);
+            if (ok) a_issued = l + 2;
+        }
+        // the down groups, in ring order
 #pragma unroll 1
         for (int gi = 0; gi < ngr && ok; ++gi) {
             const DGroup dg = dgroup(P, gi);
@@ -1592,11 +1672,12 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             }
             ++seq;
         }
-        if (ok && l + 1 < P.L) ok = issue_seg_a(S, P, Pk.layers[l + 1], P.maps + (size_t)(l + 1) * kMaps, ring, cw, seq);
     }
     // let this thread's copies land before the CTA ends (bounded)
     for (unsigned q = seq > (unsigned)ns ? seq - (unsigned)ns : 0u; q < seq; ++q)
         mbar_drain(&S.full[q % (unsigned)ns], (q / (unsigned)ns) & 1u);
+    if (a_issued > 0)
+        for (int i = 0; i <= min(cw.nshg, P.ua); ++i) mbar_drain(&S.afull[i], (unsigned)(a_issued - 1) & 1u);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -1611,10 +1692,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], 1);
         }
+        for (int i = 0; i < kMaxA; ++i) mbar_init(&S.afull[i], 1);
+        mbar_init(&S.aempty, 1u + (unsigned)min(cta_work(Pk.c).nshg, Pk.c.ua));  // router + static shared units
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     for (int i = threadIdx.x; i < (int)(sizeof(Cfg) / 4); i += blockDim.x)
         reinterpret_cast<unsigned *>(&S.c)[i] = reinterpret_cast<const unsigned *>(&Pk.c)[i];
+    for (int i = threadIdx.x; i < kMaxA; i += blockDim.x) S.acnt[i] = 0;
     for (int i = threadIdx.x; i < kMaxSlots; i += blockDim.x) {
         S.owner[i] = 0xffffffffu;
         S.cnt[i] = 0;
@@ -1716,27 +1800,42 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     };
     const long nrows_r = (w.E + grid - 1) / grid;
     const size_t r_slot = 2 * (size_t)w.H + nrows_r * w.H + 2 * al(nrows_r * P.GH * 2 + 32, 16);
+    // static region: the router rows and this CTA's shared gate/up units of one layer
+    const int nshg_max = (P.units_s + grid - 1) / grid;
+    P.a_rbytes = (int)al(r_slot, 1024);
+    P.a_ubytes = (int)al(g_slot, 1024);
+    // ring: routed gate/up units and down groups
     size_t slot = g_slot;
     slot = std::max(slot, d_slot(P.dcb_s, P.sbd_s, P.pc_s));
     slot = std::max(slot, d_slot(P.dcb_r, P.sbd_r, P.pc_r));
-    slot = std::max(slot, r_slot);
     P.slot_bytes = (int)al(slot, 1024);
     const int nsl = (w.E + 31) / 32;
     P.maxc = std::min(w.E, nsl * std::min(w.k, 32));
     if (P.maxc > dec::kMaxCand) return false;
     P.yrows = 8 * dec::kMaxBlk;
-    // after the fixed part: ring (1024-aligned), x, xs, h, ybuf, candidates
+    // after the fixed part: static region and ring (1024-aligned), x, xs, h, ybuf, candidates, partials
     size_t off = al(sizeof(dec::Shared), 1024);
-    P.off_ring = (int)off;
+    P.off_a = (int)off;
     const size_t x_bytes = mma ? (size_t)T * dec::xb_token_bytes(P.CH) : (size_t)T * P.CH * dec::kXStride * 4;
     const size_t xs_bytes = mma ? (size_t)T * P.GH * 4 : (size_t)T * P.CH * 4;
-    const size_t part_per_slot = mma ? (size_t)dec::kMaxPieces * 128 * 4 : 0;
+    const size_t part_per_slot = mma ? (size_t)dec::kMaxPieces * 128 * 4 : (size_t)dec::kFfmaPart * 4;
     const size_t fixed_tail = al(x_bytes, 16) + al(xs_bytes, 16) + al((size_t)T * w.H * 2, 16) +
                               al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16) +
                               al((size_t)T * P.maxc * sizeof(dec::Cand), 16);
     const size_t budget = 227 * 1024 - 1024;  // the base is aligned to 1024 bytes inside the allocation
-    if (off + fixed_tail + 3 * ((size_t)P.slot_bytes + part_per_slot) > budget) return false;
-    long ns = (long)((budget - off - fixed_tail) / ((size_t)P.slot_bytes + part_per_slot));
+    // as many of a CTA's shared units in the static region as leave the ring 3 slots or more; else none,
+    // and 2 ring slots (every ring task is consumed in its own layer, so 2 slots cannot deadlock)
+    size_t ring_min = 3 * ((size_t)P.slot_bytes + part_per_slot);
+    int ua = std::min(nshg_max, dec::kMaxA - 1);
+    auto a_need = [&](int u) { return (size_t)P.a_rbytes + (size_t)u * (P.a_ubytes + part_per_slot); };
+    while (ua > 0 && off + a_need(ua) + fixed_tail + ring_min > budget) --ua;
+    if (off + a_need(ua) + fixed_tail + ring_min > budget) ring_min = 2 * ((size_t)P.slot_bytes + part_per_slot);
+    if (off + a_need(ua) + fixed_tail + ring_min > budget) return false;
+    P.ua = ua;
+    const size_t a_parts = (size_t)ua * part_per_slot;  // the static shared units' partial sums
+    off += (size_t)P.a_rbytes + (size_t)ua * P.a_ubytes;
+    P.off_ring = (int)off;
+    long ns = (long)((budget - off - fixed_tail - a_parts) / ((size_t)P.slot_bytes + part_per_slot));
     if (ns > dec::kMaxSlots) ns = dec::kMaxSlots;
     P.ns = (int)ns;
     off += (size_t)ns * P.slot_bytes;
@@ -1751,7 +1850,7 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     P.off_cand = (int)off;
     off += al((size_t)T * P.maxc * sizeof(dec::Cand), 16);
     P.off_part = (int)off;
-    off += (size_t)ns * part_per_slot;
+    off += (size_t)ns * part_per_slot + a_parts;  // ring slots' partials, then the shared units'
     *smem = off + 1024;
     return *smem <= 227 * 1024;
 }

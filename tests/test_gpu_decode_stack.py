@@ -37,7 +37,8 @@ def _check_stack(st, cfg, cfg_id, oracle_layers=(0,), tol=OUT_TOL):
 
 
 @pytest.mark.parametrize("cfg_id,T,L,path", [(0, 4, 3, 0), (0, 1, 2, 0), (1, 1, 4, 0), (1, 8, 2, 0), (2, 4, 3, 0),
-                                              (2, 8, 2, 0), (0, 4, 2, 1), (1, 1, 3, 2), (2, 2, 2, 1), (2, 3, 2, 2)])
+                                              (2, 8, 2, 0), (0, 4, 2, 1), (1, 1, 3, 2), (2, 2, 2, 1), (2, 3, 2, 2),
+                                              (2, 8, 2, 1)])
 def test_decode_stack_matches_per_layer_path_and_oracle(cfg_id, T, L, path):
     """path 0: automatic (CUDA-core FMAs for T = 1, tensor cores for T >= 2);
     1 and 2 force the CUDA-core and the tensor-core variants."""
