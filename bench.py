@@ -252,7 +252,7 @@ def _e2e(st, cfg, T, K, W, inputs, dev):
 
 
 def decode_measure(cfg_id, T, K, W, dev, rank=0, world=1, clocks=False, cpu_budget=3.0, layers=None,
-                   share=None, want_cpu=True):
+                   share=None, want_cpu=True, force_path=0):
     """One decode configuration: K timed steps of T tokens through the whole
     stack (device-resident inputs), its HBM roofline, the end-to-end number
     and the oracle on the host cores.  Returns (result, stack)."""
@@ -260,7 +260,7 @@ def decode_measure(cfg_id, T, K, W, dev, rank=0, world=1, clocks=False, cpu_budg
     from int4_routed_expert_02_b200.stack import MoEStack
     cfg = synth.CONFIGS[cfg_id]
     st = MoEStack(cfg, cfg_id, T=T, layers=layers, device=dev, keep_router_codes=cfg.zipf > 0,
-                  device_layers=None if share is None else share.layers)
+                  device_layers=None if share is None else share.layers, opts=moe.make_opts(force_path=force_path))
     inputs = Inputs(cfg, cfg_id, st, T, W + K, rank, dev)
     stream = torch.cuda.current_stream(dev)
     st.capture()
@@ -623,7 +623,7 @@ def run_ours(args, rank, world, local_rank):
     K, W = args.steps, args.warmup
     head_res, st = decode_measure(args.config, T, K, W, dev, rank, world, clocks=(rank == 0),
                                   cpu_budget=0 if args.no_cpu_baseline else args.cpu_budget,
-                                  layers=args.layers or None)
+                                  layers=args.layers or None, force_path=args.expert_path)
     cfg = synth.CONFIGS[args.config]
     res = {
         "metric": METRIC, "value": head_res["value"], "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -689,7 +689,7 @@ def main():
     ap.add_argument("--prefill-only", action="store_true",
                     help="profiling only: the 128-token prefill chunks alone (with --layers, --expert-path)")
     ap.add_argument("--expert-path", type=int, default=0, choices=[0, 1, 2, 3],
-                    help="with --prefill-only: force_path of the expert FFN (0 automatic)")
+                    help="profiling only: force_path of the expert FFN (0 automatic) for --prefill-only or the headline")
     ap.add_argument("--headline-only", dest="all_configs", action="store_false",
                     help="only the headline configuration (skip the other configurations of the line)")
     args = ap.parse_args()
