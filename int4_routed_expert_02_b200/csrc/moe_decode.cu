@@ -138,8 +138,8 @@ struct Shared {
     int acnt[kMaxA];                       // pieces of a shared unit that are done
     volatile int tables_layer;             // 1 + the layer whose routing tables are ready
     volatile int verdict;                  // consumers: 1 while no error is recorded
+    volatile int kverdict;                 // the token warps' verdict on this layer's routing
     int D;                                 // distinct experts of the current layer
-    int ccount[kMaxT];                     // top-k candidates per token
     int slot_e[kMaxPairs], slot_off[kMaxPairs], slot_n[kMaxPairs];
     int pos_tok[kMaxPairs];                // bucketed position -> token
     int pos_pair[kMaxPairs];               // bucketed position -> pair id t*k + s
@@ -261,6 +261,9 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, i
 
 // Named barrier of the 15 consumer warps.
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCThreads) : "memory"); }
+
+// Named barrier of the T token warps (the top-k and the buckets).
+__device__ __forceinline__ void token_warps_sync(int T) { asm volatile("bar.sync 2, %0;" ::"r"(T * 32) : "memory"); }
 
 // ------------------------------------------------------------------ grid barrier (split phase)
 
@@ -920,8 +923,9 @@ struct Cand {
 //   3. lanes r < k form the softmax weights (one exp per lane);
 // then, over the whole block, the buckets by counting over the T*k pairs.
 __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, const uint16_t *pes, unsigned tag) {
+    // called by the T token warps only (T * k <= 32 T pairs: one per thread at most)
     const int T = P.T, E = P.E, k = P.k, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    if (wid < T) {
+    {
         const int t = wid, nsl = (E + 31) / 32;
         Cand *cw = cand + (size_t)t * P.maxc;
         int nc = 0;
@@ -999,7 +1003,7 @@ __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, co
             S.wts[t * k + r] = (float)(q / z * (double)bf16_bits_to_float(pes[S.idx[t * k + r]]));
         }
     }
-    consumer_sync();
+    token_warps_sync(T);
     const int n = T * k;
 #pragma unroll 1
     for (int p = threadIdx.x; p < n; p += kCThreads) {
@@ -1018,7 +1022,7 @@ __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, co
         S.slot_off[p] = less;  // scratch: moved to the slot's entry below
         S.slot_n[p] = cnt;
     }
-    consumer_sync();
+    token_warps_sync(T);
     int my_slot = -1, my_e = 0, my_off = 0, my_n = 0;
     if (threadIdx.x < n && S.first[threadIdx.x]) {
         const int p = threadIdx.x, e = S.idx[p];
@@ -1030,7 +1034,7 @@ __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, co
         my_off = S.slot_off[p];
         my_n = S.slot_n[p];
     }
-    consumer_sync();
+    token_warps_sync(T);
     if (my_slot >= 0) {
         S.slot_e[my_slot] = my_e;
         S.slot_off[my_slot] = my_off;
@@ -1041,7 +1045,7 @@ __device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, co
         for (int q = 0; q < n; ++q) d += S.first[q];
         S.D = d;
     }
-    consumer_sync();
+    token_warps_sync(T);
 }
 
 // ------------------------------------------------------------------ work bookkeeping
@@ -1156,9 +1160,12 @@ __device__ __noinline__ bool stage_a(Shared &S, const Cfg &P, int s, bool shd, i
     return ok != 0;
 }
 
-// This CTA's 8-row output blocks [b0, b1) and its shared-expert units.
+// This CTA's 8-row output blocks [b0, b1), its shared-expert units, and its
+// rank rk for the routed gate/up units (unit u goes to the CTA of rank u mod
+// G): the CTAs with one output block fewer rank first, so the down blocks and
+// the gate/up units even out over the grid.
 struct CtaWork {
-    int b0, nblk, nshg;
+    int b0, nblk, nshg, rk;
 };
 
 __device__ __forceinline__ CtaWork cta_work(const Cfg &P) {
@@ -1167,6 +1174,9 @@ __device__ __forceinline__ CtaWork cta_work(const Cfg &P) {
     w.b0 = (int)((long long)P.nrb8 * c / G);
     w.nblk = (int)((long long)P.nrb8 * (c + 1) / G) - w.b0;
     w.nshg = c < P.units_s ? (P.units_s - 1 - c) / G + 1 : 0;
+    const int q = P.nrb8 / G, nhigh = P.nrb8 - q * G;  // CTAs with q + 1 blocks
+    const int hb = w.b0 - q * c;                       // of them before this CTA
+    w.rk = w.nblk == q ? c - hb : (G - nhigh) + hb;
     return w;
 }
 
@@ -1361,32 +1371,28 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
             consumer_sync();
             if (threadIdx.x == 0) mbar_arrive(&S.aempty);
         }
-        // ---------------------------------------------------------- K: top-k and buckets
-        // (the logits carry the layer's tag: no barrier before reading them)
-        topk_bucket(P, S, cand, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
-        if (threadIdx.x == 0) S.verdict = ldcg_int(P.err) == 0;
-        consumer_sync();
-        if (!(ok = S.verdict != 0)) break;
-        if (threadIdx.x == 0) {
-            S.exp_ready[0] += (unsigned)P.units_s;
-            for (int j = 0; j < S.D; ++j) S.exp_ready[1 + j] += (unsigned)P.units_r;
-            __threadfence_block();
-            S.tables_layer = l + 1;  // the producer may issue this layer's routed copies
-        }
-        consumer_sync();
-        // ---------------------------------------------------------- S, G and D
-        // the shared units already in the static region first (they overlap the routed copies), then the
-        // gate/up units of the ring (routed, then shared ones that did not fit), then the down blocks
-        const int D = S.D, nu = D * P.units_r;
-        const int nrg = c < nu ? (nu - 1 - c) / G + 1 : 0;
-        const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
-        const int nss = min(cw.nshg, P.ua), ngu = nrg + (cw.nshg - nss);  // ring gate/up units: routed, shared
-        const int nun = nss + ngu;
-        const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(nun, 1) - 1) / max(nun, 1))) : 8;
-        const int nitems = nun * npc + ngr * cw.nblk;
+        // ---------------------------------------------------------- K (token warps) and S (the others)
+        // The T token warps rank the logits (they carry the layer's tag: no barrier before reading them)
+        // and publish the routing tables; meanwhile the other warps run the shared units already in the
+        // static region, which need only xe.
+        const int nss = min(cw.nshg, P.ua);
+        if (wid < T) {
+            topk_bucket(P, S, cand, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
+            if (threadIdx.x == 0) {
+                const int good = ldcg_int(P.err) == 0;
+                S.kverdict = good;
+                if (good) {
+                    S.exp_ready[0] += (unsigned)P.units_s;
+                    for (int j = 0; j < S.D; ++j) S.exp_ready[1 + j] += (unsigned)P.units_r;
+                }
+                __threadfence_block();
+                S.tables_layer = l + 1;  // the producer and the other warps may go on
+            }
+        } else {
+            const int nsw = kCW - T;  // warps on the shared units
+            const int npc = kMma ? min(kMaxPieces, max(1, (nsw + max(nss, 1) - 1) / max(nss, 1))) : 8;
 #pragma unroll 1
-        for (int i = wid; i < nitems; i += kCW) {
-            if (i < nss * npc) {
+            for (int i = wid - T; i < nss * npc; i += nsw) {
                 const int ui = i / npc, pi = i - ui * npc;
                 if (!wait_a(S, P, 1 + ui, l)) break;
                 const unsigned char *unit = abase + P.a_rbytes + (size_t)ui * P.a_ubytes;
@@ -1403,8 +1409,37 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                     piece_done_ffma<NT>(part + (size_t)(ns + ui) * kFfmaPart, &S.acnt[1 + ui], &S.aempty, P.ready, pi,
                                         T, g, u, P.a_sh, S.toks_sh, P.Is, row0);
                 }
-            } else if (i < nun * npc) {
-                const int ii = i - nss * npc, ui = ii / npc, pi = ii - ui * npc;
+            }
+        }
+        // every warp: this layer's routing tables (bounded wait), then the ring items
+        {
+            int seen = 1;
+            if (lane == 0) {
+                const unsigned long long t0 = globaltimer();
+                for (unsigned it = 0; S.tables_layer < l + 1; ++it)
+                    if ((it & 63u) == 63u && (ldcg_int(P.err) != 0 || globaltimer() - t0 > kWaitNs)) {
+                        atomicCAS(P.err, 0, kErrTables);
+                        seen = 0;
+                        break;
+                    }
+                __threadfence_block();
+            }
+            seen = __shfl_sync(0xffffffffu, seen, 0);
+            if (!(ok = seen && S.kverdict != 0)) break;
+        }
+        // ---------------------------------------------------------- G and D
+        // the gate/up units of the ring (routed, then shared ones that did not fit the static region),
+        // then the down blocks
+        const int D = S.D, nu = D * P.units_r;
+        const int nrg = cw.rk < nu ? (nu - 1 - cw.rk) / G + 1 : 0;
+        const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
+        const int ngu = nrg + (cw.nshg - nss);  // ring gate/up units: routed, shared
+        const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(ngu, 1) - 1) / max(ngu, 1))) : 8;
+        const int nitems = ngu * npc + ngr * cw.nblk;
+#pragma unroll 1
+        for (int i = wid; i < nitems; i += kCW) {
+            if (i < ngu * npc) {
+                const int ui = i / npc, pi = i - ui * npc;
                 const unsigned tseq = seq + (unsigned)ui;
                 if (!wait_task(S, P, tseq)) break;
                 int n, row0, lda;
@@ -1412,7 +1447,7 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                 float *adst;
                 unsigned *rdy;
                 if (ui < nrg) {  // routed unit: slot j's rows sub*8 .. sub*8+7
-                    const int u = c + ui * G, j = u / P.units_r, sub = u - j * P.units_r, off = S.slot_off[j];
+                    const int u = cw.rk + ui * G, j = u / P.units_r, sub = u - j * P.units_r, off = S.slot_off[j];
                     n = S.slot_n[j];
                     tp = S.pos_tok + off;
                     ip = S.pos_idx + off;
@@ -1442,7 +1477,7 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                                         ip, lda, row0);
                 }
             } else {
-                const int di = i - nun * npc, gi = di / cw.nblk, bi = di - gi * cw.nblk;
+                const int di = i - ngu * npc, gi = di / cw.nblk, bi = di - gi * cw.nblk;
                 const unsigned tseq = seq + (unsigned)(ngu + gi);
                 if (!wait_task(S, P, tseq)) break;
                 const DGroup dg = dgroup(P, gi);
@@ -1599,10 +1634,14 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             }
             if (!ok) break;
             __threadfence_block();
+            if (!S.kverdict) {  // the routing of this layer failed: the consumers stop
+                ok = false;
+                break;
+            }
         }
         const CUtensorMap *mp = P.maps + (size_t)l * kMaps;
         const int D = S.D, nu = D * P.units_r;
-        const int nrg = c < nu ? (nu - 1 - c) / G + 1 : 0;
+        const int nrg = cw.rk < nu ? (nu - 1 - cw.rk) / G + 1 : 0;
         const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
         // routed gate/up units first (the layer's critical path); once the ring is full, the rest of them
         // are asked into L2 before the loop waits for free slots
@@ -1613,12 +1652,12 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             if (ui == ns) {
 #pragma unroll 1
                 for (int uj = ns; uj < nrg; ++uj) {
-                    routed_unit(P, S, c + uj * G, rb, x);
+                    routed_unit(P, S, cw.rk + uj * G, rb, x);
                     tma_prefetch_3d(mp + kMapGateQ, 32 * x, 0, rb);
                     tma_prefetch_3d(mp + kMapUpQ, 32 * x, 0, rb);
                 }
             }
-            routed_unit(P, S, c + ui * G, rb, x);
+            routed_unit(P, S, cw.rk + ui * G, rb, x);
             unsigned char *dst = claim(S, P, ring, seq, ubytes);
             if (!dst) {
                 ok = false;
