@@ -331,10 +331,16 @@ def expert_flops(cfg, T: int) -> float:
 
 
 PREFILL_KERNELS = {
-    0: "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
     2: "expert_mma_kernel (tcgen05 grouped GEMM, FP16 operands) x2 + gather + combine",
     3: "gateup_kernel + down_kernel (weight-stationary warp MMA, exact FP16 codes) + gather + combine",
 }
+
+
+def expert_path_of(force_path, T):
+    """The expert path a call of T tokens takes (the library's automatic rule when force_path is 0)."""
+    if force_path:
+        return force_path
+    return 1 if T < 32 else (3 if T <= 512 else 2)
 
 
 def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0):
@@ -372,15 +378,16 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0
     tflops = fl / (roof["us_per_launch"] / 1e6) / 1e12
     peak_t = hbm["bf16_tflops"]  # FP16 and BF16 share the dense tensor rate
     fused = T != cfg.T
+    path = expert_path_of(force_path, T)
     traffic = (PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER if fused else PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK) \
-        if force_path in (0, 2) else None
+        if path == 2 else None
     name = (workload_name(cfg, T) + ", the rows of 8 chunks of 128 through each layer in one call") if fused else \
         (workload_name(cfg, T) + f", {chunks} chunks chunk-major")
     bound_us = max(roof["bytes_per_launch"] / (hbm["hbm_gbs"] * 1e3), fl / (peak_t * 1e6))
     return {"workload": name, "tok_s": round(chunks * T / (ms / 1e3), 1),
             "ms_per_chunk": round(ms / chunks, 4),
             "force_path": force_path,
-            "expert_ffn": {"kernel": PREFILL_KERNELS[force_path],
+            "expert_ffn": {"kernel": PREFILL_KERNELS[path],
                            "us_per_launch": roof["us_per_launch"], "flops_per_launch": fl,
                            "tflops": round(tflops, 2), "tensor_peak_tflops": peak_t,
                            "tensor_frac": round(tflops / peak_t, 4), "hbm_gbs": roof["achieved"],
@@ -659,7 +666,8 @@ def run_ours(args, rank, world, local_rank):
     prefill, pst = prefill_measure(dev)
     res["prefill"] = prefill
     res["prefill_fused"], _ = prefill_measure(dev, chunks=2, T=1024, share=pst)
-    res["prefill_ws"], _ = prefill_measure(dev, share=pst, force_path=3)
+    # the other tensor-core path at each size, for comparison
+    res["prefill_tcgen05"], _ = prefill_measure(dev, share=pst, force_path=2)
     res["prefill_fused_ws"], _ = prefill_measure(dev, chunks=2, T=1024, share=pst, force_path=3)
     r64, s64 = decode_measure(4, 64, 32, W, dev, cpu_budget=args.sub_cpu_budget, share=pst)
     r64["workload"] += " (64-token decode batches on the Gemma shape)"

@@ -98,7 +98,8 @@ typedef struct {
     int post_norm;      /* 1: out = (h + rmsnorm_no_scale(m)) * layer_scalar; 0: (h + m) * layer_scalar */
     float layer_scalar; /* default 1.0 */
     float eps;          /* default 1e-6, inside every RMS */
-    int force_path;     /* 0 auto (tensor-core grouped GEMM from T >= 32 on, else dequant-GEMV),
+    int force_path;     /* 0 auto: dequant-GEMV below 32 tokens, the weight-stationary warp-level MMA
+                           for 32..512, the tcgen05 grouped GEMM above;
                            1 CUDA-core dequant-GEMV, 2 tensor-core (tcgen05) grouped GEMM,
                            3 weight-stationary warp-level MMA (exact codes, FP32 scale/bias) */
 } moe_opts;
@@ -192,7 +193,7 @@ MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets
  * weights are MLX affine 4-bit, groups of 64, a BF16 scale and bias per
  * group, section "How TurboFieldfare saves memory".)
  * Path: force_path 1, or T < 32 in auto mode, is the CUDA-core dequant-GEMV
- * (fp32 sums of exact products).  force_path 2, or T >= 32, is the tcgen05
+ * (fp32 sums of exact products).  force_path 2, or T > 512 in auto mode, is the tcgen05
  * grouped GEMM on FP16 operands: it needs every weight s*q + b and every
  * SwiGLU value within the FP16 range (|v| <= 65504).  A layer outside that
  * range is not computed approximately: the kernel records MOE_EDEVICE
@@ -202,7 +203,8 @@ MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets
  * weight read once per group of 8 (gate/up) or 16 (down) tokens of an expert:
  * codes enter as exact FP16 values, scale and bias stay FP32, so only the
  * token rows and SwiGLU outputs are FP16 (a SwiGLU value beyond 65504 is
- * reported as above; weights have no range limit).  E <= 1024.
+ * reported as above; weights have no range limit).  E <= 1024.  Auto mode takes
+ * it for 32 <= T <= 512.
  */
 MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *idx, const float *wts,
                    const int32_t *offsets, const int32_t *perm, const int32_t *active, int with_shared,
@@ -389,7 +391,7 @@ MOE_API int moe_qmat_gemv(const moe_qmat *w, int rows, int cols, const uint16_t 
  *   - The looked-up address is kept for the life of the process.  It does not
  *     survive cudaDeviceReset (or any other teardown of the device's primary
  *     context): do not call this entry point after one.
- *   - The tensor-core path (T >= 32, or force_path 2) leaves its status words
+ *   - The tensor-core paths (T >= 32, or force_path 2 or 3) leave their status words
  *     in the scratch; moe_noalloc_status reads them.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)

@@ -113,7 +113,8 @@ struct WsLayout {
 };
 
 constexpr size_t kStatusOffset = 4;
-constexpr int kMmaMinT = 32;  // auto path: tensor-core grouped GEMM from this many tokens on
+constexpr int kMmaMinT = 32;   // auto path: tensor cores from this many tokens on (else the dequant-GEMV)
+constexpr int kWsMaxT = 512;   // ... the weight-stationary warp-MMA path up to this many, the tcgen05 GEMM above
 
 WsLayout ws_layout(const moe_layer_w *w, int T) {
     WsLayout L;
@@ -183,7 +184,8 @@ enum Path { kPathGemv = 1, kPathTc = 2, kPathWs = 3 };
 
 Path expert_path(const moe_opts &o, int T) {
     if (o.force_path != 0) return static_cast<Path>(o.force_path);
-    return T >= kMmaMinT ? kPathTc : kPathGemv;
+    if (T < kMmaMinT) return kPathGemv;
+    return T <= kWsMaxT ? kPathWs : kPathTc;
 }
 
 // Expert part of a call: the SwiGLU FFNs of the routed and shared experts into

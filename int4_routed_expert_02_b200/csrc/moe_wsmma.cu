@@ -345,19 +345,28 @@ __device__ __forceinline__ void d_compute(const DStage &s, float (&y)[4][4]) {
     }
 }
 
+// Down items are 4 row blocks (128 output rows) of one matrix and 16 tokens: warp pair p = w >> 1 owns
+// row block 4*ib + p and its two warps split the block's 64-column groups of K, so the sum at the end of
+// an item runs over 2 warps.
+constexpr int kDownRbs = 4;
+
 __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
     __shared__ int cum[kMaxSlots + 1];
     __shared__ float red[kWarps][16][32];
     const int na = __ldg(P.active);
     const int units = build_prefix(P, cum);
-    const int rbs_s = P.rows_s / 32, rbs_r = P.rows_r / 32;
+    // items per token tile: the row blocks in runs of kDownRbs
+    const int rbs_s = (P.rows_s / 32 + kDownRbs - 1) / kDownRbs, rbs_r = (P.rows_r / 32 + kDownRbs - 1) / kDownRbs;
     const int nsh = P.with_shared ? rbs_s * ((P.T + P.ntok - 1) / P.ntok) : 0;
     const int total = nsh + units * rbs_r;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int pair = warp >> 1, half = warp & 1;
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Item it = get_item(P, cum, na, id, nsh, rbs_s, rbs_r);
+        const Item it = get_item(P, cum, na, id, nsh, rbs_s, rbs_r);  // it.rb: the run of row blocks
         const int K = it.shared ? P.K_s : P.K_r, C = K / 32, G = K / 64, rows = it.shared ? P.rows_s : P.rows_r;
-        const size_t mrb = it.shared ? (size_t)it.rb : (size_t)it.e * (rows / 32) + it.rb;
+        const int rb = it.rb * kDownRbs + pair;  // this pair's row block
+        const bool live = rb < rows / 32;
+        const size_t mrb = it.shared ? (size_t)rb : (size_t)it.e * (rows / 32) + rb;
         DView v;
         v.q = (it.shared ? P.sq[0] : P.q[0]) + (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
         v.sb = (it.shared ? P.ssb[0] : P.sb[0]) + mrb * G * 32 + 2 * t;
@@ -369,12 +378,12 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
         float y[4][4];
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) y[sl][0] = y[sl][1] = y[sl][2] = y[sl][3] = 0.f;
-        int gi = warp;
-        if (gi < G) {
+        int gi = half;
+        if (live && gi < G) {
             DStage cur, nxt;
             d_load(v, gi, cur);
-            for (; gi + kWarps < G; gi += kWarps) {
-                d_load(v, gi + kWarps, nxt);
+            for (; gi + 2 < G; gi += 2) {
+                d_load(v, gi + 2, nxt);
                 d_compute(cur, y);
                 cur = nxt;
             }
@@ -385,21 +394,19 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) red[warp][sl * 4 + c][lane] = y[sl][c];
         __syncthreads();
-        {
-            // warp w: slice w & 3, token j0 (w < 4) or j1; rows 2t, 2t+1 of the slice
-            const int sl = warp & 3, h = warp >> 2;
-            float o0 = 0.f, o1 = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-                o0 += red[w][sl * 4 + 2 * h][lane];
-                o1 += red[w][sl * 4 + 2 * h + 1][lane];
-            }
-            const int j = g + 8 * h;
+        if (live) {
+            // warp 2p: token g, warp 2p + 1: token g + 8; rows 2t, 2t+1 of each slice of row block rb
+            const int h = half, j = g + 8 * h;
             if (j < it.n) {
                 float *dst = it.shared ? P.sh + (size_t)(it.seg + j) * P.H
                                        : P.y + (size_t)__ldg(P.perm + it.seg + j) * P.H;
-                const int r = it.rb * 32 + sl * 8 + 2 * t;
-                *reinterpret_cast<float2 *>(dst + r) = make_float2(o0, o1);
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    const float o0 = red[2 * pair][sl * 4 + 2 * h][lane] + red[2 * pair + 1][sl * 4 + 2 * h][lane];
+                    const float o1 =
+                        red[2 * pair][sl * 4 + 2 * h + 1][lane] + red[2 * pair + 1][sl * 4 + 2 * h + 1][lane];
+                    *reinterpret_cast<float2 *>(dst + rb * 32 + sl * 8 + 2 * t) = make_float2(o0, o1);
+                }
             }
         }
         __syncthreads();
@@ -478,7 +485,8 @@ cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T,
     P.xin = b.act;
     P.ld_in = Kmax;
     P.ntok = 16;
-    items = (with_shared ? (long long)(H / 32) * ((T + 15) / 16) : 0) + (pairs / 16 + max_active) * (H / 32);
+    const long long drun = (H / 32 + kDownRbs - 1) / kDownRbs;
+    items = (with_shared ? drun * ((T + 15) / 16) : 0) + (pairs / 16 + max_active) * drun;
     grid = (int)(items < 2LL * sms ? items : 2LL * sms);
     if (grid > 0) {
         down_kernel<<<grid, kThreads, 0, st>>>(P);

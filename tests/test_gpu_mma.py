@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from int4_routed_expert_02_b200 import synth
-from tests.moe_cases import OUT_TOL, bf16_host, hidden_with_gap, host, max_err_vs_rms, oracle_layer
+from tests.moe_cases import OUT_TOL, assert_same_up_to_one_rounding, bf16_host, hidden_with_gap, host, max_err_vs_rms, oracle_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -121,26 +121,33 @@ def test_mma_edge_shapes(dims):
     assert max_err_vs_rms(bf16_host(out)[rows], ref["out_f64"]) <= OUT_TOL
 
 
-def test_prefill_chunk_layer_auto_path_is_deterministic():
-    """A 128-token chunk at the Gemma shape takes the tensor-core path by
-    default; reruns are bit-identical and sampled rows match the oracle."""
+def test_prefill_chunk_layer_paths_are_deterministic():
+    """A 128-token chunk at the Gemma shape, on the automatic path (the
+    weight-stationary warp-MMA path at this size) and on the tcgen05 path:
+    reruns are bit-identical, sampled rows match the oracle, and the two paths
+    agree to one bf16 ulp element by element."""
     cfg = synth.CONFIGS[4]
     w, D, OL = _layer(synth.CONFIGS[1], 1, layer=3)
     T = 128
     h = synth.gen_hidden(cfg, 4, 2, T)
     hd = h.cuda()
     ws = moe.workspace(D, T)
-    outs = []
-    for _ in range(2):
-        out = torch.empty_like(hd)
-        moe.moe_layer_forward(D, hd, out, T, ws)
-        torch.cuda.synchronize()
-        moe.moe_workspace_status(ws)
-        outs.append(out)
-    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     rows = [3, 64, 100]
     ref = oracle.layer_forward(OL, h[rows])
-    assert max_err_vs_rms(bf16_host(outs[0])[rows], ref["out_f64"]) <= OUT_TOL
+    first = {}
+    for path in (0, MMA):
+        outs = []
+        for _ in range(2):
+            out = torch.empty_like(hd)
+            moe.moe_layer_forward(D, hd, out, T, ws, moe.make_opts(force_path=path))
+            torch.cuda.synchronize()
+            moe.moe_workspace_status(ws)
+            outs.append(out)
+        assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+        assert max_err_vs_rms(bf16_host(outs[0])[rows], ref["out_f64"]) <= OUT_TOL
+        first[path] = outs[0]
+    # the two paths accumulate in another order: rounding flips only
+    assert_same_up_to_one_rounding(first[0], first[MMA], max_frac=0.25)
 
 
 def test_prefill_rows_of_eight_chunks_in_one_call():
@@ -166,7 +173,8 @@ def test_prefill_rows_of_eight_chunks_in_one_call():
         moe.moe_layer_forward(D, hd[c * 128:(c + 1) * 128], chunked[c * 128:(c + 1) * 128], 128, ws128)
     torch.cuda.synchronize()
     moe.moe_workspace_status(ws128)
-    assert max_err_vs_rms(bf16_host(out), bf16_host(chunked)) <= 5e-3
+    # one call of 1024 rows and the 128-row chunks may take different expert paths
+    assert_same_up_to_one_rounding(out, chunked, max_frac=0.25)
 
 
 def test_grouped_gemm_wait_timeout_is_reported_and_the_next_call_is_fine(monkeypatch):

@@ -9,7 +9,7 @@ output against moe_layer_forward with a caller-provided workspace, on two
 calls in a row (the scratch keeps the first call's contents when the second
 one starts).  Both run the same kernels on the same inputs, so the outputs
 must be bit-identical.  The cases cover the CUDA-core path (T < 32) and the
-tensor-core path (T >= 32 in auto mode, and force_path 2), whose status words
+tensor-core paths (T >= 32 in auto mode, and force_path 2 and 3), whose status words
 live in the static scratch and are read back with moe_noalloc_status.  It
 lives in its own file, collected last.
 """
