@@ -76,7 +76,7 @@ constexpr int kMaxParts = 8;                  // K-parts of a down matrix
 constexpr int kPartChunks = 32;               // at most 32 chunks (1024 columns) per K-part
 constexpr int kBarCtrs = 1;                   // grid-barrier counters, 128 bytes apart (one polls fastest)
 constexpr int kMaxStageTH = 24576;            // largest T * H
-constexpr int kMaxCand = 512;                 // top-k candidates per token
+constexpr int kMaxSl = 16;                    // groups of 32 experts (E <= 512)
 constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s
 
 enum { kErrBarrier = 1, kErrFull, kErrEmpty, kErrReady, kErrOwner, kErrTables, kErrStage, kErrLogits };
@@ -107,8 +107,7 @@ struct Cfg {
     int sbs;                     // bytes of one matrix's (scale, bias) words in a gate/up slot (128-aligned)
     int dcb_s, dcb_r;            // bytes of one 8-row block's codes in a down slot (1024-aligned)
     int sbd_s, sbd_r;            // bytes of one 8-row block's words in a down slot (128-aligned)
-    int maxc;                    // top-k candidate capacity per token
-    int off_a, off_ring, off_x, off_xs, off_h, off_y, off_cand, off_part;  // dynamic shared memory offsets
+    int off_a, off_ring, off_x, off_xs, off_h, off_y, off_part;  // dynamic shared memory offsets
     int yrows;                   // rows per ybuf entry (8 * kMaxBlk)
     unsigned *bar;               // [kBarCtrs * 32] monotonic arrival counters
     unsigned bar_extra;          // arrivals beyond the grid the barriers wait for (tests of the timeout path)
@@ -628,38 +627,43 @@ __device__ __forceinline__ void g_piece(const Cfg &P, const unsigned char *slot,
 #pragma unroll 1
     for (int c = lane; c < CH; c += 32) {
         const int sw = (row ^ (c & 7)) << 4;
+        // gate and up rows of the chunk against one read of the inputs
+        const uint4 qg = *reinterpret_cast<const uint4 *>(slot + c * 128 + sw);
+        const uint4 qu = *reinterpret_cast<const uint4 *>(slot + gcb + c * 128 + sw);
+        const uint32_t sbg = *reinterpret_cast<const uint32_t *>(sbb + (c >> 1) * 32 + row * 4);
+        const uint32_t sbu = *reinterpret_cast<const uint32_t *>(sbb + sbs + (c >> 1) * 32 + row * 4);
+        const uint32_t wg[4] = {qg.x, qg.y, qg.z, qg.w}, wu[4] = {qu.x, qu.y, qu.z, qu.w};
+        float2 g0[NT], g1[NT], u0[NT], u1[NT];
 #pragma unroll
-        for (int mat = 0; mat < 2; ++mat) {
-            const uint4 q = *reinterpret_cast<const uint4 *>(slot + mat * gcb + c * 128 + sw);
-            const uint32_t sbw = *reinterpret_cast<const uint32_t *>(sbb + mat * sbs + (c >> 1) * 32 + row * 4);
-            const float s = bf16_bits_to_float(sbw & 0xffffu) * kCodeUnscale, b = bf16_bits_to_float(sbw >> 16);
-            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
-            float2 a0[NT], a1[NT];
+        for (int tt = 0; tt < NT; ++tt) g0[tt] = g1[tt] = u0[tt] = u1[tt] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int tt = 0; tt < NT; ++tt) a0[tt] = a1[tt] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-                const Decoded8 d = decode_word(wv[wi]);
-#pragma unroll
-                for (int tt = 0; tt < NT; ++tt) {
-                    if (tt < n) {
-                        const float4 *xp =
-                            reinterpret_cast<const float4 *>(x + ((size_t)tk[tt] * CH + c) * kXStride + wi * 8);
-                        const float4 xa = xp[0], xb = xp[1];
-                        a0[tt] = ffma2(make_float2(d.f[0], d.f[1]), make_float2(xa.x, xa.y), a0[tt]);
-                        a1[tt] = ffma2(make_float2(d.f[2], d.f[3]), make_float2(xa.z, xa.w), a1[tt]);
-                        a0[tt] = ffma2(make_float2(d.f[4], d.f[5]), make_float2(xb.x, xb.y), a0[tt]);
-                        a1[tt] = ffma2(make_float2(d.f[6], d.f[7]), make_float2(xb.z, xb.w), a1[tt]);
-                    }
-                }
-            }
+        for (int wi = 0; wi < 4; ++wi) {
+            const Decoded8 dg = decode_word(wg[wi]), du = decode_word(wu[wi]);
 #pragma unroll
             for (int tt = 0; tt < NT; ++tt) {
                 if (tt < n) {
-                    const float dsum = (a0[tt].x + a0[tt].y) + (a1[tt].x + a1[tt].y);
-                    float &acc = mat ? u[tt] : g[tt];
-                    acc = fmaf(s, dsum, fmaf(b, xs[tk[tt] * CH + c], acc));
+                    const float4 *xp =
+                        reinterpret_cast<const float4 *>(x + ((size_t)tk[tt] * CH + c) * kXStride + wi * 8);
+                    const float4 xa = xp[0], xb = xp[1];
+                    g0[tt] = ffma2(make_float2(dg.f[0], dg.f[1]), make_float2(xa.x, xa.y), g0[tt]);
+                    g1[tt] = ffma2(make_float2(dg.f[2], dg.f[3]), make_float2(xa.z, xa.w), g1[tt]);
+                    g0[tt] = ffma2(make_float2(dg.f[4], dg.f[5]), make_float2(xb.x, xb.y), g0[tt]);
+                    g1[tt] = ffma2(make_float2(dg.f[6], dg.f[7]), make_float2(xb.z, xb.w), g1[tt]);
+                    u0[tt] = ffma2(make_float2(du.f[0], du.f[1]), make_float2(xa.x, xa.y), u0[tt]);
+                    u1[tt] = ffma2(make_float2(du.f[2], du.f[3]), make_float2(xa.z, xa.w), u1[tt]);
+                    u0[tt] = ffma2(make_float2(du.f[4], du.f[5]), make_float2(xb.x, xb.y), u0[tt]);
+                    u1[tt] = ffma2(make_float2(du.f[6], du.f[7]), make_float2(xb.z, xb.w), u1[tt]);
                 }
+            }
+        }
+        const float s_g = bf16_bits_to_float(sbg & 0xffffu) * kCodeUnscale, b_g = bf16_bits_to_float(sbg >> 16);
+        const float s_u = bf16_bits_to_float(sbu & 0xffffu) * kCodeUnscale, b_u = bf16_bits_to_float(sbu >> 16);
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+            if (tt < n) {
+                const float xsum = xs[tk[tt] * CH + c];
+                g[tt] = fmaf(s_g, (g0[tt].x + g0[tt].y) + (g1[tt].x + g1[tt].y), fmaf(b_g, xsum, g[tt]));
+                u[tt] = fmaf(s_u, (u0[tt].x + u0[tt].y) + (u1[tt].x + u1[tt].y), fmaf(b_u, xsum, u[tt]));
             }
         }
     }
@@ -905,86 +909,82 @@ __device__ __forceinline__ double key_logit(unsigned long long k) {
     return __longlong_as_double((long long)b);
 }
 
-struct Cand {
-    unsigned long long key;
-    int e, pad;
-};
-
 // K: top-k of every token (ties to the lower expert index; ordered by logit
 // desc, index asc), gate weights softmax(logits[top-k]) * per_expert_scale
 // in fp64, and the bucketing of the T*k pairs by expert (stable by pair id).
 // Every CTA computes the same result from the same logits.  Warp t handles
 // token t alone, with no block-wide barrier until the bucketing:
-//   1. per group of 32 experts, each lane polls one logit and ranks it among
-//      the group by shuffles; only those ranked below k can be in the top k
-//      of all E, and they are appended (ballot order) to the warp's candidate
-//      list (everything that beats a top-k logit is itself a candidate);
-//   2. each candidate's rank among the candidates is its rank among all E;
+//   1. lane j polls the logits of experts j, 32 + j, ... (all of them in
+//      flight at once) and keeps them as order-preserving 64-bit keys;
+//   2. k rounds of selection: each lane offers its largest remaining key
+//      (the lower expert on equal keys), the warp takes the maximum with two
+//      32-bit max-reductions (high word, then low word among the lanes that
+//      hold the high word) and the lowest expert index among the lanes that
+//      hold the maximum with a min-reduction; the winning lane drops it;
 //   3. lanes r < k form the softmax weights (one exp per lane);
 // then, over the whole block, the buckets by counting over the T*k pairs.
-__device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, Cand *cand, const uint16_t *pes, unsigned tag) {
-    // called by the T token warps only (T * k <= 32 T pairs: one per thread at most)
+template <int NSL>
+__device__ __noinline__ void topk_bucket(const Cfg &P, Shared &S, const uint16_t *pes, unsigned tag) {
+    // called by the T token warps only (T * k <= 32 T pairs: one per thread at most); E <= 32 * NSL
     const int T = P.T, E = P.E, k = P.k, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     {
         const int t = wid, nsl = (E + 31) / 32;
-        Cand *cw = cand + (size_t)t * P.maxc;
-        int nc = 0;
-        // the lane's logits in batches of 8 groups (one round trip per batch when they are all there)
-        constexpr int kPoll = 8;
-#pragma unroll 1
-        for (int sb = 0; sb < nsl; sb += kPoll) {
-            unsigned long long w0[kPoll], w1[kPoll];
+        unsigned long long key[NSL];
+        // the lane's logits, four groups of 32 experts per batch of loads (one round trip when they are all there)
 #pragma unroll
-            for (int q = 0; q < kPoll; ++q) {
-                const int e = (sb + q) * 32 + lane;
-                w0[q] = w1[q] = 0ull;
-                if (sb + q < nsl && e < E) {
-                    const unsigned long long *w = P.logit_ll + 2 * ((size_t)t * E + e);
-                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w0[q]) : "l"(w) : "memory");
-                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w1[q]) : "l"(w + 1) : "memory");
-                }
-            }
+        for (int sb = 0; sb < NSL; sb += 4) {
+            if (sb < nsl) {
+                unsigned long long w0[4], w1[4];
 #pragma unroll
-            for (int q = 0; q < kPoll; ++q) {
-                const int sl = sb + q;
-                if (sl >= nsl) break;
-                const int e = sl * 32 + lane;
-                const bool valid = e < E;
-                double v = 0.0;
-                if (valid) {
-                    if ((unsigned)(w0[q] >> 32) == tag && (unsigned)(w1[q] >> 32) == tag)
-                        v = __longlong_as_double((long long)((w0[q] & 0xffffffffull) | (w1[q] << 32)));
-                    else if (!get_logit(P, t, e, tag, v))
-                        v = 0.0;  // an error is recorded; the layer's result is void
+                for (int q = 0; q < 4; ++q) {
+                    const int e = (sb + q) * 32 + lane;
+                    w0[q] = w1[q] = 0ull;
+                    if (sb + q < nsl && e < E) {
+                        const unsigned long long *w = P.logit_ll + 2 * ((size_t)t * E + e);
+                        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w0[q]) : "l"(w) : "memory");
+                        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w1[q]) : "l"(w + 1) : "memory");
+                    }
                 }
-                const unsigned long long key = valid ? logit_key(v) : 0ull;
-                int rank = 0;
-#pragma unroll 8
-                for (int j = 0; j < 32; ++j) {
-                    const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
-                    rank += (kj > key) | ((kj == key) & (j < lane));
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int e = (sb + q) * 32 + lane;
+                    key[sb + q] = 0ull;  // below every logit's key: never selected while k <= E
+                    if (sb + q < nsl && e < E) {
+                        double v;
+                        if ((unsigned)(w0[q] >> 32) == tag && (unsigned)(w1[q] >> 32) == tag)
+                            v = __longlong_as_double((long long)((w0[q] & 0xffffffffull) | (w1[q] << 32)));
+                        else if (!get_logit(P, t, e, tag, v))
+                            v = 0.0;  // an error is recorded; the layer's result is void
+                        key[sb + q] = logit_key(v);
+                    }
                 }
-                const bool cnd = valid && rank < k;
-                const unsigned mask = __ballot_sync(0xffffffffu, cnd);
-                const int pos = nc + __popc(mask & ((1u << lane) - 1u));
-                if (cnd && pos < P.maxc) cw[pos] = Cand{key, e, 0};
-                nc += __popc(mask);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) key[sb + q] = 0ull;
             }
         }
-        nc = min(nc, P.maxc);
-        __syncwarp();
 #pragma unroll 1
-        for (int ci = lane; ci < nc; ci += 32) {
-            const Cand me = cw[ci];
-            int rank = 0;
-#pragma unroll 4
-            for (int j = 0; j < nc; ++j) {
-                const Cand o = cw[j];
-                rank += (o.key > me.key) | ((o.key == me.key) & (o.e < me.e));
+        for (int r = 0; r < k; ++r) {
+            unsigned long long best = 0ull;
+            int bsl = 0;
+#pragma unroll
+            for (int sl = 0; sl < NSL; ++sl)
+                if (key[sl] > best) {  // strict: the lower group (expert) on equal keys
+                    best = key[sl];
+                    bsl = sl;
+                }
+            const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(best >> 32));
+            const unsigned lo = __reduce_max_sync(0xffffffffu, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
+            const unsigned long long top = ((unsigned long long)hi << 32) | lo;
+            const unsigned e = __reduce_min_sync(0xffffffffu, best == top ? (unsigned)(bsl * 32 + lane) : 0xffffffffu);
+            if (lane == (int)(e & 31u)) {
+#pragma unroll
+                for (int sl = 0; sl < NSL; ++sl)
+                    if (sl == bsl) key[sl] = 0ull;
             }
-            if (rank < k) {
-                S.idx[t * k + rank] = me.e;
-                S.selv[t * k + rank] = key_logit(me.key);
+            if (lane == 0) {
+                S.idx[t * k + r] = (int)e;
+                S.selv[t * k + r] = key_logit(top);
             }
         }
         __syncwarp();
@@ -1345,7 +1345,6 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
     float *xs = reinterpret_cast<float *>(base + P.off_xs); // chunk sums (FFMA) or group sums (MMA)
     uint16_t *hs = reinterpret_cast<uint16_t *>(base + P.off_h);
     float *ybuf = reinterpret_cast<float *>(base + P.off_y);
-    Cand *cand = reinterpret_cast<Cand *>(base + P.off_cand);
     float *part = reinterpret_cast<float *>(base + P.off_part);
     const CtaWork cw = cta_work(P);
     unsigned seq = 0, nbar = 0;
@@ -1377,7 +1376,12 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
         // static region, which need only xe.
         const int nss = min(cw.nshg, P.ua);
         if (wid < T) {
-            topk_bucket(P, S, cand, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
+            if (P.E <= 128)
+                topk_bucket<4>(P, S, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
+            else if (P.E <= 256)
+                topk_bucket<8>(P, S, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
+            else
+                topk_bucket<kMaxSl>(P, S, Pk.layers[l].per_expert_scale, (unsigned)l + 1u);
             if (threadIdx.x == 0) {
                 const int good = ldcg_int(P.err) == 0;
                 S.kverdict = good;
@@ -1848,19 +1852,16 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     slot = std::max(slot, d_slot(P.dcb_s, P.sbd_s, P.pc_s));
     slot = std::max(slot, d_slot(P.dcb_r, P.sbd_r, P.pc_r));
     P.slot_bytes = (int)al(slot, 1024);
-    const int nsl = (w.E + 31) / 32;
-    P.maxc = std::min(w.E, nsl * std::min(w.k, 32));
-    if (P.maxc > dec::kMaxCand) return false;
+    if ((w.E + 31) / 32 > dec::kMaxSl) return false;
     P.yrows = 8 * dec::kMaxBlk;
-    // after the fixed part: static region and ring (1024-aligned), x, xs, h, ybuf, candidates, partials
+    // after the fixed part: static region and ring (1024-aligned), x, xs, h, ybuf, partials
     size_t off = al(sizeof(dec::Shared), 1024);
     P.off_a = (int)off;
     const size_t x_bytes = mma ? (size_t)T * dec::xb_token_bytes(P.CH) : (size_t)T * P.CH * dec::kXStride * 4;
     const size_t xs_bytes = mma ? (size_t)T * P.GH * 4 : (size_t)T * P.CH * 4;
     const size_t part_per_slot = mma ? (size_t)dec::kMaxPieces * 128 * 4 : (size_t)dec::kFfmaPart * 4;
     const size_t fixed_tail = al(x_bytes, 16) + al(xs_bytes, 16) + al((size_t)T * w.H * 2, 16) +
-                              al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16) +
-                              al((size_t)T * P.maxc * sizeof(dec::Cand), 16);
+                              al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16);
     const size_t budget = 227 * 1024 - 1024;  // the base is aligned to 1024 bytes inside the allocation
     // as many of a CTA's shared units in the static region as leave the ring 3 slots or more; else none,
     // and 2 ring slots (every ring task is consumed in its own layer, so 2 slots cannot deadlock)
@@ -1886,8 +1887,6 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     off += al((size_t)T * w.H * 2, 16);
     P.off_y = (int)off;
     off += al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16);
-    P.off_cand = (int)off;
-    off += al((size_t)T * P.maxc * sizeof(dec::Cand), 16);
     P.off_part = (int)off;
     off += (size_t)ns * part_per_slot + a_parts;  // ring slots' partials, then the shared units'
     *smem = off + 1024;
