@@ -1222,10 +1222,11 @@ __device__ __noinline__ bool stage_a_mma(Shared &S, const Cfg &P, int s, bool sh
         ok = __shfl_sync(0xffffffffu, ok, 0);
         __syncwarp();  // the other lanes' loads below come after lane 0's acquire
         if (!ok) return false;
+        // (token, chunk) pairs over the lanes: pcv is even, so lanes w and w ^ 1 hold the two chunks of a group
 #pragma unroll 1
-        for (int tt = 0; tt < n; ++tt) {
+        for (int w0 = 0; w0 < n * pcv; w0 += 32) {
+            const int wq = w0 + lane, tt = wq < n * pcv ? wq / pcv : 0, c = wq < n * pcv ? wq - tt * pcv : pcv;
             const float *src = shd ? P.a_sh + (size_t)tt * P.Is : P.a_r + (size_t)(off + tt) * P.I;
-            const int c = lane;
             float sum = 0.f;
             if (c < pcv) {
                 const float4 *s4 = reinterpret_cast<const float4 *>(src + (p * pc + c) * 32);
@@ -1438,7 +1439,9 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
         const int nrg = cw.rk < nu ? (nu - 1 - cw.rk) / G + 1 : 0;
         const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
         const int ngu = nrg + (cw.nshg - nss);  // ring gate/up units: routed, shared
-        const int npc = kMma ? min(kMaxPieces, max(1, (kCW + max(ngu, 1) - 1) / max(ngu, 1))) : 8;
+        // K-pieces per ring unit: enough for every warp while at most ns units are resident at once
+        const int nres = max(1, min(ngu, ns));
+        const int npc = kMma ? min(kMaxPieces, (kCW + nres - 1) / nres) : 8;
         const int nitems = ngu * npc + ngr * cw.nblk;
 #pragma unroll 1
         for (int i = wid; i < nitems; i += kCW) {

@@ -261,6 +261,33 @@ def test_empty_call_and_output_canaries_and_determinism():
     assert torch.equal(out.view(torch.int16), first.view(torch.int16))   # bit-identical reruns
 
 
+@pytest.mark.parametrize("T,force_path", [(8, 0), (40, 0), (40, 2), (40, 3), (600, 0)])
+def test_layer_forward_replays_from_a_cuda_graph(T, force_path):
+    """Every expert path (GEMV, warp-MMA, tcgen05, and the automatic choice at
+    8, 40 and 600 tokens) can be captured in a CUDA graph after one eager
+    call: the host side of a call queries nothing that a capture refuses, and
+    the replay gives the eager output bit for bit."""
+    cfg = synth.CONFIGS[0]
+    D = moe.DeviceLayer.from_config(synth.gen_layer(cfg, 0, 0, device="cuda"), cfg)
+    h = synth.gen_hidden(cfg, 0, 5, T).cuda()
+    ws = moe.workspace(D, T)
+    opts = moe.make_opts(force_path=force_path)
+    eager = torch.empty_like(h)
+    moe.moe_layer_forward(D, h, eager, T, ws, opts)
+    torch.cuda.synchronize()
+    moe.moe_workspace_status(ws)
+    out = torch.full_like(h, float("nan"))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        moe.moe_layer_forward(D, h, out, T, ws, opts)
+    g.replay()
+    torch.cuda.synchronize()
+    moe.moe_workspace_status(ws)
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+
+
 # ------------------------------------------------------------------ full-size stack
 
 def test_full_decode_stack_teacher_forced_on_sampled_layers():
