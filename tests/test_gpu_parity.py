@@ -70,7 +70,7 @@ def test_prepare_qmat_matches_the_documented_tiled_layout():
 
 # ------------------------------------------------------------------ router
 
-@pytest.mark.parametrize("cfg_id,T", [(0, 4), (1, 8), (2, 8), (3, 4), (4, 37)])
+@pytest.mark.parametrize("cfg_id,T", [(0, 4), (1, 8), (2, 8), (3, 4), (4, 37), (2, 16), (3, 20)])
 def test_router_matches_oracle(cfg_id, T):
     cfg, w, D, OL = case(cfg_id if cfg_id != 4 else 1)
     h = hidden(cfg_id, cfg, OL, T, stream=3, layer_w=w)
