@@ -148,7 +148,7 @@ cudaError_t launch_fill(const moe_layer_w *w, const moe_qmat pool[3], const moe_
         a.total += per[k];
     }
     int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);  // the launches' device (stream queries are refused while capturing)
+    cudaError_t e = stream_device(st, &dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     fill_kernel<<<2 * sms, 256, 0, st>>>(a, miss);

@@ -388,9 +388,8 @@ static cudaError_t launch_qmat_gemv_nt(const moe_qmat &w, int rows, int cols, co
     cudaError_t e = ensure_smem(fn, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per = 0;
-    // the SM count of the current device, which runs the kernel (no stream query: a CUDA-graph capture
-    // refuses those)
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    // the SM count of the device that runs the kernel
+    if ((e = stream_device(st, &dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kQgWarps * 32, smem)) != cudaSuccess) return e;
     const int nrb = rows / kRowBlock;

@@ -12,6 +12,21 @@ namespace moe {
 // Record `msg` as this host thread's moe_last_error() text; returns `code`.
 int set_last_error(int code, const char *msg);
 
+// The device that runs launches on `st`: the stream's own (NULL: the current
+// device).  While `st` is being captured into a CUDA graph the current device
+// is taken instead (the captured launches run there): asking a capturing
+// stream for its device ended the capture on the warp-MMA path, and the
+// capture-status query is the one stream query a capture allows.
+inline cudaError_t stream_device(cudaStream_t st, int *dev) {
+    if (st) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        const cudaError_t e = cudaStreamIsCapturing(st, &cs);
+        if (e != cudaSuccess) return e;
+        if (cs == cudaStreamCaptureStatusNone) return cudaStreamGetDevice(st, dev);
+    }
+    return cudaGetDevice(dev);
+}
+
 // Raise a kernel's dynamic shared memory limit once (per process) to at
 // least `bytes`.  A no-op below 48 KiB.
 cudaError_t ensure_smem(const void *kernel, size_t bytes);

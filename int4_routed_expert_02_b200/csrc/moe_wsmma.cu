@@ -413,12 +413,10 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
     }
 }
 
-// SM count of the current device (the launches go to its streams).  Stream
-// queries are not used: they are refused while a stream is being captured
-// into a CUDA graph.
-int sms_of() {
+// SM count of the device that runs launches on `st`.
+int sms_of(cudaStream_t st) {
     int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (stream_device(st, &dev) != cudaSuccess) return 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     return n;
 }
@@ -436,7 +434,7 @@ cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T,
     const int Kmax = I > Is ? I : Is;
     cudaError_t e = launch_gather_tokens(xe, perm, T, k, H, b.xg, st);
     if (e != cudaSuccess) return e;
-    const int sms = sms_of();
+    const int sms = sms_of(st);
     if (sms <= 0) return cudaErrorNoDevice;
     const long long pairs = (long long)T * k;
     const long long max_active = pairs < w->E ? pairs : w->E;

@@ -86,3 +86,26 @@ def test_qmat_gemv_rejects_bad_arguments():
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_qmat_gemv(qt, sbt, rows, cols, x, 1, y, ws[:8])
     assert ei.value.code == moe.MOE_EWORKSPACE
+
+
+def test_qmat_gemv_replays_from_a_cuda_graph_on_a_side_stream():
+    """Captured on a non-default stream after one eager call, the head GEMV
+    replays to the eager result bit for bit (the launch sizes its grid for
+    the stream's device without a query that the capture refuses)."""
+    rows, cols, T = 1024, 2816, 2
+    _, qt, sbt = _head(rows, cols, 5)
+    x = _x(T, cols, 6).cuda()
+    ws = moe.qmat_gemv_workspace()
+    eager = torch.empty(T, rows, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.moe_qmat_gemv(qt, sbt, rows, cols, x, T, eager, ws, stream=s)
+    s.synchronize()
+    out = torch.full_like(eager, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        moe.moe_qmat_gemv(qt, sbt, rows, cols, x, T, out, ws, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
