@@ -180,10 +180,12 @@ def _distinct_experts(st, moe, cfg, T):
     return tot / st.L
 
 
-def _expert_roofline(st, moe, cfg, T, hbm, dev, opts=None):
+def _expert_roofline(st, moe, cfg, T, hbm, dev, opts=None, split_shared=False):
     """Per-launch time of the expert part (moe_expert_ffn: gate/up + down +
     weighted sum) on each layer's real input, against the HBM roofline of
-    the distinct experts it reads."""
+    the distinct experts it reads.  split_shared: also time the same calls
+    without the shared expert, so that its share can be reported apart (the
+    time with it minus the time without it)."""
     L = st.L
     bufs = []
     for l in range(L):
@@ -201,25 +203,33 @@ def _expert_roofline(st, moe, cfg, T, hbm, dev, opts=None):
     ws2 = moe.workspace(st.layers[0], T, device=dev)
     stream = torch.cuda.current_stream(dev)
     reps = 3
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L * reps)]
-    for r in range(reps):
-        for l in range(L):
-            xe, idx, wts, offsets, perm, active = bufs[l]
-            a, b = evs[r * L + l]
-            a.record(stream)
-            moe.moe_expert_ffn(st.layers[l], xe, T, idx, wts, offsets, perm, active, 1, m, ws2, opts)
-            b.record(stream)
-    torch.cuda.synchronize(dev)
-    moe.moe_workspace_status(ws2)
-    times = [a.elapsed_time(b) for a, b in evs[L:]]  # drop the first (warm) repetition
-    us = statistics.mean(times) * 1e3
+
+    def timed(with_shared):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L * reps)]
+        for r in range(reps):
+            for l in range(L):
+                xe, idx, wts, offsets, perm, active = bufs[l]
+                a, b = evs[r * L + l]
+                a.record(stream)
+                moe.moe_expert_ffn(st.layers[l], xe, T, idx, wts, offsets, perm, active, with_shared, m, ws2, opts)
+                b.record(stream)
+        torch.cuda.synchronize(dev)
+        moe.moe_workspace_status(ws2)
+        times = [a.elapsed_time(b) for a, b in evs[L:]]  # drop the first (warm) repetition
+        return statistics.mean(times) * 1e3
+
+    us = timed(1)
+    us_routed = timed(0) if split_shared else None
     d = statistics.mean(int(torch.unique(bufs[l][1]).numel()) for l in range(L))
     nbytes = d * expert_bytes(3 * cfg.I * cfg.H) + expert_bytes(3 * cfg.Is * cfg.H)
     achieved = nbytes / (us / 1e6) / 1e9
-    return {"kernel": "expert FFN per layer call (moe_expert_ffn)", "bound": "hbm", "achieved": round(achieved, 1),
-            "peak": hbm["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / hbm["hbm_gbs"], 4),
-            "peak_source": hbm["source"] + " (burst copy)", "traffic": None, "bytes_per_launch": int(nbytes),
-            "us_per_launch": round(us, 3), "distinct_experts": round(d, 2)}
+    out = {"kernel": "expert FFN per layer call (moe_expert_ffn)", "bound": "hbm", "achieved": round(achieved, 1),
+           "peak": hbm["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / hbm["hbm_gbs"], 4),
+           "peak_source": hbm["source"] + " (burst copy)", "traffic": None, "bytes_per_launch": int(nbytes),
+           "us_per_launch": round(us, 3), "distinct_experts": round(d, 2)}
+    if us_routed is not None:
+        out["us_routed_only"] = round(us_routed, 3)
+    return out
 
 
 def _e2e(st, cfg, T, K, W, inputs, dev):
@@ -373,7 +383,7 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0
     ms = e0.elapsed_time(e1)
     st.status()
     hbm = peaks()
-    roof = _expert_roofline(st, moe, cfg, T, hbm, dev, opts)
+    roof = _expert_roofline(st, moe, cfg, T, hbm, dev, opts, split_shared=True)
     fl = expert_flops(cfg, T)
     tflops = fl / (roof["us_per_launch"] / 1e6) / 1e12
     peak_t = hbm["bf16_tflops"]  # FP16 and BF16 share the dense tensor rate
@@ -394,7 +404,22 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0
                            "hbm_frac": roof["frac"], "bytes_per_launch": roof["bytes_per_launch"],
                            "binding_roof_frac": round(bound_us / roof["us_per_launch"], 4),
                            "traffic": traffic,
-                           "peak_source": hbm["source"] + " (bf16 dense burst; FP16 same rate; copy bandwidth)"}}, st
+                           "peak_source": hbm["source"] + " (bf16 dense burst; FP16 same rate; copy bandwidth)",
+                           "split": split_roofline(cfg, T, roof, peak_t)}}, st
+
+
+def split_roofline(cfg, T, roof, peak_t):
+    """The routed experts and the shared expert apart: the routed part is the
+    same call without the shared expert; the shared part is the difference
+    (time with it minus time without it)."""
+    us_r = roof["us_routed_only"]
+    us_s = roof["us_per_launch"] - us_r
+    fl_r = 2.0 * T * 3.0 * cfg.I * cfg.H * cfg.k
+    fl_s = 2.0 * T * 3.0 * cfg.Is * cfg.H
+    part = lambda fl, us: ({"us": round(us, 3), "tflops": round(fl / (us / 1e6) / 1e12, 2),
+                           "tensor_frac": round(fl / (us / 1e6) / 1e12 / peak_t, 4)} if us > 0 else {"us": round(us, 3)})
+    return {"routed": part(fl_r, us_r), "shared_expert": part(fl_s, us_s),
+            "how": "routed: the call without the shared expert; shared: the call's time with it minus without it"}
 
 
 HEAD_ROWS = 262_144  # vocabulary rows of the output head (synthetic: the pages give no vocabulary size)
