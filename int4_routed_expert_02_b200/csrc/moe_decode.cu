@@ -548,7 +548,11 @@ __device__ __noinline__ void router_compute(const Cfg &P, Shared &S, const unsig
     const RouterCopy rc = router_copy(P);
     const int items = rc.nrows * T;
     if (items > 0) {
-        const int parts = items >= kCW ? 1 : kCW / items, units = items * parts, nch = H / 16;
+        // the K-split is the one of the CTAs with the most rows, in every CTA: a logit's summation order
+        // then does not depend on which CTA computes it, so experts with equal router rows get equal
+        // logits (and the tie rule decides between them, as in the per-layer router)
+        const int maxi = (P.E + (int)gridDim.x - 1) / (int)gridDim.x * T;
+        const int parts = maxi >= kCW ? 1 : kCW / maxi, units = items * parts, nch = H / 16;
         const uint16_t *rsc = reinterpret_cast<const uint16_t *>(slot);
         const unsigned char *rows = slot + 2 * H;
         const int sb_skip = (int)((size_t)rc.e0 * G * 2) - (int)rc.sb_lo;

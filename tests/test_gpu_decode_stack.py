@@ -52,15 +52,63 @@ def test_decode_stack_matches_per_layer_path_and_oracle(cfg_id, T, L, path):
         _check_stack(st, cfg, cfg_id, oracle_layers=(0, L - 1) if step == 1 else ())
 
 
-def test_decode_stack_unchained_zipf_inputs():
+@pytest.mark.parametrize("T", [1, 2])
+def test_decode_stack_unchained_zipf_inputs(T):
+    """512 experts (16 groups of 32 in the kernel's top-k) with the Zipf-routed
+    inputs, on the CUDA-core (T = 1) and the tensor-core (T = 2) variants."""
     cfg = synth.CONFIGS[3]
-    L, T = 3, 2
+    L = 3
     st = MoEStack(cfg, 3, T=T, layers=L, keep_router_codes=True)
     h = torch.stack([synth.gen_zipf_hidden(cfg, 3, l, 0, st.router_codes[l], T=T)[0] for l in range(L)])
     st.set_input(h.cuda())
     st.run()
     torch.cuda.synchronize()
     _check_stack(st, cfg, 3, oracle_layers=(1,))
+
+
+@pytest.mark.parametrize("cfg_id,T,tie", [(1, 1, "all"), (1, 2, "pairs"), (2, 1, "pairs"), (3, 1, "all"),
+                                           (3, 2, "pairs")])
+def test_decode_stack_top_k_ties_go_to_the_lower_index(cfg_id, T, tie):
+    """Router rows made identical, so that logits tie exactly: "all" (every
+    expert the same: the top k must be experts 0..k-1) or "pairs" (expert e
+    and e + E/2 the same: the two sit in different groups of 32 for E >= 64,
+    and the lower one must win where the pair straddles the k-th place).  The
+    experts' own weights differ, so a wrong pick changes the output far beyond
+    the bar; the kernel is checked against the oracle and the per-layer path."""
+    cfg = synth.CONFIGS[cfg_id]
+    L = 2
+    ws_, OLs, Ds = [], [], []
+    for l in range(L):
+        w = synth.gen_layer(cfg, cfg_id, l, device="cuda")
+        if tie == "all":
+            for key in ("router_q", "router_s", "router_b"):
+                w[key][:] = w[key][0]
+        else:
+            half = cfg.E // 2
+            for key in ("router_q", "router_s", "router_b"):
+                w[key][half:] = w[key][:half]
+        Ds.append(moe.DeviceLayer.from_config(w, cfg))
+        OLs.append(oracle_layer(host(w), cfg))
+    st = MoEStack(cfg, cfg_id, T=T, layers=L, device_layers=Ds)
+    assert st.persistent
+    h = synth.gen_hidden(cfg, cfg_id, 900, T).cuda()
+    if not cfg.chained:
+        h = h.unsqueeze(0).expand(L, T, cfg.H).contiguous()
+    st.set_input(h)
+    st.run()
+    torch.cuda.synchronize()
+    st.status()
+    ws = moe.workspace(st.layers[0], T)
+    for l in range(L):
+        h_in = st.inputs[l]
+        ref = torch.empty_like(h_in)
+        moe.moe_layer_forward(st.layers[l], h_in, ref, T, ws)
+        torch.cuda.synchronize()
+        assert_same_up_to_one_rounding(st.outputs[l], ref)
+        out = oracle.layer_forward(OLs[l], h_in.cpu())
+        if tie == "all":
+            assert all(list(r) == list(range(cfg.k)) for r in out["idx"])
+        assert max_err_vs_rms(bf16_host(st.outputs[l]), out["out_f64"]) <= OUT_TOL
 
 
 @pytest.mark.parametrize("dims", [
