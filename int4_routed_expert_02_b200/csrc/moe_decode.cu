@@ -70,6 +70,8 @@ constexpr int kMaxLayers = 64;
 constexpr int kMaxPairs = kMaxT * kMaxK;      // 256
 constexpr int kMaxSlots = 16;                 // ring slots
 constexpr int kMaxA = 9;                      // the static region's tasks: router rows + up to 8 shared units
+constexpr int kXmBlk = 4;                     // expert-major down items: 8-row blocks per item (one 32-row block)
+constexpr int kMaxStage = 3;                  // expert-major down: experts whose SwiGLU input a CTA stages per layer
 constexpr int kMaps = 12;                     // TMA tensor maps per layer
 constexpr int kMaxBlk = 4;                    // 8-row output blocks per CTA (H <= 4096 on >= 128 SMs)
 constexpr int kMaxParts = 8;                  // K-parts of a down matrix
@@ -118,6 +120,11 @@ struct Cfg {
     float *a_r;                  // [T*k,I]  of the routed experts, by bucketed position
     float *m;                    // [T,H]    combine of the current layer
     const CUtensorMap *maps;     // [L][kMaps]
+    int xm;                      // tensor-core variant: routed down work by expert (see consumer_main)
+    int ipe;                     // expert-major down items per expert (H / 32)
+    int stage_bytes, off_stage;  // expert-major down: one expert's staged input, and where they sit
+    int nstage;                  // expert-major down: staged experts a CTA has room for (<= kMaxStage)
+    float *y_r;                  // [T*k,H]  expert-major down: routed outputs by pair id
 };
 
 struct Params {
@@ -153,6 +160,7 @@ struct Shared {
     double rpart[kCW];                     // router partial sums (fewer items than warps)
     int toks_sh[kMaxT];                    // 0, 1, ..., T-1
     Cfg c;
+    volatile int xstate[kMaxStage];        // expert-major down: as astate, for each staged expert
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -1214,11 +1222,11 @@ __device__ __forceinline__ DGroup dgroup(const Cfg &P, int gi) {
 // ([n][pc][t][16 bf16] + padding per token) and the 64-column sums of hi + lo
 // ([n][pc/2], fp32).  One lane per 32-column chunk; the first warp of the
 // group stages, the others wait (as stage_a).
-__device__ __noinline__ bool stage_a_mma(Shared &S, const Cfg &P, int s, bool shd, int j, int p, int pc, int pcv,
-                                         int n, int off, unsigned char *ahl, float *asg) {
+__device__ __noinline__ bool stage_a_mma(Shared &S, const Cfg &P, volatile int *state, bool shd, int j, int p, int pc,
+                                         int pcv, int n, int off, unsigned char *ahl, float *asg) {
     const int lane = threadIdx.x & 31;
     int mine = 0, ok = 1;
-    if (lane == 0) mine = atomicCAS(const_cast<int *>(&S.astate[s]), 0, 1) == 0;
+    if (lane == 0) mine = atomicCAS(const_cast<int *>(state), 0, 1) == 0;
     mine = __shfl_sync(0xffffffffu, mine, 0);
     if (mine) {
         const int ri = shd ? 0 : 1 + j;
@@ -1259,12 +1267,12 @@ __device__ __noinline__ bool stage_a_mma(Shared &S, const Cfg &P, int s, bool sh
         }
         __syncwarp();
         __threadfence_block();
-        if (lane == 0) S.astate[s] = 2;
+        if (lane == 0) *state = 2;
         return true;
     }
     if (lane == 0) {
         const unsigned long long t0 = globaltimer();
-        for (unsigned it = 0; S.astate[s] != 2; ++it) {
+        for (unsigned it = 0; *state != 2; ++it) {
             if ((it & 63u) == 63u && (ldcg_int(P.err) != 0 || globaltimer() - t0 > kWaitNs)) {
                 atomicCAS(P.err, 0, kErrStage);
                 ok = 0;
@@ -1394,6 +1402,8 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                     S.exp_ready[0] += (unsigned)P.units_s;
                     for (int j = 0; j < S.D; ++j) S.exp_ready[1 + j] += (unsigned)P.units_r;
                 }
+                if (P.xm)
+                    for (int i = 0; i < kMaxStage; ++i) S.xstate[i] = 0;  // this layer's experts are not staged yet
                 __threadfence_block();
                 S.tables_layer = l + 1;  // the producer and the other warps may go on
             }
@@ -1441,12 +1451,18 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
         // then the down blocks
         const int D = S.D, nu = D * P.units_r;
         const int nrg = cw.rk < nu ? (nu - 1 - cw.rk) / G + 1 : 0;
-        const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
+        // down groups by output rows: the shared expert's, and (unless the routed down work goes by
+        // expert) every routed slot's
+        const int ngr = cw.nblk > 0 ? P.parts_s + ((kMma && P.xm) ? 0 : D * P.parts_r) : 0;
         const int ngu = nrg + (cw.nshg - nss);  // ring gate/up units: routed, shared
+        // expert-major routed down items [xg0, xg1) of the grid's D * ipe (expert, 32-row block) items
+        const int xtot = (kMma && P.xm) ? D * P.ipe : 0;
+        const int xg0 = kMma ? (int)((long long)xtot * c / G) : 0, xg1 = kMma ? (int)((long long)xtot * (c + 1) / G) : 0;
+        const int nxm = xg1 - xg0, xj0 = kMma && nxm > 0 ? xg0 / P.ipe : 0;
         // K-pieces per ring unit: enough for every warp while at most ns units are resident at once
         const int nres = max(1, min(ngu, ns));
         const int npc = kMma ? min(kMaxPieces, (kCW + nres - 1) / nres) : 8;
-        const int nitems = ngu * npc + ngr * cw.nblk;
+        const int nitems = ngu * npc + ngr * cw.nblk + nxm * kXmBlk;
 #pragma unroll 1
         for (int i = wid; i < nitems; i += kCW) {
             if (i < ngu * npc) {
@@ -1487,6 +1503,32 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                     piece_done_ffma<NT>(part + (size_t)s * kFfmaPart, &S.cnt[s], &S.empty[s], rdy, pi, n, g, uu, adst,
                                         ip, lda, row0);
                 }
+            } else if (kMma && i >= ngu * npc + ngr * cw.nblk) {
+                // expert-major routed down: item xi (expert j, 32-row block q), block bi of it, against the
+                // expert's input staged once in this CTA
+                const int xi = (i - ngu * npc - ngr * cw.nblk) / kXmBlk, bi = (i - ngu * npc - ngr * cw.nblk) % kXmBlk;
+                const int g = xg0 + xi, j = g / P.ipe, q = g - j * P.ipe;
+                const unsigned tseq = seq + (unsigned)(ngu + ngr + xi);
+                if (!wait_task(S, P, tseq)) break;
+                const int n = S.slot_n[j], off = S.slot_off[j], si = j - xj0;
+                if (si >= P.nstage) {  // the plan bounds the experts per CTA; never expected
+                    if (lane == 0) atomicCAS(P.err, 0, kErrStage);
+                    break;
+                }
+                unsigned char *area = base + P.off_stage + (size_t)si * P.stage_bytes;
+                float *asg = reinterpret_cast<float *>(area + (size_t)n * ahl_token_bytes(P.pc_r));
+                if (!stage_a_mma(S, P, &S.xstate[si], false, j, 0, P.pc_r, P.pc_r, n, off, area, asg)) break;
+                const int s = (int)(tseq % (unsigned)ns);
+                const unsigned char *slot = ring + (size_t)s * P.slot_bytes;
+                float y[2];
+                d_block_mma(slot + bi * P.dcb_r, slot + kXmBlk * P.dcb_r + bi * P.sbd_r, area, asg, P.pc_r, P.pc_r, n,
+                            y);
+                const int g8 = lane >> 2, t4 = lane & 3;
+                if (g8 < n) {
+                    float *dst = P.y_r + (size_t)S.pos_pair[off + g8] * H + (q * kXmBlk + bi) * 8 + 2 * t4;
+                    *reinterpret_cast<float2 *>(dst) = make_float2(y[0], y[1]);
+                }
+                block_done(S, P, tseq, kXmBlk);
             } else {
                 const int di = i - ngu * npc, gi = di / cw.nblk, bi = di - gi * cw.nblk;
                 const unsigned tseq = seq + (unsigned)(ngu + gi);
@@ -1499,12 +1541,13 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                 const unsigned char *codes = slot + bi * dg.dcb, *sbp = slot + cw.nblk * dg.dcb + bi * dg.sbd;
                 if (kMma) {
                     float *asg = reinterpret_cast<float *>(area + (size_t)n * ahl_token_bytes(dg.pc));
-                    if (!stage_a_mma(S, P, s, dg.shd, dg.j, dg.p, dg.pc, dg.pcv, n, off, area, asg)) break;
+                    if (!stage_a_mma(S, P, &S.astate[s], dg.shd, dg.j, dg.p, dg.pc, dg.pcv, n, off, area, asg)) break;
                     float y[2];
                     d_block_mma(codes, sbp, area, asg, dg.pc, dg.pcv, n, y);
                     const int g8 = lane >> 2, t4 = lane & 3;
                     if (g8 < n) {
-                        const int entry = dg.shd ? T * P.k * P.parts_r + dg.p * T + g8
+                        // by expert, the routed outputs go to global memory and ybuf keeps the shared ones only
+                        const int entry = dg.shd ? (P.xm ? 0 : T * P.k * P.parts_r) + dg.p * T + g8
                                                  : S.pos_pair[off + g8] * P.parts_r + dg.p;
                         ybuf[(size_t)entry * P.yrows + bi * 8 + 2 * t4] = y[0];
                         ybuf[(size_t)entry * P.yrows + bi * 8 + 2 * t4 + 1] = y[1];
@@ -1530,8 +1573,13 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
                 block_done(S, P, tseq, cw.nblk);
             }
         }
-        seq += (unsigned)(ngu + ngr);
+        seq += (unsigned)(ngu + ngr + nxm);
         consumer_sync();
+        if (kMma && P.xm) {  // every CTA's routed outputs are written before any CTA sums its rows
+            if (!ok) break;
+            if (threadIdx.x == 0) grid_arrive(P);
+            if (!(ok = grid_wait(P, S, ++nbar))) break;
+        }
         // ---------------------------------------------------------- the combine of this CTA's rows
         if (cw.nblk > 0) {
             const int nrows = cw.nblk * 8, r0 = cw.b0 * 8, k = P.k, pr = P.parts_r;
@@ -1542,11 +1590,15 @@ __device__ __noinline__ void consumer_main(const Params &Pk, Shared &S, unsigned
 #pragma unroll 1
                 for (int s2 = 0; s2 < k; ++s2) {
                     float ys = 0.f;
-                    for (int p = 0; p < pr; ++p) ys += ybuf[(size_t)((t * k + s2) * pr + p) * P.yrows + r];
+                    if (kMma && P.xm)  // written by the CTAs that own the expert's rows (before the barrier above)
+                        ys = __ldcg(P.y_r + (size_t)(t * k + s2) * H + r0 + r);
+                    else
+                        for (int p = 0; p < pr; ++p) ys += ybuf[(size_t)((t * k + s2) * pr + p) * P.yrows + r];
                     acc = fmaf(S.wts[t * k + s2], ys, acc);
                 }
                 float sh = 0.f;
-                for (int p = 0; p < P.parts_s; ++p) sh += ybuf[(size_t)(T * k * pr + p * T + t) * P.yrows + r];
+                const int sh0 = (kMma && P.xm) ? 0 : T * k * pr;
+                for (int p = 0; p < P.parts_s; ++p) sh += ybuf[(size_t)(sh0 + p * T + t) * P.yrows + r];
                 P.m[(size_t)t * H + r0 + r] = acc + sh;
             }
         }
@@ -1617,6 +1669,7 @@ __device__ __forceinline__ int down_rb(const Cfg &P, const Shared &S, const DGro
     return (dg.shd ? 0 : S.slot_e[dg.j] * (P.H / 32)) + (b >> 2);
 }
 
+template <bool kMma>
 __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned char *base) {
     if ((threadIdx.x & 31) != 0) return;
     const Cfg &P = S.c;
@@ -1653,7 +1706,9 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
         const CUtensorMap *mp = P.maps + (size_t)l * kMaps;
         const int D = S.D, nu = D * P.units_r;
         const int nrg = cw.rk < nu ? (nu - 1 - cw.rk) / G + 1 : 0;
-        const int ngr = cw.nblk > 0 ? P.parts_s + D * P.parts_r : 0;
+        const int ngr = cw.nblk > 0 ? P.parts_s + ((kMma && P.xm) ? 0 : D * P.parts_r) : 0;
+        const int xtot = (kMma && P.xm) ? D * P.ipe : 0;
+        const int xg0 = kMma ? (int)((long long)xtot * c / G) : 0, xg1 = kMma ? (int)((long long)xtot * (c + 1) / G) : 0;
         // routed gate/up units first (the layer's critical path); once the ring is full, the rest of them
         // are asked into L2 before the loop waits for free slots
         const unsigned ubytes = 2u * P.CH * 128u + 2u * P.GH * 32u;
@@ -1722,6 +1777,22 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             }
             ++seq;
         }
+        // expert-major routed down items: expert j's 32-row block q (four 8-row blocks), in item order
+#pragma unroll 1
+        for (int g = xg0; g < xg1 && ok; ++g) {
+            const int j = g / P.ipe, q = g - j * P.ipe, rb = S.slot_e[j] * (P.H / 32) + q;
+            unsigned char *dst = claim(S, P, ring, seq, (unsigned)kXmBlk * (unsigned)(P.pc_r * 128 + P.pc_r * 16));
+            if (!dst) {
+                ok = false;
+                break;
+            }
+            unsigned long long *fb = &S.full[seq % (unsigned)ns];
+            for (int bi = 0; bi < kXmBlk; ++bi) {
+                tma_load_3d(dst + bi * P.dcb_r, mp + kMapDownQ, 32 * bi, 0, rb, fb);
+                tma_load_3d(dst + kXmBlk * P.dcb_r + bi * P.sbd_r, mp + kMapDownSb, 8 * bi, 0, rb, fb);
+            }
+            ++seq;
+        }
     }
     // let this thread's copies land before the CTA ends (bounded)
     for (unsigned q = seq > (unsigned)ns ? seq - (unsigned)ns : 0u; q < seq; ++q)
@@ -1763,7 +1834,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     }
     __syncthreads();
     if ((threadIdx.x >> 5) == kProdWarp) {
-        producer_main(Pk, S, base);  // lane 0 works, the other lanes return at once
+        producer_main<MMA>(Pk, S, base);  // lane 0 works, the other lanes return at once
         __syncwarp();
     } else {
         consumer_main<NT, MMA>(Pk, S, base);
@@ -1780,7 +1851,7 @@ namespace {
 size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct DecodeWs {
-    size_t ctl, ready, zero_bytes, logits, a_sh, a_r, m, maps, total;
+    size_t ctl, ready, zero_bytes, logits, a_sh, a_r, m, y_r, maps, total;
 };
 
 // Workspace: control words (barrier counters 128 bytes apart; the status word
@@ -1802,6 +1873,9 @@ DecodeWs decode_ws(const moe_layer_w *w, int T) {
     d.a_r = take(sizeof(float) * (size_t)T * w->k * w->I);
     d.m = take(sizeof(float) * (size_t)T * w->H);
     d.maps = take(sizeof(CUtensorMap) * dec::kMaxLayers * dec::kMaps, 128);
+    // expert-major down (T >= 4 only): routed outputs by pair.  Below that the workspace keeps its size
+    // (and its control words their placement: one 90 KB larger at T = 1 timed 1.5 % slower)
+    d.y_r = take(T >= 4 ? sizeof(float) * (size_t)T * w->k * w->H : 0);
     d.total = al(off, 256);
     return d;
 }
@@ -1817,7 +1891,7 @@ void down_parts(int K, int *parts, int *pc) {
 
 // The kernel's shared-memory plan for layers shaped like w, T tokens, a grid
 // of `grid` CTAs; false if it does not fit.
-bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, size_t *smem) {
+bool decode_plan_xm(const moe_layer_w &w, int T, int grid, bool mma, bool allow_xm, dec::Cfg &P, size_t *smem) {
     if (grid <= 0 || T < 1 || T > dec::kMaxT || (long)T * w.H > dec::kMaxStageTH || w.H > 4096) return false;
     if ((long)T * w.k > dec::kMaxPairs) return false;
     P.H = w.H;
@@ -1854,10 +1928,31 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     const int nshg_max = (P.units_s + grid - 1) / grid;
     P.a_rbytes = (int)al(r_slot, 1024);
     P.a_ubytes = (int)al(g_slot, 1024);
-    // ring: routed gate/up units and down groups
+    // from 4 tokens on, the tensor-core variant does the routed down work by expert: a CTA takes a run
+    // of (expert, 32-row block) items and stages each of its experts' input once; it needs one K-part per
+    // routed down matrix, and room for the experts a run can reach (measured: T = 8 1592 -> 1948 tok/s,
+    // T = 4 1630 -> 1716 on the Qwen-35B shape; T = 2 slower, 1270 -> 1203)
+    P.xm = 0;
+    P.ipe = w.H / 32;
+    P.nstage = 0;
+    P.stage_bytes = 0;
+    if (allow_xm && mma && T >= 4 && P.parts_r == 1) {
+        const long dmax = std::min((long)w.E, (long)T * w.k);
+        const long itmax = (dmax * P.ipe + grid - 1) / grid;
+        const long reach = (itmax + P.ipe - 1) / P.ipe + 1;
+        if (reach <= dec::kMaxStage) {
+            P.xm = 1;
+            P.nstage = (int)reach;
+            P.stage_bytes = (int)al((size_t)T * dec::ahl_token_bytes(P.pc_r) + (size_t)T * (P.pc_r / 2) * 4, 128);
+        }
+    }
+    // ring: routed gate/up units and down groups (by output rows, or by expert)
     size_t slot = g_slot;
     slot = std::max(slot, d_slot(P.dcb_s, P.sbd_s, P.pc_s));
-    slot = std::max(slot, d_slot(P.dcb_r, P.sbd_r, P.pc_r));
+    if (P.xm)
+        slot = std::max(slot, (size_t)dec::kXmBlk * (P.dcb_r + P.sbd_r));
+    else
+        slot = std::max(slot, d_slot(P.dcb_r, P.sbd_r, P.pc_r));
     P.slot_bytes = (int)al(slot, 1024);
     if ((w.E + 31) / 32 > dec::kMaxSl) return false;
     P.yrows = 8 * dec::kMaxBlk;
@@ -1867,8 +1962,11 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     const size_t x_bytes = mma ? (size_t)T * dec::xb_token_bytes(P.CH) : (size_t)T * P.CH * dec::kXStride * 4;
     const size_t xs_bytes = mma ? (size_t)T * P.GH * 4 : (size_t)T * P.CH * 4;
     const size_t part_per_slot = mma ? (size_t)dec::kMaxPieces * 128 * 4 : (size_t)dec::kFfmaPart * 4;
+    const size_t stage_all = (size_t)P.nstage * P.stage_bytes;
+    // down outputs of this CTA's rows: routed by pair and shared, or (by expert) the shared ones only
+    const size_t ybuf_bytes = (size_t)((P.xm ? 0 : T * w.k * P.parts_r) + P.parts_s * T) * P.yrows * 4;
     const size_t fixed_tail = al(x_bytes, 16) + al(xs_bytes, 16) + al((size_t)T * w.H * 2, 16) +
-                              al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16);
+                              al(ybuf_bytes, 16) + (stage_all ? stage_all + 128 : 0);
     const size_t budget = 227 * 1024 - 1024;  // the base is aligned to 1024 bytes inside the allocation
     // as many of a CTA's shared units in the static region as leave the ring 3 slots or more; else none,
     // and 2 ring slots (every ring task is consumed in its own layer, so 2 slots cannot deadlock)
@@ -1893,11 +1991,19 @@ bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, s
     P.off_h = (int)off;
     off += al((size_t)T * w.H * 2, 16);
     P.off_y = (int)off;
-    off += al((size_t)(T * w.k * P.parts_r + P.parts_s * T) * P.yrows * 4, 16);
+    off += al(ybuf_bytes, 16);
     P.off_part = (int)off;
     off += (size_t)ns * part_per_slot + a_parts;  // ring slots' partials, then the shared units'
+    if (stage_all) off = al(off, 128);
+    P.off_stage = (int)off;
+    off += stage_all;
     *smem = off + 1024;
     return *smem <= 227 * 1024;
+}
+
+// The plan with the routed down work by expert where it fits, else by output rows.
+bool decode_plan(const moe_layer_w &w, int T, int grid, bool mma, dec::Cfg &P, size_t *smem) {
+    return decode_plan_xm(w, T, grid, mma, true, P, smem) || decode_plan_xm(w, T, grid, mma, false, P, smem);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -2074,6 +2180,7 @@ cudaError_t launch_decode_stack(const moe_layer_w *layers, int L, const uint16_t
     P.a_sh = reinterpret_cast<float *>(base + d.a_sh);
     P.a_r = reinterpret_cast<float *>(base + d.a_r);
     P.m = reinterpret_cast<float *>(base + d.m);
+    P.y_r = reinterpret_cast<float *>(base + d.y_r);
     P.maps = reinterpret_cast<const CUtensorMap *>(base + d.maps);
 
     const void *fn = kernel_for(T, mma);
