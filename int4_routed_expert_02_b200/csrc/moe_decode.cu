@@ -70,7 +70,7 @@ constexpr int kMaxLayers = 64;
 constexpr int kMaxPairs = kMaxT * kMaxK;      // 256
 constexpr int kMaxSlots = 16;                 // ring slots
 constexpr int kMaxA = 9;                      // the static region's tasks: router rows + up to 8 shared units
-constexpr int kXmBlk = 4;                     // expert-major down items: 8-row blocks per item (one 32-row block)
+constexpr int kXmBlk = 8;                     // expert-major down items: 8-row blocks per item (a multiple of 4)
 constexpr int kMaxStage = 3;                  // expert-major down: experts whose SwiGLU input a CTA stages per layer
 constexpr int kMaps = 12;                     // TMA tensor maps per layer
 constexpr int kMaxBlk = 4;                    // 8-row output blocks per CTA (H <= 4096 on >= 128 SMs)
@@ -121,7 +121,7 @@ struct Cfg {
     float *m;                    // [T,H]    combine of the current layer
     const CUtensorMap *maps;     // [L][kMaps]
     int xm;                      // tensor-core variant: routed down work by expert (see consumer_main)
-    int ipe;                     // expert-major down items per expert (H / 32)
+    int ipe;                     // expert-major down items per expert (H / (8 kXmBlk))
     int stage_bytes, off_stage;  // expert-major down: one expert's staged input, and where they sit
     int nstage;                  // expert-major down: staged experts a CTA has room for (<= kMaxStage)
     float *y_r;                  // [T*k,H]  expert-major down: routed outputs by pair id
@@ -1777,10 +1777,10 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             }
             ++seq;
         }
-        // expert-major routed down items: expert j's 32-row block q (four 8-row blocks), in item order
+        // expert-major routed down items: expert j's kXmBlk 8-row blocks from block q * kXmBlk, in item order
 #pragma unroll 1
         for (int g = xg0; g < xg1 && ok; ++g) {
-            const int j = g / P.ipe, q = g - j * P.ipe, rb = S.slot_e[j] * (P.H / 32) + q;
+            const int j = g / P.ipe, q = g - j * P.ipe;
             unsigned char *dst = claim(S, P, ring, seq, (unsigned)kXmBlk * (unsigned)(P.pc_r * 128 + P.pc_r * 16));
             if (!dst) {
                 ok = false;
@@ -1788,8 +1788,9 @@ __device__ __noinline__ void producer_main(const Params &Pk, Shared &S, unsigned
             }
             unsigned long long *fb = &S.full[seq % (unsigned)ns];
             for (int bi = 0; bi < kXmBlk; ++bi) {
-                tma_load_3d(dst + bi * P.dcb_r, mp + kMapDownQ, 32 * bi, 0, rb, fb);
-                tma_load_3d(dst + kXmBlk * P.dcb_r + bi * P.sbd_r, mp + kMapDownSb, 8 * bi, 0, rb, fb);
+                const int b = q * kXmBlk + bi, rb = S.slot_e[j] * (P.H / 32) + (b >> 2);  // b: 8-row block
+                tma_load_3d(dst + bi * P.dcb_r, mp + kMapDownQ, 32 * (b & 3), 0, rb, fb);
+                tma_load_3d(dst + kXmBlk * P.dcb_r + bi * P.sbd_r, mp + kMapDownSb, 8 * (b & 3), 0, rb, fb);
             }
             ++seq;
         }
@@ -1933,10 +1934,10 @@ bool decode_plan_xm(const moe_layer_w &w, int T, int grid, bool mma, bool allow_
     // routed down matrix, and room for the experts a run can reach (measured: T = 8 1592 -> 1948 tok/s,
     // T = 4 1630 -> 1716 on the Qwen-35B shape; T = 2 slower, 1270 -> 1203)
     P.xm = 0;
-    P.ipe = w.H / 32;
+    P.ipe = w.H / (8 * dec::kXmBlk);
     P.nstage = 0;
     P.stage_bytes = 0;
-    if (allow_xm && mma && T >= 4 && P.parts_r == 1) {
+    if (allow_xm && mma && T >= 4 && P.parts_r == 1 && w.H % (8 * dec::kXmBlk) == 0) {
         const long dmax = std::min((long)w.E, (long)T * w.k);
         const long itmax = (dmax * P.ipe + grid - 1) / grid;
         const long reach = (itmax + P.ipe - 1) / P.ipe + 1;
