@@ -58,7 +58,7 @@ def peaks():
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu
 # capture, per unit of work; None where no capture of the current kernel
 # exists.  Reset to None whenever the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = (223_313_408 + 4_422_912) / 6  # decode_stack_kernel, Gemma shape, T = 1, per layer
+DECODE_TRAFFIC_PER_LAYER = (223_362_304 + 4_370_944) / 6  # decode_stack_kernel, Gemma shape, T = 1, per layer
 HEAD_TRAFFIC_PER_CALL = 415_259_392 + 3_848_192  # moe_qmat_gemv over the 262,144 x 2816 head, one token
 PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER = 369_931_520 + 15_747_328 + 162_025_216 + 65_058_816  # one 1024-token layer call
 PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_960_000 + 5_408_000 + 147_004_672 + 8_862_720
