@@ -68,8 +68,10 @@ struct MmaBuffers {
 };
 size_t mma_xg_bytes(const moe_layer_w *w, int T);
 // FP16 token rows for the tensor-core paths: row r < T token r, row T + j the token of bucketed pair j.
+// odd_div16: the odd input columns (stored places 2, 3, 6, 7 of every 8) hold x / 16, rounded once
+// (the warp-MMA path's operand encoding); otherwise every value is x.
 cudaError_t launch_gather_tokens(const uint16_t *xe, const int32_t *perm, int T, int k, int H, uint16_t *xg,
-                                 cudaStream_t st);
+                                 cudaStream_t st, bool odd_div16 = false);
 // Weight-stationary warp-MMA expert FFN (moe_wsmma.cu): same buffers as launch_expert_mma.
 bool wsmma_supported(const moe_layer_w *w);
 cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *offsets,

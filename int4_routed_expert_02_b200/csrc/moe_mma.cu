@@ -715,9 +715,11 @@ __global__ void __launch_bounds__(kThreads, 1) expert_mma_kernel(const __grid_co
 
 // Token matrix for the gate/up GEMM, FP16: row r < T is token r, row T + j the
 // token of bucketed pair j; every 16-byte chunk stored in the order
-// (0,4,1,5,2,6,3,7).
+// (0,4,1,5,2,6,3,7).  The pairs (1,5) and (3,7) are multiplied by odd_scale
+// (1, or 1/16 for the warp-MMA path) before their one rounding to FP16.
 __global__ void __launch_bounds__(256) gather_kernel(const uint16_t *__restrict__ xe, const int32_t *__restrict__ perm,
-                                                     int T, int k, int H, int R, uint16_t *__restrict__ xg) {
+                                                     int T, int k, int H, int R, float odd_scale,
+                                                     uint16_t *__restrict__ xg) {
     const int cpr = H / 8;  // 16-byte chunks per row
     const long long total = (long long)R * cpr;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
@@ -726,9 +728,10 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint16_t *__restrict_
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xe + (size_t)tok * H) + c);
         uint4 o;  // pairs (0,4), (1,5), (2,6), (3,7), each converted BF16 -> FP16
         o.x = f16x2_from_bf16x2(__byte_perm(v.x, v.z, 0x5410));
-        o.y = f16x2_from_bf16x2(__byte_perm(v.x, v.z, 0x7632));
+        const uint32_t p15 = __byte_perm(v.x, v.z, 0x7632), p37 = __byte_perm(v.y, v.w, 0x7632);
+        o.y = f16x2_from_f32(__uint_as_float(p15 << 16) * odd_scale, __uint_as_float(p15 & 0xffff0000u) * odd_scale);
         o.z = f16x2_from_bf16x2(__byte_perm(v.y, v.w, 0x5410));
-        o.w = f16x2_from_bf16x2(__byte_perm(v.y, v.w, 0x7632));
+        o.w = f16x2_from_f32(__uint_as_float(p37 << 16) * odd_scale, __uint_as_float(p37 & 0xffff0000u) * odd_scale);
         reinterpret_cast<uint4 *>(xg + (size_t)r * H)[c] = o;
     }
 }
@@ -813,13 +816,13 @@ static cudaError_t launch_mma(Params &P, const Maps &map, int max_items, cudaStr
 }  // namespace mma
 
 cudaError_t launch_gather_tokens(const uint16_t *xe, const int32_t *perm, int T, int k, int H, uint16_t *xg,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool odd_div16) {
     const int R = T + T * k;
     const long long chunks = (long long)R * (H / 8);
     long long blocks = (chunks + 255) / 256;
     if (blocks > 4096) blocks = 4096;
     if (blocks <= 0) return cudaSuccess;
-    mma::gather_kernel<<<(int)blocks, 256, 0, st>>>(xe, perm, T, k, H, R, xg);
+    mma::gather_kernel<<<(int)blocks, 256, 0, st>>>(xe, perm, T, k, H, R, odd_div16 ? 0.0625f : 1.0f, xg);
     return cudaGetLastError();
 }
 

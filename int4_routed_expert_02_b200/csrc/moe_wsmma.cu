@@ -14,13 +14,19 @@
 // Operands (m16n8k16, FP16 inputs, FP32 accumulation):
 //   codes   a nibble q masked in place into the low bits of an FP16 half is
 //           the subnormal q * 2^-24, exact; one mask per pair of nibbles
-//           (j, j+4) of a word, and no offset that would cancel later;
+//           (j, j+4) of a word, and no offset that would cancel later.  The
+//           odd nibbles (1,5), (3,7) are masked at bits 4..7 of each half,
+//           where they read 16 q * 2^-24 (still subnormal and exact), so a
+//           word takes one shift (by 8) and four masks;
 //   inputs  the gathered token rows (FP16, every 8 columns stored in the
 //           order 0,4,1,5,2,6,3,7, as the tcgen05 path stores them), so one
 //           16-byte load gives a lane the values of one code word in the
-//           MMA's K order;
+//           MMA's K order.  The odd columns hold x / 16 (the gather and the
+//           gate/up epilogue round x / 16 once), so every product is
+//           q * 2^-24 * x, exact while x / 16 is an FP16 normal (|x| >= 2^-10);
 //   group of 64 columns:  sum_k (s q_k + b) x_k = (s 2^24) D + b sum_k x_k,
-//           D = sum_k (q_k 2^-24) x_k, with sum_k x_k from MMAs against ones.
+//           D = sum_k (q_k 2^-24) x_k, with sum_k x_k from MMAs against ones
+//           (16 against the odd columns).
 // The scale and bias stay FP32, so only the token rows and the SwiGLU values
 // are FP16 here; a SwiGLU value beyond the FP16 range is recorded in the
 // range status word (and stored as 0), as on the tcgen05 path.
@@ -47,6 +53,7 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxSlots = 1024;           // active experts a call may have (E <= 1024)
 constexpr uint32_t kOnes = 0x3C003C00u;   // FP16 pair (1, 1)
+constexpr uint32_t kSixteens = 0x4C004C00u;  // FP16 pair (16, 16): the weight of an odd column's x / 16
 constexpr float kCodeScale = 16777216.f;  // 2^24: undoes the subnormal code encoding
 
 struct Params {
@@ -144,12 +151,15 @@ __device__ __forceinline__ Item get_item(const Params &P, const int *cum, int na
     return it;
 }
 
+// Nibble pairs (0,4), (1,5), (2,6), (3,7) of a code word as FP16 pairs: q * 2^-24 for the even
+// nibbles, 16 q * 2^-24 for the odd ones (their inputs are stored divided by 16).
 __device__ __forceinline__ void code_pairs(uint32_t w, uint32_t (&p)[4]) {
-    constexpr uint32_t kM = 0x000F000Fu;
+    constexpr uint32_t kM = 0x000F000Fu, kM4 = 0x00F000F0u;
+    const uint32_t w8 = w >> 8;
     p[0] = w & kM;
-    p[1] = (w >> 4) & kM;
-    p[2] = (w >> 8) & kM;
-    p[3] = (w >> 12) & kM;
+    p[1] = w & kM4;
+    p[2] = w8 & kM;
+    p[3] = w8 & kM4;
 }
 
 __device__ __forceinline__ void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -198,10 +208,10 @@ __device__ __forceinline__ void gu_load(const GUView &v, int gi, GUStage &s) {
 
 __device__ __forceinline__ void gu_compute(const GUStage &s, float (&acc)[4][4]) {
     float dx[4] = {0.f, 0.f, 0.f, 0.f};
-    mma(dx, kOnes, kOnes, kOnes, kOnes, s.x0.x, s.x0.y);
-    mma(dx, kOnes, kOnes, kOnes, kOnes, s.x0.z, s.x0.w);
-    mma(dx, kOnes, kOnes, kOnes, kOnes, s.x1.x, s.x1.y);
-    mma(dx, kOnes, kOnes, kOnes, kOnes, s.x1.z, s.x1.w);
+    mma(dx, kOnes, kOnes, kSixteens, kSixteens, s.x0.x, s.x0.y);
+    mma(dx, kOnes, kOnes, kSixteens, kSixteens, s.x0.z, s.x0.w);
+    mma(dx, kOnes, kOnes, kSixteens, kSixteens, s.x1.x, s.x1.y);
+    mma(dx, kOnes, kOnes, kSixteens, kSixteens, s.x1.z, s.x1.w);
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -283,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
                     atomicCAS(P.range_err, 0, 2);
                     a = 0.f;
                 }
+                if (r & 1) a *= 0.0625f;  // an odd column of the down GEMM's input: a / 16
                 P.act[(size_t)(it.row0 + j) * P.act_ld + col] = __half_as_ushort(__float2half_rn(a));
             }
         }
@@ -321,10 +332,10 @@ __device__ __forceinline__ void d_load(const DView &v, int gi, DStage &s) {
 
 __device__ __forceinline__ void d_compute(const DStage &s, float (&y)[4][4]) {
     float da[4] = {0.f, 0.f, 0.f, 0.f};
-    mma(da, s.a00.x, s.a10.x, s.a00.y, s.a10.y, kOnes, kOnes);
-    mma(da, s.a00.z, s.a10.z, s.a00.w, s.a10.w, kOnes, kOnes);
-    mma(da, s.a01.x, s.a11.x, s.a01.y, s.a11.y, kOnes, kOnes);
-    mma(da, s.a01.z, s.a11.z, s.a01.w, s.a11.w, kOnes, kOnes);
+    mma(da, s.a00.x, s.a10.x, s.a00.y, s.a10.y, kOnes, kSixteens);
+    mma(da, s.a00.z, s.a10.z, s.a00.w, s.a10.w, kOnes, kSixteens);
+    mma(da, s.a01.x, s.a11.x, s.a01.y, s.a11.y, kOnes, kSixteens);
+    mma(da, s.a01.z, s.a11.z, s.a01.w, s.a11.w, kOnes, kSixteens);
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -432,7 +443,7 @@ cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T,
     if (!wsmma_supported(w)) return cudaErrorInvalidValue;
     const int H = w->H, k = w->k, I = w->I, Is = w->Is;
     const int Kmax = I > Is ? I : Is;
-    cudaError_t e = launch_gather_tokens(xe, perm, T, k, H, b.xg, st);
+    cudaError_t e = launch_gather_tokens(xe, perm, T, k, H, b.xg, st, true);
     if (e != cudaSuccess) return e;
     const int sms = sms_of(st);
     if (sms <= 0) return cudaErrorNoDevice;
