@@ -233,6 +233,24 @@ __device__ __forceinline__ void gu_compute(const GUStage &s, float (&acc)[4][4])
     }
 }
 
+__device__ __forceinline__ GUView gu_view(const Params &P, const Item &it, int lane) {
+    const int g = lane >> 2, t = lane & 3, G = P.H / 64, C = P.H / 32;
+    const int rows = it.shared ? P.rows_s : P.rows_r;
+    const size_t mrb = it.shared ? (size_t)it.rb : (size_t)it.e * (rows / 32) + it.rb;
+    // this lane's codes: chunk (t>>1) of group 0, row g of slice 0, words 2(t&1) and 2(t&1)+1
+    const size_t qoff = (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
+    GUView v;
+    v.qg = (it.shared ? P.sq[0] : P.q[0]) + qoff;
+    v.qu = (it.shared ? P.sq[1] : P.q[1]) + qoff;
+    v.sbg = (it.shared ? P.ssb[0] : P.sb[0]) + mrb * G * 32 + g;
+    v.sbu = (it.shared ? P.ssb[1] : P.sb[1]) + mrb * G * 32 + g;
+    v.xok = g < it.n;
+    v.x = P.xin + (size_t)(it.row0 + (v.xok ? g : 0)) * P.ld_in + (t >> 1) * 32 + 16 * (t & 1);
+    return v;
+}
+
+// Items are software-pipelined: the first K group of a warp's next item is loaded before the
+// current item's partial sums meet in shared memory, so the item's first HBM latency overlaps them.
 __global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
     __shared__ int cum[kMaxSlots + 1];
     __shared__ float red[kWarps][16][32];
@@ -242,33 +260,34 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
     const int nsh = P.with_shared ? rbs_s * ((P.T + P.ntok - 1) / P.ntok) : 0;
     const int total = nsh + units * rbs_r;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int G = P.H / 64, C = P.H / 32;
+    const int G = P.H / 64;
+    Item it;
+    GUView v;
+    GUStage cur;
+    if (blockIdx.x < total) {
+        it = get_item(P, cum, na, blockIdx.x, nsh, rbs_s, rbs_r);
+        v = gu_view(P, it, lane);
+        if (warp < G) gu_load(v, warp, cur);
+    }
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Item it = get_item(P, cum, na, id, nsh, rbs_s, rbs_r);
-        const int rows = it.shared ? P.rows_s : P.rows_r;
-        const size_t mrb = it.shared ? (size_t)it.rb : (size_t)it.e * (rows / 32) + it.rb;
-        // this lane's codes: chunk (t>>1) of group 0, row g of slice 0, words 2(t&1) and 2(t&1)+1
-        const size_t qoff = (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
-        GUView v;
-        v.qg = (it.shared ? P.sq[0] : P.q[0]) + qoff;
-        v.qu = (it.shared ? P.sq[1] : P.q[1]) + qoff;
-        v.sbg = (it.shared ? P.ssb[0] : P.sb[0]) + mrb * G * 32 + g;
-        v.sbu = (it.shared ? P.ssb[1] : P.sb[1]) + mrb * G * 32 + g;
-        v.xok = g < it.n;
-        v.x = P.xin + (size_t)(it.row0 + (v.xok ? g : 0)) * P.ld_in + (t >> 1) * 32 + 16 * (t & 1);
         float acc[4][4];
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) acc[sl][0] = acc[sl][1] = acc[sl][2] = acc[sl][3] = 0.f;
         int gi = warp;
         if (gi < G) {
-            GUStage cur, nxt;
-            gu_load(v, gi, cur);
+            GUStage nxt;
             for (; gi + kWarps < G; gi += kWarps) {
                 gu_load(v, gi + kWarps, nxt);
                 gu_compute(cur, acc);
                 cur = nxt;
             }
             gu_compute(cur, acc);
+        }
+        const Item ic = it;  // this item; `it`, `v` and `cur` move on to the next one
+        if (id + (int)gridDim.x < total) {
+            it = get_item(P, cum, na, id + gridDim.x, nsh, rbs_s, rbs_r);
+            v = gu_view(P, it, lane);
+            if (warp < G) gu_load(v, warp, cur);
         }
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl)
@@ -285,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
                 us += red[w][sl * 4 + 2 + h][lane];
             }
             const int j = 2 * t + h;
-            if (j < it.n) {
-                const int r = it.rb * 32 + sl * 8 + g;  // gate/up row = activation column
+            if (j < ic.n) {
+                const int r = ic.rb * 32 + sl * 8 + g;  // gate/up row = activation column
                 const int col = (r & ~7) | ((r & 3) << 1) | ((r >> 2) & 1);
                 float a = silu_mul(gs, us);
                 if (!(fabsf(a) <= 65504.f)) {
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
                     a = 0.f;
                 }
                 if (r & 1) a *= 0.0625f;  // an odd column of the down GEMM's input: a / 16
-                P.act[(size_t)(it.row0 + j) * P.act_ld + col] = __half_as_ushort(__float2half_rn(a));
+                P.act[(size_t)(ic.row0 + j) * P.act_ld + col] = __half_as_ushort(__float2half_rn(a));
             }
         }
         __syncthreads();
@@ -361,6 +380,31 @@ __device__ __forceinline__ void d_compute(const DStage &s, float (&y)[4][4]) {
 // an item runs over 2 warps.
 constexpr int kDownRbs = 4;
 
+// A warp's part of a down item: its row block, whether the block exists, the K groups, the view.
+struct DWork {
+    int rb, G;
+    bool live;
+    DView v;
+};
+
+__device__ __forceinline__ DWork d_work(const Params &P, const Item &it, int pair, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int K = it.shared ? P.K_s : P.K_r, C = K / 32, rows = it.shared ? P.rows_s : P.rows_r;
+    DWork w;
+    w.G = K / 64;
+    w.rb = it.rb * kDownRbs + pair;  // this pair's row block
+    w.live = w.rb < rows / 32;
+    const size_t mrb = it.shared ? (size_t)w.rb : (size_t)it.e * (rows / 32) + w.rb;
+    w.v.q = (it.shared ? P.sq[0] : P.q[0]) + (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
+    w.v.sb = (it.shared ? P.ssb[0] : P.sb[0]) + mrb * w.G * 32 + 2 * t;
+    w.v.ok0 = g < it.n;
+    w.v.ok1 = g + 8 < it.n;
+    const int xo = (t >> 1) * 32 + 16 * (t & 1);
+    w.v.a0 = P.xin + (size_t)(it.row0 + (w.v.ok0 ? g : 0)) * P.ld_in + xo;
+    w.v.a1 = P.xin + (size_t)(it.row0 + (w.v.ok1 ? g + 8 : 0)) * P.ld_in + xo;
+    return w;
+}
+
 __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
     __shared__ int cum[kMaxSlots + 1];
     __shared__ float red[kWarps][16][32];
@@ -372,33 +416,36 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
     const int total = nsh + units * rbs_r;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int pair = warp >> 1, half = warp & 1;
+    // software-pipelined over items like gateup_kernel
+    Item it;
+    DWork dw;
+    DStage cur;
+    if (blockIdx.x < total) {
+        it = get_item(P, cum, na, blockIdx.x, nsh, rbs_s, rbs_r);  // it.rb: the run of row blocks
+        dw = d_work(P, it, pair, lane);
+        if (dw.live && half < dw.G) d_load(dw.v, half, cur);
+    }
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Item it = get_item(P, cum, na, id, nsh, rbs_s, rbs_r);  // it.rb: the run of row blocks
-        const int K = it.shared ? P.K_s : P.K_r, C = K / 32, G = K / 64, rows = it.shared ? P.rows_s : P.rows_r;
-        const int rb = it.rb * kDownRbs + pair;  // this pair's row block
-        const bool live = rb < rows / 32;
-        const size_t mrb = it.shared ? (size_t)rb : (size_t)it.e * (rows / 32) + rb;
-        DView v;
-        v.q = (it.shared ? P.sq[0] : P.q[0]) + (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
-        v.sb = (it.shared ? P.ssb[0] : P.sb[0]) + mrb * G * 32 + 2 * t;
-        v.ok0 = g < it.n;
-        v.ok1 = g + 8 < it.n;
-        const int xo = (t >> 1) * 32 + 16 * (t & 1);
-        v.a0 = P.xin + (size_t)(it.row0 + (v.ok0 ? g : 0)) * P.ld_in + xo;
-        v.a1 = P.xin + (size_t)(it.row0 + (v.ok1 ? g + 8 : 0)) * P.ld_in + xo;
         float y[4][4];
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) y[sl][0] = y[sl][1] = y[sl][2] = y[sl][3] = 0.f;
         int gi = half;
-        if (live && gi < G) {
-            DStage cur, nxt;
-            d_load(v, gi, cur);
-            for (; gi + 2 < G; gi += 2) {
-                d_load(v, gi + 2, nxt);
+        if (dw.live && gi < dw.G) {
+            DStage nxt;
+            for (; gi + 2 < dw.G; gi += 2) {
+                d_load(dw.v, gi + 2, nxt);
                 d_compute(cur, y);
                 cur = nxt;
             }
             d_compute(cur, y);
+        }
+        const Item ic = it;  // this item; `it`, `dw` and `cur` move on to the next one
+        const int rb = dw.rb;
+        const bool live = dw.live;
+        if (id + (int)gridDim.x < total) {
+            it = get_item(P, cum, na, id + gridDim.x, nsh, rbs_s, rbs_r);
+            dw = d_work(P, it, pair, lane);
+            if (dw.live && half < dw.G) d_load(dw.v, half, cur);
         }
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl)
@@ -408,9 +455,9 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
         if (live) {
             // warp 2p: token g, warp 2p + 1: token g + 8; rows 2t, 2t+1 of each slice of row block rb
             const int h = half, j = g + 8 * h;
-            if (j < it.n) {
-                float *dst = it.shared ? P.sh + (size_t)(it.seg + j) * P.H
-                                       : P.y + (size_t)__ldg(P.perm + it.seg + j) * P.H;
+            if (j < ic.n) {
+                float *dst = ic.shared ? P.sh + (size_t)(ic.seg + j) * P.H
+                                       : P.y + (size_t)__ldg(P.perm + ic.seg + j) * P.H;
 #pragma unroll
                 for (int sl = 0; sl < 4; ++sl) {
                     const float o0 = red[2 * pair][sl * 4 + 2 * h][lane] + red[2 * pair + 1][sl * 4 + 2 * h][lane];
