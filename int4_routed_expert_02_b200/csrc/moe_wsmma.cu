@@ -31,16 +31,20 @@
 // are FP16 here; a SwiGLU value beyond the FP16 range is recorded in the
 // range status word (and stored as 0), as on the tcgen05 path.
 //
-// Work items: (32-row block, token group) of the shared expert, then of every
-// active routed expert; a persistent grid walks them.  The 8 warps of a CTA
-// split the 64-column groups of K and add their partial sums in shared memory
-// in a fixed order, so results do not depend on timing.
-//   gate/up  A = 8 gate rows (M 0..7) and the same 8 up rows (M 8..15) of one
-//            of the block's four 8-row slices, B = 8 tokens; the SwiGLU
+// Work items: (row blocks, token group) of the shared expert, then of every
+// active routed expert; a persistent grid of 4 CTAs of 4 warps per SM walks
+// them.  Every sum is taken in a fixed order, so results do not depend on
+// timing.
+//   gate/up  one 32-row block and 8 tokens: the 4 warps split the 64-column
+//            groups of K and add their partial sums in shared memory in warp
+//            order.  A = 8 gate rows (M 0..7) and the same 8 up rows (M 8..15)
+//            of one of the block's four 8-row slices, B = 8 tokens; the SwiGLU
 //            output goes to the FP16 activation buffer (the down GEMM's input,
 //            in the same 8-column order).
-//   down     A = 16 tokens' activations, B = 8 rows of one slice; the output
-//            goes to y (routed, by pair id) or sh (shared, by token).
+//   down     four 32-row blocks and 16 tokens: warp w owns block w over all
+//            of K, so its sums are the outputs.  A = 16 tokens' activations,
+//            B = 8 rows of one slice; the output goes to y (routed, by pair
+//            id) or sh (shared, by token).
 #include <cuda_fp16.h>
 
 #include "moe_common.cuh"
@@ -49,8 +53,9 @@
 namespace moe {
 namespace wsm {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
+constexpr int kCtasPerSm = 4;             // 16 warps of 128 registers per SM
 constexpr int kMaxSlots = 1024;           // active experts a call may have (E <= 1024)
 constexpr uint32_t kOnes = 0x3C003C00u;   // FP16 pair (1, 1)
 constexpr uint32_t kSixteens = 0x4C004C00u;  // FP16 pair (16, 16): the weight of an odd column's x / 16
@@ -82,11 +87,12 @@ struct Item {
 __device__ int build_prefix(const Params &P, int *cum) {
     __shared__ int wsum[kWarps];
     const int na = __ldg(P.active);
-    const int per = (na + kThreads - 1) / kThreads;  // slots per thread (<= 4)
+    constexpr int kPer = kMaxSlots / kThreads;
+    const int per = (na + kThreads - 1) / kThreads;  // slots per thread (<= kPer)
     const int s0 = threadIdx.x * per;
-    int loc[4], tot = 0;
+    int loc[kPer], tot = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kPer; ++i) {
         loc[i] = 0;
         if (i < per && s0 + i < na) {
             const int e = __ldg(P.active + 1 + s0 + i);
@@ -251,7 +257,7 @@ __device__ __forceinline__ GUView gu_view(const Params &P, const Item &it, int l
 
 // Items are software-pipelined: the first K group of a warp's next item is loaded before the
 // current item's partial sums meet in shared memory, so the item's first HBM latency overlaps them.
-__global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) gateup_kernel(const Params P) {
     __shared__ int cum[kMaxSlots + 1];
     __shared__ float red[kWarps][16][32];
     const int na = __ldg(P.active);
@@ -294,9 +300,10 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_kernel(const Params P) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) red[warp][sl * 4 + c][lane] = acc[sl][c];
         __syncthreads();
-        {
-            // warp w: slice w & 3, token column 2t + (w >> 2)
-            const int sl = warp & 3, h = warp >> 2;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            // warp w: slice w, token columns 2t and 2t + 1
+            const int sl = warp;
             float gs = 0.f, us = 0.f;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
@@ -375,10 +382,9 @@ __device__ __forceinline__ void d_compute(const DStage &s, float (&y)[4][4]) {
     }
 }
 
-// Down items are 4 row blocks (128 output rows) of one matrix and 16 tokens: warp pair p = w >> 1 owns
-// row block 4*ib + p and its two warps split the block's 64-column groups of K, so the sum at the end of
-// an item runs over 2 warps.
-constexpr int kDownRbs = 4;
+// Down items are 4 row blocks (128 output rows) of one matrix and 16 tokens: warp w owns row block
+// 4*ib + w over all of K, so its sums are the outputs (no reduction across warps).
+constexpr int kDownRbs = kWarps;
 
 // A warp's part of a down item: its row block, whether the block exists, the K groups, the view.
 struct DWork {
@@ -387,12 +393,12 @@ struct DWork {
     DView v;
 };
 
-__device__ __forceinline__ DWork d_work(const Params &P, const Item &it, int pair, int lane) {
+__device__ __forceinline__ DWork d_work(const Params &P, const Item &it, int warp, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const int K = it.shared ? P.K_s : P.K_r, C = K / 32, rows = it.shared ? P.rows_s : P.rows_r;
     DWork w;
     w.G = K / 64;
-    w.rb = it.rb * kDownRbs + pair;  // this pair's row block
+    w.rb = it.rb * kDownRbs + warp;  // this warp's row block
     w.live = w.rb < rows / 32;
     const size_t mrb = it.shared ? (size_t)w.rb : (size_t)it.e * (rows / 32) + w.rb;
     w.v.q = (it.shared ? P.sq[0] : P.q[0]) + (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
@@ -405,9 +411,8 @@ __device__ __forceinline__ DWork d_work(const Params &P, const Item &it, int pai
     return w;
 }
 
-__global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) down_kernel(const Params P) {
     __shared__ int cum[kMaxSlots + 1];
-    __shared__ float red[kWarps][16][32];
     const int na = __ldg(P.active);
     const int units = build_prefix(P, cum);
     // items per token tile: the row blocks in runs of kDownRbs
@@ -415,25 +420,24 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
     const int nsh = P.with_shared ? rbs_s * ((P.T + P.ntok - 1) / P.ntok) : 0;
     const int total = nsh + units * rbs_r;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int pair = warp >> 1, half = warp & 1;
-    // software-pipelined over items like gateup_kernel
+    // software-pipelined over items like gateup_kernel (here per warp: no step joins the warps)
     Item it;
     DWork dw;
     DStage cur;
     if (blockIdx.x < total) {
         it = get_item(P, cum, na, blockIdx.x, nsh, rbs_s, rbs_r);  // it.rb: the run of row blocks
-        dw = d_work(P, it, pair, lane);
-        if (dw.live && half < dw.G) d_load(dw.v, half, cur);
+        dw = d_work(P, it, warp, lane);
+        if (dw.live) d_load(dw.v, 0, cur);
     }
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
         float y[4][4];
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) y[sl][0] = y[sl][1] = y[sl][2] = y[sl][3] = 0.f;
-        int gi = half;
-        if (dw.live && gi < dw.G) {
+        if (dw.live) {
             DStage nxt;
-            for (; gi + 2 < dw.G; gi += 2) {
-                d_load(dw.v, gi + 2, nxt);
+            int gi = 0;
+            for (; gi + 1 < dw.G; ++gi) {
+                d_load(dw.v, gi + 1, nxt);
                 d_compute(cur, y);
                 cur = nxt;
             }
@@ -444,30 +448,24 @@ __global__ void __launch_bounds__(kThreads, 2) down_kernel(const Params P) {
         const bool live = dw.live;
         if (id + (int)gridDim.x < total) {
             it = get_item(P, cum, na, id + gridDim.x, nsh, rbs_s, rbs_r);
-            dw = d_work(P, it, pair, lane);
-            if (dw.live && half < dw.G) d_load(dw.v, half, cur);
+            dw = d_work(P, it, warp, lane);
+            if (dw.live) d_load(dw.v, 0, cur);
         }
-#pragma unroll
-        for (int sl = 0; sl < 4; ++sl)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) red[warp][sl * 4 + c][lane] = y[sl][c];
-        __syncthreads();
         if (live) {
-            // warp 2p: token g, warp 2p + 1: token g + 8; rows 2t, 2t+1 of each slice of row block rb
-            const int h = half, j = g + 8 * h;
-            if (j < ic.n) {
-                float *dst = ic.shared ? P.sh + (size_t)(ic.seg + j) * P.H
-                                       : P.y + (size_t)__ldg(P.perm + ic.seg + j) * P.H;
+            // y[sl]: token g (0, 1) and token g + 8 (2, 3), rows 2t and 2t + 1 of slice sl of row block rb
 #pragma unroll
-                for (int sl = 0; sl < 4; ++sl) {
-                    const float o0 = red[2 * pair][sl * 4 + 2 * h][lane] + red[2 * pair + 1][sl * 4 + 2 * h][lane];
-                    const float o1 =
-                        red[2 * pair][sl * 4 + 2 * h + 1][lane] + red[2 * pair + 1][sl * 4 + 2 * h + 1][lane];
-                    *reinterpret_cast<float2 *>(dst + rb * 32 + sl * 8 + 2 * t) = make_float2(o0, o1);
+            for (int h = 0; h < 2; ++h) {
+                const int j = g + 8 * h;
+                if (j < ic.n) {
+                    float *dst = ic.shared ? P.sh + (size_t)(ic.seg + j) * P.H
+                                           : P.y + (size_t)__ldg(P.perm + ic.seg + j) * P.H;
+#pragma unroll
+                    for (int sl = 0; sl < 4; ++sl)
+                        *reinterpret_cast<float2 *>(dst + rb * 32 + sl * 8 + 2 * t) =
+                            make_float2(y[sl][2 * h], y[sl][2 * h + 1]);
                 }
             }
         }
-        __syncthreads();
     }
 }
 
@@ -526,7 +524,7 @@ cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T,
     P.ntok = 8;
     long long items =
         (with_shared ? (long long)(Is / 32) * ((T + 7) / 8) : 0) + (pairs / 8 + max_active) * (I / 32);
-    int grid = (int)(items < 2LL * sms ? items : 2LL * sms);
+    int grid = (int)(items < (long long)kCtasPerSm * sms ? items : (long long)kCtasPerSm * sms);
     if (grid > 0) {
         gateup_kernel<<<grid, kThreads, 0, st>>>(P);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -546,7 +544,7 @@ cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T,
     P.ntok = 16;
     const long long drun = (H / 32 + kDownRbs - 1) / kDownRbs;
     items = (with_shared ? drun * ((T + 15) / 16) : 0) + (pairs / 16 + max_active) * drun;
-    grid = (int)(items < 2LL * sms ? items : 2LL * sms);
+    grid = (int)(items < (long long)kCtasPerSm * sms ? items : (long long)kCtasPerSm * sms);
     if (grid > 0) {
         down_kernel<<<grid, kThreads, 0, st>>>(P);
         e = cudaGetLastError();
