@@ -350,7 +350,7 @@ def expert_path_of(force_path, T):
     """The expert path a call of T tokens takes (the library's automatic rule when force_path is 0)."""
     if force_path:
         return force_path
-    return 1 if T < 32 else (3 if T <= 320 else 2)
+    return 1 if T < 32 else (3 if T <= 448 else 2)
 
 
 def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0):

@@ -99,7 +99,7 @@ typedef struct {
     float layer_scalar; /* default 1.0 */
     float eps;          /* default 1e-6, inside every RMS */
     int force_path;     /* 0 auto: dequant-GEMV below 32 tokens, the weight-stationary warp-level MMA
-                           for 32..320, the tcgen05 grouped GEMM above;
+                           for 32..448, the tcgen05 grouped GEMM above;
                            1 CUDA-core dequant-GEMV, 2 tensor-core (tcgen05) grouped GEMM,
                            3 weight-stationary warp-level MMA (exact codes, FP32 scale/bias) */
 } moe_opts;
@@ -193,7 +193,7 @@ MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets
  * weights are MLX affine 4-bit, groups of 64, a BF16 scale and bias per
  * group, section "How TurboFieldfare saves memory".)
  * Path: force_path 1, or T < 32 in auto mode, is the CUDA-core dequant-GEMV
- * (fp32 sums of exact products).  force_path 2, or T > 320 in auto mode, is the tcgen05
+ * (fp32 sums of exact products).  force_path 2, or T > 448 in auto mode, is the tcgen05
  * grouped GEMM on FP16 operands: it needs every weight s*q + b and every
  * SwiGLU value within the FP16 range (|v| <= 65504).  A layer outside that
  * range is not computed approximately: the kernel records MOE_EDEVICE
@@ -204,7 +204,7 @@ MOE_API int moe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets
  * codes enter as exact FP16 values, scale and bias stay FP32, so only the
  * token rows and SwiGLU outputs are FP16 (a SwiGLU value beyond 65504 is
  * reported as above; weights have no range limit).  E <= 1024.  Auto mode takes
- * it for 32 <= T <= 320.
+ * it for 32 <= T <= 448.
  */
 MOE_API int moe_expert_ffn(const moe_layer_w *w, const uint16_t *xe, int T, const int32_t *idx, const float *wts,
                    const int32_t *offsets, const int32_t *perm, const int32_t *active, int with_shared,

@@ -114,8 +114,8 @@ struct WsLayout {
 
 constexpr size_t kStatusOffset = 4;
 constexpr int kMmaMinT = 32;   // auto path: tensor cores from this many tokens on (else the dequant-GEMV)
-constexpr int kWsMaxT = 320;   // ... the weight-stationary warp-MMA path up to this many, the tcgen05 GEMM above
-                               // (the two measured level at 320 tokens on the Gemma shape)
+constexpr int kWsMaxT = 448;   // ... the weight-stationary warp-MMA path up to this many, the tcgen05 GEMM above
+                               // (measured on the Gemma shape: the warp-MMA path ahead up to 448 tokens)
 
 WsLayout ws_layout(const moe_layer_w *w, int T) {
     WsLayout L;
