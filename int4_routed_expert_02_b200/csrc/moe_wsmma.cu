@@ -42,7 +42,9 @@
 //            output goes to the FP16 activation buffer (the down GEMM's input,
 //            in the same 8-column order).
 //   down     four 32-row blocks and 16 tokens: warp w owns block w over all
-//            of K, so its sums are the outputs.  A = 16 tokens' activations,
+//            of K, so its sums are the outputs (a shared-expert item is one
+//            block whose K the 4 warps split, summed in shared memory in warp
+//            order).  A = 16 tokens' activations,
 //            B = 8 rows of one slice; the output goes to y (routed, by pair
 //            id) or sh (shared, by token).
 #include <cuda_fp16.h>
@@ -382,13 +384,16 @@ __device__ __forceinline__ void d_compute(const DStage &s, float (&y)[4][4]) {
     }
 }
 
-// Down items are 4 row blocks (128 output rows) of one matrix and 16 tokens: warp w owns row block
-// 4*ib + w over all of K, so its sums are the outputs (no reduction across warps).
+// Routed down items are 4 row blocks (128 output rows) of one expert and 16 tokens: warp w owns row
+// block 4*ib + w over all of K (I columns), so its sums are the outputs.  The shared expert's K (Is
+// columns) is usually several times longer, so its items are one row block whose K groups the 4 warps
+// split, adding their sums in shared memory in warp order: every item then takes about as long, and
+// the round-robin over items stays balanced.
 constexpr int kDownRbs = kWarps;
 
 // A warp's part of a down item: its row block, whether the block exists, the K groups, the view.
 struct DWork {
-    int rb, G;
+    int rb, G, gi0, step;  // row block; K groups; this warp's first group and group stride
     bool live;
     DView v;
 };
@@ -398,8 +403,10 @@ __device__ __forceinline__ DWork d_work(const Params &P, const Item &it, int war
     const int K = it.shared ? P.K_s : P.K_r, C = K / 32, rows = it.shared ? P.rows_s : P.rows_r;
     DWork w;
     w.G = K / 64;
-    w.rb = it.rb * kDownRbs + warp;  // this warp's row block
-    w.live = w.rb < rows / 32;
+    w.rb = it.shared ? it.rb : it.rb * kDownRbs + warp;  // this warp's row block
+    w.gi0 = it.shared ? warp : 0;
+    w.step = it.shared ? kWarps : 1;
+    w.live = w.rb < rows / 32 && w.gi0 < w.G;
     const size_t mrb = it.shared ? (size_t)w.rb : (size_t)it.e * (rows / 32) + w.rb;
     w.v.q = (it.shared ? P.sq[0] : P.q[0]) + (mrb * C + (t >> 1)) * 128 + g * 4 + 2 * (t & 1);
     w.v.sb = (it.shared ? P.ssb[0] : P.sb[0]) + mrb * w.G * 32 + 2 * t;
@@ -413,21 +420,22 @@ __device__ __forceinline__ DWork d_work(const Params &P, const Item &it, int war
 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) down_kernel(const Params P) {
     __shared__ int cum[kMaxSlots + 1];
+    __shared__ float red[kWarps][16][32];
     const int na = __ldg(P.active);
     const int units = build_prefix(P, cum);
-    // items per token tile: the row blocks in runs of kDownRbs
-    const int rbs_s = (P.rows_s / 32 + kDownRbs - 1) / kDownRbs, rbs_r = (P.rows_r / 32 + kDownRbs - 1) / kDownRbs;
+    // items per token tile: shared, one row block each; routed, the row blocks in runs of kDownRbs
+    const int rbs_s = P.rows_s / 32, rbs_r = (P.rows_r / 32 + kDownRbs - 1) / kDownRbs;
     const int nsh = P.with_shared ? rbs_s * ((P.T + P.ntok - 1) / P.ntok) : 0;
     const int total = nsh + units * rbs_r;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    // software-pipelined over items like gateup_kernel (here per warp: no step joins the warps)
+    // software-pipelined over items like gateup_kernel
     Item it;
     DWork dw;
     DStage cur;
     if (blockIdx.x < total) {
         it = get_item(P, cum, na, blockIdx.x, nsh, rbs_s, rbs_r);  // it.rb: the run of row blocks
         dw = d_work(P, it, warp, lane);
-        if (dw.live) d_load(dw.v, 0, cur);
+        if (dw.live) d_load(dw.v, dw.gi0, cur);
     }
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
         float y[4][4];
@@ -435,9 +443,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) down_kernel(const Params
         for (int sl = 0; sl < 4; ++sl) y[sl][0] = y[sl][1] = y[sl][2] = y[sl][3] = 0.f;
         if (dw.live) {
             DStage nxt;
-            int gi = 0;
-            for (; gi + 1 < dw.G; ++gi) {
-                d_load(dw.v, gi + 1, nxt);
+            int gi = dw.gi0;
+            for (; gi + dw.step < dw.G; gi += dw.step) {
+                d_load(dw.v, gi + dw.step, nxt);
                 d_compute(cur, y);
                 cur = nxt;
             }
@@ -449,16 +457,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) down_kernel(const Params
         if (id + (int)gridDim.x < total) {
             it = get_item(P, cum, na, id + gridDim.x, nsh, rbs_s, rbs_r);
             dw = d_work(P, it, warp, lane);
-            if (dw.live) d_load(dw.v, 0, cur);
+            if (dw.live) d_load(dw.v, dw.gi0, cur);
         }
-        if (live) {
+        if (ic.shared) {
+            // the 4 warps' partial sums of row block rb; warp w writes slice w
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) red[warp][sl * 4 + c][lane] = y[sl][c];
+            __syncthreads();
+            if (rb < P.rows_s / 32) {
+                const int sl = warp;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = g + 8 * h;
+                    float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w) {
+                        o0 += red[w][sl * 4 + 2 * h][lane];
+                        o1 += red[w][sl * 4 + 2 * h + 1][lane];
+                    }
+                    if (j < ic.n)
+                        *reinterpret_cast<float2 *>(P.sh + (size_t)(ic.seg + j) * P.H + rb * 32 + sl * 8 + 2 * t) =
+                            make_float2(o0, o1);
+                }
+            }
+            __syncthreads();
+        } else if (live) {
             // y[sl]: token g (0, 1) and token g + 8 (2, 3), rows 2t and 2t + 1 of slice sl of row block rb
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int j = g + 8 * h;
                 if (j < ic.n) {
-                    float *dst = ic.shared ? P.sh + (size_t)(ic.seg + j) * P.H
-                                           : P.y + (size_t)__ldg(P.perm + ic.seg + j) * P.H;
+                    float *dst = P.y + (size_t)__ldg(P.perm + ic.seg + j) * P.H;
 #pragma unroll
                     for (int sl = 0; sl < 4; ++sl)
                         *reinterpret_cast<float2 *>(dst + rb * 32 + sl * 8 + 2 * t) =
@@ -543,7 +574,7 @@ cudaError_t launch_expert_wsmma(const moe_layer_w *w, const uint16_t *xe, int T,
     P.ld_in = Kmax;
     P.ntok = 16;
     const long long drun = (H / 32 + kDownRbs - 1) / kDownRbs;
-    items = (with_shared ? drun * ((T + 15) / 16) : 0) + (pairs / 16 + max_active) * drun;
+    items = (with_shared ? (long long)(H / 32) * ((T + 15) / 16) : 0) + (pairs / 16 + max_active) * drun;
     grid = (int)(items < (long long)kCtasPerSm * sms ? items : (long long)kCtasPerSm * sms);
     if (grid > 0) {
         down_kernel<<<grid, kThreads, 0, st>>>(P);
