@@ -58,10 +58,20 @@ def peaks():
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu
 # capture, per unit of work; None where no capture of the current kernel
 # exists.  Reset to None whenever the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = (223_362_304 + 4_370_944) / 6  # decode_stack_kernel, Gemma shape, T = 1, per layer
+# decode_stack_kernel, per layer, keyed by (configuration, tokens per step): one launch of 6 layers (Gemma
+# shape) or 4 layers (Qwen shapes).  Only T = 1, where every layer reads exactly k experts, so bytes
+# scale with layers; from T = 4 on a layer's bytes follow its routing (the distinct experts fall from
+# ~57 in the first layers of the Qwen-35B-shaped stack to ~30 averaged over 40), so no capture stands
+# for a whole stack and those lines carry null.
+DECODE_TRAFFIC_PER_LAYER = {
+    (1, 1): (223_362_304 + 4_370_944) / 6,
+    (2, 1): (66_149_120 + 1_017_344) / 4,
+    (3, 1): (82_535_424 + 1_690_368) / 4,
+}
 HEAD_TRAFFIC_PER_CALL = 415_259_392 + 3_848_192  # moe_qmat_gemv over the 262,144 x 2816 head, one token
 PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER = 369_931_520 + 15_747_328 + 162_025_216 + 65_058_816  # one 1024-token layer call
 PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK = 296_960_000 + 5_408_000 + 147_004_672 + 8_862_720
+PREFILL_WS_TRAFFIC_PER_LAYER_CHUNK = 298_698_496 + 5_197_056 + 148_107_776 + 5_612_800  # gateup + down_kernel
 
 
 def expert_bytes(rows_cols: int) -> float:
@@ -310,8 +320,8 @@ def decode_measure(cfg_id, T, K, W, dev, rank=0, world=1, clocks=False, cpu_budg
     hbm = peaks()
     gbs = step_bytes / (ms_per_step / 1e3) / 1e9
     if st.persistent:
-        traffic = (int(DECODE_TRAFFIC_PER_LAYER * st.L)
-                   if DECODE_TRAFFIC_PER_LAYER and cfg_id == 1 and T == 1 and layers is None else None)
+        traffic = (int(DECODE_TRAFFIC_PER_LAYER[(cfg_id, T)] * st.L)
+                   if (cfg_id, T) in DECODE_TRAFFIC_PER_LAYER and layers is None else None)
         roof = {"kernel": "decode_stack_kernel (persistent: all layers of a step in one cooperative launch)",
                 "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / hbm["hbm_gbs"], 4), "peak_source": hbm["source"] + " (burst copy)",
@@ -389,8 +399,8 @@ def prefill_measure(dev, chunks=8, layers=None, T=None, share=None, force_path=0
     peak_t = hbm["bf16_tflops"]  # FP16 and BF16 share the dense tensor rate
     fused = T != cfg.T
     path = expert_path_of(force_path, T)
-    traffic = (PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER if fused else PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK) \
-        if path == 2 else None
+    traffic = ((PREFILL_FUSED_MMA_TRAFFIC_PER_LAYER if fused else PREFILL_MMA_TRAFFIC_PER_LAYER_CHUNK) if path == 2
+               else PREFILL_WS_TRAFFIC_PER_LAYER_CHUNK if path == 3 and not fused else None)
     name = (workload_name(cfg, T) + ", the rows of 8 chunks of 128 through each layer in one call") if fused else \
         (workload_name(cfg, T) + f", {chunks} chunks chunk-major")
     bound_us = max(roof["bytes_per_launch"] / (hbm["hbm_gbs"] * 1e3), fl / (peak_t * 1e6))
