@@ -206,3 +206,26 @@ def test_ws_prefill_layer_rows_match_chunked_rows():
     torch.cuda.synchronize()
     moe.moe_workspace_status(ws128)
     assert max_err_vs_rms(bf16_host(out), bf16_host(chunked)) <= 5e-3
+
+
+@pytest.mark.parametrize("T,path", [(32, WS), (448, WS), (449, TC)])
+def test_automatic_path_at_its_boundaries(T, path):
+    """force_path 0 takes this path for 32..448 tokens and the tcgen05 GEMM
+    above (both measured on B200; the GEMV below 32): the automatic output
+    equals the forced path's bit for bit, and sampled rows match the oracle."""
+    cfg = synth.CONFIGS[0]
+    w, D, OL = _layer(cfg, 0, layer=1)
+    h = hidden_with_gap(cfg, 0, OL, 11, T)
+    hd = h.cuda()
+    ws = moe.workspace(D, T)
+    outs = []
+    for fp in (0, path):
+        out = torch.empty_like(hd)
+        moe.moe_layer_forward(D, hd, out, T, ws, moe.make_opts(force_path=fp))
+        torch.cuda.synchronize()
+        moe.moe_workspace_status(ws)
+        outs.append(out)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    rows = sorted({0, T // 2, T - 1})
+    ref = oracle.layer_forward(OL, h[rows])
+    assert max_err_vs_rms(bf16_host(outs[0])[rows], ref["out_f64"]) <= OUT_TOL
