@@ -730,7 +730,8 @@ def main():
     ap.add_argument("--head-only", action="store_true",
                     help="profiling only: time the output-head GEMV alone and print its object")
     ap.add_argument("--prefill-only", action="store_true",
-                    help="profiling only: the 128-token prefill chunks alone (with --layers, --expert-path)")
+                    help="profiling only: the 128-token prefill chunks alone (with --layers, --expert-path; "
+                         "--tokens 1024 puts the rows of 8 chunks through each layer in one call)")
     ap.add_argument("--expert-path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="profiling only: force_path of the expert FFN (0 automatic) for --prefill-only or the headline")
     ap.add_argument("--headline-only", dest="all_configs", action="store_false",
@@ -754,7 +755,8 @@ def main():
             from int4_routed_expert_02_b200 import build
             build.build()
             res = {"prefill": prefill_measure(torch.device("cuda", local_rank), chunks=2, layers=args.layers or None,
-                                              force_path=args.expert_path)[0]} if rank == 0 else None
+                                              T=args.tokens or None, force_path=args.expert_path)[0]} \
+                if rank == 0 else None
         elif args.head_only:
             from int4_routed_expert_02_b200 import build
             build.build()
