@@ -250,49 +250,63 @@ router_logits_tiled_kernel(const uint32_t *__restrict__ rq, const uint16_t *__re
         }
 }
 
-// One warp per token.  k rounds of a warp-wide argmax over the logits not yet
-// taken, ordered by (logit desc, index asc), then the softmax over the k
-// selected logits in fp64, times per_expert_scale.
+// The logit as an order-preserving 64-bit key (larger logit <=> larger key;
+// -0 and +0 are the same logit).
+__device__ __forceinline__ unsigned long long topk_key(double v) {
+    unsigned long long b = (unsigned long long)__double_as_longlong(v);
+    if (b == 0x8000000000000000ull) b = 0ull;
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ double topk_logit(unsigned long long k) {
+    const unsigned long long b = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
+    return __longlong_as_double((long long)b);
+}
+
+// One warp per token, lane j holding the keys of experts j, 32 + j, ... in
+// registers.  k rounds: every lane offers its largest key not yet taken (the
+// lower expert on equal keys), two 32-bit max-reductions (high word, then low
+// word among the lanes holding the high word) give the largest key and a
+// min-reduction the lowest expert holding it; ordered by (logit desc, index
+// asc).  Then the softmax over the k selected logits in fp64, times
+// per_expert_scale.
+template <int NSL>
 __global__ void __launch_bounds__(kWarp)
 router_topk_kernel(const double *__restrict__ logits, int E, int k, const uint16_t *__restrict__ pes,
                    int32_t *__restrict__ idx, float *__restrict__ wts) {
-    __shared__ double v[kMaxE];
-    __shared__ unsigned char taken[kMaxE];
     __shared__ double selv[kMaxK];
     __shared__ int sel[kMaxK];
     const int t = blockIdx.x, lane = threadIdx.x;
-    for (int e = lane; e < E; e += kWarp) {
-        v[e] = logits[(size_t)t * E + e];
-        taken[e] = 0;
-    }
-    __syncwarp();
-    for (int s = 0; s < k; ++s) {
-        double bv = 0.0;
-        int be = 0x7fffffff;
-        for (int e = lane; e < E; e += kWarp) {
-            if (taken[e]) continue;
-            const double x = v[e];
-            if (be == 0x7fffffff || x > bv || (x == bv && e < be)) {
-                bv = x;
-                be = e;
-            }
-        }
+    unsigned long long key[NSL];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-                bv = ov;
-                be = oe;
+    for (int sl = 0; sl < NSL; ++sl) {
+        const int e = sl * kWarp + lane;
+        key[sl] = e < E ? topk_key(logits[(size_t)t * E + e]) : 0ull;  // 0: below every logit's key
+    }
+    for (int s = 0; s < k; ++s) {
+        unsigned long long best = 0ull;
+        int bsl = 0;
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl)
+            if (key[sl] > best) {  // strict: the lower expert on equal keys
+                best = key[sl];
+                bsl = sl;
             }
+        const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(best >> 32));
+        const unsigned lo = __reduce_max_sync(0xffffffffu, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
+        const unsigned long long top = ((unsigned long long)hi << 32) | lo;
+        const unsigned e = __reduce_min_sync(0xffffffffu, best == top ? (unsigned)(bsl * kWarp + lane) : 0xffffffffu);
+        if (lane == (int)(e & 31u)) {
+#pragma unroll
+            for (int sl = 0; sl < NSL; ++sl)
+                if (sl == bsl) key[sl] = 0ull;
         }
         if (lane == 0) {
-            taken[be] = 1;
-            sel[s] = be;
-            selv[s] = bv;
+            sel[s] = (int)e;
+            selv[s] = topk_logit(top);
         }
-        __syncwarp();
     }
+    __syncwarp();
     // softmax over the selected logits; selv[0] is their maximum
     const double p = lane < k ? exp(selv[lane] - selv[0]) : 0.0;
     const double z = warp_sum(p);
@@ -336,7 +350,10 @@ cudaError_t launch_router_logits(const moe_layer_w *w, const uint16_t *h, int T,
 
 cudaError_t launch_router_topk(const double *logits, int T, int E, int k, const uint16_t *pes, int32_t *idx,
                                float *wts, cudaStream_t st) {
-    router_topk_kernel<<<T, kWarp, 0, st>>>(logits, E, k, pes, idx, wts);
+    if (E <= 4 * kWarp) router_topk_kernel<4><<<T, kWarp, 0, st>>>(logits, E, k, pes, idx, wts);
+    else if (E <= 8 * kWarp) router_topk_kernel<8><<<T, kWarp, 0, st>>>(logits, E, k, pes, idx, wts);
+    else if (E <= 16 * kWarp) router_topk_kernel<16><<<T, kWarp, 0, st>>>(logits, E, k, pes, idx, wts);
+    else router_topk_kernel<32><<<T, kWarp, 0, st>>>(logits, E, k, pes, idx, wts);
     return cudaGetLastError();
 }
 
