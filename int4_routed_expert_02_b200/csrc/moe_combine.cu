@@ -14,12 +14,12 @@
 namespace moe {
 
 constexpr int kCombineMaxThreads = 1024;  // one thread per 4 columns up to H = 4096
+constexpr int kCombinePer = 2;            // groups of 4 columns per thread: H <= 8192
 
 __global__ void __launch_bounds__(kCombineMaxThreads)
 combine_kernel(const float *__restrict__ y, const float *__restrict__ sh, const float *__restrict__ wts, int H, int k,
                int with_shared, const uint16_t *__restrict__ h_in, float *__restrict__ m_out,
                uint16_t *__restrict__ h_out, int post_norm, float layer_scalar, float eps) {
-    extern __shared__ float4 msh4[];  // [H / 4]
     __shared__ float red[kCombineMaxThreads / 32];
     __shared__ float wk[kMaxK];
     const int t = blockIdx.x, H4 = H / 4;
@@ -27,11 +27,17 @@ combine_kernel(const float *__restrict__ y, const float *__restrict__ sh, const 
     __syncthreads();
     const float4 *y4 = reinterpret_cast<const float4 *>(y) + (size_t)t * k * H4;
     float ss = 0.f;
-    // four columns per thread and step; the loads of 8 routed slots (and the
-    // shared row) are issued before any is used; per column the sum runs over
-    // s = 0, 1, ... in order, then adds the shared branch
-    for (int i = threadIdx.x; i < H4; i += blockDim.x) {
+    // four columns per thread and step, kept in registers for the second half;
+    // the loads of 8 routed slots (and the shared row) are issued before any is
+    // used; per column the sum runs over s = 0, 1, ... in order, then adds the
+    // shared branch
+    float4 mv[kCombinePer];
+#pragma unroll
+    for (int r = 0; r < kCombinePer; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
         float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+        mv[r] = m;
+        if (i >= H4) continue;
         for (int s0 = 0; s0 < k; s0 += 8) {
             float4 v[8];
 #pragma unroll
@@ -58,27 +64,33 @@ combine_kernel(const float *__restrict__ y, const float *__restrict__ sh, const 
             m.w += sv.w;
         }
         if (m_out) reinterpret_cast<float4 *>(m_out)[(size_t)t * H4 + i] = m;
-        msh4[i] = m;
+        mv[r] = m;
         ss = fmaf(m.x, m.x, fmaf(m.y, m.y, fmaf(m.z, m.z, fmaf(m.w, m.w, ss))));
     }
     if (!h_out) return;
     ss = block_sum(ss, red);
     const float inv = post_norm ? 1.0f / sqrtf(ss / (float)H + eps) : 1.0f;
-    const float *msh = reinterpret_cast<const float *>(msh4);
-    for (int i = threadIdx.x; i < H; i += blockDim.x) {
-        const float v = (bf16_bits_to_float(h_in[(size_t)t * H + i]) + msh[i] * inv) * layer_scalar;
-        h_out[(size_t)t * H + i] = f32_to_bf16_bits(v);
+    // out = (h + m * inv) * layer_scalar for the thread's own columns, 4 at a time
+#pragma unroll
+    for (int r = 0; r < kCombinePer; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
+        if (i >= H4) continue;
+        const uint2 hv = __ldg(reinterpret_cast<const uint2 *>(h_in + (size_t)t * H) + i);
+        const float4 m = mv[r];
+        const uint32_t o0 = f32_to_bf16_bits((bf16_bits_to_float(hv.x & 0xffffu) + m.x * inv) * layer_scalar);
+        const uint32_t o1 = f32_to_bf16_bits((bf16_bits_to_float(hv.x >> 16) + m.y * inv) * layer_scalar);
+        const uint32_t o2 = f32_to_bf16_bits((bf16_bits_to_float(hv.y & 0xffffu) + m.z * inv) * layer_scalar);
+        const uint32_t o3 = f32_to_bf16_bits((bf16_bits_to_float(hv.y >> 16) + m.w * inv) * layer_scalar);
+        reinterpret_cast<uint2 *>(h_out + (size_t)t * H)[i] = make_uint2(o0 | (o1 << 16), o2 | (o3 << 16));
     }
 }
 
 cudaError_t launch_combine(const float *y, const float *sh, const float *wts, int T, int H, int k, int with_shared,
                            const uint16_t *h_in, float *m_out, uint16_t *h_out, int post_norm, float layer_scalar,
                            float eps, cudaStream_t st) {
-    const size_t smem = sizeof(float) * (size_t)H;
-    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(combine_kernel), smem);
-    if (e != cudaSuccess) return e;
     const int threads = min(kCombineMaxThreads, ((H / 4 + 31) / 32) * 32);
-    combine_kernel<<<T, threads, smem, st>>>(y, sh, wts, H, k, with_shared, h_in, m_out, h_out, post_norm,
+    if ((long long)threads * kCombinePer < H / 4) return cudaErrorInvalidValue;
+    combine_kernel<<<T, threads, 0, st>>>(y, sh, wts, H, k, with_shared, h_in, m_out, h_out, post_norm,
                                                      layer_scalar, eps);
     return cudaGetLastError();
 }
